@@ -1,0 +1,292 @@
+"""Float64 CPU oracle for GPTQ layer-wise INT-b weight quantization.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import this package.  It shares
+no code with the CUDA path and never imports it.
+
+Every function is a thin numpy wrapper over ``gptq_oracle.c`` (plain C,
+float64, no blocking) and cites the passage it follows:
+
+* ``hessian``      -- H accumulation, "GPTQ / AWQ / SqueezeLLM" sec. 一
+                      (H = 2 X^T X / n; here the raw sum S = X^T X).
+* ``finalize``     -- H = 2S/n, relative damping, act-order permutation
+                      (same page, sec. 一: damping, importance order).
+* ``cholesky_lower``/``trtri_lower``/``hinv_upper_chol`` -- the "decomposition"
+                      of H^-1 (same page, sec. 一; "INT4/INT8 量化推理" sec. 三).
+* ``quantize_rows`` -- the column sweep with error feedback ("INT4/INT8 量化推理"
+                      sec. 三 loop; "校准艺术" sec. 2.2 steps 1-5).
+* ``rtn``          -- round-to-nearest group min-max ("校准艺术" sec. 2.1).
+* ``pack_int4``/``unpack_int4`` -- the 66.5 B / 128-weight storage format
+                      ("INT4/INT8 量化推理" sec. 一).
+* ``trace_quadratic`` -- tr(D H D^T), the layer loss of sec. 三 of that page.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        lib.orc_half_to_double.argtypes = [ctypes.c_uint16]
+        lib.orc_half_to_double.restype = ctypes.c_double
+        lib.orc_float_to_half_rne.argtypes = [ctypes.c_float]
+        lib.orc_float_to_half_rne.restype = ctypes.c_uint16
+        lib.orc_hessian_accumulate.argtypes = [P, I64, I64, P]
+        lib.orc_hessian_accumulate.restype = None
+        lib.orc_finalize.argtypes = [P, I64, I64, ctypes.c_double, ctypes.c_int, P, P, P, P]
+        lib.orc_finalize.restype = ctypes.c_int
+        lib.orc_cholesky_lower.argtypes = [P, I64, P]
+        lib.orc_cholesky_lower.restype = ctypes.c_int
+        lib.orc_trtri_lower_T.argtypes = [P, I64, P]
+        lib.orc_trtri_lower_T.restype = None
+        lib.orc_hinv_upper_chol.argtypes = [P, I64, P]
+        lib.orc_hinv_upper_chol.restype = ctypes.c_int
+        lib.orc_quantize_rows.argtypes = [P, P, I64, I64, ctypes.c_int, I64,
+                                          P, P, P, P, P, P, P, P, P, P, P]
+        lib.orc_quantize_rows.restype = None
+        lib.orc_rtn.argtypes = [P, I64, I64, ctypes.c_int, I64, P, P, P, P]
+        lib.orc_rtn.restype = None
+        lib.orc_pack_int4.argtypes = [P, P, I64, I64, I64, P, P]
+        lib.orc_pack_int4.restype = None
+        lib.orc_unpack_int4.argtypes = [P, P, I64, I64, I64, P, P]
+        lib.orc_unpack_int4.restype = None
+        lib.orc_trace_quadratic.argtypes = [P, P, I64, I64]
+        lib.orc_trace_quadratic.restype = ctypes.c_double
+        lib.orc_num_threads.argtypes = []
+        lib.orc_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+# --------------------------------------------------------------------------
+# fp16 helpers (IEEE binary16 from the format definition)
+# --------------------------------------------------------------------------
+
+def half_bits_to_float64(h: np.ndarray) -> np.ndarray:
+    lib = _load()
+    flat = np.ascontiguousarray(h, dtype=np.uint16).ravel()
+    out = np.fromiter((lib.orc_half_to_double(int(v)) for v in flat), dtype=np.float64,
+                      count=flat.size)
+    return out.reshape(np.shape(h))
+
+
+def float32_to_half_bits(x: float) -> int:
+    return int(_load().orc_float_to_half_rne(ctypes.c_float(x)))
+
+
+def _as_half_bits(X) -> np.ndarray:
+    X = np.asarray(X)
+    if X.dtype == np.float16:
+        return np.ascontiguousarray(X).view(np.uint16)
+    if X.dtype == np.uint16:
+        return np.ascontiguousarray(X)
+    raise TypeError("X must be float16 (or its uint16 bit pattern)")
+
+
+# --------------------------------------------------------------------------
+# Hessian and its preparation
+# --------------------------------------------------------------------------
+
+def hessian(X, S: np.ndarray | None = None) -> np.ndarray:
+    """S += X^T X for X (n x d) fp16, in float64 (fp16 values promoted exactly)."""
+    Xb = _as_half_bits(X)
+    n, d = Xb.shape
+    if S is None:
+        S = np.zeros((d, d), dtype=np.float64)
+    assert S.dtype == np.float64 and S.shape == (d, d) and S.flags["C_CONTIGUOUS"]
+    _load().orc_hessian_accumulate(_p(Xb), n, d, _p(S))
+    return S
+
+
+def finalize(S: np.ndarray, n: int, damp_rel: float = 0.01, act_order: bool = False):
+    """H = 2S/n; perm (stable descending argsort of diag H when act_order);
+    H <- H[perm][:, perm]; lambda = damp_rel * mean(diag H); Hd = H + lambda I.
+
+    Returns (H, Hd, perm, lam, status) with status 0, or 3 when mean(diag H) <= 0.
+    """
+    S = np.ascontiguousarray(S, dtype=np.float64)
+    d = S.shape[0]
+    H = np.empty_like(S)
+    Hd = np.empty_like(S)
+    perm = np.empty(d, dtype=np.int32)
+    lam = ctypes.c_double(0.0)
+    st = _load().orc_finalize(_p(S), int(n), d, float(damp_rel), int(bool(act_order)),
+                              _p(H), _p(Hd), _p(perm), ctypes.byref(lam))
+    return H, Hd, perm, float(lam.value), int(st)
+
+
+def cholesky_lower(A: np.ndarray):
+    """Lower Cholesky factor; returns (L, info) with info = 1-based failing pivot or 0."""
+    A = np.ascontiguousarray(A, dtype=np.float64)
+    L = np.empty_like(A)
+    info = _load().orc_cholesky_lower(_p(A), A.shape[0], _p(L))
+    return L, int(info)
+
+
+def trtri_lower(L: np.ndarray) -> np.ndarray:
+    """Inverse of a lower-triangular matrix (returned in normal orientation)."""
+    L = np.ascontiguousarray(L, dtype=np.float64)
+    LinvT = np.empty_like(L)
+    _load().orc_trtri_lower_T(_p(L), L.shape[0], _p(LinvT))
+    return np.ascontiguousarray(LinvT.T)
+
+
+def hinv_upper_chol(Hd: np.ndarray):
+    """U upper with U^T U = Hd^-1 (plain route: chol, triangular inverse,
+    form the inverse, chol again, transpose).  Returns (U, info)."""
+    Hd = np.ascontiguousarray(Hd, dtype=np.float64)
+    U = np.empty_like(Hd)
+    info = _load().orc_hinv_upper_chol(_p(Hd), Hd.shape[0], _p(U))
+    return U, int(info)
+
+
+# --------------------------------------------------------------------------
+# Sweep, RTN, packing
+# --------------------------------------------------------------------------
+
+def n_groups(d: int, group_size: int) -> int:
+    g = d if group_size <= 0 else group_size
+    return (d + g - 1) // g
+
+
+def quantize_rows(W: np.ndarray, U: np.ndarray, bits: int = 4, group_size: int = 128,
+                  forced_codes=None, forced_scales=None, forced_zeros=None,
+                  record=False, return_wq=False):
+    """Column sweep over the rows of W (sweep order) with U (d x d upper).
+
+    Returns dict(codes uint8 m x d, scales uint16 (fp16 bits) m x G, zeros uint8
+    m x G, row_loss float64 m = sum_j (e_j / U_jj)^2, s_pre float32 m x G) and,
+    with ``record``, own_codes / tie_dist (the oracle's own decision and the
+    distance of w/s from the nearest rounding boundary) for teacher forcing.
+    """
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    U = np.ascontiguousarray(U, dtype=np.float64)
+    m, d = W.shape
+    G = n_groups(d, group_size)
+    out = dict(codes=np.empty((m, d), np.uint8), scales=np.empty((m, G), np.uint16),
+               zeros=np.empty((m, G), np.uint8), row_loss=np.empty(m, np.float64),
+               s_pre=np.empty((m, G), np.float32))
+    fc = None if forced_codes is None else np.ascontiguousarray(forced_codes, dtype=np.int16)
+    fs = None if forced_scales is None else np.ascontiguousarray(forced_scales, dtype=np.uint16)
+    fz = None if forced_zeros is None else np.ascontiguousarray(forced_zeros, dtype=np.uint8)
+    if record or fc is not None:
+        out["own_codes"] = np.empty((m, d), np.uint8)
+        out["tie_dist"] = np.empty((m, d), np.float32)
+    wq = np.empty((m, d), np.float64) if return_wq else None
+    _load().orc_quantize_rows(_p(W), _p(U), m, d, int(bits), int(group_size),
+                              _p(out["codes"]), _p(out["scales"]), _p(out["zeros"]),
+                              _p(out["row_loss"]), _p(out["s_pre"]), _p(fc), _p(fs), _p(fz),
+                              _p(out.get("own_codes")), _p(out.get("tie_dist")), _p(wq))
+    if return_wq:
+        out["wq"] = wq
+    return out
+
+
+def rtn(W: np.ndarray, bits: int = 4, group_size: int = 128):
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    m, d = W.shape
+    G = n_groups(d, group_size)
+    out = dict(codes=np.empty((m, d), np.uint8), scales=np.empty((m, G), np.uint16),
+               zeros=np.empty((m, G), np.uint8), s_pre=np.empty((m, G), np.float32))
+    _load().orc_rtn(_p(W), m, d, int(bits), int(group_size), _p(out["codes"]),
+                    _p(out["scales"]), _p(out["zeros"]), _p(out["s_pre"]))
+    return out
+
+
+def pack_int4(codes: np.ndarray, zeros: np.ndarray):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    zeros = np.ascontiguousarray(zeros, dtype=np.uint8)
+    m, d = codes.shape
+    G = zeros.shape[1]
+    assert d % 8 == 0
+    qweight = np.empty((m, d // 8), np.uint32)
+    qzeros = np.empty((m, (G + 1) // 2), np.uint8)
+    _load().orc_pack_int4(_p(codes), _p(zeros), m, d, G, _p(qweight), _p(qzeros))
+    return qweight, qzeros
+
+
+def unpack_int4(qweight: np.ndarray, qzeros: np.ndarray, d: int, G: int):
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint32)
+    qzeros = np.ascontiguousarray(qzeros, dtype=np.uint8)
+    m = qweight.shape[0]
+    codes = np.empty((m, d), np.uint8)
+    zeros = np.empty((m, G), np.uint8)
+    _load().orc_unpack_int4(_p(qweight), _p(qzeros), m, d, G, _p(codes), _p(zeros))
+    return codes, zeros
+
+
+def dequantize(codes: np.ndarray, scales16: np.ndarray, zeros: np.ndarray,
+               group_size: int, perm: np.ndarray | None = None) -> np.ndarray:
+    """Q in ORIGINAL column order: Q[:, perm[k]] = s(r, k//g) * (c[r, k] - z(r, k//g))."""
+    m, d = codes.shape
+    g = d if group_size <= 0 else group_size
+    gi = np.arange(d) // g
+    s = np.ascontiguousarray(scales16, dtype=np.uint16).view(np.float16).astype(np.float64)[:, gi]
+    z = zeros.astype(np.float64)[:, gi]
+    Qs = s * (codes.astype(np.float64) - z)
+    if perm is None:
+        return Qs
+    Q = np.empty_like(Qs)
+    Q[:, np.asarray(perm, dtype=np.int64)] = Qs
+    return Q
+
+
+def trace_quadratic(D: np.ndarray, H: np.ndarray) -> float:
+    """tr(D H D^T) in float64."""
+    D = np.ascontiguousarray(D, dtype=np.float64)
+    H = np.ascontiguousarray(H, dtype=np.float64)
+    return float(_load().orc_trace_quadratic(_p(D), _p(H), D.shape[0], D.shape[1]))
+
+
+# --------------------------------------------------------------------------
+# Whole layer
+# --------------------------------------------------------------------------
+
+def gptq_layer(W: np.ndarray, S: np.ndarray, n: int, bits: int = 4, group_size: int = 128,
+               damp_rel: float = 0.01, act_order: bool = False, record=False):
+    """Whole-layer GPTQ from the raw token sum S = X^T X over n tokens.
+
+    W is m x d (any float dtype; promoted to float64) in ORIGINAL column order.
+    Returns dict with perm, H (undamped, permuted), Hd, lam, U and the sweep
+    outputs (codes/scales/zeros in sweep order, row_loss).
+    """
+    H, Hd, perm, lam, st = finalize(S, n, damp_rel, act_order)
+    if st != 0:
+        raise ValueError("mean(diag H) <= 0: no damping can make H positive definite")
+    U, info = hinv_upper_chol(Hd)
+    if info != 0:
+        raise ValueError(f"H + lambda I is not positive definite (pivot {info})")
+    Wp = np.ascontiguousarray(np.asarray(W, dtype=np.float64)[:, perm])
+    res = quantize_rows(Wp, U, bits, group_size, record=record)
+    res.update(perm=perm, H=H, Hd=Hd, lam=lam, U=U)
+    return res
+
+
+def layer_loss(W: np.ndarray, Q: np.ndarray, H_orig: np.ndarray) -> float:
+    """tr((W-Q) H (W-Q)^T) with H in ORIGINAL column order; times n/2 this is
+    ||(W - Q) X^T||_F^2 for H = 2 X^T X / n."""
+    D = np.asarray(W, dtype=np.float64) - np.asarray(Q, dtype=np.float64)
+    return trace_quadratic(D, H_orig)
