@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""GPTQ INT4-g128 layer-quantization benchmark (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one layer whose inputs are
+resident in HBM: zero S, accumulate S = X^T X over all calibration tokens,
+prepare U (damp, factor, invert), sweep all columns with error feedback, and
+pack to INT4.  Default workload: the 7B attention projection (W 4096 x 4096
+fp16, X 262144 tokens x 4096 fp16 with 1 % outlier channels), synthetic and
+seeded.  Under torchrun every rank quantizes its own independent layer (weak
+scaling, no collective on the data path); value = weights of all ranks / the
+max-over-ranks time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the float64 CPU oracle (the only other implementation
+of this path) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+METRIC = "GPTQ INT4-g128 weights quantized/sec per layer"
+UNIT = "weights/s"
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="attn7b")
+    p.add_argument("--layer", type=int, default=0)
+    p.add_argument("--tokens", type=int, default=0, help="override token count (0: workload's)")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+
+def _dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# clocks sampler
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), hw=f[5], hwt=f[6], swt=f[7],
+                                 pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        reasons = set()
+        for r in rows:
+            if r["hw"] == "Active":
+                reasons.add("hw_slowdown")
+            if r["hwt"] == "Active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active":
+                reasons.add("sw_thermal_slowdown")
+            if r["pcap"] == "Active":
+                reasons.add("sw_power_cap")
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# workload
+# --------------------------------------------------------------------------
+
+def _workload(name, layer, tokens):
+    from post_weight_quantization_11_b200 import inputs
+    wl = inputs.WORKLOADS[name]
+    spec = wl.layers[layer]
+    n = tokens or spec.n_tokens
+    return wl, spec, n
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+def _traffic_for(kernel_file: str, summary_name: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    src = os.path.join(ROOT, "post_weight_quantization_11_b200", "csrc", kernel_file)
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if rec.get("source_sha") != sha:
+            return None
+        return rec.get("dram_bytes_per_launch_full_size")
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+class Layer:
+    """Preallocated buffers and one step of the path through the C ABI."""
+
+    def __init__(self, spec, n, dev, seed_offset=0):
+        from post_weight_quantization_11_b200 import gptq as G
+        from post_weight_quantization_11_b200 import inputs
+        self.G = G
+        self.m, self.d, self.n = spec.d_out, spec.d_in, n
+        self.act_order = spec.act_order
+        m, d = self.m, self.d
+        self.W = inputs.weights(spec, device=dev, seed_offset=seed_offset)
+        self.X = inputs.calibration_x(spec, n_tokens=n, device=dev)
+        self.S = torch.zeros(d, d, dtype=torch.float32, device=dev)
+        self.perm = torch.empty(d, dtype=torch.int32, device=dev)
+        self.U = torch.empty(d, d, dtype=torch.float32, device=dev)
+        self.info = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ws_p = torch.empty(G.gptq_prepare_workspace_bytes(d), dtype=torch.uint8, device=dev)
+        self.ws_q = torch.empty(G.gptq_quantize_workspace_bytes(m, d, 128), dtype=torch.uint8,
+                                device=dev)
+        self.codes = torch.empty(m, d, dtype=torch.uint8, device=dev)
+        self.scales = torch.empty(m, d // 128, dtype=torch.float16, device=dev)
+        self.zeros = torch.empty(m, d // 128, dtype=torch.uint8, device=dev)
+        self.loss = torch.empty(m, dtype=torch.float32, device=dev)
+        self.qweight = torch.empty(m, d // 8, dtype=torch.int32, device=dev)
+        self.qzeros = torch.empty(m, (d // 128 + 1) // 2, dtype=torch.uint8, device=dev)
+
+    def step(self, ev_k1=None):
+        G = self.G
+        self.S.zero_()
+        if ev_k1 is not None:
+            ev_k1[0].record()
+        G.gptq_hessian_accumulate(self.S, self.X)
+        if ev_k1 is not None:
+            ev_k1[1].record()
+        G.gptq_prepare_hinv(self.S, self.n, 0.01, self.act_order, self.perm, self.U, self.info,
+                            self.ws_p)
+        G.gptq_quantize_layer(self.W, self.U, self.perm if self.act_order else None, 4, 128, 128,
+                              self.codes, self.scales, self.zeros, self.loss, self.ws_q)
+        G.gptq_pack_int4(self.codes, self.zeros, self.qweight, self.qzeros)
+
+
+def _cpu_baseline(spec, n, reps=1):
+    """The float64 oracle, as it stands, on a bounded sample of the workload:
+    S over n_s tokens, the full d x d preparation, the sweep and packing of m_s
+    rows; the token and row parts are scaled linearly to the full layer (their
+    cost is exactly linear in tokens and rows)."""
+    import oracle
+    from post_weight_quantization_11_b200 import inputs
+    m, d = spec.d_out, spec.d_in
+    n_s = max(8, min(n, int(2 ** 22 // d)))       # ~4M token-features
+    m_s = min(m, 64)
+    X = inputs.calibration_x(spec, n_tokens=n_s, device="cpu").numpy()
+    W = inputs.weights(spec, device="cpu")[:m_s].double().numpy()
+    t0 = time.perf_counter()
+    S = oracle.hessian(X)
+    t_s = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    H, Hd, perm, lam, st = oracle.finalize(S, n_s, 0.01, spec.act_order)
+    U, info = oracle.hinv_upper_chol(Hd)
+    t_p = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    r = oracle.quantize_rows(np.ascontiguousarray(W[:, perm]), U, 4, 128)
+    oracle.pack_int4(r["codes"], r["zeros"])
+    t_q = time.perf_counter() - t0
+    total = t_s * (n / n_s) + t_p + t_q * (m / m_s)
+    return dict(value=m * d / total, unit=UNIT, cores=oracle.num_threads(), kind="oracle",
+                sample=f"S over {n_s} of {n} tokens (x{n / n_s:.0f}), full {d}x{d} prepare, "
+                       f"sweep+pack of {m_s} of {m} rows (x{m / m_s:.0f}); "
+                       f"measured {t_s + t_p + t_q:.1f} s, extrapolated layer {total:.0f} s",
+                seconds=dict(hessian_sample=t_s, prepare=t_p, sweep_pack_sample=t_q,
+                             layer_extrapolated=total))
+
+
+def run_ours(a):
+    ws, rank, local = _dist_init()
+    from post_weight_quantization_11_b200 import gptq as G
+    G.load_library()
+    dev = torch.device("cuda", local)
+    wl, spec, n = _workload(a.workload, a.layer, a.tokens)
+    lay = Layer(spec, n, dev, seed_offset=rank)
+    m, d = lay.m, lay.d
+    torch.cuda.synchronize()
+    for _ in range(max(3, a.warmup)):
+        lay.step()
+    torch.cuda.synchronize()
+    assert int(lay.info.item()) == 0, "non-positive pivot in the workload"
+
+    n_ev = a.steps
+    k1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n_ev)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = G.gptq_debug_launch_count()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for i in range(a.steps):
+            lay.step(k1[i])
+        end.record()
+        torch.cuda.synchronize()
+    _barrier(ws)
+    launches = G.gptq_debug_launch_count() - launches0
+    ms = start.elapsed_time(end) / a.steps
+    ms = _max_over_ranks(ms, ws)
+    k1_ms = statistics.mean(s.elapsed_time(e) for s, e in k1)
+
+    # end to end through the public API from pinned host memory
+    Xh = lay.X.cpu().pin_memory()
+    Wh = lay.W.cpu().pin_memory()
+    qwh = torch.empty_like(lay.qweight, device="cpu").pin_memory()
+    qzh = torch.empty_like(lay.qzeros, device="cpu").pin_memory()
+    sch = torch.empty_like(lay.scales, device="cpu").pin_memory()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    torch.cuda.synchronize()
+    e_start.record()
+    for _ in range(a.e2e_steps):
+        lay.X.copy_(Xh, non_blocking=True)
+        lay.W.copy_(Wh, non_blocking=True)
+        lay.step()
+        qwh.copy_(lay.qweight, non_blocking=True)
+        qzh.copy_(lay.qzeros, non_blocking=True)
+        sch.copy_(lay.scales, non_blocking=True)
+    e_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e_start.elapsed_time(e_end) / a.e2e_steps, ws)
+    h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in (qwh, qzh, sch))
+
+    peaks, src = _peaks()
+    flops = float(n) * d * d                         # SYRK, upper triangle: n d^2
+    achieved = flops / (k1_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    traffic = _traffic_for("hessian.cu", "hessian_syrk_attn7b.json")
+    line = {
+        "metric": METRIC,
+        "value": ws * m * d / (ms * 1e-3),
+        "unit": UNIT,
+        "n_gpus": ws,
+        "steps": a.steps,
+        "warmup": a.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; random-init weights, Gaussian calibration inputs with "
+                "outlier channels)",
+        "config": {"workload": f"{spec.name} ({a.workload}): W {m}x{d} fp16, X {n}x{d} fp16, "
+                               f"INT4 g128, damp 0.01, act_order={spec.act_order}",
+                   "layers_per_rank": 1, "tokens": n,
+                   "l2": "inputs larger than L2 (X %.2f GB re-read every step)" %
+                         (n * d * 2 / 1e9)},
+        "e2e": {"value": ws * m * d / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "roofline": {"bound": "tensor", "kernel": "hessian_accumulate (S += X^T X)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"bf16_tflops_sustained of {src} (fp16 = bf16 rate)",
+                     "kernel_ms": k1_ms},
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+        cb = _cpu_baseline(spec, n)
+        cb.pop("seconds", None)
+        line["cpu_baseline"] = cb
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# --------------------------------------------------------------------------
+
+def run_reference(a):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl, spec, n = _workload(a.workload, a.layer, a.tokens)
+    for _ in range(a.warmup):
+        _cpu_baseline(spec, n)
+    vals, samples = [], None
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        r = _cpu_baseline(spec, n)
+        vals.append(r["value"])
+        samples = r
+    wall = time.perf_counter() - t0
+    v = statistics.median(vals)
+    m, d = spec.d_out, spec.d_in
+    line = {
+        "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": ws, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": m * d / v * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "impl": "reference",
+        "config": {"workload": f"{spec.name} ({a.workload}): W {m}x{d} fp16, X {n}x{d} fp16, "
+                               f"INT4 g128, damp 0.01, act_order={spec.act_order}",
+                   "tokens": n},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": samples["cores"], "kind": "oracle",
+                         "sample": samples["sample"]},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

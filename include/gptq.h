@@ -1,0 +1,167 @@
+/*
+ * gptq.h -- C ABI of the B200 (sm_100a) GPTQ layer-quantization library
+ * (libgptq.so).
+ *
+ * The operation is GPTQ layer-wise weight quantization as described on the
+ * pages "GPTQ / AWQ / SqueezeLLM" (sec. 一: H = 2 X^T X / n from the
+ * calibration inputs, damping, block-wise processing, importance order),
+ * "INT4/INT8 量化推理：从 GPTQ 到 AWQ 的取舍" (sec. 一: groups of 128
+ * consecutive weights with an fp16 scale and a 4-bit zero point, 66.5 bytes
+ * per 128 weights; sec. 三: quantize column by column and push each column's
+ * error onto the not-yet-quantized columns through H^-1) and
+ * "大模型量化的“校准”艺术" (sec. 2.1 min-max mapping; sec. 2.2 the loop).
+ *
+ * Conventions shared by every call:
+ *  - All array arguments are DEVICE pointers to caller-owned memory (the
+ *    library never allocates, frees or synchronizes).  Scratch memory, where
+ *    a call needs it, is passed as (ws, ws_bytes); the matching
+ *    *_workspace_bytes() call gives the size.
+ *  - Matrices are row-major and densely packed (leading dimension = number of
+ *    columns).  W is d_out x d_in like a torch Linear weight: a "column" is an
+ *    input channel.  X is n_tokens x d_in (token-major).
+ *  - fp16 data is passed as its 16-bit IEEE pattern (uint16_t).
+ *  - `stream` is a cudaStream_t (0 = legacy default stream).  Every call is
+ *    asynchronous on it; device-side outcomes (non-positive pivot) are
+ *    reported through a device int the caller may read after synchronizing.
+ *  - Pointers must be 16-byte aligned.  Arguments are validated before any
+ *    launch; on error nothing is launched and the status says why.
+ *  - Return value: a gptq_status.  GPTQ_ERR_CUDA means a launch failed; the
+ *    CUDA error is left for the caller to inspect with cudaGetLastError().
+ */
+#ifndef GPTQ_B200_GPTQ_H
+#define GPTQ_B200_GPTQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GPTQ_OK = 0,
+    GPTQ_ERR_INVALID_ARG = 1,   /* null pointer, bad enum, misaligned pointer */
+    GPTQ_ERR_SHAPE = 2,         /* sizes outside what the call supports */
+    GPTQ_ERR_NOT_PD = 3,        /* (host-detectable) no positive definite H */
+    GPTQ_ERR_UNSUPPORTED = 4,   /* valid but not implemented (e.g. bits=5) */
+    GPTQ_ERR_CUDA = 5,          /* a kernel launch failed */
+    GPTQ_ERR_TIMEOUT = 6        /* reserved: a bounded device wait expired */
+} gptq_status;
+
+enum { GPTQ_DTYPE_F32 = 0, GPTQ_DTYPE_F16 = 1 };
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gptq_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int gptq_abi_version(void);
+
+/* Diagnostics: number of kernel launches this process has issued through the
+ * library so far (all devices, all calls).  Host-only, never synchronizes. */
+uint64_t gptq_debug_launch_count(void);
+
+/*
+ * Hessian accumulation -- "GPTQ / AWQ / SqueezeLLM" sec. 一 (H from the
+ * calibration inputs; the 2/n factor is applied later by gptq_prepare_hinv).
+ *
+ *   S[i][j] += sum_t X[t][i] * X[t][j]      for 0 <= i <= j < d
+ *
+ * S: d x d fp32, in/out.  Only the upper triangle (i <= j) is read and
+ *    written; the strictly-lower triangle is left untouched.  Zero S before
+ *    the first batch; call once per calibration batch.
+ * X: n_tokens x d fp16 (token-major).
+ * n_seen: optional HOST counter, incremented by n_tokens on success.
+ * Requires d % 128 == 0, 128 <= d <= 32768, n_tokens >= 0 (0: no-op).
+ * Accumulation is fp32 on the tensor cores with fp16 inputs.
+ */
+int gptq_hessian_accumulate(float* S, const uint16_t* X, int64_t n_tokens, int64_t d,
+                            int64_t* n_seen, void* stream);
+
+/*
+ * Prepare the inverse-Hessian factor -- "GPTQ / AWQ / SqueezeLLM" sec. 一
+ * (H = 2 X^T X / n, damping, decomposition of H^-1, importance order) and
+ * "INT4/INT8 量化推理" sec. 三 (rows of H^-1 carry the error feedback).
+ *
+ *   H   = (2 / n) * S, symmetric (upper triangle of S mirrored)
+ *   perm = stable descending argsort of diag(H) if act_order, else identity
+ *   H   <- H[perm][:, perm];  lambda = damp_rel * mean(diag H);  Hd = H + lambda I
+ *   U   = upper-triangular Cholesky factor of Hd^-1  (U^T U = Hd^-1)
+ *
+ * S: d x d fp32 from gptq_hessian_accumulate (upper triangle read, not written).
+ * n_tokens: total tokens accumulated into S (> 0).
+ * perm: d int32 output (written whenever non-NULL; required if act_order).
+ * U: d x d fp32 output, row-major; strictly-lower triangle written as 0.
+ * info: device int32 output: 0 on success, else a 1-based pivot index of Hd
+ *       where the factorization met a non-positive pivot (U then undefined).
+ * ws: scratch of gptq_prepare_workspace_bytes(d) bytes.
+ * Requires d % 128 == 0, 128 <= d <= 32768, damp_rel >= 0.
+ */
+size_t gptq_prepare_workspace_bytes(int64_t d);
+int gptq_prepare_hinv(const float* S, int64_t d, int64_t n_tokens, float damp_rel,
+                      int act_order, int32_t* perm, float* U, int32_t* info,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Quantize one layer -- "INT4/INT8 量化推理" sec. 三 (column loop with error
+ * compensation), "GPTQ / AWQ / SqueezeLLM" sec. 一 (blocks), "校准艺术"
+ * sec. 2.1 (min-max), "INT4/INT8 量化推理" sec. 一 (group layout).
+ *
+ * For every row r, columns j = 0..d_in-1 in sweep order (W's columns taken
+ * through perm when non-NULL):
+ *   at a group start: mn = min(0, min w[j:j+g]), mx = max(0, max w[j:j+g])
+ *                     (all zero: [-1, 1]); s = fp16(fp32(mx - mn) / maxq)
+ *                     clamped to [2^-24, 65504]; z = clamp(rne(-mn / s), 0, maxq)
+ *   c = clamp(rne(w_j / s) + z, 0, maxq);   e = w_j - s (c - z)
+ *   E_j = e / U[j][j];  w[k] -= E_j U[j][k] for k > j;  row_loss[r] += E_j^2
+ * (decisions in IEEE fp32; maxq = 2^bits - 1).  The feedback inside each
+ * block of block_size columns is applied column by column on the CUDA cores;
+ * the feedback onto later blocks is one tensor-core product per block.
+ *
+ * W: d_out x d_in, dtype GPTQ_DTYPE_F16 or GPTQ_DTYPE_F32 (read only).
+ * U: d_in x d_in fp32 from gptq_prepare_hinv (upper triangle read).
+ * perm: d_in int32 or NULL (identity).
+ * codes: d_out x d_in uint8 output, sweep order (code of column perm[k] at k).
+ * scales: d_out x G fp16 output (G = d_in / group_size), zeros: d_out x G uint8.
+ * row_loss: d_out fp32 output or NULL: sum_j E_j^2 (= tr(D Hd D^T) per row).
+ * bits in {2,3,4,8}; group_size in {32, 64, 128}; block_size == 128.
+ * Requires d_in % 128 == 0, 128 <= d_in <= 32768, 1 <= d_out <= 2^24.
+ */
+size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, int block_size);
+int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
+                        const float* U, const int32_t* perm, int bits, int group_size,
+                        int block_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
+                        float* row_loss, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Pack INT4 -- "INT4/INT8 量化推理" sec. 一 (64 B of codes + 0.5 B zero point
+ * + 2 B fp16 scale per 128 weights).
+ *   qweight[r][w] = sum_k codes[r][8w + k] << 4k        (uint32, k = 0..7)
+ *   qzeros[r][b]  = zeros[r][2b] | zeros[r][2b+1] << 4   (odd G: high nibble 0)
+ * codes: d_out x d_in uint8 (values 0..15), zeros: d_out x G uint8.
+ * qweight: d_out x d_in/8 uint32 out, qzeros: d_out x ceil(G/2) uint8 out.
+ * Requires d_in % 8 == 0, G >= 1.
+ */
+int gptq_pack_int4(const uint8_t* codes, const uint8_t* zeros, int64_t d_out, int64_t d_in,
+                   int64_t n_groups, uint32_t* qweight, uint8_t* qzeros, void* stream);
+
+/* Inverse of gptq_pack_int4 (bit-exact round trip). */
+int gptq_unpack_int4(const uint32_t* qweight, const uint8_t* qzeros, int64_t d_out,
+                     int64_t d_in, int64_t n_groups, uint8_t* codes, uint8_t* zeros,
+                     void* stream);
+
+/*
+ * Round-to-nearest baseline -- "大模型量化实战（上）" (RTN: every weight
+ * rounded on its own) with the min-max group quantizer of "校准艺术" sec. 2.1:
+ * the same group parameters and codes as gptq_quantize_layer, taken on the
+ * original W with no error feedback.  Same argument meaning and limits as
+ * gptq_quantize_layer (natural column order, no U, no workspace).
+ */
+int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bits,
+                 int group_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
+                 void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_GPTQ_H */

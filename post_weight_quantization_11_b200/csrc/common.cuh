@@ -1,0 +1,36 @@
+// Shared host/device helpers of libgptq (sm_100a).  No quantization
+// arithmetic lives here.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+#include <algorithm>
+#include <cstring>
+
+#include "../../include/gptq.h"
+
+#define GPTQ_ABI_VERSION 100
+
+namespace gptq {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Process-wide count of kernel launches issued by the library (diagnostics).
+void count_launches(int n = 1);
+
+inline int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Supported problem limits (validated at the ABI).
+constexpr int64_t kMaxDim = 32768;
+constexpr int64_t kMaxRows = int64_t(1) << 24;
+
+}  // namespace gptq

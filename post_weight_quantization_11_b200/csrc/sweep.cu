@@ -1,0 +1,318 @@
+// Layer quantization driver and the intra-block column sweep -- "INT4/INT8
+// 量化推理" sec. 三 (quantize column by column, push the error onto the
+// not-yet-quantized columns), "GPTQ / AWQ / SqueezeLLM" sec. 一 (process in
+// blocks), "大模型量化的“校准”艺术" sec. 2.2 steps 1-5.
+//
+// Per 128-column block b (columns j0 .. j0+127, sweep order):
+//   block_sweep:  every row runs the 128 sequential steps with the block's
+//                 columns in registers (4 lanes per row, 32 columns per lane)
+//                 and U's 128x128 diagonal block in shared memory; writes the
+//                 codes, group scales/zeros, the scaled errors E (rows x 128)
+//                 and accumulates sum E_j^2 per row.
+//   block_update: W[:, j0+128:] -= E . U[j0:j0+128, j0+128:]
+// Rows are independent given U, so a block's sweep is parallel over rows and
+// only the chain of blocks is sequential.
+#include "common.cuh"
+#include "quant_common.cuh"
+#include "simt_gemm.cuh"
+#include "update.cuh"
+
+namespace gptq {
+
+constexpr int SW_B = 128;          // block width (columns)
+constexpr int SW_ROWS = 32;        // rows per CTA (4 lanes each, 128 threads)
+constexpr unsigned FULL = 0xffffffffu;
+
+// W_work[r][k] = float(W[r][perm[k]])
+template <typename T>
+__global__ void init_work_kernel(const T* __restrict__ W, const int32_t* __restrict__ perm,
+                                 int64_t m, int64_t d, float* __restrict__ Wk)
+{
+    const int64_t total = m * d;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = i / d, k = i - r * d;
+        const int64_t src = perm ? int64_t(perm[k]) : k;
+        Wk[i] = float(W[r * d + src]);
+    }
+}
+
+template <int GS>
+__global__ void __launch_bounds__(128)
+block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
+                   int64_t j0, float maxqf, uint8_t* __restrict__ codes,
+                   __half* __restrict__ scales, uint8_t* __restrict__ zeros,
+                   float* __restrict__ E_out, float* __restrict__ row_loss, int first_block)
+{
+    extern __shared__ __align__(16) float smem[];
+    float* Us = smem;                        // 128 x 128, strictly-lower part zeroed
+    float* rdiag = smem + SW_B * SW_B;       // 128: 1 / U_jj
+    const int tid = threadIdx.x;
+    for (int idx = tid * 4; idx < SW_B * SW_B; idx += 128 * 4) {
+        const int a = idx / SW_B, b = idx % SW_B;
+        float4 v = *reinterpret_cast<const float4*>(U + (j0 + a) * d + j0 + b);
+        if (b + 0 < a) v.x = 0.f;
+        if (b + 1 < a) v.y = 0.f;
+        if (b + 2 < a) v.z = 0.f;
+        if (b + 3 < a) v.w = 0.f;
+        *reinterpret_cast<float4*>(Us + idx) = v;
+    }
+    __syncthreads();
+    if (tid < SW_B) rdiag[tid] = 1.0f / Us[tid * SW_B + tid];
+
+    const int lane = tid & 31, sub = lane & 3;
+    const int src_base = lane & ~3;
+    const int64_t row = int64_t(blockIdx.x) * SW_ROWS + (tid >> 2);
+    const bool valid = row < m;
+    const int64_t G = d / GS;
+
+    float w[32];
+    if (valid) {
+        const float4* p = reinterpret_cast<const float4*>(Wk + row * d + j0 + 32 * sub);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            float4 v = p[q];
+            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) w[q] = 0.f;
+    }
+    __syncthreads();
+
+    float Ev[32];
+    uint32_t cp[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) cp[q] = 0u;
+    float loss = 0.f;
+    GroupQ gq;
+    gq.s = 1.f; gq.z = 0.f; gq.h = __float2half(1.f);
+
+#pragma unroll
+    for (int j = 0; j < SW_B; ++j) {
+        if (j % GS == 0) {
+            constexpr int span = GS / 32;
+            const int lo = j / 32;
+            float mn = 0.f, mx = 0.f;
+            if (sub >= lo && sub < lo + span) {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) { mn = fminf(mn, w[q]); mx = fmaxf(mx, w[q]); }
+            }
+            mn = fminf(mn, __shfl_xor_sync(FULL, mn, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+            mn = fminf(mn, __shfl_xor_sync(FULL, mn, 2));
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+            gq = group_params(mn, mx, maxqf);
+            if (valid && sub == lo) {
+                const int64_t gi = (j0 + j) / GS;
+                scales[row * G + gi] = gq.h;
+                zeros[row * G + gi] = (uint8_t)gq.z;
+            }
+        }
+        const int owner = j / 32, idx = j % 32;
+        const float x = __shfl_sync(FULL, w[idx], src_base | owner);
+        const float c = quant_code(x, gq, maxqf);
+        const float q = gq.s * (c - gq.z);
+        const float e = x - q;
+        const float Ej = e * rdiag[j];
+        loss = fmaf(Ej, Ej, loss);
+        if (sub == owner) {
+            Ev[idx] = Ej;
+            cp[idx / 4] |= uint32_t(c) << (8 * (idx % 4));
+        }
+        const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B + 32 * sub);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 u = urow[q4];
+            w[4 * q4 + 0] = fmaf(-Ej, u.x, w[4 * q4 + 0]);
+            w[4 * q4 + 1] = fmaf(-Ej, u.y, w[4 * q4 + 1]);
+            w[4 * q4 + 2] = fmaf(-Ej, u.z, w[4 * q4 + 2]);
+            w[4 * q4 + 3] = fmaf(-Ej, u.w, w[4 * q4 + 3]);
+        }
+    }
+    if (!valid) return;
+    uint4* cdst = reinterpret_cast<uint4*>(codes + row * d + j0 + 32 * sub);
+    cdst[0] = make_uint4(cp[0], cp[1], cp[2], cp[3]);
+    cdst[1] = make_uint4(cp[4], cp[5], cp[6], cp[7]);
+    float4* edst = reinterpret_cast<float4*>(E_out + row * SW_B + 32 * sub);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+        edst[q] = make_float4(Ev[4 * q], Ev[4 * q + 1], Ev[4 * q + 2], Ev[4 * q + 3]);
+    if (row_loss && sub == 0) row_loss[row] = first_block ? loss : row_loss[row] + loss;
+}
+
+// Round-to-nearest: one warp per (row, 128-column segment), 4 columns per lane.
+template <int GS, typename T>
+__global__ void __launch_bounds__(256)
+rtn_kernel(const T* __restrict__ W, int64_t m, int64_t d, float maxqf,
+           uint8_t* __restrict__ codes, __half* __restrict__ scales, uint8_t* __restrict__ zeros)
+{
+    const int64_t seg = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t segs_per_row = d / 128;
+    if (seg >= m * segs_per_row) return;   // whole warp exits together
+    const int64_t row = seg / segs_per_row;
+    const int64_t c0 = (seg - row * segs_per_row) * 128 + 4 * lane;
+    float x[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) x[q] = float(W[row * d + c0 + q]);
+    float mn = 0.f, mx = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) { mn = fminf(mn, x[q]); mx = fmaxf(mx, x[q]); }
+#pragma unroll
+    for (int o = 1; o < GS / 4; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+    }
+    const GroupQ gq = group_params(mn, mx, maxqf);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) packed |= uint32_t(quant_code(x[q], gq, maxqf)) << (8 * q);
+    *reinterpret_cast<uint32_t*>(codes + row * d + c0) = packed;
+    if ((lane % (GS / 4)) == 0) {
+        const int64_t G = d / GS;
+        const int64_t gi = c0 / GS;
+        scales[row * G + gi] = gq.h;
+        zeros[row * G + gi] = (uint8_t)gq.z;
+    }
+}
+
+struct QuantWs {
+    float* Wk;     // d_out x d_in working copy (sweep order)
+    float* E;      // d_out x 128 scaled errors of the current block
+    UpdateWs upd;  // tensor-core update scratch
+};
+
+static size_t quant_layout(int64_t m, int64_t d, char* base, QuantWs* w)
+{
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 1024); return o; };
+    size_t oW = take(sizeof(float) * m * d);
+    size_t oE = take(sizeof(float) * m * SW_B);
+    size_t oU = take(update_ws_bytes(m, d));
+    if (w && base) {
+        w->Wk = reinterpret_cast<float*>(base + oW);
+        w->E = reinterpret_cast<float*>(base + oE);
+        update_ws_bind(m, d, base + oU, &w->upd);
+    }
+    return off;
+}
+
+static int check_quant_args(int w_dtype, int64_t m, int64_t d, int bits, int group_size)
+{
+    if (w_dtype != GPTQ_DTYPE_F16 && w_dtype != GPTQ_DTYPE_F32) return GPTQ_ERR_INVALID_ARG;
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8)) return GPTQ_ERR_UNSUPPORTED;
+    if (!(group_size == 32 || group_size == 64 || group_size == 128)) return GPTQ_ERR_UNSUPPORTED;
+    if (d < 128 || d > kMaxDim || d % 128 != 0) return GPTQ_ERR_SHAPE;
+    if (m < 1 || m > kMaxRows) return GPTQ_ERR_SHAPE;
+    return GPTQ_OK;
+}
+
+template <int GS>
+static void launch_sweep(dim3 grid, size_t smem, cudaStream_t st, const float* Wk, const float* U,
+                         int64_t m, int64_t d, int64_t j0, float maxqf, uint8_t* codes,
+                         __half* scales, uint8_t* zeros, float* E, float* row_loss, int first)
+{
+    cudaFuncSetAttribute(block_sweep_kernel<GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    block_sweep_kernel<GS><<<grid, 128, smem, st>>>(Wk, U, m, d, j0, maxqf, codes, scales, zeros,
+                                                   E, row_loss, first);
+    count_launches();
+}
+
+}  // namespace gptq
+
+extern "C" size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, int block_size)
+{
+    if (d_out <= 0 || d_in <= 0 || block_size != gptq::SW_B) return 0;
+    return gptq::quant_layout(d_out, d_in, nullptr, nullptr);
+}
+
+extern "C" int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
+                                   const float* U, const int32_t* perm, int bits, int group_size,
+                                   int block_size, uint8_t* codes, uint16_t* scales,
+                                   uint8_t* zeros, float* row_loss, void* ws, size_t ws_bytes,
+                                   void* stream)
+{
+    using namespace gptq;
+    if (!W || !U || !codes || !scales || !zeros || !ws) return GPTQ_ERR_INVALID_ARG;
+    int rc = check_quant_args(w_dtype, d_out, d_in, bits, group_size);
+    if (rc != GPTQ_OK) return rc;
+    if (block_size != SW_B) return GPTQ_ERR_UNSUPPORTED;
+    if (!aligned16(W) || !aligned16(U) || !aligned16(codes) || !aligned16(scales) ||
+        !aligned16(zeros) || !aligned16(ws) || (perm && !aligned16(perm)) ||
+        (row_loss && !aligned16(row_loss)))
+        return GPTQ_ERR_INVALID_ARG;
+    if (ws_bytes < gptq_quantize_workspace_bytes(d_out, d_in, block_size))
+        return GPTQ_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    QuantWs w;
+    quant_layout(d_out, d_in, reinterpret_cast<char*>(ws), &w);
+    const int64_t m = d_out, d = d_in;
+    {
+        const int64_t total = m * d;
+        const unsigned grid = (unsigned)std::min<int64_t>(ceil_div(total, 256), 148 * 16);
+        if (w_dtype == GPTQ_DTYPE_F16)
+            init_work_kernel<__half><<<grid, 256, 0, st>>>(reinterpret_cast<const __half*>(W), perm,
+                                                           m, d, w.Wk);
+        else
+            init_work_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(W), perm,
+                                                          m, d, w.Wk);
+        count_launches();
+    }
+    rc = update_prepare_u(U, d, &w.upd, st);
+    if (rc != GPTQ_OK) return rc;
+    const float maxqf = float((1 << bits) - 1);
+    const dim3 grid((unsigned)ceil_div(m, SW_ROWS));
+    const size_t smem = sizeof(float) * (SW_B * SW_B + SW_B);
+    __half* sc = reinterpret_cast<__half*>(scales);
+    const int64_t nblk = d / SW_B;
+    for (int64_t b = 0; b < nblk; ++b) {
+        const int64_t j0 = b * SW_B;
+        switch (group_size) {
+            case 32: launch_sweep<32>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
+                                      w.E, row_loss, b == 0); break;
+            case 64: launch_sweep<64>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
+                                      w.E, row_loss, b == 0); break;
+            default: launch_sweep<128>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
+                                       w.E, row_loss, b == 0); break;
+        }
+        if (b + 1 < nblk) {
+            rc = block_update(w.Wk, w.E, U, m, d, j0, &w.upd, st);
+            if (rc != GPTQ_OK) return rc;
+        }
+    }
+    return launch_status();
+}
+
+extern "C" int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bits,
+                            int group_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
+                            void* stream)
+{
+    using namespace gptq;
+    if (!W || !codes || !scales || !zeros) return GPTQ_ERR_INVALID_ARG;
+    int rc = check_quant_args(w_dtype, d_out, d_in, bits, group_size);
+    if (rc != GPTQ_OK) return rc;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros))
+        return GPTQ_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    const float maxqf = float((1 << bits) - 1);
+    const int64_t warps = d_out * (d_in / 128);
+    const unsigned grid = (unsigned)ceil_div(warps * 32, 256);
+    __half* sc = reinterpret_cast<__half*>(scales);
+#define GPTQ_RTN_LAUNCH(GSV)                                                                     \
+    if (w_dtype == GPTQ_DTYPE_F16)                                                               \
+        rtn_kernel<GSV, __half><<<grid, 256, 0, st>>>(reinterpret_cast<const __half*>(W), d_out, \
+                                                      d_in, maxqf, codes, sc, zeros);            \
+    else                                                                                         \
+        rtn_kernel<GSV, float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(W), d_out,   \
+                                                     d_in, maxqf, codes, sc, zeros);
+    switch (group_size) {
+        case 32: GPTQ_RTN_LAUNCH(32) break;
+        case 64: GPTQ_RTN_LAUNCH(64) break;
+        default: GPTQ_RTN_LAUNCH(128) break;
+    }
+#undef GPTQ_RTN_LAUNCH
+    count_launches();
+    return launch_status();
+}

@@ -1,0 +1,260 @@
+"""Thin Python binding of libgptq.so (include/gptq.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+torch is used for device memory and the current stream.  The functions carry
+the names of the C entry points; each checks dtypes/devices/contiguity,
+allocates outputs and workspace with torch when they are not given, passes
+raw pointers and sizes, and raises GptqError on a non-zero status.
+
+There is no CPU fallback: if libgptq.so is missing or cannot be loaded, the
+first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgptq.so")
+
+GPTQ_DTYPE_F32 = 0
+GPTQ_DTYPE_F16 = 1
+
+_STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_SHAPE", 3: "GPTQ_ERR_NOT_PD",
+           4: "GPTQ_ERR_UNSUPPORTED", 5: "GPTQ_ERR_CUDA", 6: "GPTQ_ERR_TIMEOUT"}
+
+# every symbol include/gptq.h declares
+EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
+            "gptq_hessian_accumulate",
+            "gptq_prepare_workspace_bytes", "gptq_prepare_hinv",
+            "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_pack_int4",
+            "gptq_unpack_int4", "rtn_quantize")
+
+
+class GptqError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {_STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libgptq.so (raises OSError when it is missing: no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"libgptq.so not found at {path}; build it with "
+                      f"`python -m post_weight_quantization_11_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I64, I32, F32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    SZ = ctypes.c_size_t
+    sig = {
+        "gptq_status_string": ([I32], ctypes.c_char_p),
+        "gptq_abi_version": ([], I32),
+        "gptq_debug_launch_count": ([], ctypes.c_uint64),
+        "gptq_hessian_accumulate": ([P, P, I64, I64, P, P], I32),
+        "gptq_prepare_workspace_bytes": ([I64], SZ),
+        "gptq_prepare_hinv": ([P, I64, I64, F32, I32, P, P, P, P, SZ, P], I32),
+        "gptq_quantize_workspace_bytes": ([I64, I64, I32], SZ),
+        "gptq_quantize_layer": ([P, I32, I64, I64, P, P, I32, I32, I32, P, P, P, P, P, SZ, P],
+                                I32),
+        "gptq_pack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
+        "gptq_unpack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
+        "rtn_quantize": ([P, I32, I64, I64, I32, I32, P, P, P, P], I32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise GptqError(fn, status)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _wdtype(W: torch.Tensor) -> int:
+    if W.dtype == torch.float16:
+        return GPTQ_DTYPE_F16
+    if W.dtype == torch.float32:
+        return GPTQ_DTYPE_F32
+    raise ValueError("W must be float16 or float32")
+
+
+# --------------------------------------------------------------------------
+# Entry points
+# --------------------------------------------------------------------------
+
+def gptq_abi_version() -> int:
+    return int(load_library().gptq_abi_version())
+
+
+def gptq_debug_launch_count() -> int:
+    return int(load_library().gptq_debug_launch_count())
+
+
+def gptq_status_string(status: int) -> str:
+    return load_library().gptq_status_string(int(status)).decode()
+
+
+def gptq_hessian_accumulate(S: torch.Tensor, X: torch.Tensor) -> int:
+    """S (d x d fp32, upper triangle) += X^T X for X (n x d fp16). Returns n."""
+    _need(S, "S", torch.float32)
+    _need(X, "X", torch.float16)
+    n, d = X.shape
+    if S.shape != (d, d):
+        raise ValueError("S must be d x d")
+    _check("gptq_hessian_accumulate",
+           load_library().gptq_hessian_accumulate(_ptr(S), _ptr(X), n, d, None, _stream(S)))
+    return n
+
+
+def gptq_prepare_workspace_bytes(d: int) -> int:
+    return int(load_library().gptq_prepare_workspace_bytes(int(d)))
+
+
+def gptq_prepare_hinv(S: torch.Tensor, n_tokens: int, damp_rel: float = 0.01,
+                      act_order: bool = False, perm=None, U=None, info=None, ws=None):
+    """Returns (perm int32 d, U fp32 d x d, info int32[1] device)."""
+    _need(S, "S", torch.float32)
+    d = S.shape[0]
+    dev = S.device
+    perm = torch.empty(d, dtype=torch.int32, device=dev) if perm is None else perm
+    U = torch.empty(d, d, dtype=torch.float32, device=dev) if U is None else U
+    info = torch.zeros(1, dtype=torch.int32, device=dev) if info is None else info
+    nb = gptq_prepare_workspace_bytes(d)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev) if ws is None else ws
+    for t, nm in ((perm, "perm"), (U, "U"), (info, "info"), (ws, "ws")):
+        _need(t, nm)
+    _check("gptq_prepare_hinv",
+           load_library().gptq_prepare_hinv(_ptr(S), d, int(n_tokens), float(damp_rel),
+                                            int(bool(act_order)), _ptr(perm), _ptr(U), _ptr(info),
+                                            _ptr(ws), ws.numel() * ws.element_size(), _stream(S)))
+    return perm, U, info
+
+
+def gptq_quantize_workspace_bytes(d_out: int, d_in: int, block_size: int = 128) -> int:
+    return int(load_library().gptq_quantize_workspace_bytes(int(d_out), int(d_in),
+                                                            int(block_size)))
+
+
+def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm=None, bits: int = 4,
+                        group_size: int = 128, block_size: int = 128, codes=None, scales=None,
+                        zeros=None, row_loss=None, ws=None):
+    """Returns (codes uint8 m x d, scales fp16 m x G, zeros uint8 m x G, row_loss fp32 m)."""
+    _need(W, "W")
+    _need(U, "U", torch.float32)
+    m, d = W.shape
+    dev = W.device
+    G = d // group_size
+    codes = torch.empty(m, d, dtype=torch.uint8, device=dev) if codes is None else codes
+    scales = torch.empty(m, G, dtype=torch.float16, device=dev) if scales is None else scales
+    zeros = torch.empty(m, G, dtype=torch.uint8, device=dev) if zeros is None else zeros
+    row_loss = torch.empty(m, dtype=torch.float32, device=dev) if row_loss is None else row_loss
+    nb = gptq_quantize_workspace_bytes(m, d, block_size)
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev) if ws is None else ws
+    if perm is not None:
+        _need(perm, "perm", torch.int32)
+    _check("gptq_quantize_layer",
+           load_library().gptq_quantize_layer(_ptr(W), _wdtype(W), m, d, _ptr(U), _ptr(perm),
+                                              int(bits), int(group_size), int(block_size),
+                                              _ptr(codes), _ptr(scales), _ptr(zeros),
+                                              _ptr(row_loss), _ptr(ws),
+                                              ws.numel() * ws.element_size(), _stream(W)))
+    return codes, scales, zeros, row_loss
+
+
+def gptq_pack_int4(codes: torch.Tensor, zeros: torch.Tensor, qweight=None, qzeros=None):
+    _need(codes, "codes", torch.uint8)
+    _need(zeros, "zeros", torch.uint8)
+    m, d = codes.shape
+    G = zeros.shape[1]
+    dev = codes.device
+    qweight = torch.empty(m, d // 8, dtype=torch.int32, device=dev) if qweight is None else qweight
+    qzeros = torch.empty(m, (G + 1) // 2, dtype=torch.uint8, device=dev) if qzeros is None else qzeros
+    _check("gptq_pack_int4",
+           load_library().gptq_pack_int4(_ptr(codes), _ptr(zeros), m, d, G, _ptr(qweight),
+                                         _ptr(qzeros), _stream(codes)))
+    return qweight, qzeros
+
+
+def gptq_unpack_int4(qweight: torch.Tensor, qzeros: torch.Tensor, d_in: int, n_groups: int):
+    _need(qweight, "qweight")
+    _need(qzeros, "qzeros", torch.uint8)
+    m = qweight.shape[0]
+    dev = qweight.device
+    codes = torch.empty(m, d_in, dtype=torch.uint8, device=dev)
+    zeros = torch.empty(m, n_groups, dtype=torch.uint8, device=dev)
+    _check("gptq_unpack_int4",
+           load_library().gptq_unpack_int4(_ptr(qweight), _ptr(qzeros), m, d_in, n_groups,
+                                           _ptr(codes), _ptr(zeros), _stream(qweight)))
+    return codes, zeros
+
+
+def rtn_quantize(W: torch.Tensor, bits: int = 4, group_size: int = 128):
+    _need(W, "W")
+    m, d = W.shape
+    dev = W.device
+    G = d // group_size
+    codes = torch.empty(m, d, dtype=torch.uint8, device=dev)
+    scales = torch.empty(m, G, dtype=torch.float16, device=dev)
+    zeros = torch.empty(m, G, dtype=torch.uint8, device=dev)
+    _check("rtn_quantize",
+           load_library().rtn_quantize(_ptr(W), _wdtype(W), m, d, int(bits), int(group_size),
+                                       _ptr(codes), _ptr(scales), _ptr(zeros), _stream(W)))
+    return codes, scales, zeros
+
+
+# --------------------------------------------------------------------------
+# Whole layer (the four calls in order)
+# --------------------------------------------------------------------------
+
+class LayerResult:
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def quantize_layer_from_inputs(W: torch.Tensor, X_batches, bits: int = 4, group_size: int = 128,
+                               damp_rel: float = 0.01, act_order: bool = False,
+                               pack: bool = True) -> LayerResult:
+    """GPTQ on one layer: accumulate S over the calibration batches, prepare U,
+    sweep, and pack.  X_batches: a CUDA fp16 tensor (n x d) or an iterable of them."""
+    m, d = W.shape
+    S = torch.zeros(d, d, dtype=torch.float32, device=W.device)
+    n = 0
+    if isinstance(X_batches, torch.Tensor):
+        X_batches = [X_batches]
+    for X in X_batches:
+        n += gptq_hessian_accumulate(S, X)
+    perm, U, info = gptq_prepare_hinv(S, n, damp_rel, act_order)
+    codes, scales, zeros, row_loss = gptq_quantize_layer(
+        W, U, perm if act_order else None, bits, group_size)
+    res = LayerResult(S=S, n=n, perm=perm, U=U, info=info, codes=codes, scales=scales,
+                      zeros=zeros, row_loss=row_loss)
+    if pack and bits == 4:
+        res.qweight, res.qzeros = gptq_pack_int4(codes, zeros)
+    return res

@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+symbol include/gptq.h declares, and rejects bad arguments before launching
+anything (every call below returns during validation)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_weight_quantization_11_b200 import gptq as G
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "gptq.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|uint64_t|char\s*\*|void)\s*\**\s*(\w+)\s*\(", txt,
+                       flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from post_weight_quantization_11_b200 import build
+    build.build()
+    return G.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 10
+    assert sorted(names) == sorted(G.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+    out = os.popen(f"nm -D --defined-only {G.LIB_PATH}").read()
+    for n in names:
+        assert re.search(rf"\bT {n}\b", out), n
+
+
+def test_status_strings_and_version(lib):
+    assert G.gptq_abi_version() == 100
+    for code, name in G._STATUS.items():
+        assert G.gptq_status_string(code) == name
+    assert G.gptq_status_string(99) == "GPTQ_ERR_UNKNOWN"
+    assert G.gptq_debug_launch_count() >= 0
+
+
+def test_workspace_sizes(lib):
+    for d in (128, 256, 4096, 14336):
+        b = G.gptq_prepare_workspace_bytes(d)
+        assert b >= 2 * 4 * d * d and b % 256 == 0
+    for m, d in ((1, 128), (300, 256), (4096, 4096), (14336, 4096)):
+        b = G.gptq_quantize_workspace_bytes(m, d, 128)
+        assert b >= 4 * m * d + 4 * m * 128
+    assert G.gptq_quantize_workspace_bytes(64, 256, 64) == 0
+    assert G.gptq_prepare_workspace_bytes(0) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)          # 16-byte aligned, never dereferenced
+MIS = ctypes.c_void_p((1 << 20) + 4)     # misaligned
+
+
+def test_validation_rejects_before_launch(lib):
+    n0 = ctypes.c_int64(0)
+    # null / misaligned pointers
+    assert lib.gptq_hessian_accumulate(None, FAKE, 10, 256, None, None) == 1
+    assert lib.gptq_hessian_accumulate(MIS, FAKE, 10, 256, None, None) == 1
+    # shapes
+    assert lib.gptq_hessian_accumulate(FAKE, FAKE, 10, 200, None, None) == 2
+    assert lib.gptq_hessian_accumulate(FAKE, FAKE, -1, 256, None, None) == 2
+    assert lib.gptq_hessian_accumulate(FAKE, FAKE, 10, 64, None, None) == 2
+    # n_tokens == 0 is a no-op that still counts nothing
+    assert lib.gptq_hessian_accumulate(FAKE, FAKE, 0, 256, ctypes.byref(n0), None) == 0
+    assert n0.value == 0
+    ws = G.gptq_prepare_workspace_bytes(256)
+    assert lib.gptq_prepare_hinv(FAKE, 256, 0, 0.01, 0, None, FAKE, FAKE, FAKE, ws, None) == 2
+    assert lib.gptq_prepare_hinv(FAKE, 256, 10, 0.01, 1, None, FAKE, FAKE, FAKE, ws, None) == 1
+    assert lib.gptq_prepare_hinv(FAKE, 256, 10, -1.0, 0, None, FAKE, FAKE, FAKE, ws, None) == 1
+    assert lib.gptq_prepare_hinv(FAKE, 256, 10, 0.01, 0, None, FAKE, FAKE, FAKE, 16, None) == 1
+    assert lib.gptq_prepare_hinv(FAKE, 300, 10, 0.01, 0, None, FAKE, FAKE, FAKE, ws, None) == 2
+    wq = G.gptq_quantize_workspace_bytes(64, 256, 128)
+    args = lambda **k: dict(dict(W=FAKE, dt=1, m=64, d=256, U=FAKE, perm=None, bits=4, g=128,
+                                 B=128, codes=FAKE, scales=FAKE, zeros=FAKE, loss=None, ws=FAKE,
+                                 wsb=wq), **k)
+
+    def q(**k):
+        a = args(**k)
+        return lib.gptq_quantize_layer(a["W"], a["dt"], a["m"], a["d"], a["U"], a["perm"],
+                                       a["bits"], a["g"], a["B"], a["codes"], a["scales"],
+                                       a["zeros"], a["loss"], a["ws"], a["wsb"], None)
+    assert q(bits=5) == 4
+    assert q(g=96) == 4
+    assert q(B=64) == 4
+    assert q(dt=7) == 1
+    assert q(d=200) == 2
+    assert q(m=0) == 2
+    assert q(W=None) == 1
+    assert q(U=MIS) == 1
+    assert q(wsb=100) == 1
+    assert lib.rtn_quantize(FAKE, 1, 64, 256, 3, 48, FAKE, FAKE, FAKE, None) == 4
+    assert lib.rtn_quantize(None, 1, 64, 256, 4, 128, FAKE, FAKE, FAKE, None) == 1
+    assert lib.gptq_pack_int4(FAKE, FAKE, 4, 12, 1, FAKE, FAKE, None) == 2
+    assert lib.gptq_pack_int4(FAKE, FAKE, 4, 16, 0, FAKE, FAKE, None) == 2
+    assert lib.gptq_unpack_int4(FAKE, FAKE, 0, 16, 1, FAKE, FAKE, None) == 2

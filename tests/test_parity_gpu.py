@@ -1,0 +1,192 @@
+"""GPU parity: the CUDA path (through the C ABI binding) against the float64
+oracle on the same seeded inputs.  Tolerances are stated in tests/parity.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_weight_quantization_11_b200 import gptq as G
+from post_weight_quantization_11_b200 import inputs
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from post_weight_quantization_11_b200 import build
+    build.build()
+    G.load_library()
+
+
+def _gauss_x(n, d, n_out, fac, seed):
+    spec = inputs.LayerSpec("t", 1, d, 0.02, "fp16", n, "gauss", n_out, fac, fac, False, seed)
+    return inputs.calibration_x(spec, device="cpu")
+
+
+def _weights(m, d, dtype, seed, std=0.02):
+    spec = inputs.LayerSpec("t", m, d, std, "fp32" if dtype == torch.float32 else "fp16", 1,
+                            "gauss", 0, 1, 1, False, seed)
+    return inputs.weights(spec, device="cpu")
+
+
+def _gpu_layer(W, X, bits=4, group_size=128, act_order=False, damp=0.01):
+    Wd, Xd = W.to(DEV), X.to(DEV)
+    d = W.shape[1]
+    S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    G.gptq_hessian_accumulate(S, Xd)
+    perm, U, info = G.gptq_prepare_hinv(S, X.shape[0], damp, act_order)
+    codes, scales, zeros, loss = G.gptq_quantize_layer(Wd, U, perm if act_order else None,
+                                                       bits, group_size)
+    torch.cuda.synchronize()
+    return dict(S=P.to_np(S), perm=P.to_np(perm), U=P.to_np(U), info=int(info.item()),
+                codes=P.to_np(codes), scales=P.to_np(scales), zeros=P.to_np(zeros),
+                row_loss=P.to_np(loss))
+
+
+def _check_layer(W, X, bits=4, group_size=128, act_order=False, rows=None):
+    """H-forced protocol: the oracle takes the GPU's S (promoted to fp64)."""
+    n = X.shape[0]
+    g = _gpu_layer(W, X, bits, group_size, act_order)
+    assert g["info"] == 0
+    S_or = oracle.hessian(X.numpy())
+    S_gpu = P.mirror_upper(g["S"])
+    assert P.rel_fro(S_gpu, S_or) <= P.S_TOL
+    W64 = W.double().numpy()
+    ref = oracle.gptq_layer(W64, S_gpu, n, bits, group_size, 0.01, act_order)
+    assert np.array_equal(g["perm"], ref["perm"]) if act_order else True
+    assert P.rel_fro(g["U"].astype(np.float64), ref["U"]) <= P.U_TOL
+    st = P.compare_sweep(g, dict(codes=ref["codes"], scales=ref["scales"], zeros=ref["zeros"],
+                                 s_pre=ref["s_pre"]), group_size)
+    H64 = 2.0 * S_gpu / n
+    perm = ref["perm"]
+    lg = P.layer_loss_of(W64, g["codes"], g["scales"], g["zeros"], group_size, perm, H64)
+    lo = P.layer_loss_of(W64, ref["codes"], ref["scales"], ref["zeros"], group_size, perm, H64)
+    assert abs(lg - lo) <= P.LOSS_REL * lo, (lg, lo)
+    # the GPU's own bookkeeping: sum E_j^2 = tr(D Hd D^T)
+    assert abs(g["row_loss"].sum() - ref["row_loss"].sum()) <= P.LOSS_REL * ref["row_loss"].sum()
+    Wp = np.ascontiguousarray(W64[:, perm])
+    n_ties = P.teacher_forced_check(Wp, ref["U"], g, bits, group_size, rows)
+    st.update(loss_gpu=lg, loss_oracle=lo, teacher_forced_ties=n_ties)
+    return st, g, ref
+
+
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,gs", [(4, 128), (4, 64), (3, 32), (2, 128), (8, 64)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16])
+def test_rtn_bit_exact(bits, gs, dtype):
+    W = _weights(300, 384, dtype, 3)
+    W[5, :] = 0                       # an all-zero row: degenerate groups
+    W[7, :128] = -0.01                # one-signed group
+    c, s, z = G.rtn_quantize(W.to(DEV), bits, gs)
+    ref = oracle.rtn(W.double().numpy(), bits, gs)
+    assert np.array_equal(P.to_np(c), ref["codes"])
+    assert np.array_equal(P.to_np(s), ref["scales"])
+    assert np.array_equal(P.to_np(z), ref["zeros"])
+
+
+@pytest.mark.parametrize("m,d,G_", [(1, 128, 1), (300, 1024, 8), (77, 256, 3), (5, 8, 1)])
+def test_pack_bit_exact(m, d, G_):
+    rng = np.random.default_rng(m + d)
+    codes = rng.integers(0, 16, (m, d), dtype=np.uint8)
+    zeros = rng.integers(0, 16, (m, G_), dtype=np.uint8)
+    qw, qz = G.gptq_pack_int4(torch.from_numpy(codes).to(DEV), torch.from_numpy(zeros).to(DEV))
+    rq, rz = oracle.pack_int4(codes, zeros)
+    assert np.array_equal(P.to_np(qw).view(np.uint32), rq)
+    assert np.array_equal(P.to_np(qz), rz)
+    c2, z2 = G.gptq_unpack_int4(qw, qz, d, G_)
+    assert np.array_equal(P.to_np(c2), codes) and np.array_equal(P.to_np(z2), zeros)
+
+
+@pytest.mark.parametrize("n,d", [(512, 256), (777, 384), (64, 128), (4099, 1024)])
+def test_hessian_parity(n, d):
+    X = _gauss_x(n, d, 3, 50.0, d + n)
+    S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    S.fill_(0)
+    Xd = X.to(DEV)
+    # two batches accumulate into the same S
+    G.gptq_hessian_accumulate(S, Xd[: n // 3])
+    G.gptq_hessian_accumulate(S, Xd[n // 3:])
+    G.gptq_hessian_accumulate(S, Xd[:0])  # empty batch: no-op
+    Sg = P.to_np(S)
+    ref = oracle.hessian(X.numpy())
+    assert P.rel_fro(np.triu(Sg.astype(np.float64)), np.triu(ref)) <= P.S_TOL
+    assert np.all(np.tril(Sg, -1) == 0)   # lower triangle untouched
+
+
+@pytest.mark.parametrize("act_order", [False, True])
+def test_prepare_parity(act_order):
+    n, d = 2048, 512
+    X = _gauss_x(n, d, 5, 40.0, 11)
+    S = torch.from_numpy(oracle.hessian(X.numpy()).astype(np.float32)).to(DEV)
+    perm, U, info = G.gptq_prepare_hinv(S, n, 0.01, act_order)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    S64 = P.mirror_upper(P.to_np(S))
+    H, Hd, rperm, lam, st = oracle.finalize(S64, n, 0.01, act_order)
+    U64, inf = oracle.hinv_upper_chol(Hd)
+    assert np.array_equal(P.to_np(perm), rperm)
+    Ug = P.to_np(U).astype(np.float64)
+    assert np.all(np.tril(Ug, -1) == 0)
+    assert P.rel_fro(Ug, U64) <= P.U_TOL
+
+
+def test_prepare_reports_non_pd():
+    d = 256
+    S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    _, _, info = G.gptq_prepare_hinv(S, 100, 0.01, False)
+    torch.cuda.synchronize()
+    assert int(info.item()) != 0
+
+
+def test_tiny_layer_end_to_end():
+    """The tiny workload: W 256x256 fp32, X 512x256 fp16 with 3 outlier channels x50."""
+    wl = inputs.WORKLOADS["tiny"]
+    spec = wl.layers[0]
+    W = inputs.weights(spec)
+    X = inputs.calibration_x(spec)
+    st, g, ref = _check_layer(W, X, 4, 128)
+    # against the oracle's OWN Hessian as well (end to end)
+    S_or = oracle.hessian(X.numpy())
+    own = oracle.gptq_layer(W.double().numpy(), S_or, X.shape[0], 4, 128)
+    H64 = 2.0 * S_or / X.shape[0]
+    lg = P.layer_loss_of(W.double().numpy(), g["codes"], g["scales"], g["zeros"], 128, None, H64)
+    lo = P.layer_loss_of(W.double().numpy(), own["codes"], own["scales"], own["zeros"], 128, None,
+                         H64)
+    assert abs(lg - lo) <= P.LOSS_REL * lo
+    # GPTQ beats RTN on this outlier workload
+    r = oracle.rtn(W.double().numpy(), 4, 128)
+    lr = P.layer_loss_of(W.double().numpy(), r["codes"], r["scales"], r["zeros"], 128, None, H64)
+    assert lg < lr
+    print("tiny:", st)
+
+
+@pytest.mark.parametrize("m,d,n,bits,gs,act,dtype", [
+    (1, 128, 300, 4, 128, False, torch.float16),      # single row, single block
+    (300, 256, 700, 4, 128, False, torch.float16),    # ragged rows and tokens
+    (129, 384, 1000, 3, 64, True, torch.float32),     # act-order, 3-bit, g64
+    (64, 512, 1500, 2, 32, False, torch.float16),     # 2-bit, g32
+    (1000, 1024, 4096, 4, 128, False, torch.float16), # several tiles in every dimension
+])
+def test_layer_parity_cases(m, d, n, bits, gs, act, dtype):
+    W = _weights(m, d, dtype, m + d)
+    X = _gauss_x(n, d, max(1, d // 100), 30.0, n + d)
+    st, _, _ = _check_layer(W, X, bits, gs, act)
+    print((m, d, n, bits, gs, act), st)
+
+
+def test_pack_of_gptq_result_matches_storage_format():
+    wl = inputs.WORKLOADS["tiny"]
+    spec = wl.layers[0]
+    W, X = inputs.weights(spec).to(DEV), inputs.calibration_x(spec).to(DEV)
+    res = G.quantize_layer_from_inputs(W, X, 4, 128)
+    torch.cuda.synchronize()
+    qw, qz = P.to_np(res.qweight).view(np.uint32), P.to_np(res.qzeros)
+    rq, rz = oracle.pack_int4(P.to_np(res.codes), P.to_np(res.zeros))
+    assert np.array_equal(qw, rq) and np.array_equal(qz, rz)
+    m, d = W.shape
+    nbytes = qw.nbytes + qz.nbytes + res.scales.numel() * 2
+    assert nbytes == 66.5 * m * d / 128
