@@ -60,6 +60,12 @@ int gptq_abi_version(void);
  * library so far (all devices, all calls).  Host-only, never synchronizes. */
 uint64_t gptq_debug_launch_count(void);
 
+/* Device status of the current device: 0, or the code a bounded device-side
+ * wait recorded when it gave up (the kernel then returned early and its
+ * outputs are invalid).  Synchronous (reads a device word); reset != 0 clears
+ * it.  Returns GPTQ_OK or GPTQ_ERR_CUDA / GPTQ_ERR_INVALID_ARG. */
+int gptq_device_status(int32_t* status_out, int reset);
+
 /*
  * Hessian accumulation -- "GPTQ / AWQ / SqueezeLLM" sec. 一 (H from the
  * calibration inputs; the 2/n factor is applied later by gptq_prepare_hinv).

@@ -22,7 +22,8 @@ LIB = os.path.join(PKG, "libgptq.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-Xcompiler", "-fPIC",
+         "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]
 
 
@@ -64,7 +65,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
             if log.strip():
                 print(log)
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + [o for o, _ in results] + ["-lcudart"]
+    cmd = [NVCC] + ARCH + ["-shared", "-rdc=true", "-o", tmp] + [o for o, _ in results] + \
+        ["-lcudart"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

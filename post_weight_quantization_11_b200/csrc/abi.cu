@@ -1,9 +1,38 @@
 // Library-wide C entry points: status names, ABI version, launch counter.
 #include <atomic>
 
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace gptq {
+
+__device__ int g_device_status = 0;
+
+int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swz)
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !p)
+            return GPTQ_ERR_CUDA;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
 
 static std::atomic<unsigned long long> g_launches{0};
 
@@ -28,3 +57,18 @@ extern "C" const char* gptq_status_string(int status)
 extern "C" int gptq_abi_version(void) { return GPTQ_ABI_VERSION; }
 
 extern "C" uint64_t gptq_debug_launch_count(void) { return gptq::g_launches.load(); }
+
+extern "C" int gptq_device_status(int32_t* status_out, int reset)
+{
+    if (!status_out) return GPTQ_ERR_INVALID_ARG;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, gptq::g_device_status, sizeof(int)) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    *status_out = v;
+    if (reset && v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(gptq::g_device_status, &zero, sizeof(int)) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+    }
+    return GPTQ_OK;
+}

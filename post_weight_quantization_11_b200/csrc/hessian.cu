@@ -1,67 +1,220 @@
 // Hessian accumulation S += X^T X (upper triangle) -- "GPTQ / AWQ /
 // SqueezeLLM" sec. 一 (H from the calibration inputs).
 //
-// First version: CUDA-core fp32 FMA of fp16 inputs, 64x64 upper tiles,
-// token range split across grid.y with fp32 atomic accumulation.
+// sm_100a design: 5th-generation tensor cores, fp16 x fp16 -> fp32.
+//  * Output tiles of 128 (rows i) x 256 (columns j) covering the upper
+//    triangle; the work items are (token split, tile) pairs handed out
+//    round-robin to one persistent CTA per SM.  Items of one round share the
+//    same token window, so concurrently running CTAs re-read X from L2.
+//  * X is token-major (n x d), so both operands of S = X^T X are "MN-major":
+//    a TMA box of 64 features x 64 tokens (128-byte swizzle) is exactly one
+//    canonical MN-major atom column; A = X[t, i0:i0+128] (2 boxes) and
+//    B = X[t, j0:j0+256] (4 boxes) per 64-token stage, 4 stages.
+//  * warp 0 issues TMA, warp 1 issues tcgen05.mma (M=128, N=256, K=16).
+//  * Accuracy: the tensor core's fp32 accumulator loses low-order bits on
+//    every accumulate (measured: about 1.5e-3 relative after 262144 tokens in
+//    one accumulator).  So a TMEM accumulator only ever sums one chunk of 512
+//    tokens (32 MMAs); eight epilogue warps (warps 2-9, two per TMEM lane
+//    quarter, 128 columns each) fold every chunk into fp32 registers with
+//    round-to-nearest adds while the MMAs fill the other of two TMEM
+//    accumulators, and add the item's sum into S with vector atomics.
+//  * Every mbarrier wait is bounded (see tc_common.cuh).
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace gptq {
 
-constexpr int HS_B = 64, HS_BK = 32;
+constexpr int HB_M = 128, HB_N = 256, HB_K = 64, HB_STAGES = 4;
+constexpr int HB_A_BYTES = HB_M * HB_K * 2;                 // 16 KB
+constexpr int HB_B_BYTES = HB_N * HB_K * 2;                 // 32 KB
+constexpr int HB_STAGE_BYTES = HB_A_BYTES + HB_B_BYTES;     // 48 KB
+constexpr int HB_THREADS = 320;
+constexpr int HB_EPI_THREADS = 256;
+constexpr int HB_CHUNK = 512;                                // tokens per TMEM accumulation
+constexpr int HB_SMEM = HB_STAGES * HB_STAGE_BYTES + 1024 + 256;
+constexpr uint32_t HB_IDESC = make_idesc(0 /*f16*/, HB_M, HB_N, 1 /*A MN-major*/, 1 /*B MN*/);
+constexpr uint32_t HB_TMEM_COLS = 512;
 
-__global__ void __launch_bounds__(256)
-hessian_simt_kernel(float* __restrict__ S, const __half* __restrict__ X, int64_t n, int64_t d,
-                    int64_t tokens_per_split)
+struct SyrkParams {
+    float* S;
+    int64_t d, n;
+    int64_t per;      // tokens per split (multiple of 64)
+    int nbi;          // row blocks of 128
+    int tiles;        // upper-triangle tiles
+    int items;        // tiles * splits
+};
+
+// Tiles are enumerated column-block-major: column block bj (256 wide) holds
+// row blocks bi = 0 .. 2 bj + 1 (the last one possibly truncated to nbi).
+__device__ __forceinline__ void tile_coords(int t, int& bi, int& bj)
 {
-    const int nb = (int)(d / HS_B);
-    const int bi = blockIdx.x / nb, bj = blockIdx.x % nb;
-    if (bi > bj) return;
-    const int64_t t_begin = int64_t(blockIdx.y) * tokens_per_split;
-    const int64_t t_end = min(n, t_begin + tokens_per_split);
-    if (t_begin >= t_end) return;
-    __shared__ __align__(16) float As[HS_BK][HS_B + 4];
-    __shared__ __align__(16) float Bs[HS_BK][HS_B + 4];
-    const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
-    const int64_t i0 = int64_t(bi) * HS_B, j0 = int64_t(bj) * HS_B;
-    float acc[4][4] = {};
-    for (int64_t t0 = t_begin; t0 < t_end; t0 += HS_BK) {
-        // 32 tokens x 64 features per operand: 256 threads x 8 halves
-        int r = tid / 8, c8 = (tid % 8) * 8;
-        int64_t t = t0 + r;
-        __half2 va[4], vb[4];
-        if (t < t_end) {
-            uint4 ua = *reinterpret_cast<const uint4*>(X + t * d + i0 + c8);
-            uint4 ub = *reinterpret_cast<const uint4*>(X + t * d + j0 + c8);
-            memcpy(va, &ua, 16);
-            memcpy(vb, &ub, 16);
-        } else {
-            for (int q = 0; q < 4; ++q) { va[q] = __float2half2_rn(0.f); vb[q] = va[q]; }
-        }
-        for (int q = 0; q < 4; ++q) {
-            float2 fa = __half22float2(va[q]), fb = __half22float2(vb[q]);
-            As[r][c8 + 2 * q] = fa.x; As[r][c8 + 2 * q + 1] = fa.y;
-            Bs[r][c8 + 2 * q] = fb.x; Bs[r][c8 + 2 * q + 1] = fb.y;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int k = 0; k < HS_BK; ++k) {
-            float4 a = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
-            float4 b = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
-            float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
-        }
-        __syncthreads();
+    int b = (int)((sqrtf(4.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while ((b + 1) * (b + 2) <= t) ++b;
+    while (b > 0 && b * (b + 1) > t) --b;
+    bj = b;
+    bi = t - b * (b + 1);
+}
+
+__global__ void __launch_bounds__(HB_THREADS, 1)
+hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, const SyrkParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + HB_STAGES * HB_STAGE_BYTES);
+    uint64_t* empty_bar = full_bar + HB_STAGES;
+    uint64_t* accf_bar = empty_bar + HB_STAGES;
+    uint64_t* acce_bar = accf_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + 2);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < HB_STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&accf_bar[a], 1); mbar_init(&acce_bar[a], HB_EPI_THREADS); }
+        *abort = 0;
+        fence_mbar_init();
     }
-    for (int p = 0; p < 4; ++p) {
-        int64_t gi = i0 + ty * 4 + p;
-        for (int q = 0; q < 4; ++q) {
-            int64_t gj = j0 + tx * 4 + q;
-            if (gi <= gj) atomicAdd(S + gi * d + gj, acc[p][q]);
+    if (warp == 1) tmem_alloc(tmem_slot, HB_TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int P = gridDim.x;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmX);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0, armed_par = 0;   // per-stage: armed at least once / last parity
+            bool ok = true;
+            for (int q = blockIdx.x; q < p.items && ok; q += P) {
+                const int s = q / p.tiles, t = q - s * p.tiles;
+                int bi, bj;
+                tile_coords(t, bi, bj);
+                const int64_t t0 = int64_t(s) * p.per, t1 = min(p.n, t0 + p.per);
+                for (int64_t k = t0; k < t1; k += HB_K) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, kErrWaitEmpty, abort)) { ok = false; break; }
+                    uint8_t* sa = smem + stage * HB_STAGE_BYTES;
+                    uint8_t* sb = sa + HB_A_BYTES;
+                    mbar_arrive_expect_tx(&full_bar[stage], HB_STAGE_BYTES);
+                    tma_load_2d(sa, &tmX, &full_bar[stage], bi * HB_M, (int)k);
+                    tma_load_2d(sa + 8192, &tmX, &full_bar[stage], bi * HB_M + 64, (int)k);
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        tma_load_2d(sb + h * 8192, &tmX, &full_bar[stage], bj * HB_N + 64 * h, (int)k);
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == HB_STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            // every copy this thread issued has landed before the CTA exits
+            for (int s = 0; s < HB_STAGES; ++s)
+                if (armed & (1u << s)) mbar_drain(&full_bar[s], (armed_par >> s) & 1u);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0, ch = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int q = blockIdx.x; q < p.items && ok; q += P) {
+                const int s = q / p.tiles;
+                const int64_t t0 = int64_t(s) * p.per, t1 = min(p.n, t0 + p.per);
+                for (int64_t c0 = t0; c0 < t1 && ok; c0 += HB_CHUNK, ++ch) {
+                    const int64_t c1 = min(t1, c0 + HB_CHUNK);
+                    const int a = ch & 1;
+                    const uint32_t aph = (ch >> 1) & 1;
+                    if (!mbar_wait(&acce_bar[a], aph ^ 1, kErrWaitAccEmpty, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem + uint32_t(a * HB_N);
+                    uint32_t acc = 0;
+                    for (int64_t k = c0; k < c1; k += HB_K) {
+                        if (!mbar_wait(&full_bar[stage], phase, kErrWaitFull, abort)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t sa = smem_u32(smem + stage * HB_STAGE_BYTES);
+                        const uint32_t sb = sa + HB_A_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < HB_K / 16; ++kk) {
+                            const uint64_t da = smem_desc_sw128(sa + kk * 2048, 8192, 1024);
+                            const uint64_t db = smem_desc_sw128(sb + kk * 2048, 8192, 1024);
+                            mma_f16(d_tmem, da, db, HB_IDESC, acc);
+                            acc = 1;
+                        }
+                        mma_commit(&empty_bar[stage]);
+                        if (++stage == HB_STAGES) { stage = 0; phase ^= 1; }
+                    }
+                    mma_commit(&accf_bar[a]);
+                }
+            }
+        }
+    } else {
+        const int ew = warp - 2;                 // 0..7
+        const int qr = warp & 3;                 // TMEM lane quarter of this warp
+        const int half = ew >> 2;                // columns [128*half, 128*half + 128)
+        int ch = 0;
+        bool ok = true;
+        for (int q = blockIdx.x; q < p.items && ok; q += P) {
+            const int s = q / p.tiles, t = q - s * p.tiles;
+            int bi, bj;
+            tile_coords(t, bi, bj);
+            const int64_t t0 = int64_t(s) * p.per, t1 = min(p.n, t0 + p.per);
+            float sum[128];
+#pragma unroll
+            for (int u = 0; u < 128; ++u) sum[u] = 0.f;
+            for (int64_t c0 = t0; c0 < t1; c0 += HB_CHUNK, ++ch) {
+                const int a = ch & 1;
+                const uint32_t aph = (ch >> 1) & 1;
+                if (!mbar_wait(&accf_bar[a], aph, kErrWaitAccFull, abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t base = tmem + uint32_t(a * HB_N + half * 128) + (uint32_t(qr * 32) << 16);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(base + uint32_t(c * 32), v);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) sum[c * 32 + u] = __fadd_rn(sum[c * 32 + u], v[u]);
+                }
+                tc_fence_before();
+                mbar_arrive(&acce_bar[a]);
+            }
+            if (!ok) break;
+            const int64_t i = int64_t(bi) * HB_M + qr * 32 + lane;
+            float* Srow = p.S + i * p.d;
+            const int64_t jb = int64_t(bj) * HB_N + half * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int64_t j0 = jb + c * 32;
+                if (j0 >= p.d || j0 + 31 < i) continue;
+#pragma unroll
+                for (int u = 0; u < 32; u += 4) {
+                    const int64_t j = j0 + u;
+                    const float* v = sum + c * 32 + u;
+                    if (j >= i) {
+                        atomicAdd(reinterpret_cast<float4*>(Srow + j),
+                                  make_float4(v[0], v[1], v[2], v[3]));
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (j + e >= i) atomicAdd(Srow + j + e, v[e]);
+                    }
+                }
+            }
         }
     }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, HB_TMEM_COLS);
+    }
+}
+
+static int sm_count()
+{
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
 }
 
 }  // namespace gptq
@@ -72,17 +225,42 @@ extern "C" int gptq_hessian_accumulate(float* S, const uint16_t* X, int64_t n_to
     using namespace gptq;
     if (!S || (!X && n_tokens > 0)) return GPTQ_ERR_INVALID_ARG;
     if (!aligned16(S) || (X && !aligned16(X))) return GPTQ_ERR_INVALID_ARG;
-    if (d < 128 || d > kMaxDim || d % 128 != 0 || n_tokens < 0) return GPTQ_ERR_SHAPE;
+    if (d < 128 || d > kMaxDim || d % 128 != 0 || n_tokens < 0 || n_tokens > (int64_t(1) << 31))
+        return GPTQ_ERR_SHAPE;
     if (n_tokens == 0) return GPTQ_OK;
     cudaStream_t st = as_stream(stream);
-    const int nb = (int)(d / HS_B);
-    const int64_t tiles = int64_t(nb) * (nb + 1) / 2;
-    int64_t splits = ceil_div(4 * 148, tiles);
-    splits = std::max<int64_t>(1, std::min<int64_t>(splits, ceil_div(n_tokens, 1024)));
-    int64_t per = ceil_div(ceil_div(n_tokens, splits), HS_BK) * HS_BK;
-    splits = ceil_div(n_tokens, per);
-    dim3 grid((unsigned)(nb * nb), (unsigned)splits);
-    hessian_simt_kernel<<<grid, 256, 0, st>>>(S, reinterpret_cast<const __half*>(X), n_tokens, d, per);
+
+    SyrkParams p{};
+    p.S = S;
+    p.d = d;
+    p.n = n_tokens;
+    p.nbi = (int)(d / HB_M);
+    const int nbj = (int)ceil_div(d, HB_N);
+    p.tiles = (nbj - 1) * nbj + std::min(2 * nbj, p.nbi);
+    const int P = sm_count();
+    const int64_t ksteps = ceil_div(n_tokens, HB_K);
+    // smallest token split count whose round-robin over P CTAs is >= 90 % busy
+    int64_t best_s = 1;
+    double best_eff = 0.0;
+    for (int64_t s = 1; s <= std::min<int64_t>(ksteps, 64); ++s) {
+        const int64_t items = p.tiles * s;
+        const double eff = double(items) / double(ceil_div(items, P) * P);
+        if (eff > best_eff + 1e-9) { best_eff = eff; best_s = s; }
+        if (eff >= 0.9) { best_s = s; break; }
+    }
+    p.per = ceil_div(ksteps, best_s) * HB_K;
+    const int64_t splits = ceil_div(n_tokens, p.per);
+    p.items = (int)(p.tiles * splits);
+
+    CUtensorMap tm;
+    if (encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, (uint64_t)d, (uint64_t)n_tokens,
+                       (uint64_t)d * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK)
+        return GPTQ_ERR_CUDA;
+    if (cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             HB_SMEM) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    const int grid = std::min(p.items, P);
+    hessian_tc_kernel<<<grid, HB_THREADS, HB_SMEM, st>>>(tm, p);
     count_launches();
     int rc = launch_status();
     if (rc == GPTQ_OK && n_seen) *n_seen += n_tokens;

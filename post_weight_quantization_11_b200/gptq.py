@@ -27,6 +27,7 @@ _STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_SHAPE", 3: "GPT
 
 # every symbol include/gptq.h declares
 EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
+            "gptq_device_status",
             "gptq_hessian_accumulate",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_pack_int4",
@@ -57,6 +58,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_status_string": ([I32], ctypes.c_char_p),
         "gptq_abi_version": ([], I32),
         "gptq_debug_launch_count": ([], ctypes.c_uint64),
+        "gptq_device_status": ([P, I32], I32),
         "gptq_hessian_accumulate": ([P, P, I64, I64, P, P], I32),
         "gptq_prepare_workspace_bytes": ([I64], SZ),
         "gptq_prepare_hinv": ([P, I64, I64, F32, I32, P, P, P, P, SZ, P], I32),
@@ -115,6 +117,13 @@ def gptq_abi_version() -> int:
 
 def gptq_debug_launch_count() -> int:
     return int(load_library().gptq_debug_launch_count())
+
+
+def gptq_device_status(reset: bool = True) -> int:
+    """0, or the error code a bounded device-side wait recorded (synchronous)."""
+    v = ctypes.c_int32(0)
+    _check("gptq_device_status", load_library().gptq_device_status(ctypes.byref(v), int(reset)))
+    return int(v.value)
 
 
 def gptq_status_string(status: int) -> str:

@@ -1,0 +1,98 @@
+"""Full-size parity in the launch configuration bench.py times: the 7B
+attention projection (W 4096x4096 fp16, X 262144 x 4096 fp16 with 1 % outlier
+channels), one Hessian call over all tokens, prepare, sweep, pack.
+
+The oracle computes what it can at this size: a 96-column block of S (every
+token), the full float64 U from the GPU's S (the H-forced protocol), and the
+sweep of a seeded sample of rows (rows are independent given U).  Tolerances
+are those of tests/parity.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_weight_quantization_11_b200 import gptq as G
+from post_weight_quantization_11_b200 import inputs
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def attn7b():
+    from post_weight_quantization_11_b200 import build
+    build.build()
+    spec = inputs.WORKLOADS["attn7b"].layers[0]
+    W = inputs.weights(spec, device=DEV)
+    X = inputs.calibration_x(spec, device=DEV)
+    n = X.shape[0]
+    m, d = W.shape
+    S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    G.gptq_hessian_accumulate(S, X)
+    perm, U, info = G.gptq_prepare_hinv(S, n, 0.01, False)
+    codes, scales, zeros, loss = G.gptq_quantize_layer(W, U, None, 4, 128)
+    qw, qz = G.gptq_pack_int4(codes, zeros)
+    torch.cuda.synchronize()
+    assert G.gptq_device_status(reset=True) == 0
+    assert int(info.item()) == 0
+    ch, _ = inputs.outlier_channels(spec)
+    rng = np.random.default_rng(1234)
+    cols = np.unique(np.concatenate([ch[:8], rng.choice(d, 88, replace=False)]))
+    Xc = X[:, torch.as_tensor(cols, device=DEV)].contiguous().cpu().numpy()
+    rows = np.sort(rng.choice(m, 48, replace=False))
+    out = dict(spec=spec, n=n, m=m, d=d, cols=cols, Xc=Xc, rows=rows,
+               W64=W.double().cpu().numpy(), S=P.to_np(S), U=P.to_np(U),
+               codes=P.to_np(codes), scales=P.to_np(scales), zeros=P.to_np(zeros),
+               loss=P.to_np(loss), qw=P.to_np(qw).view(np.uint32), qz=P.to_np(qz))
+    del X
+    torch.cuda.empty_cache()
+    return out
+
+
+def test_hessian_block_full_tokens(attn7b):
+    a = attn7b
+    ref = oracle.hessian(a["Xc"])                               # 96 x 96 over all tokens
+    got = P.mirror_upper(a["S"])[np.ix_(a["cols"], a["cols"])]
+    assert P.rel_fro(got, ref) <= P.S_TOL
+    # lower triangle of S is never written
+    assert np.all(np.tril(a["S"], -1) == 0)
+
+
+@pytest.fixture(scope="module")
+def oracle_from_gpu_S(attn7b):
+    a = attn7b
+    S64 = P.mirror_upper(a["S"])
+    H, Hd, perm, lam, st = oracle.finalize(S64, a["n"], 0.01, False)
+    U64, info = oracle.hinv_upper_chol(Hd)
+    assert st == 0 and info == 0
+    return dict(H=H, Hd=Hd, U=U64, perm=perm)
+
+
+def test_u_full_size(attn7b, oracle_from_gpu_S):
+    Ug = attn7b["U"].astype(np.float64)
+    assert np.all(np.tril(Ug, -1) == 0)
+    assert P.rel_fro(Ug, oracle_from_gpu_S["U"]) <= P.U_TOL
+
+
+def test_sweep_sampled_rows_full_size(attn7b, oracle_from_gpu_S):
+    a, o = attn7b, oracle_from_gpu_S
+    r = a["rows"]
+    ref = oracle.quantize_rows(a["W64"][r], o["U"], 4, 128)
+    gpu = dict(codes=a["codes"][r], scales=a["scales"][r], zeros=a["zeros"][r])
+    st = P.compare_sweep(gpu, ref, 128)
+    assert abs(a["loss"][r].sum() - ref["row_loss"].sum()) <= P.LOSS_REL * ref["row_loss"].sum()
+    H64 = o["H"]
+    lg = P.layer_loss_of(a["W64"][r], gpu["codes"], gpu["scales"], gpu["zeros"], 128, None, H64)
+    lo = P.layer_loss_of(a["W64"][r], ref["codes"], ref["scales"], ref["zeros"], 128, None, H64)
+    assert abs(lg - lo) <= P.LOSS_REL * lo
+    ties = P.teacher_forced_check(np.ascontiguousarray(a["W64"][r]), o["U"], gpu, 4, 128)
+    print("attn7b sampled rows:", st, "ties", ties, "loss", lg, lo)
+
+
+def test_pack_full_size(attn7b):
+    a = attn7b
+    rq, rz = oracle.pack_int4(a["codes"], a["zeros"])
+    assert np.array_equal(a["qw"], rq) and np.array_equal(a["qz"], rz)
+    nbytes = a["qw"].nbytes + a["qz"].nbytes + a["scales"].nbytes
+    assert nbytes == 66.5 * a["m"] * a["d"] / 128

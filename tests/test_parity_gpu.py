@@ -21,6 +21,13 @@ def _lib():
     G.load_library()
 
 
+@pytest.fixture(autouse=True)
+def _device_status_clean():
+    yield
+    torch.cuda.synchronize()
+    assert G.gptq_device_status(reset=True) == 0, "a bounded device wait gave up"
+
+
 def _gauss_x(n, d, n_out, fac, seed):
     spec = inputs.LayerSpec("t", 1, d, 0.02, "fp16", n, "gauss", n_out, fac, fac, False, seed)
     return inputs.calibration_x(spec, device="cpu")
