@@ -215,19 +215,26 @@ class Layer:
         self.qweight = torch.empty(m, d // 8, dtype=torch.int32, device=dev)
         self.qzeros = torch.empty(m, (d // 128 + 1) // 2, dtype=torch.uint8, device=dev)
 
-    def step(self, ev_k1=None):
+    def step(self, ev=None):
+        """ev: None or 5 CUDA events recorded at the phase boundaries."""
         G = self.G
         self.S.zero_()
-        if ev_k1 is not None:
-            ev_k1[0].record()
+        if ev is not None:
+            ev[0].record()
         G.gptq_hessian_accumulate(self.S, self.X)
-        if ev_k1 is not None:
-            ev_k1[1].record()
+        if ev is not None:
+            ev[1].record()
         G.gptq_prepare_hinv(self.S, self.n, 0.01, self.act_order, self.perm, self.U, self.info,
                             self.ws_p)
+        if ev is not None:
+            ev[2].record()
         G.gptq_quantize_layer(self.W, self.U, self.perm if self.act_order else None, 4, 128, 128,
                               self.codes, self.scales, self.zeros, self.loss, self.ws_q)
+        if ev is not None:
+            ev[3].record()
         G.gptq_pack_int4(self.codes, self.zeros, self.qweight, self.qzeros)
+        if ev is not None:
+            ev[4].record()
 
 
 def _cpu_baseline(spec, n, reps=1):
@@ -277,8 +284,7 @@ def run_ours(a):
     assert int(lay.info.item()) == 0, "non-positive pivot in the workload"
 
     n_ev = a.steps
-    k1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(n_ev)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_ev)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = G.gptq_debug_launch_count()
     _barrier(ws)
@@ -286,14 +292,16 @@ def run_ours(a):
     with ClockSampler(local) as clk:
         start.record()
         for i in range(a.steps):
-            lay.step(k1[i])
+            lay.step(evs[i])
         end.record()
         torch.cuda.synchronize()
     _barrier(ws)
     launches = G.gptq_debug_launch_count() - launches0
     ms = start.elapsed_time(end) / a.steps
     ms = _max_over_ranks(ms, ws)
-    k1_ms = statistics.mean(s.elapsed_time(e) for s, e in k1)
+    phase = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in evs)
+             for k, name in enumerate(("hessian", "prepare", "quantize", "pack"))}
+    k1_ms = phase["hessian"]
 
     # end to end through the public API from pinned host memory
     Xh = lay.X.cpu().pin_memory()
@@ -351,6 +359,8 @@ def run_ours(a):
                      "peak_source": f"bf16_tflops_sustained of {src} (fp16 = bf16 rate)",
                      "kernel_ms": k1_ms},
         "clocks": clk.summary(),
+        "phase_ms": phase,
+        "layer_ms_without_hessian": phase["prepare"] + phase["quantize"] + phase["pack"],
     }
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         cb = _cpu_baseline(spec, n)

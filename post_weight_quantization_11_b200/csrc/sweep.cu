@@ -14,7 +14,6 @@
 // only the chain of blocks is sequential.
 #include "common.cuh"
 #include "quant_common.cuh"
-#include "simt_gemm.cuh"
 #include "update.cuh"
 
 namespace gptq {
@@ -42,7 +41,8 @@ __global__ void __launch_bounds__(128)
 block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
                    int64_t j0, float maxqf, uint8_t* __restrict__ codes,
                    __half* __restrict__ scales, uint8_t* __restrict__ zeros,
-                   float* __restrict__ E_out, float* __restrict__ row_loss, int first_block)
+                   float* __restrict__ Eh_out, float* __restrict__ El_out,
+                   float* __restrict__ row_loss, int first_block)
 {
     extern __shared__ __align__(16) float smem[];
     float* Us = smem;                        // 128 x 128, strictly-lower part zeroed
@@ -134,10 +134,19 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     uint4* cdst = reinterpret_cast<uint4*>(codes + row * d + j0 + 32 * sub);
     cdst[0] = make_uint4(cp[0], cp[1], cp[2], cp[3]);
     cdst[1] = make_uint4(cp[4], cp[5], cp[6], cp[7]);
-    float4* edst = reinterpret_cast<float4*>(E_out + row * SW_B + 32 * sub);
+    // E split into its TF32 head and fp32 remainder for the tensor-core update
+    float4* hdst = reinterpret_cast<float4*>(Eh_out + row * SW_B + 32 * sub);
+    float4* ldst = reinterpret_cast<float4*>(El_out + row * SW_B + 32 * sub);
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-        edst[q] = make_float4(Ev[4 * q], Ev[4 * q + 1], Ev[4 * q + 2], Ev[4 * q + 3]);
+    for (int q = 0; q < 8; ++q) {
+        float4 h, l;
+        h.x = tf32_round(Ev[4 * q + 0]); l.x = Ev[4 * q + 0] - h.x;
+        h.y = tf32_round(Ev[4 * q + 1]); l.y = Ev[4 * q + 1] - h.y;
+        h.z = tf32_round(Ev[4 * q + 2]); l.z = Ev[4 * q + 2] - h.z;
+        h.w = tf32_round(Ev[4 * q + 3]); l.w = Ev[4 * q + 3] - h.w;
+        hdst[q] = h;
+        ldst[q] = l;
+    }
     if (row_loss && sub == 0) row_loss[row] = first_block ? loss : row_loss[row] + loss;
 }
 
@@ -179,8 +188,7 @@ rtn_kernel(const T* __restrict__ W, int64_t m, int64_t d, float maxqf,
 
 struct QuantWs {
     float* Wk;     // d_out x d_in working copy (sweep order)
-    float* E;      // d_out x 128 scaled errors of the current block
-    UpdateWs upd;  // tensor-core update scratch
+    UpdateWs upd;  // split U and the current block's split errors
 };
 
 static size_t quant_layout(int64_t m, int64_t d, char* base, QuantWs* w)
@@ -188,11 +196,9 @@ static size_t quant_layout(int64_t m, int64_t d, char* base, QuantWs* w)
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 1024); return o; };
     size_t oW = take(sizeof(float) * m * d);
-    size_t oE = take(sizeof(float) * m * SW_B);
     size_t oU = take(update_ws_bytes(m, d));
     if (w && base) {
         w->Wk = reinterpret_cast<float*>(base + oW);
-        w->E = reinterpret_cast<float*>(base + oE);
         update_ws_bind(m, d, base + oU, &w->upd);
     }
     return off;
@@ -211,12 +217,13 @@ static int check_quant_args(int w_dtype, int64_t m, int64_t d, int bits, int gro
 template <int GS>
 static void launch_sweep(dim3 grid, size_t smem, cudaStream_t st, const float* Wk, const float* U,
                          int64_t m, int64_t d, int64_t j0, float maxqf, uint8_t* codes,
-                         __half* scales, uint8_t* zeros, float* E, float* row_loss, int first)
+                         __half* scales, uint8_t* zeros, float* Eh, float* El, float* row_loss,
+                         int first)
 {
     cudaFuncSetAttribute(block_sweep_kernel<GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     block_sweep_kernel<GS><<<grid, 128, smem, st>>>(Wk, U, m, d, j0, maxqf, codes, scales, zeros,
-                                                   E, row_loss, first);
+                                                   Eh, El, row_loss, first);
     count_launches();
 }
 
@@ -271,14 +278,14 @@ extern "C" int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, in
         const int64_t j0 = b * SW_B;
         switch (group_size) {
             case 32: launch_sweep<32>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                      w.E, row_loss, b == 0); break;
+                                      w.upd.Eh, w.upd.El, row_loss, b == 0); break;
             case 64: launch_sweep<64>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                      w.E, row_loss, b == 0); break;
+                                      w.upd.Eh, w.upd.El, row_loss, b == 0); break;
             default: launch_sweep<128>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                       w.E, row_loss, b == 0); break;
+                                       w.upd.Eh, w.upd.El, row_loss, b == 0); break;
         }
         if (b + 1 < nblk) {
-            rc = block_update(w.Wk, w.E, U, m, d, j0, &w.upd, st);
+            rc = block_update(w.Wk, &w.upd, m, d, j0, st);
             if (rc != GPTQ_OK) return rc;
         }
     }

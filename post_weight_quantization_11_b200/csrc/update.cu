@@ -1,0 +1,257 @@
+// Inter-block update W[:, c0:] -= E . U[j0:j0+128, c0:], c0 = j0 + 128, on
+// tcgen05 tensor cores in split-TF32 (three kind::tf32 products, fp32
+// accumulation in TMEM).
+//
+//  * Items are 128-row x 256-column output tiles of the trailing columns,
+//    handed round-robin to one persistent CTA per SM.
+//  * K = 128 (one block) in 4 stages of 32: E_hi, E_lo tiles (rows x 32) and
+//    U_hi^T, U_lo^T tiles (256 columns x 32), all K-major with 128-byte
+//    swizzle, one TMA box each.  U is stored transposed because an MN-major
+//    tf32 operand would need the 32-byte-atom swizzle; K-major is the plain
+//    layout for both.  2 stages of 96 KB.
+//  * warp 0: TMA; warp 1: per 8-wide k-step E_hi U_hi + E_hi U_lo + E_lo U_hi
+//    into one of two TMEM accumulators (2 x 256 columns); warps 2-5: read the
+//    accumulator (tcgen05.ld) and write W - D back, overlapping the next
+//    tile's MMAs.
+//  * Every mbarrier wait is bounded (see tc_common.cuh).
+#include "common.cuh"
+#include "tc_common.cuh"
+#include "update.cuh"
+
+namespace gptq {
+
+constexpr int UB_M = 128, UB_N = 256, UB_KC = 32, UB_STAGES = 2, UB_KTOT = 128;
+constexpr int UB_A_BYTES = UB_M * UB_KC * 4;                  // 16 KB per E tile
+constexpr int UB_B_BYTES = UB_KC * UB_N * 4;                  // 32 KB per U tile
+constexpr int UB_STAGE_BYTES = 2 * UB_A_BYTES + 2 * UB_B_BYTES;  // 96 KB
+constexpr int UB_THREADS = 192;
+constexpr int UB_SMEM = UB_STAGES * UB_STAGE_BYTES + 1024 + 256;
+constexpr uint32_t UB_IDESC = make_idesc(2 /*tf32*/, UB_M, UB_N, 0 /*A K-major*/, 0 /*B K-major*/);
+
+struct UpdParams {
+    float* W;
+    int64_t m, d, j0, c0;
+    int n_rt, n_ct, items;
+};
+
+__global__ void __launch_bounds__(UB_THREADS, 1)
+block_update_tc_kernel(const __grid_constant__ CUtensorMap tmEh,
+                       const __grid_constant__ CUtensorMap tmEl,
+                       const __grid_constant__ CUtensorMap tmUh,
+                       const __grid_constant__ CUtensorMap tmUl, const UpdParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + UB_STAGES * UB_STAGE_BYTES);
+    uint64_t* empty_bar = full_bar + UB_STAGES;
+    uint64_t* accf_bar = empty_bar + UB_STAGES;
+    uint64_t* acce_bar = accf_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + 2);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < UB_STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&accf_bar[a], 1); mbar_init(&acce_bar[a], 128); }
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int P = gridDim.x;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmEh); prefetch_tmap(&tmEl); prefetch_tmap(&tmUh); prefetch_tmap(&tmUl);
+            int stage = 0;
+            uint32_t phase = 0, armed = 0, armed_par = 0;
+            bool ok = true;
+            for (int q = blockIdx.x; q < p.items && ok; q += P) {
+                const int rt = q % p.n_rt, ct = q / p.n_rt;
+                const int y_e = rt * UB_M;
+                const int x_u = (int)(p.c0 + int64_t(ct) * UB_N);
+                for (int kc = 0; kc < UB_KTOT / UB_KC; ++kc) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, kErrWaitEmpty, abort)) { ok = false; break; }
+                    uint8_t* sEh = smem + stage * UB_STAGE_BYTES;
+                    uint8_t* sEl = sEh + UB_A_BYTES;
+                    uint8_t* sUh = sEl + UB_A_BYTES;
+                    uint8_t* sUl = sUh + UB_B_BYTES;
+                    mbar_arrive_expect_tx(&full_bar[stage], UB_STAGE_BYTES);
+                    tma_load_2d(sEh, &tmEh, &full_bar[stage], kc * UB_KC, y_e);
+                    tma_load_2d(sEl, &tmEl, &full_bar[stage], kc * UB_KC, y_e);
+                    const int k_u = (int)(p.j0 + kc * UB_KC);
+                    tma_load_2d(sUh, &tmUh, &full_bar[stage], k_u, x_u);
+                    tma_load_2d(sUl, &tmUl, &full_bar[stage], k_u, x_u);
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == UB_STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            for (int s = 0; s < UB_STAGES; ++s)
+                if (armed & (1u << s)) mbar_drain(&full_bar[s], (armed_par >> s) & 1u);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0, it = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int q = blockIdx.x; q < p.items && ok; q += P, ++it) {
+                const int a = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (!mbar_wait(&acce_bar[a], aph ^ 1, kErrWaitAccEmpty, abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + uint32_t(a * UB_N);
+                uint32_t acc = 0;
+                for (int kc = 0; kc < UB_KTOT / UB_KC; ++kc) {
+                    if (!mbar_wait(&full_bar[stage], phase, kErrWaitFull, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sEh = smem_u32(smem + stage * UB_STAGE_BYTES);
+                    const uint32_t sEl = sEh + UB_A_BYTES;
+                    const uint32_t sUh = sEl + UB_A_BYTES;
+                    const uint32_t sUl = sUh + UB_B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < UB_KC / 8; ++kk) {
+                        // A: K-major rows of 128 B; an 8-wide k-step is 32 B along the row
+                        const uint64_t aH = smem_desc_sw128(sEh + kk * 32, 16, 1024);
+                        const uint64_t aL = smem_desc_sw128(sEl + kk * 32, 16, 1024);
+                        const uint64_t bH = smem_desc_sw128(sUh + kk * 32, 16, 1024);
+                        const uint64_t bL = smem_desc_sw128(sUl + kk * 32, 16, 1024);
+                        mma_tf32(d_tmem, aH, bH, UB_IDESC, acc);
+                        mma_tf32(d_tmem, aH, bL, UB_IDESC, 1u);
+                        mma_tf32(d_tmem, aL, bH, UB_IDESC, 1u);
+                        acc = 1;
+                    }
+                    mma_commit(&empty_bar[stage]);
+                    if (++stage == UB_STAGES) { stage = 0; phase ^= 1; }
+                }
+                mma_commit(&accf_bar[a]);
+            }
+        }
+    } else {
+        const int qr = warp & 3;
+        int it = 0;
+        for (int q = blockIdx.x; q < p.items; q += P, ++it) {
+            const int rt = q % p.n_rt, ct = q / p.n_rt;
+            const int a = it & 1;
+            const uint32_t aph = (it >> 1) & 1;
+            if (!mbar_wait(&accf_bar[a], aph, kErrWaitAccFull, abort)) break;
+            tc_fence_after();
+            const int64_t i = int64_t(rt) * UB_M + qr * 32 + lane;
+            const bool row_ok = i < p.m;
+            float* Wrow = p.W + i * p.d;
+#pragma unroll 1
+            for (int c = 0; c < UB_N / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + uint32_t(a * UB_N + c * 32) + (uint32_t(qr * 32) << 16), v);
+                const int64_t col = p.c0 + int64_t(ct) * UB_N + c * 32;
+                if (!row_ok || col >= p.d) continue;
+                float4* wp = reinterpret_cast<float4*>(Wrow + col);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    float4 w4 = wp[u];
+                    w4.x -= v[4 * u + 0];
+                    w4.y -= v[4 * u + 1];
+                    w4.z -= v[4 * u + 2];
+                    w4.w -= v[4 * u + 3];
+                    wp[u] = w4;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acce_bar[a]);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// hiT[c][k] = tf32(U[k][c]), loT[c][k] = U[k][c] - hiT[c][k]: 32x32 tiles
+// through shared memory so both the reads and the writes are coalesced.
+__global__ void __launch_bounds__(256)
+split_tf32_transpose_kernel(const float* __restrict__ U, int64_t d, float* __restrict__ hiT,
+                            float* __restrict__ loT)
+{
+    __shared__ float t[32][33];
+    const int64_t r0 = int64_t(blockIdx.y) * 32, c0 = int64_t(blockIdx.x) * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8
+#pragma unroll
+    for (int k = 0; k < 32; k += 8) t[ty + k][tx] = U[(r0 + ty + k) * d + c0 + tx];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 32; k += 8) {
+        const float v = t[tx][ty + k];               // U[r0 + tx][c0 + ty + k]
+        const float h = tf32_round(v);
+        hiT[(c0 + ty + k) * d + r0 + tx] = h;
+        loT[(c0 + ty + k) * d + r0 + tx] = v - h;
+    }
+}
+
+static int num_sms()
+{
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+size_t update_ws_bytes(int64_t m, int64_t d)
+{
+    return align_up(sizeof(float) * d * d, 1024) * 2 + align_up(sizeof(float) * m * 128, 1024) * 2;
+}
+
+void update_ws_bind(int64_t m, int64_t d, char* base, UpdateWs* w)
+{
+    const size_t u = align_up(sizeof(float) * d * d, 1024);
+    const size_t e = align_up(sizeof(float) * m * 128, 1024);
+    w->Uh = reinterpret_cast<float*>(base);
+    w->Ul = reinterpret_cast<float*>(base + u);
+    w->Eh = reinterpret_cast<float*>(base + 2 * u);
+    w->El = reinterpret_cast<float*>(base + 2 * u + e);
+}
+
+int update_prepare_u(const float* U, int64_t d, UpdateWs* w, cudaStream_t st)
+{
+    const dim3 grid((unsigned)(d / 32), (unsigned)(d / 32));
+    split_tf32_transpose_kernel<<<grid, 256, 0, st>>>(U, d, w->Uh, w->Ul);
+    count_launches();
+    return launch_status();
+}
+
+int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t j0, cudaStream_t st)
+{
+    UpdParams p{};
+    p.W = Wk;
+    p.m = m;
+    p.d = d;
+    p.j0 = j0;
+    p.c0 = j0 + UB_KTOT;
+    if (p.c0 >= d) return GPTQ_OK;
+    p.n_rt = (int)ceil_div(m, UB_M);
+    p.n_ct = (int)ceil_div(d - p.c0, UB_N);
+    p.items = p.n_rt * p.n_ct;
+    CUtensorMap tEh, tEl, tUh, tUl;
+    if (encode_tmap_2d(&tEh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Eh, 128, (uint64_t)m, 512, 32,
+                       128, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
+        encode_tmap_2d(&tEl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->El, 128, (uint64_t)m, 512, 32,
+                       128, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
+        encode_tmap_2d(&tUh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Uh, (uint64_t)d, (uint64_t)d,
+                       (uint64_t)d * 4, 32, UB_N, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
+        encode_tmap_2d(&tUl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Ul, (uint64_t)d, (uint64_t)d,
+                       (uint64_t)d * 4, 32, UB_N, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK)
+        return GPTQ_ERR_CUDA;
+    if (cudaFuncSetAttribute(block_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             UB_SMEM) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    const int grid = std::min(p.items, num_sms());
+    block_update_tc_kernel<<<grid, UB_THREADS, UB_SMEM, st>>>(tEh, tEl, tUh, tUl, p);
+    count_launches();
+    return launch_status();
+}
+
+}  // namespace gptq

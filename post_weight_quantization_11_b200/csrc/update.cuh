@@ -2,33 +2,34 @@
 // err * H_inv[j, j+1:]) applied a block at a time ("GPTQ / AWQ / SqueezeLLM"
 // sec. 一, blocks):
 //   W[:, j0+128:] -= E . U[j0:j0+128, j0+128:]
-// First version: fp32 CUDA-core GEMM.
+// on the tensor cores in split-TF32: with x = x_hi + x_lo (x_hi rounded to
+// TF32, x_lo the exact fp32 remainder), E U ~ E_hi U_hi + E_hi U_lo + E_lo U_hi
+// (the error-corrected TF32 product of Ootomo & Yokota, 2022), fp32 accuracy.
 #pragma once
 
 #include "common.cuh"
-#include "simt_gemm.cuh"
 
 namespace gptq {
 
 struct UpdateWs {
-    int unused;
+    float* Uh;   // d x d, TF32-rounded U, TRANSPOSED (Uh[c][k] ~ U[k][c])
+    float* Ul;   // d x d, U^T - Uh
+    float* Eh;   // m x 128, TF32-rounded scaled errors of the current block
+    float* El;   // m x 128, remainder
 };
 
-inline size_t update_ws_bytes(int64_t, int64_t) { return 256; }
-inline void update_ws_bind(int64_t, int64_t, char*, UpdateWs* w) { w->unused = 0; }
-inline int update_prepare_u(const float*, int64_t, UpdateWs*, cudaStream_t) { return GPTQ_OK; }
+size_t update_ws_bytes(int64_t m, int64_t d);
+void update_ws_bind(int64_t m, int64_t d, char* base, UpdateWs* w);
+// Split U into its TF32 head and fp32 remainder, transposed (once per layer).
+int update_prepare_u(const float* U, int64_t d, UpdateWs* w, cudaStream_t st);
+// W[:, j0+128:] -= (Eh + El) . (Uh + Ul)[j0:j0+128, j0+128:]  (lo x lo dropped)
+int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t j0, cudaStream_t st);
 
-inline int block_update(float* Wk, const float* E, const float* U, int64_t m, int64_t d,
-                        int64_t j0, UpdateWs*, cudaStream_t st)
+__device__ __forceinline__ float tf32_round(float x)
 {
-    const int64_t c0 = j0 + 128;
-    GemmArgs g{};
-    g.A = E; g.lda = 128;
-    g.B = U + j0 * d + c0; g.ldb = d;
-    g.C = Wk + c0; g.ldc = d;
-    g.M = m; g.N = d - c0; g.K = 128;
-    g.alpha = -1.f; g.beta = 1.f;
-    return simt_gemm(g, st);
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
 }
 
 }  // namespace gptq
