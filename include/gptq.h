@@ -108,6 +108,26 @@ int gptq_prepare_hinv(const float* S, int64_t d, int64_t n_tokens, float damp_re
                       void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * gptq_prepare_hinv without a workspace argument, for callers that cannot
+ * allocate device memory (code running while a stream is captured into a
+ * CUDA graph, where cudaMalloc is not allowed, or a plug-in inside an engine
+ * that owns the whole device memory pool).  The pages have no counterpart:
+ * this is an interface convenience of the library.
+ *
+ * Same arguments, results and errors as gptq_prepare_hinv, minus (ws,
+ * ws_bytes).  Scratch is a fixed 16 MiB array inside the library that every
+ * GPU loading the library holds until the process exits; it limits d to
+ * 1024 (larger d returns GPTQ_ERR_SHAPE before anything is launched).  The
+ * first call on a device looks up the array's device address (make it before
+ * any stream capture begins).  All calls share the one array, so calls that
+ * overlap on the GPU (e.g. on two streams at once) race: serialize them.
+ * Nothing is allocated or freed.
+ */
+int gptq_prepare_hinv_static(const float* S, int64_t d, int64_t n_tokens, float damp_rel,
+                             int act_order, int32_t* perm, float* U, int32_t* info,
+                             void* stream);
+
+/*
  * Quantize one layer -- "INT4/INT8 量化推理" sec. 三 (column loop with error
  * compensation), "GPTQ / AWQ / SqueezeLLM" sec. 一 (blocks), "校准艺术"
  * sec. 2.1 (min-max), "INT4/INT8 量化推理" sec. 一 (group layout).

@@ -29,7 +29,7 @@ _STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_SHAPE", 3: "GPT
 EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_device_status",
             "gptq_hessian_accumulate",
-            "gptq_prepare_workspace_bytes", "gptq_prepare_hinv",
+            "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_pack_int4",
             "gptq_unpack_int4", "rtn_quantize")
 
@@ -62,6 +62,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_hessian_accumulate": ([P, P, I64, I64, P, P], I32),
         "gptq_prepare_workspace_bytes": ([I64], SZ),
         "gptq_prepare_hinv": ([P, I64, I64, F32, I32, P, P, P, P, SZ, P], I32),
+        "gptq_prepare_hinv_static": ([P, I64, I64, F32, I32, P, P, P, P], I32),
         "gptq_quantize_workspace_bytes": ([I64, I64, I32], SZ),
         "gptq_quantize_layer": ([P, I32, I64, I64, P, P, I32, I32, I32, P, P, P, P, P, SZ, P],
                                 I32),
@@ -163,6 +164,22 @@ def gptq_prepare_hinv(S: torch.Tensor, n_tokens: int, damp_rel: float = 0.01,
            load_library().gptq_prepare_hinv(_ptr(S), d, int(n_tokens), float(damp_rel),
                                             int(bool(act_order)), _ptr(perm), _ptr(U), _ptr(info),
                                             _ptr(ws), ws.numel() * ws.element_size(), _stream(S)))
+    return perm, U, info
+
+
+def gptq_prepare_hinv_static(S: torch.Tensor, n_tokens: int, damp_rel: float = 0.01,
+                             act_order: bool = False, perm=None, U=None, info=None):
+    """gptq_prepare_hinv on the library's fixed scratch (no workspace; d <= 1024)."""
+    _need(S, "S", torch.float32)
+    d = S.shape[0]
+    dev = S.device
+    perm = torch.empty(d, dtype=torch.int32, device=dev) if perm is None else perm
+    U = torch.empty(d, d, dtype=torch.float32, device=dev) if U is None else U
+    info = torch.zeros(1, dtype=torch.int32, device=dev) if info is None else info
+    _check("gptq_prepare_hinv_static",
+           load_library().gptq_prepare_hinv_static(_ptr(S), d, int(n_tokens), float(damp_rel),
+                                                   int(bool(act_order)), _ptr(perm), _ptr(U),
+                                                   _ptr(info), _stream(S)))
     return perm, U, info
 
 
