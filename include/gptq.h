@@ -186,6 +186,19 @@ int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bi
                  int group_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
                  void* stream);
 
+/*
+ * Test hook (no counterpart on the pages): the split-TF32 tensor-core GEMM the
+ * library uses for the Cholesky / triangular-inverse updates, exposed so it
+ * can be checked on its own.
+ *   C = beta * C + alpha * A * B^T
+ * A: M x K (lda), B: N x K (ldb), C: M x N (ldc), dense row-major fp32 device
+ * arrays; K % 32 == 0; leading dimensions multiples of 4.  lower != 0
+ * computes only 128x128 output tiles on or below the diagonal (M == N).
+ */
+int gptq_debug_gemm_nt(const float* A, int64_t lda, const float* B, int64_t ldb, float* C,
+                       int64_t ldc, int64_t M, int64_t N, int64_t K, float alpha, float beta,
+                       int lower, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -4,28 +4,42 @@
 // U = upper Cholesky factor of Hd^-1 is taken by the reverse-order route:
 // with J the exchange matrix, A = J Hd J = L L^T (lower Cholesky), and
 // U = J L^-1 J is upper with U^T U = Hd^-1 (uniqueness of the Cholesky
-// factor).  One factorization and one triangular inverse instead of
-// factor / invert / factor.
+// factor): one factorization and one triangular inverse.
 //
 // Steps (all on the device):
 //   1. keys + lambda: diag(S), lambda = damp * mean(2 S_ii / n)
 //   2. perm: stable descending rank of S_ii (act-order) or identity
 //   3. A[i][j] = Hd[d-1-i][d-1-j], Hd = (2/n) S[perm][:, perm] + lambda I
-//   4. blocked right-looking Cholesky of A (64-wide panels): panel factor and
-//      its inverse in one CTA, TRSM and trailing SYRK as fp32 GEMMs
-//   5. blocked triangular inverse X = L^-1 by block rows
+//   4. blocked right-looking Cholesky of A with 128-wide panels:
+//        leaf:  one CTA factors the 128x128 diagonal block and inverts it
+//               (L_kk, X_kk = L_kk^-1, Y_kk = X_kk^T), register tiles,
+//               one barrier per column step
+//        TRSM:  A[below, k] <- A[below, k] X_kk^T       (tensor-core GEMM)
+//        SYRK:  A[below, below] -= L21 L21^T, lower tiles (tensor-core GEMM)
+//   5. X = L^-1 by recursive doubling: for blocks [[A,0],[B,C]] (A of size s,
+//      C of size c <= s),  T^T = Y_A B^T,  X_BC = -X_C T,  Y_BC = X_BC^T;
+//      all full pairs of one level in one batched GEMM, ceil(log2(d/128))
+//      levels
 //   6. U[i][j] = X[d-1-i][d-1-j] (upper), 0 below the diagonal
+// The GEMMs are split-TF32 on tcgen05 (gemm_nt.cu), fp32-level accuracy.
 #include "common.cuh"
-#include "simt_gemm.cuh"
+#include "gemm_nt.cuh"
 
 namespace gptq {
 
-constexpr int PN = 64;   // panel width
+constexpr int PN = 128;            // panel / leaf width
+constexpr int LT = 4;              // register tile edge in the leaf
+constexpr int LNT = PN / LT;       // 32 tile rows
+constexpr int LTILES = LNT * (LNT + 1) / 2;   // 528 lower tiles
+constexpr int LTHREADS = 544;
+constexpr int LSTRIDE = PN + 4;    // row stride of the transposed L in shared memory
+constexpr size_t LSMEM = sizeof(float) * (PN * LSTRIDE + 4 * PN + PN);
 
 struct PrepWs {
     float* A;      // d x d working matrix, then L in its lower triangle
-    float* X;      // d x d, L^-1
-    float* T;      // PN x d temporary
+    float* X;      // d x d, L^-1 (lower)
+    float* Y;      // d x d, L^-T (upper)
+    float* T;      // d x (d/2) temporary of the inverse's levels
     float* keys;   // d
     float* lam;    // 1
 };
@@ -33,15 +47,18 @@ struct PrepWs {
 static size_t prep_layout(int64_t d, char* base, PrepWs* w)
 {
     size_t off = 0;
-    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 1024); return o; };
+    const int64_t h = std::max<int64_t>(d / 2, 128);
     size_t oA = take(sizeof(float) * d * d);
     size_t oX = take(sizeof(float) * d * d);
-    size_t oT = take(sizeof(float) * PN * d);
+    size_t oY = take(sizeof(float) * d * d);
+    size_t oT = take(sizeof(float) * d * h);
     size_t oK = take(sizeof(float) * d);
     size_t oL = take(sizeof(float) * 4);
     if (w && base) {
         w->A = reinterpret_cast<float*>(base + oA);
         w->X = reinterpret_cast<float*>(base + oX);
+        w->Y = reinterpret_cast<float*>(base + oY);
         w->T = reinterpret_cast<float*>(base + oT);
         w->keys = reinterpret_cast<float*>(base + oK);
         w->lam = reinterpret_cast<float*>(base + oL);
@@ -118,54 +135,164 @@ __global__ void build_reversed_kernel(const float* __restrict__ S, const int32_t
     }
 }
 
-// Factor the PN x PN diagonal block k of A (lower), record the first
-// non-positive pivot, write L_kk back to A and L_kk^-1 into X's diagonal block.
-__global__ void __launch_bounds__(256)
-potrf_panel_kernel(float* __restrict__ A, float* __restrict__ X, int64_t d, int64_t k0,
-                   int32_t* __restrict__ info)
+// Leaf: factor the 128x128 diagonal block at (k0, k0) of A and invert it.
+// Thread t < 528 owns the 4x4 tile (R, C), R >= C, of the lower triangle in
+// registers.  Factorization (unscaled right-looking): at step j every tile
+// subtracts col_j[r] col_j[c] / d_j from its elements with c > j, r >= c;
+// the owners of column j+1 then publish it; one barrier per step.  The
+// inverse runs the same way by rows (X[k][:] = B[k][:] / L_kk, then
+// B[r][c] -= L[r][k] X[k][c] for r > k).
+__global__ void __launch_bounds__(LTHREADS, 1)
+leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __restrict__ Y,
+                      int64_t d, int64_t k0, int32_t* __restrict__ info)
 {
-    __shared__ float a[PN][PN + 1];
-    __shared__ float x[PN][PN + 1];
+    extern __shared__ __align__(16) float lsm[];
+    float* Lt = lsm;                                  // Lt[c * LSTRIDE + r] = L[r][c]
+    float* colbuf = lsm + PN * LSTRIDE;               // [2][PN]
+    float* rowbuf = colbuf + 2 * PN;                  // [2][PN]
+    float* piv = rowbuf + 2 * PN;                     // [PN]
+
     const int tid = threadIdx.x;
-    for (int idx = tid; idx < PN * PN; idx += blockDim.x) {
-        int r = idx / PN, c = idx % PN;
-        a[r][c] = (c <= r) ? A[(k0 + r) * d + k0 + c] : 0.f;
+    const bool valid = tid < LTILES;
+    int R = 0, C = 0;
+    if (valid) {
+        int r = (int)((sqrtf(8.f * (float)tid + 1.f) - 1.f) * 0.5f);
+        while ((r + 1) * (r + 2) / 2 <= tid) ++r;
+        while (r > 0 && r * (r + 1) / 2 > tid) --r;
+        R = r;
+        C = tid - r * (r + 1) / 2;
     }
+    const int r0 = R * LT, c0 = C * LT;
+    float v[LT][LT];
+#pragma unroll
+    for (int i = 0; i < LT; ++i) {
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) t = *reinterpret_cast<const float4*>(A + (k0 + r0 + i) * d + k0 + c0);
+        v[i][0] = (c0 + 0 <= r0 + i) ? t.x : 0.f;
+        v[i][1] = (c0 + 1 <= r0 + i) ? t.y : 0.f;
+        v[i][2] = (c0 + 2 <= r0 + i) ? t.z : 0.f;
+        v[i][3] = (c0 + 3 <= r0 + i) ? t.w : 0.f;
+    }
+    if (valid && C == 0) {
+#pragma unroll
+        for (int i = 0; i < LT; ++i) colbuf[r0 + i] = v[i][0];
+    }
+    __syncthreads();
+
     for (int j = 0; j < PN; ++j) {
+        const float* cb = colbuf + (j & 1) * PN;
+        const float dj = cb[j];
+        const bool bad = !(dj > 0.f);
+        if (tid == 0) {
+            piv[j] = dj;
+            if (bad && info) atomicCAS(reinterpret_cast<int*>(info), 0, (int)(d - (k0 + j)));
+        }
+        const float inv = bad ? __int_as_float(0x7fc00000) : 1.0f / dj;
+        if (valid && c0 + LT - 1 > j) {
+            const float4 cr = *reinterpret_cast<const float4*>(cb + r0);
+            const float4 cc = *reinterpret_cast<const float4*>(cb + c0);
+            const float crv[4] = {cr.x, cr.y, cr.z, cr.w};
+            const float ccv[4] = {cc.x * inv, cc.y * inv, cc.z * inv, cc.w * inv};
+#pragma unroll
+            for (int i = 0; i < LT; ++i)
+#pragma unroll
+                for (int q = 0; q < LT; ++q)
+                    if (c0 + q > j && r0 + i >= c0 + q) v[i][q] = fmaf(-crv[i], ccv[q], v[i][q]);
+        }
+        if (j + 1 < PN && valid && C == (j + 1) / LT) {
+            float* nb = colbuf + ((j + 1) & 1) * PN;
+            const int qq = (j + 1) % LT;
+#pragma unroll
+            for (int i = 0; i < LT; ++i) {
+                const float val = qq == 0 ? v[i][0] : qq == 1 ? v[i][1] : qq == 2 ? v[i][2] : v[i][3];
+                if (r0 + i >= j + 1) nb[r0 + i] = val;
+            }
+        }
         __syncthreads();
-        const float piv = a[j][j];
-        const bool bad = !(piv > 0.f);
-        const float sq = bad ? __int_as_float(0x7fc00000) : sqrtf(piv);
-        if (tid == 0 && bad && info)
-            atomicCAS(reinterpret_cast<int*>(info), 0, (int)(d - (k0 + j)));
+    }
+
+    // scale into L, keep L transposed in shared memory, write L back to A
+    if (valid) {
+#pragma unroll
+        for (int q = 0; q < LT; ++q) {
+            const float sq = sqrtf(piv[c0 + q]);
+#pragma unroll
+            for (int i = 0; i < LT; ++i) {
+                const int r = r0 + i, c = c0 + q;
+                float l = 0.f;
+                if (r == c) l = sq;
+                else if (r > c) l = v[i][q] / sq;
+                v[i][q] = l;
+                Lt[c * LSTRIDE + r] = l;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < LT; ++i)
+            *reinterpret_cast<float4*>(A + (k0 + r0 + i) * d + k0 + c0) =
+                make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
+    }
+    // B = I, then X = L^-1 row by row
+#pragma unroll
+    for (int i = 0; i < LT; ++i)
+#pragma unroll
+        for (int q = 0; q < LT; ++q) v[i][q] = (r0 + i == c0 + q) ? 1.f : 0.f;
+    __syncthreads();
+    for (int k = 0; k < PN; ++k) {
+        float* rb = rowbuf + (k & 1) * PN;
+        if (valid && R == k / LT) {
+            const float lkk = Lt[k * LSTRIDE + k];
+            const int ii = k % LT;
+#pragma unroll
+            for (int i = 0; i < LT; ++i) {
+#pragma unroll
+                for (int q = 0; q < LT; ++q) {
+                    const bool on = (i == ii) && (c0 + q <= k);
+                    const float x = v[i][q] / lkk;
+                    v[i][q] = on ? x : v[i][q];
+                    if (on) rb[c0 + q] = x;
+                }
+            }
+        }
         __syncthreads();
-        if (tid == 0) a[j][j] = sq;
-        for (int r = j + 1 + tid; r < PN; r += blockDim.x) a[r][j] = a[r][j] / sq;
-        __syncthreads();
-        const int cnt = PN - 1 - j;
-        for (int idx = tid; idx < cnt * cnt; idx += blockDim.x) {
-            int r = j + 1 + idx / cnt, c = j + 1 + idx % cnt;
-            if (c <= r) a[r][c] = fmaf(-a[r][j], a[c][j], a[r][c]);
+        if (valid && r0 + LT - 1 > k && c0 <= k) {
+            const float4 lc = *reinterpret_cast<const float4*>(Lt + k * LSTRIDE + r0);
+            const float4 xr = *reinterpret_cast<const float4*>(rb + c0);
+            const float lv[4] = {lc.x, lc.y, lc.z, lc.w};
+            const float xv[4] = {xr.x, xr.y, xr.z, xr.w};
+#pragma unroll
+            for (int i = 0; i < LT; ++i)
+#pragma unroll
+                for (int q = 0; q < LT; ++q)
+                    if (r0 + i > k && c0 + q <= k) v[i][q] = fmaf(-lv[i], xv[q], v[i][q]);
         }
     }
-    __syncthreads();
-    // inverse of the lower-triangular block, one column per thread
-    if (tid < PN) {
-        const int c = tid;
-        for (int r = 0; r < PN; ++r) x[r][c] = 0.f;
-        x[c][c] = 1.f / a[c][c];
-        for (int r = c + 1; r < PN; ++r) {
-            float t = 0.f;
-            for (int k = c; k < r; ++k) t = fmaf(a[r][k], x[k][c], t);
-            x[r][c] = -t / a[r][r];
-        }
+    if (valid) {
+#pragma unroll
+        for (int i = 0; i < LT; ++i)
+            *reinterpret_cast<float4*>(X + (k0 + r0 + i) * d + k0 + c0) =
+                make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
+#pragma unroll
+        for (int q = 0; q < LT; ++q)
+            *reinterpret_cast<float4*>(Y + (k0 + c0 + q) * d + k0 + r0) =
+                make_float4(v[0][q], v[1][q], v[2][q], v[3][q]);
     }
+}
+
+// Y[o : o+s, o+s : o+s+c] = X[o+s : o+s+c, o : o+s]^T for every node
+// o = o0 + 2 s b (grid.x = s/32 column tiles of X_BC, grid.y = c/32 row tiles).
+__global__ void __launch_bounds__(256)
+transpose_nodes_kernel(const float* __restrict__ X, float* __restrict__ Y, int64_t d, int64_t s,
+                       int64_t o0)
+{
+    __shared__ float t[32][33];
+    const int64_t o = o0 + 2 * s * blockIdx.z;
+    const int64_t r0 = int64_t(blockIdx.y) * 32, c0 = int64_t(blockIdx.x) * 32;   // within X_BC
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+#pragma unroll
+    for (int k = 0; k < 32; k += 8) t[ty + k][tx] = X[(o + s + r0 + ty + k) * d + o + c0 + tx];
     __syncthreads();
-    for (int idx = tid; idx < PN * PN; idx += blockDim.x) {
-        int r = idx / PN, c = idx % PN;
-        if (c <= r) A[(k0 + r) * d + k0 + c] = a[r][c];
-        X[(k0 + r) * d + k0 + c] = x[r][c];
-    }
+#pragma unroll
+    for (int k = 0; k < 32; k += 8) Y[(o + c0 + ty + k) * d + o + s + r0 + tx] = t[tx][ty + k];
 }
 
 __global__ void write_u_kernel(const float* __restrict__ X, int64_t d, float* __restrict__ U)
@@ -210,43 +337,68 @@ extern "C" int gptq_prepare_hinv(const float* S, int64_t d, int64_t n_tokens, fl
         build_reversed_kernel<<<grid, 256, 0, st>>>(S, p, w.lam, d, 2.0f / float(n_tokens), w.A);
         count_launches();
     }
-    if (cudaMemsetAsync(w.X, 0, sizeof(float) * d * d, st) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (cudaMemsetAsync(w.X, 0, sizeof(float) * d * d, st) != cudaSuccess ||
+        cudaMemsetAsync(w.Y, 0, sizeof(float) * d * d, st) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
     if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
+    if (cudaFuncSetAttribute(leaf_potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)LSMEM) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+
+    const NtBuffer bufA{w.A, d, d, d}, bufX{w.X, d, d, d}, bufY{w.Y, d, d, d};
+    const int64_t h = std::max<int64_t>(d / 2, 128);
+    const NtBuffer bufT{w.T, d, h, h};
     const int64_t nblk = d / PN;
     for (int64_t k = 0; k < nblk; ++k) {
         const int64_t k0 = k * PN;
-        potrf_panel_kernel<<<1, 256, 0, st>>>(w.A, w.X, d, k0, info);
+        leaf_potrf_inv_kernel<<<1, LTHREADS, LSMEM, st>>>(w.A, w.X, w.Y, d, k0, info);
         count_launches();
         const int64_t R = d - k0 - PN;
-        if (R > 0) {
-            GemmArgs t{};
-            t.A = w.A + (k0 + PN) * d + k0; t.lda = d;
-            t.B = w.X + k0 * d + k0; t.ldb = d; t.b_trans = 1;
-            t.C = w.A + (k0 + PN) * d + k0; t.ldc = d;
-            t.M = R; t.N = PN; t.K = PN; t.alpha = 1.f; t.beta = 0.f;
-            if (simt_gemm(t, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
-            GemmArgs s{};
-            s.A = w.A + (k0 + PN) * d + k0; s.lda = d;
-            s.B = w.A + (k0 + PN) * d + k0; s.ldb = d; s.b_trans = 1;
-            s.C = w.A + (k0 + PN) * d + (k0 + PN); s.ldc = d;
-            s.M = R; s.N = R; s.K = PN; s.alpha = -1.f; s.beta = 1.f; s.lower_tiles = 1;
-            if (simt_gemm(s, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
-        }
+        if (R <= 0) continue;
+        NtGemm t{};                               // TRSM: A21 <- A21 X_kk^T
+        t.A = bufA; t.a_row0 = k0 + PN; t.a_col0 = k0;
+        t.B = bufX; t.b_row0 = k0; t.b_col0 = k0;
+        t.C = w.A; t.ldc = d; t.c_row0 = k0 + PN; t.c_col0 = k0;
+        t.M = R; t.N = PN; t.K = PN; t.batch = 1; t.alpha = 1.f; t.beta = 0.f;
+        if (gemm_nt_tf32x3(t, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
+        NtGemm s{};                               // SYRK: A22 -= L21 L21^T (lower tiles)
+        s.A = bufA; s.a_row0 = k0 + PN; s.a_col0 = k0;
+        s.B = bufA; s.b_row0 = k0 + PN; s.b_col0 = k0;
+        s.C = w.A; s.ldc = d; s.c_row0 = k0 + PN; s.c_col0 = k0 + PN;
+        s.M = R; s.N = R; s.K = PN; s.batch = 1; s.alpha = -1.f; s.beta = 1.f; s.lower = 1;
+        if (gemm_nt_tf32x3(s, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
     }
-    for (int64_t i = 1; i < nblk; ++i) {
-        const int64_t i0 = i * PN;
-        GemmArgs t{};
-        t.A = w.A + i0 * d; t.lda = d;          // L[i-block, 0:i0]
-        t.B = w.X; t.ldb = d; t.b_lower = 1;    // X[0:i0, 0:i0]
-        t.C = w.T; t.ldc = d;
-        t.M = PN; t.N = i0; t.K = i0; t.alpha = 1.f; t.beta = 0.f;
-        if (simt_gemm(t, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
-        GemmArgs x{};
-        x.A = w.X + i0 * d + i0; x.lda = d;     // L_ii^-1
-        x.B = w.T; x.ldb = d;
-        x.C = w.X + i0 * d; x.ldc = d;
-        x.M = PN; x.N = i0; x.K = PN; x.alpha = -1.f; x.beta = 0.f;
-        if (simt_gemm(x, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
+    // X = L^-1 by recursive doubling over block pairs.  Level sz merges the
+    // inverted blocks [o, o+sz) and [o+sz, o+sz+c) for o = 2 sz b; when d/128 is
+    // not a power of two the last pair has a shorter second block (c < sz).
+    auto merge = [&](int64_t o0, int64_t sz, int64_t c, int nodes) -> int {
+        NtGemm g1{};                              // T^T_b (sz x c) = Y_A B^T
+        g1.A = bufY; g1.a_row0 = o0; g1.a_col0 = o0; g1.a_row_step = 2 * sz; g1.a_col_step = 2 * sz;
+        g1.B = bufA; g1.b_row0 = o0 + sz; g1.b_col0 = o0; g1.b_row_step = 2 * sz;
+        g1.b_col_step = 2 * sz;
+        g1.C = w.T; g1.ldc = h; g1.c_row0 = 0; g1.c_col0 = 0; g1.c_row_step = sz; g1.c_col_step = 0;
+        g1.M = sz; g1.N = c; g1.K = sz; g1.batch = nodes; g1.alpha = 1.f; g1.beta = 0.f;
+        if (gemm_nt_tf32x3(g1, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
+        NtGemm g2{};                              // X_BC (c x sz) = -X_C T, T = (T^T)^T
+        g2.A = bufX; g2.a_row0 = o0 + sz; g2.a_col0 = o0 + sz; g2.a_row_step = 2 * sz;
+        g2.a_col_step = 2 * sz;
+        g2.B = bufT; g2.b_row0 = 0; g2.b_col0 = 0; g2.b_row_step = sz; g2.b_col_step = 0;
+        g2.C = w.X; g2.ldc = d; g2.c_row0 = o0 + sz; g2.c_col0 = o0; g2.c_row_step = 2 * sz;
+        g2.c_col_step = 2 * sz;
+        g2.M = c; g2.N = sz; g2.K = c; g2.batch = nodes; g2.alpha = -1.f; g2.beta = 0.f;
+        if (gemm_nt_tf32x3(g2, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
+        if (!(o0 == 0 && nodes == 1 && sz + c == d)) {   // Y is read by later levels only
+            dim3 grid((unsigned)(sz / 32), (unsigned)(c / 32), (unsigned)nodes);
+            transpose_nodes_kernel<<<grid, 256, 0, st>>>(w.X, w.Y, d, sz, o0);
+            count_launches();
+        }
+        return GPTQ_OK;
+    };
+    for (int64_t sz = PN; sz < d; sz *= 2) {
+        const int full = (int)(d / (2 * sz));
+        if (full > 0 && merge(0, sz, sz, full) != GPTQ_OK) return GPTQ_ERR_CUDA;
+        const int64_t o = int64_t(full) * 2 * sz;
+        if (o + sz < d && merge(o, sz, d - o - sz, 1) != GPTQ_OK) return GPTQ_ERR_CUDA;
     }
     {
         dim3 grid((unsigned)std::min<int64_t>(ceil_div(d, 256), 16), (unsigned)d);

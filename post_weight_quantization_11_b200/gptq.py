@@ -31,7 +31,7 @@ EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_hessian_accumulate",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_pack_int4",
-            "gptq_unpack_int4", "rtn_quantize")
+            "gptq_unpack_int4", "rtn_quantize", "gptq_debug_gemm_nt")
 
 
 class GptqError(RuntimeError):
@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_pack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "gptq_unpack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "rtn_quantize": ([P, I32, I64, I64, I32, I32, P, P, P, P], I32),
+        "gptq_debug_gemm_nt": ([P, I64, P, I64, P, I64, I64, I64, I64, F32, F32, I32, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -253,6 +254,20 @@ def rtn_quantize(W: torch.Tensor, bits: int = 4, group_size: int = 128):
            load_library().rtn_quantize(_ptr(W), _wdtype(W), m, d, int(bits), int(group_size),
                                        _ptr(codes), _ptr(scales), _ptr(zeros), _stream(W)))
     return codes, scales, zeros
+
+
+def gptq_debug_gemm_nt(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor, alpha: float = 1.0,
+                       beta: float = 0.0, lower: bool = False):
+    """C = beta C + alpha A B^T on the split-TF32 tensor-core GEMM (test hook)."""
+    for t, nm in ((A, "A"), (B, "B"), (C, "C")):
+        _need(t, nm, torch.float32)
+    M, K = A.shape
+    N = B.shape[0]
+    _check("gptq_debug_gemm_nt",
+           load_library().gptq_debug_gemm_nt(_ptr(A), A.stride(0), _ptr(B), B.stride(0), _ptr(C),
+                                             C.stride(0), M, N, K, float(alpha), float(beta),
+                                             int(bool(lower)), _stream(A)))
+    return C
 
 
 # --------------------------------------------------------------------------

@@ -124,9 +124,9 @@ def test_hessian_parity(n, d):
     assert np.all(np.tril(Sg, -1) == 0)   # lower triangle untouched
 
 
-@pytest.mark.parametrize("act_order", [False, True])
-def test_prepare_parity(act_order):
-    n, d = 2048, 512
+@pytest.mark.parametrize("act_order,d", [(False, 512), (True, 512), (False, 640), (True, 1152)])
+def test_prepare_parity(act_order, d):
+    n = 2048
     X = _gauss_x(n, d, 5, 40.0, 11)
     S = torch.from_numpy(oracle.hessian(X.numpy()).astype(np.float32)).to(DEV)
     perm, U, info = G.gptq_prepare_hinv(S, n, 0.01, act_order)
