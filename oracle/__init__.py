@@ -47,6 +47,8 @@ def _load():
         lib.orc_hessian_accumulate.restype = None
         lib.orc_finalize.argtypes = [P, I64, I64, ctypes.c_double, ctypes.c_int, P, P, P, P]
         lib.orc_finalize.restype = ctypes.c_int
+        lib.orc_act_order_perm.argtypes = [P, I64, P]
+        lib.orc_act_order_perm.restype = None
         lib.orc_cholesky_lower.argtypes = [P, I64, P]
         lib.orc_cholesky_lower.restype = ctypes.c_int
         lib.orc_trtri_lower_T.argtypes = [P, I64, P]
@@ -136,6 +138,14 @@ def finalize(S: np.ndarray, n: int, damp_rel: float = 0.01, act_order: bool = Fa
     st = _load().orc_finalize(_p(S), int(n), d, float(damp_rel), int(bool(act_order)),
                               _p(H), _p(Hd), _p(perm), ctypes.byref(lam))
     return H, Hd, perm, float(lam.value), int(st)
+
+
+def act_order_perm(diag: np.ndarray) -> np.ndarray:
+    """Stable descending argsort of diag(H) (ties: lower index first)."""
+    diag = np.ascontiguousarray(diag, dtype=np.float64)
+    perm = np.empty(diag.shape[0], dtype=np.int32)
+    _load().orc_act_order_perm(_p(diag), diag.shape[0], _p(perm))
+    return perm
 
 
 def cholesky_lower(A: np.ndarray):

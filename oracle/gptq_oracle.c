@@ -179,6 +179,14 @@ static int orc_cmp_desc_stable(const void* a, const void* b)
     return (ia < ib) ? -1 : (ia > ib);
 }
 
+/* The act-order permutation alone (stable descending argsort of diag). */
+void orc_act_order_perm(const double* diag, int64_t d, int32_t* perm)
+{
+    for (int64_t i = 0; i < d; ++i) perm[i] = (int32_t)i;
+    orc_sort_keys = diag;
+    qsort(perm, (size_t)d, sizeof(int32_t), orc_cmp_desc_stable);
+}
+
 int orc_finalize(const double* S, int64_t n, int64_t d, double damp_rel,
                  int act_order, double* H, double* Hd, int32_t* perm, double* lam_out)
 {

@@ -38,6 +38,19 @@ static std::atomic<unsigned long long> g_launches{0};
 
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
+int device_sm_count()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 }  // namespace gptq
 
 extern "C" const char* gptq_status_string(int status)

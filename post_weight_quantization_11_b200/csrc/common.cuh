@@ -29,6 +29,9 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Number of SMs of the current device (cached per device after the first query).
+int device_sm_count();
+
 // Supported problem limits (validated at the ABI).
 constexpr int64_t kMaxDim = 32768;
 constexpr int64_t kMaxRows = int64_t(1) << 24;

@@ -235,14 +235,6 @@ gemm_nt_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
-static int gn_sms()
-{
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
-
 int gemm_nt_tf32x3(const NtGemm& g, cudaStream_t st)
 {
     if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return GPTQ_OK;
@@ -275,7 +267,7 @@ int gemm_nt_tf32x3(const NtGemm& g, cudaStream_t st)
     if (cudaFuncSetAttribute(gemm_nt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GN_SMEM) != cudaSuccess)
         return GPTQ_ERR_CUDA;
-    const int grid = std::min(p.items, gn_sms());
+    const int grid = std::min(p.items, device_sm_count());
     gemm_nt_kernel<<<grid, GN_THREADS, GN_SMEM, st>>>(tA, tB, p);
     count_launches();
     return launch_status();

@@ -209,14 +209,6 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, const SyrkParams p)
     }
 }
 
-static int sm_count()
-{
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
-
 }  // namespace gptq
 
 extern "C" int gptq_hessian_accumulate(float* S, const uint16_t* X, int64_t n_tokens, int64_t d,
@@ -237,7 +229,7 @@ extern "C" int gptq_hessian_accumulate(float* S, const uint16_t* X, int64_t n_to
     p.nbi = (int)(d / HB_M);
     const int nbj = (int)ceil_div(d, HB_N);
     p.tiles = (nbj - 1) * nbj + std::min(2 * nbj, p.nbi);
-    const int P = sm_count();
+    const int P = device_sm_count();
     const int64_t ksteps = ceil_div(n_tokens, HB_K);
     // smallest token split count whose round-robin over P CTAs is >= 90 % busy
     int64_t best_s = 1;

@@ -136,12 +136,24 @@ __global__ void build_reversed_kernel(const float* __restrict__ S, const int32_t
 }
 
 // Leaf: factor the 128x128 diagonal block at (k0, k0) of A and invert it.
-// Thread t < 528 owns the 4x4 tile (R, C), R >= C, of the lower triangle in
-// registers.  Factorization (unscaled right-looking): at step j every tile
-// subtracts col_j[r] col_j[c] / d_j from its elements with c > j, r >= c;
-// the owners of column j+1 then publish it; one barrier per step.  The
-// inverse runs the same way by rows (X[k][:] = B[k][:] / L_kk, then
-// B[r][c] -= L[r][k] X[k][c] for r > k).
+// Each of the first 528 threads owns one 4x4 tile (R >= C) of the lower
+// triangle in registers; one barrier per column step.
+//  * Factorization (unscaled right-looking): at step j every tile subtracts
+//    col_j[r] col_j[c] / d_j from its elements with c > j, r >= c, then the
+//    owners of column j+1 publish it.  Tiles are handed to threads in
+//    descending column order, so the tiles still active at step j are the
+//    first threads (whole warps fall idle as the trailing block shrinks).
+//  * Inverse, by rows: X[k][:] = B[k][:] / L_kk, then B[r][c] -= L[r][k] X[k][c]
+//    for r > k; tiles handed out in descending row order for the same reason.
+__device__ __forceinline__ void tri_index(int t, int& r, int& c)
+{
+    int u = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while ((u + 1) * (u + 2) / 2 <= t) ++u;
+    while (u > 0 && u * (u + 1) / 2 > t) --u;
+    r = u;
+    c = t - u * (u + 1) / 2;
+}
+
 __global__ void __launch_bounds__(LTHREADS, 1)
 leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __restrict__ Y,
                       int64_t d, int64_t k0, int32_t* __restrict__ info)
@@ -154,15 +166,15 @@ leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __res
 
     const int tid = threadIdx.x;
     const bool valid = tid < LTILES;
+    // factorization order: column C = 31 - u descending, rows C..31
     int R = 0, C = 0;
     if (valid) {
-        int r = (int)((sqrtf(8.f * (float)tid + 1.f) - 1.f) * 0.5f);
-        while ((r + 1) * (r + 2) / 2 <= tid) ++r;
-        while (r > 0 && r * (r + 1) / 2 > tid) --r;
-        R = r;
-        C = tid - r * (r + 1) / 2;
+        int u, w;
+        tri_index(tid, u, w);
+        C = (LNT - 1) - u;
+        R = C + w;
     }
-    const int r0 = R * LT, c0 = C * LT;
+    int r0 = R * LT, c0 = C * LT;
     float v[LT][LT];
 #pragma unroll
     for (int i = 0; i < LT; ++i) {
@@ -187,17 +199,26 @@ leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __res
             piv[j] = dj;
             if (bad && info) atomicCAS(reinterpret_cast<int*>(info), 0, (int)(d - (k0 + j)));
         }
-        const float inv = bad ? __int_as_float(0x7fc00000) : 1.0f / dj;
         if (valid && c0 + LT - 1 > j) {
+            const float inv = bad ? __int_as_float(0x7fc00000) : __frcp_rn(dj);
             const float4 cr = *reinterpret_cast<const float4*>(cb + r0);
             const float4 cc = *reinterpret_cast<const float4*>(cb + c0);
             const float crv[4] = {cr.x, cr.y, cr.z, cr.w};
             const float ccv[4] = {cc.x * inv, cc.y * inv, cc.z * inv, cc.w * inv};
+            if (c0 > j && R > C) {                    // whole tile trails column j
 #pragma unroll
-            for (int i = 0; i < LT; ++i)
+                for (int i = 0; i < LT; ++i)
 #pragma unroll
-                for (int q = 0; q < LT; ++q)
-                    if (c0 + q > j && r0 + i >= c0 + q) v[i][q] = fmaf(-crv[i], ccv[q], v[i][q]);
+                    for (int q = 0; q < LT; ++q) v[i][q] = fmaf(-crv[i], ccv[q], v[i][q]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < LT; ++i)
+#pragma unroll
+                    for (int q = 0; q < LT; ++q) {
+                        const float m = (c0 + q > j && r0 + i >= c0 + q) ? crv[i] : 0.f;
+                        v[i][q] = fmaf(-m, ccv[q], v[i][q]);
+                    }
+            }
         }
         if (j + 1 < PN && valid && C == (j + 1) / LT) {
             float* nb = colbuf + ((j + 1) & 1) * PN;
@@ -231,6 +252,10 @@ leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __res
             *reinterpret_cast<float4*>(A + (k0 + r0 + i) * d + k0 + c0) =
                 make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
     }
+    // inverse order: row R = 31 - u descending
+    if (valid) tri_index(LTILES - 1 - tid, R, C);
+    r0 = R * LT;
+    c0 = C * LT;
     // B = I, then X = L^-1 row by row
 #pragma unroll
     for (int i = 0; i < LT; ++i)
@@ -241,13 +266,14 @@ leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __res
         float* rb = rowbuf + (k & 1) * PN;
         if (valid && R == k / LT) {
             const float lkk = Lt[k * LSTRIDE + k];
+            const float rl = __frcp_rn(lkk);
             const int ii = k % LT;
 #pragma unroll
             for (int i = 0; i < LT; ++i) {
 #pragma unroll
                 for (int q = 0; q < LT; ++q) {
                     const bool on = (i == ii) && (c0 + q <= k);
-                    const float x = v[i][q] / lkk;
+                    const float x = v[i][q] * rl;
                     v[i][q] = on ? x : v[i][q];
                     if (on) rb[c0 + q] = x;
                 }
@@ -259,11 +285,20 @@ leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __res
             const float4 xr = *reinterpret_cast<const float4*>(rb + c0);
             const float lv[4] = {lc.x, lc.y, lc.z, lc.w};
             const float xv[4] = {xr.x, xr.y, xr.z, xr.w};
+            if (r0 > k && c0 + LT - 1 <= k) {          // whole tile below row k, left of k
 #pragma unroll
-            for (int i = 0; i < LT; ++i)
+                for (int i = 0; i < LT; ++i)
 #pragma unroll
-                for (int q = 0; q < LT; ++q)
-                    if (r0 + i > k && c0 + q <= k) v[i][q] = fmaf(-lv[i], xv[q], v[i][q]);
+                    for (int q = 0; q < LT; ++q) v[i][q] = fmaf(-lv[i], xv[q], v[i][q]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < LT; ++i)
+#pragma unroll
+                    for (int q = 0; q < LT; ++q) {
+                        const float m = (r0 + i > k && c0 + q <= k) ? lv[i] : 0.f;
+                        v[i][q] = fmaf(-m, xv[q], v[i][q]);
+                    }
+            }
         }
     }
     if (valid) {

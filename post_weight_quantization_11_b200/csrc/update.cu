@@ -192,14 +192,6 @@ split_tf32_transpose_kernel(const float* __restrict__ U, int64_t d, float* __res
     }
 }
 
-static int num_sms()
-{
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
-
 size_t update_ws_bytes(int64_t m, int64_t d)
 {
     return align_up(sizeof(float) * d * d, 1024) * 2 + align_up(sizeof(float) * m * 128, 1024) * 2;
@@ -248,7 +240,7 @@ int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t j0,
     if (cudaFuncSetAttribute(block_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              UB_SMEM) != cudaSuccess)
         return GPTQ_ERR_CUDA;
-    const int grid = std::min(p.items, num_sms());
+    const int grid = std::min(p.items, device_sm_count());
     block_update_tc_kernel<<<grid, UB_THREADS, UB_SMEM, st>>>(tEh, tEl, tUh, tUl, p);
     count_launches();
     return launch_status();
