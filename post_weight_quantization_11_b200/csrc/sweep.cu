@@ -19,7 +19,10 @@
 namespace gptq {
 
 constexpr int SW_B = 128;          // block width (columns)
-constexpr int SW_ROWS = 32;        // rows per CTA (4 lanes each, 128 threads)
+constexpr int SW_LPR = 16;         // lanes per row
+constexpr int SW_CPL = SW_B / SW_LPR;   // columns per lane (8)
+constexpr int SW_THREADS = 256;
+constexpr int SW_ROWS = SW_THREADS / SW_LPR;   // rows per CTA (16)
 constexpr unsigned FULL = 0xffffffffu;
 
 // W_work[r][k] = float(W[r][perm[k]])
@@ -36,8 +39,17 @@ __global__ void init_work_kernel(const T* __restrict__ W, const int32_t* __restr
     }
 }
 
+// One 128-column block of the sweep for all rows.  16 lanes per row, each
+// holding 8 consecutive columns in registers; U's 128x128 diagonal block (its
+// strictly-lower part zeroed) and 1/U_jj in shared memory.  Step j: the owner
+// lane's w_j is broadcast with a shuffle, every lane of the row takes the same
+// fp32 decision, and each lane applies w[k] -= E_j U[j][k] to its columns.
+// At a group's first column the group's min/max is reduced over the row's
+// lanes (lanes outside the group contribute 0, neutral since the range
+// includes 0).  The outer loop over the 16 owner lanes is not unrolled, which
+// keeps the kernel's code small.
 template <int GS>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(SW_THREADS)
 block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
                    int64_t j0, float maxqf, uint8_t* __restrict__ codes,
                    __half* __restrict__ scales, uint8_t* __restrict__ zeros,
@@ -48,7 +60,7 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     float* Us = smem;                        // 128 x 128, strictly-lower part zeroed
     float* rdiag = smem + SW_B * SW_B;       // 128: 1 / U_jj
     const int tid = threadIdx.x;
-    for (int idx = tid * 4; idx < SW_B * SW_B; idx += 128 * 4) {
+    for (int idx = tid * 4; idx < SW_B * SW_B; idx += SW_THREADS * 4) {
         const int a = idx / SW_B, b = idx % SW_B;
         float4 v = *reinterpret_cast<const float4*>(U + (j0 + a) * d + j0 + b);
         if (b + 0 < a) v.x = 0.f;
@@ -60,85 +72,86 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     __syncthreads();
     if (tid < SW_B) rdiag[tid] = 1.0f / Us[tid * SW_B + tid];
 
-    const int lane = tid & 31, sub = lane & 3;
-    const int src_base = lane & ~3;
-    const int64_t row = int64_t(blockIdx.x) * SW_ROWS + (tid >> 2);
+    const int lane = tid & 31, sub = lane & (SW_LPR - 1);
+    const int src_base = lane & ~(SW_LPR - 1);
+    const int64_t row = int64_t(blockIdx.x) * SW_ROWS + (tid / SW_LPR);
     const bool valid = row < m;
     const int64_t G = d / GS;
 
-    float w[32];
+    float w[SW_CPL];
     if (valid) {
-        const float4* p = reinterpret_cast<const float4*>(Wk + row * d + j0 + 32 * sub);
+        const float4* p = reinterpret_cast<const float4*>(Wk + row * d + j0 + SW_CPL * sub);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            float4 v = p[q];
+        for (int q = 0; q < SW_CPL / 4; ++q) {
+            const float4 v = p[q];
             w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
         }
     } else {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) w[q] = 0.f;
+        for (int q = 0; q < SW_CPL; ++q) w[q] = 0.f;
     }
     __syncthreads();
 
-    float Ev[32];
-    uint32_t cp[8];
+    float Ev[SW_CPL];
+    uint32_t cp[SW_CPL / 4];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) cp[q] = 0u;
+    for (int q = 0; q < SW_CPL / 4; ++q) cp[q] = 0u;
     float loss = 0.f;
     GroupQ gq;
     gq.s = 1.f; gq.z = 0.f; gq.h = __float2half(1.f);
 
+#pragma unroll 1
+    for (int jo = 0; jo < SW_LPR; ++jo) {
 #pragma unroll
-    for (int j = 0; j < SW_B; ++j) {
-        if (j % GS == 0) {
-            constexpr int span = GS / 32;
-            const int lo = j / 32;
-            float mn = 0.f, mx = 0.f;
-            if (sub >= lo && sub < lo + span) {
+        for (int ji = 0; ji < SW_CPL; ++ji) {
+            const int j = jo * SW_CPL + ji;
+            if (ji == 0 && (jo * SW_CPL) % GS == 0) {
+                constexpr int span = GS / SW_CPL;            // lanes covering one group
+                float mn = 0.f, mx = 0.f;
+                if (sub >= jo && sub < jo + span) {
 #pragma unroll
-                for (int q = 0; q < 32; ++q) { mn = fminf(mn, w[q]); mx = fmaxf(mx, w[q]); }
+                    for (int q = 0; q < SW_CPL; ++q) { mn = fminf(mn, w[q]); mx = fmaxf(mx, w[q]); }
+                }
+#pragma unroll
+                for (int o = 1; o < SW_LPR; o <<= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+                    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+                }
+                gq = group_params(mn, mx, maxqf);
+                if (valid && sub == jo) {
+                    const int64_t gi = (j0 + j) / GS;
+                    scales[row * G + gi] = gq.h;
+                    zeros[row * G + gi] = (uint8_t)gq.z;
+                }
             }
-            mn = fminf(mn, __shfl_xor_sync(FULL, mn, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
-            mn = fminf(mn, __shfl_xor_sync(FULL, mn, 2));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
-            gq = group_params(mn, mx, maxqf);
-            if (valid && sub == lo) {
-                const int64_t gi = (j0 + j) / GS;
-                scales[row * G + gi] = gq.h;
-                zeros[row * G + gi] = (uint8_t)gq.z;
+            const float x = __shfl_sync(FULL, w[ji], src_base | jo);
+            const float c = quant_code(x, gq, maxqf);
+            const float q = gq.s * (c - gq.z);
+            const float e = x - q;
+            const float Ej = e * rdiag[j];
+            loss = fmaf(Ej, Ej, loss);
+            if (sub == jo) {
+                Ev[ji] = Ej;
+                cp[ji / 4] |= uint32_t(c) << (8 * (ji % 4));
             }
-        }
-        const int owner = j / 32, idx = j % 32;
-        const float x = __shfl_sync(FULL, w[idx], src_base | owner);
-        const float c = quant_code(x, gq, maxqf);
-        const float q = gq.s * (c - gq.z);
-        const float e = x - q;
-        const float Ej = e * rdiag[j];
-        loss = fmaf(Ej, Ej, loss);
-        if (sub == owner) {
-            Ev[idx] = Ej;
-            cp[idx / 4] |= uint32_t(c) << (8 * (idx % 4));
-        }
-        const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B + 32 * sub);
+            const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B + SW_CPL * sub);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 u = urow[q4];
-            w[4 * q4 + 0] = fmaf(-Ej, u.x, w[4 * q4 + 0]);
-            w[4 * q4 + 1] = fmaf(-Ej, u.y, w[4 * q4 + 1]);
-            w[4 * q4 + 2] = fmaf(-Ej, u.z, w[4 * q4 + 2]);
-            w[4 * q4 + 3] = fmaf(-Ej, u.w, w[4 * q4 + 3]);
+            for (int q4 = 0; q4 < SW_CPL / 4; ++q4) {
+                const float4 u = urow[q4];
+                w[4 * q4 + 0] = fmaf(-Ej, u.x, w[4 * q4 + 0]);
+                w[4 * q4 + 1] = fmaf(-Ej, u.y, w[4 * q4 + 1]);
+                w[4 * q4 + 2] = fmaf(-Ej, u.z, w[4 * q4 + 2]);
+                w[4 * q4 + 3] = fmaf(-Ej, u.w, w[4 * q4 + 3]);
+            }
         }
     }
     if (!valid) return;
-    uint4* cdst = reinterpret_cast<uint4*>(codes + row * d + j0 + 32 * sub);
-    cdst[0] = make_uint4(cp[0], cp[1], cp[2], cp[3]);
-    cdst[1] = make_uint4(cp[4], cp[5], cp[6], cp[7]);
+    *reinterpret_cast<uint2*>(codes + row * d + j0 + SW_CPL * sub) = make_uint2(cp[0], cp[1]);
     // E split into its TF32 head and fp32 remainder for the tensor-core update
-    float4* hdst = reinterpret_cast<float4*>(Eh_out + row * SW_B + 32 * sub);
-    float4* ldst = reinterpret_cast<float4*>(El_out + row * SW_B + 32 * sub);
+    float4* hdst = reinterpret_cast<float4*>(Eh_out + row * SW_B + SW_CPL * sub);
+    float4* ldst = reinterpret_cast<float4*>(El_out + row * SW_B + SW_CPL * sub);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < SW_CPL / 4; ++q) {
         float4 h, l;
         h.x = tf32_round(Ev[4 * q + 0]); l.x = Ev[4 * q + 0] - h.x;
         h.y = tf32_round(Ev[4 * q + 1]); l.y = Ev[4 * q + 1] - h.y;
@@ -222,7 +235,8 @@ static void launch_sweep(dim3 grid, size_t smem, cudaStream_t st, const float* W
 {
     cudaFuncSetAttribute(block_sweep_kernel<GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    block_sweep_kernel<GS><<<grid, 128, smem, st>>>(Wk, U, m, d, j0, maxqf, codes, scales, zeros,
+    block_sweep_kernel<GS><<<grid, SW_THREADS, smem, st>>>(Wk, U, m, d, j0, maxqf, codes, scales,
+                                                          zeros,
                                                    Eh, El, row_loss, first);
     count_launches();
 }
