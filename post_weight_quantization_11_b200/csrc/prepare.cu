@@ -12,8 +12,9 @@
 //   3. A[i][j] = Hd[d-1-i][d-1-j], Hd = (2/n) S[perm][:, perm] + lambda I
 //   4. blocked right-looking Cholesky of A with 128-wide panels:
 //        leaf:  one CTA factors the 128x128 diagonal block and inverts it
-//               (L_kk, X_kk = L_kk^-1, Y_kk = X_kk^T), register tiles,
-//               one barrier per column step
+//               (L_kk, X_kk = L_kk^-1, Y_kk = X_kk^T): 32-column sub-panels
+//               factored and inverted by one warp with shuffles, panel solve
+//               and rank-32 updates by the whole CTA
 //        TRSM:  A[below, k] <- A[below, k] X_kk^T       (tensor-core GEMM)
 //        SYRK:  A[below, below] -= L21 L21^T, lower tiles (tensor-core GEMM)
 //   5. X = L^-1 by recursive doubling: for blocks [[A,0],[B,C]] (A of size s,
@@ -28,12 +29,6 @@
 namespace gptq {
 
 constexpr int PN = 128;            // panel / leaf width
-constexpr int LT = 4;              // register tile edge in the leaf
-constexpr int LNT = PN / LT;       // 32 tile rows
-constexpr int LTILES = LNT * (LNT + 1) / 2;   // 528 lower tiles
-constexpr int LTHREADS = 544;
-constexpr int LSTRIDE = PN + 4;    // row stride of the transposed L in shared memory
-constexpr size_t LSMEM = sizeof(float) * (PN * LSTRIDE + 4 * PN + PN);
 
 struct PrepWs {
     float* A;      // d x d working matrix, then L in its lower triangle
@@ -135,16 +130,20 @@ __global__ void build_reversed_kernel(const float* __restrict__ S, const int32_t
     }
 }
 
-// Leaf: factor the 128x128 diagonal block at (k0, k0) of A and invert it.
-// Each of the first 528 threads owns one 4x4 tile (R >= C) of the lower
-// triangle in registers; one barrier per column step.
-//  * Factorization (unscaled right-looking): at step j every tile subtracts
-//    col_j[r] col_j[c] / d_j from its elements with c > j, r >= c, then the
-//    owners of column j+1 publish it.  Tiles are handed to threads in
-//    descending column order, so the tiles still active at step j are the
-//    first threads (whole warps fall idle as the trailing block shrinks).
-//  * Inverse, by rows: X[k][:] = B[k][:] / L_kk, then B[r][c] -= L[r][k] X[k][c]
-//    for r > k; tiles handed out in descending row order for the same reason.
+// Leaf: factor the 128x128 diagonal block at (k0, k0) of A and invert it
+// (L_kk into A, X_kk = L_kk^-1 into X, X_kk^T into Y), one CTA of 8 warps,
+// every thread busy at every step:
+//   * 4 columns per step: every thread factors and inverts the 4x4 diagonal
+//     block itself (10 shared-memory reads, no broadcast), one thread per row
+//     solves the 4 panel entries of its row, then a rank-4 update of the
+//     trailing lower triangle in 4x4 tiles -- two barriers per 4 columns;
+//   * X is assembled from the 4x4 diagonal inverses by five doubling levels,
+//     X_BC = -X_C (B X_A), as small GEMMs in shared memory.
+constexpr int LDA = PN + 4;                  // row stride of the shared 128x128 blocks
+constexpr int LDT = 68;                      // row stride of the doubling temporary
+constexpr int LTHREADS = 256;
+constexpr size_t LSMEM = sizeof(float) * (2 * PN * LDA + 64 * LDT);
+
 __device__ __forceinline__ void tri_index(int t, int& r, int& c)
 {
     int u = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
@@ -154,162 +153,194 @@ __device__ __forceinline__ void tri_index(int t, int& r, int& c)
     c = t - u * (u + 1) / 2;
 }
 
+// C (4x4 tile at rows i0.., cols j0..) = sum over k in [kb, ke) of P[i][k] Q[k][j]
+// with P, Q in shared memory (row strides ldp, ldq; k range a multiple of 4).
+__device__ __forceinline__ void tile_gemm4(const float* P, int ldp, const float* Q, int ldq,
+                                           int i0, int j0, int kb, int ke, float (&acc)[4][4])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int k = kb; k < ke; k += 4) {
+        float4 pr[4], qr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pr[i] = *reinterpret_cast<const float4*>(P + (i0 + i) * ldp + k);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) qr[q] = *reinterpret_cast<const float4*>(Q + (k + q) * ldq + j0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float pv[4] = {pr[i].x, pr[i].y, pr[i].z, pr[i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc[i][0] = fmaf(pv[q], qr[q].x, acc[i][0]);
+                acc[i][1] = fmaf(pv[q], qr[q].y, acc[i][1]);
+                acc[i][2] = fmaf(pv[q], qr[q].z, acc[i][2]);
+                acc[i][3] = fmaf(pv[q], qr[q].w, acc[i][3]);
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(LTHREADS, 1)
 leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __restrict__ Y,
                       int64_t d, int64_t k0, int32_t* __restrict__ info)
 {
     extern __shared__ __align__(16) float lsm[];
-    float* Lt = lsm;                                  // Lt[c * LSTRIDE + r] = L[r][c]
-    float* colbuf = lsm + PN * LSTRIDE;               // [2][PN]
-    float* rowbuf = colbuf + 2 * PN;                  // [2][PN]
-    float* piv = rowbuf + 2 * PN;                     // [PN]
-
+    float* a = lsm;                    // 128 x LDA: the block, then L (lower)
+    float* xs = a + PN * LDA;          // 128 x LDA: X = L^-1 (lower)
+    float* tb = xs + PN * LDA;         // 64 x LDT temporary
     const int tid = threadIdx.x;
-    const bool valid = tid < LTILES;
-    // factorization order: column C = 31 - u descending, rows C..31
-    int R = 0, C = 0;
-    if (valid) {
-        int u, w;
-        tri_index(tid, u, w);
-        C = (LNT - 1) - u;
-        R = C + w;
-    }
-    int r0 = R * LT, c0 = C * LT;
-    float v[LT][LT];
-#pragma unroll
-    for (int i = 0; i < LT; ++i) {
-        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (valid) t = *reinterpret_cast<const float4*>(A + (k0 + r0 + i) * d + k0 + c0);
-        v[i][0] = (c0 + 0 <= r0 + i) ? t.x : 0.f;
-        v[i][1] = (c0 + 1 <= r0 + i) ? t.y : 0.f;
-        v[i][2] = (c0 + 2 <= r0 + i) ? t.z : 0.f;
-        v[i][3] = (c0 + 3 <= r0 + i) ? t.w : 0.f;
-    }
-    if (valid && C == 0) {
-#pragma unroll
-        for (int i = 0; i < LT; ++i) colbuf[r0 + i] = v[i][0];
+
+    for (int idx = tid * 4; idx < PN * PN; idx += LTHREADS * 4) {
+        const int r = idx / PN, c = idx % PN;
+        *reinterpret_cast<float4*>(a + r * LDA + c) =
+            *reinterpret_cast<const float4*>(A + (k0 + r) * d + k0 + c);
+        *reinterpret_cast<float4*>(xs + r * LDA + c) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
 
-    for (int j = 0; j < PN; ++j) {
-        const float* cb = colbuf + (j & 1) * PN;
-        const float dj = cb[j];
-        const bool bad = !(dj > 0.f);
+    for (int c0 = 0; c0 < PN; c0 += 4) {
+        // 4x4 diagonal block: Cholesky factor g and its inverse h, in registers
+        float g[4][4], h[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) g[i][j] = (j <= i) ? a[(c0 + i) * LDA + c0 + j] : 0.f;
+        float rd[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float djj = g[j][j];
+            const bool bad = !(djj > 0.f);
+            if (bad && tid == 0 && info)
+                atomicCAS(reinterpret_cast<int*>(info), 0, (int)(d - (k0 + c0 + j)));
+            const float sq = bad ? __int_as_float(0x7fc00000) : sqrtf(djj);
+            rd[j] = __frcp_rn(sq);
+            g[j][j] = sq;
+#pragma unroll
+            for (int i = j + 1; i < 4; ++i) g[i][j] *= rd[j];
+#pragma unroll
+            for (int i = j + 1; i < 4; ++i)
+#pragma unroll
+                for (int k = j + 1; k <= i; ++k) g[i][k] = fmaf(-g[i][j], g[k][j], g[i][k]);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {                 // forward substitution, column c
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r < c) { h[r][c] = 0.f; continue; }
+                float t = (r == c) ? 1.f : 0.f;
+#pragma unroll
+                for (int k = c; k < r; ++k) t = fmaf(-g[r][k], h[k][c], t);
+                h[r][c] = t * rd[r];
+            }
+        }
+        // panel rows below: L[r][c0..c0+3] = A[r][c0..c0+3] h^T, one row per thread
+        const int rows = PN - c0 - 4;
+        if (tid < rows) {
+            const int r = c0 + 4 + tid;
+            const float4 v = *reinterpret_cast<const float4*>(a + r * LDA + c0);
+            const float av[4] = {v.x, v.y, v.z, v.w};
+            float o[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float t = 0.f;
+#pragma unroll
+                for (int k = 0; k <= c; ++k) t = fmaf(av[k], h[c][k], t);
+                o[c] = t;
+            }
+            *reinterpret_cast<float4*>(a + r * LDA + c0) = make_float4(o[0], o[1], o[2], o[3]);
+        }
         if (tid == 0) {
-            piv[j] = dj;
-            if (bad && info) atomicCAS(reinterpret_cast<int*>(info), 0, (int)(d - (k0 + j)));
-        }
-        if (valid && c0 + LT - 1 > j) {
-            const float inv = bad ? __int_as_float(0x7fc00000) : __frcp_rn(dj);
-            const float4 cr = *reinterpret_cast<const float4*>(cb + r0);
-            const float4 cc = *reinterpret_cast<const float4*>(cb + c0);
-            const float crv[4] = {cr.x, cr.y, cr.z, cr.w};
-            const float ccv[4] = {cc.x * inv, cc.y * inv, cc.z * inv, cc.w * inv};
-            if (c0 > j && R > C) {                    // whole tile trails column j
 #pragma unroll
-                for (int i = 0; i < LT; ++i)
-#pragma unroll
-                    for (int q = 0; q < LT; ++q) v[i][q] = fmaf(-crv[i], ccv[q], v[i][q]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < LT; ++i)
-#pragma unroll
-                    for (int q = 0; q < LT; ++q) {
-                        const float m = (c0 + q > j && r0 + i >= c0 + q) ? crv[i] : 0.f;
-                        v[i][q] = fmaf(-m, ccv[q], v[i][q]);
-                    }
+            for (int i = 0; i < 4; ++i) {
+                *reinterpret_cast<float4*>(a + (c0 + i) * LDA + c0) =
+                    make_float4(g[i][0], g[i][1], g[i][2], g[i][3]);
+                *reinterpret_cast<float4*>(xs + (c0 + i) * LDA + c0) =
+                    make_float4(h[i][0], h[i][1], h[i][2], h[i][3]);
             }
         }
-        if (j + 1 < PN && valid && C == (j + 1) / LT) {
-            float* nb = colbuf + ((j + 1) & 1) * PN;
-            const int qq = (j + 1) % LT;
+        __syncthreads();
+        // rank-4 update of the trailing lower triangle [c0+4, 128)
+        const int nt = rows / 4, tiles = nt * (nt + 1) / 2;
+        for (int t = tid; t < tiles; t += LTHREADS) {
+            int ti, tj;
+            tri_index(t, ti, tj);
+            const int r0 = c0 + 4 + 4 * ti, q0 = c0 + 4 + 4 * tj;
+            float4 lr[4], lc[4];
 #pragma unroll
-            for (int i = 0; i < LT; ++i) {
-                const float val = qq == 0 ? v[i][0] : qq == 1 ? v[i][1] : qq == 2 ? v[i][2] : v[i][3];
-                if (r0 + i >= j + 1) nb[r0 + i] = val;
+            for (int i = 0; i < 4; ++i) {
+                lr[i] = *reinterpret_cast<const float4*>(a + (r0 + i) * LDA + c0);
+                lc[i] = *reinterpret_cast<const float4*>(a + (q0 + i) * LDA + c0);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float4 cur = *reinterpret_cast<const float4*>(a + (r0 + i) * LDA + q0);
+                float cv[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float t2 = cv[j];
+                    t2 = fmaf(-lr[i].x, lc[j].x, t2);
+                    t2 = fmaf(-lr[i].y, lc[j].y, t2);
+                    t2 = fmaf(-lr[i].z, lc[j].z, t2);
+                    t2 = fmaf(-lr[i].w, lc[j].w, t2);
+                    cv[j] = t2;
+                }
+                *reinterpret_cast<float4*>(a + (r0 + i) * LDA + q0) =
+                    make_float4(cv[0], cv[1], cv[2], cv[3]);
             }
         }
         __syncthreads();
     }
 
-    // scale into L, keep L transposed in shared memory, write L back to A
-    if (valid) {
+    // X from the 4x4 diagonal inverses by doubling: s = 4, 8, ..., 64
+    for (int s = 4; s < PN; s *= 2) {
+        const int pairs = PN / (2 * s);
+        const int ts = s / 4, tpp = ts * ts;               // 4x4 tiles per pair
+        // T = B X_A, B = L[o+s+i][o+k], X_A = X[o+k][o+j] (zero for k < j)
+        for (int t = tid; t < pairs * tpp; t += LTHREADS) {
+            const int pr = t / tpp, tt = t % tpp;
+            const int o = pr * 2 * s;
+            const int i0 = (tt / ts) * 4, j0 = (tt % ts) * 4;
+            float acc[4][4];
+            tile_gemm4(a + (o + s) * LDA + o, LDA, xs + o * LDA + o, LDA, i0, j0, j0, s, acc);
 #pragma unroll
-        for (int q = 0; q < LT; ++q) {
-            const float sq = sqrtf(piv[c0 + q]);
-#pragma unroll
-            for (int i = 0; i < LT; ++i) {
-                const int r = r0 + i, c = c0 + q;
-                float l = 0.f;
-                if (r == c) l = sq;
-                else if (r > c) l = v[i][q] / sq;
-                v[i][q] = l;
-                Lt[c * LSTRIDE + r] = l;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < LT; ++i)
-            *reinterpret_cast<float4*>(A + (k0 + r0 + i) * d + k0 + c0) =
-                make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
-    }
-    // inverse order: row R = 31 - u descending
-    if (valid) tri_index(LTILES - 1 - tid, R, C);
-    r0 = R * LT;
-    c0 = C * LT;
-    // B = I, then X = L^-1 row by row
-#pragma unroll
-    for (int i = 0; i < LT; ++i)
-#pragma unroll
-        for (int q = 0; q < LT; ++q) v[i][q] = (r0 + i == c0 + q) ? 1.f : 0.f;
-    __syncthreads();
-    for (int k = 0; k < PN; ++k) {
-        float* rb = rowbuf + (k & 1) * PN;
-        if (valid && R == k / LT) {
-            const float lkk = Lt[k * LSTRIDE + k];
-            const float rl = __frcp_rn(lkk);
-            const int ii = k % LT;
-#pragma unroll
-            for (int i = 0; i < LT; ++i) {
-#pragma unroll
-                for (int q = 0; q < LT; ++q) {
-                    const bool on = (i == ii) && (c0 + q <= k);
-                    const float x = v[i][q] * rl;
-                    v[i][q] = on ? x : v[i][q];
-                    if (on) rb[c0 + q] = x;
-                }
-            }
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4*>(tb + (pr * s + i0 + i) * LDT + j0) =
+                    make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         }
         __syncthreads();
-        if (valid && r0 + LT - 1 > k && c0 <= k) {
-            const float4 lc = *reinterpret_cast<const float4*>(Lt + k * LSTRIDE + r0);
-            const float4 xr = *reinterpret_cast<const float4*>(rb + c0);
-            const float lv[4] = {lc.x, lc.y, lc.z, lc.w};
-            const float xv[4] = {xr.x, xr.y, xr.z, xr.w};
-            if (r0 > k && c0 + LT - 1 <= k) {          // whole tile below row k, left of k
+        // X_BC = -X_C T, X_C = X[o+s+i][o+s+k] (zero for k > i)
+        for (int t = tid; t < pairs * tpp; t += LTHREADS) {
+            const int pr = t / tpp, tt = t % tpp;
+            const int o = pr * 2 * s;
+            const int i0 = (tt / ts) * 4, j0 = (tt % ts) * 4;
+            float acc[4][4];
+            tile_gemm4(xs + (o + s) * LDA + o + s, LDA, tb + pr * s * LDT, LDT, i0, j0, 0, i0 + 4,
+                       acc);
 #pragma unroll
-                for (int i = 0; i < LT; ++i)
-#pragma unroll
-                    for (int q = 0; q < LT; ++q) v[i][q] = fmaf(-lv[i], xv[q], v[i][q]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < LT; ++i)
-#pragma unroll
-                    for (int q = 0; q < LT; ++q) {
-                        const float m = (r0 + i > k && c0 + q <= k) ? lv[i] : 0.f;
-                        v[i][q] = fmaf(-m, xv[q], v[i][q]);
-                    }
-            }
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4*>(xs + (o + s + i0 + i) * LDA + o + j0) =
+                    make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
         }
+        __syncthreads();
     }
-    if (valid) {
-#pragma unroll
-        for (int i = 0; i < LT; ++i)
-            *reinterpret_cast<float4*>(X + (k0 + r0 + i) * d + k0 + c0) =
-                make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
-#pragma unroll
-        for (int q = 0; q < LT; ++q)
-            *reinterpret_cast<float4*>(Y + (k0 + c0 + q) * d + k0 + r0) =
-                make_float4(v[0][q], v[1][q], v[2][q], v[3][q]);
+
+    // write L (lower, zeros above within the block), X and Y = X^T
+    for (int idx = tid * 4; idx < PN * PN; idx += LTHREADS * 4) {
+        const int r = idx / PN, c = idx % PN;
+        float4 lv = *reinterpret_cast<const float4*>(a + r * LDA + c);
+        if (c + 0 > r) lv.x = 0.f;
+        if (c + 1 > r) lv.y = 0.f;
+        if (c + 2 > r) lv.z = 0.f;
+        if (c + 3 > r) lv.w = 0.f;
+        *reinterpret_cast<float4*>(A + (k0 + r) * d + k0 + c) = lv;
+        *reinterpret_cast<float4*>(X + (k0 + r) * d + k0 + c) =
+            *reinterpret_cast<const float4*>(xs + r * LDA + c);
+        // Y row r holds column r of X: X[c..c+3][r]
+        *reinterpret_cast<float4*>(Y + (k0 + r) * d + k0 + c) =
+            make_float4(xs[(c + 0) * LDA + r], xs[(c + 1) * LDA + r], xs[(c + 2) * LDA + r],
+                        xs[(c + 3) * LDA + r]);
     }
 }
 
