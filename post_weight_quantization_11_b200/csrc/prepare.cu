@@ -146,7 +146,8 @@ constexpr size_t LSMEM = sizeof(float) * (2 * PN * LDA + 64 * LDT);
 
 __device__ __forceinline__ void tri_index(int t, int& r, int& c)
 {
-    int u = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    const float x = 8.f * (float)t + 1.f;                 // estimate, corrected below
+    int u = (int)((x * rsqrtf(x) - 1.f) * 0.5f);
     while ((u + 1) * (u + 2) / 2 <= t) ++u;
     while (u > 0 && u * (u + 1) / 2 > t) --u;
     r = u;
@@ -214,9 +215,12 @@ leaf_potrf_inv_kernel(float* __restrict__ A, float* __restrict__ X, float* __res
             const bool bad = !(djj > 0.f);
             if (bad && tid == 0 && info)
                 atomicCAS(reinterpret_cast<int*>(info), 0, (int)(d - (k0 + c0 + j)));
-            const float sq = bad ? __int_as_float(0x7fc00000) : sqrtf(djj);
-            rd[j] = __frcp_rn(sq);
-            g[j][j] = sq;
+            // 1/sqrt(d) from the hardware estimate plus one Newton step (~1 ulp)
+            float y = rsqrtf(djj);
+            y = y * fmaf(-0.5f * djj * y, y, 1.5f);
+            if (bad) y = __int_as_float(0x7fc00000);
+            rd[j] = y;
+            g[j][j] = djj * y;
 #pragma unroll
             for (int i = j + 1; i < 4; ++i) g[i][j] *= rd[j];
 #pragma unroll
