@@ -53,13 +53,16 @@ __global__ void __launch_bounds__(SW_THREADS)
 block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
                    int64_t j0, float maxqf, uint8_t* __restrict__ codes,
                    __half* __restrict__ scales, uint8_t* __restrict__ zeros,
-                   float* __restrict__ Eh_out, float* __restrict__ El_out,
+                   float* __restrict__ Eh_out, float* __restrict__ El_out, int64_t ldE,
                    float* __restrict__ row_loss, int first_block)
 {
     extern __shared__ __align__(16) float smem[];
-    float* Us = smem;                        // 128 x 128, strictly-lower part zeroed
+    float* Us = smem;                        // 128 x 128, strictly-lower part zeroed, swizzled
     float* rdiag = smem + SW_B * SW_B;       // 128: 1 / U_jj
     const int tid = threadIdx.x;
+    // Row j of the block is stored chunk-major: float4 chunk q of lane `sub`'s
+    // 8 columns at position q*16 + sub, so the 16 lanes of a row read 256
+    // contiguous bytes per float4 load (no bank conflicts).
     for (int idx = tid * 4; idx < SW_B * SW_B; idx += SW_THREADS * 4) {
         const int a = idx / SW_B, b = idx % SW_B;
         float4 v = *reinterpret_cast<const float4*>(U + (j0 + a) * d + j0 + b);
@@ -67,10 +70,11 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
         if (b + 1 < a) v.y = 0.f;
         if (b + 2 < a) v.z = 0.f;
         if (b + 3 < a) v.w = 0.f;
-        *reinterpret_cast<float4*>(Us + idx) = v;
+        const int f = b / 4;                 // natural float4 index in the row
+        *reinterpret_cast<float4*>(Us + a * SW_B + ((f & 1) * 16 + (f >> 1)) * 4) = v;
     }
+    if (tid < SW_B) rdiag[tid] = 1.0f / U[(j0 + tid) * d + j0 + tid];
     __syncthreads();
-    if (tid < SW_B) rdiag[tid] = 1.0f / Us[tid * SW_B + tid];
 
     const int lane = tid & 31, sub = lane & (SW_LPR - 1);
     const int src_base = lane & ~(SW_LPR - 1);
@@ -134,10 +138,10 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
                 Ev[ji] = Ej;
                 cp[ji / 4] |= uint32_t(c) << (8 * (ji % 4));
             }
-            const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B + SW_CPL * sub);
+            const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B);
 #pragma unroll
             for (int q4 = 0; q4 < SW_CPL / 4; ++q4) {
-                const float4 u = urow[q4];
+                const float4 u = urow[q4 * 16 + sub];
                 w[4 * q4 + 0] = fmaf(-Ej, u.x, w[4 * q4 + 0]);
                 w[4 * q4 + 1] = fmaf(-Ej, u.y, w[4 * q4 + 1]);
                 w[4 * q4 + 2] = fmaf(-Ej, u.z, w[4 * q4 + 2]);
@@ -148,8 +152,8 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     if (!valid) return;
     *reinterpret_cast<uint2*>(codes + row * d + j0 + SW_CPL * sub) = make_uint2(cp[0], cp[1]);
     // E split into its TF32 head and fp32 remainder for the tensor-core update
-    float4* hdst = reinterpret_cast<float4*>(Eh_out + row * SW_B + SW_CPL * sub);
-    float4* ldst = reinterpret_cast<float4*>(El_out + row * SW_B + SW_CPL * sub);
+    float4* hdst = reinterpret_cast<float4*>(Eh_out + row * ldE + SW_CPL * sub);
+    float4* ldst = reinterpret_cast<float4*>(El_out + row * ldE + SW_CPL * sub);
 #pragma unroll
     for (int q = 0; q < SW_CPL / 4; ++q) {
         float4 h, l;
@@ -230,14 +234,14 @@ static int check_quant_args(int w_dtype, int64_t m, int64_t d, int bits, int gro
 template <int GS>
 static void launch_sweep(dim3 grid, size_t smem, cudaStream_t st, const float* Wk, const float* U,
                          int64_t m, int64_t d, int64_t j0, float maxqf, uint8_t* codes,
-                         __half* scales, uint8_t* zeros, float* Eh, float* El, float* row_loss,
-                         int first)
+                         __half* scales, uint8_t* zeros, float* Eh, float* El, int64_t ldE,
+                         float* row_loss, int first)
 {
     cudaFuncSetAttribute(block_sweep_kernel<GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     block_sweep_kernel<GS><<<grid, SW_THREADS, smem, st>>>(Wk, U, m, d, j0, maxqf, codes, scales,
                                                           zeros,
-                                                   Eh, El, row_loss, first);
+                                                   Eh, El, ldE, row_loss, first);
     count_launches();
 }
 
@@ -287,19 +291,35 @@ extern "C" int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, in
     const dim3 grid((unsigned)ceil_div(m, SW_ROWS));
     const size_t smem = sizeof(float) * (SW_B * SW_B + SW_B);
     __half* sc = reinterpret_cast<__half*>(scales);
+    // Deferred (two-level) error feedback: after each 128-column block only the
+    // rest of its 512-column outer block is updated (K = 128); the columns
+    // beyond an outer block get the outer block's four blocks at once
+    // (K = 512) when it completes.  Every column still receives every earlier
+    // column's correction before its own block is swept.
     const int64_t nblk = d / SW_B;
     for (int64_t b = 0; b < nblk; ++b) {
         const int64_t j0 = b * SW_B;
+        const int64_t ob0 = (b / UPD_OUTER) * UPD_OUTER * SW_B;            // outer block start
+        const int64_t ob1 = std::min<int64_t>(d, ob0 + UPD_OUTER * SW_B);  // and end
+        const int64_t ecol = j0 - ob0;                                     // E column of this block
+        float* Eh = w.upd.Eh + ecol;
+        float* El = w.upd.El + ecol;
         switch (group_size) {
             case 32: launch_sweep<32>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                      w.upd.Eh, w.upd.El, row_loss, b == 0); break;
+                                      Eh, El, UPD_LDE, row_loss, b == 0); break;
             case 64: launch_sweep<64>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                      w.upd.Eh, w.upd.El, row_loss, b == 0); break;
+                                      Eh, El, UPD_LDE, row_loss, b == 0); break;
             default: launch_sweep<128>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                       w.upd.Eh, w.upd.El, row_loss, b == 0); break;
+                                       Eh, El, UPD_LDE, row_loss, b == 0); break;
         }
-        if (b + 1 < nblk) {
-            rc = block_update(w.Wk, &w.upd, m, d, j0, st);
+        if (j0 + SW_B < ob1) {                                   // near: rest of the outer block
+            rc = block_update(w.Wk, &w.upd, m, d, /*e_col0=*/ecol, /*k_rows=*/SW_B, /*u_row0=*/j0,
+                              /*c_begin=*/j0 + SW_B, /*c_end=*/ob1, st);
+            if (rc != GPTQ_OK) return rc;
+        }
+        if (j0 + SW_B == ob1 && ob1 < d) {                       // far: everything beyond it
+            rc = block_update(w.Wk, &w.upd, m, d, /*e_col0=*/0, /*k_rows=*/ob1 - ob0,
+                              /*u_row0=*/ob0, /*c_begin=*/ob1, /*c_end=*/d, st);
             if (rc != GPTQ_OK) return rc;
         }
     }

@@ -1,10 +1,10 @@
-// Inter-block update W[:, c0:] -= E . U[j0:j0+128, c0:], c0 = j0 + 128, on
-// tcgen05 tensor cores in split-TF32 (three kind::tf32 products, fp32
-// accumulation in TMEM).
+// Error-feedback update W[:, c0:c1] -= E[:, e0:e0+K] . U[u0:u0+K, c0:c1] on tcgen05
+// tensor cores in split-TF32 (three kind::tf32 products, fp32 accumulation in
+// TMEM); K = 128 (the rest of an outer block) or 512 (a whole outer block).
 //
 //  * Items are 128-row x 256-column output tiles of the trailing columns,
 //    handed round-robin to one persistent CTA per SM.
-//  * K = 128 (one block) in 4 stages of 32: E_hi, E_lo tiles (rows x 32) and
+//  * K in chunks of 32 through 2 stages: E_hi, E_lo tiles (rows x 32) and
 //    U_hi^T, U_lo^T tiles (256 columns x 32), all K-major with 128-byte
 //    swizzle, one TMA box each.  U is stored transposed because an MN-major
 //    tf32 operand would need the 32-byte-atom swizzle; K-major is the plain
@@ -20,7 +20,7 @@
 
 namespace gptq {
 
-constexpr int UB_M = 128, UB_N = 256, UB_KC = 32, UB_STAGES = 2, UB_KTOT = 128;
+constexpr int UB_M = 128, UB_N = 256, UB_KC = 32, UB_STAGES = 2;
 constexpr int UB_A_BYTES = UB_M * UB_KC * 4;                  // 16 KB per E tile
 constexpr int UB_B_BYTES = UB_KC * UB_N * 4;                  // 32 KB per U tile
 constexpr int UB_STAGE_BYTES = 2 * UB_A_BYTES + 2 * UB_B_BYTES;  // 96 KB
@@ -30,7 +30,8 @@ constexpr uint32_t UB_IDESC = make_idesc(2 /*tf32*/, UB_M, UB_N, 0 /*A K-major*/
 
 struct UpdParams {
     float* W;
-    int64_t m, d, j0, c0;
+    int64_t m, d, e0, u0, c0, c1;
+    int kchunks;
     int n_rt, n_ct, items;
 };
 
@@ -74,16 +75,16 @@ block_update_tc_kernel(const __grid_constant__ CUtensorMap tmEh,
                 const int rt = q % p.n_rt, ct = q / p.n_rt;
                 const int y_e = rt * UB_M;
                 const int x_u = (int)(p.c0 + int64_t(ct) * UB_N);
-                for (int kc = 0; kc < UB_KTOT / UB_KC; ++kc) {
+                for (int kc = 0; kc < p.kchunks; ++kc) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, kErrWaitEmpty, abort)) { ok = false; break; }
                     uint8_t* sEh = smem + stage * UB_STAGE_BYTES;
                     uint8_t* sEl = sEh + UB_A_BYTES;
                     uint8_t* sUh = sEl + UB_A_BYTES;
                     uint8_t* sUl = sUh + UB_B_BYTES;
                     mbar_arrive_expect_tx(&full_bar[stage], UB_STAGE_BYTES);
-                    tma_load_2d(sEh, &tmEh, &full_bar[stage], kc * UB_KC, y_e);
-                    tma_load_2d(sEl, &tmEl, &full_bar[stage], kc * UB_KC, y_e);
-                    const int k_u = (int)(p.j0 + kc * UB_KC);
+                    tma_load_2d(sEh, &tmEh, &full_bar[stage], (int)(p.e0 + kc * UB_KC), y_e);
+                    tma_load_2d(sEl, &tmEl, &full_bar[stage], (int)(p.e0 + kc * UB_KC), y_e);
+                    const int k_u = (int)(p.u0 + kc * UB_KC);
                     tma_load_2d(sUh, &tmUh, &full_bar[stage], k_u, x_u);
                     tma_load_2d(sUl, &tmUl, &full_bar[stage], k_u, x_u);
                     armed |= 1u << stage;
@@ -106,7 +107,7 @@ block_update_tc_kernel(const __grid_constant__ CUtensorMap tmEh,
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + uint32_t(a * UB_N);
                 uint32_t acc = 0;
-                for (int kc = 0; kc < UB_KTOT / UB_KC; ++kc) {
+                for (int kc = 0; kc < p.kchunks; ++kc) {
                     if (!mbar_wait(&full_bar[stage], phase, kErrWaitFull, abort)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sEh = smem_u32(smem + stage * UB_STAGE_BYTES);
@@ -148,7 +149,7 @@ block_update_tc_kernel(const __grid_constant__ CUtensorMap tmEh,
                 float v[32];
                 tmem_ld32(tmem + uint32_t(a * UB_N + c * 32) + (uint32_t(qr * 32) << 16), v);
                 const int64_t col = p.c0 + int64_t(ct) * UB_N + c * 32;
-                if (!row_ok || col >= p.d) continue;
+                if (!row_ok || col >= p.c1) continue;
                 float4* wp = reinterpret_cast<float4*>(Wrow + col);
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
@@ -194,13 +195,14 @@ split_tf32_transpose_kernel(const float* __restrict__ U, int64_t d, float* __res
 
 size_t update_ws_bytes(int64_t m, int64_t d)
 {
-    return align_up(sizeof(float) * d * d, 1024) * 2 + align_up(sizeof(float) * m * 128, 1024) * 2;
+    return align_up(sizeof(float) * d * d, 1024) * 2 +
+           align_up(sizeof(float) * m * UPD_LDE, 1024) * 2;
 }
 
 void update_ws_bind(int64_t m, int64_t d, char* base, UpdateWs* w)
 {
     const size_t u = align_up(sizeof(float) * d * d, 1024);
-    const size_t e = align_up(sizeof(float) * m * 128, 1024);
+    const size_t e = align_up(sizeof(float) * m * UPD_LDE, 1024);
     w->Uh = reinterpret_cast<float*>(base);
     w->Ul = reinterpret_cast<float*>(base + u);
     w->Eh = reinterpret_cast<float*>(base + 2 * u);
@@ -215,23 +217,28 @@ int update_prepare_u(const float* U, int64_t d, UpdateWs* w, cudaStream_t st)
     return launch_status();
 }
 
-int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t j0, cudaStream_t st)
+int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t e_col0,
+                 int64_t k_rows, int64_t u_row0, int64_t c_begin, int64_t c_end, cudaStream_t st)
 {
+    if (c_end <= c_begin) return GPTQ_OK;
+    if (k_rows <= 0 || k_rows % UB_KC != 0 || e_col0 + k_rows > UPD_LDE) return GPTQ_ERR_SHAPE;
     UpdParams p{};
     p.W = Wk;
     p.m = m;
     p.d = d;
-    p.j0 = j0;
-    p.c0 = j0 + UB_KTOT;
-    if (p.c0 >= d) return GPTQ_OK;
+    p.e0 = e_col0;
+    p.u0 = u_row0;
+    p.c0 = c_begin;
+    p.c1 = c_end;
+    p.kchunks = (int)(k_rows / UB_KC);
     p.n_rt = (int)ceil_div(m, UB_M);
-    p.n_ct = (int)ceil_div(d - p.c0, UB_N);
+    p.n_ct = (int)ceil_div(c_end - c_begin, UB_N);
     p.items = p.n_rt * p.n_ct;
     CUtensorMap tEh, tEl, tUh, tUl;
-    if (encode_tmap_2d(&tEh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Eh, 128, (uint64_t)m, 512, 32,
-                       128, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
-        encode_tmap_2d(&tEl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->El, 128, (uint64_t)m, 512, 32,
-                       128, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
+    if (encode_tmap_2d(&tEh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Eh, UPD_LDE, (uint64_t)m,
+                       UPD_LDE * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
+        encode_tmap_2d(&tEl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->El, UPD_LDE, (uint64_t)m,
+                       UPD_LDE * 4, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
         encode_tmap_2d(&tUh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Uh, (uint64_t)d, (uint64_t)d,
                        (uint64_t)d * 4, 32, UB_N, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
         encode_tmap_2d(&tUl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Ul, (uint64_t)d, (uint64_t)d,

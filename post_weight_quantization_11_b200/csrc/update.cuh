@@ -11,19 +11,24 @@
 
 namespace gptq {
 
+constexpr int UPD_OUTER = 4;                 // 128-column blocks per deferred outer block
+constexpr int64_t UPD_LDE = 128 * UPD_OUTER;  // row stride of the E buffers (512)
+
 struct UpdateWs {
     float* Uh;   // d x d, TF32-rounded U, TRANSPOSED (Uh[c][k] ~ U[k][c])
     float* Ul;   // d x d, U^T - Uh
-    float* Eh;   // m x 128, TF32-rounded scaled errors of the current block
-    float* El;   // m x 128, remainder
+    float* Eh;   // m x 512, TF32-rounded scaled errors of the current outer block
+    float* El;   // m x 512, remainder
 };
 
 size_t update_ws_bytes(int64_t m, int64_t d);
 void update_ws_bind(int64_t m, int64_t d, char* base, UpdateWs* w);
 // Split U into its TF32 head and fp32 remainder, transposed (once per layer).
 int update_prepare_u(const float* U, int64_t d, UpdateWs* w, cudaStream_t st);
-// W[:, j0+128:] -= (Eh + El) . (Uh + Ul)[j0:j0+128, j0+128:]  (lo x lo dropped)
-int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t j0, cudaStream_t st);
+// W[:, c_begin:c_end] -= E[:, e_col0 : e_col0+k_rows] . U[u_row0 : u_row0+k_rows, c_begin:c_end]
+// with E = Eh + El, U = Uh + Ul (lo x lo dropped); k_rows a multiple of 32.
+int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t e_col0,
+                 int64_t k_rows, int64_t u_row0, int64_t c_begin, int64_t c_end, cudaStream_t st);
 
 __device__ __forceinline__ float tf32_round(float x)
 {

@@ -9,8 +9,10 @@ Tolerances (written here, used by every parity test):
             feedback flips codes that sit at a rounding tie)
   * scales: for every group of a row before that row's first code mismatch,
             the GPU's fp16 scale is the fp16 rounding of some value within
-            1e-4 relative of the oracle's pre-fp16 scale; zero points equal
-            when the scales are equal
+            1e-4 relative of the oracle's pre-fp16 scale
+  * zero points: z = rne(-mn/s) is a rounding decision like the codes; under
+            equal scales they are equal except at most 1e-3 of the groups,
+            and those differ by one step
   * loss:   the layer loss tr(D H D^T) of the GPU's dequantized weights,
             evaluated in float64, within 1e-3 relative of the oracle's
   * teacher-forced diagnostic: with the GPU's decisions forced into the
@@ -68,8 +70,11 @@ def compare_sweep(gpu: dict, orc: dict, group_size: int, report: dict | None = N
     bad = ok_groups & ~in_range
     assert not bad.any(), f"{int(bad.sum())} scales outside 1e-4 of the oracle's pre-fp16 scale"
     same_s = gpu["scales"] == orc["scales"]
-    zbad = ok_groups & same_s & (gpu["zeros"] != orc["zeros"])
-    assert not zbad.any(), f"{int(zbad.sum())} zero points differ under equal scales"
+    zdiff = ok_groups & same_s & (gpu["zeros"] != orc["zeros"])
+    assert zdiff.sum() <= CODE_FRAC * max(1, ok_groups.sum()) + 1, \
+        f"{int(zdiff.sum())} zero points differ under equal scales"
+    zstep = np.abs(gpu["zeros"].astype(np.int32) - orc["zeros"].astype(np.int32))
+    assert (zstep[zdiff] <= 1).all(), "a zero point differs by more than one step"
     st = dict(code_mismatch_frac=frac, rows_with_mismatch=int((first < d).sum()),
               scale_exact_frac=float(same_s[ok_groups].mean()) if ok_groups.any() else 1.0)
     if report is not None:
