@@ -12,9 +12,9 @@
 //   3. A[i][j] = Hd[d-1-i][d-1-j], Hd = (2/n) S[perm][:, perm] + lambda I
 //   4. blocked right-looking Cholesky of A with 128-wide panels:
 //        leaf:  one CTA factors the 128x128 diagonal block and inverts it
-//               (L_kk, X_kk = L_kk^-1, Y_kk = X_kk^T): 32-column sub-panels
-//               factored and inverted by one warp with shuffles, panel solve
-//               and rank-32 updates by the whole CTA
+//               (L_kk, X_kk = L_kk^-1, Y_kk = X_kk^T): 4-column steps with a
+//               rank-4 trailing update, then the inverse from the 4x4
+//               diagonal inverses by doubling
 //        TRSM:  A[below, k] <- A[below, k] X_kk^T       (tensor-core GEMM)
 //        SYRK:  A[below, below] -= L21 L21^T, lower tiles (tensor-core GEMM)
 //   5. X = L^-1 by recursive doubling: for blocks [[A,0],[B,C]] (A of size s,

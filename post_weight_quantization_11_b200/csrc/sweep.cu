@@ -5,11 +5,12 @@
 //
 // Per 128-column block b (columns j0 .. j0+127, sweep order):
 //   block_sweep:  every row runs the 128 sequential steps with the block's
-//                 columns in registers (4 lanes per row, 32 columns per lane)
+//                 columns in registers (16 lanes per row, 8 columns per lane)
 //                 and U's 128x128 diagonal block in shared memory; writes the
 //                 codes, group scales/zeros, the scaled errors E (rows x 128)
 //                 and accumulates sum E_j^2 per row.
-//   block_update: W[:, j0+128:] -= E . U[j0:j0+128, j0+128:]
+//   block_update: W[:, cols] -= E . U[rows of E, cols], deferred in two
+//                 levels (see gptq_quantize_layer below)
 // Rows are independent given U, so a block's sweep is parallel over rows and
 // only the chain of blocks is sequential.
 #include "common.cuh"
