@@ -1,0 +1,496 @@
+// Cholesky factorization and triangular inverse of the damped Hessian as one
+// persistent, dependency-driven kernel -- "GPTQ / AWQ / SqueezeLLM" sec. 一
+// (decomposition of H^-1) and sec. 三 of "INT4/INT8 量化推理" (rows of H^-1
+// carry the error).
+//
+// The matrix is cut into 128x128 tiles, T = d / 128 per dimension.  Each
+// tile of L and of X = L^-1 is one task, left-looking:
+//   F(j)    diagonal:  B = A_jj - sum_{k<j} L_jk L_jk^T, then the one-CTA leaf
+//                      factors B = L_jj L_jj^T and inverts it (X_jj)
+//   S(i,j)  i > j:     L_ij = (A_ij - sum_{k<j} L_ik L_jk^T) X_jj^T
+//   I(i,j)  i > j:     X_ij = -X_ii sum_{j<=k<i} L_ik X_kj
+// Every sum runs on the tensor cores (split-TF32: A_hi B_hi + A_hi B_lo +
+// A_lo B_hi, fp32 accumulation in TMEM), one 128-deep product at a time,
+// folded into fp32 registers after each product.  The I tasks accumulate
+// the transpose, sum_k (X_kj)^T L_ik^T, so that every operand is read
+// K-major: they read Y = X^T, which they also write.
+//
+// Scheduling: tasks are numbered in an order in which every dependency of
+// a task has a smaller number, and each CTA claims the next number from an
+// atomic counter.  A CTA waits (bounded) only for tasks with smaller
+// numbers, which CTAs that already run hold, so the smallest unfinished task
+// can always proceed: no co-residency of the CTAs is needed.  Completion
+// flags are released at GPU scope after the task's stores; a consumer
+// acquires them and issues a proxy fence before its TMA loads read the data.
+//
+// Order of the numbers, phase p = 0 .. T-1 (the critical chain
+// F(p) -> S(p+1,p) -> F(p+1) is claimed early):
+//   phase 0:  F(0), S(1,0), F(1), S(2,0) .. S(T-1,0)
+//   phase p:  S(p+1,p), F(p+1), S(p+2,p) .. S(T-1,p), I(p,p-1) .. I(p,0)
+//   phase T-1: I(T-1,T-2) .. I(T-1,0)
+//
+// CTA roles (320 threads): warp 0 TMA producer (also waits for the
+// dependencies), warp 1 MMA issuer, warps 2-5 split the landed fp32 tiles
+// into TF32 head / remainder, warps 6-9 fold TMEM into registers and write
+// the task's results.  The leaf runs on all 320 threads.
+#include "chol_dag.cuh"
+#include "leaf.cuh"
+#include "tc_common.cuh"
+#include "update.cuh"
+
+namespace gptq {
+
+constexpr int CD_T = 128, CD_KC = 32, CD_STAGES = 3;
+constexpr int CD_TILE_BYTES = CD_T * CD_KC * 4;             // 16 KB
+constexpr int CD_STAGE_BYTES = 4 * CD_TILE_BYTES;           // A hi, A lo, B hi, B lo
+constexpr int CD_PIPE_BYTES = CD_STAGES * CD_STAGE_BYTES;   // 192 KB
+constexpr int CD_THREADS = 320;
+constexpr int CD_SMEM = CD_PIPE_BYTES + 1024 + 256;
+constexpr uint32_t CD_IDESC = make_idesc(2 /*tf32*/, CD_T, CD_T, 0, 0);
+static_assert(LSMEM <= (size_t)CD_PIPE_BYTES, "the leaf reuses the pipeline's shared memory");
+
+enum : int { kTaskF = 0, kTaskS = 1, kTaskI = 2 };
+enum : int { kMapA = 0, kMapX = 1, kMapY = 2 };
+
+struct CdParams {
+    float* A;
+    float* Xc;
+    float* Y;
+    float* U;
+    int* flagL;      // T x T: L_ij (and for i == j also X_jj, Y_jj) is final
+    int* flagY;      // T x T: Y_jk (k > j) is final
+    int* ticket;
+    int* gabort;     // set by a CTA that gave up: the others stop waiting
+    int32_t* info;
+    int64_t d;
+    int T, total;
+};
+
+struct CdProduct {
+    int ma, ra, ca;      // A operand: tensor map, first row, first column
+    int mb, rb, cb;      // B operand
+    const int* f1;       // flags to acquire first (nullptr: none)
+    const int* f2;
+};
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int* p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait for a completion flag (acquire).
+__device__ __forceinline__ bool cd_wait_flag(const int* f, volatile int* abort, const int* gabort)
+{
+    if (ld_acquire_gpu(f)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (unsigned it = 1;; ++it) {
+        __nanosleep(32);
+        if (ld_acquire_gpu(f)) return true;
+        if ((it & 15u) == 0) {
+            if (*abort || *reinterpret_cast<const volatile int*>(gabort)) {
+                *abort = 1;
+                return false;
+            }
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicCAS(&g_device_status, 0, kErrWaitDep);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Task number -> (type, i, j); see the order above.
+__device__ __forceinline__ void cd_decode(int t, int T, int& type, int& i, int& j)
+{
+    if (T == 1) { type = kTaskF; i = j = 0; return; }
+    if (t < T + 1) {
+        if (t == 0) { type = kTaskF; i = j = 0; }
+        else if (t == 1) { type = kTaskS; i = 1; j = 0; }
+        else if (t == 2) { type = kTaskF; i = j = 1; }
+        else { type = kTaskS; i = t - 1; j = 0; }
+        return;
+    }
+    const int r = t - (T + 1);
+    const int p = 1 + r / T, u = r % T;
+    if (p == T - 1) { type = kTaskI; i = p; j = p - 1 - u; return; }
+    if (u == 0) { type = kTaskS; i = p + 1; j = p; }
+    else if (u == 1) { type = kTaskF; i = j = p + 1; }
+    else if (u < T - p) { type = kTaskS; i = p + u; j = p; }
+    else { type = kTaskI; i = p; j = p - 1 - (u - (T - p)); }
+}
+
+// q-th product of a task's pass (pass 1: the sum; pass 2: the final product).
+__device__ __forceinline__ CdProduct cd_product(const CdParams& p, int type, int i, int j,
+                                                int pass, int q)
+{
+    const int T = p.T;
+    CdProduct r;
+    if (pass == 1) {
+        if (type == kTaskI) {               // (X_kj)^T L_ik^T: A = Y_jk, B = L_ik
+            const int k = j + q;
+            r = CdProduct{kMapY, j * CD_T, k * CD_T, kMapA, i * CD_T, k * CD_T,
+                          (k == j) ? &p.flagL[j * T + j] : &p.flagY[j * T + k],
+                          &p.flagL[i * T + k]};
+        } else {                            // L_ik L_jk^T
+            const int k = q;
+            r = CdProduct{kMapA, i * CD_T, k * CD_T, kMapA, j * CD_T, k * CD_T,
+                          &p.flagL[i * T + k], &p.flagL[j * T + k]};
+        }
+    } else if (type == kTaskS) {            // (A_ij - sum) X_jj^T
+        r = CdProduct{kMapA, i * CD_T, j * CD_T, kMapX, j * CD_T, 0, nullptr,
+                      &p.flagL[j * T + j]};
+    } else {                                // X_ii (sum^T)^T
+        r = CdProduct{kMapX, i * CD_T, 0, kMapY, j * CD_T, i * CD_T, &p.flagL[i * T + i],
+                      nullptr};
+    }
+    return r;
+}
+
+__global__ void __launch_bounds__(CD_THREADS, 1)
+chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
+                const __grid_constant__ CUtensorMap tmY, const CdParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + CD_PIPE_BYTES);
+    uint64_t* conv_bar = full_bar + CD_STAGES;
+    uint64_t* empty_bar = conv_bar + CD_STAGES;
+    uint64_t* accf_bar = empty_bar + CD_STAGES;
+    uint64_t* acce_bar = accf_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + 2);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* s_task = abort + 1;
+    float* la = reinterpret_cast<float*>(smem);          // leaf: block, then L
+    float* lx = la + PN * LDA;                           // leaf: X = L^-1
+    float* lt = lx + PN * LDA;                           // leaf: temporary
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t d = p.d;
+    const int T = p.T;
+    if (tid == 0) {
+        for (int s = 0; s < CD_STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&conv_bar[s], 256);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) { mbar_init(&accf_bar[a], 1); mbar_init(&acce_bar[a], 256); }
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // pipeline state of each role, carried across tasks
+    int pr_stage = 0, cv_stage = 0, mm_stage = 0;
+    uint32_t pr_phase = 0, cv_phase = 0, mm_phase = 0;
+    uint32_t armed = 0, armed_par = 0;
+    int mm_it = 0, ep_it = 0;
+    // warps 2-9: tile row m = qrow*32 + lane (TMEM lane quarter of the warp),
+    // columns [64 half, 64 half + 64)
+    const int qrow = warp & 3, half = (warp - 2) >> 2;
+    const int m = qrow * 32 + lane;
+    float acc[CD_T / 2];
+
+    // one pass of n products through the pipeline; warps 2-9 call epi(v, cc)
+    // with accumulator columns 64 half + 32 cc .. + 31 of each product, in order
+    auto run_pass = [&](int type, int ti, int tj, int pass, int n, auto&& epi) {
+        if (warp == 0) {
+            if (lane == 0) {
+                for (int q = 0; q < n; ++q) {
+                    const CdProduct pr = cd_product(p, type, ti, tj, pass, q);
+                    if (pr.f1 && !cd_wait_flag(pr.f1, abort, p.gabort)) break;
+                    if (pr.f2 && !cd_wait_flag(pr.f2, abort, p.gabort)) break;
+                    fence_proxy_async_global();
+                    const CUtensorMap* ma = pr.ma == kMapA ? &tmA : pr.ma == kMapX ? &tmX : &tmY;
+                    const CUtensorMap* mb = pr.mb == kMapA ? &tmA : pr.mb == kMapX ? &tmX : &tmY;
+                    bool ok = true;
+                    for (int kc = 0; kc < CD_T / CD_KC; ++kc) {
+                        if (!mbar_wait(&empty_bar[pr_stage], pr_phase ^ 1, kErrWaitEmpty, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t* st = smem + pr_stage * CD_STAGE_BYTES;
+                        mbar_arrive_expect_tx(&full_bar[pr_stage], 2 * CD_TILE_BYTES);
+                        tma_load_2d(st, ma, &full_bar[pr_stage], pr.ca + kc * CD_KC, pr.ra);
+                        tma_load_2d(st + 2 * CD_TILE_BYTES, mb, &full_bar[pr_stage],
+                                    pr.cb + kc * CD_KC, pr.rb);
+                        armed |= 1u << pr_stage;
+                        armed_par = (armed_par & ~(1u << pr_stage)) | (pr_phase << pr_stage);
+                        if (++pr_stage == CD_STAGES) { pr_stage = 0; pr_phase ^= 1; }
+                    }
+                    if (!ok) break;
+                }
+            }
+        } else if (warp == 1) {
+            if (lane == 0) {
+                bool ok = true;
+                for (int q = 0; q < n && ok; ++q, ++mm_it) {
+                    const int a = mm_it & 1;
+                    const uint32_t aph = (mm_it >> 1) & 1;
+                    if (!mbar_wait(&acce_bar[a], aph ^ 1, kErrWaitAccEmpty, abort)) break;
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem + uint32_t(a * CD_T);
+                    uint32_t accum = 0;
+                    for (int kc = 0; kc < CD_T / CD_KC; ++kc) {
+                        if (!mbar_wait(&conv_bar[mm_stage], mm_phase, kErrWaitFull, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t sAh = smem_u32(smem + mm_stage * CD_STAGE_BYTES);
+                        const uint32_t sAl = sAh + CD_TILE_BYTES;
+                        const uint32_t sBh = sAh + 2 * CD_TILE_BYTES;
+                        const uint32_t sBl = sAh + 3 * CD_TILE_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < CD_KC / 8; ++kk) {
+                            const uint64_t aH = smem_desc_sw128(sAh + kk * 32, 16, 1024);
+                            const uint64_t aL = smem_desc_sw128(sAl + kk * 32, 16, 1024);
+                            const uint64_t bH = smem_desc_sw128(sBh + kk * 32, 16, 1024);
+                            const uint64_t bL = smem_desc_sw128(sBl + kk * 32, 16, 1024);
+                            mma_tf32(d_tmem, aH, bH, CD_IDESC, accum);
+                            mma_tf32(d_tmem, aH, bL, CD_IDESC, 1u);
+                            mma_tf32(d_tmem, aL, bH, CD_IDESC, 1u);
+                            accum = 1;
+                        }
+                        mma_commit(&empty_bar[mm_stage]);
+                        if (++mm_stage == CD_STAGES) { mm_stage = 0; mm_phase ^= 1; }
+                    }
+                    if (ok) mma_commit(&accf_bar[a]);
+                }
+            }
+        } else {
+            // warps 2-9: split the chunks of product q, then fold product q-1
+            // (the MMA of q-1 overlaps the split of q)
+            const int ct = tid - 64;
+            bool ok = true;
+            for (int q = 0; q <= n && ok; ++q) {
+                if (q < n) {
+                    for (int kc = 0; kc < CD_T / CD_KC; ++kc) {
+                        if (!mbar_wait(&full_bar[cv_stage], cv_phase, kErrWaitFull, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t* st = smem + cv_stage * CD_STAGE_BYTES;
+#pragma unroll
+                        for (int op = 0; op < 2; ++op) {
+                            float4* hi = reinterpret_cast<float4*>(st + op * 2 * CD_TILE_BYTES);
+                            float4* lo = reinterpret_cast<float4*>(st + op * 2 * CD_TILE_BYTES +
+                                                                   CD_TILE_BYTES);
+#pragma unroll
+                            for (int u = 0; u < CD_TILE_BYTES / 16 / 256; ++u) {
+                                const int e = ct + 256 * u;
+                                const float4 x = hi[e];
+                                float4 hv, lv;
+                                hv.x = tf32_round(x.x); lv.x = x.x - hv.x;
+                                hv.y = tf32_round(x.y); lv.y = x.y - hv.y;
+                                hv.z = tf32_round(x.z); lv.z = x.z - hv.z;
+                                hv.w = tf32_round(x.w); lv.w = x.w - hv.w;
+                                hi[e] = hv;
+                                lo[e] = lv;
+                            }
+                        }
+                        fence_proxy_async_smem();
+                        mbar_arrive(&conv_bar[cv_stage]);
+                        if (++cv_stage == CD_STAGES) { cv_stage = 0; cv_phase ^= 1; }
+                    }
+                    if (!ok) break;
+                }
+                if (q > 0) {
+                    const int a = ep_it & 1;
+                    const uint32_t aph = (ep_it >> 1) & 1;
+                    ++ep_it;
+                    if (!mbar_wait(&accf_bar[a], aph, kErrWaitAccFull, abort)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float v[32];
+                        tmem_ld32(tmem + uint32_t(a * CD_T + (2 * half + cc) * 32) +
+                                      (uint32_t(qrow * 32) << 16), v);
+                        epi(v, cc);
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&acce_bar[a]);
+                }
+            }
+        }
+    };
+
+    for (;;) {
+        if (tid == 0) {
+            int t = p.total;
+            if (*abort) atomicExch(p.gabort, 1);
+            else if (!*reinterpret_cast<const volatile int*>(p.gabort)) t = atomicAdd(p.ticket, 1);
+            *s_task = t;
+        }
+        __syncthreads();
+        const int t = *s_task;
+        if (t >= p.total) break;
+        int type, ti, tj;
+        cd_decode(t, T, type, ti, tj);
+        const int n1 = (type == kTaskI) ? ti - tj : tj;
+        const int64_t r0 = int64_t(ti) * CD_T, c0 = int64_t(tj) * CD_T;
+
+        // ---- pass 1: the sum, folded into acc (row m, 64 columns per thread)
+        const int cb = 64 * half;                          // first column of this thread
+#pragma unroll
+        for (int u = 0; u < CD_T / 2; ++u) acc[u] = 0.f;
+        run_pass(type, ti, tj, 1, n1, [&](const float (&v)[32], int cc) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) acc[cc * 32 + u] += v[u];
+        });
+        if (warp >= 2) {
+            if (type == kTaskF) {
+                // leaf input B = A_jj - sum, X zeroed
+                const float4* src = reinterpret_cast<const float4*>(p.A + (c0 + m) * d + c0 + cb);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const float4 x = src[u];
+                    *reinterpret_cast<float4*>(la + m * LDA + cb + 4 * u) =
+                        make_float4(x.x - acc[4 * u], x.y - acc[4 * u + 1], x.z - acc[4 * u + 2],
+                                    x.w - acc[4 * u + 3]);
+                    *reinterpret_cast<float4*>(lx + m * LDA + cb + 4 * u) =
+                        make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            } else if (type == kTaskS && n1 > 0) {
+                // A_ij - sum, in place: the final product reads it back by TMA
+                float4* dst = reinterpret_cast<float4*>(p.A + (r0 + m) * d + c0 + cb);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const float4 x = dst[u];
+                    dst[u] = make_float4(x.x - acc[4 * u], x.y - acc[4 * u + 1],
+                                         x.z - acc[4 * u + 2], x.w - acc[4 * u + 3]);
+                }
+                fence_proxy_async_global();
+            } else if (type == kTaskI) {
+                // the sum's transpose (row m = column m of the sum) into the Y_ji
+                // tile, read back by TMA
+                float4* dst = reinterpret_cast<float4*>(p.Y + (c0 + m) * d + r0 + cb);
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    dst[u] = make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
+                fence_proxy_async_global();
+            }
+        }
+        __syncthreads();
+
+        if (type == kTaskF) {
+            leaf_factor_invert<CD_THREADS>(la, lx, lt, tid, p.info, d - c0);
+            // X_jj -> Xc, X_jj^T -> Y_jj, reversed X_jj -> the diagonal tile of U
+            const int64_t u0 = d - CD_T - c0;                 // U tile origin (row = column)
+            for (int idx = tid * 4; idx < CD_T * CD_T; idx += CD_THREADS * 4) {
+                const int r = idx / CD_T, c = idx % CD_T;
+                const float4 xv = *reinterpret_cast<const float4*>(lx + r * LDA + c);
+                *reinterpret_cast<float4*>(p.Xc + (c0 + r) * CD_T + c) = xv;
+                *reinterpret_cast<float4*>(p.Y + (c0 + r) * d + c0 + c) =
+                    make_float4(lx[(c + 0) * LDA + r], lx[(c + 1) * LDA + r],
+                                lx[(c + 2) * LDA + r], lx[(c + 3) * LDA + r]);
+                *reinterpret_cast<float4*>(p.U + (u0 + CD_T - 1 - r) * d + u0 + CD_T - 4 - c) =
+                    make_float4(xv.w, xv.z, xv.y, xv.x);
+            }
+            fence_proxy_async_global();
+            fence_proxy_async_smem();            // the pipeline's TMA reuses this memory
+        } else if (type == kTaskS) {
+            // L_ij = (A_ij - sum) X_jj^T into A; the mirrored tile of U is zero
+            float* lrow = p.A + (r0 + m) * d + c0 + cb;
+            float* zrow = p.U + (d - CD_T - c0 + m) * d + (d - CD_T - r0) + cb;
+            run_pass(type, ti, tj, 2, 1, [&](const float (&v)[32], int cc) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    reinterpret_cast<float4*>(lrow + cc * 32)[u] =
+                        make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                    reinterpret_cast<float4*>(zrow + cc * 32)[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            });
+            if (warp >= 2) fence_proxy_async_global();
+        } else {
+            // X_ij = -X_ii sum: Y_ji = X_ij^T, U gets X_ij reversed
+            float* urow = p.U + (d - 1 - r0 - m) * d + (d - c0);   // column of n: d - c0 - 1 - n
+            run_pass(type, ti, tj, 2, 1, [&](const float (&v)[32], int cc) {
+                const int nb = cb + cc * 32;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) p.Y[(c0 + nb + u) * d + r0 + m] = -v[u];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const int n0 = nb + 4 * g;                        // columns n0 .. n0+3
+                    *reinterpret_cast<float4*>(urow - n0 - 4) =
+                        make_float4(-v[4 * g + 3], -v[4 * g + 2], -v[4 * g + 1], -v[4 * g]);
+                }
+            });
+            if (warp >= 2) fence_proxy_async_global();
+        }
+        __syncthreads();
+        if (tid == 0 && !*abort) {
+            __threadfence();
+            int* f = (type == kTaskI) ? &p.flagY[tj * T + ti] : &p.flagL[ti * T + tj];
+            st_release_gpu(f, 1);
+        }
+    }
+
+    if (warp == 0 && lane == 0)
+        for (int s = 0; s < CD_STAGES; ++s)
+            if (armed & (1u << s)) mbar_drain(&full_bar[s], (armed_par >> s) & 1u);
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+size_t chol_dag_sync_bytes(int64_t d)
+{
+    const int64_t T = d / CD_T;
+    return sizeof(int) * size_t(2 * T * T + 32);
+}
+
+int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d, int32_t* info,
+                 cudaStream_t st)
+{
+    if (d < CD_T || d % CD_T) return GPTQ_ERR_SHAPE;
+    const int T = (int)(d / CD_T);
+    CdParams p{};
+    p.A = A; p.Xc = Xc; p.Y = Y; p.U = U;
+    int* s = reinterpret_cast<int*>(sync);
+    p.flagL = s;
+    p.flagY = s + size_t(T) * T;
+    p.ticket = s + size_t(2) * T * T;
+    p.gabort = p.ticket + 1;
+    p.info = info;
+    p.d = d;
+    p.T = T;
+    p.total = T * T;
+    if (cudaMemsetAsync(sync, 0, chol_dag_sync_bytes(d), st) != cudaSuccess) return GPTQ_ERR_CUDA;
+    CUtensorMap tA, tX, tY;
+    if (encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, A, (uint64_t)d, (uint64_t)d,
+                       (uint64_t)d * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
+        encode_tmap_2d(&tX, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Xc, (uint64_t)CD_T, (uint64_t)d,
+                       (uint64_t)CD_T * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
+        encode_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, (uint64_t)d, (uint64_t)d,
+                       (uint64_t)d * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK)
+        return GPTQ_ERR_CUDA;
+    if (cudaFuncSetAttribute(chol_dag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CD_SMEM) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    const int grid = std::min(p.total, device_sm_count());
+    chol_dag_kernel<<<grid, CD_THREADS, CD_SMEM, st>>>(tA, tX, tY, p);
+    count_launches();
+    return launch_status();
+}
+
+}  // namespace gptq

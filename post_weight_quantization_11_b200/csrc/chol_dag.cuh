@@ -1,0 +1,26 @@
+// Tiled Cholesky factorization + triangular inverse as one dependency-driven
+// persistent kernel (chol_dag.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace gptq {
+
+// Bytes of the synchronization area chol_inv_dag needs for T = d / 128
+// tiles per dimension (tile flags + the task ticket counter).
+size_t chol_dag_sync_bytes(int64_t d);
+
+// A (d x d, row-major): on entry its lower 128x128 tiles hold the symmetric
+// positive definite matrix to factor (the upper tiles are never read); on
+// exit its strictly-lower tiles hold those of L (A = L L^T), its diagonal
+// tiles are unspecified.
+// Xc (d x 128): on exit rows [128 j, 128 j + 128) hold X_jj = L_jj^-1.
+// Y (d x d): on exit its upper tiles (block row j <= block column k) hold
+// (L^-1)^T; the lower tiles are not touched.
+// U (d x d): on exit U[i][j] = (L^-1)[d-1-i][d-1-j] (upper; zeros below).
+// sync: chol_dag_sync_bytes(d) bytes of scratch (cleared here).
+// info: a non-positive pivot stores its position (as the leaf reports it).
+int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d, int32_t* info,
+                 cudaStream_t st);
+
+}  // namespace gptq

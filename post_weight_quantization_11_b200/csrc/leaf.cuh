@@ -1,0 +1,205 @@
+// 128x128 leaf of the blocked Cholesky factorization, on one CTA, in shared
+// memory -- "GPTQ / AWQ / SqueezeLLM" sec. 一 (decomposition of H^-1).
+//
+#pragma once
+
+#include "common.cuh"
+
+namespace gptq {
+
+constexpr int PN = 128;            // panel / leaf width
+// leaf_factor_invert: factor the symmetric block held in `a` (lower triangle
+// read) into L (lower, in `a`) and write X = L^-1 into `xs` (which the caller
+// zeroed), with every thread of the CTA busy at every step:
+//   * 4 columns per step: every thread factors and inverts the 4x4 diagonal
+//     block itself (10 shared-memory reads, no broadcast), one thread per row
+//     solves the 4 panel entries of its row, then a rank-4 update of the
+//     trailing lower triangle in 4x4 tiles -- two barriers per 4 columns;
+//   * X is assembled from the 4x4 diagonal inverses by five doubling levels,
+//     X_BC = -X_C (B X_A), as small GEMMs in shared memory.
+constexpr int LDA = PN + 4;                  // row stride of the shared 128x128 blocks
+constexpr int LDT = 68;                      // row stride of the doubling temporary
+constexpr size_t LSMEM = sizeof(float) * (2 * PN * LDA + 64 * LDT);
+
+__device__ __forceinline__ void tri_index(int t, int& r, int& c)
+{
+    const float x = 8.f * (float)t + 1.f;                 // estimate, corrected below
+    int u = (int)((x * rsqrtf(x) - 1.f) * 0.5f);
+    while ((u + 1) * (u + 2) / 2 <= t) ++u;
+    while (u > 0 && u * (u + 1) / 2 > t) --u;
+    r = u;
+    c = t - u * (u + 1) / 2;
+}
+
+// C (4x4 tile at rows i0.., cols j0..) = sum over k in [kb, ke) of P[i][k] Q[k][j]
+// with P, Q in shared memory (row strides ldp, ldq; k range a multiple of 4).
+__device__ __forceinline__ void tile_gemm4(const float* P, int ldp, const float* Q, int ldq,
+                                           int i0, int j0, int kb, int ke, float (&acc)[4][4])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int k = kb; k < ke; k += 4) {
+        float4 pr[4], qr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pr[i] = *reinterpret_cast<const float4*>(P + (i0 + i) * ldp + k);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) qr[q] = *reinterpret_cast<const float4*>(Q + (k + q) * ldq + j0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float pv[4] = {pr[i].x, pr[i].y, pr[i].z, pr[i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc[i][0] = fmaf(pv[q], qr[q].x, acc[i][0]);
+                acc[i][1] = fmaf(pv[q], qr[q].y, acc[i][1]);
+                acc[i][2] = fmaf(pv[q], qr[q].z, acc[i][2]);
+                acc[i][3] = fmaf(pv[q], qr[q].w, acc[i][3]);
+            }
+        }
+    }
+}
+
+// Shared memory: a (128 x LDA), xs (128 x LDA), tb (64 x LDT), 16-byte aligned.
+// A non-positive pivot at column c of the block stores piv0 - c into *info
+// (first one wins) and the factorization continues with NaN.  NT = threads of
+// the CTA; every thread must call (the function contains __syncthreads).
+template <int NT>
+__device__ __forceinline__ void leaf_factor_invert(float* __restrict__ a, float* __restrict__ xs,
+                                                   float* __restrict__ tb, int tid,
+                                                   int32_t* __restrict__ info, int64_t piv0)
+{
+    for (int c0 = 0; c0 < PN; c0 += 4) {
+        // 4x4 diagonal block: Cholesky factor g and its inverse h, in registers
+        float g[4][4], h[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) g[i][j] = (j <= i) ? a[(c0 + i) * LDA + c0 + j] : 0.f;
+        float rd[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float djj = g[j][j];
+            const bool bad = !(djj > 0.f);
+            if (bad && tid == 0 && info)
+                atomicCAS(reinterpret_cast<int*>(info), 0, (int)(piv0 - (c0 + j)));
+            // 1/sqrt(d) from the hardware estimate plus one Newton step (~1 ulp)
+            float y = rsqrtf(djj);
+            y = y * fmaf(-0.5f * djj * y, y, 1.5f);
+            if (bad) y = __int_as_float(0x7fc00000);
+            rd[j] = y;
+            g[j][j] = djj * y;
+#pragma unroll
+            for (int i = j + 1; i < 4; ++i) g[i][j] *= rd[j];
+#pragma unroll
+            for (int i = j + 1; i < 4; ++i)
+#pragma unroll
+                for (int k = j + 1; k <= i; ++k) g[i][k] = fmaf(-g[i][j], g[k][j], g[i][k]);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {                 // forward substitution, column c
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r < c) { h[r][c] = 0.f; continue; }
+                float t = (r == c) ? 1.f : 0.f;
+#pragma unroll
+                for (int k = c; k < r; ++k) t = fmaf(-g[r][k], h[k][c], t);
+                h[r][c] = t * rd[r];
+            }
+        }
+        // panel rows below: L[r][c0..c0+3] = A[r][c0..c0+3] h^T, one row per thread
+        const int rows = PN - c0 - 4;
+        if (tid < rows) {
+            const int r = c0 + 4 + tid;
+            const float4 v = *reinterpret_cast<const float4*>(a + r * LDA + c0);
+            const float av[4] = {v.x, v.y, v.z, v.w};
+            float o[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float t = 0.f;
+#pragma unroll
+                for (int k = 0; k <= c; ++k) t = fmaf(av[k], h[c][k], t);
+                o[c] = t;
+            }
+            *reinterpret_cast<float4*>(a + r * LDA + c0) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+        __syncthreads();
+        // the factored diagonal block replaces its input only now: every thread
+        // has read that input, and the rest of the step reads rows >= c0 + 4
+        if (tid == NT - 1) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                *reinterpret_cast<float4*>(a + (c0 + i) * LDA + c0) =
+                    make_float4(g[i][0], g[i][1], g[i][2], g[i][3]);
+                *reinterpret_cast<float4*>(xs + (c0 + i) * LDA + c0) =
+                    make_float4(h[i][0], h[i][1], h[i][2], h[i][3]);
+            }
+        }
+        // rank-4 update of the trailing lower triangle [c0+4, 128)
+        const int nt = rows / 4, tiles = nt * (nt + 1) / 2;
+        for (int t = tid; t < tiles; t += NT) {
+            int ti, tj;
+            tri_index(t, ti, tj);
+            const int r0 = c0 + 4 + 4 * ti, q0 = c0 + 4 + 4 * tj;
+            float4 lr[4], lc[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                lr[i] = *reinterpret_cast<const float4*>(a + (r0 + i) * LDA + c0);
+                lc[i] = *reinterpret_cast<const float4*>(a + (q0 + i) * LDA + c0);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float4 cur = *reinterpret_cast<const float4*>(a + (r0 + i) * LDA + q0);
+                float cv[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float t2 = cv[j];
+                    t2 = fmaf(-lr[i].x, lc[j].x, t2);
+                    t2 = fmaf(-lr[i].y, lc[j].y, t2);
+                    t2 = fmaf(-lr[i].z, lc[j].z, t2);
+                    t2 = fmaf(-lr[i].w, lc[j].w, t2);
+                    cv[j] = t2;
+                }
+                *reinterpret_cast<float4*>(a + (r0 + i) * LDA + q0) =
+                    make_float4(cv[0], cv[1], cv[2], cv[3]);
+            }
+        }
+        __syncthreads();
+    }
+
+    // X from the 4x4 diagonal inverses by doubling: s = 4, 8, ..., 64
+    for (int s = 4; s < PN; s *= 2) {
+        const int pairs = PN / (2 * s);
+        const int ts = s / 4, tpp = ts * ts;               // 4x4 tiles per pair
+        // T = B X_A, B = L[o+s+i][o+k], X_A = X[o+k][o+j] (zero for k < j)
+        for (int t = tid; t < pairs * tpp; t += NT) {
+            const int pr = t / tpp, tt = t % tpp;
+            const int o = pr * 2 * s;
+            const int i0 = (tt / ts) * 4, j0 = (tt % ts) * 4;
+            float acc[4][4];
+            tile_gemm4(a + (o + s) * LDA + o, LDA, xs + o * LDA + o, LDA, i0, j0, j0, s, acc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4*>(tb + (pr * s + i0 + i) * LDT + j0) =
+                    make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        }
+        __syncthreads();
+        // X_BC = -X_C T, X_C = X[o+s+i][o+s+k] (zero for k > i)
+        for (int t = tid; t < pairs * tpp; t += NT) {
+            const int pr = t / tpp, tt = t % tpp;
+            const int o = pr * 2 * s;
+            const int i0 = (tt / ts) * 4, j0 = (tt % ts) * 4;
+            float acc[4][4];
+            tile_gemm4(xs + (o + s) * LDA + o + s, LDA, tb + pr * s * LDT, LDT, i0, j0, 0, i0 + 4,
+                       acc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4*>(xs + (o + s + i0 + i) * LDA + o + j0) =
+                    make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
+        }
+        __syncthreads();
+    }
+
+}
+
+}  // namespace gptq

@@ -27,6 +27,7 @@ enum DeviceError : int {
     kErrWaitEmpty = 0x102,    // producer waited too long for a free stage
     kErrWaitAccFull = 0x103,  // epilogue waited too long for an accumulator
     kErrWaitAccEmpty = 0x104, // MMA waited too long for a drained accumulator
+    kErrWaitDep = 0x105,      // a task waited too long for a task it depends on
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
