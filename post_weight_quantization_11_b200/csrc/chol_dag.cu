@@ -57,8 +57,8 @@ struct CdParams {
     float* Xc;
     float* Y;
     float* U;
-    int* flagL;      // T x T: L_ij (and for i == j also X_jj, Y_jj) is final
-    int* flagY;      // T x T: Y_jk (k > j) is final
+    int* flagL;      // T x T: L_ij is final (for i == j: X_jj is in Xc)
+    int* flagY;      // T x T: Y_jk (k >= j) is final
     int* ticket;
     int* gabort;     // set by a CTA that gave up: the others stop waiting
     int32_t* info;
@@ -142,7 +142,7 @@ __device__ __forceinline__ CdProduct cd_product(const CdParams& p, int type, int
         if (type == kTaskI) {               // (X_kj)^T L_ik^T: A = Y_jk, B = L_ik
             const int k = j + q;
             r = CdProduct{kMapY, j * CD_T, k * CD_T, kMapA, i * CD_T, k * CD_T,
-                          (k == j) ? &p.flagL[j * T + j] : &p.flagY[j * T + k],
+                          &p.flagY[j * T + k],
                           &p.flagL[i * T + k]};
         } else {                            // L_ik L_jk^T
             const int k = q;
@@ -157,6 +157,42 @@ __device__ __forceinline__ CdProduct cd_product(const CdParams& p, int type, int
                       nullptr};
     }
     return r;
+}
+
+// Tile copies between the shared staging tile sb (128 x LDA floats) and
+// global memory, one warp per row so that every store is coalesced.
+__device__ __forceinline__ void cd_tile_out(const float* sb, float* dst, int64_t ld, int warp,
+                                            int lane)
+{
+    for (int r = warp; r < CD_T; r += CD_THREADS / 32)
+        *reinterpret_cast<float4*>(dst + r * ld + 4 * lane) =
+            *reinterpret_cast<const float4*>(sb + r * LDA + 4 * lane);
+}
+
+// dst[127 - r][127 - c] = sb[r][c]  (a tile of U from a tile of X)
+__device__ __forceinline__ void cd_tile_out_reversed(const float* sb, float* dst, int64_t ld,
+                                                     int warp, int lane)
+{
+    for (int r = warp; r < CD_T; r += CD_THREADS / 32) {
+        const float4 v = *reinterpret_cast<const float4*>(sb + r * LDA + 4 * lane);
+        *reinterpret_cast<float4*>(dst + (CD_T - 1 - r) * ld + CD_T - 4 - 4 * lane) =
+            make_float4(v.w, v.z, v.y, v.x);
+    }
+}
+
+// dst[c][r] = sb[r][c]  (lanes along r: coalesced stores, 4-way bank conflicts)
+__device__ __forceinline__ void cd_tile_out_transposed(const float* sb, float* dst, int64_t ld,
+                                                       int warp, int lane)
+{
+    for (int c = warp; c < CD_T; c += CD_THREADS / 32)
+#pragma unroll
+        for (int q = 0; q < CD_T / 32; ++q) dst[c * ld + 32 * q + lane] = sb[(32 * q + lane) * LDA + c];
+}
+
+__device__ __forceinline__ void cd_tile_zero(float* dst, int64_t ld, int warp, int lane)
+{
+    for (int r = warp; r < CD_T; r += CD_THREADS / 32)
+        *reinterpret_cast<float4*>(dst + r * ld + 4 * lane) = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 __global__ void __launch_bounds__(CD_THREADS, 1)
@@ -347,99 +383,111 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int n1 = (type == kTaskI) ? ti - tj : tj;
         const int64_t r0 = int64_t(ti) * CD_T, c0 = int64_t(tj) * CD_T;
 
-        // ---- pass 1: the sum, folded into acc (row m, 64 columns per thread)
         const int cb = 64 * half;                          // first column of this thread
-#pragma unroll
-        for (int u = 0; u < CD_T / 2; ++u) acc[u] = 0.f;
-        run_pass(type, ti, tj, 1, n1, [&](const float (&v)[32], int cc) {
-#pragma unroll
-            for (int u = 0; u < 32; ++u) acc[cc * 32 + u] += v[u];
-        });
-        if (warp >= 2) {
-            if (type == kTaskF) {
-                // leaf input B = A_jj - sum, X zeroed
-                const float4* src = reinterpret_cast<const float4*>(p.A + (c0 + m) * d + c0 + cb);
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const float4 x = src[u];
-                    *reinterpret_cast<float4*>(la + m * LDA + cb + 4 * u) =
-                        make_float4(x.x - acc[4 * u], x.y - acc[4 * u + 1], x.z - acc[4 * u + 2],
-                                    x.w - acc[4 * u + 3]);
-                    *reinterpret_cast<float4*>(lx + m * LDA + cb + 4 * u) =
-                        make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            } else if (type == kTaskS && n1 > 0) {
-                // A_ij - sum, in place: the final product reads it back by TMA
-                float4* dst = reinterpret_cast<float4*>(p.A + (r0 + m) * d + c0 + cb);
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const float4 x = dst[u];
-                    dst[u] = make_float4(x.x - acc[4 * u], x.y - acc[4 * u + 1],
-                                         x.z - acc[4 * u + 2], x.w - acc[4 * u + 3]);
-                }
-                fence_proxy_async_global();
-            } else if (type == kTaskI) {
-                // the sum's transpose (row m = column m of the sum) into the Y_ji
-                // tile, read back by TMA
-                float4* dst = reinterpret_cast<float4*>(p.Y + (c0 + m) * d + r0 + cb);
+        float* sb = la;                                    // staging tile (pipeline memory)
+        auto stage_acc = [&]() {                           // acc rows -> sb
+            if (warp >= 2) {
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
-                    dst[u] = make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
-                fence_proxy_async_global();
+                    *reinterpret_cast<float4*>(sb + m * LDA + cb + 4 * u) =
+                        make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
+            }
+        };
+        auto release = [&](int* f) {                       // after the task's stores
+            fence_proxy_async_global();
+            fence_proxy_async_smem();                      // the pipeline reuses sb
+            __syncthreads();
+            if (tid == 0 && !*abort) {
+                __threadfence();
+                st_release_gpu(f, 1);
+            }
+        };
+
+        // ---- pass 1: acc = A_ij - sum (F, S) or the sum's transpose (I), row m
+        if (type == kTaskI) {
+#pragma unroll
+            for (int u = 0; u < CD_T / 2; ++u) acc[u] = 0.f;
+        } else if (warp >= 2) {
+            const float4* src = reinterpret_cast<const float4*>(p.A + (r0 + m) * d + c0 + cb);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const float4 x = src[u];
+                acc[4 * u] = x.x; acc[4 * u + 1] = x.y; acc[4 * u + 2] = x.z; acc[4 * u + 3] = x.w;
             }
         }
-        __syncthreads();
+        if (type == kTaskS)           // the mirrored tile of U is zero
+            cd_tile_zero(p.U + (d - CD_T - c0) * d + (d - CD_T - r0), d, warp, lane);
+        const float sgn = (type == kTaskI) ? 1.f : -1.f;
+        run_pass(type, ti, tj, 1, n1, [&](const float (&v)[32], int cc) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) acc[cc * 32 + u] = fmaf(sgn, v[u], acc[cc * 32 + u]);
+        });
 
         if (type == kTaskF) {
+            // leaf on B = A_jj - sum, X zeroed
+            if (warp >= 2) {
+                stage_acc();
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    *reinterpret_cast<float4*>(lx + m * LDA + cb + 4 * u) =
+                        make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            __syncthreads();
             leaf_factor_invert<CD_THREADS>(la, lx, lt, tid, p.info, d - c0);
-            // X_jj -> Xc, X_jj^T -> Y_jj, reversed X_jj -> the diagonal tile of U
-            const int64_t u0 = d - CD_T - c0;                 // U tile origin (row = column)
+            // X_jj first: the S tasks of column j wait only for it
             for (int idx = tid * 4; idx < CD_T * CD_T; idx += CD_THREADS * 4) {
                 const int r = idx / CD_T, c = idx % CD_T;
-                const float4 xv = *reinterpret_cast<const float4*>(lx + r * LDA + c);
-                *reinterpret_cast<float4*>(p.Xc + (c0 + r) * CD_T + c) = xv;
-                *reinterpret_cast<float4*>(p.Y + (c0 + r) * d + c0 + c) =
-                    make_float4(lx[(c + 0) * LDA + r], lx[(c + 1) * LDA + r],
-                                lx[(c + 2) * LDA + r], lx[(c + 3) * LDA + r]);
-                *reinterpret_cast<float4*>(p.U + (u0 + CD_T - 1 - r) * d + u0 + CD_T - 4 - c) =
-                    make_float4(xv.w, xv.z, xv.y, xv.x);
+                *reinterpret_cast<float4*>(p.Xc + (c0 + r) * CD_T + c) =
+                    *reinterpret_cast<const float4*>(lx + r * LDA + c);
             }
             fence_proxy_async_global();
-            fence_proxy_async_smem();            // the pipeline's TMA reuses this memory
+            __syncthreads();
+            if (tid == 0 && !*abort) {
+                __threadfence();
+                st_release_gpu(&p.flagL[tj * T + tj], 1);
+            }
+            // then Y_jj = X_jj^T and the diagonal tile of U
+            cd_tile_out_transposed(lx, p.Y + c0 * d + c0, d, warp, lane);
+            cd_tile_out_reversed(lx, p.U + (d - CD_T - c0) * d + (d - CD_T - c0), d, warp, lane);
+            release(&p.flagY[tj * T + tj]);
         } else if (type == kTaskS) {
-            // L_ij = (A_ij - sum) X_jj^T into A; the mirrored tile of U is zero
-            float* lrow = p.A + (r0 + m) * d + c0 + cb;
-            float* zrow = p.U + (d - CD_T - c0 + m) * d + (d - CD_T - r0) + cb;
+            if (n1 > 0) {             // A_ij - sum back into A: the final product reads it
+                stage_acc();
+                __syncthreads();
+                cd_tile_out(sb, p.A + r0 * d + c0, d, warp, lane);
+                fence_proxy_async_global();
+                fence_proxy_async_smem();
+                __syncthreads();
+            }
+            // L_ij = (A_ij - sum) X_jj^T into A
             run_pass(type, ti, tj, 2, 1, [&](const float (&v)[32], int cc) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    reinterpret_cast<float4*>(lrow + cc * 32)[u] =
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<float4*>(sb + m * LDA + cb + cc * 32 + 4 * u) =
                         make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-                    reinterpret_cast<float4*>(zrow + cc * 32)[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
             });
-            if (warp >= 2) fence_proxy_async_global();
+            __syncthreads();
+            cd_tile_out(sb, p.A + r0 * d + c0, d, warp, lane);
+            release(&p.flagL[ti * T + tj]);
         } else {
+            // the sum's transpose into the Y_ji tile: the final product reads it
+            stage_acc();
+            __syncthreads();
+            cd_tile_out(sb, p.Y + c0 * d + r0, d, warp, lane);
+            fence_proxy_async_global();
+            fence_proxy_async_smem();
+            __syncthreads();
             // X_ij = -X_ii sum: Y_ji = X_ij^T, U gets X_ij reversed
-            float* urow = p.U + (d - 1 - r0 - m) * d + (d - c0);   // column of n: d - c0 - 1 - n
             run_pass(type, ti, tj, 2, 1, [&](const float (&v)[32], int cc) {
-                const int nb = cb + cc * 32;
 #pragma unroll
-                for (int u = 0; u < 32; ++u) p.Y[(c0 + nb + u) * d + r0 + m] = -v[u];
-#pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const int n0 = nb + 4 * g;                        // columns n0 .. n0+3
-                    *reinterpret_cast<float4*>(urow - n0 - 4) =
-                        make_float4(-v[4 * g + 3], -v[4 * g + 2], -v[4 * g + 1], -v[4 * g]);
-                }
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<float4*>(sb + m * LDA + cb + cc * 32 + 4 * u) =
+                        make_float4(-v[4 * u], -v[4 * u + 1], -v[4 * u + 2], -v[4 * u + 3]);
             });
-            if (warp >= 2) fence_proxy_async_global();
-        }
-        __syncthreads();
-        if (tid == 0 && !*abort) {
-            __threadfence();
-            int* f = (type == kTaskI) ? &p.flagY[tj * T + ti] : &p.flagL[ti * T + tj];
-            st_release_gpu(f, 1);
+            __syncthreads();
+            cd_tile_out_transposed(sb, p.Y + c0 * d + r0, d, warp, lane);
+            cd_tile_out_reversed(sb, p.U + (d - CD_T - r0) * d + (d - CD_T - c0), d, warp, lane);
+            release(&p.flagY[tj * T + ti]);
         }
     }
 
