@@ -433,7 +433,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         make_float4(0.f, 0.f, 0.f, 0.f);
             }
             __syncthreads();
-            leaf_factor_invert<CD_THREADS>(la, lx, lt, tid, p.info, d - c0);
+            leaf_factor_invert<CD_THREADS>(la, lx, lt, tid, p.info, d - c0, abort);
             // X_jj first: the S tasks of column j wait only for it
             for (int idx = tid * 4; idx < CD_T * CD_T; idx += CD_THREADS * 4) {
                 const int r = idx / CD_T, c = idx % CD_T;

@@ -4,22 +4,22 @@
 #pragma once
 
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace gptq {
 
 constexpr int PN = 128;            // panel / leaf width
 // leaf_factor_invert: factor the symmetric block held in `a` (lower triangle
 // read) into L (lower, in `a`) and write X = L^-1 into `xs` (which the caller
-// zeroed), with every thread of the CTA busy at every step:
-//   * 4 columns per step: every thread factors and inverts the 4x4 diagonal
-//     block itself (10 shared-memory reads, no broadcast), one thread per row
-//     solves the 4 panel entries of its row, then a rank-4 update of the
-//     trailing lower triangle in 4x4 tiles -- two barriers per 4 columns;
-//   * X is assembled from the 4x4 diagonal inverses by five doubling levels,
-//     X_BC = -X_C (B X_A), as small GEMMs in shared memory.
+// zeroed): a 4-column right-looking factorization pipelined between a panel
+// warp and update warps (below), then X from the 4x4 diagonal inverses by
+// five doubling levels, X_BC = -X_C (B X_A), as small GEMMs in shared memory.
 constexpr int LDA = PN + 4;                  // row stride of the shared 128x128 blocks
 constexpr int LDT = 68;                      // row stride of the doubling temporary
-constexpr size_t LSMEM = sizeof(float) * (2 * PN * LDA + 64 * LDT);
+constexpr int LPC_BYTES = 2 * PN * 16;       // two compact copies of a 4-column panel
+constexpr int LTB_BYTES = 64 * LDT * 4;      // tb: doubling temporary, or panel copies + mbarriers
+static_assert(LPC_BYTES + 64 <= LTB_BYTES, "panel copies and barriers fit in tb");
+constexpr size_t LSMEM = sizeof(float) * 2 * PN * LDA + LTB_BYTES;
 
 __device__ __forceinline__ void tri_index(int t, int& r, int& c)
 {
@@ -64,108 +64,183 @@ __device__ __forceinline__ void tile_gemm4(const float* P, int ldp, const float*
 // A non-positive pivot at column c of the block stores piv0 - c into *info
 // (first one wins) and the factorization continues with NaN.  NT = threads of
 // the CTA; every thread must call (the function contains __syncthreads).
+// Slot of row r in the compact copy of a panel: rows 4 apart (the rows one
+// warp's tiles read together) fall into distinct 16-byte slots of a 128-byte
+// line, so the float4 loads below take the minimum number of wavefronts.
+__device__ __forceinline__ int panel_slot(int r) { return r ^ ((r >> 3) & 7); }
+
+// a[r0..r0+3][q0..q0+3] -= L[r0..r0+3][c0..c0+3] L[q0..q0+3][c0..c0+3]^T, with
+// the panel's L rows read from its compact copy pc
+__device__ __forceinline__ void rank4_tile(float* __restrict__ a, const float4* __restrict__ pc,
+                                           int r0, int q0)
+{
+    float4 lr[4], lc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        lr[i] = pc[panel_slot(r0 + i)];
+        lc[i] = pc[panel_slot(q0 + i)];
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float4 cur = *reinterpret_cast<const float4*>(a + (r0 + i) * LDA + q0);
+        float cv[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float t2 = cv[j];
+            t2 = fmaf(-lr[i].x, lc[j].x, t2);
+            t2 = fmaf(-lr[i].y, lc[j].y, t2);
+            t2 = fmaf(-lr[i].z, lc[j].z, t2);
+            t2 = fmaf(-lr[i].w, lc[j].w, t2);
+            cv[j] = t2;
+        }
+        *reinterpret_cast<float4*>(a + (r0 + i) * LDA + q0) = make_float4(cv[0], cv[1], cv[2], cv[3]);
+    }
+}
+
+// Shared memory: a (128 x LDA), xs (128 x LDA), tb (LTB_BYTES), 16-byte
+// aligned.  A non-positive pivot at column c of the block stores piv0 - c
+// into *info (first one wins) and the factorization continues with NaN.
+// NT = threads of the CTA (a multiple of 32, at least 64); every thread must
+// call (the function uses __syncthreads).  `abort` is the CTA's abort flag of
+// the bounded waits (tc_common.cuh): a wait that gives up records
+// kErrWaitLeaf and every role leaves early; the block is then garbage.
+//
+// Factorization, 4 columns per step c0, software-pipelined across two roles:
+//   warp 0 (panel):   factor and invert the 4x4 pivot block in registers,
+//                     solve the 4 panel entries of every row below (into a,
+//                     and into a compact copy in tb, double-buffered by step
+//                     parity) and publish;
+//   warps 1.. (update): after the publish, first apply the panel's rank-4
+//                     update to the next panel's 4 columns and signal that
+//                     the panel warp may go on, then apply it to the rest of
+//                     the trailing triangle (columns >= c0 + 8, which the
+//                     panel warp neither reads nor writes in its next step).
+// The hand-offs are mbarriers alternating by step parity: pub[parity]
+// completes when the panel warp has published step c0 and every update warp
+// has finished the trailing update of step c0 - 4 (which orders the updates
+// of consecutive steps), nxt[parity] when every update warp has updated the
+// next panel's columns.  The next use of a barrier always follows a wait that
+// saw its previous phase complete.
 template <int NT>
 __device__ __forceinline__ void leaf_factor_invert(float* __restrict__ a, float* __restrict__ xs,
                                                    float* __restrict__ tb, int tid,
-                                                   int32_t* __restrict__ info, int64_t piv0)
+                                                   int32_t* __restrict__ info, int64_t piv0,
+                                                   volatile int* abort)
 {
-    for (int c0 = 0; c0 < PN; c0 += 4) {
-        // 4x4 diagonal block: Cholesky factor g and its inverse h, in registers
-        float g[4][4], h[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) g[i][j] = (j <= i) ? a[(c0 + i) * LDA + c0 + j] : 0.f;
-        float rd[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float djj = g[j][j];
-            const bool bad = !(djj > 0.f);
-            if (bad && tid == 0 && info)
-                atomicCAS(reinterpret_cast<int*>(info), 0, (int)(piv0 - (c0 + j)));
-            // 1/sqrt(d) from the hardware estimate plus one Newton step (~1 ulp)
-            float y = rsqrtf(djj);
-            y = y * fmaf(-0.5f * djj * y, y, 1.5f);
-            if (bad) y = __int_as_float(0x7fc00000);
-            rd[j] = y;
-            g[j][j] = djj * y;
-#pragma unroll
-            for (int i = j + 1; i < 4; ++i) g[i][j] *= rd[j];
-#pragma unroll
-            for (int i = j + 1; i < 4; ++i)
-#pragma unroll
-                for (int k = j + 1; k <= i; ++k) g[i][k] = fmaf(-g[i][j], g[k][j], g[i][k]);
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {                 // forward substitution, column c
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                if (r < c) { h[r][c] = 0.f; continue; }
-                float t = (r == c) ? 1.f : 0.f;
-#pragma unroll
-                for (int k = c; k < r; ++k) t = fmaf(-g[r][k], h[k][c], t);
-                h[r][c] = t * rd[r];
-            }
-        }
-        // panel rows below: L[r][c0..c0+3] = A[r][c0..c0+3] h^T, one row per thread
-        const int rows = PN - c0 - 4;
-        if (tid < rows) {
-            const int r = c0 + 4 + tid;
-            const float4 v = *reinterpret_cast<const float4*>(a + r * LDA + c0);
-            const float av[4] = {v.x, v.y, v.z, v.w};
-            float o[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float t = 0.f;
-#pragma unroll
-                for (int k = 0; k <= c; ++k) t = fmaf(av[k], h[c][k], t);
-                o[c] = t;
-            }
-            *reinterpret_cast<float4*>(a + r * LDA + c0) = make_float4(o[0], o[1], o[2], o[3]);
-        }
-        __syncthreads();
-        // the factored diagonal block replaces its input only now: every thread
-        // has read that input, and the rest of the step reads rows >= c0 + 4
-        if (tid == NT - 1) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                *reinterpret_cast<float4*>(a + (c0 + i) * LDA + c0) =
-                    make_float4(g[i][0], g[i][1], g[i][2], g[i][3]);
-                *reinterpret_cast<float4*>(xs + (c0 + i) * LDA + c0) =
-                    make_float4(h[i][0], h[i][1], h[i][2], h[i][3]);
-            }
-        }
-        // rank-4 update of the trailing lower triangle [c0+4, 128)
-        const int nt = rows / 4, tiles = nt * (nt + 1) / 2;
-        for (int t = tid; t < tiles; t += NT) {
-            int ti, tj;
-            tri_index(t, ti, tj);
-            const int r0 = c0 + 4 + 4 * ti, q0 = c0 + 4 + 4 * tj;
-            float4 lr[4], lc[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                lr[i] = *reinterpret_cast<const float4*>(a + (r0 + i) * LDA + c0);
-                lc[i] = *reinterpret_cast<const float4*>(a + (q0 + i) * LDA + c0);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float4 cur = *reinterpret_cast<const float4*>(a + (r0 + i) * LDA + q0);
-                float cv[4] = {cur.x, cur.y, cur.z, cur.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float t2 = cv[j];
-                    t2 = fmaf(-lr[i].x, lc[j].x, t2);
-                    t2 = fmaf(-lr[i].y, lc[j].y, t2);
-                    t2 = fmaf(-lr[i].z, lc[j].z, t2);
-                    t2 = fmaf(-lr[i].w, lc[j].w, t2);
-                    cv[j] = t2;
-                }
-                *reinterpret_cast<float4*>(a + (r0 + i) * LDA + q0) =
-                    make_float4(cv[0], cv[1], cv[2], cv[3]);
-            }
-        }
-        __syncthreads();
+    static_assert(NT % 32 == 0 && NT >= 64, "one panel warp and at least one update warp");
+    constexpr int NU = NT - 32;
+    const int warp = tid >> 5, lane = tid & 31;
+    float4* const pcb = reinterpret_cast<float4*>(tb);     // 2 x 128 compact panel copies
+    uint64_t* const pub = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(tb) + LPC_BYTES);
+    uint64_t* const nxt = pub + 2;
+    if (tid == 0) {
+        mbar_init(&pub[0], 1 + NU / 32);
+        mbar_init(&pub[1], 1 + NU / 32);
+        mbar_init(&nxt[0], NU / 32);
+        mbar_init(&nxt[1], NU / 32);
+        fence_mbar_init();
     }
+    __syncthreads();
+    if (warp == 0) {
+        for (int c0 = 0; c0 < PN; c0 += 4) {
+            const int st = c0 >> 2;
+            if (c0 > 0 && !mbar_wait(&nxt[(st - 1) & 1], ((st - 1) >> 1) & 1, kErrWaitLeaf, abort))
+                break;
+            // 4x4 diagonal block: Cholesky factor g and its inverse h, in registers
+            float g[4][4], h[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) g[i][j] = (j <= i) ? a[(c0 + i) * LDA + c0 + j] : 0.f;
+            float rd[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float djj = g[j][j];
+                const bool bad = !(djj > 0.f);
+                if (bad && lane == 0 && info)
+                    atomicCAS(reinterpret_cast<int*>(info), 0, (int)(piv0 - (c0 + j)));
+                // 1/sqrt(d) from the hardware estimate plus one Newton step (~1 ulp)
+                float y = rsqrtf(djj);
+                y = y * fmaf(-0.5f * djj * y, y, 1.5f);
+                if (bad) y = __int_as_float(0x7fc00000);
+                rd[j] = y;
+                g[j][j] = djj * y;
+#pragma unroll
+                for (int i = j + 1; i < 4; ++i) g[i][j] *= rd[j];
+#pragma unroll
+                for (int i = j + 1; i < 4; ++i)
+#pragma unroll
+                    for (int k = j + 1; k <= i; ++k) g[i][k] = fmaf(-g[i][j], g[k][j], g[i][k]);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {                 // forward substitution, column c
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (r < c) { h[r][c] = 0.f; continue; }
+                    float t = (r == c) ? 1.f : 0.f;
+#pragma unroll
+                    for (int k = c; k < r; ++k) t = fmaf(-g[r][k], h[k][c], t);
+                    h[r][c] = t * rd[r];
+                }
+            }
+            // panel rows below: L[r][c0..c0+3] = A[r][c0..c0+3] h^T
+            float4* pc = pcb + (st & 1) * PN;
+            for (int r = c0 + 4 + lane; r < PN; r += 32) {
+                const float4 v = *reinterpret_cast<const float4*>(a + r * LDA + c0);
+                const float av[4] = {v.x, v.y, v.z, v.w};
+                float o[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float t = 0.f;
+#pragma unroll
+                    for (int k = 0; k <= c; ++k) t = fmaf(av[k], h[c][k], t);
+                    o[c] = t;
+                }
+                const float4 lv = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4*>(a + r * LDA + c0) = lv;
+                pc[panel_slot(r)] = lv;
+            }
+            __syncwarp();                                  // every lane has read the pivot block
+            if (lane < 4) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (lane == i) {
+                        *reinterpret_cast<float4*>(a + (c0 + i) * LDA + c0) =
+                            make_float4(g[i][0], g[i][1], g[i][2], g[i][3]);
+                        *reinterpret_cast<float4*>(xs + (c0 + i) * LDA + c0) =
+                            make_float4(h[i][0], h[i][1], h[i][2], h[i][3]);
+                    }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pub[st & 1]);      // panel published
+        }
+    } else {
+        const int ut = tid - 32;
+        if (lane == 0) mbar_arrive(&pub[0]);              // nothing before step 0
+        for (int c0 = 0; c0 < PN; c0 += 4) {
+            const int st = c0 >> 2;
+            if (!mbar_wait(&pub[st & 1], (st >> 1) & 1, kErrWaitLeaf, abort)) break;
+            const int nt = (PN - c0 - 4) / 4;              // 4-row tiles below the panel
+            const float4* pc = pcb + (st & 1) * PN;
+            if (ut < nt) rank4_tile(a, pc, c0 + 4 + 4 * ut, c0 + 4);
+            __syncwarp();
+            if (c0 + 4 < PN && lane == 0) mbar_arrive(&nxt[st & 1]);   // next panel's columns
+            const int tiles = nt * (nt - 1) / 2;           // tile columns >= 1: columns >= c0 + 8
+            for (int t = ut; t < tiles; t += NU) {
+                int ti, tj;
+                tri_index(t, ti, tj);
+                rank4_tile(a, pc, c0 + 8 + 4 * ti, c0 + 8 + 4 * tj);
+            }
+            __syncwarp();
+            if (c0 + 4 < PN && lane == 0) mbar_arrive(&pub[(st + 1) & 1]);   // next step
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {                     // tb becomes the doubling temporary
+#pragma unroll
+        for (int b = 0; b < 4; ++b) mbar_inval(&pub[b]);
+    }
+    __syncthreads();
 
     // X from the 4x4 diagonal inverses by doubling: s = 4, 8, ..., 64
     for (int s = 4; s < PN; s *= 2) {

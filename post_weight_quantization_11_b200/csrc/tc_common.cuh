@@ -28,6 +28,7 @@ enum DeviceError : int {
     kErrWaitAccFull = 0x103,  // epilogue waited too long for an accumulator
     kErrWaitAccEmpty = 0x104, // MMA waited too long for a drained accumulator
     kErrWaitDep = 0x105,      // a task waited too long for a task it depends on
+    kErrWaitLeaf = 0x106,     // a role of the factorization leaf waited too long
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
@@ -39,6 +40,12 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                  : "memory");
+}
+
+// The memory of an mbarrier may serve another purpose only after this.
+__device__ __forceinline__ void mbar_inval(uint64_t* bar)
+{
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void fence_mbar_init()
