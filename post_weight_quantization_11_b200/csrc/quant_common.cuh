@@ -13,6 +13,7 @@ namespace gptq {
 struct GroupQ {
     float s;      // fp16 scale as fp32 (exact)
     float z;      // zero point as an integral fp32
+    float r;      // fl(1 / s), for quant_code_fast
     __half h;     // fp16 scale
 };
 
@@ -31,6 +32,7 @@ __device__ __forceinline__ GroupQ group_params(float mn, float mx, float maxqf)
     g.s = __half2float(h);
     float zf = rintf(__fdiv_rn(-mn, g.s));
     g.z = fminf(fmaxf(zf, 0.f), maxqf);
+    g.r = __frcp_rn(g.s);
     return g;
 }
 
@@ -38,6 +40,26 @@ __device__ __forceinline__ GroupQ group_params(float mn, float mx, float maxqf)
 __device__ __forceinline__ float quant_code(float x, const GroupQ& g, float maxqf)
 {
     float c = __fadd_rn(rintf(__fdiv_rn(x, g.s)), g.z);
+    return fminf(fmaxf(c, 0.f), maxqf);
+}
+
+// The same value as quant_code, without a division: with r = RN(1/s) and a
+// quotient q within one ulp of x/s, RN(q + RN(x - q s) r) is the correctly
+// rounded quotient RN(x/s) (Markstein's theorem for division with a
+// correctly rounded reciprocal; x - q s is exact in one FMA).  x r alone can
+// be 1.5 ulp off, so the correction is applied twice: the first brings q
+// within one ulp, the second rounds it correctly.  No overflow or underflow
+// can occur: s is a finite fp16 value >= 2^-24.
+__device__ __forceinline__ float div_rn_recip(float x, float s, float r)
+{
+    float q = x * r;
+    q = fmaf(fmaf(-q, s, x), r, q);
+    return fmaf(fmaf(-q, s, x), r, q);
+}
+
+__device__ __forceinline__ float quant_code_fast(float x, const GroupQ& g, float maxqf)
+{
+    const float c = __fadd_rn(rintf(div_rn_recip(x, g.s, g.r)), g.z);
     return fminf(fmaxf(c, 0.f), maxqf);
 }
 

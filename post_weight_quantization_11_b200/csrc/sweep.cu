@@ -20,10 +20,11 @@
 namespace gptq {
 
 constexpr int SW_B = 128;          // block width (columns)
-constexpr int SW_LPR = 16;         // lanes per row
-constexpr int SW_CPL = SW_B / SW_LPR;   // columns per lane (8)
+constexpr int SW_LPR = 8;          // lanes per row
+constexpr int SW_CPL = SW_B / SW_LPR;   // columns per lane (16)
+constexpr int SW_Q4 = SW_CPL / 4;       // float4 chunks per lane (4)
 constexpr int SW_THREADS = 256;
-constexpr int SW_ROWS = SW_THREADS / SW_LPR;   // rows per CTA (16)
+constexpr int SW_ROWS = SW_THREADS / SW_LPR;   // rows per CTA (32)
 constexpr unsigned FULL = 0xffffffffu;
 
 // W_work[r][k] = float(W[r][perm[k]])
@@ -40,11 +41,13 @@ __global__ void init_work_kernel(const T* __restrict__ W, const int32_t* __restr
     }
 }
 
-// One 128-column block of the sweep for all rows.  16 lanes per row, each
-// holding 8 consecutive columns in registers; U's 128x128 diagonal block (its
+// One 128-column block of the sweep for all rows.  8 lanes per row (4 rows per
+// warp, so the per-column decision is issued once for 4 rows), each holding 16
+// consecutive columns in registers; U's 128x128 diagonal block (its
 // strictly-lower part zeroed) and 1/U_jj in shared memory.  Step j: the owner
 // lane's w_j is broadcast with a shuffle, every lane of the row takes the same
-// fp32 decision, and each lane applies w[k] -= E_j U[j][k] to its columns.
+// fp32 decision (quant_code_fast: no division on the common path), and each
+// lane applies w[k] -= E_j U[j][k] to its columns.
 // At a group's first column the group's min/max is reduced over the row's
 // lanes (lanes outside the group contribute 0, neutral since the range
 // includes 0).  The outer loop over the 16 owner lanes is not unrolled, which
@@ -62,19 +65,31 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     float* rdiag = smem + SW_B * SW_B;       // 128: 1 / U_jj
     const int tid = threadIdx.x;
     // Row j of the block is stored chunk-major: float4 chunk q of lane `sub`'s
-    // 8 columns at position q*16 + sub, so the 16 lanes of a row read 256
-    // contiguous bytes per float4 load (no bank conflicts).
-    for (int idx = tid * 4; idx < SW_B * SW_B; idx += SW_THREADS * 4) {
+    // 16 columns at position q*8 + sub, so the 8 lanes of a row read 128
+    // contiguous bytes per float4 load (no bank conflicts; the 4 rows of a
+    // warp read the same U row).
+    // all loads of the block first (16 per thread in flight), then the stores
+    constexpr int UPT = SW_B * SW_B / 4 / SW_THREADS;   // float4 per thread
+    float4 uv[UPT];
+#pragma unroll
+    for (int i = 0; i < UPT; ++i) {
+        const int idx = (tid + i * SW_THREADS) * 4;
+        uv[i] = *reinterpret_cast<const float4*>(U + (j0 + idx / SW_B) * d + j0 + idx % SW_B);
+    }
+    const float udiag = (tid < SW_B) ? U[(j0 + tid) * d + j0 + tid] : 1.f;
+#pragma unroll
+    for (int i = 0; i < UPT; ++i) {
+        const int idx = (tid + i * SW_THREADS) * 4;
         const int a = idx / SW_B, b = idx % SW_B;
-        float4 v = *reinterpret_cast<const float4*>(U + (j0 + a) * d + j0 + b);
+        float4 v = uv[i];
         if (b + 0 < a) v.x = 0.f;
         if (b + 1 < a) v.y = 0.f;
         if (b + 2 < a) v.z = 0.f;
         if (b + 3 < a) v.w = 0.f;
         const int f = b / 4;                 // natural float4 index in the row
-        *reinterpret_cast<float4*>(Us + a * SW_B + ((f & 1) * 16 + (f >> 1)) * 4) = v;
+        *reinterpret_cast<float4*>(Us + a * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4) = v;
     }
-    if (tid < SW_B) rdiag[tid] = 1.0f / U[(j0 + tid) * d + j0 + tid];
+    if (tid < SW_B) rdiag[tid] = 1.0f / udiag;
     __syncthreads();
 
     const int lane = tid & 31, sub = lane & (SW_LPR - 1);
@@ -103,8 +118,14 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     for (int q = 0; q < SW_CPL / 4; ++q) cp[q] = 0u;
     float loss = 0.f;
     GroupQ gq;
-    gq.s = 1.f; gq.z = 0.f; gq.h = __float2half(1.f);
+    gq.s = 1.f; gq.z = 0.f; gq.r = 1.f; gq.h = __float2half(1.f);
 
+    // Look-ahead broadcast: xn is the value of the next column to quantize,
+    // identical on the row's 8 lanes.  The pre-update value of column j+1 is
+    // shuffled from its owner while column j is decided, and every lane then
+    // applies column j's single correction to it itself (the owner applies the
+    // same FMA to its register), so the shuffle is off the dependency chain.
+    float xn = __shfl_sync(FULL, w[0], src_base);
 #pragma unroll 1
     for (int jo = 0; jo < SW_LPR; ++jo) {
 #pragma unroll
@@ -129,8 +150,19 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
                     zeros[row * G + gi] = (uint8_t)gq.z;
                 }
             }
-            const float x = __shfl_sync(FULL, w[ji], src_base | jo);
-            const float c = quant_code(x, gq, maxqf);
+            // next column's value before this column's correction (off the chain)
+            float xpre = 0.f, unext = 0.f;
+            if (ji + 1 < SW_CPL) {
+                xpre = __shfl_sync(FULL, w[ji + 1], src_base | jo);
+            } else if (jo + 1 < SW_LPR) {
+                xpre = __shfl_sync(FULL, w[0], src_base | (jo + 1));
+            }
+            if (j + 1 < SW_B) {
+                const int f = (j + 1) >> 2;
+                unext = Us[j * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 + ((j + 1) & 3)];
+            }
+            const float x = xn;
+            const float c = quant_code_fast(x, gq, maxqf);
             const float q = gq.s * (c - gq.z);
             const float e = x - q;
             const float Ej = e * rdiag[j];
@@ -139,10 +171,11 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
                 Ev[ji] = Ej;
                 cp[ji / 4] |= uint32_t(c) << (8 * (ji % 4));
             }
+            xn = fmaf(-Ej, unext, xpre);
             const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B);
 #pragma unroll
-            for (int q4 = 0; q4 < SW_CPL / 4; ++q4) {
-                const float4 u = urow[q4 * 16 + sub];
+            for (int q4 = 0; q4 < SW_Q4; ++q4) {
+                const float4 u = urow[q4 * SW_LPR + sub];
                 w[4 * q4 + 0] = fmaf(-Ej, u.x, w[4 * q4 + 0]);
                 w[4 * q4 + 1] = fmaf(-Ej, u.y, w[4 * q4 + 1]);
                 w[4 * q4 + 2] = fmaf(-Ej, u.z, w[4 * q4 + 2]);
@@ -151,7 +184,9 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
         }
     }
     if (!valid) return;
-    *reinterpret_cast<uint2*>(codes + row * d + j0 + SW_CPL * sub) = make_uint2(cp[0], cp[1]);
+    static_assert(SW_CPL == 16, "codes of a lane are stored as one uint4");
+    *reinterpret_cast<uint4*>(codes + row * d + j0 + SW_CPL * sub) =
+        make_uint4(cp[0], cp[1], cp[2], cp[3]);
     // E split into its TF32 head and fp32 remainder for the tensor-core update
     float4* hdst = reinterpret_cast<float4*>(Eh_out + row * ldE + SW_CPL * sub);
     float4* ldst = reinterpret_cast<float4*>(El_out + row * ldE + SW_CPL * sub);
