@@ -23,8 +23,8 @@ constexpr int SW_B = 128;          // block width (columns)
 constexpr int SW_LPR = 8;          // lanes per row
 constexpr int SW_CPL = SW_B / SW_LPR;   // columns per lane (16)
 constexpr int SW_Q4 = SW_CPL / 4;       // float4 chunks per lane (4)
-constexpr int SW_THREADS = 256;
-constexpr int SW_ROWS = SW_THREADS / SW_LPR;   // rows per CTA (32)
+constexpr int SW_THREADS = 128;
+constexpr int SW_ROWS = 2 * SW_THREADS / SW_LPR;   // rows per CTA (32: two per lane group)
 constexpr unsigned FULL = 0xffffffffu;
 
 // W_work[r][k] = float(W[r][perm[k]])
@@ -41,17 +41,19 @@ __global__ void init_work_kernel(const T* __restrict__ W, const int32_t* __restr
     }
 }
 
-// One 128-column block of the sweep for all rows.  8 lanes per row (4 rows per
-// warp, so the per-column decision is issued once for 4 rows), each holding 16
-// consecutive columns in registers; U's 128x128 diagonal block (its
-// strictly-lower part zeroed) and 1/U_jj in shared memory.  Step j: the owner
-// lane's w_j is broadcast with a shuffle, every lane of the row takes the same
-// fp32 decision (quant_code_fast: no division on the common path), and each
-// lane applies w[k] -= E_j U[j][k] to its columns.
-// At a group's first column the group's min/max is reduced over the row's
-// lanes (lanes outside the group contribute 0, neutral since the range
-// includes 0).  The outer loop over the 16 owner lanes is not unrolled, which
-// keeps the kernel's code small.
+// One 128-column block of the sweep for all rows.  8 lanes per row, each lane
+// holding 16 consecutive columns of TWO rows in registers (rows g and g+4 of
+// its warp's 8), so every U value a lane reads from shared memory serves two
+// rows and each warp carries two independent decision chains.  U's 128x128
+// diagonal block (its strictly-lower part zeroed) and 1/U_jj live in shared
+// memory.  Step j: every lane of a row takes the same fp32 decision on column
+// j (quant_code_fast: no division) and applies w[k] -= E_j U[j][k] to its
+// columns; the next column's value is shuffled from its owner before the
+// decision and each lane applies the one correction itself, so the shuffle
+// is off the dependency chain.  At a group's first column the group's
+// min/max is reduced over the row's lanes (lanes outside the group
+// contribute 0, neutral since the range includes 0).  The outer loop over the
+// 8 owner lanes is not unrolled, which keeps the kernel's code small.
 template <int GS>
 __global__ void __launch_bounds__(SW_THREADS)
 block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
@@ -66,66 +68,72 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     const int tid = threadIdx.x;
     // Row j of the block is stored chunk-major: float4 chunk q of lane `sub`'s
     // 16 columns at position q*8 + sub, so the 8 lanes of a row read 128
-    // contiguous bytes per float4 load (no bank conflicts; the 4 rows of a
-    // warp read the same U row).
-    // all loads of the block first (16 per thread in flight), then the stores
-    constexpr int UPT = SW_B * SW_B / 4 / SW_THREADS;   // float4 per thread
-    float4 uv[UPT];
+    // contiguous bytes per float4 load.  All loads of a half block first, then
+    // the stores.
+    constexpr int UPT = SW_B * SW_B / 4 / SW_THREADS / 2;   // float4 per thread per half
 #pragma unroll
-    for (int i = 0; i < UPT; ++i) {
-        const int idx = (tid + i * SW_THREADS) * 4;
-        uv[i] = *reinterpret_cast<const float4*>(U + (j0 + idx / SW_B) * d + j0 + idx % SW_B);
-    }
-    const float udiag = (tid < SW_B) ? U[(j0 + tid) * d + j0 + tid] : 1.f;
+    for (int hb = 0; hb < 2; ++hb) {
+        float4 uv[UPT];
 #pragma unroll
-    for (int i = 0; i < UPT; ++i) {
-        const int idx = (tid + i * SW_THREADS) * 4;
-        const int a = idx / SW_B, b = idx % SW_B;
-        float4 v = uv[i];
-        if (b + 0 < a) v.x = 0.f;
-        if (b + 1 < a) v.y = 0.f;
-        if (b + 2 < a) v.z = 0.f;
-        if (b + 3 < a) v.w = 0.f;
-        const int f = b / 4;                 // natural float4 index in the row
-        *reinterpret_cast<float4*>(Us + a * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4) = v;
+        for (int i = 0; i < UPT; ++i) {
+            const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
+            uv[i] = *reinterpret_cast<const float4*>(U + (j0 + idx / SW_B) * d + j0 + idx % SW_B);
+        }
+#pragma unroll
+        for (int i = 0; i < UPT; ++i) {
+            const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
+            const int a = idx / SW_B, b = idx % SW_B;
+            float4 v = uv[i];
+            if (b + 0 < a) v.x = 0.f;
+            if (b + 1 < a) v.y = 0.f;
+            if (b + 2 < a) v.z = 0.f;
+            if (b + 3 < a) v.w = 0.f;
+            const int f = b / 4;                 // natural float4 index in the row
+            *reinterpret_cast<float4*>(Us + a * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4) = v;
+        }
     }
-    if (tid < SW_B) rdiag[tid] = 1.0f / udiag;
-    __syncthreads();
+    if (tid < SW_B) rdiag[tid] = 1.0f / U[(j0 + tid) * d + j0 + tid];
 
     const int lane = tid & 31, sub = lane & (SW_LPR - 1);
     const int src_base = lane & ~(SW_LPR - 1);
-    const int64_t row = int64_t(blockIdx.x) * SW_ROWS + (tid / SW_LPR);
-    const bool valid = row < m;
+    const int64_t rbase = int64_t(blockIdx.x) * SW_ROWS + (tid >> 5) * 8 + (lane >> 3);
+    int64_t row[2];
+    bool valid[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) { row[r] = rbase + 4 * r; valid[r] = row[r] < m; }
     const int64_t G = d / GS;
 
-    float w[SW_CPL];
-    if (valid) {
-        const float4* p = reinterpret_cast<const float4*>(Wk + row * d + j0 + SW_CPL * sub);
+    float w[2][SW_CPL];
 #pragma unroll
-        for (int q = 0; q < SW_CPL / 4; ++q) {
-            const float4 v = p[q];
-            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+    for (int r = 0; r < 2; ++r) {
+        if (valid[r]) {
+            const float4* p = reinterpret_cast<const float4*>(Wk + row[r] * d + j0 + SW_CPL * sub);
+#pragma unroll
+            for (int q = 0; q < SW_Q4; ++q) {
+                const float4 v = p[q];
+                w[r][4 * q] = v.x; w[r][4 * q + 1] = v.y; w[r][4 * q + 2] = v.z; w[r][4 * q + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < SW_CPL; ++q) w[r][q] = 0.f;
         }
-    } else {
-#pragma unroll
-        for (int q = 0; q < SW_CPL; ++q) w[q] = 0.f;
     }
     __syncthreads();
 
-    float Ev[SW_CPL];
-    uint32_t cp[SW_CPL / 4];
+    float Ev[2][SW_CPL];
+    uint32_t cp[2][SW_Q4];
+    float loss[2] = {0.f, 0.f};
+    GroupQ gq[2];
 #pragma unroll
-    for (int q = 0; q < SW_CPL / 4; ++q) cp[q] = 0u;
-    float loss = 0.f;
-    GroupQ gq;
-    gq.s = 1.f; gq.z = 0.f; gq.r = 1.f; gq.h = __float2half(1.f);
+    for (int r = 0; r < 2; ++r) {
+#pragma unroll
+        for (int q = 0; q < SW_Q4; ++q) cp[r][q] = 0u;
+        gq[r].s = 1.f; gq[r].z = 0.f; gq[r].r = 1.f; gq[r].h = __float2half(1.f);
+    }
+    float xn[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) xn[r] = __shfl_sync(FULL, w[r][0], src_base);
 
-    // Look-ahead broadcast: xn is the value of the next column to quantize,
-    // identical on the row's 8 lanes.  The pre-update value of column j+1 is
-    // shuffled from its owner while column j is decided, and every lane then
-    // applies column j's single correction to it itself (the owner applies the
-    // same FMA to its register), so the shuffle is off the dependency chain.
-    float xn = __shfl_sync(FULL, w[0], src_base);
 #pragma unroll 1
     for (int jo = 0; jo < SW_LPR; ++jo) {
 #pragma unroll
@@ -133,74 +141,90 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
             const int j = jo * SW_CPL + ji;
             if (ji == 0 && (jo * SW_CPL) % GS == 0) {
                 constexpr int span = GS / SW_CPL;            // lanes covering one group
-                float mn = 0.f, mx = 0.f;
-                if (sub >= jo && sub < jo + span) {
+                const bool in_group = sub >= jo && sub < jo + span;
 #pragma unroll
-                    for (int q = 0; q < SW_CPL; ++q) { mn = fminf(mn, w[q]); mx = fmaxf(mx, w[q]); }
-                }
+                for (int r = 0; r < 2; ++r) {
+                    float mn = 0.f, mx = 0.f;
+                    if (in_group) {
 #pragma unroll
-                for (int o = 1; o < SW_LPR; o <<= 1) {
-                    mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
-                    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-                }
-                gq = group_params(mn, mx, maxqf);
-                if (valid && sub == jo) {
-                    const int64_t gi = (j0 + j) / GS;
-                    scales[row * G + gi] = gq.h;
-                    zeros[row * G + gi] = (uint8_t)gq.z;
+                        for (int q = 0; q < SW_CPL; ++q) { mn = fminf(mn, w[r][q]); mx = fmaxf(mx, w[r][q]); }
+                    }
+#pragma unroll
+                    for (int o = 1; o < SW_LPR; o <<= 1) {
+                        mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+                        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+                    }
+                    gq[r] = group_params(mn, mx, maxqf);
+                    if (valid[r] && sub == jo) {
+                        const int64_t gi = (j0 + j) / GS;
+                        scales[row[r] * G + gi] = gq[r].h;
+                        zeros[row[r] * G + gi] = (uint8_t)gq[r].z;
+                    }
                 }
             }
-            // next column's value before this column's correction (off the chain)
-            float xpre = 0.f, unext = 0.f;
-            if (ji + 1 < SW_CPL) {
-                xpre = __shfl_sync(FULL, w[ji + 1], src_base | jo);
-            } else if (jo + 1 < SW_LPR) {
-                xpre = __shfl_sync(FULL, w[0], src_base | (jo + 1));
+            // next column's values before this column's correction (off the chain)
+            float xpre[2] = {0.f, 0.f};
+            float unext = 0.f;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                if (ji + 1 < SW_CPL) xpre[r] = __shfl_sync(FULL, w[r][ji + 1], src_base | jo);
+                else if (jo + 1 < SW_LPR) xpre[r] = __shfl_sync(FULL, w[r][0], src_base | (jo + 1));
             }
             if (j + 1 < SW_B) {
                 const int f = (j + 1) >> 2;
                 unext = Us[j * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 + ((j + 1) & 3)];
             }
-            const float x = xn;
-            const float c = quant_code_fast(x, gq, maxqf);
-            const float q = gq.s * (c - gq.z);
-            const float e = x - q;
-            const float Ej = e * rdiag[j];
-            loss = fmaf(Ej, Ej, loss);
-            if (sub == jo) {
-                Ev[ji] = Ej;
-                cp[ji / 4] |= uint32_t(c) << (8 * (ji % 4));
+            const float rdj = rdiag[j];
+            float Ej[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const float x = xn[r];
+                const float c = quant_code_fast(x, gq[r], maxqf);
+                const float q = gq[r].s * (c - gq[r].z);
+                Ej[r] = (x - q) * rdj;
+                loss[r] = fmaf(Ej[r], Ej[r], loss[r]);
+                if (sub == jo) {
+                    Ev[r][ji] = Ej[r];
+                    cp[r][ji / 4] |= uint32_t(c) << (8 * (ji % 4));
+                }
+                xn[r] = fmaf(-Ej[r], unext, xpre[r]);
             }
-            xn = fmaf(-Ej, unext, xpre);
             const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B);
 #pragma unroll
             for (int q4 = 0; q4 < SW_Q4; ++q4) {
                 const float4 u = urow[q4 * SW_LPR + sub];
-                w[4 * q4 + 0] = fmaf(-Ej, u.x, w[4 * q4 + 0]);
-                w[4 * q4 + 1] = fmaf(-Ej, u.y, w[4 * q4 + 1]);
-                w[4 * q4 + 2] = fmaf(-Ej, u.z, w[4 * q4 + 2]);
-                w[4 * q4 + 3] = fmaf(-Ej, u.w, w[4 * q4 + 3]);
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    w[r][4 * q4 + 0] = fmaf(-Ej[r], u.x, w[r][4 * q4 + 0]);
+                    w[r][4 * q4 + 1] = fmaf(-Ej[r], u.y, w[r][4 * q4 + 1]);
+                    w[r][4 * q4 + 2] = fmaf(-Ej[r], u.z, w[r][4 * q4 + 2]);
+                    w[r][4 * q4 + 3] = fmaf(-Ej[r], u.w, w[r][4 * q4 + 3]);
+                }
             }
         }
     }
-    if (!valid) return;
-    static_assert(SW_CPL == 16, "codes of a lane are stored as one uint4");
-    *reinterpret_cast<uint4*>(codes + row * d + j0 + SW_CPL * sub) =
-        make_uint4(cp[0], cp[1], cp[2], cp[3]);
-    // E split into its TF32 head and fp32 remainder for the tensor-core update
-    float4* hdst = reinterpret_cast<float4*>(Eh_out + row * ldE + SW_CPL * sub);
-    float4* ldst = reinterpret_cast<float4*>(El_out + row * ldE + SW_CPL * sub);
 #pragma unroll
-    for (int q = 0; q < SW_CPL / 4; ++q) {
-        float4 h, l;
-        h.x = tf32_round(Ev[4 * q + 0]); l.x = Ev[4 * q + 0] - h.x;
-        h.y = tf32_round(Ev[4 * q + 1]); l.y = Ev[4 * q + 1] - h.y;
-        h.z = tf32_round(Ev[4 * q + 2]); l.z = Ev[4 * q + 2] - h.z;
-        h.w = tf32_round(Ev[4 * q + 3]); l.w = Ev[4 * q + 3] - h.w;
-        hdst[q] = h;
-        ldst[q] = l;
+    for (int r = 0; r < 2; ++r) {
+        if (!valid[r]) continue;
+        static_assert(SW_CPL == 16, "codes of a lane are stored as one uint4");
+        *reinterpret_cast<uint4*>(codes + row[r] * d + j0 + SW_CPL * sub) =
+            make_uint4(cp[r][0], cp[r][1], cp[r][2], cp[r][3]);
+        // E split into its TF32 head and fp32 remainder for the tensor-core update
+        float4* hdst = reinterpret_cast<float4*>(Eh_out + row[r] * ldE + SW_CPL * sub);
+        float4* ldst = reinterpret_cast<float4*>(El_out + row[r] * ldE + SW_CPL * sub);
+#pragma unroll
+        for (int q = 0; q < SW_Q4; ++q) {
+            float4 h, l;
+            h.x = tf32_round(Ev[r][4 * q + 0]); l.x = Ev[r][4 * q + 0] - h.x;
+            h.y = tf32_round(Ev[r][4 * q + 1]); l.y = Ev[r][4 * q + 1] - h.y;
+            h.z = tf32_round(Ev[r][4 * q + 2]); l.z = Ev[r][4 * q + 2] - h.z;
+            h.w = tf32_round(Ev[r][4 * q + 3]); l.w = Ev[r][4 * q + 3] - h.w;
+            hdst[q] = h;
+            ldst[q] = l;
+        }
+        if (row_loss && sub == 0)
+            row_loss[row[r]] = first_block ? loss[r] : row_loss[row[r]] + loss[r];
     }
-    if (row_loss && sub == 0) row_loss[row] = first_block ? loss : row_loss[row] + loss;
 }
 
 // Round-to-nearest: one warp per (row, 128-column segment), 4 columns per lane.
