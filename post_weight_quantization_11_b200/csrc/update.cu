@@ -12,7 +12,8 @@
 //  * warp 0: TMA; warp 1: per 8-wide k-step E_hi U_hi + E_hi U_lo + E_lo U_hi
 //    into one of two TMEM accumulators (2 x 256 columns); warps 2-5: read the
 //    accumulator (tcgen05.ld) and write W - D back, overlapping the next
-//    tile's MMAs.
+//    tile's MMAs; each thread's row of W is read two 32-column chunks ahead,
+//    the first two before the accumulator is ready.
 //  * Every mbarrier wait is bounded (see tc_common.cuh).
 #include "common.cuh"
 #include "tc_common.cuh"
@@ -139,27 +140,46 @@ block_update_tc_kernel(const __grid_constant__ CUtensorMap tmEh,
             const int rt = q % p.n_rt, ct = q / p.n_rt;
             const int a = it & 1;
             const uint32_t aph = (it >> 1) & 1;
-            if (!mbar_wait(&accf_bar[a], aph, kErrWaitAccFull, abort)) break;
-            tc_fence_after();
             const int64_t i = int64_t(rt) * UB_M + qr * 32 + lane;
             const bool row_ok = i < p.m;
             float* Wrow = p.W + i * p.d;
-#pragma unroll 1
-            for (int c = 0; c < UB_N / 32; ++c) {
+            const int64_t col0 = p.c0 + int64_t(ct) * UB_N;
+            // W is read two 32-column chunks ahead; the first two are requested
+            // before the accumulator is ready, so their latency hides behind the
+            // tile's MMAs.
+            constexpr int NCH = UB_N / 32;
+            float4 wbuf[2][8];
+            auto load_chunk = [&](int c, float4 (&dst)[8]) {
+                const int64_t col = col0 + c * 32;
+                if (row_ok && col < p.c1) {
+                    const float4* wp = reinterpret_cast<const float4*>(Wrow + col);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) dst[u] = wp[u];
+                }
+            };
+            load_chunk(0, wbuf[0]);
+            load_chunk(1, wbuf[1]);
+            if (!mbar_wait(&accf_bar[a], aph, kErrWaitAccFull, abort)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
                 float v[32];
                 tmem_ld32(tmem + uint32_t(a * UB_N + c * 32) + (uint32_t(qr * 32) << 16), v);
-                const int64_t col = p.c0 + int64_t(ct) * UB_N + c * 32;
-                if (!row_ok || col >= p.c1) continue;
-                float4* wp = reinterpret_cast<float4*>(Wrow + col);
+                const int64_t col = col0 + c * 32;
+                float4 (&cur)[8] = wbuf[c & 1];
+                if (row_ok && col < p.c1) {
+                    float4* wp = reinterpret_cast<float4*>(Wrow + col);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    float4 w4 = wp[u];
-                    w4.x -= v[4 * u + 0];
-                    w4.y -= v[4 * u + 1];
-                    w4.z -= v[4 * u + 2];
-                    w4.w -= v[4 * u + 3];
-                    wp[u] = w4;
+                    for (int u = 0; u < 8; ++u) {
+                        float4 w4 = cur[u];
+                        w4.x -= v[4 * u + 0];
+                        w4.y -= v[4 * u + 1];
+                        w4.z -= v[4 * u + 2];
+                        w4.w -= v[4 * u + 3];
+                        wp[u] = w4;
+                    }
                 }
+                if (c + 2 < NCH) load_chunk(c + 2, cur);
             }
             tc_fence_before();
             mbar_arrive(&acce_bar[a]);
