@@ -9,7 +9,8 @@
 // Steps (all on the device):
 //   1. keys + lambda: diag(S), lambda = damp * mean(2 S_ii / n)
 //   2. perm: stable descending rank of S_ii (act-order) or identity
-//   3. A[i][j] = Hd[d-1-i][d-1-j], Hd = (2/n) S[perm][:, perm] + lambda I
+//   3. A[i][j] = Hd[d-1-i][d-1-j], Hd = (2/n) S[perm][:, perm] + lambda I,
+//      for the lower 128x128 tiles (the only ones the factorization reads)
 //   4. L (A = L L^T) and X = L^-1 by 128x128 tiles in one dependency-driven
 //      persistent kernel (chol_dag.cu): a one-CTA leaf factors and inverts
 //      each diagonal tile, the off-diagonal tiles of L and X are split-TF32
@@ -105,6 +106,10 @@ __global__ void rank_perm_kernel(const float* __restrict__ keys, int64_t d, int 
     if (i < d) perm[rank] = (int32_t)i;
 }
 
+// A[i][j] = Hd[d-1-i][d-1-j] for the lower tiles only (j < 128 (i/128 + 1)):
+// the factorization reads nothing else.  Inside a diagonal tile the entries
+// above the diagonal are set to 0.  For j <= i (b >= a) the source is S's
+// upper triangle read along row a (coalesced for the identity permutation).
 __global__ void build_reversed_kernel(const float* __restrict__ S, const int32_t* __restrict__ perm,
                                       const float* __restrict__ lam, int64_t d, float scale,
                                       float* __restrict__ A)
@@ -113,13 +118,17 @@ __global__ void build_reversed_kernel(const float* __restrict__ S, const int32_t
     const int64_t a = d - 1 - i;
     const int32_t pa = perm[a];
     const float l = lam[0];
-    for (int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; j < d;
+    const int64_t jend = (i / 128 + 1) * 128;
+    for (int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; j < jend;
          j += int64_t(gridDim.x) * blockDim.x) {
-        const int64_t b = d - 1 - j;
-        const int32_t pb = perm[b];
-        const int64_t r = min(pa, pb), c = max(pa, pb);
-        float v = scale * S[r * d + c];
-        if (a == b) v += l;
+        float v = 0.f;
+        if (j <= i) {
+            const int64_t b = d - 1 - j;
+            const int32_t pb = perm[b];
+            const int64_t r = min(pa, pb), c = max(pa, pb);
+            v = scale * S[r * d + c];
+            if (a == b) v += l;
+        }
         A[i * d + j] = v;
     }
 }
