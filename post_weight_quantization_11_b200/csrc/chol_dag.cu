@@ -73,45 +73,6 @@ struct CdProduct {
     const int* f2;
 };
 
-__device__ __forceinline__ int ld_acquire_gpu(const int* p)
-{
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(int* p, int v)
-{
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_global()
-{
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Bounded wait for a completion flag (acquire).
-__device__ __forceinline__ bool cd_wait_flag(const int* f, volatile int* abort, const int* gabort)
-{
-    if (ld_acquire_gpu(f)) return true;
-    const unsigned long long t0 = globaltimer_ns();
-    for (unsigned it = 1;; ++it) {
-        __nanosleep(32);
-        if (ld_acquire_gpu(f)) return true;
-        if ((it & 15u) == 0) {
-            if (*abort || *reinterpret_cast<const volatile int*>(gabort)) {
-                *abort = 1;
-                return false;
-            }
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                atomicCAS(&g_device_status, 0, kErrWaitDep);
-                *abort = 1;
-                return false;
-            }
-        }
-    }
-}
-
 // Task number -> (type, i, j); see the order above.
 __device__ __forceinline__ void cd_decode(int t, int T, int& type, int& i, int& j)
 {

@@ -119,6 +119,51 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity)
         if (globaltimer_ns() - t0 > kWaitLimitNs) return;
 }
 
+// ---- completion flags between CTAs -------------------------------------
+// A producer CTA stores its results, fences them for the async proxy (they
+// may be read by TMA), synchronizes, and one thread releases a flag at GPU
+// scope; a consumer acquires the flag (bounded wait) and issues a proxy
+// fence before its TMA loads read the data.
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int* p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait for a completion flag (acquire).
+__device__ __forceinline__ bool cd_wait_flag(const int* f, volatile int* abort, const int* gabort)
+{
+    if (ld_acquire_gpu(f)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (unsigned it = 1;; ++it) {
+        __nanosleep(32);
+        if (ld_acquire_gpu(f)) return true;
+        if ((it & 15u) == 0) {
+            if (*abort || *reinterpret_cast<const volatile int*>(gabort)) {
+                *abort = 1;
+                return false;
+            }
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicCAS(&g_device_status, 0, kErrWaitDep);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
 // 2D tiled TMA load into shared memory, completing on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y)
