@@ -141,7 +141,9 @@ int gptq_prepare_hinv_static(const float* S, int64_t d, int64_t n_tokens, float 
  *   E_j = e / U[j][j];  w[k] -= E_j U[j][k] for k > j;  row_loss[r] += E_j^2
  * (decisions in IEEE fp32; maxq = 2^bits - 1).  The feedback inside each
  * block of block_size columns is applied column by column on the CUDA cores;
- * the feedback onto later blocks is one tensor-core product per block.
+ * the feedback onto later blocks is applied on the tensor cores in two
+ * levels: after each block onto the rest of its 512-column outer block
+ * (K = 128), and once per outer block onto every column beyond it (K = 512).
  *
  * W: d_out x d_in, dtype GPTQ_DTYPE_F16 or GPTQ_DTYPE_F32 (read only).
  * U: d_in x d_in fp32 from gptq_prepare_hinv (upper triangle read).
