@@ -104,11 +104,18 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        """Start sampling every 25 ms and return once the first sample (taken
+        before the timed region, and discarded) has arrived, so the samples
+        that follow cover the timed region even when it lasts under 100 ms."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "25"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import select
+            ready, _, _ = select.select([self.proc.stdout], [], [], 3.0)
+            if ready:
+                self.proc.stdout.readline()
         except Exception:
             self.proc = None
         return self
