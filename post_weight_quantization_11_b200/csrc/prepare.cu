@@ -163,8 +163,9 @@ extern "C" int gptq_prepare_hinv(const float* S, int64_t d, int64_t n_tokens, fl
     rank_perm_kernel<<<(unsigned)ceil_div(d, 256), 256, 0, st>>>(w.keys, d, act_order, p);
     count_launches();
     {
-        dim3 grid((unsigned)std::min<int64_t>(ceil_div(d, 256), 16), (unsigned)d);
-        build_reversed_kernel<<<grid, 256, 0, st>>>(S, p, w.lam, d, 2.0f / float(n_tokens), w.A);
+        // one CTA per row: rows hold 128 .. d entries of the lower tiles
+        build_reversed_kernel<<<dim3(1, (unsigned)d), 256, 0, st>>>(S, p, w.lam, d,
+                                                                    2.0f / float(n_tokens), w.A);
         count_launches();
     }
     if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
