@@ -3,9 +3,7 @@
 // TMEM); K = 128 (the rest of an outer block) or 512 (a whole outer block).
 //
 //  * Items are 128-row x N-column output tiles of the trailing columns
-//    (N = 256; N = 128 for the near updates, which cover at most 384
-//    columns, so they get twice the CTAs), handed round-robin to one
-//    persistent CTA per SM.
+//    (N = 128), handed round-robin to one persistent CTA per SM.
 //  * K in chunks of 32: E_hi, E_lo tiles (rows x 32) and U_hi^T, U_lo^T
 //    tiles (N columns x 32), all K-major with 128-byte swizzle, one TMA box
 //    each.  U is stored transposed because an MN-major tf32 operand would
@@ -23,9 +21,8 @@
 
 namespace gptq {
 
-// Tile width N: 256 columns (far updates, many tiles) or 128 (near updates:
-// a few hundred columns, so narrower tiles give more CTAs and a shorter MMA
-// chain per tile).
+// Tile width N (128 is the one launched: more CTAs and a shorter MMA chain
+// for the near updates, and three pipeline stages instead of two).
 constexpr int UB_M = 128, UB_KC = 32;
 constexpr int UB_A_BYTES = UB_M * UB_KC * 4;                  // 16 KB per E tile
 constexpr int UB_THREADS = 192;
@@ -284,9 +281,10 @@ int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t e_c
         kern<<<grid, UB_THREADS, smem, st>>>(tEh, tEl, tUh, tUl, p);
         return GPTQ_OK;
     };
-    // near updates (the rest of an outer block, at most 384 columns): 128-wide tiles
-    const int rc = cols <= 384 ? launch(block_update_tc_kernel<128>, 128, UbCfg<128>::SMEM)
-                               : launch(block_update_tc_kernel<256>, 256, UbCfg<256>::SMEM);
+    // 128-wide tiles for near and far updates alike: three 64 KB stages hide
+    // the operand latency better than two of 96 KB (measured faster for the
+    // far updates too, despite reading E twice as often per output column)
+    const int rc = launch(block_update_tc_kernel<128>, 128, UbCfg<128>::SMEM);
     if (rc != GPTQ_OK) return rc;
     count_launches();
     return launch_status();
