@@ -201,6 +201,22 @@ int gptq_debug_gemm_nt(const float* A, int64_t lda, const float* B, int64_t ldb,
                        int64_t ldc, int64_t M, int64_t N, int64_t K, float alpha, float beta,
                        int lower, void* stream);
 
+/*
+ * Test hooks (host only, no GPU needed; no counterpart on the pages).
+ *
+ * gptq_debug_chol_task_order: the tiled factorization's tasks of a d x d
+ * preparation in the order CTAs claim them: out[3t .. 3t+2] = (type, i, j)
+ * for task t, type 0 = diagonal tile j (factor + invert), 1 = tile (i, j) of
+ * L, 2 = tile (i, j) of L^-1.  Needs cap >= 3 (d/128)^2 int32s.  Returns the
+ * task count, or minus a status code.
+ *
+ * gptq_debug_div_rn: out[i] = the quantizer's division-free quotient
+ * x[i] / s[i] (reciprocal plus two FMA corrections) for s[i] > 0 finite,
+ * computed by the function the sweep kernel uses.  Returns a status code.
+ */
+int64_t gptq_debug_chol_task_order(int64_t d, int32_t* out, int64_t cap);
+int gptq_debug_div_rn(const float* x, const float* s, int64_t n, float* out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,6 +23,7 @@ LIB = os.path.join(PKG, "libgptq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-Xcompiler", "-fPIC",
+         "-Xcompiler", "-ffp-contract=off",
          "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]
 

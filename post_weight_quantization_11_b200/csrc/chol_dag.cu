@@ -73,8 +73,9 @@ struct CdProduct {
     const int* f2;
 };
 
-// Task number -> (type, i, j); see the order above.
-__device__ __forceinline__ void cd_decode(int t, int T, int& type, int& i, int& j)
+// Task number -> (type, i, j); see the order above.  Host and device (the
+// library's task-order test hook calls it on the host).
+__host__ __device__ __forceinline__ void cd_decode(int t, int T, int& type, int& i, int& j)
 {
     if (T == 1) { type = kTaskF; i = j = 0; return; }
     if (t < T + 1) {
@@ -503,3 +504,21 @@ int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d,
 }
 
 }  // namespace gptq
+
+// Test hook: the factorization's tasks in claim order (host only).
+extern "C" int64_t gptq_debug_chol_task_order(int64_t d, int32_t* out, int64_t cap)
+{
+    using namespace gptq;
+    if (d < CD_T || d % CD_T || d > kMaxDim) return -GPTQ_ERR_SHAPE;
+    const int T = (int)(d / CD_T);
+    const int64_t total = int64_t(T) * T;
+    if (!out || cap < 3 * total) return -GPTQ_ERR_INVALID_ARG;
+    for (int t = 0; t < (int)total; ++t) {
+        int type, i, j;
+        cd_decode(t, T, type, i, j);
+        out[3 * t] = type;
+        out[3 * t + 1] = i;
+        out[3 * t + 2] = j;
+    }
+    return total;
+}

@@ -50,7 +50,7 @@ __device__ __forceinline__ float quant_code(float x, const GroupQ& g, float maxq
 // be 1.5 ulp off, so the correction is applied twice: the first brings q
 // within one ulp, the second rounds it correctly.  No overflow or underflow
 // can occur: s is a finite fp16 value >= 2^-24.
-__device__ __forceinline__ float div_rn_recip(float x, float s, float r)
+__host__ __device__ __forceinline__ float div_rn_recip(float x, float s, float r)
 {
     float q = x * r;
     q = fmaf(fmaf(-q, s, x), r, q);

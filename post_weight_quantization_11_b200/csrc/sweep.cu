@@ -417,3 +417,16 @@ extern "C" int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d
     count_launches();
     return launch_status();
 }
+
+// Test hook: out[i] = the sweep's division-free quotient of x[i] / s[i] with
+// r = RN(1 / s[i]), computed on the host by the same function the kernels
+// use (FMAs are correctly rounded on both sides).
+extern "C" int gptq_debug_div_rn(const float* x, const float* s, int64_t n, float* out)
+{
+    if (n < 0 || (n > 0 && (!x || !s || !out))) return GPTQ_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < n; ++i) {
+        const float r = 1.0f / s[i];
+        out[i] = gptq::div_rn_recip(x[i], s[i], r);
+    }
+    return GPTQ_OK;
+}

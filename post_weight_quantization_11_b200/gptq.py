@@ -31,7 +31,8 @@ EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_hessian_accumulate",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_pack_int4",
-            "gptq_unpack_int4", "rtn_quantize", "gptq_debug_gemm_nt")
+            "gptq_unpack_int4", "rtn_quantize", "gptq_debug_gemm_nt",
+            "gptq_debug_chol_task_order", "gptq_debug_div_rn")
 
 
 class GptqError(RuntimeError):
@@ -70,6 +71,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_unpack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "rtn_quantize": ([P, I32, I64, I64, I32, I32, P, P, P, P], I32),
         "gptq_debug_gemm_nt": ([P, I64, P, I64, P, I64, I64, I64, I64, F32, F32, I32, P], I32),
+        "gptq_debug_chol_task_order": ([I64, P, I64], I64),
+        "gptq_debug_div_rn": ([P, P, I64, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -299,3 +302,27 @@ def quantize_layer_from_inputs(W: torch.Tensor, X_batches, bits: int = 4, group_
     if pack and bits == 4:
         res.qweight, res.qzeros = gptq_pack_int4(codes, zeros)
     return res
+
+
+def gptq_debug_chol_task_order(d: int):
+    """The factorization's tasks in claim order as an int32 array of shape
+    (T*T, 3): (type, i, j), type 0 = diagonal tile, 1 = tile of L, 2 = tile
+    of L^-1 (host only)."""
+    import numpy as np
+    T = d // 128
+    out = np.zeros((max(T * T, 1), 3), dtype=np.int32)
+    n = load_library().gptq_debug_chol_task_order(d, out.ctypes.data, out.size)
+    if n < 0:
+        raise GptqError("gptq_debug_chol_task_order", int(-n))
+    return out[:n]
+
+
+def gptq_debug_div_rn(x, s):
+    """The quantizer's division-free quotient x / s (host only; float32 arrays)."""
+    import numpy as np
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    out = np.empty_like(x)
+    _check("gptq_debug_div_rn",
+           load_library().gptq_debug_div_rn(x.ctypes.data, s.ctypes.data, x.size, out.ctypes.data))
+    return out

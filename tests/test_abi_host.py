@@ -15,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _declared():
     txt = open(os.path.join(ROOT, "include", "gptq.h")).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|uint64_t|char\s*\*|void)\s*\**\s*(\w+)\s*\(", txt,
+    names = re.findall(r"^\s*(?:const\s+)?(?:int64_t|int|size_t|uint64_t|char\s*\*|void)\s*\**\s*(\w+)\s*\(", txt,
                        flags=re.M)
     return sorted(set(names))
 
