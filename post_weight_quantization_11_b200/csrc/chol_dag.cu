@@ -30,9 +30,11 @@
 //   phase T-1: I(T-1,T-2) .. I(T-1,0)
 //
 // CTA roles (320 threads): warp 0 TMA producer (also waits for the
-// dependencies), warp 1 MMA issuer, warps 2-5 split the landed fp32 tiles
-// into TF32 head / remainder, warps 6-9 fold TMEM into registers and write
-// the task's results.  The leaf runs on all 320 threads.
+// dependencies), warp 1 MMA issuer, warps 2-9 split each landed fp32 chunk
+// into TF32 head / remainder and fold the previous product's TMEM
+// accumulator into registers (row m, 64 columns per thread), then write the
+// task's results through shared memory.  The leaf runs on all 320 threads
+// (warp 0 as its panel warp, warps 1-9 as its update warps).
 #include "chol_dag.cuh"
 #include "leaf.cuh"
 #include "tc_common.cuh"
