@@ -24,6 +24,9 @@ def _free_port() -> int:
 
 
 def _worker(rank: int, ws: int, port: int, out):
+    # CPU ranks even on a machine with a GPU: the plumbing picks gloo when no
+    # device is visible (NCCL would need one GPU per rank)
+    os.environ["CUDA_VISIBLE_DEVICES"] = ""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       LOCAL_RANK=str(rank), WORLD_SIZE=str(ws))
     import bench
