@@ -227,13 +227,17 @@ class Layer:
 
     def step(self, ev=None):
         """ev: None or 5 CUDA events recorded at the phase boundaries."""
-        G = self.G
         self.S.zero_()
         if ev is not None:
             ev[0].record()
-        G.gptq_hessian_accumulate(self.S, self.X)
+        self.G.gptq_hessian_accumulate(self.S, self.X)
         if ev is not None:
             ev[1].record()
+        self.after_hessian(ev)
+
+    def after_hessian(self, ev=None):
+        """Prepare, quantize and pack once S holds the layer's sum."""
+        G = self.G
         G.gptq_prepare_hinv(self.S, self.n, 0.01, self.act_order, self.perm, self.U, self.info,
                             self.ws_p)
         if ev is not None:
@@ -353,20 +357,27 @@ def run_ours(a):
     torch.cuda.synchronize()
     k1_ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in k1)
 
-    # end to end through the public API from pinned host memory
+    # end to end through the public API from pinned host memory: X streams
+    # through the library's two-slot ring (each chunk's PCIe copy overlaps the
+    # accumulation of the one before, and the next layer's copies overlap this
+    # layer's prepare / quantize / pack); W goes in and the packed result
+    # comes back with plain copies on the compute stream
     Xh = lay.X.cpu().pin_memory()
     Wh = lay.W.cpu().pin_memory()
     qwh = torch.empty_like(lay.qweight, device="cpu").pin_memory()
     qzh = torch.empty_like(lay.qzeros, device="cpu").pin_memory()
     sch = torch.empty_like(lay.scales, device="cpu").pin_memory()
+    hh = G.HostHessian(d, dev)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(ws)
     torch.cuda.synchronize()
     e_start.record()
+    hh.copy_stream.wait_stream(torch.cuda.current_stream())   # no copy starts before e_start
     for _ in range(a.e2e_steps):
-        lay.X.copy_(Xh, non_blocking=True)
+        lay.S.zero_()
+        hh.accumulate(lay.S, Xh)
         lay.W.copy_(Wh, non_blocking=True)
-        lay.step()
+        lay.after_hessian()
         qwh.copy_(lay.qweight, non_blocking=True)
         qzh.copy_(lay.qzeros, non_blocking=True)
         sch.copy_(lay.scales, non_blocking=True)

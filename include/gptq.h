@@ -84,6 +84,45 @@ int gptq_hessian_accumulate(float* S, const uint16_t* X, int64_t n_tokens, int64
                             int64_t* n_seen, void* stream);
 
 /*
+ * Hessian accumulation from HOST memory -- the same sum as
+ * gptq_hessian_accumulate ("GPTQ / AWQ / SqueezeLLM" sec. 一), for
+ * calibration inputs that live in host memory.  The pages have no
+ * counterpart: streaming the batch is an interface convenience.
+ *
+ * X_host is cut into chunks of chunk_tokens tokens.  Chunk k is copied into
+ * slot k % 2 of the device ring `stage` on copy_stream while chunk k - 1 is
+ * accumulated into S on `stream`, so the PCIe copy overlaps the tensor-core
+ * work.  Two caller-owned CUDA events order the ring:
+ *   ev_filled: recorded on copy_stream after each chunk's copy; `stream`
+ *              waits on it before accumulating that chunk;
+ *   ev_freed:  recorded on `stream` after each chunk's accumulation;
+ *              copy_stream waits on it before overwriting a slot.
+ * Reuse the same (stage, ev_filled, ev_freed) for consecutive calls: the
+ * first copy of a call waits for the last accumulation of the previous one,
+ * so the next batch's copies overlap whatever the caller queues on `stream`
+ * in between (e.g. the rest of a layer's quantization).
+ *
+ * S: d x d fp32 device, in/out (upper triangle, as gptq_hessian_accumulate).
+ * X_host: n_tokens x d fp16 host memory, token-major.  Page-locked memory is
+ *    needed for the copies to run asynchronously (pageable memory works but
+ *    each copy then blocks the calling thread).  It is read after the call
+ *    returns: keep it alive and unchanged until `stream` has passed the call.
+ * stage: device buffer of at least 2 * chunk_tokens * d fp16 (stage_bytes).
+ * chunk_tokens: tokens per chunk, 1 <= chunk_tokens <= 2^31.
+ * stream, copy_stream: cudaStream_t; create copy_stream non-blocking for the
+ *    copies to overlap (the same stream twice is allowed: no overlap).
+ * ev_filled, ev_freed: cudaEvent_t, created by the caller (timing disabled
+ *    is enough), on the device of S.
+ * n_seen: optional HOST counter, incremented by n_tokens on success.
+ * Requires the conditions of gptq_hessian_accumulate.  On GPTQ_ERR_CUDA
+ * part of the work may have been queued; S is then undefined.
+ */
+int gptq_hessian_accumulate_host(float* S, const uint16_t* X_host, int64_t n_tokens, int64_t d,
+                                 int64_t* n_seen, uint16_t* stage, size_t stage_bytes,
+                                 int64_t chunk_tokens, void* stream, void* copy_stream,
+                                 void* ev_filled, void* ev_freed);
+
+/*
  * Prepare the inverse-Hessian factor -- "GPTQ / AWQ / SqueezeLLM" sec. 一
  * (H = 2 X^T X / n, damping, decomposition of H^-1, importance order) and
  * "INT4/INT8 量化推理" sec. 三 (rows of H^-1 carry the error feedback).

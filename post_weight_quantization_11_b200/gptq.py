@@ -28,7 +28,7 @@ _STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_SHAPE", 3: "GPT
 # every symbol include/gptq.h declares
 EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_device_status",
-            "gptq_hessian_accumulate",
+            "gptq_hessian_accumulate", "gptq_hessian_accumulate_host",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_pack_int4",
             "gptq_unpack_int4", "rtn_quantize", "gptq_debug_gemm_nt",
@@ -61,6 +61,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_debug_launch_count": ([], ctypes.c_uint64),
         "gptq_device_status": ([P, I32], I32),
         "gptq_hessian_accumulate": ([P, P, I64, I64, P, P], I32),
+        "gptq_hessian_accumulate_host": ([P, P, I64, I64, P, P, SZ, I64, P, P, P, P], I32),
         "gptq_prepare_workspace_bytes": ([I64], SZ),
         "gptq_prepare_hinv": ([P, I64, I64, F32, I32, P, P, P, P, SZ, P], I32),
         "gptq_prepare_hinv_static": ([P, I64, I64, F32, I32, P, P, P, P], I32),
@@ -145,6 +146,56 @@ def gptq_hessian_accumulate(S: torch.Tensor, X: torch.Tensor) -> int:
     _check("gptq_hessian_accumulate",
            load_library().gptq_hessian_accumulate(_ptr(S), _ptr(X), n, d, None, _stream(S)))
     return n
+
+
+class HostHessian:
+    """Accumulates S += X^T X for calibration batches held in HOST memory.
+
+    Owns what gptq_hessian_accumulate_host needs across calls: a two-slot
+    device ring of chunk_tokens x d fp16, a non-blocking copy stream and the
+    two ordering events.  Each batch's PCIe copy overlaps the accumulation of
+    the previous chunk, and the copies of the next batch overlap whatever the
+    caller queues after accumulate() on the current stream.  The default
+    chunk is about 64 MiB of fp16 tokens.
+    """
+
+    def __init__(self, d: int, device=None, chunk_tokens: int | None = None):
+        dev = torch.device("cuda" if device is None else device)
+        if dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.d = int(d)
+        self.chunk = int(chunk_tokens) if chunk_tokens else max(64, (1 << 25) // self.d // 64 * 64)
+        self.device = dev
+        self.stage = torch.empty(2 * self.chunk * self.d, dtype=torch.float16, device=dev)
+        self.copy_stream = torch.cuda.Stream(device=dev)
+        self.ev_filled = torch.cuda.Event()
+        self.ev_freed = torch.cuda.Event()
+        # torch creates an event's CUDA handle at its first record
+        self.ev_filled.record(self.copy_stream)
+        self.ev_freed.record(self.copy_stream)
+
+    def accumulate(self, S: torch.Tensor, X_host: torch.Tensor) -> int:
+        """S (d x d fp32 on the device, upper triangle) += X^T X for X_host
+        (n x d fp16, CPU, contiguous; pinned for the copies to overlap).
+        Asynchronous on the current stream; keep X_host alive and unchanged
+        until that stream has passed this call.  Returns n."""
+        _need(S, "S", torch.float32)
+        if not isinstance(X_host, torch.Tensor) or X_host.is_cuda:
+            raise ValueError("X_host must be a CPU tensor")
+        if X_host.dtype != torch.float16 or not X_host.is_contiguous() or X_host.dim() != 2:
+            raise ValueError("X_host must be a contiguous n x d float16 tensor")
+        n, d = X_host.shape
+        if d != self.d or S.shape != (d, d) or S.device != self.device:
+            raise ValueError("S must be d x d on the streamer's device, X_host n x d")
+        st = torch.cuda.current_stream(self.device)
+        _check("gptq_hessian_accumulate_host",
+               load_library().gptq_hessian_accumulate_host(
+                   _ptr(S), ctypes.c_void_p(X_host.data_ptr()), n, d, None, _ptr(self.stage),
+                   self.stage.numel() * 2, self.chunk, ctypes.c_void_p(st.cuda_stream),
+                   ctypes.c_void_p(self.copy_stream.cuda_stream),
+                   ctypes.c_void_p(self.ev_filled.cuda_event),
+                   ctypes.c_void_p(self.ev_freed.cuda_event)))
+        return n
 
 
 def gptq_prepare_workspace_bytes(d: int) -> int:

@@ -73,6 +73,18 @@ def test_validation_rejects_before_launch(lib):
     # n_tokens == 0 is a no-op that still counts nothing
     assert lib.gptq_hessian_accumulate(FAKE, FAKE, 0, 256, ctypes.byref(n0), None) == 0
     assert n0.value == 0
+    # host-streamed accumulation: ring size, chunk, events
+    H = lib.gptq_hessian_accumulate_host
+    ring = 2 * 64 * 256 * 2
+    assert H(None, FAKE, 10, 256, None, FAKE, ring, 64, None, FAKE, FAKE, FAKE) == 1
+    assert H(FAKE, FAKE, 10, 256, None, MIS, ring, 64, None, FAKE, FAKE, FAKE) == 1
+    assert H(FAKE, FAKE, 10, 256, None, FAKE, ring, 64, None, FAKE, None, FAKE) == 1
+    assert H(FAKE, None, 10, 256, None, FAKE, ring, 64, None, FAKE, FAKE, FAKE) == 1
+    assert H(FAKE, FAKE, 10, 256, None, FAKE, ring - 2, 64, None, FAKE, FAKE, FAKE) == 1
+    assert H(FAKE, FAKE, 10, 200, None, FAKE, ring, 64, None, FAKE, FAKE, FAKE) == 2
+    assert H(FAKE, FAKE, 10, 256, None, FAKE, ring, 0, None, FAKE, FAKE, FAKE) == 2
+    assert H(FAKE, FAKE, 0, 256, ctypes.byref(n0), FAKE, ring, 64, None, FAKE, FAKE, FAKE) == 0
+    assert n0.value == 0
     ws = G.gptq_prepare_workspace_bytes(256)
     assert lib.gptq_prepare_hinv(FAKE, 256, 0, 0.01, 0, None, FAKE, FAKE, FAKE, ws, None) == 2
     assert lib.gptq_prepare_hinv(FAKE, 256, 10, 0.01, 1, None, FAKE, FAKE, FAKE, ws, None) == 1

@@ -124,6 +124,25 @@ def test_hessian_parity(n, d):
     assert np.all(np.tril(Sg, -1) == 0)   # lower triangle untouched
 
 
+@pytest.mark.parametrize("n,d,chunk,pinned", [(5000, 256, 1024, True), (777, 384, 4096, True),
+                                              (3000, 128, 700, False)])
+def test_hessian_from_host_memory(n, d, chunk, pinned):
+    """The host-streamed accumulation: ragged last chunks, a batch smaller
+    than one chunk, pageable memory, and a second batch through the same
+    ring (its first copies wait for the first batch's last accumulation)."""
+    X = _gauss_x(n, d, 3, 50.0, d + n + 1).contiguous()
+    Xh = X.pin_memory() if pinned else X
+    S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    hh = G.HostHessian(d, DEV, chunk_tokens=chunk)
+    assert hh.accumulate(S, Xh) == n
+    assert hh.accumulate(S, Xh[: n // 2]) == n // 2
+    torch.cuda.synchronize()
+    Sg = P.to_np(S)
+    ref = oracle.hessian(np.concatenate([X.numpy(), X.numpy()[: n // 2]]))
+    assert P.rel_fro(np.triu(Sg.astype(np.float64)), np.triu(ref)) <= P.S_TOL
+    assert np.all(np.tril(Sg, -1) == 0)
+
+
 @pytest.mark.parametrize("act_order,d", [(False, 512), (True, 512), (False, 640), (True, 1152)])
 def test_prepare_parity(act_order, d):
     n = 2048
