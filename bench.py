@@ -46,7 +46,7 @@ def _args():
     p.add_argument("--workload", default="attn7b")
     p.add_argument("--layer", type=int, default=0)
     p.add_argument("--tokens", type=int, default=0, help="override token count (0: workload's)")
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--eager", action="store_true",
                    help="launch every kernel from Python each step instead of replaying a "
