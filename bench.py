@@ -48,6 +48,10 @@ def _args():
     p.add_argument("--tokens", type=int, default=0, help="override token count (0: workload's)")
     p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shard", choices=["layers", "layer"], default="layers",
+                   help="layers: every rank quantizes its own layer (weak scaling); layer: one "
+                        "layer over all ranks, tokens and rows split, S summed by one "
+                        "all-reduce (strong scaling)")
     p.add_argument("--eager", action="store_true",
                    help="launch every kernel from Python each step instead of replaying a "
                         "CUDA graph of the step")
@@ -476,10 +480,128 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+def run_ours_one_layer(a):
+    """--shard layer: one layer per step over all ranks.  Rank r accumulates
+    S over its share of the tokens, S is summed by one all-reduce, every rank
+    prepares U from it and quantizes and packs its share of the rows."""
+    ws, rank, local = _dist_init()
+    from post_weight_quantization_11_b200 import gptq as G
+    from post_weight_quantization_11_b200 import inputs, sharded
+    G.load_library()
+    dev = torch.device("cuda", local)
+    wl, spec, n = _workload(a.workload, a.layer, a.tokens)
+    m, d = spec.d_out, spec.d_in
+    t0, t1 = sharded.share(n, ws, rank)
+    L = sharded.ShardedLayer(m, d, t1 - t0, dev, act_order=spec.act_order)
+    lo, hi = L.rows
+    W = inputs.weights(spec, device=dev)[lo:hi].contiguous()
+    X = inputs.calibration_x(spec, n_tokens=t1 - t0, device=dev, first_token=t0)
+    for _ in range(max(3, a.warmup)):
+        L.step(W, X)
+    torch.cuda.synchronize()
+    assert int(L.info.item()) == 0, "non-positive pivot in the workload"
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    start, end = ev(), ev()
+    launches0 = G.gptq_debug_launch_count()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for _ in range(a.steps):
+            L.step(W, X)
+        end.record()
+        torch.cuda.synchronize()
+    _barrier(ws)
+    launches = G.gptq_debug_launch_count() - launches0
+    ms = _max_over_ranks(start.elapsed_time(end) / a.steps, ws)
+    assert int(L.info.item()) == 0 and G.gptq_device_status(reset=True) == 0
+
+    # per-phase split (this rank): local Hessian, the all-reduce, the rest
+    evs = [[ev() for _ in range(4)] for _ in range(3)]
+    for e in evs:
+        L.S.zero_()
+        e[0].record()
+        G.gptq_hessian_accumulate(L.S, X)
+        e[1].record()
+        if ws > 1:
+            import torch.distributed as dist
+            dist.all_reduce(L.S)
+        e[2].record()
+        L.quantize(W)
+        e[3].record()
+    torch.cuda.synchronize()
+    phase = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in evs)
+             for k, name in enumerate(("hessian_local", "all_reduce_S", "prepare_quantize_pack"))}
+    k1_ms = phase["hessian_local"]
+
+    # end to end: this rank's tokens and rows from pinned host memory
+    Xh = X.cpu().pin_memory()
+    Wh = W.cpu().pin_memory()
+    outs = [L.qweight, L.qzeros, L.scales]
+    host_outs = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+    hh = G.HostHessian(d, dev)
+    e_start, e_end = ev(), ev()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    e_start.record()
+    hh.copy_stream.wait_stream(torch.cuda.current_stream())
+    for _ in range(a.e2e_steps):
+        L.hessian_from_host(hh, Xh)
+        W.copy_(Wh, non_blocking=True)
+        L.quantize(W)
+        for h_, t_ in zip(host_outs, outs):
+            h_.copy_(t_, non_blocking=True)
+    e_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e_start.elapsed_time(e_end) / a.e2e_steps, ws)
+
+    peaks, src = _peaks()
+    achieved = float(t1 - t0) * d * d / (k1_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    line = {
+        "metric": METRIC, "value": m * d / (ms * 1e-3), "unit": UNIT, "n_gpus": ws,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; random-init weights, Gaussian calibration inputs with "
+                "outlier channels)",
+        "config": {"workload": f"{spec.name} ({a.workload}): W {m}x{d} fp16, X {n}x{d} fp16, "
+                               f"INT4 g128, damp 0.01, act_order={spec.act_order}",
+                   "parallelism": f"one layer over {ws} rank(s): tokens and rows split, S "
+                                  f"summed by one all-reduce, U prepared on every rank",
+                   "tokens_per_rank": t1 - t0, "rows_per_rank": hi - lo,
+                   "l2": "inputs larger than L2" if (t1 - t0) * d * 2 > 126e6
+                         else "X share smaller than L2"},
+        "e2e": {"value": m * d / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": Xh.numel() * 2 + Wh.numel() * Wh.element_size(),
+                "d2h_bytes_per_step": sum(h_.numel() * h_.element_size() for h_ in host_outs)},
+        "gpu_launches": int(launches),
+        "roofline": {"bound": "tensor", "kernel": "hessian_accumulate (this rank's tokens)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"bf16_tflops_sustained of {src} (fp16 = bf16 rate)",
+                     "kernel_ms": k1_ms},
+        "clocks": clk.summary(),
+        "phase_ms": phase,
+        "launch_mode": "eager",
+    }
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = _cpu_baseline(spec, n)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     a = _args()
     if a.impl == "reference":
         run_reference(a)
+    elif a.shard == "layer":
+        run_ours_one_layer(a)
     else:
         run_ours(a)
 

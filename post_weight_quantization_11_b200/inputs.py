@@ -107,20 +107,22 @@ def outlier_channels(spec: LayerSpec):
 
 
 def calibration_x(spec: LayerSpec, n_tokens: int | None = None, device="cpu",
-                  chunk: int = 16384) -> torch.Tensor:
+                  chunk: int = 16384, first_token: int = 0) -> torch.Tensor:
     """X (n x d_in) fp16, token-major. Gaussian N(0,1) or silu(a)*b with a, b
     N(0,1); then the outlier channels are multiplied by their factor (the same
     factor for every token).  Drawn chunk by chunk so that any prefix of the
-    tokens is the same whatever n is asked for."""
+    tokens is the same whatever n is asked for; first_token > 0 gives rows
+    [first_token, first_token + n) of that same sequence (one rank's share)."""
     n = spec.n_tokens if n_tokens is None else int(n_tokens)
     d = spec.d_in
     ch, fac = outlier_channels(spec)
     ch_t = torch.as_tensor(ch, device=device)
     fac_t = torch.as_tensor(fac, device=device)
     out = torch.empty(n, d, dtype=torch.float16, device=device)
-    for c0 in range(0, n, chunk):
-        c1 = min(n, c0 + chunk)
-        g = _gen(1_000_003 * spec.seed + 101 + c0 // chunk, device)
+    t_end = first_token + n
+    for k in range(first_token // chunk, (t_end + chunk - 1) // chunk):
+        a0, a1 = max(first_token, k * chunk), min(t_end, (k + 1) * chunk)   # absolute rows
+        g = _gen(1_000_003 * spec.seed + 101 + k, device)
         if spec.x_kind == "gauss":
             x = torch.randn(chunk, d, generator=g, device=device, dtype=torch.float32)
         elif spec.x_kind == "silu":
@@ -132,7 +134,7 @@ def calibration_x(spec: LayerSpec, n_tokens: int | None = None, device="cpu",
             raise ValueError(spec.x_kind)
         if len(ch):
             x[:, ch_t] *= fac_t
-        out[c0:c1] = x[: c1 - c0].to(torch.float16)
+        out[a0 - first_token:a1 - first_token] = x[a0 - k * chunk:a1 - k * chunk].to(torch.float16)
         del x
     return out
 
