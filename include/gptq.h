@@ -256,6 +256,22 @@ int gptq_debug_gemm_nt(const float* A, int64_t lda, const float* B, int64_t ldb,
 int64_t gptq_debug_chol_task_order(int64_t d, int32_t* out, int64_t cap);
 int gptq_debug_div_rn(const float* x, const float* s, int64_t n, float* out);
 
+/*
+ * Test hook (no counterpart on the pages): failure detection without a GPU
+ * fault.  Runs one of the library's bounded waits against a condition that
+ * never comes true, with a wait limit of limit_ns nanoseconds instead of
+ * the kernels' 4 s:
+ *   which = 0: the completion-flag wait tasks use for their dependencies,
+ *              on the device int32 *flag (returns at once when it is
+ *              non-zero; otherwise gives up and records 0x105);
+ *   which = 1: the mbarrier wait of the TMA pipelines, on a fresh barrier
+ *              nobody arrives on (gives up and records 0x101; flag unused).
+ * The recorded code is read (and cleared) with gptq_device_status; the
+ * kernel returns normally either way.  Asynchronous on `stream`.
+ * Requires 1e6 <= limit_ns <= 1e9; flag 4-byte aligned when which = 0.
+ */
+int gptq_debug_bounded_wait(const int32_t* flag, int which, int64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

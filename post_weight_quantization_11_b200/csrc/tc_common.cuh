@@ -93,7 +93,8 @@ __device__ __forceinline__ unsigned long long globaltimer_ns()
 // Bounded wait for the phase with the given parity to complete.  `abort` is
 // a CTA-shared flag: set by whichever role of the CTA gave up first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int err,
-                                          volatile int* abort)
+                                          volatile int* abort,
+                                          unsigned long long limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
@@ -101,7 +102,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int er
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 atomicCAS(&g_device_status, 0, err);
                 *abort = 1;
                 return false;
@@ -143,7 +144,8 @@ __device__ __forceinline__ void fence_proxy_async_global()
 }
 
 // Bounded wait for a completion flag (acquire).
-__device__ __forceinline__ bool cd_wait_flag(const int* f, volatile int* abort, const int* gabort)
+__device__ __forceinline__ bool cd_wait_flag(const int* f, volatile int* abort, const int* gabort,
+                                             unsigned long long limit_ns = kWaitLimitNs)
 {
     if (ld_acquire_gpu(f)) return true;
     const unsigned long long t0 = globaltimer_ns();
@@ -155,7 +157,7 @@ __device__ __forceinline__ bool cd_wait_flag(const int* f, volatile int* abort, 
                 *abort = 1;
                 return false;
             }
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 atomicCAS(&g_device_status, 0, kErrWaitDep);
                 *abort = 1;
                 return false;

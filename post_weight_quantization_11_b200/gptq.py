@@ -32,7 +32,7 @@ EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_pack_int4",
             "gptq_unpack_int4", "rtn_quantize", "gptq_debug_gemm_nt",
-            "gptq_debug_chol_task_order", "gptq_debug_div_rn")
+            "gptq_debug_chol_task_order", "gptq_debug_div_rn", "gptq_debug_bounded_wait")
 
 
 class GptqError(RuntimeError):
@@ -74,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_debug_gemm_nt": ([P, I64, P, I64, P, I64, I64, I64, I64, F32, F32, I32, P], I32),
         "gptq_debug_chol_task_order": ([I64, P, I64], I64),
         "gptq_debug_div_rn": ([P, P, I64, P], I32),
+        "gptq_debug_bounded_wait": ([P, I32, I64, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -379,3 +380,15 @@ def gptq_debug_div_rn(x, s):
     _check("gptq_debug_div_rn",
            load_library().gptq_debug_div_rn(x.ctypes.data, s.ctypes.data, x.size, out.ctypes.data))
     return out
+
+
+def gptq_debug_bounded_wait(flag: torch.Tensor | None, which: int, limit_ns: int) -> None:
+    """Run a bounded wait that never succeeds (unless which == 0 and flag is
+    non-zero) with the given limit; the outcome is read with
+    gptq_device_status().  Asynchronous on the current stream."""
+    if flag is not None:
+        _need(flag, "flag", torch.int32)
+    st = torch.cuda.current_stream() if flag is None else torch.cuda.current_stream(flag.device)
+    _check("gptq_debug_bounded_wait",
+           load_library().gptq_debug_bounded_wait(_ptr(flag), int(which), int(limit_ns),
+                                                  ctypes.c_void_p(st.cuda_stream)))

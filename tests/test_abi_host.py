@@ -85,6 +85,11 @@ def test_validation_rejects_before_launch(lib):
     assert H(FAKE, FAKE, 10, 256, None, FAKE, ring, 0, None, FAKE, FAKE, FAKE) == 2
     assert H(FAKE, FAKE, 0, 256, ctypes.byref(n0), FAKE, ring, 64, None, FAKE, FAKE, FAKE) == 0
     assert n0.value == 0
+    # failure-detection probe: argument checks
+    assert lib.gptq_debug_bounded_wait(FAKE, 2, 50_000_000, None) == 1
+    assert lib.gptq_debug_bounded_wait(None, 0, 50_000_000, None) == 1
+    assert lib.gptq_debug_bounded_wait(FAKE, 0, 10, None) == 1
+    assert lib.gptq_debug_bounded_wait(FAKE, 1, 2_000_000_000, None) == 1
     ws = G.gptq_prepare_workspace_bytes(256)
     assert lib.gptq_prepare_hinv(FAKE, 256, 0, 0.01, 0, None, FAKE, FAKE, FAKE, ws, None) == 2
     assert lib.gptq_prepare_hinv(FAKE, 256, 10, 0.01, 1, None, FAKE, FAKE, FAKE, ws, None) == 1
