@@ -228,9 +228,12 @@ int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bi
                  void* stream);
 
 /*
- * Test hook (no counterpart on the pages): the split-TF32 tensor-core GEMM the
- * library uses for the Cholesky / triangular-inverse updates, exposed so it
- * can be checked on its own.
+ * Test hook (no counterpart on the pages): a stand-alone split-TF32
+ * tensor-core GEMM.  It takes every product the way the factorization and
+ * the block update do (x = x_hi + x_lo, x_hi rounded to TF32; three
+ * kind::tf32 MMAs A_hi B_hi + A_hi B_lo + A_lo B_hi accumulated in TMEM), so
+ * a test can check on its own that this arithmetic keeps fp32-level accuracy
+ * on the hardware.  The library's kernels do not call it.
  *   C = beta * C + alpha * A * B^T
  * A: M x K (lda), B: N x K (ldb), C: M x N (ldc), dense row-major fp32 device
  * arrays; K % 32 == 0; leading dimensions multiples of 4.  lower != 0

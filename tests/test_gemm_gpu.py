@@ -1,6 +1,6 @@
-"""The split-TF32 tensor-core GEMM (C = beta C + alpha A B^T) used by the
-Cholesky / triangular-inverse updates, checked directly against a float64
-product.  Split-TF32 (Ootomo & Yokota 2022) keeps about fp32 accuracy: the
+"""The stand-alone split-TF32 tensor-core GEMM (C = beta C + alpha A B^T),
+which takes its products the way the factorization and the block update do,
+checked directly against a float64 product.  Split-TF32 (Ootomo & Yokota 2022) keeps about fp32 accuracy: the
 test bound is 2e-6 * max(1, sqrt(K / 512)) of |alpha| |A| |B|^T + |beta C| per
 element (accumulation error grows like sqrt(K); a lost hi/lo term would show
 as ~5e-4)."""
