@@ -143,6 +143,26 @@ def test_hessian_from_host_memory(n, d, chunk, pinned):
     assert np.all(np.tril(Sg, -1) == 0)
 
 
+def test_sharded_layer_on_one_process_matches_the_direct_path():
+    """The one-layer-over-ranks driver without a process group: the same
+    library calls as quantize_layer_from_inputs, on real kernels."""
+    from post_weight_quantization_11_b200 import sharded
+    W = _weights(300, 512, torch.float16, 21)
+    X = _gauss_x(3000, 512, 3, 50.0, 22)
+    Wd, Xd = W.to(DEV), X.to(DEV)
+    L = sharded.ShardedLayer(300, 512, 3000, DEV)
+    assert L.rows == (0, 300) and L.n_total == 3000
+    L.step(Wd, Xd)
+    ref = G.quantize_layer_from_inputs(Wd, Xd)
+    torch.cuda.synchronize()
+    assert int(L.info.item()) == 0
+    S1, S2 = P.to_np(L.S).astype(np.float64), P.to_np(ref.S).astype(np.float64)
+    assert P.rel_fro(np.triu(S1), np.triu(S2)) <= 1e-6
+    assert float((P.to_np(L.codes) != P.to_np(ref.codes)).mean()) <= 1e-3
+    qw, qz = G.gptq_pack_int4(L.codes, L.zeros)
+    assert torch.equal(qw, L.qweight) and torch.equal(qz, L.qzeros)
+
+
 @pytest.mark.parametrize("act_order,d", [(False, 512), (True, 512), (False, 640), (True, 1152)])
 def test_prepare_parity(act_order, d):
     n = 2048
