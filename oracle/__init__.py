@@ -19,6 +19,8 @@ float64, no blocking) and cites the passage it follows:
 * ``pack_int4``/``unpack_int4`` -- the 66.5 B / 128-weight storage format
                       ("INT4/INT8 量化推理" sec. 一).
 * ``trace_quadratic`` -- tr(D H D^T), the layer loss of sec. 三 of that page.
+* ``w4a16_matmul`` -- y = x Q^T from the packed layer (weight-only INT4 with
+                      fp16 activations, "INT4/INT8 量化推理" sec. 六).
 """
 from __future__ import annotations
 
@@ -262,6 +264,26 @@ def dequantize(codes: np.ndarray, scales16: np.ndarray, zeros: np.ndarray,
     Q = np.empty_like(Qs)
     Q[:, np.asarray(perm, dtype=np.int64)] = Qs
     return Q
+
+
+def w4a16_matmul(x, qweight: np.ndarray, qzeros: np.ndarray, scales16: np.ndarray, d: int,
+                 group_size: int, perm: np.ndarray | None = None) -> np.ndarray:
+    """y = x Q^T straight from the packed INT4 layer, in float64: the
+    weight-only-quantized product (W4A16) of "INT4/INT8 量化推理" sec. 六,
+    on the storage of sec. 一 of the same page.
+
+    x: b x d fp16 activations (original column order); qweight / qzeros /
+    scales16 as gptq_pack_int4 and the sweep write them (codes in sweep
+    order); Q[:, perm[k]] = s (c_k - z) as in ``dequantize``.
+    """
+    xb = np.asarray(x)
+    if xb.dtype == np.uint16:
+        xb = xb.view(np.float16)
+    xb = xb.astype(np.float64)
+    G = n_groups(d, group_size)
+    codes, zeros = unpack_int4(qweight, qzeros, d, G)
+    Q = dequantize(codes, scales16, zeros, group_size, perm)
+    return xb @ Q.T
 
 
 def trace_quadratic(D: np.ndarray, H: np.ndarray) -> float:

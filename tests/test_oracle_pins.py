@@ -124,6 +124,40 @@ def test_pack_hand_examples_and_roundtrip():
         assert np.array_equal(c2, codes) and np.array_equal(z2, zeros)
 
 
+def test_w4a16_hand_example_and_one_hot_columns():
+    rows = {}
+    cases = []
+    for row in _read_golden("w4a16_example.txt"):
+        f = [p.strip() for p in row.split("|")]
+        if f[0] == "case":
+            cases.append(f[1:])
+        else:
+            rows[f[0]] = [[int(v, 16) for v in part.split(",")] for part in f[1].split(";")]
+    qw = np.array(rows["qweight"], np.uint32)
+    qz = np.array(rows["qzeros"], np.uint8)
+    sc = np.array(rows["scales"], np.uint16)
+    xs = {"ones": np.ones(16), "ramp": np.arange(16.0)}
+    for xname, pname, want in cases:
+        perm = {"none": None, "reversed": np.arange(15, -1, -1, dtype=np.int32),
+                "cyclic": ((np.arange(16) + 1) % 16).astype(np.int32)}[pname]
+        x = xs[xname].astype(np.float16)[None, :]
+        y = oracle.w4a16_matmul(x, qw, qz, sc, 16, 8, perm)
+        assert y[0].tolist() == [float(v) for v in want.split(",")]
+    # one-hot activations pick out columns of the dequantized layer
+    rng = _rng(17)
+    m, d, g = 5, 256, 64
+    codes = rng.integers(0, 16, (m, d), dtype=np.uint8)
+    zeros = rng.integers(0, 16, (m, d // g), dtype=np.uint8)
+    sc = rng.uniform(1e-3, 1e-1, (m, d // g)).astype(np.float16).view(np.uint16)
+    perm = rng.permutation(d).astype(np.int32)
+    qw, qz = oracle.pack_int4(codes, zeros)
+    Q = oracle.dequantize(codes, sc, zeros, g, perm)
+    for j in (0, 1, 77, 255):
+        e = np.zeros((1, d), np.float16)
+        e[0, j] = 1
+        assert np.array_equal(oracle.w4a16_matmul(e, qw, qz, sc, d, g, perm)[0], Q[:, j])
+
+
 # --------------------------------------------------------------------------
 # Hessian
 # --------------------------------------------------------------------------
