@@ -217,6 +217,21 @@ def quantize_rows(W: np.ndarray, U: np.ndarray, bits: int = 4, group_size: int =
     return out
 
 
+def quantize_rows_static(W: np.ndarray, U: np.ndarray, bits: int = 4, group_size: int = 128):
+    """The column sweep with STATIC groups: every group's scale and zero point
+    are taken from the rows as they are before the sweep (the original W in
+    sweep order, i.e. the round-to-nearest parameters of ``rtn``) instead of
+    from the corrected values at the group's first column; the codes and the
+    error feedback are those of ``quantize_rows``.  The pages fix the group
+    parameters only by the min-max rule ("校准艺术" sec. 2.1); taking them
+    before any correction is the alternative reading to the default one."""
+    p = rtn(W, bits, group_size)
+    out = quantize_rows(W, U, bits, group_size, forced_scales=p["scales"],
+                        forced_zeros=p["zeros"])
+    out["s_pre"] = p["s_pre"]
+    return out
+
+
 def rtn(W: np.ndarray, bits: int = 4, group_size: int = 128):
     W = np.ascontiguousarray(W, dtype=np.float64)
     m, d = W.shape

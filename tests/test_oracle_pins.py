@@ -294,6 +294,41 @@ def test_gptq_equals_rtn_when_hessian_is_isotropic():
     assert np.array_equal(res["codes"], r["codes"])
 
 
+def test_static_groups_special_cases():
+    """Static groups take every group's parameters from the uncorrected row:
+    with a diagonal U (no feedback) they equal the dynamic ones and RTN; per
+    channel (one group per row, parameterized at column 0 before any
+    correction) the two readings coincide for any U; otherwise the scales are
+    RTN's and the feedback still obeys the loss identity."""
+    rng = _rng(23)
+    m, d = 48, 128
+    W = 0.02 * rng.standard_normal((m, d))
+    Ud = np.diag(rng.uniform(0.2, 2.0, d))
+    st = oracle.quantize_rows_static(W, Ud, 4, 32)
+    dy = oracle.quantize_rows(W, Ud, 4, 32)
+    r = oracle.rtn(W, 4, 32)
+    for k in ("codes", "scales", "zeros"):
+        assert np.array_equal(st[k], dy[k]) and np.array_equal(st[k], r[k])
+    X = rng.standard_normal((400, d)).astype(np.float16)
+    X[:, 5] *= 30
+    S = oracle.hessian(X)
+    _, Hd, _, _, _ = oracle.finalize(S, 400, 0.01, False)
+    U, info = oracle.hinv_upper_chol(Hd)
+    assert info == 0
+    for g in (d, -1):
+        st = oracle.quantize_rows_static(W, U, 4, g)
+        dy = oracle.quantize_rows(W, U, 4, g)
+        for k in ("codes", "scales", "zeros"):
+            assert np.array_equal(st[k], dy[k])
+    st = oracle.quantize_rows_static(W, U, 4, 32)
+    dy = oracle.quantize_rows(W, U, 4, 32)
+    assert np.array_equal(st["scales"], oracle.rtn(W, 4, 32)["scales"])
+    assert not np.array_equal(st["scales"], dy["scales"])
+    Q = oracle.dequantize(st["codes"], st["scales"], st["zeros"], 32)
+    D = W - Q
+    assert abs(st["row_loss"].sum() - oracle.trace_quadratic(D, Hd)) <= 1e-9 * st["row_loss"].sum()
+
+
 def test_loss_closed_form_identity():
     # sum_j (e_j/U_jj)^2 = tr(D Hd D^T) = (2/n)||D X^T||^2 + lam ||D||^2, and
     # D = E U (the accumulated corrections): exact for any quantizer decisions.
