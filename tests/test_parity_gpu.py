@@ -180,6 +180,27 @@ def test_prepare_parity(act_order, d):
     assert P.rel_fro(Ug, U64) <= P.U_TOL
 
 
+def test_prepare_kms_closed_form():
+    """The GPU's U for H = KMS(0.7) (H_ij = 0.7^|i-j|, no damping) against
+    its closed form, an upper bidiagonal matrix (every entry checked, the
+    zeros included): no oracle involved."""
+    d, n, rho = 512, 1000, 0.7
+    i = np.arange(d)
+    H = rho ** np.abs(i[:, None] - i[None, :])
+    S = torch.from_numpy((n / 2.0) * H).float().to(DEV)
+    perm, U, info = G.gptq_prepare_hinv(S, n, 0.0, False)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    c = np.sqrt(1.0 - rho * rho)
+    ref = np.zeros((d, d))
+    ref[i[:-1], i[:-1]] = 1.0 / c
+    ref[d - 1, d - 1] = 1.0
+    ref[i[:-1], i[1:]] = -rho / c
+    Ug = P.to_np(U).astype(np.float64)
+    assert np.abs(Ug - ref).max() <= 1e-5 * np.abs(ref).max()
+    assert np.array_equal(P.to_np(perm), np.arange(d, dtype=np.int32))
+
+
 def test_prepare_reports_non_pd():
     d = 256
     S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
