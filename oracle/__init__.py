@@ -8,11 +8,13 @@ Every function is a thin numpy wrapper over ``gptq_oracle.c`` (plain C,
 float64, no blocking) and cites the passage it follows:
 
 * ``hessian``      -- H accumulation, "GPTQ / AWQ / SqueezeLLM" sec. 一
-                      (H = 2 X^T X / n; here the raw sum S = X^T X).
+                      (H = 2 X^T X / n; here the raw sum S = X^T X);
+                      ``hessian_syrk`` the same sum through BLAS for full-size X.
 * ``finalize``     -- H = 2S/n, relative damping, act-order permutation
                       (same page, sec. 一: damping, importance order).
 * ``cholesky_lower``/``trtri_lower``/``hinv_upper_chol`` -- the "decomposition"
-                      of H^-1 (same page, sec. 一; "INT4/INT8 量化推理" sec. 三).
+                      of H^-1 (same page, sec. 一; "INT4/INT8 量化推理" sec. 三);
+                      ``u_rows`` selected rows of it from their definition.
 * ``quantize_rows`` -- the column sweep with error feedback ("INT4/INT8 量化推理"
                       sec. 三 loop; "校准艺术" sec. 2.2 steps 1-5).
 * ``rtn``          -- round-to-nearest group min-max ("校准艺术" sec. 2.1).
@@ -61,7 +63,7 @@ def _load():
         lib.orc_hinv_upper_chol.argtypes = [P, I64, P]
         lib.orc_hinv_upper_chol.restype = ctypes.c_int
         lib.orc_quantize_rows.argtypes = [P, P, I64, I64, ctypes.c_int, I64,
-                                          P, P, P, P, P, P, P, P, P, P, P]
+                                          P, P, P, P, P, P, P, P, P, P, P, P, P, P]
         lib.orc_quantize_rows.restype = None
         lib.orc_rtn.argtypes = [P, I64, I64, ctypes.c_int, I64, P, P, P, P]
         lib.orc_rtn.restype = None
@@ -128,6 +130,26 @@ def hessian(X, S: np.ndarray | None = None) -> np.ndarray:
     return S
 
 
+
+def hessian_syrk(X, chunk: int = 16384) -> np.ndarray:
+    """S = X^T X for X (n x d) fp16 in float64 through the BLAS rank-k update
+    (dsyrk) over token chunks: the same sum as ``hessian`` (every fp16 value is
+    exact in float64; only the float64 summation order differs), for inputs
+    where the plain loop takes minutes.  X may be a numpy array or a CPU torch
+    tensor of float16.  Returns the full symmetric matrix."""
+    from scipy.linalg import blas
+    if hasattr(X, "numpy"):
+        X = X.numpy()
+    X = np.asarray(X)
+    assert X.dtype == np.float16
+    n, d = X.shape
+    S = np.zeros((d, d), dtype=np.float64, order="F")
+    for t0 in range(0, n, chunk):
+        Xc = np.asfortranarray(X[t0:t0 + chunk].astype(np.float64))
+        S = blas.dsyrk(1.0, Xc, beta=1.0, c=S, trans=1, lower=0, overwrite_c=1)
+    S = np.ascontiguousarray(S)
+    return np.triu(S) + np.triu(S, 1).T
+
 def finalize(S: np.ndarray, n: int, damp_rel: float = 0.01, act_order: bool = False):
     """H = 2S/n; perm (stable descending argsort of diag H when act_order);
     H <- H[perm][:, perm]; lambda = damp_rel * mean(diag H); Hd = H + lambda I.
@@ -178,6 +200,30 @@ def hinv_upper_chol(Hd: np.ndarray):
     return U, int(info)
 
 
+
+def u_rows(Hd: np.ndarray, rows) -> np.ndarray:
+    """Selected rows of U (upper, U^T U = Hd^-1) from their definition: row j
+    of U is the first row of the inverse of the trailing sub-Hessian
+    Hd[j:, j:] (the Hessian of the not-yet-quantized columns once columns
+    0..j-1 are fixed) divided by the square root of its first entry ("GPTQ /
+    AWQ / SqueezeLLM" sec. 一: the decomposition of H^-1 the sweep reads
+    row by row).  Each row is one float64 solve with that sub-matrix (a
+    library Cholesky solve as the step), so a few rows of a d = 14336 factor
+    cost seconds where the whole factor costs minutes.  Returns a
+    len(rows) x d array, zero left of the diagonal."""
+    from scipy.linalg import cho_factor, cho_solve
+    Hd = np.asarray(Hd, dtype=np.float64)
+    d = Hd.shape[0]
+    out = np.zeros((len(rows), d), dtype=np.float64)
+    for i, j in enumerate(rows):
+        j = int(j)
+        e = np.zeros(d - j)
+        e[0] = 1.0
+        x = cho_solve(cho_factor(Hd[j:, j:], lower=False, check_finite=False), e,
+                      check_finite=False)
+        out[i, j:] = x / np.sqrt(x[0])
+    return out
+
 # --------------------------------------------------------------------------
 # Sweep, RTN, packing
 # --------------------------------------------------------------------------
@@ -195,7 +241,10 @@ def quantize_rows(W: np.ndarray, U: np.ndarray, bits: int = 4, group_size: int =
     Returns dict(codes uint8 m x d, scales uint16 (fp16 bits) m x G, zeros uint8
     m x G, row_loss float64 m = sum_j (e_j / U_jj)^2, s_pre float32 m x G) and,
     with ``record``, own_codes / tie_dist (the oracle's own decision and the
-    distance of w/s from the nearest rounding boundary) for teacher forcing.
+    distance of w/s from the nearest rounding boundary) and, per group,
+    own_scales / own_zeros / zero_tie_dist (the oracle's own fp16 scale and
+    zero point on this trajectory, and the distance of -mn/s from the nearest
+    rounding boundary) for teacher forcing.
     """
     W = np.ascontiguousarray(W, dtype=np.float64)
     U = np.ascontiguousarray(U, dtype=np.float64)
@@ -210,11 +259,16 @@ def quantize_rows(W: np.ndarray, U: np.ndarray, bits: int = 4, group_size: int =
     if record or fc is not None:
         out["own_codes"] = np.empty((m, d), np.uint8)
         out["tie_dist"] = np.empty((m, d), np.float32)
+        out["own_scales"] = np.empty((m, G), np.uint16)
+        out["own_zeros"] = np.empty((m, G), np.uint8)
+        out["zero_tie_dist"] = np.empty((m, G), np.float32)
     wq = np.empty((m, d), np.float64) if return_wq else None
     _load().orc_quantize_rows(_p(W), _p(U), m, d, int(bits), int(group_size),
                               _p(out["codes"]), _p(out["scales"]), _p(out["zeros"]),
                               _p(out["row_loss"]), _p(out["s_pre"]), _p(fc), _p(fs), _p(fz),
-                              _p(out.get("own_codes")), _p(out.get("tie_dist")), _p(wq))
+                              _p(out.get("own_codes")), _p(out.get("tie_dist")),
+                              _p(out.get("own_scales")), _p(out.get("own_zeros")),
+                              _p(out.get("zero_tie_dist")), _p(wq))
     if return_wq:
         out["wq"] = wq
     return out

@@ -100,6 +100,7 @@ typedef struct {
     float s;        /* the same scale as fp32 (exact) */
     float s_pre;    /* fp32 scale before fp16 rounding */
     int z;          /* zero point, 0..maxq */
+    float zq;       /* -mn / s in fp32, the value the zero point rounds */
 } orc_gparams;
 
 static orc_gparams orc_group_params(const double* w, int len, int maxq)
@@ -118,7 +119,8 @@ static orc_gparams orc_group_params(const double* w, int len, int maxq)
     if ((h & 0x7fff) >= 0x7c00) h = 0x7bff;       /* largest finite fp16 */
     g.s16 = h;
     g.s = (float)orc_half_to_double(h);
-    float zf = rintf(-mn / g.s);
+    g.zq = -mn / g.s;
+    float zf = rintf(g.zq);
     if (zf < 0.0f) zf = 0.0f;
     if (zf > (float)maxq) zf = (float)maxq;
     g.z = (int)zf;
@@ -301,7 +303,10 @@ int orc_hinv_upper_chol(const double* Hd, int64_t d, double* U)
 /* Teacher forcing (all nullable): when forced_codes[r*d+j] >= 0 the code is */
 /* taken from it; when forced_s16 is given the group parameters are taken    */
 /* from forced_s16/forced_z.  own_codes/tie_dist record the oracle's own     */
-/* decision and the distance of w/s from the nearest rounding boundary.      */
+/* decision and the distance of w/s from the nearest rounding boundary;      */
+/* own_s16/own_z/z_tie (m x G) record the oracle's own group parameters on   */
+/* the (forced) trajectory and the distance of -mn/s from the nearest        */
+/* rounding boundary k + 0.5 (nullable; bookkeeping only).                  */
 /* ------------------------------------------------------------------------ */
 
 void orc_quantize_rows(const double* W, const double* U, int64_t m, int64_t d,
@@ -310,6 +315,7 @@ void orc_quantize_rows(const double* W, const double* U, int64_t m, int64_t d,
                        double* row_loss, float* s_pre,
                        const int16_t* forced_codes, const uint16_t* forced_s16,
                        const uint8_t* forced_z, uint8_t* own_codes, float* tie_dist,
+                       uint16_t* own_s16, uint8_t* own_z, float* z_tie,
                        double* Wq_out)
 {
     int maxq = (1 << bits) - 1;
@@ -319,7 +325,7 @@ void orc_quantize_rows(const double* W, const double* U, int64_t m, int64_t d,
     for (int64_t r = 0; r < m; ++r) {
         double* w = (double*)malloc(sizeof(double) * (size_t)d);
         memcpy(w, W + r * d, sizeof(double) * (size_t)d);
-        orc_gparams gp = {0, 1.0f, 1.0f, 0};
+        orc_gparams gp = {0, 1.0f, 1.0f, 0, 0.0f};
         double loss = 0.0;
         for (int64_t j = 0; j < d; ++j) {
             if (j % g == 0) {
@@ -327,6 +333,9 @@ void orc_quantize_rows(const double* W, const double* U, int64_t m, int64_t d,
                 int64_t gi = j / g;
                 orc_gparams own = orc_group_params(w + j, (int)len, maxq);
                 if (s_pre) s_pre[r * G + gi] = own.s_pre;
+                if (own_s16) own_s16[r * G + gi] = own.s16;
+                if (own_z) own_z[r * G + gi] = (uint8_t)own.z;
+                if (z_tie) z_tie[r * G + gi] = fabsf((own.zq - floorf(own.zq)) - 0.5f);
                 gp = own;
                 if (forced_s16) {
                     gp.s16 = forced_s16[r * G + gi];

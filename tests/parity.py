@@ -10,14 +10,21 @@ Tolerances (written here, used by every parity test):
   * scales: for every group of a row before that row's first code mismatch,
             the GPU's fp16 scale is the fp16 rounding of some value within
             1e-4 relative of the oracle's pre-fp16 scale
-  * zero points: z = rne(-mn/s) is a rounding decision like the codes; under
-            equal scales they are equal except at most 1e-3 of the groups,
-            and those differ by one step
+  * zero points: z = rne(-mn/s) is an integer rounding decision like the
+            codes; under equal scales they are equal except at most 1e-3 of
+            the groups, those differ by one step, and the teacher-forced run
+            shows each such flip to be a near-tie: |frac(-mn/s) - 0.5| <= 1e-3
+            on the oracle's side of the same trajectory
   * loss:   the layer loss tr(D H D^T) of the GPU's dequantized weights,
             evaluated in float64, within 1e-3 relative of the oracle's
   * teacher-forced diagnostic: with the GPU's decisions forced into the
             oracle, every code where the oracle would have decided otherwise
-            is a near-tie: |frac(w/s) - 0.5| <= 1e-3
+            is a near-tie: |frac(w/s) - 0.5| <= 1e-3; every zero point where it
+            would have decided otherwise under the same fp16 scale is a
+            near-tie of -mn/s; and every fp16 scale where it would have
+            decided otherwise rounds a value within 1e-4 of the oracle's
+            pre-fp16 scale (the oracle's value sits that close to an fp16
+            rounding boundary)
 """
 from __future__ import annotations
 
@@ -83,9 +90,12 @@ def compare_sweep(gpu: dict, orc: dict, group_size: int, report: dict | None = N
 
 
 def teacher_forced_check(Wp64: np.ndarray, U64: np.ndarray, gpu: dict, bits: int,
-                         group_size: int, rows=None):
+                         group_size: int, rows=None, report: dict | None = None):
     """Force the GPU's codes/scales/zeros into the oracle sweep; every place
-    where the oracle's own code differs must be a near-tie."""
+    where the oracle's own decision differs must be a near-tie: codes by
+    |frac(w/s) - 0.5|, zero points (under the same fp16 scale) by
+    |frac(-mn/s) - 0.5|, scales by the fp16 rounding of a value within 1e-4
+    of the oracle's pre-fp16 scale."""
     sl = slice(None) if rows is None else rows
     f = oracle.quantize_rows(Wp64[sl], U64, bits, group_size,
                              forced_codes=gpu["codes"][sl].astype(np.int16),
@@ -99,6 +109,17 @@ def teacher_forced_check(Wp64: np.ndarray, U64: np.ndarray, gpu: dict, bits: int
     sg = gpu["scales"][sl].view(np.float16).astype(np.float32)
     lo, hi = fp16_range(f["s_pre"], SCALE_REL)
     assert ((sg >= lo) & (sg <= hi)).all(), "scale outside range on the forced trajectory"
+    s_flip = f["own_scales"] != gpu["scales"][sl]
+    # zero points decided under the same fp16 scale: a flip must sit at a tie of -mn/s
+    z_flip = ~s_flip & (f["own_zeros"] != gpu["zeros"][sl])
+    if z_flip.any():
+        zt = f["zero_tie_dist"][z_flip]
+        assert (zt <= TIE).all(), (f"{int((zt > TIE).sum())} zero points differ off a tie "
+                                   f"(max tie distance {float(zt.max()):.3g})")
+    if report is not None:
+        report.update(forced_code_ties=int(diff.sum()), forced_zero_ties=int(z_flip.sum()),
+                      forced_scale_flips=int(s_flip.sum()),
+                      max_zero_tie_dist=float(f["zero_tie_dist"][z_flip].max()) if z_flip.any() else 0.0)
     return int(diff.sum())
 
 

@@ -194,6 +194,19 @@ def test_hessian_closed_forms():
     assert np.linalg.eigvalsh(S1).min() > -1e-9 * np.abs(S1).max()
 
 
+
+def test_hessian_syrk_closed_forms_and_plain_loop():
+    """The BLAS route of S (full-size checks) against the Hadamard closed form
+    and against the plain column loop on ragged chunking."""
+    Had = _sylvester(5)                      # 32 x 32 entries +-1: X^T X = 32 I
+    assert np.array_equal(oracle.hessian_syrk(Had.astype(np.float16), chunk=7),
+                          32.0 * np.eye(32))
+    X = _spd_from_tokens(1000, 40, 5, outliers=3)
+    S1 = oracle.hessian(X)
+    S2 = oracle.hessian_syrk(X, chunk=333)
+    assert np.array_equal(S2, S2.T)
+    assert np.abs(S1 - S2).max() <= 1e-13 * np.abs(S1).max()
+
 def test_finalize_damping_and_perm():
     X = _spd_from_tokens(64, 9, 4, outliers=2)
     S = oracle.hessian(X)
@@ -312,6 +325,23 @@ def test_upper_chol_of_inverse_kms_closed_form():
             if j + 1 < d:
                 w[j + 1] -= E * U[j, j + 1]
 
+
+
+def test_u_rows_closed_form_and_full_factor():
+    """Rows of U from the trailing sub-Hessians against the KMS closed form
+    (upper bidiagonal) and against the full factor of the plain route."""
+    d, rho = 200, 0.6
+    i = np.arange(d)
+    H = rho ** np.abs(i[:, None] - i[None, :])
+    rows = [0, 1, 77, 198, 199]
+    assert np.abs(oracle.u_rows(H, rows) - _kms_u(d, rho)[rows]).max() <= 1e-12
+    X = _spd_from_tokens(600, 150, 6, outliers=3).astype(np.float64)
+    Hd = 2.0 * X.T @ X / 600
+    Hd += 0.01 * np.diag(Hd).mean() * np.eye(150)
+    U, info = oracle.hinv_upper_chol(Hd)
+    assert info == 0
+    rows = [0, 64, 100, 149]
+    assert np.abs(oracle.u_rows(Hd, rows) - U[rows]).max() <= 1e-10 * np.abs(U).max()
 
 # --------------------------------------------------------------------------
 # The sweep
