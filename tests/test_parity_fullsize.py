@@ -3,9 +3,10 @@ attention projection (W 4096x4096 fp16, X 262144 x 4096 fp16 with 1 % outlier
 channels), one Hessian call over all tokens, prepare, sweep, pack.
 
 The oracle computes what it can at this size: a 96-column block of S (every
-token), the full float64 U from the GPU's S (the H-forced protocol), and the
-sweep of a seeded sample of rows (rows are independent given U).  Tolerances
-are those of tests/parity.py."""
+token) with its plain loop, the whole of S through BLAS (end to end: the
+oracle's own S, U and sweep), the full float64 U from the GPU's S (the
+H-forced protocol), and the sweep of a seeded sample of rows (rows are
+independent given U).  Tolerances are those of tests/parity.py."""
 import numpy as np
 import pytest
 import torch
@@ -41,7 +42,7 @@ def attn7b():
     cols = np.unique(np.concatenate([ch[:8], rng.choice(d, 88, replace=False)]))
     Xc = X[:, torch.as_tensor(cols, device=DEV)].contiguous().cpu().numpy()
     rows = np.sort(rng.choice(m, 48, replace=False))
-    out = dict(spec=spec, n=n, m=m, d=d, cols=cols, Xc=Xc, rows=rows,
+    out = dict(spec=spec, n=n, m=m, d=d, cols=cols, Xc=Xc, rows=rows, Xcpu=X.cpu(),
                W64=W.double().cpu().numpy(), S=P.to_np(S), U=P.to_np(U),
                codes=P.to_np(codes), scales=P.to_np(scales), zeros=P.to_np(zeros),
                loss=P.to_np(loss), qw=P.to_np(qw).view(np.uint32), qz=P.to_np(qz))
@@ -88,6 +89,31 @@ def test_sweep_sampled_rows_full_size(attn7b, oracle_from_gpu_S):
     assert abs(lg - lo) <= P.LOSS_REL * lo
     ties = P.teacher_forced_check(np.ascontiguousarray(a["W64"][r]), o["U"], gpu, 4, 128)
     print("attn7b sampled rows:", st, "ties", ties, "loss", lg, lo)
+
+
+def test_end_to_end_against_the_oracles_own_hessian(attn7b):
+    """End to end: the oracle's own S over all 262144 tokens (float64 BLAS
+    rank-k updates), its own damping and U, and its sweep of the sampled rows,
+    against the GPU's whole pipeline.  S is compared over the whole matrix.
+    Codes, scales, zero points and the layer loss take the tolerances of
+    tests/parity.py; the two sides now differ by S's fp32 summation as well,
+    so no teacher-forced run is made on this trajectory (the H-forced tests
+    above make it)."""
+    a = attn7b
+    S_or = oracle.hessian_syrk(a["Xcpu"])
+    assert P.rel_fro(P.mirror_upper(a["S"]), S_or) <= P.S_TOL
+    H, Hd, perm, lam, st = oracle.finalize(S_or, a["n"], 0.01, False)
+    U64, info = oracle.hinv_upper_chol(Hd)
+    assert st == 0 and info == 0
+    assert P.rel_fro(a["U"].astype(np.float64), U64) <= P.U_TOL
+    r = a["rows"]
+    ref = oracle.quantize_rows(a["W64"][r], U64, 4, 128)
+    gpu = dict(codes=a["codes"][r], scales=a["scales"][r], zeros=a["zeros"][r])
+    st = P.compare_sweep(gpu, ref, 128)
+    lg = P.layer_loss_of(a["W64"][r], gpu["codes"], gpu["scales"], gpu["zeros"], 128, None, H)
+    lo = P.layer_loss_of(a["W64"][r], ref["codes"], ref["scales"], ref["zeros"], 128, None, H)
+    assert abs(lg - lo) <= P.LOSS_REL * lo
+    print("attn7b end to end:", st, "loss", lg, lo)
 
 
 def test_pack_full_size(attn7b):

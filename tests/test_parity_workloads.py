@@ -4,8 +4,8 @@ prepare, sweep, pack):
 
   * mlp7b: 7B MLP pair, up 11008x4096 and down 4096x11008 (SiLU-gated X)
   * mlp8b_act: 8B MLP with act-order, 14336x4096 and 4096x14336
-  * moe8: two of the eight 14336x4096 experts -- the hottest and the coldest
-    (capped at 2048 routed tokens, so its Hessian is rank-deficient)
+  * moe8: all eight 14336x4096 experts, each on its routed tokens (the
+    coldest capped at 2048 routed tokens, so its Hessian is rank-deficient)
 
 At these sizes the oracle computes what it can one piece at a time:
   * S: a 96-column block (outlier channels included) over all tokens;
@@ -13,9 +13,11 @@ At these sizes the oracle computes what it can one piece at a time:
   * U: a size-independent backward-error property of the Cholesky factor of
     Hd^-1: U^-1 U^-T v = Hd v for random v (float64 triangular solves with the
     GPU's U), |residual| <= 1e-4 |Hd v|; plus triangular shape and U_jj > 0;
-    the oracle's own float64 U at d = 4096 is compared in
-    test_parity_fullsize.py (a full float64 U at d = 11008 / 14336 takes
-    minutes of host time);
+    and sampled rows of U (the first, the last 128, and seeded ones between)
+    against the oracle's rows from the same Hd, each the normalized first
+    row of the inverse of a trailing sub-Hessian, within the U tolerance
+    (the oracle's whole float64 U at d = 4096 is compared in
+    test_parity_fullsize.py; at d = 11008 / 14336 it takes minutes);
   * sweep: a seeded sample of rows through the oracle's sweep with the GPU's
     U promoted to float64 (rows are independent given U), the same code,
     scale, zero and loss tolerances as everywhere, plus the teacher-forced
@@ -84,6 +86,15 @@ def _check(spec, W, X, g, seed):
         hv = (2.0 / n) * (S64 @ w)[perm] + lam * v
         z = sla.solve_triangular(U64, sla.solve_triangular(U64, v, trans="T"), trans="N")
         assert np.linalg.norm(z - hv) <= 1e-4 * np.linalg.norm(hv)
+    # U: sampled rows against the oracle's rows of the same Hd
+    Hd = (2.0 / n) * S64[np.ix_(perm, perm)]
+    Hd[np.arange(d), np.arange(d)] += lam
+    urows = np.unique(np.concatenate([[0, 1, d // 3, (2 * d) // 3], np.arange(d - 128, d),
+                                      rng.choice(d, 4, replace=False)]))
+    R = oracle.u_rows(Hd, urows)
+    del Hd
+    u_err = P.rel_fro(U64[urows], R)
+    assert u_err <= P.U_TOL, u_err
     # sweep on sampled rows with the GPU's U
     rows = np.sort(rng.choice(m, 24, replace=False))
     W64 = W[torch.as_tensor(rows, device=DEV)].double().cpu().numpy()
@@ -92,7 +103,9 @@ def _check(spec, W, X, g, seed):
     gpu = dict(codes=g["codes"][rows], scales=g["scales"][rows], zeros=g["zeros"][rows])
     st = P.compare_sweep(gpu, res, 128)
     assert abs(g["loss"][rows].sum() - res["row_loss"].sum()) <= P.LOSS_REL * res["row_loss"].sum()
-    P.teacher_forced_check(Wp, U64, gpu, 4, 128)
+    tf = {}
+    P.teacher_forced_check(Wp, U64, gpu, 4, 128, report=tf)
+    st.update(tf, u_rows_rel_err=u_err)
     # packing of the whole layer
     rq, rz = oracle.pack_int4(g["codes"], g["zeros"])
     assert np.array_equal(g["qw"], rq) and np.array_equal(g["qz"], rz)
@@ -112,18 +125,31 @@ def test_dense_workload_layer(workload, layer):
     torch.cuda.empty_cache()
 
 
-def test_moe_hottest_and_coldest_expert():
+@pytest.mark.parametrize("expert", range(8))
+def test_moe_expert(expert):
+    """Every expert of the MoE layer on its own routed tokens (the coldest
+    capped at 2048, rank-deficient before damping)."""
     wl = inputs.WORKLOADS["moe8"]
-    spec0 = wl.layers[0]
-    X = inputs.calibration_x(spec0, device=DEV)
-    lists = inputs.moe_routing(X.shape[0], wl.n_experts, wl.zipf_s, wl.top_k, wl.cold_cap,
-                               spec0.seed)
+    X, lists = _moe_inputs()
     counts = [len(x) for x in lists]
     assert sum(counts) <= 2 * X.shape[0] and min(counts) == wl.cold_cap
-    for e in (int(np.argmax(counts)), int(np.argmin(counts))):
-        spec = wl.layers[e]
-        W = inputs.weights(spec, device=DEV)
-        Xe = X.index_select(0, torch.as_tensor(lists[e], device=DEV)).contiguous()
-        g = _run_layer(W, Xe, Xe.shape[0], False)
-        st = _check(spec, W, Xe, g, 200 + e)
-        print("expert", e, "tokens", counts[e], st)
+    spec = wl.layers[expert]
+    W = inputs.weights(spec, device=DEV)
+    Xe = X.index_select(0, torch.as_tensor(lists[expert], device=DEV)).contiguous()
+    g = _run_layer(W, Xe, Xe.shape[0], False)
+    st = _check(spec, W, Xe, g, 200 + expert)
+    print("expert", expert, "tokens", counts[expert], st)
+
+
+_MOE = {}
+
+
+def _moe_inputs():
+    if "X" not in _MOE:
+        wl = inputs.WORKLOADS["moe8"]
+        spec0 = wl.layers[0]
+        X = inputs.calibration_x(spec0, device=DEV)
+        _MOE["X"] = X
+        _MOE["lists"] = inputs.moe_routing(X.shape[0], wl.n_experts, wl.zipf_s, wl.top_k,
+                                           wl.cold_cap, spec0.seed)
+    return _MOE["X"], _MOE["lists"]
