@@ -190,7 +190,10 @@ int gptq_prepare_hinv_static(const float* S, int64_t d, int64_t n_tokens, float 
  * codes: d_out x d_in uint8 output, sweep order (code of column perm[k] at k).
  * scales: d_out x G fp16 output (G = d_in / group_size), zeros: d_out x G uint8.
  * row_loss: d_out fp32 output or NULL: sum_j E_j^2 (= tr(D Hd D^T) per row).
- * bits in {2,3,4,8}; group_size in {32, 64, 128}; block_size == 128.
+ * bits in {2,3,4,8}; group_size in {32, 64, 128}, or -1 (or d_in) for one
+ * group per row (G = 1: its parameters come from the row before any
+ * correction, which is what "at the group's first column" means for column
+ * 0); block_size == 128.
  * Requires d_in % 128 == 0, 128 <= d_in <= 32768, 1 <= d_out <= 2^24.
  */
 size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, int block_size);
@@ -198,6 +201,22 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
                         const float* U, const int32_t* perm, int bits, int group_size,
                         int block_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
                         float* row_loss, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * gptq_quantize_layer with STATIC groups: every group's scale and zero point
+ * are taken, by the same min-max rule ("校准艺术" sec. 2.1), from the row as
+ * it is before the sweep (W's columns in sweep order, no correction yet),
+ * instead of from the corrected values at the group's first column.  The
+ * codes, the error feedback and every other output are as in
+ * gptq_quantize_layer.  The pages fix the group parameters only by the
+ * min-max rule; this is the reading that parameterizes before correcting.
+ * Same arguments and errors as gptq_quantize_layer, except group_size: 32,
+ * 64, any multiple of 128 that divides d_in, or -1 (one group per row).
+ */
+int gptq_quantize_layer_static(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
+                               const float* U, const int32_t* perm, int bits, int group_size,
+                               int block_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
+                               float* row_loss, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Pack INT4 -- "INT4/INT8 量化推理" sec. 一 (64 B of codes + 0.5 B zero point

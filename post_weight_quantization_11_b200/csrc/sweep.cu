@@ -54,10 +54,14 @@ __global__ void init_work_kernel(const T* __restrict__ W, const int32_t* __restr
 // min/max is reduced over the row's lanes (lanes outside the group
 // contribute 0, neutral since the range includes 0).  The outer loop over the
 // 8 owner lanes is not unrolled, which keeps the kernel's code small.
-template <int GS>
+// STATIC: the group parameters were set before the sweep (static groups, or
+// one group per row); the kernel loads them at each group start inside the
+// block and at the block's first column instead of reducing min/max.  GS is
+// then min(group size, 128) and gsz the group size.
+template <int GS, bool STATIC>
 __global__ void __launch_bounds__(SW_THREADS)
 block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
-                   int64_t j0, float maxqf, uint8_t* __restrict__ codes,
+                   int64_t gsz, int64_t j0, float maxqf, uint8_t* __restrict__ codes,
                    __half* __restrict__ scales, uint8_t* __restrict__ zeros,
                    float* __restrict__ Eh_out, float* __restrict__ El_out, int64_t ldE,
                    float* __restrict__ row_loss, int first_block)
@@ -101,7 +105,7 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     bool valid[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) { row[r] = rbase + 4 * r; valid[r] = row[r] < m; }
-    const int64_t G = d / GS;
+    const int64_t G = d / gsz;
 
     float w[2][SW_CPL];
 #pragma unroll
@@ -139,7 +143,19 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
 #pragma unroll
         for (int ji = 0; ji < SW_CPL; ++ji) {
             const int j = jo * SW_CPL + ji;
-            if (ji == 0 && (jo * SW_CPL) % GS == 0) {
+            if (STATIC && ji == 0 && (jo * SW_CPL) % GS == 0) {
+                const int64_t gi = (j0 + j) / gsz;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    if (valid[r]) {
+                        const __half h = scales[row[r] * G + gi];
+                        gq[r].h = h;
+                        gq[r].s = __half2float(h);
+                        gq[r].z = float(zeros[row[r] * G + gi]);
+                        gq[r].r = __frcp_rn(gq[r].s);
+                    }
+                }
+            } else if (ji == 0 && (jo * SW_CPL) % GS == 0) {
                 constexpr int span = GS / SW_CPL;            // lanes covering one group
                 const bool in_group = sub >= jo && sub < jo + span;
 #pragma unroll
@@ -263,6 +279,37 @@ rtn_kernel(const T* __restrict__ W, int64_t m, int64_t d, float maxqf,
     }
 }
 
+// Static group parameters: one warp per (row, group) of the working copy
+// (sweep order, before any correction); min/max over the group with the
+// range including 0, then the same group_params as the sweep and RTN.
+__global__ void __launch_bounds__(256)
+static_params_kernel(const float* __restrict__ Wk, int64_t m, int64_t d, int64_t gsz,
+                     float maxqf, __half* __restrict__ scales, uint8_t* __restrict__ zeros)
+{
+    const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t G = d / gsz;
+    if (wid >= m * G) return;               // whole warp exits together
+    const int64_t row = wid / G, gi = wid - row * G;
+    const float* p = Wk + row * d + gi * gsz;
+    float mn = 0.f, mx = 0.f;
+    for (int64_t c = 4 * lane; c < gsz; c += 128) {
+        const float4 v = *reinterpret_cast<const float4*>(p + c);
+        mn = fminf(fminf(mn, v.x), fminf(v.y, fminf(v.z, v.w)));
+        mx = fmaxf(fmaxf(mx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+    }
+    if (lane == 0) {
+        const GroupQ gq = group_params(mn, mx, maxqf);
+        scales[row * G + gi] = gq.h;
+        zeros[row * G + gi] = (uint8_t)gq.z;
+    }
+}
+
 struct QuantWs {
     float* Wk;     // d_out x d_in working copy (sweep order)
     UpdateWs upd;  // split U and the current block's split errors
@@ -281,27 +328,25 @@ static size_t quant_layout(int64_t m, int64_t d, char* base, QuantWs* w)
     return off;
 }
 
-static int check_quant_args(int w_dtype, int64_t m, int64_t d, int bits, int group_size)
+static int check_quant_args(int w_dtype, int64_t m, int64_t d, int bits)
 {
     if (w_dtype != GPTQ_DTYPE_F16 && w_dtype != GPTQ_DTYPE_F32) return GPTQ_ERR_INVALID_ARG;
     if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8)) return GPTQ_ERR_UNSUPPORTED;
-    if (!(group_size == 32 || group_size == 64 || group_size == 128)) return GPTQ_ERR_UNSUPPORTED;
     if (d < 128 || d > kMaxDim || d % 128 != 0) return GPTQ_ERR_SHAPE;
     if (m < 1 || m > kMaxRows) return GPTQ_ERR_SHAPE;
     return GPTQ_OK;
 }
 
-template <int GS>
+template <int GS, bool STATIC>
 static void launch_sweep(dim3 grid, size_t smem, cudaStream_t st, const float* Wk, const float* U,
-                         int64_t m, int64_t d, int64_t j0, float maxqf, uint8_t* codes,
-                         __half* scales, uint8_t* zeros, float* Eh, float* El, int64_t ldE,
-                         float* row_loss, int first)
+                         int64_t m, int64_t d, int64_t gsz, int64_t j0, float maxqf,
+                         uint8_t* codes, __half* scales, uint8_t* zeros, float* Eh, float* El,
+                         int64_t ldE, float* row_loss, int first)
 {
-    cudaFuncSetAttribute(block_sweep_kernel<GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    block_sweep_kernel<GS><<<grid, SW_THREADS, smem, st>>>(Wk, U, m, d, j0, maxqf, codes, scales,
-                                                          zeros,
-                                                   Eh, El, ldE, row_loss, first);
+    cudaFuncSetAttribute(block_sweep_kernel<GS, STATIC>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    block_sweep_kernel<GS, STATIC><<<grid, SW_THREADS, smem, st>>>(
+        Wk, U, m, d, gsz, j0, maxqf, codes, scales, zeros, Eh, El, ldE, row_loss, first);
     count_launches();
 }
 
@@ -313,16 +358,37 @@ extern "C" size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, int
     return gptq::quant_layout(d_out, d_in, nullptr, nullptr);
 }
 
-extern "C" int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
-                                   const float* U, const int32_t* perm, int bits, int group_size,
-                                   int block_size, uint8_t* codes, uint16_t* scales,
-                                   uint8_t* zeros, float* row_loss, void* ws, size_t ws_bytes,
-                                   void* stream)
+namespace gptq {
+
+// Group sizes the sweep takes: dynamic groups (parameters at each group's
+// first column from the corrected row) in {32, 64, 128}; static groups
+// (parameters from the rows before the sweep) in {32, 64} or any multiple of
+// 128 dividing d; one group per row (-1 or d) is the static case, since at
+// column 0 no correction has happened yet.
+static int sweep_group_size(int64_t d, int group_size, bool static_groups, int64_t* gsz)
 {
-    using namespace gptq;
+    if (group_size == -1 || group_size == d) { *gsz = d; return GPTQ_OK; }
+    if (group_size == 32 || group_size == 64 || group_size == 128) { *gsz = group_size; return GPTQ_OK; }
+    if (static_groups && group_size > 128 && group_size % 128 == 0 && d % group_size == 0) {
+        *gsz = group_size;
+        return GPTQ_OK;
+    }
+    return GPTQ_ERR_UNSUPPORTED;
+}
+
+static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
+                         const float* U, const int32_t* perm, int bits, int group_size,
+                         int block_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
+                         float* row_loss, void* ws, size_t ws_bytes, void* stream,
+                         bool static_groups)
+{
     if (!W || !U || !codes || !scales || !zeros || !ws) return GPTQ_ERR_INVALID_ARG;
-    int rc = check_quant_args(w_dtype, d_out, d_in, bits, group_size);
+    int rc = check_quant_args(w_dtype, d_out, d_in, bits);
     if (rc != GPTQ_OK) return rc;
+    int64_t gsz = 0;
+    rc = sweep_group_size(d_in, group_size, static_groups, &gsz);
+    if (rc != GPTQ_OK) return rc;
+    const bool stat = static_groups || gsz == d_in;
     if (block_size != SW_B) return GPTQ_ERR_UNSUPPORTED;
     if (!aligned16(W) || !aligned16(U) || !aligned16(codes) || !aligned16(scales) ||
         !aligned16(zeros) || !aligned16(ws) || (perm && !aligned16(perm)) ||
@@ -345,12 +411,18 @@ extern "C" int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, in
                                                           m, d, w.Wk);
         count_launches();
     }
+    const float maxqf = float((1 << bits) - 1);
+    __half* sc = reinterpret_cast<__half*>(scales);
+    if (stat) {
+        const int64_t warps = m * (d / gsz);
+        static_params_kernel<<<(unsigned)ceil_div(warps * 32, 256), 256, 0, st>>>(
+            w.Wk, m, d, gsz, maxqf, sc, zeros);
+        count_launches();
+    }
     rc = update_prepare_u(U, d, &w.upd, st);
     if (rc != GPTQ_OK) return rc;
-    const float maxqf = float((1 << bits) - 1);
     const dim3 grid((unsigned)ceil_div(m, SW_ROWS));
     const size_t smem = sizeof(float) * (SW_B * SW_B + SW_B);
-    __half* sc = reinterpret_cast<__half*>(scales);
     // Deferred (two-level) error feedback: after each 128-column block only the
     // rest of its 512-column outer block is updated (K = 128); the columns
     // beyond an outer block get the outer block's four blocks at once
@@ -364,14 +436,23 @@ extern "C" int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, in
         const int64_t ecol = j0 - ob0;                                     // E column of this block
         float* Eh = w.upd.Eh + ecol;
         float* El = w.upd.El + ecol;
-        switch (group_size) {
-            case 32: launch_sweep<32>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                      Eh, El, UPD_LDE, row_loss, b == 0); break;
-            case 64: launch_sweep<64>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                      Eh, El, UPD_LDE, row_loss, b == 0); break;
-            default: launch_sweep<128>(grid, smem, st, w.Wk, U, m, d, j0, maxqf, codes, sc, zeros,
-                                       Eh, El, UPD_LDE, row_loss, b == 0); break;
+#define GPTQ_SWEEP(GSV, STAT)                                                                   \
+        launch_sweep<GSV, STAT>(grid, smem, st, w.Wk, U, m, d, gsz, j0, maxqf, codes, sc, zeros, \
+                                Eh, El, UPD_LDE, row_loss, b == 0)
+        if (stat) {
+            switch (gsz) {
+                case 32: GPTQ_SWEEP(32, true); break;
+                case 64: GPTQ_SWEEP(64, true); break;
+                default: GPTQ_SWEEP(128, true); break;     // groups of 128 or more
+            }
+        } else {
+            switch (gsz) {
+                case 32: GPTQ_SWEEP(32, false); break;
+                case 64: GPTQ_SWEEP(64, false); break;
+                default: GPTQ_SWEEP(128, false); break;
+            }
         }
+#undef GPTQ_SWEEP
         if (j0 + SW_B < ob1) {                                   // near: rest of the outer block
             rc = block_update(w.Wk, &w.upd, m, d, /*e_col0=*/ecol, /*k_rows=*/SW_B, /*u_row0=*/j0,
                               /*c_begin=*/j0 + SW_B, /*c_end=*/ob1, st);
@@ -386,14 +467,38 @@ extern "C" int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, in
     return launch_status();
 }
 
+}  // namespace gptq
+
+extern "C" int gptq_quantize_layer(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
+                                   const float* U, const int32_t* perm, int bits, int group_size,
+                                   int block_size, uint8_t* codes, uint16_t* scales,
+                                   uint8_t* zeros, float* row_loss, void* ws, size_t ws_bytes,
+                                   void* stream)
+{
+    return gptq::quantize_impl(W, w_dtype, d_out, d_in, U, perm, bits, group_size, block_size,
+                               codes, scales, zeros, row_loss, ws, ws_bytes, stream, false);
+}
+
+extern "C" int gptq_quantize_layer_static(const void* W, int w_dtype, int64_t d_out,
+                                          int64_t d_in, const float* U, const int32_t* perm,
+                                          int bits, int group_size, int block_size,
+                                          uint8_t* codes, uint16_t* scales, uint8_t* zeros,
+                                          float* row_loss, void* ws, size_t ws_bytes,
+                                          void* stream)
+{
+    return gptq::quantize_impl(W, w_dtype, d_out, d_in, U, perm, bits, group_size, block_size,
+                               codes, scales, zeros, row_loss, ws, ws_bytes, stream, true);
+}
+
 extern "C" int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bits,
                             int group_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
                             void* stream)
 {
     using namespace gptq;
     if (!W || !codes || !scales || !zeros) return GPTQ_ERR_INVALID_ARG;
-    int rc = check_quant_args(w_dtype, d_out, d_in, bits, group_size);
+    int rc = check_quant_args(w_dtype, d_out, d_in, bits);
     if (rc != GPTQ_OK) return rc;
+    if (!(group_size == 32 || group_size == 64 || group_size == 128)) return GPTQ_ERR_UNSUPPORTED;
     if (!aligned16(W) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros))
         return GPTQ_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);

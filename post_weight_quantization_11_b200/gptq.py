@@ -30,7 +30,8 @@ EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_device_status",
             "gptq_hessian_accumulate", "gptq_hessian_accumulate_host",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
-            "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_pack_int4",
+            "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_quantize_layer_static",
+            "gptq_pack_int4",
             "gptq_unpack_int4", "rtn_quantize", "gptq_debug_gemm_nt",
             "gptq_debug_chol_task_order", "gptq_debug_div_rn", "gptq_debug_bounded_wait")
 
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_quantize_workspace_bytes": ([I64, I64, I32], SZ),
         "gptq_quantize_layer": ([P, I32, I64, I64, P, P, I32, I32, I32, P, P, P, P, P, SZ, P],
                                 I32),
+        "gptq_quantize_layer_static": ([P, I32, I64, I64, P, P, I32, I32, I32, P, P, P, P, P, SZ,
+                                        P], I32),
         "gptq_pack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "gptq_unpack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "rtn_quantize": ([P, I32, I64, I64, I32, I32, P, P, P, P], I32),
@@ -254,13 +257,15 @@ def gptq_quantize_workspace_bytes(d_out: int, d_in: int, block_size: int = 128) 
 
 def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm=None, bits: int = 4,
                         group_size: int = 128, block_size: int = 128, codes=None, scales=None,
-                        zeros=None, row_loss=None, ws=None):
-    """Returns (codes uint8 m x d, scales fp16 m x G, zeros uint8 m x G, row_loss fp32 m)."""
+                        zeros=None, row_loss=None, ws=None, static_groups: bool = False):
+    """Returns (codes uint8 m x d, scales fp16 m x G, zeros uint8 m x G, row_loss fp32 m).
+    group_size -1: one group per row.  static_groups: group parameters from
+    the rows before the sweep (gptq_quantize_layer_static)."""
     _need(W, "W")
     _need(U, "U", torch.float32)
     m, d = W.shape
     dev = W.device
-    G = d // group_size
+    G = 1 if group_size in (-1, d) else d // group_size
     codes = torch.empty(m, d, dtype=torch.uint8, device=dev) if codes is None else codes
     scales = torch.empty(m, G, dtype=torch.float16, device=dev) if scales is None else scales
     zeros = torch.empty(m, G, dtype=torch.uint8, device=dev) if zeros is None else zeros
@@ -269,12 +274,12 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm=None, bits: int =
     ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev) if ws is None else ws
     if perm is not None:
         _need(perm, "perm", torch.int32)
-    _check("gptq_quantize_layer",
-           load_library().gptq_quantize_layer(_ptr(W), _wdtype(W), m, d, _ptr(U), _ptr(perm),
-                                              int(bits), int(group_size), int(block_size),
-                                              _ptr(codes), _ptr(scales), _ptr(zeros),
-                                              _ptr(row_loss), _ptr(ws),
-                                              ws.numel() * ws.element_size(), _stream(W)))
+    name = "gptq_quantize_layer_static" if static_groups else "gptq_quantize_layer"
+    _check(name, getattr(load_library(), name)(_ptr(W), _wdtype(W), m, d, _ptr(U), _ptr(perm),
+                                               int(bits), int(group_size), int(block_size),
+                                               _ptr(codes), _ptr(scales), _ptr(zeros),
+                                               _ptr(row_loss), _ptr(ws),
+                                               ws.numel() * ws.element_size(), _stream(W)))
     return codes, scales, zeros, row_loss
 
 

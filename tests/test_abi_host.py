@@ -121,6 +121,18 @@ def test_validation_rejects_before_launch(lib):
     assert q(W=None) == 1
     assert q(U=MIS) == 1
     assert q(wsb=100) == 1
+    assert q(g=256, d=512) == 4               # dynamic groups span one block at most
+    assert q(g=-1, wsb=100) == 1              # one group per row: accepted up to the ws check
+
+    def qs(**k):
+        a = args(**k)
+        return lib.gptq_quantize_layer_static(a["W"], a["dt"], a["m"], a["d"], a["U"], a["perm"],
+                                              a["bits"], a["g"], a["B"], a["codes"], a["scales"],
+                                              a["zeros"], a["loss"], a["ws"], a["wsb"], None)
+    assert qs(g=96) == 4
+    assert qs(g=384) == 4                     # must divide d_in
+    assert qs(g=256, wsb=100) == 1            # accepted up to the ws check
+    assert qs(bits=5) == 4 and qs(d=200) == 2 and qs(W=None) == 1
     assert lib.rtn_quantize(FAKE, 1, 64, 256, 3, 48, FAKE, FAKE, FAKE, None) == 4
     assert lib.rtn_quantize(None, 1, 64, 256, 4, 128, FAKE, FAKE, FAKE, None) == 1
     assert lib.gptq_pack_int4(FAKE, FAKE, 4, 12, 1, FAKE, FAKE, None) == 2

@@ -163,6 +163,41 @@ def test_sharded_layer_on_one_process_matches_the_direct_path():
     assert torch.equal(qw, L.qweight) and torch.equal(qz, L.qzeros)
 
 
+@pytest.mark.parametrize("gs,static,act", [(32, True, False), (128, True, True), (256, True, False),
+                                           (-1, True, False), (-1, False, True)])
+def test_static_and_per_channel_groups(gs, static, act):
+    """Static groups (parameters from the rows before the sweep) and one
+    group per row, against the oracle on the GPU's S: the parameters come
+    from the uncorrected weights, so scales and zero points are bit-exact;
+    codes and loss as in every layer test.  d = 1024 takes the far update."""
+    m, d, n = 200, 1024, 2048
+    W = _weights(m, d, torch.float16, 31)
+    X = _gauss_x(n, d, 3, 50.0, 32)
+    Wd, Xd = W.to(DEV), X.to(DEV)
+    S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    G.gptq_hessian_accumulate(S, Xd)
+    perm, U, info = G.gptq_prepare_hinv(S, n, 0.01, act)
+    codes, scales, zeros, _ = G.gptq_quantize_layer(Wd, U, perm if act else None, 4, gs,
+                                                    static_groups=static)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    S64 = P.mirror_upper(P.to_np(S))
+    _, Hd, perm_o, _, st = oracle.finalize(S64, n, 0.01, act)
+    U_o, inf = oracle.hinv_upper_chol(Hd)
+    assert st == 0 and inf == 0
+    assert np.array_equal(P.to_np(perm), perm_o)
+    W64 = W.double().numpy()
+    Wp = np.ascontiguousarray(W64[:, perm_o])
+    ref = (oracle.quantize_rows_static if static else oracle.quantize_rows)(Wp, U_o, 4, gs)
+    sc, zr, cd = P.to_np(scales), P.to_np(zeros), P.to_np(codes)
+    assert np.array_equal(sc, ref["scales"]) and np.array_equal(zr, ref["zeros"])
+    assert float((cd != ref["codes"]).mean()) <= P.CODE_FRAC
+    H64 = 2.0 * S64 / n
+    lg = P.layer_loss_of(W64, cd, sc, zr, gs, perm_o, H64)
+    lo = P.layer_loss_of(W64, ref["codes"], ref["scales"], ref["zeros"], gs, perm_o, H64)
+    assert abs(lg - lo) <= P.LOSS_REL * lo, (lg, lo)
+
+
 @pytest.mark.parametrize("act_order,d", [(False, 512), (True, 512), (False, 640), (True, 1152)])
 def test_prepare_parity(act_order, d):
     n = 2048
