@@ -67,6 +67,19 @@ uint64_t gptq_debug_launch_count(void);
 int gptq_device_status(int32_t* status_out, int reset);
 
 /*
+ * Launch configuration (no counterpart on the pages): caps the CTAs of the
+ * library's persistent kernels of one kind -- GPTQ_CTAS_HESSIAN (the Hessian
+ * accumulation) or GPTQ_CTAS_PREPARE (the factorization in
+ * gptq_prepare_hinv) -- at max_ctas (0: one per SM, the default).  A caller
+ * that runs one layer's preparation beside the next layer's Hessian on two
+ * streams gives each a share of the SMs this way; both kernels are correct
+ * for any count.  Process-wide, read at each launch; not synchronized with
+ * launches in flight.  Returns GPTQ_OK or GPTQ_ERR_INVALID_ARG.
+ */
+enum { GPTQ_CTAS_HESSIAN = 0, GPTQ_CTAS_PREPARE = 1 };
+int gptq_set_max_ctas(int kind, int max_ctas);
+
+/*
  * Hessian accumulation -- "GPTQ / AWQ / SqueezeLLM" sec. 一 (H from the
  * calibration inputs; the 2/n factor is applied later by gptq_prepare_hinv).
  *

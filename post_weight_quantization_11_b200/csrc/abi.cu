@@ -51,7 +51,23 @@ int device_sm_count()
     return n;
 }
 
+static std::atomic<int> g_cta_cap[kCtaKinds];
+
+int persistent_ctas(int kind)
+{
+    const int sms = device_sm_count();
+    const int cap = (kind >= 0 && kind < kCtaKinds) ? g_cta_cap[kind].load() : 0;
+    return cap > 0 ? std::min(cap, sms) : sms;
+}
+
 }  // namespace gptq
+
+extern "C" int gptq_set_max_ctas(int kind, int max_ctas)
+{
+    if (kind < 0 || kind >= gptq::kCtaKinds || max_ctas < 0) return GPTQ_ERR_INVALID_ARG;
+    gptq::g_cta_cap[kind].store(max_ctas);
+    return GPTQ_OK;
+}
 
 extern "C" const char* gptq_status_string(int status)
 {

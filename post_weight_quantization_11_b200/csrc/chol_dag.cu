@@ -499,7 +499,7 @@ int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d,
     if (cudaFuncSetAttribute(chol_dag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CD_SMEM) != cudaSuccess)
         return GPTQ_ERR_CUDA;
-    const int grid = std::min(p.total, device_sm_count());
+    const int grid = std::min(p.total, persistent_ctas(kCtaPrepare));
     chol_dag_kernel<<<grid, CD_THREADS, CD_SMEM, st>>>(tA, tX, tY, p);
     count_launches();
     return launch_status();

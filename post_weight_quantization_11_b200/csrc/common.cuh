@@ -32,6 +32,11 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Number of SMs of the current device (cached per device after the first query).
 int device_sm_count();
 
+// Persistent-grid caps set by gptq_set_max_ctas (0: none): the CTAs a
+// persistent kernel of that kind launches are min(SMs, cap).
+enum CtaKind : int { kCtaHessian = 0, kCtaPrepare = 1, kCtaKinds = 2 };
+int persistent_ctas(int kind);
+
 // Supported problem limits (validated at the ABI).
 constexpr int64_t kMaxDim = 32768;
 constexpr int64_t kMaxRows = int64_t(1) << 24;

@@ -229,7 +229,7 @@ extern "C" int gptq_hessian_accumulate(float* S, const uint16_t* X, int64_t n_to
     p.nbi = (int)(d / HB_M);
     const int nbj = (int)ceil_div(d, HB_N);
     p.tiles = (nbj - 1) * nbj + std::min(2 * nbj, p.nbi);
-    const int P = device_sm_count();
+    const int P = persistent_ctas(kCtaHessian);
     const int64_t ksteps = ceil_div(n_tokens, HB_K);
     // smallest token split count whose round-robin over P CTAs is >= 90 % busy
     int64_t best_s = 1;

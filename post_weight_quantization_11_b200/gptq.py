@@ -27,7 +27,7 @@ _STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_SHAPE", 3: "GPT
 
 # every symbol include/gptq.h declares
 EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
-            "gptq_device_status",
+            "gptq_device_status", "gptq_set_max_ctas",
             "gptq_hessian_accumulate", "gptq_hessian_accumulate_host",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_quantize_layer_static",
@@ -61,6 +61,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_abi_version": ([], I32),
         "gptq_debug_launch_count": ([], ctypes.c_uint64),
         "gptq_device_status": ([P, I32], I32),
+        "gptq_set_max_ctas": ([I32, I32], I32),
         "gptq_hessian_accumulate": ([P, P, I64, I64, P, P], I32),
         "gptq_hessian_accumulate_host": ([P, P, I64, I64, P, P, SZ, I64, P, P, P, P], I32),
         "gptq_prepare_workspace_bytes": ([I64], SZ),
@@ -134,6 +135,15 @@ def gptq_device_status(reset: bool = True) -> int:
     v = ctypes.c_int32(0)
     _check("gptq_device_status", load_library().gptq_device_status(ctypes.byref(v), int(reset)))
     return int(v.value)
+
+
+GPTQ_CTAS_HESSIAN, GPTQ_CTAS_PREPARE = 0, 1
+
+
+def gptq_set_max_ctas(kind: int, max_ctas: int) -> None:
+    """Cap the CTAs of the persistent Hessian (kind 0) or factorization
+    (kind 1) kernels; 0 restores one per SM."""
+    _check("gptq_set_max_ctas", load_library().gptq_set_max_ctas(int(kind), int(max_ctas)))
 
 
 def gptq_status_string(status: int) -> str:

@@ -38,6 +38,13 @@ def test_exports_every_declared_symbol(lib):
         assert re.search(rf"\bT {n}\b", out), n
 
 
+def test_cta_caps(lib):
+    assert lib.gptq_set_max_ctas(2, 10) == 1 and lib.gptq_set_max_ctas(-1, 10) == 1
+    assert lib.gptq_set_max_ctas(0, -1) == 1
+    assert lib.gptq_set_max_ctas(0, 32) == 0 and lib.gptq_set_max_ctas(1, 16) == 0
+    assert lib.gptq_set_max_ctas(0, 0) == 0 and lib.gptq_set_max_ctas(1, 0) == 0
+
+
 def test_status_strings_and_version(lib):
     assert G.gptq_abi_version() == 100
     for code, name in G._STATUS.items():

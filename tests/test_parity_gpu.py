@@ -267,6 +267,31 @@ def test_gptq_equals_rtn_when_hessian_is_isotropic():
         assert np.array_equal(P.to_np(sc), P.to_np(rs)) and np.array_equal(P.to_np(z), P.to_np(rz))
 
 
+def test_cta_caps_keep_the_results():
+    """The persistent kernels on fewer CTAs than SMs: the Hessian sums in
+    another order (within fp32 rounding), the factorization's tasks do the
+    same arithmetic whichever CTA runs them (U bit for bit)."""
+    d, n = 1024, 4096
+    X = _gauss_x(n, d, 3, 50.0, 51).to(DEV)
+    S0 = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    G.gptq_hessian_accumulate(S0, X)
+    _, U0, info0 = G.gptq_prepare_hinv(S0, n, 0.01, False)
+    try:
+        G.gptq_set_max_ctas(G.GPTQ_CTAS_HESSIAN, 24)
+        G.gptq_set_max_ctas(G.GPTQ_CTAS_PREPARE, 7)
+        S1 = torch.zeros_like(S0)
+        G.gptq_hessian_accumulate(S1, X)
+        _, U1, info1 = G.gptq_prepare_hinv(S0, n, 0.01, False)
+        torch.cuda.synchronize()
+    finally:
+        G.gptq_set_max_ctas(G.GPTQ_CTAS_HESSIAN, 0)
+        G.gptq_set_max_ctas(G.GPTQ_CTAS_PREPARE, 0)
+    assert int(info0.item()) == 0 and int(info1.item()) == 0
+    a, b = P.to_np(S1).astype(np.float64), P.to_np(S0).astype(np.float64)
+    assert P.rel_fro(np.triu(a), np.triu(b)) <= 1e-6
+    assert torch.equal(U1, U0)
+
+
 def test_prepare_reports_non_pd():
     d = 256
     S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
