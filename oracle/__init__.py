@@ -21,6 +21,9 @@ float64, no blocking) and cites the passage it follows:
 * ``trace_quadratic`` -- tr(D H D^T), the layer loss of sec. 三 of that page.
 * ``w4a16_matmul`` -- y = x Q^T from the packed layer (weight-only INT4 with
                       fp16 activations, "INT4/INT8 量化推理" sec. 六).
+* ``channel_magnitude``/``awq_search``/``awq_then_gptq`` -- activation-aware
+                      channel scaling ahead of the sweep ("GPTQ / AWQ /
+                      SqueezeLLM" sec. 二; "INT4/INT8 量化推理" sec. 四).
 """
 from __future__ import annotations
 
@@ -337,3 +340,80 @@ def layer_loss(W: np.ndarray, Q: np.ndarray, H_orig: np.ndarray) -> float:
     ||(W - Q) X^T||_F^2 for H = 2 X^T X / n."""
     D = np.asarray(W, dtype=np.float64) - np.asarray(Q, dtype=np.float64)
     return trace_quadratic(D, H_orig)
+
+
+# --------------------------------------------------------------------------
+# Activation-aware channel scaling ahead of the sweep
+# --------------------------------------------------------------------------
+
+def channel_magnitude(X) -> np.ndarray:
+    """a_j = mean over tokens of |X[t, j]|: the per-input-channel activation
+    magnitude AWQ scales by ("GPTQ / AWQ / SqueezeLLM" sec. 二: the mean of
+    the absolute activations per channel)."""
+    Xf = np.asarray(X)
+    if Xf.dtype == np.uint16:
+        Xf = Xf.view(np.float16)
+    return np.abs(Xf.astype(np.float64)).mean(axis=0)
+
+
+def awq_candidate_scales(a: np.ndarray, alpha: float) -> np.ndarray:
+    """s = (a / mean(a))^alpha per input channel; a channel whose magnitude is
+    0 takes the smallest positive one instead (the pages do not say; a zero
+    scale would erase the channel)."""
+    a = np.asarray(a, dtype=np.float64)
+    pos = a[a > 0]
+    floor = pos.min() if pos.size else 1.0
+    a = np.where(a > 0, a, floor)
+    return (a / a.mean()) ** alpha
+
+
+def awq_search(W: np.ndarray, S: np.ndarray, n: int, a: np.ndarray, bits: int = 4,
+               group_size: int = 128, n_grid: int = 20):
+    """Choose the channel scaling by the output error, "GPTQ / AWQ /
+    SqueezeLLM" sec. 二 (scale each input channel's weights up by its
+    activation magnitude before quantizing, divide back afterwards; pick
+    among candidate scalings the one with the smallest output error) and
+    "INT4/INT8 量化推理" sec. 四 (the transform is exact before quantization).
+
+    For alpha = k / n_grid, k = 0 .. n_grid - 1: s = awq_candidate_scales(a,
+    alpha), W' = W diag(s), Q' = the group round-to-nearest of W' (the
+    quantizer AWQ uses, no error feedback), D = Q' diag(s)^-1 - W, loss =
+    tr(D H D^T) with H = 2 S / n (= (2/n) ||D X^T||^2).  alpha = 0 (no
+    scaling) is a candidate, so the choice never loses to round-to-nearest
+    on the calibration loss.  Ties go to the smaller alpha.
+
+    Returns dict(alpha, s, losses (n_grid,), alphas (n_grid,)).
+    """
+    W = np.asarray(W, dtype=np.float64)
+    S = np.ascontiguousarray(S, dtype=np.float64)
+    H = 2.0 * S / n
+    alphas = np.arange(n_grid, dtype=np.float64) / n_grid
+    losses = np.empty(n_grid)
+    for k, al in enumerate(alphas):
+        s = awq_candidate_scales(a, al)
+        Ws = np.ascontiguousarray(W * s[None, :])
+        r = rtn(Ws, bits, group_size)
+        Qs = dequantize(r["codes"], r["scales"], r["zeros"], group_size)
+        losses[k] = layer_loss(W, Qs / s[None, :], H)
+    k = int(np.argmin(losses))
+    return dict(alpha=float(alphas[k]), s=awq_candidate_scales(a, alphas[k]), losses=losses,
+                alphas=alphas)
+
+
+def awq_then_gptq(W: np.ndarray, S: np.ndarray, n: int, a: np.ndarray, bits: int = 4,
+                  group_size: int = 128, damp_rel: float = 0.01, act_order: bool = False,
+                  n_grid: int = 20):
+    """The combination the pages suggest ("GPTQ / AWQ / SqueezeLLM" sec. 二:
+    first the AWQ scaling, then GPTQ's error compensation): with s from
+    awq_search, GPTQ quantizes W' = W diag(s) against the inputs X' = X
+    diag(s)^-1, i.e. S' = diag(s)^-1 S diag(s)^-1.  The dequantized layer is
+    Q' diag(s)^-1; at inference the 1/s is folded into whatever produces X.
+
+    Returns gptq_layer's dict for (W', S') plus s and alpha."""
+    sr = awq_search(W, S, n, a, bits, group_size, n_grid)
+    s = sr["s"]
+    Wp = np.asarray(W, dtype=np.float64) * s[None, :]
+    Sp = np.asarray(S, dtype=np.float64) / np.outer(s, s)
+    res = gptq_layer(Wp, Sp, n, bits, group_size, damp_rel, act_order)
+    res.update(s=s, alpha=sr["alpha"], awq_losses=sr["losses"])
+    return res

@@ -62,6 +62,12 @@ MIS = ctypes.c_void_p((1 << 20) + 4)     # misaligned
 
 
 def test_validation_rejects_before_launch(lib):
+    # The calls below pass fake device addresses and rely on the library
+    # rejecting them before any launch; where a GPU is visible a call that
+    # wrongly passed would launch on them, so these checks run without one.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-side argument checks with fake pointers run where no GPU is visible")
     n0 = ctypes.c_int64(0)
     # null / misaligned pointers
     assert lib.gptq_hessian_accumulate(None, FAKE, 10, 256, None, None) == 1

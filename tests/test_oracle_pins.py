@@ -329,6 +329,71 @@ def test_static_groups_special_cases():
     assert abs(st["row_loss"].sum() - oracle.trace_quadratic(D, Hd)) <= 1e-9 * st["row_loss"].sum()
 
 
+def test_awq_search_pins():
+    """The channel-scaling search: the alpha = 0 candidate is round-to-nearest,
+    every candidate's loss equals the output error evaluated through X itself,
+    the choice is the first minimizer, and the search depends on the
+    activations only through a / mean(a)."""
+    rng = _rng(31)
+    n, m, d, g = 600, 40, 128, 32
+    X = rng.standard_normal((n, d))
+    X[:, [3, 50]] *= 40.0
+    X = X.astype(np.float16)
+    W = 0.02 * rng.standard_normal((m, d))
+    S = oracle.hessian(X)
+    a = oracle.channel_magnitude(X)
+    r = oracle.awq_search(W, S, n, a, 4, g, n_grid=10)
+    X64 = X.astype(np.float64)
+
+    def through_x(alpha):
+        sc = oracle.awq_candidate_scales(a, alpha)
+        q = oracle.rtn(W * sc, 4, g)
+        Q = oracle.dequantize(q["codes"], q["scales"], q["zeros"], g) / sc
+        return (2.0 / n) * float(np.sum(((W - Q) @ X64.T) ** 2))
+
+    rt = oracle.rtn(W, 4, g)
+    Q0 = oracle.dequantize(rt["codes"], rt["scales"], rt["zeros"], g)
+    l0 = (2.0 / n) * float(np.sum(((W - Q0) @ X64.T) ** 2))
+    assert abs(r["losses"][0] - l0) <= 1e-9 * l0
+    for k in (3, 7, 9):
+        lk = through_x(r["alphas"][k])
+        assert abs(r["losses"][k] - lk) <= 1e-9 * lk
+    assert r["alpha"] == r["alphas"][int(np.argmin(r["losses"]))]
+    assert r["losses"].min() <= r["losses"][0]
+    # two channels with 40x activations: protecting them pays off here
+    assert r["alpha"] > 0 and r["losses"].min() < r["losses"][0]
+    # X -> 4 X: S -> 16 S, a -> 4 a; the scales and choice are unchanged, the
+    # losses x16 (up to the summation order of the oracle's threaded trace)
+    r2 = oracle.awq_search(W, 16.0 * S, n, 4.0 * a, 4, g, n_grid=10)
+    assert r2["alpha"] == r["alpha"]
+    assert np.allclose(r2["losses"], 16.0 * r["losses"], rtol=1e-12, atol=0)
+
+
+def test_awq_then_gptq_pins():
+    """GPTQ after the scaling works on W' = W diag(s) and S' = diag(s)^-1 S
+    diag(s)^-1: with one candidate (alpha = 0, s = 1) it is plain GPTQ, and
+    the loss of the layer mapped back, Q' diag(s)^-1, against the original
+    H equals the loss in the scaled coordinates."""
+    rng = _rng(37)
+    n, m, d, g = 500, 24, 128, 32
+    X = rng.standard_normal((n, d))
+    X[:, [9]] *= 30.0
+    X = X.astype(np.float16)
+    W = 0.02 * rng.standard_normal((m, d))
+    S = oracle.hessian(X)
+    a = oracle.channel_magnitude(X)
+    one = oracle.awq_then_gptq(W, S, n, a, 4, g, n_grid=1)
+    ref = oracle.gptq_layer(W, S, n, 4, g)
+    assert np.all(one["s"] == 1.0) and np.array_equal(one["codes"], ref["codes"])
+    res = oracle.awq_then_gptq(W, S, n, a, 4, g, n_grid=10)
+    s = res["s"]
+    Qp = oracle.dequantize(res["codes"], res["scales"], res["zeros"], g, res["perm"])
+    H = 2.0 * S / n
+    l_orig = oracle.layer_loss(W, Qp / s[None, :], H)
+    l_scaled = oracle.layer_loss(W * s[None, :], Qp, H / np.outer(s, s))
+    assert abs(l_orig - l_scaled) <= 1e-10 * l_orig
+
+
 def test_loss_closed_form_identity():
     # sum_j (e_j/U_jj)^2 = tr(D Hd D^T) = (2/n)||D X^T||^2 + lam ||D||^2, and
     # D = E U (the accumulated corrections): exact for any quantizer decisions.
