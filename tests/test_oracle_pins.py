@@ -269,6 +269,50 @@ def test_upper_chol_of_inverse_properties():
     assert np.allclose(U, np.diag(1 / np.sqrt(h)), rtol=1e-15, atol=0)
 
 
+def _kms_u(d, rho):
+    """Closed form for H = KMS(rho), H_ij = rho^|i-j|: chol(H) = L with
+    L[i][0] = rho^i and L[i][j] = rho^(i-j) sqrt(1 - rho^2) (j >= 1), so L^-1
+    is lower bidiagonal (1, then 1/c on the diagonal and -rho/c below it,
+    c = sqrt(1 - rho^2)); H is persymmetric (J H J = H), so the upper factor
+    of H^-1 is U = J L^-1 J: upper bidiagonal, U_ii = 1/c except U_{d-1,d-1}
+    = 1, and U_{i,i+1} = -rho/c."""
+    c = np.sqrt(1.0 - rho * rho)
+    U = np.zeros((d, d))
+    U[np.arange(d - 1), np.arange(d - 1)] = 1.0 / c
+    U[d - 1, d - 1] = 1.0
+    U[np.arange(d - 1), np.arange(1, d)] = -rho / c
+    return U
+
+
+def test_upper_chol_of_inverse_kms_closed_form():
+    """U for a Kac-Murdock-Szego matrix at d = 256 against its closed form
+    (every entry, the zeros beyond the first superdiagonal included); and
+    the sweep with that U against a scalar recursion in which each column's
+    error reaches the next column only (U[j][j+1], row j of U, not column j)."""
+    d, rho, g = 256, 0.7, 64
+    i = np.arange(d)
+    H = rho ** np.abs(i[:, None] - i[None, :])
+    U, info = oracle.hinv_upper_chol(H)
+    assert info == 0
+    assert np.abs(U - _kms_u(d, rho)).max() <= 1e-12
+    rng = _rng(41)
+    W = 0.02 * rng.standard_normal((5, d))
+    r = oracle.quantize_rows(W, U, 4, g)
+    for row in range(W.shape[0]):
+        w = W[row].copy()
+        for j in range(d):
+            if j % g == 0:                       # parameters from the values as they stand
+                p = oracle.rtn(w[None, j:j + g], 4, g)
+                s = float(p["scales"].view(np.float16)[0, 0])
+                z = int(p["zeros"][0, 0])
+            x = np.float32(w[j])
+            c = int(min(max(np.rint(np.float32(x / np.float32(s))) + z, 0), 15))
+            assert c == r["codes"][row, j], (row, j)
+            E = (w[j] - s * (c - z)) / U[j, j]
+            if j + 1 < d:
+                w[j + 1] -= E * U[j, j + 1]
+
+
 # --------------------------------------------------------------------------
 # The sweep
 # --------------------------------------------------------------------------

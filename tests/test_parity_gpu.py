@@ -180,6 +180,58 @@ def test_prepare_parity(act_order, d):
     assert P.rel_fro(Ug, U64) <= P.U_TOL
 
 
+def test_prepare_kms_closed_form():
+    """The GPU's U for H = KMS(0.7) (H_ij = 0.7^|i-j|, no damping) against
+    its closed form, an upper bidiagonal matrix (every entry checked, the
+    zeros included): no oracle involved."""
+    d, n, rho = 512, 1000, 0.7
+    i = np.arange(d)
+    H = rho ** np.abs(i[:, None] - i[None, :])
+    S = torch.from_numpy((n / 2.0) * H).float().to(DEV)
+    perm, U, info = G.gptq_prepare_hinv(S, n, 0.0, False)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    c = np.sqrt(1.0 - rho * rho)
+    ref = np.zeros((d, d))
+    ref[i[:-1], i[:-1]] = 1.0 / c
+    ref[d - 1, d - 1] = 1.0
+    ref[i[:-1], i[1:]] = -rho / c
+    Ug = P.to_np(U).astype(np.float64)
+    assert np.abs(Ug - ref).max() <= 1e-5 * np.abs(ref).max()
+    assert np.array_equal(P.to_np(perm), np.arange(d, dtype=np.int32))
+
+
+def test_gptq_equals_rtn_when_hessian_is_isotropic():
+    """X of Hadamard rows: X^T X = n I exactly (integer sums), so U is diagonal
+    and the error feedback vanishes; the GPU's GPTQ must then give the GPU's
+    and the oracle's round-to-nearest codes, scales and zero points bit for
+    bit, with and without act-order (equal diagonal: identity order)."""
+    d, reps = 256, 2
+    Hd_ = np.array([[1.0]])
+    while Hd_.shape[0] < d:
+        Hd_ = np.block([[Hd_, Hd_], [Hd_, -Hd_]])
+    X = torch.from_numpy(np.vstack([Hd_] * reps).astype(np.float16)).to(DEV)
+    n = X.shape[0]
+    W = _weights(96, d, torch.float16, 43).to(DEV)
+    S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    G.gptq_hessian_accumulate(S, X)
+    Sg = P.to_np(S)
+    assert np.array_equal(np.triu(Sg), n * np.eye(d, dtype=np.float32))
+    rc, rs, rz = G.rtn_quantize(W, 4, 128)
+    ref = oracle.rtn(W.double().cpu().numpy(), 4, 128)
+    assert np.array_equal(P.to_np(rc), ref["codes"])
+    for act in (False, True):
+        perm, U, info = G.gptq_prepare_hinv(S, n, 0.01, act)
+        c, sc, z, _ = G.gptq_quantize_layer(W, U, perm if act else None, 4, 128)
+        torch.cuda.synchronize()
+        assert int(info.item()) == 0
+        Ug = P.to_np(U)
+        assert np.array_equal(Ug, np.diag(np.diag(Ug)))
+        assert np.array_equal(P.to_np(perm), np.arange(d, dtype=np.int32))
+        assert np.array_equal(P.to_np(c), P.to_np(rc))
+        assert np.array_equal(P.to_np(sc), P.to_np(rs)) and np.array_equal(P.to_np(z), P.to_np(rz))
+
+
 def test_prepare_reports_non_pd():
     d = 256
     S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
