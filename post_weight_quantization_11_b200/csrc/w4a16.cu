@@ -71,16 +71,10 @@ w4a16_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight,
 #pragma unroll
         for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
 
-    for (int c = lane; c < nch; c += 32) {
+    // one chunk of 16 codes for the warp's rows, packed words already loaded
+    auto chunk = [&](int c, const uint2 (&q)[W4_ROWS]) {
         const int64_t gc = k0 / W4_CHUNK + c;                   // chunk index in the row
         const int64_t gi = gc * W4_CHUNK / g;                   // its group
-        uint2 q[W4_ROWS];
-#pragma unroll
-        for (int r = 0; r < W4_ROWS; ++r) {
-            const int64_t row = row0 + r;
-            q[r] = row < m ? *reinterpret_cast<const uint2*>(qweight + row * (d / 8) + 2 * gc)
-                           : make_uint2(0u, 0u);
-        }
         float xv[B][W4_CHUNK];
 #pragma unroll
         for (int b = 0; b < B; ++b)
@@ -117,6 +111,25 @@ w4a16_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight,
 #pragma unroll
             for (int b = 0; b < B; ++b) acc[r][b] = fmaf(s, fmaf(-z, xsum[b][c], a[b]), acc[r][b]);
         }
+    };
+    auto load = [&](int c, uint2 (&q)[W4_ROWS]) {
+        const int64_t gc = k0 / W4_CHUNK + c;
+#pragma unroll
+        for (int r = 0; r < W4_ROWS; ++r) {
+            const int64_t row = row0 + r;
+            q[r] = row < m ? *reinterpret_cast<const uint2*>(qweight + row * (d / 8) + 2 * gc)
+                           : make_uint2(0u, 0u);
+        }
+    };
+    // two chunks per step, both chunks' words requested before either is used,
+    // so each warp keeps 2 KB of weight loads in flight
+    for (int c = lane; c < nch; c += 64) {
+        uint2 q0[W4_ROWS], q1[W4_ROWS];
+        const bool two = c + 32 < nch;
+        load(c, q0);
+        if (two) load(c + 32, q1);
+        chunk(c, q0);
+        if (two) chunk(c + 32, q1);
     }
 #pragma unroll
     for (int r = 0; r < W4_ROWS; ++r)
