@@ -177,12 +177,14 @@ class HostHessian:
         # torch creates an event's CUDA handle at its first record
         self.ev_filled.record(self.copy_stream)
         self.ev_freed.record(self.copy_stream)
+        self._inflight = []          # (event, host tensor) until that tensor's copies are done
 
     def accumulate(self, S: torch.Tensor, X_host: torch.Tensor) -> int:
         """S (d x d fp32 on the device, upper triangle) += X^T X for X_host
         (n x d fp16, CPU, contiguous; pinned for the copies to overlap).
-        Asynchronous on the current stream; keep X_host alive and unchanged
-        until that stream has passed this call.  Returns n."""
+        Asynchronous on the current stream.  The streamer keeps a reference to
+        X_host until its copies have completed; do not modify it before then.
+        Returns n."""
         _need(S, "S", torch.float32)
         if not isinstance(X_host, torch.Tensor) or X_host.is_cuda:
             raise ValueError("X_host must be a CPU tensor")
@@ -199,6 +201,10 @@ class HostHessian:
                    ctypes.c_void_p(self.copy_stream.cuda_stream),
                    ctypes.c_void_p(self.ev_filled.cuda_event),
                    ctypes.c_void_p(self.ev_freed.cuda_event)))
+        done = torch.cuda.Event()
+        done.record(self.copy_stream)        # after this call's last copy
+        self._inflight = [(e, t) for e, t in self._inflight if not e.query()]
+        self._inflight.append((done, X_host))
         return n
 
 
