@@ -52,6 +52,9 @@ def _args():
                    help="overlap each layer's preparation with the next layer's Hessian on two "
                         "streams, the Hessian on at most H CTAs and the factorization on at "
                         "most P (e.g. 116,32)")
+    p.add_argument("--w4a16", type=int, default=0, metavar="BATCH",
+                   help="time the W4A16 product of packed layers shaped like the workload's "
+                        "instead of the quantization step (batch 1-4 activation rows)")
     p.add_argument("--shard", choices=["layers", "layer"], default="layers",
                    help="layers: every rank quantizes its own layer (weak scaling); layer: one "
                         "layer over all ranks, tokens and rows split, S summed by one "
@@ -695,12 +698,72 @@ def run_ours_pipelined(a):
         dist.destroy_process_group()
 
 
+def run_w4a16(a):
+    """The W4A16 product y = x Q^T of packed INT4 layers (batch a.w4a16 rows
+    of fp16 activations).  Enough distinct layers rotate through the timed
+    loop that their packed bytes exceed L2, so every launch streams its
+    weights from HBM; the roofline is HBM bytes (packed weights, scales, zero
+    points, activations, outputs) per launch over its CUDA-event time."""
+    ws, rank, local = _dist_init()
+    from post_weight_quantization_11_b200 import gptq as G
+    G.load_library()
+    dev = torch.device("cuda", local)
+    wl, spec, n = _workload(a.workload, a.layer, a.tokens)
+    m, d, b, g = spec.d_out, spec.d_in, a.w4a16, 128
+    ng = d // g
+    per_layer = m * d // 2 + m * ng * 2 + m * ((ng + 1) // 2)
+    L = max(2, int(4 * 126e6 // per_layer) + 1)
+    gen = torch.Generator(device=dev).manual_seed(5)
+    layers = []
+    for _ in range(L):
+        qw = torch.randint(-2**31, 2**31 - 1, (m, d // 8), generator=gen, device=dev,
+                           dtype=torch.int32)
+        sc = (torch.rand(m, ng, generator=gen, device=dev) * 0.05 + 1e-3).half()
+        qz = torch.randint(0, 256, (m, (ng + 1) // 2), generator=gen, device=dev,
+                           dtype=torch.uint8)
+        layers.append((qw, sc, qz))
+    x = torch.randn(b, d, generator=gen, device=dev).half()
+    y = torch.empty(b, m, dtype=torch.float32, device=dev)
+    for i in range(max(3, a.warmup) * L):
+        qw, sc, qz = layers[i % L]
+        G.gptq_w4a16_gemm(x, qw, sc, qz, g, None, y)
+    torch.cuda.synchronize()
+    reps = max(a.steps, 1) * L
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    with ClockSampler(local) as clk:
+        start.record()
+        for i in range(reps):
+            qw, sc, qz = layers[i % L]
+            G.gptq_w4a16_gemm(x, qw, sc, qz, g, None, y)
+        end.record()
+        torch.cuda.synchronize()
+    us = _max_over_ranks(start.elapsed_time(end) * 1e3 / reps, ws)
+    peaks, src = _peaks()
+    bytes_ = per_layer + b * d * 2 + b * m * 4
+    gbs = bytes_ / (us * 1e-6) / 1e9
+    line = {"metric": "W4A16 product weights/s", "value": ws * m * d / (us * 1e-6),
+            "unit": "weights/s", "n_gpus": ws, "steps": a.steps, "warmup": a.warmup,
+            "us_per_launch": us, "higher_is_better": True, "scaling": "weak", "dtype": "f32",
+            "data": "synthetic packed layers", "vs_baseline": None,
+            "config": {"workload": f"{spec.name} ({a.workload}) packed: W {m}x{d} INT4 g{g}, "
+                                   f"batch {b}", "layers_rotated": L},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks.get("hbm_gbs"),
+                         "unit": "GB/s", "frac": gbs / peaks.get("hbm_gbs"),
+                         "bytes_per_launch": bytes_, "peak_source": f"hbm_gbs of {src}"},
+            "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     a = _args()
     if a.impl == "reference":
         run_reference(a)
     elif a.pipeline:
         run_ours_pipelined(a)
+    elif a.w4a16:
+        run_w4a16(a)
     elif a.shard == "layer":
         run_ours_one_layer(a)
     else:

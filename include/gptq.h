@@ -249,6 +249,24 @@ int gptq_unpack_int4(const uint32_t* qweight, const uint8_t* qzeros, int64_t d_o
                      void* stream);
 
 /*
+ * Weight-only INT4 product on the packed layer (W4A16) -- "INT4/INT8 量化推理"
+ * sec. 六 (weights in 4 bits, activations in fp16), on the storage of sec. 一
+ * of the same page:
+ *   y[b][r] = sum_j x[b][j] Q[r][j],  Q[r][perm[k]] = s[r][k/g] (c[r][k] - z[r][k/g])
+ * with c, z unpacked from qweight / qzeros (gptq_pack_int4's layout, codes in
+ * sweep order) and s the fp16 scales.  Products and sums are fp32; the
+ * dequantized weights are exact.
+ * x: batch x d_in fp16 (original column order); y: batch x d_out fp32 output
+ * (overwritten).  perm: d_in int32 or NULL (identity), as gptq_prepare_hinv
+ * returned it.  group_size: a multiple of 32 dividing d_in, or -1 (one group
+ * per row).  batch in 1..4 (decode-sized; larger batches are UNSUPPORTED).
+ * Requires d_in % 128 == 0, 128 <= d_in <= 32768, 1 <= d_out <= 2^24.
+ */
+int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t* qweight,
+                    const uint16_t* scales, const uint8_t* qzeros, const int32_t* perm,
+                    int64_t d_out, int64_t d_in, int group_size, float* y, void* stream);
+
+/*
  * Round-to-nearest baseline -- "大模型量化实战（上）" (RTN: every weight
  * rounded on its own) with the min-max group quantizer of "校准艺术" sec. 2.1:
  * the same group parameters and codes as gptq_quantize_layer, taken on the

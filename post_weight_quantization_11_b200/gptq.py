@@ -32,7 +32,7 @@ EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_quantize_layer_static",
             "gptq_pack_int4",
-            "gptq_unpack_int4", "rtn_quantize", "gptq_debug_gemm_nt",
+            "gptq_unpack_int4", "gptq_w4a16_gemm", "rtn_quantize", "gptq_debug_gemm_nt",
             "gptq_debug_chol_task_order", "gptq_debug_div_rn", "gptq_debug_bounded_wait")
 
 
@@ -75,6 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_pack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "gptq_unpack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "rtn_quantize": ([P, I32, I64, I64, I32, I32, P, P, P, P], I32),
+        "gptq_w4a16_gemm": ([P, I64, P, P, P, P, I64, I64, I32, P, P], I32),
         "gptq_debug_gemm_nt": ([P, I64, P, I64, P, I64, I64, I64, I64, F32, F32, I32, P], I32),
         "gptq_debug_chol_task_order": ([I64, P, I64], I64),
         "gptq_debug_div_rn": ([P, P, I64, P], I32),
@@ -305,6 +306,26 @@ def gptq_pack_int4(codes: torch.Tensor, zeros: torch.Tensor, qweight=None, qzero
            load_library().gptq_pack_int4(_ptr(codes), _ptr(zeros), m, d, G, _ptr(qweight),
                                          _ptr(qzeros), _stream(codes)))
     return qweight, qzeros
+
+
+def gptq_w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                    qzeros: torch.Tensor, group_size: int = 128, perm=None, y=None):
+    """y = x Q^T (batch x d_out fp32) from the packed INT4 layer; x: batch x
+    d_in fp16 in original column order, batch 1..4."""
+    _need(x, "x", torch.float16)
+    _need(qweight, "qweight")
+    _need(scales, "scales", torch.float16)
+    _need(qzeros, "qzeros", torch.uint8)
+    b, d = x.shape
+    m = qweight.shape[0]
+    y = torch.empty(b, m, dtype=torch.float32, device=x.device) if y is None else y
+    _need(y, "y", torch.float32)
+    if perm is not None:
+        _need(perm, "perm", torch.int32)
+    _check("gptq_w4a16_gemm",
+           load_library().gptq_w4a16_gemm(_ptr(x), b, _ptr(qweight), _ptr(scales), _ptr(qzeros),
+                                          _ptr(perm), m, d, int(group_size), _ptr(y), _stream(x)))
+    return y
 
 
 def gptq_unpack_int4(qweight: torch.Tensor, qzeros: torch.Tensor, d_in: int, n_groups: int):

@@ -142,6 +142,15 @@ def test_validation_rejects_before_launch(lib):
     assert qs(bits=5) == 4 and qs(d=200) == 2 and qs(W=None) == 1
     assert lib.rtn_quantize(FAKE, 1, 64, 256, 3, 48, FAKE, FAKE, FAKE, None) == 4
     assert lib.rtn_quantize(None, 1, 64, 256, 4, 128, FAKE, FAKE, FAKE, None) == 1
+    W4 = lib.gptq_w4a16_gemm
+    assert W4(None, 1, FAKE, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 1
+    assert W4(FAKE, 1, MIS, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 1
+    assert W4(FAKE, 5, FAKE, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 4
+    assert W4(FAKE, 0, FAKE, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 4
+    assert W4(FAKE, 1, FAKE, FAKE, FAKE, None, 64, 200, 128, FAKE, None) == 2
+    assert W4(FAKE, 1, FAKE, FAKE, FAKE, None, 0, 256, 128, FAKE, None) == 2
+    assert W4(FAKE, 1, FAKE, FAKE, FAKE, None, 64, 256, 48, FAKE, None) == 4
+    assert W4(FAKE, 1, FAKE, FAKE, FAKE, None, 64, 384, 256, FAKE, None) == 4
     assert lib.gptq_pack_int4(FAKE, FAKE, 4, 12, 1, FAKE, FAKE, None) == 2
     assert lib.gptq_pack_int4(FAKE, FAKE, 4, 16, 0, FAKE, FAKE, None) == 2
     assert lib.gptq_unpack_int4(FAKE, FAKE, 0, 16, 1, FAKE, FAKE, None) == 2
