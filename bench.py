@@ -48,6 +48,8 @@ def _args():
     p.add_argument("--tokens", type=int, default=0, help="override token count (0: workload's)")
     p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the per-config summary (every workload of the pages' shapes)")
     p.add_argument("--pipeline", default="", metavar="H,P",
                    help="overlap each layer's preparation with the next layer's Hessian on two "
                         "streams, the Hessian on at most H CTAs and the factorization on at "
@@ -262,6 +264,297 @@ class Layer:
             ev[4].record()
 
 
+class MoeLayer:
+    """The mixture-of-experts layer (all experts at once) through the
+    batched entry points: routed rows gathered expert-major, one grouped
+    Hessian launch, one factorization launch for every expert, the batched
+    sweep, one pack of the stacked codes."""
+
+    def __init__(self, wl, dev, seed_offset=0):
+        from post_weight_quantization_11_b200 import gptq as G
+        from post_weight_quantization_11_b200 import inputs
+        self.G = G
+        spec0 = wl.layers[0]
+        self.E = wl.n_experts
+        self.m, self.d = spec0.d_out, spec0.d_in
+        self.act_order = spec0.act_order
+        E, m, d = self.E, self.m, self.d
+        self.W = torch.stack([inputs.weights(sp, device=dev, seed_offset=seed_offset)
+                              for sp in wl.layers]).contiguous()
+        self.X = inputs.calibration_x(spec0, device=dev)
+        lists = inputs.moe_routing(self.X.shape[0], wl.n_experts, wl.zipf_s, wl.top_k,
+                                   wl.cold_cap, spec0.seed)
+        self.counts = [len(x) for x in lists]
+        self.offsets = np.concatenate([[0], np.cumsum(self.counts)]).astype(np.int64)
+        self.idx = torch.as_tensor(np.concatenate(lists), dtype=torch.int32, device=dev)
+        self.n = int(self.offsets[-1])               # routed rows (token-expert pairs)
+        self.Xr = torch.empty(self.n, d, dtype=torch.float16, device=dev)
+        self.S = torch.zeros(E, d, d, dtype=torch.float32, device=dev)
+        self.perm = torch.empty(E, d, dtype=torch.int32, device=dev)
+        self.U = torch.empty(E, d, d, dtype=torch.float32, device=dev)
+        self.info = torch.zeros(E, dtype=torch.int32, device=dev)
+        self.ws_p = torch.empty(G.gptq_prepare_batched_workspace_bytes(d, E), dtype=torch.uint8,
+                                device=dev)
+        self.ws_q = torch.empty(G.gptq_quantize_workspace_bytes(m, d, 128), dtype=torch.uint8,
+                                device=dev)
+        self.codes = torch.empty(E, m, d, dtype=torch.uint8, device=dev)
+        self.scales = torch.empty(E, m, d // 128, dtype=torch.float16, device=dev)
+        self.zeros = torch.empty(E, m, d // 128, dtype=torch.uint8, device=dev)
+        self.loss = torch.empty(E, m, dtype=torch.float32, device=dev)
+        self.qweight = torch.empty(E * m, d // 8, dtype=torch.int32, device=dev)
+        self.qzeros = torch.empty(E * m, (d // 128 + 1) // 2, dtype=torch.uint8, device=dev)
+
+    def step(self, ev=None):
+        G = self.G
+        self.S.zero_()
+        if ev is not None:
+            ev[0].record()
+        G.gptq_gather_rows(self.X, self.idx, self.Xr)
+        G.gptq_hessian_accumulate_grouped(self.S, self.Xr, self.offsets)
+        if ev is not None:
+            ev[1].record()
+        self.after_hessian(ev)
+
+    def after_hessian(self, ev=None):
+        G = self.G
+        G.gptq_prepare_hinv_batched(self.S, self.counts, 0.01, self.act_order, self.perm, self.U,
+                                    self.info, self.ws_p)
+        if ev is not None:
+            ev[2].record()
+        G.gptq_quantize_layer_batched(self.W, self.U, self.perm if self.act_order else None, 4,
+                                      128, 128, self.codes, self.scales, self.zeros, self.loss,
+                                      self.ws_q)
+        if ev is not None:
+            ev[3].record()
+        G.gptq_pack_int4(self.codes.view(self.E * self.m, self.d),
+                         self.zeros.view(self.E * self.m, -1), self.qweight, self.qzeros)
+        if ev is not None:
+            ev[4].record()
+
+
+def _make_layer(workload: str, layer: int, tokens: int, dev, seed_offset=0):
+    """(layer object, description dict) for a workload of inputs.WORKLOADS."""
+    from post_weight_quantization_11_b200 import inputs
+    wl = inputs.WORKLOADS[workload]
+    if getattr(wl, "n_experts", 0):
+        lay = MoeLayer(wl, dev, seed_offset)
+        lay.mats, lay.tokens = lay.E, lay.counts
+        desc = (f"{wl.layers[0].name} ({workload}): {lay.E} experts x W {lay.m}x{lay.d} fp16, "
+                f"X {lay.X.shape[0]}x{lay.d} fp16, top-{wl.top_k} routed ({lay.n} rows, "
+                f"{min(lay.counts)}..{max(lay.counts)} per expert), INT4 g128, damp 0.01, "
+                f"batched")
+        return lay, desc
+    spec = wl.layers[layer]
+    n = tokens or spec.n_tokens
+    lay = Layer(spec, n, dev, seed_offset=seed_offset)
+    lay.mats, lay.tokens = 1, [n]
+    desc = (f"{spec.name} ({workload}): W {lay.m}x{lay.d} fp16, X {n}x{lay.d} fp16, INT4 g128, "
+            f"damp 0.01, act_order={spec.act_order}")
+    return lay, desc
+
+
+def _update_flops(m: int, d: int, B: int = 128, outer: int = 4) -> float:
+    """Algorithmic flops of the lazy-batch feedback onto later blocks, as the
+    library schedules it: after each block of B columns the rest of its
+    outer block of outer*B columns (K = B), and after each outer block every
+    column beyond it (K = outer*B); 2 m K N per product."""
+    f = 0.0
+    ob = outer * B
+    for j0 in range(0, d, B):
+        o0 = j0 // ob * ob
+        o1 = min(d, o0 + ob)
+        if j0 + B < o1:
+            f += 2.0 * m * B * (o1 - j0 - B)
+        if j0 + B == o1 and o1 < d:
+            f += 2.0 * m * (o1 - o0) * (d - o1)
+    return f
+
+
+def _tf32_peak(peaks) -> float:
+    """TF32 dense peak from the measured bf16 burst peak and the nominal
+    TF32 : bf16 ratio (1.1 : 2.25 PFLOP/s)."""
+    return float(peaks["bf16_tflops"]) * (1.1 / 2.25)
+
+
+def _phase_bounds(lay, peaks) -> dict:
+    """Lower bounds (ms) of each phase at the measured burst peaks: the
+    Hessian at the bf16 rate (fp16 runs at it) or its HBM bytes, whichever
+    is larger; the factorization's and the updates' split-TF32 tensor flops
+    (three MMAs per product) at the TF32 peak; the sweep's and pack's HBM
+    bytes."""
+    m, d, E = lay.m, lay.d, lay.mats
+    hbm = float(peaks["hbm_gbs"]) * 1e9
+    bf16 = float(peaks["bf16_tflops"]) * 1e12
+    tf32 = _tf32_peak(peaks) * 1e12
+    ntok = float(sum(lay.tokens))
+    gather = 2.0 * ntok * d * 2 if E > 1 else 0.0
+    hess = max(ntok * d * d / bf16, (2.0 * ntok * d + gather) / hbm)
+    fact = E * 3 * (2.0 / 3.0) * d ** 3 / tf32
+    upd = E * 3 * _update_flops(m, d) / tf32
+    sweep_b = E * (13.0 * m * d + 4.0 * d * d)
+    pack_b = E * 1.53 * m * d
+    return {"hessian": hess * 1e3, "prepare": fact * 1e3, "quantize": (upd + sweep_b / hbm) * 1e3,
+            "pack": pack_b / hbm * 1e3}
+
+
+def _kernel_entries(lay, peaks, times: dict, steps: int) -> dict:
+    """Per-kernel roofline entries from the library's per-kind event timing
+    (ms per step = summed kernel time / steps)."""
+    m, d, E = lay.m, lay.d, lay.mats
+    hbm = float(peaks["hbm_gbs"])
+    bf16 = float(peaks["bf16_tflops"])
+    tf32 = _tf32_peak(peaks)
+    ntok = float(sum(lay.tokens))
+
+    def t(kind):
+        v = times.get(kind)
+        return (v[0] / steps, v[1] // steps) if v else (None, 0)
+
+    out = {}
+    ms, nl = t("hessian")
+    if ms:
+        a = ntok * d * d / (ms * 1e-3) / 1e12
+        out["hessian"] = {"bound": "tensor", "ms": ms, "launches": nl, "achieved": a,
+                          "peak": bf16, "unit": "TFLOP/s", "frac": a / bf16,
+                          "work": "n d^2 flops (fp16 in, fp32 accumulate)"}
+    ms, nl = t("factorization")
+    if ms:
+        a = E * 3 * (2.0 / 3.0) * d ** 3 / (ms * 1e-3) / 1e12
+        out["factorization"] = {"bound": "tensor", "ms": ms, "launches": nl, "achieved": a,
+                                "peak": tf32, "unit": "TFLOP/s", "frac": a / tf32,
+                                "work": "3 x (d^3/3 factor + d^3/3 inverse) split-TF32 flops "
+                                        "per matrix; a latency chain of d/128 diagonal tiles"}
+    un, nn = t("update_near")
+    uf, nf = t("update_far")
+    if un or uf:
+        ms = (un or 0.0) + (uf or 0.0)
+        a = E * 3 * _update_flops(m, d) / (ms * 1e-3) / 1e12
+        out["update"] = {"bound": "tensor", "ms": ms, "launches": nn + nf, "achieved": a,
+                         "peak": tf32, "unit": "TFLOP/s", "frac": a / tf32,
+                         "near_ms": un, "far_ms": uf,
+                         "work": "3 x sum of 2 m K N split-TF32 flops of the lazy-batch "
+                                 "schedule (K = 128 near, 512 far)"}
+    ms, nl = t("sweep")
+    if ms:
+        b = E * (13.0 * m * d + 4.0 * d * d)
+        a = b / (ms * 1e-3) / 1e9
+        out["sweep"] = {"bound": "hbm", "ms": ms, "launches": nl, "achieved": a, "peak": hbm,
+                        "unit": "GB/s", "frac": a / hbm,
+                        "work": "W fp32 in (4 B), codes (1 B) and E split (8 B) out per weight, "
+                                "U diagonal blocks in; issue-bound in practice"}
+    ms, nl = t("pack")
+    if ms:
+        b = E * 1.53 * m * d
+        a = b / (ms * 1e-3) / 1e9
+        out["pack"] = {"bound": "hbm", "ms": ms, "launches": nl, "achieved": a, "peak": hbm,
+                       "unit": "GB/s", "frac": a / hbm,
+                       "work": "codes in (1 B per weight), packed nibbles out (0.5 B), zero "
+                               "points and their packing (0.03 B)"}
+    ms, nl = t("gather")
+    if ms:
+        b = 2.0 * ntok * d * 2
+        a = b / (ms * 1e-3) / 1e9
+        out["gather"] = {"bound": "hbm", "ms": ms, "launches": nl, "achieved": a, "peak": hbm,
+                         "unit": "GB/s", "frac": a / hbm, "work": "routed rows read and written"}
+    for k in ("finalize", "init_work", "split_u"):
+        ms, nl = t(k)
+        if ms:
+            out[k] = {"ms": ms, "launches": nl}
+    return out
+
+
+def _time_layer(lay, steps: int, warmup: int, eager: bool = False):
+    """(ms per step, launches per step, graph or None): the step captured
+    once as a CUDA graph and replayed between CUDA events (the library's
+    calls never synchronize or allocate, so they capture)."""
+    G = lay.G
+    c0 = G.gptq_debug_launch_count()
+    lay.step()
+    per_step = G.gptq_debug_launch_count() - c0
+    torch.cuda.synchronize()
+    graph = None
+    if not eager:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            lay.step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            lay.step()
+        torch.cuda.synchronize()
+        for _ in range(max(3, warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        if graph is not None:
+            graph.replay()
+        else:
+            lay.step()
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps, per_step, graph
+
+
+def _phase_split(lay, reps: int = 3) -> dict:
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps)]
+    for e in evs:
+        lay.step(e)
+    torch.cuda.synchronize()
+    return {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in evs)
+            for k, name in enumerate(("hessian", "prepare", "quantize", "pack"))}
+
+
+def _kernel_times(lay, reps: int = 2) -> dict:
+    G = lay.G
+    G.gptq_debug_kernel_times()                  # drop older records
+    G.gptq_debug_kernel_timing(True)
+    try:
+        for _ in range(reps):
+            lay.step()
+        torch.cuda.synchronize()
+    finally:
+        G.gptq_debug_kernel_timing(False)
+    return G.gptq_debug_kernel_times()
+
+
+CONFIGS = (("tiny", 0), ("attn7b", 0), ("mlp7b", 0), ("mlp7b", 1), ("mlp8b_act", 0),
+           ("mlp8b_act", 1), ("moe8", 0))
+
+
+def _configs_summary(dev, peaks, steps: int, warmup: int, skip=None) -> dict:
+    """Every workload of the pages' shapes, each timed the way the headline
+    is (graph replay, inputs resident): ms per layer, weights/s, the phase
+    split and the whole-layer fraction of its roofline (the sum of the
+    phase bounds at the measured peaks over the measured step)."""
+    out = {}
+    for wname, li in CONFIGS:
+        key = f"{wname}/{li}" if wname not in ("tiny", "moe8") else wname
+        if skip == (wname, li):
+            continue
+        lay, desc = _make_layer(wname, li, 0, dev)
+        for _ in range(max(3, warmup)):
+            lay.step()
+        torch.cuda.synchronize()
+        ok = not bool(lay.info.any().item())
+        k = max(steps, 200) if wname == "tiny" else steps
+        ms, launches, graph = _time_layer(lay, k, warmup)
+        phase = _phase_split(lay, 2)
+        bounds = _phase_bounds(lay, peaks)
+        units = lay.mats * lay.m * lay.d
+        out[key] = {"workload": desc, "ms_per_layer": ms, "weights_per_s": units / (ms * 1e-3),
+                    "steps": k, "launches_per_step": launches, "phase_ms": phase,
+                    "phase_bound_ms": bounds, "whole_layer_frac": sum(bounds.values()) / ms,
+                    "info_ok": ok}
+        del graph, lay
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
 def _cpu_baseline(spec, n, reps=1):
     """The float64 oracle, as it stands, on a bounded sample of the workload:
     S over n_s tokens, the full d x d preparation, the sweep and packing of m_s
@@ -298,114 +591,59 @@ def run_ours(a):
     from post_weight_quantization_11_b200 import gptq as G
     G.load_library()
     dev = torch.device("cuda", local)
-    wl, spec, n = _workload(a.workload, a.layer, a.tokens)
-    lay = Layer(spec, n, dev, seed_offset=rank)
-    m, d = lay.m, lay.d
+    lay, desc = _make_layer(a.workload, a.layer, a.tokens, dev, seed_offset=rank)
+    m, d, E = lay.m, lay.d, lay.mats
+    units = E * m * d
     torch.cuda.synchronize()
     for _ in range(max(3, a.warmup)):
         lay.step()
     torch.cuda.synchronize()
-    assert int(lay.info.item()) == 0, "non-positive pivot in the workload"
-    c0 = G.gptq_debug_launch_count()
-    lay.step()
-    graph_launches = G.gptq_debug_launch_count() - c0
-    torch.cuda.synchronize()
+    assert not bool(lay.info.any().item()), "non-positive pivot in the workload"
 
     # per-phase split (eager launches, CUDA events between the ABI calls)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(3)]
-    for e in evs:
-        lay.step(e)
-    torch.cuda.synchronize()
-    phase = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in evs)
-             for k, name in enumerate(("hessian", "prepare", "quantize", "pack"))}
+    phase = _phase_split(lay, 3)
 
     # the timed region: the step captured once as a CUDA graph and replayed
-    # (the library's calls never synchronize or allocate, so they capture)
-    graph = None
-    if not a.eager:
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            lay.step()
-        torch.cuda.current_stream().wait_stream(side)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            lay.step()
-        torch.cuda.synchronize()
-        for _ in range(max(3, a.warmup)):
-            graph.replay()
-        torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = G.gptq_debug_launch_count()
     _barrier(ws)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        start.record()
-        for i in range(a.steps):
-            if graph is not None:
-                graph.replay()
-            else:
-                lay.step()
-        end.record()
-        torch.cuda.synchronize()
+        ms, graph_launches, graph = _time_layer(lay, a.steps, a.warmup, a.eager)
     _barrier(ws)
-    launches = G.gptq_debug_launch_count() - launches0
-    if graph is not None:
-        launches = graph_launches * a.steps
-    ms = start.elapsed_time(end) / a.steps
+    launches = graph_launches * a.steps
     ms = _max_over_ranks(ms, ws)
-    assert int(lay.info.item()) == 0 and G.gptq_device_status(reset=True) == 0
-    # the dominant kernel's time inside the same timed loop: one more eager
-    # pass with events around the Hessian call only
+    assert not bool(lay.info.any().item()) and G.gptq_device_status(reset=True) == 0
+    del graph
+
+    # every kernel's time: one eager pass with the library's per-kind event
+    # timing, plus the dominant kernel alone in a loop of its own
+    ktimes = _kernel_times(lay, 2)
     k1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(a.steps)]
     for i in range(a.steps):
         lay.S.zero_()
         k1[i][0].record()
-        G.gptq_hessian_accumulate(lay.S, lay.X)
+        if E > 1:
+            G.gptq_hessian_accumulate_grouped(lay.S, lay.Xr, lay.offsets)
+        else:
+            G.gptq_hessian_accumulate(lay.S, lay.X)
         k1[i][1].record()
     torch.cuda.synchronize()
     k1_ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in k1)
 
-    # end to end through the public API from pinned host memory: X streams
-    # through the library's two-slot ring (each chunk's PCIe copy overlaps the
-    # accumulation of the one before, and the next layer's copies overlap this
-    # layer's prepare / quantize / pack); W goes in and the packed result
-    # comes back with plain copies on the compute stream
-    Xh = lay.X.cpu().pin_memory()
-    Wh = lay.W.cpu().pin_memory()
-    qwh = torch.empty_like(lay.qweight, device="cpu").pin_memory()
-    qzh = torch.empty_like(lay.qzeros, device="cpu").pin_memory()
-    sch = torch.empty_like(lay.scales, device="cpu").pin_memory()
-    hh = G.HostHessian(d, dev)
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    _barrier(ws)
-    torch.cuda.synchronize()
-    e_start.record()
-    hh.copy_stream.wait_stream(torch.cuda.current_stream())   # no copy starts before e_start
-    for _ in range(a.e2e_steps):
-        lay.S.zero_()
-        hh.accumulate(lay.S, Xh)
-        lay.W.copy_(Wh, non_blocking=True)
-        lay.after_hessian()
-        qwh.copy_(lay.qweight, non_blocking=True)
-        qzh.copy_(lay.qzeros, non_blocking=True)
-        sch.copy_(lay.scales, non_blocking=True)
-    e_end.record()
-    torch.cuda.synchronize()
-    e2e_ms = _max_over_ranks(e_start.elapsed_time(e_end) / a.e2e_steps, ws)
-    h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
-    d2h = sum(t.numel() * t.element_size() for t in (qwh, qzh, sch))
+    # end to end through the public API from pinned host memory
+    e2e = _e2e(lay, a, ws, dev)
 
     peaks, src = _peaks()
-    flops = float(n) * d * d                         # SYRK, upper triangle: n d^2
+    ntok = float(sum(lay.tokens))
+    flops = ntok * d * d                         # SYRK, upper triangle: n d^2
     achieved = flops / (k1_ms * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    traffic = _traffic_for("hessian.cu", "hessian_syrk_attn7b.json")
+    peak = float(peaks["bf16_tflops"])
+    traffic = _traffic_for("hessian.cu", "hessian_syrk_attn7b.json") if a.workload == "attn7b" \
+        else None
+    bounds = _phase_bounds(lay, peaks)
     line = {
         "metric": METRIC,
-        "value": ws * m * d / (ms * 1e-3),
+        "value": ws * units / (ms * 1e-3),
         "unit": UNIT,
         "n_gpus": ws,
         "steps": a.steps,
@@ -417,37 +655,96 @@ def run_ours(a):
         "dtype": "f32",
         "data": "synthetic (seeded; random-init weights, Gaussian calibration inputs with "
                 "outlier channels)",
-        "config": {"workload": f"{spec.name} ({a.workload}): W {m}x{d} fp16, X {n}x{d} fp16, "
-                               f"INT4 g128, damp 0.01, act_order={spec.act_order}",
-                   "layers_per_rank": 1, "tokens": n,
+        "config": {"workload": desc, "layers_per_rank": 1, "tokens": int(ntok),
                    "l2": "inputs larger than L2 (X %.2f GB re-read every step)" %
-                         (n * d * 2 / 1e9)},
-        "e2e": {"value": ws * m * d / (e2e_ms * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                         (ntok * d * 2 / 1e9)},
+        "e2e": e2e,
         "gpu_launches": int(launches),
         "roofline": {"bound": "tensor", "kernel": "hessian_accumulate (S += X^T X)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"bf16_tflops_sustained of {src} (fp16 = bf16 rate)",
+                     "peak_source": f"bf16_tflops (burst) of {src}: fp16 runs at the bf16 rate; "
+                                    f"the kernel is timed alone, {a.steps} launches",
                      "kernel_ms": k1_ms},
+        "kernels": _kernel_entries(lay, peaks, ktimes, 2),
+        "whole_layer": {"bound_ms": sum(bounds.values()), "phase_bound_ms": bounds,
+                        "frac": sum(bounds.values()) / ms,
+                        "note": "sum of the phase bounds at the measured burst peaks (TF32 = "
+                                "bf16 x 1.1/2.25) over the measured step"},
         "clocks": clk.summary(),
         "phase_ms": phase,
         "phase_note": "per-phase split from eager launches; the timed steps replay a CUDA graph"
-                      if graph is not None else "eager launches",
-        "launch_mode": "cuda_graph" if graph is not None else "eager",
+                      if not a.eager else "eager launches",
+        "launch_mode": "cuda_graph" if not a.eager else "eager",
         # one Hessian serves q/k/v (or up/gate) in a model: the rate of the
         # rest of the path, from the per-phase split
         "without_hessian": {
-            "value": m * d / (1e-3 * (phase["prepare"] + phase["quantize"] + phase["pack"])),
+            "value": units / (1e-3 * (phase["prepare"] + phase["quantize"] + phase["pack"])),
             "unit": UNIT, "note": "prepare + quantize + pack of the eager per-phase split"},
     }
-    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not a.no_configs:
+        head = {"workload": desc, "ms_per_layer": ms, "weights_per_s": units / (ms * 1e-3),
+                "steps": a.steps, "launches_per_step": graph_launches, "phase_ms": phase,
+                "phase_bound_ms": bounds, "whole_layer_frac": sum(bounds.values()) / ms,
+                "info_ok": True, "note": "the headline measurement above"}
+        del lay
+        torch.cuda.empty_cache()
+        cfg = _configs_summary(dev, peaks, max(3, min(a.steps, 5)), a.warmup,
+                               skip=(a.workload, a.layer))
+        hk = a.workload if a.workload in ("tiny", "moe8") else f"{a.workload}/{a.layer}"
+        line["configs"] = {hk: head, **cfg}
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline and a.workload != "moe8":
+        wl, spec, n = _workload(a.workload, a.layer, a.tokens)
         line["cpu_baseline"] = _cpu_baseline(spec, n)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def _e2e(lay, a, ws, dev):
+    """The same step through the public API from pinned host memory: X
+    (dense layers) streams through the library's two-slot ring -- each
+    chunk's PCIe copy overlaps the accumulation of the one before, and the
+    next layer's copies overlap this layer's prepare / quantize / pack; W
+    (and for the MoE layer X) go in with plain copies on the compute stream,
+    the packed result comes back inside the timed region."""
+    from post_weight_quantization_11_b200 import gptq as G
+    Xh = lay.X.cpu().pin_memory()
+    Wh = lay.W.cpu().pin_memory()
+    qwh = torch.empty_like(lay.qweight, device="cpu").pin_memory()
+    qzh = torch.empty_like(lay.qzeros, device="cpu").pin_memory()
+    sch = torch.empty_like(lay.scales, device="cpu").pin_memory()
+    dense = lay.mats == 1
+    hh = G.HostHessian(lay.d, dev) if dense else None
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    torch.cuda.synchronize()
+    e_start.record()
+    if dense:
+        hh.copy_stream.wait_stream(torch.cuda.current_stream())   # no copy before e_start
+    for _ in range(a.e2e_steps):
+        if dense:
+            lay.S.zero_()
+            hh.accumulate(lay.S, Xh)
+            lay.W.copy_(Wh, non_blocking=True)
+            lay.after_hessian()
+        else:
+            lay.X.copy_(Xh, non_blocking=True)
+            lay.W.copy_(Wh, non_blocking=True)
+            lay.step()
+        qwh.copy_(lay.qweight, non_blocking=True)
+        qzh.copy_(lay.qzeros, non_blocking=True)
+        sch.copy_(lay.scales, non_blocking=True)
+    e_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e_start.elapsed_time(e_end) / a.e2e_steps, ws)
+    h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in (qwh, qzh, sch))
+    units = lay.mats * lay.m * lay.d
+    return {"value": ws * units / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
 
 
 # --------------------------------------------------------------------------

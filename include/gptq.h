@@ -136,6 +136,46 @@ int gptq_hessian_accumulate_host(float* S, const uint16_t* X_host, int64_t n_tok
                                  void* ev_filled, void* ev_freed);
 
 /*
+ * Grouped Hessian accumulation -- the sum of gptq_hessian_accumulate ("GPTQ /
+ * AWQ / SqueezeLLM" sec. 一) for several independent groups of tokens at
+ * once: the experts of a mixture-of-experts layer, each calibrated on the
+ * tokens routed to it ("INT4/INT8 量化推理" sec. 五).
+ *
+ *   S_e[i][j] += sum_{offsets[e] <= t < offsets[e+1]} X[t][i] * X[t][j]
+ *                                          0 <= i <= j < d, 0 <= e < n_groups
+ *
+ * S: n_groups x d x d fp32, in/out (S_e at S + e d^2; upper triangles only,
+ *    as gptq_hessian_accumulate).
+ * X: n_rows x d fp16, the groups' rows one after the other (e.g. the output
+ *    of gptq_gather_rows).
+ * offsets: HOST array of n_groups + 1 int64: offsets[0] == 0, non-decreasing,
+ *    offsets[n_groups] == n_rows.  Empty groups are allowed (S_e unchanged).
+ * n_seen: optional HOST array of n_groups counters, each incremented by its
+ *    group's row count on success.
+ * One kernel launch per 64 groups; its work items run over (group, token
+ * split, output tile), so small and large groups share the SMs.  A group's
+ * last box of 64 rows is cut at the group's end on the device (the next
+ * group's rows never enter its sum).
+ * Requires the d limits of gptq_hessian_accumulate, 0 <= n_rows <= 2^31,
+ * 1 <= n_groups <= 2^20.
+ */
+int gptq_hessian_accumulate_grouped(float* S, const uint16_t* X, int64_t n_rows, int64_t d,
+                                    const int64_t* offsets, int64_t n_groups, int64_t* n_seen,
+                                    void* stream);
+
+/*
+ * Row gather -- the dispatch of routed tokens to experts that precedes the
+ * per-expert Hessians ("INT4/INT8 量化推理" sec. 五):
+ *   out[r][:] = X[idx[r]][:]      0 <= r < n_idx
+ * X: n_rows x d fp16; idx: n_idx int32 (device, 4-byte aligned); out:
+ * n_idx x d fp16.  An index outside [0, n_rows) is not followed: its row of
+ * `out` is written as zeros and the device status (gptq_device_status)
+ * records 0x201.  Requires d % 8 == 0, 8 <= d <= 32768.
+ */
+int gptq_gather_rows(const uint16_t* X, int64_t n_rows, int64_t d, const int32_t* idx,
+                     int64_t n_idx, uint16_t* out, void* stream);
+
+/*
  * Prepare the inverse-Hessian factor -- "GPTQ / AWQ / SqueezeLLM" sec. 一
  * (H = 2 X^T X / n, damping, decomposition of H^-1, importance order) and
  * "INT4/INT8 量化推理" sec. 三 (rows of H^-1 carry the error feedback).
@@ -178,6 +218,28 @@ int gptq_prepare_hinv(const float* S, int64_t d, int64_t n_tokens, float damp_re
 int gptq_prepare_hinv_static(const float* S, int64_t d, int64_t n_tokens, float damp_rel,
                              int act_order, int32_t* perm, float* U, int32_t* info,
                              void* stream);
+
+/*
+ * Batched preparation -- gptq_prepare_hinv ("GPTQ / AWQ / SqueezeLLM"
+ * sec. 一) for n_mats independent Hessians of the same size, e.g. the
+ * experts of a mixture-of-experts layer ("INT4/INT8 量化推理" sec. 五).
+ * Every matrix gets exactly the result gptq_prepare_hinv gives it; the
+ * factorizations of all matrices run in ONE persistent launch whose task
+ * queue interleaves the matrices, so their latency chains overlap.
+ *
+ * S: n_mats x d x d fp32 (S_e at S + e d^2, upper triangles read).
+ * n_tokens: HOST array of n_mats token counts (each > 0).
+ * perm: n_mats x d int32 output or NULL (required if act_order).
+ * U: n_mats x d x d fp32 output; info: n_mats device int32 outputs.
+ * ws: gptq_prepare_batched_workspace_bytes(d, n_mats) bytes of scratch
+ *    (n_mats times the single-matrix workspace, about 2 d^2 fp32 each).
+ * Requires the d limits of gptq_prepare_hinv, 1 <= n_mats <= 4096 and
+ * n_mats * d < 2^31.
+ */
+size_t gptq_prepare_batched_workspace_bytes(int64_t d, int64_t n_mats);
+int gptq_prepare_hinv_batched(const float* S, int64_t n_mats, int64_t d, const int64_t* n_tokens,
+                              float damp_rel, int act_order, int32_t* perm, float* U,
+                              int32_t* info, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Quantize one layer -- "INT4/INT8 量化推理" sec. 三 (column loop with error
@@ -230,6 +292,30 @@ int gptq_quantize_layer_static(const void* W, int w_dtype, int64_t d_out, int64_
                                const float* U, const int32_t* perm, int bits, int group_size,
                                int block_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
                                float* row_loss, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Batched quantization -- gptq_quantize_layer ("INT4/INT8 量化推理" sec. 三)
+ * for n_mats stacked layers of the same shape (the experts of a
+ * mixture-of-experts layer, sec. 五 of the same page), each with its own U
+ * and perm:
+ *   W: n_mats x d_out x d_in (layer e at e d_out d_in elements),
+ *   U: n_mats x d_in x d_in, perm: n_mats x d_in or NULL,
+ *   codes: n_mats x d_out x d_in, scales / zeros: n_mats x d_out x G,
+ *   row_loss: n_mats x d_out or NULL.
+ * Each layer gets exactly the result of gptq_quantize_layer.  The layers
+ * run one after the other on the stream and share ONE workspace of
+ * gptq_quantize_workspace_bytes(d_out, d_in, block_size) bytes: at these
+ * sizes one layer's sweep already fills the GPU (d_out / 32 CTAs per block).
+ * Dynamic groups only (group_size as gptq_quantize_layer).  Every layer's
+ * slice must stay 16-byte aligned (GPTQ_ERR_SHAPE otherwise).
+ * Pack the stacked codes and zero points with one gptq_pack_int4 call of
+ * n_mats * d_out rows.
+ */
+int gptq_quantize_layer_batched(const void* W, int w_dtype, int64_t n_mats, int64_t d_out,
+                                int64_t d_in, const float* U, const int32_t* perm, int bits,
+                                int group_size, int block_size, uint8_t* codes, uint16_t* scales,
+                                uint8_t* zeros, float* row_loss, void* ws, size_t ws_bytes,
+                                void* stream);
 
 /*
  * Pack INT4 -- "INT4/INT8 量化推理" sec. 一 (64 B of codes + 0.5 B zero point
@@ -292,6 +378,23 @@ int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bi
 int gptq_debug_gemm_nt(const float* A, int64_t lda, const float* B, int64_t ldb, float* C,
                        int64_t ldc, int64_t M, int64_t N, int64_t K, float alpha, float beta,
                        int lower, void* stream);
+
+/*
+ * Diagnostics (no counterpart on the pages): per-kind kernel timing.
+ * gptq_debug_kernel_timing(1) makes every later launch of the library
+ * bracket itself with two CUDA events on its stream; gptq_debug_kernel_times
+ * waits for the recorded events, returns per kind the summed milliseconds
+ * (ms[k]) and the number of timed launch sites (spans[k]), and forgets the
+ * records.  Kinds, in order (n_kinds >= 15): hessian, gather, finalize,
+ * factorization, init_work, split_u, static_params, sweep, update_near,
+ * update_far, pack, unpack, rtn, w4a16, probe (names from
+ * gptq_debug_kernel_kind_name).  Use it on eager launches only, never while
+ * a stream is being captured; it creates two CUDA events per launch site
+ * while enabled.  Disabled (the default) it costs one flag test per launch.
+ */
+int gptq_debug_kernel_timing(int enable);
+int gptq_debug_kernel_times(double* ms, int64_t* spans, int n_kinds);
+const char* gptq_debug_kernel_kind_name(int kind);
 
 /*
  * Test hooks (host only, no GPU needed; no counterpart on the pages).

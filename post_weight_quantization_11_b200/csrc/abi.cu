@@ -1,5 +1,8 @@
-// Library-wide C entry points: status names, ABI version, launch counter.
+// Library-wide C entry points: status names, ABI version, launch counter,
+// per-kind kernel timing (diagnostics).
 #include <atomic>
+#include <mutex>
+#include <vector>
 
 #include <cudaTypedefs.h>
 
@@ -51,6 +54,33 @@ int device_sm_count()
     return n;
 }
 
+// ---- per-kind kernel timing (diagnostics) --------------------------------
+
+static std::atomic<int> g_timing{0};
+static std::mutex g_timing_mu;
+struct TimedSpan { int kind; cudaEvent_t a, b; };
+static std::vector<TimedSpan> g_spans;
+
+KernelTimer::KernelTimer(int kind, cudaStream_t st) : kind_(kind), st_(st)
+{
+    if (!g_timing.load(std::memory_order_relaxed)) return;
+    if (cudaEventCreate(&ev0_) != cudaSuccess) { ev0_ = nullptr; return; }
+    if (cudaEventRecord(ev0_, st_) != cudaSuccess) { cudaEventDestroy(ev0_); ev0_ = nullptr; }
+}
+
+KernelTimer::~KernelTimer()
+{
+    if (!ev0_) return;
+    cudaEvent_t ev1 = nullptr;
+    if (cudaEventCreate(&ev1) != cudaSuccess || cudaEventRecord(ev1, st_) != cudaSuccess) {
+        if (ev1) cudaEventDestroy(ev1);
+        cudaEventDestroy(ev0_);
+        return;
+    }
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    g_spans.push_back(TimedSpan{kind_, ev0_, ev1});
+}
+
 static std::atomic<int> g_cta_cap[kCtaKinds];
 
 int persistent_ctas(int kind)
@@ -67,6 +97,47 @@ extern "C" int gptq_set_max_ctas(int kind, int max_ctas)
     if (kind < 0 || kind >= gptq::kCtaKinds || max_ctas < 0) return GPTQ_ERR_INVALID_ARG;
     gptq::g_cta_cap[kind].store(max_ctas);
     return GPTQ_OK;
+}
+
+extern "C" int gptq_debug_kernel_timing(int enable)
+{
+    gptq::g_timing.store(enable ? 1 : 0);
+    return GPTQ_OK;
+}
+
+extern "C" int gptq_debug_kernel_times(double* ms, int64_t* spans, int n_kinds)
+{
+    using namespace gptq;
+    if (!ms || !spans || n_kinds < kKKinds) return GPTQ_ERR_INVALID_ARG;
+    for (int k = 0; k < n_kinds; ++k) { ms[k] = 0.0; spans[k] = 0; }
+    std::vector<TimedSpan> take;
+    {
+        std::lock_guard<std::mutex> lock(g_timing_mu);
+        take.swap(g_spans);
+    }
+    int rc = GPTQ_OK;
+    for (const TimedSpan& t : take) {
+        float v = 0.f;
+        if (cudaEventSynchronize(t.b) != cudaSuccess ||
+            cudaEventElapsedTime(&v, t.a, t.b) != cudaSuccess)
+            rc = GPTQ_ERR_CUDA;
+        else if (t.kind >= 0 && t.kind < n_kinds) {
+            ms[t.kind] += double(v);
+            spans[t.kind] += 1;
+        }
+        cudaEventDestroy(t.a);
+        cudaEventDestroy(t.b);
+    }
+    return rc;
+}
+
+extern "C" const char* gptq_debug_kernel_kind_name(int kind)
+{
+    static const char* names[gptq::kKKinds] = {
+        "hessian", "gather", "finalize", "factorization", "init_work", "split_u",
+        "static_params", "sweep", "update_near", "update_far", "pack", "unpack", "rtn",
+        "w4a16", "probe"};
+    return (kind >= 0 && kind < gptq::kKKinds) ? names[kind] : "unknown";
 }
 
 extern "C" const char* gptq_status_string(int status)

@@ -29,6 +29,12 @@
 //   phase p:  S(p+1,p), F(p+1), S(p+2,p) .. S(T-1,p), I(p,p-1) .. I(p,0)
 //   phase T-1: I(T-1,T-2) .. I(T-1,0)
 //
+// Batches: one launch can factor E independent matrices of the same size
+// (the per-expert Hessians of a mixture-of-experts layer), stacked E high
+// in A, Xc, Y and U.  Task number t is local task t / E of matrix t % E, so
+// every matrix's tasks keep their topological order and the chains of all
+// E matrices advance side by side on the SMs.
+//
 // CTA roles (320 threads): warp 0 TMA producer (also waits for the
 // dependencies), warp 1 MMA issuer, warps 2-9 split each landed fp32 chunk
 // into TF32 head / remainder and fold the previous product's TMEM
@@ -66,7 +72,26 @@ struct CdParams {
     int32_t* info;
     int64_t d;
     int T, total;
+    int E;           // matrices in the batch (pointers above are matrix 0's)
+    int roff;        // first row of this matrix in the stacked tensor maps
 };
+
+// The view of matrix e of a batch: its arrays, flags and info word, and the
+// row offset of its tiles in the stacked tensor maps.
+__device__ __forceinline__ CdParams cd_matrix(const CdParams& p, int e)
+{
+    CdParams q = p;
+    const int64_t dd = p.d * p.d, TT = int64_t(p.T) * p.T;
+    q.A = p.A + e * dd;
+    q.Xc = p.Xc + e * p.d * 128;
+    q.Y = p.Y + e * dd;
+    q.U = p.U + e * dd;
+    q.flagL = p.flagL + e * 2 * TT;
+    q.flagY = q.flagL + TT;
+    q.info = p.info + e;
+    q.roff = (int)(int64_t(e) * p.d);
+    return q;
+}
 
 struct CdProduct {
     int ma, ra, ca;      // A operand: tensor map, first row, first column
@@ -120,6 +145,8 @@ __device__ __forceinline__ CdProduct cd_product(const CdParams& p, int type, int
         r = CdProduct{kMapX, i * CD_T, 0, kMapY, j * CD_T, i * CD_T, &p.flagL[i * T + i],
                       nullptr};
     }
+    r.ra += p.roff;
+    r.rb += p.roff;
     return r;
 }
 
@@ -181,6 +208,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t d = p.d;
     const int T = p.T;
+    CdParams q = p;                 // the matrix of the current task (see cd_matrix)
     if (tid == 0) {
         for (int s = 0; s < CD_STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
@@ -213,8 +241,8 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     auto run_pass = [&](int type, int ti, int tj, int pass, int n, auto&& epi) {
         if (warp == 0) {
             if (lane == 0) {
-                for (int q = 0; q < n; ++q) {
-                    const CdProduct pr = cd_product(p, type, ti, tj, pass, q);
+                for (int qi = 0; qi < n; ++qi) {
+                    const CdProduct pr = cd_product(q, type, ti, tj, pass, qi);
                     if (pr.f1 && !cd_wait_flag(pr.f1, abort, p.gabort)) break;
                     if (pr.f2 && !cd_wait_flag(pr.f2, abort, p.gabort)) break;
                     fence_proxy_async_global();
@@ -241,7 +269,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         } else if (warp == 1) {
             if (lane == 0) {
                 bool ok = true;
-                for (int q = 0; q < n && ok; ++q, ++mm_it) {
+                for (int qi = 0; qi < n && ok; ++qi, ++mm_it) {
                     const int a = mm_it & 1;
                     const uint32_t aph = (mm_it >> 1) & 1;
                     if (!mbar_wait(&acce_bar[a], aph ^ 1, kErrWaitAccEmpty, abort)) break;
@@ -280,8 +308,8 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             // (the MMA of q-1 overlaps the split of q)
             const int ct = tid - 64;
             bool ok = true;
-            for (int q = 0; q <= n && ok; ++q) {
-                if (q < n) {
+            for (int qi = 0; qi <= n && ok; ++qi) {
+                if (qi < n) {
                     for (int kc = 0; kc < CD_T / CD_KC; ++kc) {
                         if (!mbar_wait(&full_bar[cv_stage], cv_phase, kErrWaitFull, abort)) {
                             ok = false;
@@ -312,7 +340,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     }
                     if (!ok) break;
                 }
-                if (q > 0) {
+                if (qi > 0) {
                     const int a = ep_it & 1;
                     const uint32_t aph = (ep_it >> 1) & 1;
                     ++ep_it;
@@ -342,8 +370,9 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         __syncthreads();
         const int t = *s_task;
         if (t >= p.total) break;
+        q = cd_matrix(p, t % p.E);
         int type, ti, tj;
-        cd_decode(t, T, type, ti, tj);
+        cd_decode(t / p.E, T, type, ti, tj);
         const int n1 = (type == kTaskI) ? ti - tj : tj;
         const int64_t r0 = int64_t(ti) * CD_T, c0 = int64_t(tj) * CD_T;
 
@@ -372,7 +401,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
             for (int u = 0; u < CD_T / 2; ++u) acc[u] = 0.f;
         } else if (warp >= 2) {
-            const float4* src = reinterpret_cast<const float4*>(p.A + (r0 + m) * d + c0 + cb);
+            const float4* src = reinterpret_cast<const float4*>(q.A + (r0 + m) * d + c0 + cb);
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const float4 x = src[u];
@@ -380,7 +409,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             }
         }
         if (type == kTaskS)           // the mirrored tile of U is zero
-            cd_tile_zero(p.U + (d - CD_T - c0) * d + (d - CD_T - r0), d, warp, lane);
+            cd_tile_zero(q.U + (d - CD_T - c0) * d + (d - CD_T - r0), d, warp, lane);
         const float sgn = (type == kTaskI) ? 1.f : -1.f;
         run_pass(type, ti, tj, 1, n1, [&](const float (&v)[32], int cc) {
 #pragma unroll
@@ -397,28 +426,28 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         make_float4(0.f, 0.f, 0.f, 0.f);
             }
             __syncthreads();
-            leaf_factor_invert<CD_THREADS>(la, lx, lt, tid, p.info, d - c0, abort);
+            leaf_factor_invert<CD_THREADS>(la, lx, lt, tid, q.info, d - c0, abort);
             // X_jj first: the S tasks of column j wait only for it
             for (int idx = tid * 4; idx < CD_T * CD_T; idx += CD_THREADS * 4) {
                 const int r = idx / CD_T, c = idx % CD_T;
-                *reinterpret_cast<float4*>(p.Xc + (c0 + r) * CD_T + c) =
+                *reinterpret_cast<float4*>(q.Xc + (c0 + r) * CD_T + c) =
                     *reinterpret_cast<const float4*>(lx + r * LDA + c);
             }
             fence_proxy_async_global();
             __syncthreads();
             if (tid == 0 && !*abort) {
                 __threadfence();
-                st_release_gpu(&p.flagL[tj * T + tj], 1);
+                st_release_gpu(&q.flagL[tj * T + tj], 1);
             }
             // then Y_jj = X_jj^T and the diagonal tile of U
-            cd_tile_out_transposed(lx, p.Y + c0 * d + c0, d, warp, lane);
-            cd_tile_out_reversed(lx, p.U + (d - CD_T - c0) * d + (d - CD_T - c0), d, warp, lane);
-            release(&p.flagY[tj * T + tj]);
+            cd_tile_out_transposed(lx, q.Y + c0 * d + c0, d, warp, lane);
+            cd_tile_out_reversed(lx, q.U + (d - CD_T - c0) * d + (d - CD_T - c0), d, warp, lane);
+            release(&q.flagY[tj * T + tj]);
         } else if (type == kTaskS) {
             if (n1 > 0) {             // A_ij - sum back into A: the final product reads it
                 stage_acc();
                 __syncthreads();
-                cd_tile_out(sb, p.A + r0 * d + c0, d, warp, lane);
+                cd_tile_out(sb, q.A + r0 * d + c0, d, warp, lane);
                 fence_proxy_async_global();
                 fence_proxy_async_smem();
                 __syncthreads();
@@ -431,13 +460,13 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
             });
             __syncthreads();
-            cd_tile_out(sb, p.A + r0 * d + c0, d, warp, lane);
-            release(&p.flagL[ti * T + tj]);
+            cd_tile_out(sb, q.A + r0 * d + c0, d, warp, lane);
+            release(&q.flagL[ti * T + tj]);
         } else {
             // the sum's transpose into the Y_ji tile: the final product reads it
             stage_acc();
             __syncthreads();
-            cd_tile_out(sb, p.Y + c0 * d + r0, d, warp, lane);
+            cd_tile_out(sb, q.Y + c0 * d + r0, d, warp, lane);
             fence_proxy_async_global();
             fence_proxy_async_smem();
             __syncthreads();
@@ -449,9 +478,9 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         make_float4(-v[4 * u], -v[4 * u + 1], -v[4 * u + 2], -v[4 * u + 3]);
             });
             __syncthreads();
-            cd_tile_out_transposed(sb, p.Y + c0 * d + r0, d, warp, lane);
-            cd_tile_out_reversed(sb, p.U + (d - CD_T - r0) * d + (d - CD_T - c0), d, warp, lane);
-            release(&p.flagY[tj * T + ti]);
+            cd_tile_out_transposed(sb, q.Y + c0 * d + r0, d, warp, lane);
+            cd_tile_out_reversed(sb, q.U + (d - CD_T - r0) * d + (d - CD_T - c0), d, warp, lane);
+            release(&q.flagY[tj * T + ti]);
         }
     }
 
@@ -465,35 +494,41 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
 }
 
-size_t chol_dag_sync_bytes(int64_t d)
+size_t chol_dag_sync_bytes(int64_t d, int64_t E)
 {
     const int64_t T = d / CD_T;
-    return sizeof(int) * size_t(2 * T * T + 32);
+    return sizeof(int) * size_t(2 * T * T * E + 32);
 }
 
-int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d, int32_t* info,
-                 cudaStream_t st)
+int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d, int64_t E,
+                 int32_t* info, cudaStream_t st)
 {
     if (d < CD_T || d % CD_T) return GPTQ_ERR_SHAPE;
     const int T = (int)(d / CD_T);
+    if (E < 1 || E * d > (int64_t(1) << 31) - 1 || E * T * T > (int64_t(1) << 30))
+        return GPTQ_ERR_SHAPE;
     CdParams p{};
     p.A = A; p.Xc = Xc; p.Y = Y; p.U = U;
     int* s = reinterpret_cast<int*>(sync);
     p.flagL = s;
     p.flagY = s + size_t(T) * T;
-    p.ticket = s + size_t(2) * T * T;
+    p.ticket = s + size_t(2) * T * T * E;
     p.gabort = p.ticket + 1;
     p.info = info;
     p.d = d;
     p.T = T;
-    p.total = T * T;
-    if (cudaMemsetAsync(sync, 0, chol_dag_sync_bytes(d), st) != cudaSuccess) return GPTQ_ERR_CUDA;
+    p.E = (int)E;
+    p.total = (int)(E * T * T);
+    p.roff = 0;
+    if (cudaMemsetAsync(sync, 0, chol_dag_sync_bytes(d, E), st) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
     CUtensorMap tA, tX, tY;
-    if (encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, A, (uint64_t)d, (uint64_t)d,
+    const uint64_t rows = uint64_t(E) * uint64_t(d);
+    if (encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, A, (uint64_t)d, rows,
                        (uint64_t)d * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
-        encode_tmap_2d(&tX, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Xc, (uint64_t)CD_T, (uint64_t)d,
+        encode_tmap_2d(&tX, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Xc, (uint64_t)CD_T, rows,
                        (uint64_t)CD_T * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
-        encode_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, (uint64_t)d, (uint64_t)d,
+        encode_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, (uint64_t)d, rows,
                        (uint64_t)d * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK)
         return GPTQ_ERR_CUDA;
     if (cudaFuncSetAttribute(chol_dag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -6,9 +6,10 @@
 
 namespace gptq {
 
-// Bytes of the synchronization area chol_inv_dag needs for T = d / 128
-// tiles per dimension (tile flags + the task ticket counter).
-size_t chol_dag_sync_bytes(int64_t d);
+// Bytes of the synchronization area chol_inv_dag needs for a batch of E
+// matrices with T = d / 128 tiles per dimension (tile flags + the task
+// ticket counter).
+size_t chol_dag_sync_bytes(int64_t d, int64_t E = 1);
 
 // A (d x d, row-major): on entry its lower 128x128 tiles hold the symmetric
 // positive definite matrix to factor (the upper tiles are never read); on
@@ -20,7 +21,9 @@ size_t chol_dag_sync_bytes(int64_t d);
 // U (d x d): on exit U[i][j] = (L^-1)[d-1-i][d-1-j] (upper; zeros below).
 // sync: chol_dag_sync_bytes(d) bytes of scratch (cleared here).
 // info: a non-positive pivot stores its position (as the leaf reports it).
-int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d, int32_t* info,
-                 cudaStream_t st);
+// Batches: E matrices stacked E high in A, Xc, Y, U (matrix e at rows
+// [e d, e d + d)), one info word each (info[e]); one launch factors them all.
+int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d, int64_t E,
+                 int32_t* info, cudaStream_t st);
 
 }  // namespace gptq

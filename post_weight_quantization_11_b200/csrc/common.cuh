@@ -37,6 +37,27 @@ int device_sm_count();
 enum CtaKind : int { kCtaHessian = 0, kCtaPrepare = 1, kCtaKinds = 2 };
 int persistent_ctas(int kind);
 
+// Diagnostics (gptq_debug_kernel_timing): kinds of the library's launches.
+enum KernelKind : int {
+    kKHessian = 0, kKGather, kKFinalize, kKFactor, kKInitWork, kKSplitU, kKStaticParams,
+    kKSweep, kKUpdateNear, kKUpdateFar, kKPack, kKUnpack, kKRtn, kKW4A16, kKProbe, kKKinds
+};
+
+// While timing is enabled, the launches issued in this object's lifetime are
+// bracketed by two CUDA events on `st` and their time is added to `kind`.
+// Otherwise it does nothing.  For eager use (not under stream capture).
+class KernelTimer {
+public:
+    KernelTimer(int kind, cudaStream_t st);
+    ~KernelTimer();
+    KernelTimer(const KernelTimer&) = delete;
+    KernelTimer& operator=(const KernelTimer&) = delete;
+private:
+    int kind_;
+    cudaStream_t st_;
+    cudaEvent_t ev0_ = nullptr;
+};
+
 // Supported problem limits (validated at the ABI).
 constexpr int64_t kMaxDim = 32768;
 constexpr int64_t kMaxRows = int64_t(1) << 24;

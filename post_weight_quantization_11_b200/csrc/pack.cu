@@ -101,6 +101,7 @@ extern "C" int gptq_pack_int4(const uint8_t* codes, const uint8_t* zeros, int64_
         return GPTQ_ERR_SHAPE;
     cudaStream_t st = as_stream(stream);
     const int64_t words = d_out * d_in / 8;
+    KernelTimer kt(kKPack, st);
     if (words % 4 == 0)
         pack_codes_kernel<<<grid_for(words / 4, 256), 256, 0, st>>>(codes, words / 4, d_in / 8,
                                                                     qweight);
@@ -124,6 +125,7 @@ extern "C" int gptq_unpack_int4(const uint32_t* qweight, const uint8_t* qzeros, 
         return GPTQ_ERR_SHAPE;
     cudaStream_t st = as_stream(stream);
     const int64_t words = d_out * d_in / 8;
+    KernelTimer kt(kKUnpack, st);
     unpack_codes_kernel<<<grid_for(words, 256), 256, 0, st>>>(qweight, words, codes);
     count_launches();
     unpack_zeros_kernel<<<grid_for(d_out * n_groups, 256), 256, 0, st>>>(qzeros, d_out, n_groups,

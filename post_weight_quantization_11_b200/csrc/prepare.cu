@@ -33,17 +33,19 @@ struct PrepWs {
     int32_t* pid;  // d, identity permutation when the caller passes none
 };
 
-static size_t prep_layout(int64_t d, char* base, PrepWs* w)
+// Workspace of a batch of E matrices (E = 1: one layer); matrix e's parts at
+// e d^2 (A, Y), e d 128 (Xc), e d (keys, pid) and 4 e (lam).
+static size_t prep_layout(int64_t d, int64_t E, char* base, PrepWs* w)
 {
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 1024); return o; };
-    size_t oA = take(sizeof(float) * d * d);
-    size_t oY = take(sizeof(float) * d * d);
-    size_t oX = take(sizeof(float) * d * TW);
-    size_t oS = take(chol_dag_sync_bytes(d));
-    size_t oK = take(sizeof(float) * d);
-    size_t oL = take(sizeof(float) * 4);
-    size_t oP = take(sizeof(int32_t) * d);
+    size_t oA = take(sizeof(float) * d * d * E);
+    size_t oY = take(sizeof(float) * d * d * E);
+    size_t oX = take(sizeof(float) * d * TW * E);
+    size_t oS = take(chol_dag_sync_bytes(d, E));
+    size_t oK = take(sizeof(float) * d * E);
+    size_t oL = take(sizeof(float) * 4 * E);
+    size_t oP = take(sizeof(int32_t) * d * E);
     if (w && base) {
         w->A = reinterpret_cast<float*>(base + oA);
         w->Y = reinterpret_cast<float*>(base + oY);
@@ -133,12 +135,53 @@ __global__ void build_reversed_kernel(const float* __restrict__ S, const int32_t
     }
 }
 
+// Argument checks shared by every preparation entry point (before any launch).
+int prepare_check_args(const float* S, int64_t d, float damp_rel, int act_order,
+                       const int32_t* perm, const float* U, const int32_t* info)
+{
+    if (!S || !U || !info) return GPTQ_ERR_INVALID_ARG;
+    if (act_order && !perm) return GPTQ_ERR_INVALID_ARG;
+    if (!aligned16(S) || !aligned16(U) || (perm && !aligned16(perm)))
+        return GPTQ_ERR_INVALID_ARG;
+    if (!(damp_rel >= 0.f)) return GPTQ_ERR_INVALID_ARG;
+    if (d < 128 || d > kMaxDim || d % 128 != 0) return GPTQ_ERR_SHAPE;
+    return GPTQ_OK;
+}
+
+// The finalize steps of matrix e: lambda, perm, the reversed damped Hessian.
+static int prepare_finalize(const float* S, int64_t d, int64_t n_tokens, float damp_rel,
+                            int act_order, int32_t* perm, int32_t* info, const PrepWs& w,
+                            int64_t e, cudaStream_t st)
+{
+    const float* Se = S + e * d * d;
+    float* keys = w.keys + e * d;
+    float* lam = w.lam + 4 * e;
+    int32_t* p = perm ? perm + e * d : w.pid + e * d;
+    KernelTimer kt(kKFinalize, st);
+    diag_lambda_kernel<<<1, 1024, 0, st>>>(Se, d, n_tokens, damp_rel, keys, lam, info + e);
+    count_launches();
+    rank_perm_kernel<<<(unsigned)ceil_div(d, 256), 256, 0, st>>>(keys, d, act_order, p);
+    count_launches();
+    // one CTA per row: rows hold 128 .. d entries of the lower tiles
+    build_reversed_kernel<<<dim3(1, (unsigned)d), 256, 0, st>>>(Se, p, lam, d,
+                                                                2.0f / float(n_tokens),
+                                                                w.A + e * d * d);
+    count_launches();
+    return launch_status();
+}
+
 }  // namespace gptq
 
 extern "C" size_t gptq_prepare_workspace_bytes(int64_t d)
 {
     if (d <= 0) return 0;
-    return gptq::prep_layout(d, nullptr, nullptr);
+    return gptq::prep_layout(d, 1, nullptr, nullptr);
+}
+
+extern "C" size_t gptq_prepare_batched_workspace_bytes(int64_t d, int64_t n_mats)
+{
+    if (d <= 0 || n_mats <= 0) return 0;
+    return gptq::prep_layout(d, n_mats, nullptr, nullptr);
 }
 
 extern "C" int gptq_prepare_hinv(const float* S, int64_t d, int64_t n_tokens, float damp_rel,
@@ -146,29 +189,49 @@ extern "C" int gptq_prepare_hinv(const float* S, int64_t d, int64_t n_tokens, fl
                                  void* ws, size_t ws_bytes, void* stream)
 {
     using namespace gptq;
-    if (!S || !U || !info || !ws) return GPTQ_ERR_INVALID_ARG;
-    if (act_order && !perm) return GPTQ_ERR_INVALID_ARG;
-    if (!aligned16(S) || !aligned16(U) || !aligned16(ws) || (perm && !aligned16(perm)))
-        return GPTQ_ERR_INVALID_ARG;
-    if (!(damp_rel >= 0.f)) return GPTQ_ERR_INVALID_ARG;
-    if (d < 128 || d > kMaxDim || d % 128 != 0) return GPTQ_ERR_SHAPE;
+    int rc = prepare_check_args(S, d, damp_rel, act_order, perm, U, info);
+    if (rc != GPTQ_OK) return rc;
+    if (!ws || !aligned16(ws)) return GPTQ_ERR_INVALID_ARG;
     if (n_tokens <= 0) return GPTQ_ERR_SHAPE;
     if (ws_bytes < gptq_prepare_workspace_bytes(d)) return GPTQ_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     PrepWs w;
-    prep_layout(d, reinterpret_cast<char*>(ws), &w);
-    int32_t* p = perm ? perm : w.pid;
-    diag_lambda_kernel<<<1, 1024, 0, st>>>(S, d, n_tokens, damp_rel, w.keys, w.lam, info);
-    count_launches();
-    rank_perm_kernel<<<(unsigned)ceil_div(d, 256), 256, 0, st>>>(w.keys, d, act_order, p);
-    count_launches();
+    prep_layout(d, 1, reinterpret_cast<char*>(ws), &w);
+    rc = prepare_finalize(S, d, n_tokens, damp_rel, act_order, perm, info, w, 0, st);
+    if (rc != GPTQ_OK) return rc;
     {
-        // one CTA per row: rows hold 128 .. d entries of the lower tiles
-        build_reversed_kernel<<<dim3(1, (unsigned)d), 256, 0, st>>>(S, p, w.lam, d,
-                                                                    2.0f / float(n_tokens), w.A);
-        count_launches();
+        KernelTimer kt(kKFactor, st);
+        if (chol_inv_dag(w.A, w.Xc, w.Y, U, w.sync, d, 1, info, st) != GPTQ_OK)
+            return GPTQ_ERR_CUDA;
     }
-    if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
-    if (chol_inv_dag(w.A, w.Xc, w.Y, U, w.sync, d, info, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
+    return launch_status();
+}
+
+extern "C" int gptq_prepare_hinv_batched(const float* S, int64_t n_mats, int64_t d,
+                                         const int64_t* n_tokens, float damp_rel, int act_order,
+                                         int32_t* perm, float* U, int32_t* info, void* ws,
+                                         size_t ws_bytes, void* stream)
+{
+    using namespace gptq;
+    int rc = prepare_check_args(S, d, damp_rel, act_order, perm, U, info);
+    if (rc != GPTQ_OK) return rc;
+    if (!n_tokens || !ws || !aligned16(ws)) return GPTQ_ERR_INVALID_ARG;
+    if (n_mats < 1 || n_mats > 4096 || n_mats * d > (int64_t(1) << 31) - 1)
+        return GPTQ_ERR_SHAPE;
+    for (int64_t e = 0; e < n_mats; ++e)
+        if (n_tokens[e] <= 0) return GPTQ_ERR_SHAPE;
+    if (ws_bytes < gptq_prepare_batched_workspace_bytes(d, n_mats)) return GPTQ_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    PrepWs w;
+    prep_layout(d, n_mats, reinterpret_cast<char*>(ws), &w);
+    for (int64_t e = 0; e < n_mats; ++e) {
+        rc = prepare_finalize(S, d, n_tokens[e], damp_rel, act_order, perm, info, w, e, st);
+        if (rc != GPTQ_OK) return rc;
+    }
+    {
+        KernelTimer kt(kKFactor, st);
+        if (chol_inv_dag(w.A, w.Xc, w.Y, U, w.sync, d, n_mats, info, st) != GPTQ_OK)
+            return GPTQ_ERR_CUDA;
+    }
     return launch_status();
 }

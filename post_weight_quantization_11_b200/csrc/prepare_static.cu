@@ -21,6 +21,9 @@
 
 namespace gptq {
 
+int prepare_check_args(const float* S, int64_t d, float damp_rel, int act_order,
+                       const int32_t* perm, const float* U, const int32_t* info);
+
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB
 constexpr int64_t kStaticMaxDim = 1024;
 constexpr int kMaxDevices = 64;
@@ -58,6 +61,11 @@ extern "C" int gptq_prepare_hinv_static(const float* S, int64_t d, int64_t n_tok
                                         int32_t* info, void* stream)
 {
     using namespace gptq;
+    // the argument checks of gptq_prepare_hinv first, so both entry points
+    // return the same status for the same bad argument
+    int rc = prepare_check_args(S, d, damp_rel, act_order, perm, U, info);
+    if (rc != GPTQ_OK) return rc;
+    if (n_tokens <= 0) return GPTQ_ERR_SHAPE;
     if (d > kStaticMaxDim) return GPTQ_ERR_SHAPE;               // beyond the fixed scratch
     const size_t need = gptq_prepare_workspace_bytes(d);
     if (need > kStaticScratchBytes) return GPTQ_ERR_SHAPE;

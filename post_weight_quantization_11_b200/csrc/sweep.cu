@@ -345,6 +345,7 @@ static void launch_sweep(dim3 grid, size_t smem, cudaStream_t st, const float* W
 {
     cudaFuncSetAttribute(block_sweep_kernel<GS, STATIC>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    KernelTimer kt(kKSweep, st);
     block_sweep_kernel<GS, STATIC><<<grid, SW_THREADS, smem, st>>>(
         Wk, U, m, d, gsz, j0, maxqf, codes, scales, zeros, Eh, El, ldE, row_loss, first);
     count_launches();
@@ -403,6 +404,7 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
     {
         const int64_t total = m * d;
         const unsigned grid = (unsigned)std::min<int64_t>(ceil_div(total, 256), 148 * 16);
+        KernelTimer kt(kKInitWork, st);
         if (w_dtype == GPTQ_DTYPE_F16)
             init_work_kernel<__half><<<grid, 256, 0, st>>>(reinterpret_cast<const __half*>(W), perm,
                                                            m, d, w.Wk);
@@ -415,11 +417,15 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
     __half* sc = reinterpret_cast<__half*>(scales);
     if (stat) {
         const int64_t warps = m * (d / gsz);
+        KernelTimer kt(kKStaticParams, st);
         static_params_kernel<<<(unsigned)ceil_div(warps * 32, 256), 256, 0, st>>>(
             w.Wk, m, d, gsz, maxqf, sc, zeros);
         count_launches();
     }
-    rc = update_prepare_u(U, d, &w.upd, st);
+    {
+        KernelTimer kt(kKSplitU, st);
+        rc = update_prepare_u(U, d, &w.upd, st);
+    }
     if (rc != GPTQ_OK) return rc;
     const dim3 grid((unsigned)ceil_div(m, SW_ROWS));
     const size_t smem = sizeof(float) * (SW_B * SW_B + SW_B);
@@ -454,11 +460,13 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
         }
 #undef GPTQ_SWEEP
         if (j0 + SW_B < ob1) {                                   // near: rest of the outer block
+            KernelTimer kt(kKUpdateNear, st);
             rc = block_update(w.Wk, &w.upd, m, d, /*e_col0=*/ecol, /*k_rows=*/SW_B, /*u_row0=*/j0,
                               /*c_begin=*/j0 + SW_B, /*c_end=*/ob1, st);
             if (rc != GPTQ_OK) return rc;
         }
         if (j0 + SW_B == ob1 && ob1 < d) {                       // far: everything beyond it
+            KernelTimer kt(kKUpdateFar, st);
             rc = block_update(w.Wk, &w.upd, m, d, /*e_col0=*/0, /*k_rows=*/ob1 - ob0,
                               /*u_row0=*/ob0, /*c_begin=*/ob1, /*c_end=*/d, st);
             if (rc != GPTQ_OK) return rc;
@@ -490,6 +498,38 @@ extern "C" int gptq_quantize_layer_static(const void* W, int w_dtype, int64_t d_
                                codes, scales, zeros, row_loss, ws, ws_bytes, stream, true);
 }
 
+extern "C" int gptq_quantize_layer_batched(const void* W, int w_dtype, int64_t n_mats,
+                                           int64_t d_out, int64_t d_in, const float* U,
+                                           const int32_t* perm, int bits, int group_size,
+                                           int block_size, uint8_t* codes, uint16_t* scales,
+                                           uint8_t* zeros, float* row_loss, void* ws,
+                                           size_t ws_bytes, void* stream)
+{
+    using namespace gptq;
+    if (n_mats < 1 || n_mats > 4096) return GPTQ_ERR_SHAPE;
+    if (!W || !U || !codes || !scales || !zeros) return GPTQ_ERR_INVALID_ARG;
+    int64_t gsz = 0;
+    int rc = sweep_group_size(d_in, group_size, false, &gsz);
+    if (rc != GPTQ_OK) return rc;
+    const int64_t G = d_in / gsz;
+    const size_t wb = (w_dtype == GPTQ_DTYPE_F16) ? 2 : 4;
+    // every matrix's arrays must stay 16-byte aligned at their offsets
+    if ((d_out * d_in * int64_t(wb)) % 16 || (d_out * G * 2) % 16 || (d_out * G) % 16 ||
+        (row_loss && (d_out * 4) % 16) || (perm && (d_in * 4) % 16))
+        return GPTQ_ERR_SHAPE;
+    // one layer after the other on the stream: each fills the GPU on its own
+    // (d_out / 32 sweep CTAs per block), and they share the one workspace
+    for (int64_t e = 0; e < n_mats; ++e) {
+        rc = quantize_impl(reinterpret_cast<const char*>(W) + e * d_out * d_in * int64_t(wb),
+                           w_dtype, d_out, d_in, U + e * d_in * d_in,
+                           perm ? perm + e * d_in : nullptr, bits, group_size, block_size,
+                           codes + e * d_out * d_in, scales + e * d_out * G, zeros + e * d_out * G,
+                           row_loss ? row_loss + e * d_out : nullptr, ws, ws_bytes, stream, false);
+        if (rc != GPTQ_OK) return rc;
+    }
+    return GPTQ_OK;
+}
+
 extern "C" int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bits,
                             int group_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
                             void* stream)
@@ -506,6 +546,7 @@ extern "C" int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d
     const int64_t warps = d_out * (d_in / 128);
     const unsigned grid = (unsigned)ceil_div(warps * 32, 256);
     __half* sc = reinterpret_cast<__half*>(scales);
+    KernelTimer kt(kKRtn, st);
 #define GPTQ_RTN_LAUNCH(GSV)                                                                     \
     if (w_dtype == GPTQ_DTYPE_F16)                                                               \
         rtn_kernel<GSV, __half><<<grid, 256, 0, st>>>(reinterpret_cast<const __half*>(W), d_out, \

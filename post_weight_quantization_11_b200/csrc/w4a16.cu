@@ -169,6 +169,7 @@ extern "C" int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t*
     const int64_t g = (group_size == -1) ? d_in : group_size;
     if (g < 32 || g % 32 != 0 || d_in % g != 0) return GPTQ_ERR_UNSUPPORTED;
     cudaStream_t st = as_stream(stream);
+    KernelTimer kt(kKW4A16, st);
     if (cudaMemsetAsync(y, 0, sizeof(float) * size_t(batch) * size_t(d_out), st) != cudaSuccess)
         return GPTQ_ERR_CUDA;
     const dim3 grid((unsigned)ceil_div(d_out, W4_WARPS * W4_ROWS), (unsigned)ceil_div(d_in, W4_KS));

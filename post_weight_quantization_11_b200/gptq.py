@@ -29,11 +29,15 @@ _STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_SHAPE", 3: "GPT
 EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_device_status", "gptq_set_max_ctas",
             "gptq_hessian_accumulate", "gptq_hessian_accumulate_host",
+            "gptq_hessian_accumulate_grouped", "gptq_gather_rows",
             "gptq_prepare_workspace_bytes", "gptq_prepare_hinv", "gptq_prepare_hinv_static",
+            "gptq_prepare_batched_workspace_bytes", "gptq_prepare_hinv_batched",
+            "gptq_quantize_layer_batched",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_quantize_layer_static",
             "gptq_pack_int4",
             "gptq_unpack_int4", "gptq_w4a16_gemm", "rtn_quantize", "gptq_debug_gemm_nt",
-            "gptq_debug_chol_task_order", "gptq_debug_div_rn", "gptq_debug_bounded_wait")
+            "gptq_debug_chol_task_order", "gptq_debug_div_rn", "gptq_debug_bounded_wait",
+            "gptq_debug_kernel_timing", "gptq_debug_kernel_times", "gptq_debug_kernel_kind_name")
 
 
 class GptqError(RuntimeError):
@@ -64,7 +68,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_set_max_ctas": ([I32, I32], I32),
         "gptq_hessian_accumulate": ([P, P, I64, I64, P, P], I32),
         "gptq_hessian_accumulate_host": ([P, P, I64, I64, P, P, SZ, I64, P, P, P, P], I32),
+        "gptq_hessian_accumulate_grouped": ([P, P, I64, I64, P, I64, P, P], I32),
+        "gptq_gather_rows": ([P, I64, I64, P, I64, P, P], I32),
         "gptq_prepare_workspace_bytes": ([I64], SZ),
+        "gptq_prepare_batched_workspace_bytes": ([I64, I64], SZ),
+        "gptq_prepare_hinv_batched": ([P, I64, I64, P, F32, I32, P, P, P, P, SZ, P], I32),
+        "gptq_quantize_layer_batched": ([P, I32, I64, I64, I64, P, P, I32, I32, I32, P, P, P, P,
+                                         P, SZ, P], I32),
         "gptq_prepare_hinv": ([P, I64, I64, F32, I32, P, P, P, P, SZ, P], I32),
         "gptq_prepare_hinv_static": ([P, I64, I64, F32, I32, P, P, P, P], I32),
         "gptq_quantize_workspace_bytes": ([I64, I64, I32], SZ),
@@ -80,6 +90,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_debug_chol_task_order": ([I64, P, I64], I64),
         "gptq_debug_div_rn": ([P, P, I64, P], I32),
         "gptq_debug_bounded_wait": ([P, I32, I64, P], I32),
+        "gptq_debug_kernel_timing": ([I32], I32),
+        "gptq_debug_kernel_times": ([P, P, I32], I32),
+        "gptq_debug_kernel_kind_name": ([I32], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -147,6 +160,27 @@ def gptq_set_max_ctas(kind: int, max_ctas: int) -> None:
     _check("gptq_set_max_ctas", load_library().gptq_set_max_ctas(int(kind), int(max_ctas)))
 
 
+N_KERNEL_KINDS = 15
+
+
+def gptq_debug_kernel_timing(enable: bool) -> None:
+    """Per-kind CUDA-event timing of the library's launches (eager use only)."""
+    _check("gptq_debug_kernel_timing", load_library().gptq_debug_kernel_timing(int(bool(enable))))
+
+
+def gptq_debug_kernel_times() -> dict:
+    """{kind: (milliseconds, timed launch sites)} since the last call (waits for the events)."""
+    import numpy as np
+    ms = np.zeros(N_KERNEL_KINDS, dtype=np.float64)
+    sp = np.zeros(N_KERNEL_KINDS, dtype=np.int64)
+    lib = load_library()
+    _check("gptq_debug_kernel_times",
+           lib.gptq_debug_kernel_times(ctypes.c_void_p(ms.ctypes.data),
+                                       ctypes.c_void_p(sp.ctypes.data), N_KERNEL_KINDS))
+    return {lib.gptq_debug_kernel_kind_name(k).decode(): (float(ms[k]), int(sp[k]))
+            for k in range(N_KERNEL_KINDS) if sp[k]}
+
+
 def gptq_status_string(status: int) -> str:
     return load_library().gptq_status_string(int(status)).decode()
 
@@ -161,6 +195,38 @@ def gptq_hessian_accumulate(S: torch.Tensor, X: torch.Tensor) -> int:
     _check("gptq_hessian_accumulate",
            load_library().gptq_hessian_accumulate(_ptr(S), _ptr(X), n, d, None, _stream(S)))
     return n
+
+
+def gptq_gather_rows(X: torch.Tensor, idx: torch.Tensor, out=None) -> torch.Tensor:
+    """out[r] = X[idx[r]] (the routed tokens' rows, e.g. expert-major)."""
+    _need(X, "X", torch.float16)
+    _need(idx, "idx", torch.int32)
+    n, d = X.shape
+    k = idx.numel()
+    out = torch.empty(k, d, dtype=torch.float16, device=X.device) if out is None else out
+    _need(out, "out", torch.float16)
+    _check("gptq_gather_rows",
+           load_library().gptq_gather_rows(_ptr(X), n, d, _ptr(idx), k, _ptr(out), _stream(X)))
+    return out
+
+
+def gptq_hessian_accumulate_grouped(S: torch.Tensor, X: torch.Tensor, offsets) -> list:
+    """S[e] (E x d x d fp32, upper triangles) += X[o_e:o_{e+1}]^T X[o_e:o_{e+1}]
+    for the row segments given by the host offsets (E + 1 non-decreasing
+    ints, 0 .. n).  One launch for up to 64 segments.  Returns the
+    segments' token counts."""
+    import numpy as np
+    _need(S, "S", torch.float32)
+    _need(X, "X", torch.float16)
+    n, d = X.shape
+    off = np.ascontiguousarray(np.asarray(offsets, dtype=np.int64))
+    E = off.size - 1
+    if S.shape != (E, d, d):
+        raise ValueError("S must be E x d x d")
+    _check("gptq_hessian_accumulate_grouped",
+           load_library().gptq_hessian_accumulate_grouped(
+               _ptr(S), _ptr(X), n, d, ctypes.c_void_p(off.ctypes.data), E, None, _stream(S)))
+    return [int(v) for v in np.diff(off)]
 
 
 class HostHessian:
@@ -259,6 +325,64 @@ def gptq_prepare_hinv_static(S: torch.Tensor, n_tokens: int, damp_rel: float = 0
                                                    int(bool(act_order)), _ptr(perm), _ptr(U),
                                                    _ptr(info), _stream(S)))
     return perm, U, info
+
+
+def gptq_prepare_batched_workspace_bytes(d: int, n_mats: int) -> int:
+    return int(load_library().gptq_prepare_batched_workspace_bytes(int(d), int(n_mats)))
+
+
+def gptq_prepare_hinv_batched(S: torch.Tensor, n_tokens, damp_rel: float = 0.01,
+                              act_order: bool = False, perm=None, U=None, info=None, ws=None):
+    """The preparation of E Hessians at once (one factorization launch).
+    S: E x d x d fp32; n_tokens: E host ints.  Returns (perm E x d int32,
+    U E x d x d fp32, info E int32 on the device)."""
+    import numpy as np
+    _need(S, "S", torch.float32)
+    E, d = S.shape[0], S.shape[1]
+    dev = S.device
+    nt = np.ascontiguousarray(np.asarray(n_tokens, dtype=np.int64))
+    if nt.size != E:
+        raise ValueError("n_tokens must have one entry per matrix")
+    perm = torch.empty(E, d, dtype=torch.int32, device=dev) if perm is None else perm
+    U = torch.empty(E, d, d, dtype=torch.float32, device=dev) if U is None else U
+    info = torch.zeros(E, dtype=torch.int32, device=dev) if info is None else info
+    nb = gptq_prepare_batched_workspace_bytes(d, E)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev) if ws is None else ws
+    for t, nm in ((perm, "perm"), (U, "U"), (info, "info"), (ws, "ws")):
+        _need(t, nm)
+    _check("gptq_prepare_hinv_batched",
+           load_library().gptq_prepare_hinv_batched(
+               _ptr(S), E, d, ctypes.c_void_p(nt.ctypes.data), float(damp_rel),
+               int(bool(act_order)), _ptr(perm), _ptr(U), _ptr(info), _ptr(ws),
+               ws.numel() * ws.element_size(), _stream(S)))
+    return perm, U, info
+
+
+def gptq_quantize_layer_batched(W: torch.Tensor, U: torch.Tensor, perm=None, bits: int = 4,
+                                group_size: int = 128, block_size: int = 128, codes=None,
+                                scales=None, zeros=None, row_loss=None, ws=None):
+    """gptq_quantize_layer over E stacked layers (W: E x m x d, U: E x d x d,
+    perm: E x d or None) sharing one workspace.  Returns (codes E x m x d,
+    scales E x m x G, zeros E x m x G, row_loss E x m)."""
+    _need(W, "W")
+    _need(U, "U", torch.float32)
+    E, m, d = W.shape
+    dev = W.device
+    G = 1 if group_size in (-1, d) else d // group_size
+    codes = torch.empty(E, m, d, dtype=torch.uint8, device=dev) if codes is None else codes
+    scales = torch.empty(E, m, G, dtype=torch.float16, device=dev) if scales is None else scales
+    zeros = torch.empty(E, m, G, dtype=torch.uint8, device=dev) if zeros is None else zeros
+    row_loss = torch.empty(E, m, dtype=torch.float32, device=dev) if row_loss is None else row_loss
+    nb = gptq_quantize_workspace_bytes(m, d, block_size)
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev) if ws is None else ws
+    if perm is not None:
+        _need(perm, "perm", torch.int32)
+    _check("gptq_quantize_layer_batched",
+           load_library().gptq_quantize_layer_batched(
+               _ptr(W), _wdtype(W), E, m, d, _ptr(U), _ptr(perm), int(bits), int(group_size),
+               int(block_size), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(row_loss), _ptr(ws),
+               ws.numel() * ws.element_size(), _stream(W)))
+    return codes, scales, zeros, row_loss
 
 
 def gptq_quantize_workspace_bytes(d_out: int, d_in: int, block_size: int = 128) -> int:
@@ -397,6 +521,36 @@ def quantize_layer_from_inputs(W: torch.Tensor, X_batches, bits: int = 4, group_
                       zeros=zeros, row_loss=row_loss)
     if pack and bits == 4:
         res.qweight, res.qzeros = gptq_pack_int4(codes, zeros)
+    return res
+
+
+def quantize_moe_from_inputs(W: torch.Tensor, X: torch.Tensor, routes, bits: int = 4,
+                             group_size: int = 128, damp_rel: float = 0.01,
+                             act_order: bool = False, pack: bool = True) -> LayerResult:
+    """GPTQ on every expert of a mixture-of-experts layer at once.
+    W: E x m x d (the experts' weights); X: n x d fp16 calibration tokens;
+    routes: E int32 CUDA tensors, the tokens routed to each expert.  The
+    routed rows are gathered expert-major, the E Hessians accumulated in one
+    launch, prepared in one factorization launch, and the layers swept and
+    packed."""
+    E, m, d = W.shape
+    dev = W.device
+    counts = [int(r.numel()) for r in routes]
+    offsets = [0]
+    for c in counts:
+        offsets.append(offsets[-1] + c)
+    idx = torch.cat([r.to(device=dev, dtype=torch.int32) for r in routes]).contiguous()
+    Xr = gptq_gather_rows(X, idx)
+    S = torch.zeros(E, d, d, dtype=torch.float32, device=dev)
+    gptq_hessian_accumulate_grouped(S, Xr, offsets)
+    perm, U, info = gptq_prepare_hinv_batched(S, counts, damp_rel, act_order)
+    codes, scales, zeros, row_loss = gptq_quantize_layer_batched(
+        W, U, perm if act_order else None, bits, group_size)
+    res = LayerResult(S=S, counts=counts, perm=perm, U=U, info=info, codes=codes, scales=scales,
+                      zeros=zeros, row_loss=row_loss)
+    if pack and bits == 4:
+        qw, qz = gptq_pack_int4(codes.view(E * m, d), zeros.view(E * m, -1))
+        res.qweight, res.qzeros = qw.view(E, m, -1), qz.view(E, m, -1)
     return res
 
 

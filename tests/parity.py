@@ -123,6 +123,17 @@ def teacher_forced_check(Wp64: np.ndarray, U64: np.ndarray, gpu: dict, bits: int
     return int(diff.sum())
 
 
+def mismatch_report(gpu: dict, orc: dict) -> dict:
+    """Where the free-running comparison parts: per row the first mismatching
+    column and the number of mismatches from there to the row's end (the
+    cascade a legitimate tie flip starts)."""
+    mism = gpu["codes"] != orc["codes"]
+    rows = np.nonzero(mism.any(axis=1))[0]
+    first = mism.argmax(axis=1)
+    return dict(weights=int(mism.size), mismatches=int(mism.sum()), rows=int(rows.size),
+                cascades=[(int(r), int(first[r]), int(mism[r].sum())) for r in rows[:20]])
+
+
 def to_np(t: torch.Tensor) -> np.ndarray:
     t = t.detach().cpu()
     if t.dtype == torch.float16:

@@ -154,3 +154,73 @@ def test_validation_rejects_before_launch(lib):
     assert lib.gptq_pack_int4(FAKE, FAKE, 4, 12, 1, FAKE, FAKE, None) == 2
     assert lib.gptq_pack_int4(FAKE, FAKE, 4, 16, 0, FAKE, FAKE, None) == 2
     assert lib.gptq_unpack_int4(FAKE, FAKE, 0, 16, 1, FAKE, FAKE, None) == 2
+
+
+def test_batched_entry_points_validate_before_launch(lib):
+    """The grouped / batched entry points for mixture-of-experts layers
+    reject bad arguments before launching (fake pointers; no GPU)."""
+    import numpy as np
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-side argument checks with fake pointers run where no GPU is visible")
+    I64P = lambda a: ctypes.c_void_p(a.ctypes.data)
+    off = np.array([0, 10, 10, 40], dtype=np.int64)
+    Hg = lib.gptq_hessian_accumulate_grouped
+    assert Hg(None, FAKE, 40, 256, I64P(off), 3, None, None) == 1
+    assert Hg(FAKE, FAKE, 40, 256, None, 3, None, None) == 1
+    assert Hg(MIS, FAKE, 40, 256, I64P(off), 3, None, None) == 1
+    assert Hg(FAKE, FAKE, 40, 200, I64P(off), 3, None, None) == 2
+    assert Hg(FAKE, FAKE, 41, 256, I64P(off), 3, None, None) == 2       # offsets[E] != n
+    bad = np.array([0, 20, 10, 40], dtype=np.int64)                      # decreasing
+    assert Hg(FAKE, FAKE, 40, 256, I64P(bad), 3, None, None) == 2
+    assert Hg(FAKE, FAKE, 40, 256, I64P(off), 0, None, None) == 2
+    # all groups empty: a no-op that counts nothing
+    z = np.zeros(4, dtype=np.int64)
+    seen = np.zeros(3, dtype=np.int64)
+    assert Hg(FAKE, FAKE, 0, 256, I64P(z), 3, I64P(seen), None) == 0
+    assert not seen.any()
+    Gr = lib.gptq_gather_rows
+    assert Gr(None, 10, 256, FAKE, 5, FAKE, None) == 1
+    assert Gr(FAKE, 10, 256, FAKE, 5, MIS, None) == 1
+    assert Gr(FAKE, 10, 252, FAKE, 5, FAKE, None) == 2
+    assert Gr(FAKE, 10, 256, FAKE, -1, FAKE, None) == 2
+    assert Gr(None, 10, 256, None, 0, None, None) == 0                   # nothing to gather
+    ws = G.gptq_prepare_batched_workspace_bytes(256, 3)
+    assert ws >= 3 * 2 * 4 * 256 * 256
+    assert G.gptq_prepare_batched_workspace_bytes(256, 1) == G.gptq_prepare_workspace_bytes(256)
+    nt = np.array([100, 50, 7], dtype=np.int64)
+    Pb = lib.gptq_prepare_hinv_batched
+    assert Pb(FAKE, 3, 256, None, 0.01, 0, None, FAKE, FAKE, FAKE, ws, None) == 1
+    assert Pb(FAKE, 3, 256, I64P(nt), 0.01, 1, None, FAKE, FAKE, FAKE, ws, None) == 1
+    assert Pb(FAKE, 3, 256, I64P(nt), 0.01, 0, None, FAKE, FAKE, FAKE, ws - 1, None) == 1
+    assert Pb(FAKE, 0, 256, I64P(nt), 0.01, 0, None, FAKE, FAKE, FAKE, ws, None) == 2
+    nt0 = np.array([100, 0, 7], dtype=np.int64)
+    assert Pb(FAKE, 3, 256, I64P(nt0), 0.01, 0, None, FAKE, FAKE, FAKE, ws, None) == 2
+    assert Pb(FAKE, 3, 200, I64P(nt), 0.01, 0, None, FAKE, FAKE, FAKE, ws, None) == 2
+    wq = G.gptq_quantize_workspace_bytes(64, 256, 128)
+    Qb = lib.gptq_quantize_layer_batched
+    assert Qb(FAKE, 1, 0, 64, 256, FAKE, None, 4, 128, 128, FAKE, FAKE, FAKE, None, FAKE, wq,
+              None) == 2
+    assert Qb(None, 1, 2, 64, 256, FAKE, None, 4, 128, 128, FAKE, FAKE, FAKE, None, FAKE, wq,
+              None) == 1
+    assert Qb(FAKE, 1, 2, 64, 256, FAKE, None, 4, 96, 128, FAKE, FAKE, FAKE, None, FAKE, wq,
+              None) == 4
+    # a layer slice that would leave the next one misaligned: 3 rows of fp16 scales
+    assert Qb(FAKE, 1, 2, 3, 256, FAKE, None, 4, 128, 128, FAKE, FAKE, FAKE, None, FAKE, wq,
+              None) == 2
+
+
+def test_static_entry_checks_arguments_like_the_workspace_one(lib):
+    """gptq_prepare_hinv_static returns the status gptq_prepare_hinv gives for
+    the same bad argument, before its size limit and its scratch lookup."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-side argument checks with fake pointers run where no GPU is visible")
+    S = lib.gptq_prepare_hinv_static
+    assert S(None, 2048, 10, 0.01, 0, None, FAKE, FAKE, None) == 1
+    assert S(FAKE, 2048, 10, 0.01, 1, None, FAKE, FAKE, None) == 1
+    assert S(FAKE, 2048, 10, -1.0, 0, None, FAKE, FAKE, None) == 1
+    assert S(MIS, 512, 10, 0.01, 0, None, FAKE, FAKE, None) == 1
+    assert S(FAKE, 300, 10, 0.01, 0, None, FAKE, FAKE, None) == 2
+    assert S(FAKE, 512, 0, 0.01, 0, None, FAKE, FAKE, None) == 2
+    assert S(FAKE, 2048, 10, 0.01, 0, None, FAKE, FAKE, None) == 2    # beyond the scratch

@@ -8,8 +8,28 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from tests import parity as P
-from tests.test_parity_gpu import _check_layer, _gauss_x, _weights
+from tests.test_parity_gpu import _check_layer, _gauss_x, _gpu_layer, _weights
+
+
+def _diagnose(W, X, bits, gs, act):
+    """The teacher-forced tie check and the mismatch cascades, printed before
+    _check_layer asserts the tolerances (a failure then shows whether the
+    disagreements are near-ties and how far each one cascades)."""
+    g = _gpu_layer(W, X, bits, gs, act)
+    S_gpu = P.mirror_upper(g["S"])
+    W64 = W.double().numpy()
+    ref = oracle.gptq_layer(W64, S_gpu, X.shape[0], bits, gs, 0.01, act)
+    Wp = np.ascontiguousarray(W64[:, ref["perm"]])
+    rep = {}
+    try:
+        P.teacher_forced_check(Wp, ref["U"], g, bits, gs, report=rep)
+        rep["forced_check"] = "passed"
+    except AssertionError as e:
+        rep["forced_check"] = f"FAILED: {e}"
+    rep.update(P.mismatch_report(g, ref))
+    print("diagnosis", (bits, gs, act), rep)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,6 +57,7 @@ def test_sweep_degenerate_rows(bits, gs, act, dtype):
     m, d, n = 200, 512, 1500
     W = _degenerate_rows(_weights(m, d, dtype, 900 + bits + gs), gs)
     X = _gauss_x(n, d, 5, 40.0, 901 + bits)
+    _diagnose(W, X, bits, gs, act)
     st, g, ref = _check_layer(W, X, bits, gs, act)
     # the all-zero row quantizes to exact zeros: codes equal the zero points
     # and every group's scale is the [-1, 1] range's
@@ -57,5 +78,6 @@ def test_sweep_bits8_tolerances_hold_on_outlier_inputs():
     most often part at ties."""
     W = _weights(384, 1024, torch.float16, 77)
     X = _gauss_x(3000, 1024, 10, 60.0, 78)
+    _diagnose(W, X, 8, 128, False)
     st, _, _ = _check_layer(W, X, 8, 128, False)
     print("bits 8:", st)

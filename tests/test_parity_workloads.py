@@ -125,31 +125,43 @@ def test_dense_workload_layer(workload, layer):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("expert", range(8))
-def test_moe_expert(expert):
-    """Every expert of the MoE layer on its own routed tokens (the coldest
-    capped at 2048, rank-deficient before damping)."""
+@pytest.fixture(scope="module")
+def moe8_batched():
+    """The whole MoE layer through the batched path, as bench.py runs it:
+    routed rows gathered expert-major, one grouped Hessian launch, one
+    factorization launch for the eight experts, the batched sweep, one pack."""
     wl = inputs.WORKLOADS["moe8"]
-    X, lists = _moe_inputs()
-    counts = [len(x) for x in lists]
-    assert sum(counts) <= 2 * X.shape[0] and min(counts) == wl.cold_cap
+    spec0 = wl.layers[0]
+    X = inputs.calibration_x(spec0, device=DEV)
+    lists = inputs.moe_routing(X.shape[0], wl.n_experts, wl.zipf_s, wl.top_k, wl.cold_cap,
+                               spec0.seed)
+    W = torch.stack([inputs.weights(sp, device=DEV) for sp in wl.layers]).contiguous()
+    routes = [torch.as_tensor(np.asarray(r), dtype=torch.int32, device=DEV) for r in lists]
+    res = G.quantize_moe_from_inputs(W, X, routes)
+    torch.cuda.synchronize()
+    assert G.gptq_device_status(reset=True) == 0
+    assert not P.to_np(res.info).any()
+    out = dict(wl=wl, X=X, lists=lists, W=W, res=res)
+    yield out
+    del out, X, W, res
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("expert", range(8))
+def test_moe_expert(moe8_batched, expert):
+    """Every expert of the MoE layer on its own routed tokens (the coldest
+    capped at 2048, rank-deficient before damping), all eight quantized by
+    the batched entry points in one pass."""
+    b = moe8_batched
+    wl, res = b["wl"], b["res"]
+    counts = [len(x) for x in b["lists"]]
+    assert sum(counts) <= 2 * b["X"].shape[0] and min(counts) == wl.cold_cap
     spec = wl.layers[expert]
-    W = inputs.weights(spec, device=DEV)
-    Xe = X.index_select(0, torch.as_tensor(lists[expert], device=DEV)).contiguous()
-    g = _run_layer(W, Xe, Xe.shape[0], False)
-    st = _check(spec, W, Xe, g, 200 + expert)
-    print("expert", expert, "tokens", counts[expert], st)
-
-
-_MOE = {}
-
-
-def _moe_inputs():
-    if "X" not in _MOE:
-        wl = inputs.WORKLOADS["moe8"]
-        spec0 = wl.layers[0]
-        X = inputs.calibration_x(spec0, device=DEV)
-        _MOE["X"] = X
-        _MOE["lists"] = inputs.moe_routing(X.shape[0], wl.n_experts, wl.zipf_s, wl.top_k,
-                                           wl.cold_cap, spec0.seed)
-    return _MOE["X"], _MOE["lists"]
+    Xe = b["X"].index_select(0, torch.as_tensor(b["lists"][expert], device=DEV)).contiguous()
+    e = expert
+    g = dict(S=P.to_np(res.S[e]), perm=P.to_np(res.perm[e]), U=P.to_np(res.U[e]),
+             codes=P.to_np(res.codes[e]), scales=P.to_np(res.scales[e]),
+             zeros=P.to_np(res.zeros[e]), loss=P.to_np(res.row_loss[e]),
+             qw=P.to_np(res.qweight[e]).view(np.uint32), qz=P.to_np(res.qzeros[e]))
+    st = _check(spec, b["W"][e], Xe, g, 200 + e)
+    print("expert", e, "tokens", counts[e], st)
