@@ -19,7 +19,8 @@ float64, no blocking) and cites the passage it follows:
                       sec. 三 loop; "校准艺术" sec. 2.2 steps 1-5).
 * ``rtn``          -- round-to-nearest group min-max ("校准艺术" sec. 2.1).
 * ``pack_int4``/``unpack_int4`` -- the 66.5 B / 128-weight storage format
-                      ("INT4/INT8 量化推理" sec. 一).
+                      ("INT4/INT8 量化推理" sec. 一); ``pack_bits``/``unpack_bits``
+                      the same layout as one bit stream per row for 2..8 bits.
 * ``trace_quadratic`` -- tr(D H D^T), the layer loss of sec. 三 of that page.
 * ``w4a16_matmul`` -- y = x Q^T from the packed layer (weight-only INT4 with
                       fp16 activations, "INT4/INT8 量化推理" sec. 六).
@@ -71,6 +72,10 @@ def _load():
         lib.orc_pack_int4.restype = None
         lib.orc_unpack_int4.argtypes = [P, P, I64, I64, I64, P, P]
         lib.orc_unpack_int4.restype = None
+        lib.orc_pack_bits.argtypes = [P, P, I64, I64, I64, ctypes.c_int, P, P]
+        lib.orc_pack_bits.restype = None
+        lib.orc_unpack_bits.argtypes = [P, P, I64, I64, I64, ctypes.c_int, P, P]
+        lib.orc_unpack_bits.restype = None
         lib.orc_trace_quadratic.argtypes = [P, P, I64, I64]
         lib.orc_trace_quadratic.restype = ctypes.c_double
         lib.orc_num_threads.argtypes = []
@@ -319,6 +324,32 @@ def unpack_int4(qweight: np.ndarray, qzeros: np.ndarray, d: int, G: int):
     codes = np.empty((m, d), np.uint8)
     zeros = np.empty((m, G), np.uint8)
     _load().orc_unpack_int4(_p(qweight), _p(qzeros), m, d, G, _p(codes), _p(zeros))
+    return codes, zeros
+
+
+def pack_bits(codes: np.ndarray, zeros: np.ndarray, bits: int):
+    """b-bit storage (b in 2..8): each row's codes as one little-endian bit
+    stream in uint32 words (d * b / 32 per row), its zero points as a second
+    stream in bytes (ceil(G b / 8) per row).  b = 4 is the INT4 layout of
+    ``pack_int4`` ("INT4/INT8 量化推理" sec. 一); other widths extend it."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    zeros = np.ascontiguousarray(zeros, dtype=np.uint8)
+    m, d = codes.shape
+    G = zeros.shape[1]
+    assert (d * bits) % 32 == 0 and 2 <= bits <= 8
+    qweight = np.empty((m, d * bits // 32), np.uint32)
+    qzeros = np.empty((m, (G * bits + 7) // 8), np.uint8)
+    _load().orc_pack_bits(_p(codes), _p(zeros), m, d, G, int(bits), _p(qweight), _p(qzeros))
+    return qweight, qzeros
+
+
+def unpack_bits(qweight: np.ndarray, qzeros: np.ndarray, d: int, G: int, bits: int):
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint32)
+    qzeros = np.ascontiguousarray(qzeros, dtype=np.uint8)
+    m = qweight.shape[0]
+    codes = np.empty((m, d), np.uint8)
+    zeros = np.empty((m, G), np.uint8)
+    _load().orc_unpack_bits(_p(qweight), _p(qzeros), m, d, G, int(bits), _p(codes), _p(zeros))
     return codes, zeros
 
 

@@ -430,6 +430,65 @@ void orc_unpack_int4(const uint32_t* qweight, const uint8_t* qzeros, int64_t m, 
 }
 
 /* ------------------------------------------------------------------------ */
+/* b-bit packing (b in 2..8) for the other widths the INT4/INT8 page names   */
+/* beside the 4-bit storage of its sec. 一: each row's codes form one        */
+/* little-endian bit stream, code k in bits [b k, b k + b), stored as uint32 */
+/* words; the row's zero points form a second stream stored as bytes, its    */
+/* last byte padded with zero bits.  For b = 4 this is the INT4 layout.      */
+/* ------------------------------------------------------------------------ */
+
+void orc_pack_bits(const uint8_t* codes, const uint8_t* zeros, int64_t m, int64_t d, int64_t G,
+                   int bits, uint32_t* qweight, uint8_t* qzeros)
+{
+    int64_t nw = d * bits / 32, nb = (G * bits + 7) / 8;
+    uint32_t mask = (1u << bits) - 1u;
+    for (int64_t r = 0; r < m; ++r) {
+        for (int64_t w = 0; w < nw; ++w) qweight[r * nw + w] = 0;
+        for (int64_t k = 0; k < d; ++k) {
+            uint64_t bit = (uint64_t)k * (uint64_t)bits;
+            uint32_t c = codes[r * d + k] & mask;
+            for (int t = 0; t < bits; ++t) {            /* one bit at a time */
+                uint64_t pos = bit + (uint64_t)t;
+                if ((c >> t) & 1u) qweight[r * nw + (int64_t)(pos / 32)] |= 1u << (pos % 32);
+            }
+        }
+        for (int64_t b = 0; b < nb; ++b) qzeros[r * nb + b] = 0;
+        for (int64_t gi = 0; gi < G; ++gi) {
+            uint64_t bit = (uint64_t)gi * (uint64_t)bits;
+            uint32_t z = zeros[r * G + gi] & mask;
+            for (int t = 0; t < bits; ++t) {
+                uint64_t pos = bit + (uint64_t)t;
+                if ((z >> t) & 1u) qzeros[r * nb + (int64_t)(pos / 8)] |= (uint8_t)(1u << (pos % 8));
+            }
+        }
+    }
+}
+
+void orc_unpack_bits(const uint32_t* qweight, const uint8_t* qzeros, int64_t m, int64_t d,
+                     int64_t G, int bits, uint8_t* codes, uint8_t* zeros)
+{
+    int64_t nw = d * bits / 32, nb = (G * bits + 7) / 8;
+    for (int64_t r = 0; r < m; ++r) {
+        for (int64_t k = 0; k < d; ++k) {
+            uint32_t c = 0;
+            for (int t = 0; t < bits; ++t) {
+                uint64_t pos = (uint64_t)k * (uint64_t)bits + (uint64_t)t;
+                c |= ((qweight[r * nw + (int64_t)(pos / 32)] >> (pos % 32)) & 1u) << t;
+            }
+            codes[r * d + k] = (uint8_t)c;
+        }
+        for (int64_t gi = 0; gi < G; ++gi) {
+            uint32_t z = 0;
+            for (int t = 0; t < bits; ++t) {
+                uint64_t pos = (uint64_t)gi * (uint64_t)bits + (uint64_t)t;
+                z |= ((uint32_t)(qzeros[r * nb + (int64_t)(pos / 8)] >> (pos % 8)) & 1u) << t;
+            }
+            zeros[r * G + gi] = (uint8_t)z;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Layer loss ([P3] sec. 三 objective, [P5] sec. 一 "F-norm squared"):       */
 /* tr(D H D^T) with D = W - Q, for a symmetric H (fp64).                     */
 /* ------------------------------------------------------------------------ */

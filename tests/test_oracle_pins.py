@@ -124,6 +124,39 @@ def test_pack_hand_examples_and_roundtrip():
         assert np.array_equal(c2, codes) and np.array_equal(z2, zeros)
 
 
+def test_pack_bits_hand_examples_roundtrip_and_int4_layout():
+    """b-bit packing: hand-worked words and bytes (tests/golden), the round
+    trip at every width, the storage arithmetic, and b = 4 equal to the INT4
+    layout (pinned on its own by pack_examples.txt)."""
+    for row in _read_golden("pack_bits_examples.txt"):
+        kind, bits, vals, packed = [p.strip() for p in row.split("|")]
+        b = int(bits)
+        v = [int(x) for x in vals.split(",")]
+        want = [int(x, 16) for x in packed.split(",")]
+        if kind == "codes":
+            d = len(v)
+            qw, _ = oracle.pack_bits(np.array([v], np.uint8), np.zeros((1, 1), np.uint8), b)
+            assert [int(x) for x in qw[0]] == want + [0] * (qw.shape[1] - len(want))
+        else:
+            _, qz = oracle.pack_bits(np.zeros((1, 32), np.uint8), np.array([v], np.uint8), b)
+            assert [int(x) for x in qz[0]] == want
+    rng = _rng(6)
+    for b in (2, 3, 4, 5, 8):
+        for (m, d, G) in [(3, 256, 2), (5, 384, 3), (2, 32, 1), (4, 4096, 32)]:
+            codes = rng.integers(0, 1 << b, (m, d), dtype=np.uint8)
+            zeros = rng.integers(0, 1 << b, (m, G), dtype=np.uint8)
+            qw, qz = oracle.pack_bits(codes, zeros, b)
+            assert qw.nbytes == m * d * b // 8 and qz.shape[1] == (G * b + 7) // 8
+            c2, z2 = oracle.unpack_bits(qw, qz, d, G, b)
+            assert np.array_equal(c2, codes) and np.array_equal(z2, zeros)
+            if b == 4:
+                q4w, q4z = oracle.pack_int4(codes, zeros)
+                assert np.array_equal(qw, q4w) and np.array_equal(qz, q4z)
+    # storage: b bits per weight + (b + 16) bits per group of 128
+    for b, total in ((3, 50.375), (4, 66.5), (8, 131.0)):
+        assert (128 * b + b + 16) / 8 == total
+
+
 def test_w4a16_hand_example_and_one_hot_columns():
     rows = {}
     cases = []
