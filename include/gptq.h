@@ -265,10 +265,14 @@ int gptq_prepare_hinv_batched(const float* S, int64_t n_mats, int64_t d, const i
  * codes: d_out x d_in uint8 output, sweep order (code of column perm[k] at k).
  * scales: d_out x G fp16 output (G = d_in / group_size), zeros: d_out x G uint8.
  * row_loss: d_out fp32 output or NULL: sum_j E_j^2 (= tr(D Hd D^T) per row).
- * bits in {2,3,4,8}; group_size in {32, 64, 128}, or -1 (or d_in) for one
- * group per row (G = 1: its parameters come from the row before any
- * correction, which is what "at the group's first column" means for column
- * 0); block_size == 128.
+ * bits in {2,3,4,8}; group_size in {32, 64, 128}; or a multiple of 128
+ * dividing d_in that divides 512 or is a multiple of 512 (256, 512, 1024,
+ * ...: such a group never straddles the 512-column deferred-update block,
+ * so at its first column every column of the group holds every earlier
+ * column's correction and its parameters are taken there, as in the
+ * unblocked sweep); or -1 (or d_in) for one group per row (G = 1: its
+ * parameters come from the row before any correction, which is what "at the
+ * group's first column" means for column 0); block_size == 128.
  * Requires d_in % 128 == 0, 128 <= d_in <= 32768, 1 <= d_out <= 2^24.
  */
 size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, int block_size);
@@ -335,6 +339,28 @@ int gptq_unpack_int4(const uint32_t* qweight, const uint8_t* qzeros, int64_t d_o
                      void* stream);
 
 /*
+ * Pack b-bit codes -- the storage of "INT4/INT8 量化推理" sec. 一 for the
+ * page's other widths (INT8 beside INT4; 2 and 3 bits for the low-bit
+ * cases), read as one little-endian bit stream per row:
+ *   code k of row r occupies bits [b k, b k + b) of row r's stream, stored
+ *   as d_in * b / 32 uint32 words (word w = bits [32 w, 32 w + 32));
+ *   zero point g of row r occupies bits [b g, b g + b) of a second stream,
+ *   stored as ceil(G b / 8) bytes (the last byte padded with zero bits).
+ * For b = 4 this is exactly gptq_pack_int4's layout (66.5 B per 128 weights
+ * with the fp16 scale); b = 3 gives 50.375 B, b = 8 131 B per 128 weights.
+ * codes: d_out x d_in uint8 (values masked to b bits), zeros: d_out x G.
+ * qweight: d_out x (d_in b / 32) uint32 out (4-byte aligned), qzeros:
+ * d_out x ceil(G b / 8) uint8 out.  bits in 2..8 (else UNSUPPORTED);
+ * requires d_in % 32 == 0, 1 <= G <= d_in, codes 16-byte aligned.
+ */
+int gptq_pack_bits(const uint8_t* codes, const uint8_t* zeros, int64_t d_out, int64_t d_in,
+                   int64_t n_groups, int bits, uint32_t* qweight, uint8_t* qzeros, void* stream);
+
+/* Inverse of gptq_pack_bits (bit-exact round trip). */
+int gptq_unpack_bits(const uint32_t* qweight, const uint8_t* qzeros, int64_t d_out, int64_t d_in,
+                     int64_t n_groups, int bits, uint8_t* codes, uint8_t* zeros, void* stream);
+
+/*
  * Weight-only INT4 product on the packed layer (W4A16) -- "INT4/INT8 量化推理"
  * sec. 六 (weights in 4 bits, activations in fp16), on the storage of sec. 一
  * of the same page:
@@ -357,7 +383,8 @@ int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t* qweight,
  * rounded on its own) with the min-max group quantizer of "校准艺术" sec. 2.1:
  * the same group parameters and codes as gptq_quantize_layer, taken on the
  * original W with no error feedback.  Same argument meaning and limits as
- * gptq_quantize_layer (natural column order, no U, no workspace).
+ * gptq_quantize_layer (natural column order, no U, no workspace), except
+ * group_size: 32, 64, 128, any multiple of 128 dividing d_in, or -1.
  */
 int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bits,
                  int group_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,

@@ -88,6 +88,94 @@ static unsigned grid_for(int64_t n, int threads)
     return (unsigned)std::max<int64_t>(1, std::min<int64_t>(ceil_div(n, threads), 148 * 32));
 }
 
+// b-bit storage for the other widths (b = 2..8): each row's codes form one
+// little-endian bit stream, code k in bits [b k, b k + b), stored as uint32
+// words; b = 4 is the INT4 layout above.  One thread per 32-code chunk of a
+// row: two 16-byte loads of codes, b words out (32 codes = 32 b bits).
+template <int B>
+__global__ void pack_bits_kernel(const uint8_t* __restrict__ codes, int64_t chunks,
+                                 uint32_t* __restrict__ qweight)
+{
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks;
+         i += int64_t(gridDim.x) * blockDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(codes + 32 * i);
+    const uint4 v0 = src[0], v1 = src[1];
+    const uint32_t c4[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t wd[B];
+#pragma unroll
+    for (int t = 0; t < B; ++t) wd[t] = 0u;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const uint32_t c = (c4[k >> 2] >> (8 * (k & 3))) & ((1u << B) - 1u);
+        const int bit = B * k, w = bit >> 5, sh = bit & 31;
+        wd[w] |= c << sh;
+        if (sh + B > 32) wd[w + 1] |= c >> (32 - sh);
+    }
+    uint32_t* dst = qweight + int64_t(B) * i;
+#pragma unroll
+    for (int t = 0; t < B; ++t) dst[t] = wd[t];
+    }
+}
+
+template <int B>
+__global__ void unpack_bits_kernel(const uint32_t* __restrict__ qweight, int64_t chunks,
+                                   uint8_t* __restrict__ codes)
+{
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks;
+         i += int64_t(gridDim.x) * blockDim.x) {
+    uint32_t wd[B + 1];
+#pragma unroll
+    for (int t = 0; t < B; ++t) wd[t] = qweight[int64_t(B) * i + t];
+    wd[B] = 0u;
+    uint32_t c4[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) c4[q] = 0u;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const int bit = B * k, w = bit >> 5, sh = bit & 31;
+        uint32_t c = wd[w] >> sh;
+        if (sh + B > 32) c |= wd[w + 1] << (32 - sh);
+        c4[k >> 2] |= (c & ((1u << B) - 1u)) << (8 * (k & 3));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(codes + 32 * i);
+    dst[0] = make_uint4(c4[0], c4[1], c4[2], c4[3]);
+    dst[1] = make_uint4(c4[4], c4[5], c4[6], c4[7]);
+    }
+}
+
+// Zero points: the row's stream of G b-bit values in ceil(G b / 8) bytes;
+// one thread per output byte (pack) or per zero point (unpack).
+__global__ void pack_zero_bits_kernel(const uint8_t* __restrict__ zeros, int64_t m, int64_t G,
+                                      int b, uint8_t* __restrict__ qzeros)
+{
+    const int64_t nb = (G * b + 7) / 8;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < m * nb;
+         i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / nb, byte = i - r * nb;
+    uint32_t v = 0u;
+    for (int64_t g = (8 * byte) / b; g < G && g * b < 8 * byte + 8; ++g) {
+        const uint32_t z = zeros[r * G + g] & ((1u << b) - 1u);
+        const int64_t sh = g * b - 8 * byte;           // may be negative
+        v |= sh >= 0 ? (z << sh) : (z >> (-sh));
+    }
+    qzeros[i] = uint8_t(v & 0xffu);
+    }
+}
+
+__global__ void unpack_zero_bits_kernel(const uint8_t* __restrict__ qzeros, int64_t m, int64_t G,
+                                        int b, uint8_t* __restrict__ zeros)
+{
+    const int64_t nb = (G * b + 7) / 8;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < m * G;
+         i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / G, g = i - r * G;
+    const int64_t bit = g * b, byte = bit / 8, sh = bit % 8;
+    uint32_t v = uint32_t(qzeros[r * nb + byte]) >> sh;
+    if (sh + b > 8) v |= uint32_t(qzeros[r * nb + byte + 1]) << (8 - sh);
+    zeros[i] = uint8_t(v & ((1u << b) - 1u));
+    }
+}
+
 }  // namespace gptq
 
 extern "C" int gptq_pack_int4(const uint8_t* codes, const uint8_t* zeros, int64_t d_out,
@@ -134,3 +222,64 @@ extern "C" int gptq_unpack_int4(const uint32_t* qweight, const uint8_t* qzeros, 
     return launch_status();
 }
 
+
+extern "C" int gptq_pack_bits(const uint8_t* codes, const uint8_t* zeros, int64_t d_out,
+                              int64_t d_in, int64_t n_groups, int bits, uint32_t* qweight,
+                              uint8_t* qzeros, void* stream)
+{
+    using namespace gptq;
+    if (!codes || !zeros || !qweight || !qzeros) return GPTQ_ERR_INVALID_ARG;
+    if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(qweight) & 3u))
+        return GPTQ_ERR_INVALID_ARG;
+    if (bits < 2 || bits > 8) return GPTQ_ERR_UNSUPPORTED;
+    if (d_out < 1 || d_in < 32 || d_in % 32 != 0 || n_groups < 1 || n_groups > d_in)
+        return GPTQ_ERR_SHAPE;
+    cudaStream_t st = as_stream(stream);
+    const int64_t chunks = d_out * d_in / 32;
+    KernelTimer kt(kKPack, st);
+    switch (bits) {
+        case 2: pack_bits_kernel<2><<<grid_for(chunks, 256), 256, 0, st>>>(codes, chunks, qweight); break;
+        case 3: pack_bits_kernel<3><<<grid_for(chunks, 256), 256, 0, st>>>(codes, chunks, qweight); break;
+        case 4: pack_bits_kernel<4><<<grid_for(chunks, 256), 256, 0, st>>>(codes, chunks, qweight); break;
+        case 5: pack_bits_kernel<5><<<grid_for(chunks, 256), 256, 0, st>>>(codes, chunks, qweight); break;
+        case 6: pack_bits_kernel<6><<<grid_for(chunks, 256), 256, 0, st>>>(codes, chunks, qweight); break;
+        case 7: pack_bits_kernel<7><<<grid_for(chunks, 256), 256, 0, st>>>(codes, chunks, qweight); break;
+        default: pack_bits_kernel<8><<<grid_for(chunks, 256), 256, 0, st>>>(codes, chunks, qweight); break;
+    }
+    count_launches();
+    const int64_t nb = (n_groups * bits + 7) / 8;
+    pack_zero_bits_kernel<<<grid_for(d_out * nb, 256), 256, 0, st>>>(zeros, d_out, n_groups, bits,
+                                                                     qzeros);
+    count_launches();
+    return launch_status();
+}
+
+extern "C" int gptq_unpack_bits(const uint32_t* qweight, const uint8_t* qzeros, int64_t d_out,
+                                int64_t d_in, int64_t n_groups, int bits, uint8_t* codes,
+                                uint8_t* zeros, void* stream)
+{
+    using namespace gptq;
+    if (!codes || !zeros || !qweight || !qzeros) return GPTQ_ERR_INVALID_ARG;
+    if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(qweight) & 3u))
+        return GPTQ_ERR_INVALID_ARG;
+    if (bits < 2 || bits > 8) return GPTQ_ERR_UNSUPPORTED;
+    if (d_out < 1 || d_in < 32 || d_in % 32 != 0 || n_groups < 1 || n_groups > d_in)
+        return GPTQ_ERR_SHAPE;
+    cudaStream_t st = as_stream(stream);
+    const int64_t chunks = d_out * d_in / 32;
+    KernelTimer kt(kKUnpack, st);
+    switch (bits) {
+        case 2: unpack_bits_kernel<2><<<grid_for(chunks, 256), 256, 0, st>>>(qweight, chunks, codes); break;
+        case 3: unpack_bits_kernel<3><<<grid_for(chunks, 256), 256, 0, st>>>(qweight, chunks, codes); break;
+        case 4: unpack_bits_kernel<4><<<grid_for(chunks, 256), 256, 0, st>>>(qweight, chunks, codes); break;
+        case 5: unpack_bits_kernel<5><<<grid_for(chunks, 256), 256, 0, st>>>(qweight, chunks, codes); break;
+        case 6: unpack_bits_kernel<6><<<grid_for(chunks, 256), 256, 0, st>>>(qweight, chunks, codes); break;
+        case 7: unpack_bits_kernel<7><<<grid_for(chunks, 256), 256, 0, st>>>(qweight, chunks, codes); break;
+        default: unpack_bits_kernel<8><<<grid_for(chunks, 256), 256, 0, st>>>(qweight, chunks, codes); break;
+    }
+    count_launches();
+    unpack_zero_bits_kernel<<<grid_for(d_out * n_groups, 256), 256, 0, st>>>(qzeros, d_out,
+                                                                           n_groups, bits, zeros);
+    count_launches();
+    return launch_status();
+}

@@ -279,18 +279,22 @@ rtn_kernel(const T* __restrict__ W, int64_t m, int64_t d, float maxqf,
     }
 }
 
-// Static group parameters: one warp per (row, group) of the working copy
-// (sweep order, before any correction); min/max over the group with the
+// Group parameters from the working copy: one warp per (row, group) for the
+// groups g_first .. g_first + g_count - 1; min/max over the group with the
 // range including 0, then the same group_params as the sweep and RTN.
+// Called on the uncorrected copy for static groups (all groups at once), or
+// at a wide dynamic group's first column, when every column of the group has
+// received every earlier column's correction (see quantize_impl).
 __global__ void __launch_bounds__(256)
 static_params_kernel(const float* __restrict__ Wk, int64_t m, int64_t d, int64_t gsz,
-                     float maxqf, __half* __restrict__ scales, uint8_t* __restrict__ zeros)
+                     int64_t g_first, int64_t g_count, float maxqf, __half* __restrict__ scales,
+                     uint8_t* __restrict__ zeros)
 {
     const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t G = d / gsz;
-    if (wid >= m * G) return;               // whole warp exits together
-    const int64_t row = wid / G, gi = wid - row * G;
+    if (wid >= m * g_count) return;         // whole warp exits together
+    const int64_t row = wid / g_count, gi = g_first + (wid - row * g_count);
     const float* p = Wk + row * d + gi * gsz;
     float mn = 0.f, mx = 0.f;
     for (int64_t c = 4 * lane; c < gsz; c += 128) {
@@ -305,6 +309,44 @@ static_params_kernel(const float* __restrict__ Wk, int64_t m, int64_t d, int64_t
     }
     if (lane == 0) {
         const GroupQ gq = group_params(mn, mx, maxqf);
+        scales[row * G + gi] = gq.h;
+        zeros[row * G + gi] = (uint8_t)gq.z;
+    }
+}
+
+// Round-to-nearest for groups wider than 128 columns (or one group per
+// row): one warp per (row, group), min/max in a first pass over the group,
+// the codes in a second.
+template <typename T>
+__global__ void __launch_bounds__(256)
+rtn_wide_kernel(const T* __restrict__ W, int64_t m, int64_t d, int64_t gsz, float maxqf,
+                uint8_t* __restrict__ codes, __half* __restrict__ scales,
+                uint8_t* __restrict__ zeros)
+{
+    const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t G = d / gsz;
+    if (wid >= m * G) return;               // whole warp exits together
+    const int64_t row = wid / G, gi = wid - row * G;
+    const T* p = W + row * d + gi * gsz;
+    float mn = 0.f, mx = 0.f;
+    for (int64_t c = 4 * lane; c < gsz; c += 128) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { const float x = float(p[c + q]); mn = fminf(mn, x); mx = fmaxf(mx, x); }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+    }
+    const GroupQ gq = group_params(mn, mx, maxqf);
+    for (int64_t c = 4 * lane; c < gsz; c += 128) {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) packed |= uint32_t(quant_code(float(p[c + q]), gq, maxqf)) << (8 * q);
+        *reinterpret_cast<uint32_t*>(codes + row * d + gi * gsz + c) = packed;
+    }
+    if (lane == 0) {
         scales[row * G + gi] = gq.h;
         zeros[row * G + gi] = (uint8_t)gq.z;
     }
@@ -361,16 +403,24 @@ extern "C" size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, int
 
 namespace gptq {
 
-// Group sizes the sweep takes: dynamic groups (parameters at each group's
-// first column from the corrected row) in {32, 64, 128}; static groups
-// (parameters from the rows before the sweep) in {32, 64} or any multiple of
-// 128 dividing d; one group per row (-1 or d) is the static case, since at
-// column 0 no correction has happened yet.
+// Group sizes the sweep takes.  Dynamic groups (parameters at each group's
+// first column from the corrected row): 32, 64, 128, and the multiples of
+// 128 dividing d that either divide the 512-column outer block or are
+// multiples of it -- those groups never straddle an outer-block boundary
+// from the inside, so at a group's first column every column of the group
+// has received every earlier column's correction (the near updates cover
+// the rest of the outer block, the far updates everything beyond a finished
+// outer block) and the parameters can be taken from the working copy there.
+// Static groups (parameters from the rows before the sweep): 32, 64 or any
+// multiple of 128 dividing d.  One group per row (-1 or d) is the same in
+// both readings, since at column 0 no correction has happened yet.
 static int sweep_group_size(int64_t d, int group_size, bool static_groups, int64_t* gsz)
 {
     if (group_size == -1 || group_size == d) { *gsz = d; return GPTQ_OK; }
     if (group_size == 32 || group_size == 64 || group_size == 128) { *gsz = group_size; return GPTQ_OK; }
-    if (static_groups && group_size > 128 && group_size % 128 == 0 && d % group_size == 0) {
+    const int64_t ob = int64_t(UPD_OUTER) * SW_B;
+    if (group_size > 128 && group_size % 128 == 0 && d % group_size == 0 &&
+        (static_groups || ob % group_size == 0 || group_size % ob == 0)) {
         *gsz = group_size;
         return GPTQ_OK;
     }
@@ -389,7 +439,11 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
     int64_t gsz = 0;
     rc = sweep_group_size(d_in, group_size, static_groups, &gsz);
     if (rc != GPTQ_OK) return rc;
-    const bool stat = static_groups || gsz == d_in;
+    // the sweep reads the group parameters instead of reducing them when they
+    // are static, one per row, or dynamic but wider than a block (taken just
+    // in time at each group's first block by static_params_kernel)
+    const bool wide = !static_groups && gsz > SW_B && gsz < d_in;
+    const bool stat = static_groups || gsz == d_in || wide;
     if (block_size != SW_B) return GPTQ_ERR_UNSUPPORTED;
     if (!aligned16(W) || !aligned16(U) || !aligned16(codes) || !aligned16(scales) ||
         !aligned16(zeros) || !aligned16(ws) || (perm && !aligned16(perm)) ||
@@ -415,11 +469,11 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
     }
     const float maxqf = float((1 << bits) - 1);
     __half* sc = reinterpret_cast<__half*>(scales);
-    if (stat) {
+    if (stat && !wide) {
         const int64_t warps = m * (d / gsz);
         KernelTimer kt(kKStaticParams, st);
         static_params_kernel<<<(unsigned)ceil_div(warps * 32, 256), 256, 0, st>>>(
-            w.Wk, m, d, gsz, maxqf, sc, zeros);
+            w.Wk, m, d, gsz, 0, d / gsz, maxqf, sc, zeros);
         count_launches();
     }
     {
@@ -442,6 +496,12 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
         const int64_t ecol = j0 - ob0;                                     // E column of this block
         float* Eh = w.upd.Eh + ecol;
         float* El = w.upd.El + ecol;
+        if (wide && j0 % gsz == 0) {            // a wide dynamic group starts here
+            KernelTimer kt(kKStaticParams, st);
+            static_params_kernel<<<(unsigned)ceil_div(m * 32, 256), 256, 0, st>>>(
+                w.Wk, m, d, gsz, j0 / gsz, 1, maxqf, sc, zeros);
+            count_launches();
+        }
 #define GPTQ_SWEEP(GSV, STAT)                                                                   \
         launch_sweep<GSV, STAT>(grid, smem, st, w.Wk, U, m, d, gsz, j0, maxqf, codes, sc, zeros, \
                                 Eh, El, UPD_LDE, row_loss, b == 0)
@@ -538,11 +598,28 @@ extern "C" int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d
     if (!W || !codes || !scales || !zeros) return GPTQ_ERR_INVALID_ARG;
     int rc = check_quant_args(w_dtype, d_out, d_in, bits);
     if (rc != GPTQ_OK) return rc;
-    if (!(group_size == 32 || group_size == 64 || group_size == 128)) return GPTQ_ERR_UNSUPPORTED;
+    const int64_t gsz = (group_size == -1) ? d_in : group_size;
+    const bool narrow = gsz == 32 || gsz == 64 || gsz == 128;
+    if (!narrow && !(gsz > 128 && gsz % 128 == 0 && d_in % gsz == 0)) return GPTQ_ERR_UNSUPPORTED;
     if (!aligned16(W) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros))
         return GPTQ_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     const float maxqf = float((1 << bits) - 1);
+    if (!narrow) {
+        const int64_t warps = d_out * (d_in / gsz);
+        const unsigned grid = (unsigned)ceil_div(warps * 32, 256);
+        __half* sc = reinterpret_cast<__half*>(scales);
+        KernelTimer kt(kKRtn, st);
+        if (w_dtype == GPTQ_DTYPE_F16)
+            rtn_wide_kernel<__half><<<grid, 256, 0, st>>>(reinterpret_cast<const __half*>(W),
+                                                          d_out, d_in, gsz, maxqf, codes, sc,
+                                                          zeros);
+        else
+            rtn_wide_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(W), d_out,
+                                                         d_in, gsz, maxqf, codes, sc, zeros);
+        count_launches();
+        return launch_status();
+    }
     const int64_t warps = d_out * (d_in / 128);
     const unsigned grid = (unsigned)ceil_div(warps * 32, 256);
     __half* sc = reinterpret_cast<__half*>(scales);

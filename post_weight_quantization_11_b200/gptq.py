@@ -34,7 +34,7 @@ EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_prepare_batched_workspace_bytes", "gptq_prepare_hinv_batched",
             "gptq_quantize_layer_batched",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_quantize_layer_static",
-            "gptq_pack_int4",
+            "gptq_pack_int4", "gptq_pack_bits", "gptq_unpack_bits",
             "gptq_unpack_int4", "gptq_w4a16_gemm", "rtn_quantize", "gptq_debug_gemm_nt",
             "gptq_debug_chol_task_order", "gptq_debug_div_rn", "gptq_debug_bounded_wait",
             "gptq_debug_kernel_timing", "gptq_debug_kernel_times", "gptq_debug_kernel_kind_name")
@@ -84,6 +84,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                         P], I32),
         "gptq_pack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "gptq_unpack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
+        "gptq_pack_bits": ([P, P, I64, I64, I64, I32, P, P, P], I32),
+        "gptq_unpack_bits": ([P, P, I64, I64, I64, I32, P, P, P], I32),
         "rtn_quantize": ([P, I32, I64, I64, I32, I32, P, P, P, P], I32),
         "gptq_w4a16_gemm": ([P, I64, P, P, P, P, I64, I64, I32, P, P], I32),
         "gptq_debug_gemm_nt": ([P, I64, P, I64, P, I64, I64, I64, I64, F32, F32, I32, P], I32),
@@ -432,6 +434,39 @@ def gptq_pack_int4(codes: torch.Tensor, zeros: torch.Tensor, qweight=None, qzero
     return qweight, qzeros
 
 
+def gptq_pack_bits(codes: torch.Tensor, zeros: torch.Tensor, bits: int, qweight=None,
+                   qzeros=None):
+    """b-bit storage (one little-endian bit stream per row; b = 4 is the
+    INT4 layout).  Returns (qweight int32 m x d b/32, qzeros uint8 m x ceil(G b/8))."""
+    _need(codes, "codes", torch.uint8)
+    _need(zeros, "zeros", torch.uint8)
+    m, d = codes.shape
+    G = zeros.shape[1]
+    dev = codes.device
+    if qweight is None:
+        qweight = torch.empty(m, d * bits // 32, dtype=torch.int32, device=dev)
+    if qzeros is None:
+        qzeros = torch.empty(m, (G * bits + 7) // 8, dtype=torch.uint8, device=dev)
+    _check("gptq_pack_bits",
+           load_library().gptq_pack_bits(_ptr(codes), _ptr(zeros), m, d, G, int(bits),
+                                         _ptr(qweight), _ptr(qzeros), _stream(codes)))
+    return qweight, qzeros
+
+
+def gptq_unpack_bits(qweight: torch.Tensor, qzeros: torch.Tensor, d_in: int, n_groups: int,
+                     bits: int):
+    _need(qweight, "qweight")
+    _need(qzeros, "qzeros", torch.uint8)
+    m = qweight.shape[0]
+    dev = qweight.device
+    codes = torch.empty(m, d_in, dtype=torch.uint8, device=dev)
+    zeros = torch.empty(m, n_groups, dtype=torch.uint8, device=dev)
+    _check("gptq_unpack_bits",
+           load_library().gptq_unpack_bits(_ptr(qweight), _ptr(qzeros), m, d_in, n_groups,
+                                           int(bits), _ptr(codes), _ptr(zeros), _stream(qweight)))
+    return codes, zeros
+
+
 def gptq_w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
                     qzeros: torch.Tensor, group_size: int = 128, perm=None, y=None):
     """y = x Q^T (batch x d_out fp32) from the packed INT4 layer; x: batch x
@@ -469,7 +504,7 @@ def rtn_quantize(W: torch.Tensor, bits: int = 4, group_size: int = 128):
     _need(W, "W")
     m, d = W.shape
     dev = W.device
-    G = d // group_size
+    G = 1 if group_size in (-1, d) else d // group_size
     codes = torch.empty(m, d, dtype=torch.uint8, device=dev)
     scales = torch.empty(m, G, dtype=torch.float16, device=dev)
     zeros = torch.empty(m, G, dtype=torch.uint8, device=dev)

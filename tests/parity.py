@@ -6,7 +6,11 @@ Tolerances (written here, used by every parity test):
   * U:      relative Frobenius error <= 1e-4 against the oracle's float64 U
             computed from the SAME S (the GPU's, promoted)
   * codes:  bit-exact except at most 1e-3 of the weights (fp32 vs fp64 error
-            feedback flips codes that sit at a rounding tie)
+            feedback flips codes that sit at a rounding tie).  At 4 bits the
+            bar holds for the free-running comparison, cascades included; at
+            other widths it counts the tie flips themselves (the codes the
+            oracle decides differently on the GPU's own trajectory), since
+            one flip there moves tens to hundreds of later codes of its row
   * scales: for every group of a row before that row's first code mismatch,
             the GPU's fp16 scale is the fp16 rounding of some value within
             1e-4 relative of the oracle's pre-fp16 scale
@@ -56,15 +60,18 @@ def fp16_range(s_pre: np.ndarray, rel: float):
     return lo.astype(np.float32), hi.astype(np.float32)
 
 
-def compare_sweep(gpu: dict, orc: dict, group_size: int, report: dict | None = None):
+def compare_sweep(gpu: dict, orc: dict, group_size: int, report: dict | None = None,
+                  code_frac: float = CODE_FRAC):
     """gpu/orc: dicts with codes (m x d uint8), scales (m x G uint16 bits),
     zeros (m x G uint8); orc also has s_pre.  Asserts the code and scale
-    tolerances and returns statistics."""
+    tolerances and returns statistics.  code_frac: the bar on the free-running
+    code mismatches (1.0 where the caller takes the bar on the teacher-forced
+    run instead)."""
     cg, co = gpu["codes"], orc["codes"]
     m, d = co.shape
     mism = cg != co
     frac = float(mism.mean())
-    assert frac <= CODE_FRAC, f"code mismatch fraction {frac:.2e} > {CODE_FRAC}"
+    assert frac <= code_frac, f"code mismatch fraction {frac:.2e} > {code_frac}"
     # first mismatching column per row (d if none)
     first = np.where(mism.any(axis=1), mism.argmax(axis=1), d)
     G = co.shape[1] // group_size if group_size > 0 else 1

@@ -128,7 +128,9 @@ def test_validation_rejects_before_launch(lib):
     assert q(W=None) == 1
     assert q(U=MIS) == 1
     assert q(wsb=100) == 1
-    assert q(g=256, d=512) == 4               # dynamic groups span one block at most
+    assert q(g=384, d=768) == 4               # a dynamic group may not straddle an outer block
+    assert q(g=256, d=512, wsb=100) == 1      # wide dynamic groups: accepted up to the ws check
+    assert q(g=1024, d=2048, wsb=100) == 1
     assert q(g=-1, wsb=100) == 1              # one group per row: accepted up to the ws check
 
     def qs(**k):
@@ -141,6 +143,7 @@ def test_validation_rejects_before_launch(lib):
     assert qs(g=256, wsb=100) == 1            # accepted up to the ws check
     assert qs(bits=5) == 4 and qs(d=200) == 2 and qs(W=None) == 1
     assert lib.rtn_quantize(FAKE, 1, 64, 256, 3, 48, FAKE, FAKE, FAKE, None) == 4
+    assert lib.rtn_quantize(FAKE, 1, 64, 384, 4, 256, FAKE, FAKE, FAKE, None) == 4
     assert lib.rtn_quantize(None, 1, 64, 256, 4, 128, FAKE, FAKE, FAKE, None) == 1
     W4 = lib.gptq_w4a16_gemm
     assert W4(None, 1, FAKE, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 1
@@ -224,3 +227,18 @@ def test_static_entry_checks_arguments_like_the_workspace_one(lib):
     assert S(FAKE, 300, 10, 0.01, 0, None, FAKE, FAKE, None) == 2
     assert S(FAKE, 512, 0, 0.01, 0, None, FAKE, FAKE, None) == 2
     assert S(FAKE, 2048, 10, 0.01, 0, None, FAKE, FAKE, None) == 2    # beyond the scratch
+
+
+def test_pack_bits_validates_before_launch(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-side argument checks with fake pointers run where no GPU is visible")
+    Pk, Uk = lib.gptq_pack_bits, lib.gptq_unpack_bits
+    for f in (Pk, Uk):
+        assert f(None, FAKE, 4, 64, 1, 3, FAKE, FAKE, None) == 1
+        assert f(FAKE, FAKE, 4, 64, 1, 9, FAKE, FAKE, None) == 4
+        assert f(FAKE, FAKE, 4, 64, 1, 1, FAKE, FAKE, None) == 4
+        assert f(FAKE, FAKE, 4, 48, 1, 3, FAKE, FAKE, None) == 2
+        assert f(FAKE, FAKE, 0, 64, 1, 3, FAKE, FAKE, None) == 2
+        assert f(FAKE, FAKE, 4, 64, 0, 3, FAKE, FAKE, None) == 2
+    assert Pk(MIS, FAKE, 4, 64, 1, 3, FAKE, FAKE, None) == 1

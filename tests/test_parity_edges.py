@@ -58,7 +58,7 @@ def test_sweep_degenerate_rows(bits, gs, act, dtype):
     W = _degenerate_rows(_weights(m, d, dtype, 900 + bits + gs), gs)
     X = _gauss_x(n, d, 5, 40.0, 901 + bits)
     _diagnose(W, X, bits, gs, act)
-    st, g, ref = _check_layer(W, X, bits, gs, act)
+    st, g, ref = _check_layer(W, X, bits, gs, act, code_bar="free" if bits == 4 else "forced")
     # the all-zero row quantizes to exact zeros: codes equal the zero points
     # and every group's scale is the [-1, 1] range's
     G_ = d // gs
@@ -79,5 +79,5 @@ def test_sweep_bits8_tolerances_hold_on_outlier_inputs():
     W = _weights(384, 1024, torch.float16, 77)
     X = _gauss_x(3000, 1024, 10, 60.0, 78)
     _diagnose(W, X, 8, 128, False)
-    st, _, _ = _check_layer(W, X, 8, 128, False)
+    st, _, _ = _check_layer(W, X, 8, 128, False, code_bar="forced")
     print("bits 8:", st)
