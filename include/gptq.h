@@ -391,6 +391,49 @@ int rtn_quantize(const void* W, int w_dtype, int64_t d_out, int64_t d_in, int bi
                  void* stream);
 
 /*
+ * Channel magnitudes for activation-aware scaling -- "GPTQ / AWQ /
+ * SqueezeLLM" sec. 二 (the mean absolute activation of each input channel):
+ *   abs_sum[j] += sum_t |X[t][j]|      (fp64 accumulation; mean = abs_sum / n)
+ * X: n_tokens x d fp16; abs_sum: d fp64 device, in/out (zero it first; call
+ * once per calibration batch).  Requires d % 8 == 0, 8 <= d <= 32768.
+ */
+int gptq_channel_abs_sum(const uint16_t* X, int64_t n_tokens, int64_t d, double* abs_sum,
+                         void* stream);
+
+/*
+ * Activation-aware channel scaling chosen by output error -- "GPTQ / AWQ /
+ * SqueezeLLM" sec. 二 (scale input channels by activation magnitude, pick
+ * among candidate scalings the one with the smallest output error, then
+ * GPTQ) and "INT4/INT8 量化推理" sec. 四 (W diag(s) with X diag(s)^-1 is exact
+ * before quantization).  The pages give no candidate set; the reading is:
+ *   a_j = abs_sum_j / n_tokens, raised to the smallest positive a where 0
+ *   (all zero: a = 1); r = a / mean(a); for k = 0 .. n_grid - 1,
+ *   alpha = k / n_grid, s = r^alpha (alpha = 0 is no scaling);
+ *   W' = W diag(s) (fp64, rounded once to fp32), Q' = the group round-to-
+ *   nearest of W' (the quantizer of rtn_quantize), D = Q' diag(s)^-1 - W,
+ *   losses[k] = tr(D H D^T) with H = 2 S / n_tokens;
+ *   *best = the first k with the smallest loss; scales = s of that k.
+ * Optionally W_scaled = fp32(W diag(s)) and S_scaled = fp32(diag(s)^-1 S
+ * diag(s)^-1) (upper triangle, the strictly-lower part written as 0): the
+ * inputs of gptq_prepare_hinv / gptq_quantize_layer for GPTQ in the scaled
+ * coordinates (dequantize with Q diag(s)^-1).
+ * W: d_out x d_in (GPTQ_DTYPE_F16 / F32); S: d_in x d_in fp32 (upper
+ * triangle, from gptq_hessian_accumulate); abs_sum: d_in fp64 from
+ * gptq_channel_abs_sum; losses: n_grid fp64 out; best: 1 int32 out; scales:
+ * d_in fp64 out; W_scaled: d_out x d_in fp32 or NULL; S_scaled: d_in x d_in
+ * fp32 or NULL (all device).  ws: gptq_awq_workspace_bytes(d_out, d_in).
+ * The losses' products D H run on the tensor cores in split-TF32 (fp32-level
+ * accuracy), their sums in fp64.  bits in {2,3,4,8}; group_size a multiple
+ * of 32 dividing d_in, or -1; 1 <= n_grid <= 1000; the d limits of
+ * gptq_quantize_layer.
+ */
+size_t gptq_awq_workspace_bytes(int64_t d_out, int64_t d_in);
+int gptq_awq_search(const void* W, int w_dtype, int64_t d_out, int64_t d_in, const float* S,
+                    int64_t n_tokens, const double* abs_sum, int n_grid, int bits, int group_size,
+                    double* losses, int32_t* best, double* scales, float* W_scaled,
+                    float* S_scaled, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Test hook (no counterpart on the pages): a stand-alone split-TF32
  * tensor-core GEMM.  It takes every product the way the factorization and
  * the block update do (x = x_hi + x_lo, x_hi rounded to TF32; three
@@ -412,9 +455,9 @@ int gptq_debug_gemm_nt(const float* A, int64_t lda, const float* B, int64_t ldb,
  * bracket itself with two CUDA events on its stream; gptq_debug_kernel_times
  * waits for the recorded events, returns per kind the summed milliseconds
  * (ms[k]) and the number of timed launch sites (spans[k]), and forgets the
- * records.  Kinds, in order (n_kinds >= 15): hessian, gather, finalize,
+ * records.  Kinds, in order (n_kinds >= 16): hessian, gather, finalize,
  * factorization, init_work, split_u, static_params, sweep, update_near,
- * update_far, pack, unpack, rtn, w4a16, probe (names from
+ * update_far, pack, unpack, rtn, w4a16, probe, awq (names from
  * gptq_debug_kernel_kind_name).  Use it on eager launches only, never while
  * a stream is being captured; it creates two CUDA events per launch site
  * while enabled.  Disabled (the default) it costs one flag test per launch.

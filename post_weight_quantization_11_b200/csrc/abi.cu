@@ -136,7 +136,7 @@ extern "C" const char* gptq_debug_kernel_kind_name(int kind)
     static const char* names[gptq::kKKinds] = {
         "hessian", "gather", "finalize", "factorization", "init_work", "split_u",
         "static_params", "sweep", "update_near", "update_far", "pack", "unpack", "rtn",
-        "w4a16", "probe"};
+        "w4a16", "probe", "awq"};
     return (kind >= 0 && kind < gptq::kKKinds) ? names[kind] : "unknown";
 }
 

@@ -40,7 +40,8 @@ int persistent_ctas(int kind);
 // Diagnostics (gptq_debug_kernel_timing): kinds of the library's launches.
 enum KernelKind : int {
     kKHessian = 0, kKGather, kKFinalize, kKFactor, kKInitWork, kKSplitU, kKStaticParams,
-    kKSweep, kKUpdateNear, kKUpdateFar, kKPack, kKUnpack, kKRtn, kKW4A16, kKProbe, kKKinds
+    kKSweep, kKUpdateNear, kKUpdateFar, kKPack, kKUnpack, kKRtn, kKW4A16, kKProbe, kKAwq,
+    kKKinds
 };
 
 // While timing is enabled, the launches issued in this object's lifetime are

@@ -35,6 +35,7 @@ EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_quantize_layer_batched",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_quantize_layer_static",
             "gptq_pack_int4", "gptq_pack_bits", "gptq_unpack_bits",
+            "gptq_channel_abs_sum", "gptq_awq_workspace_bytes", "gptq_awq_search",
             "gptq_unpack_int4", "gptq_w4a16_gemm", "rtn_quantize", "gptq_debug_gemm_nt",
             "gptq_debug_chol_task_order", "gptq_debug_div_rn", "gptq_debug_bounded_wait",
             "gptq_debug_kernel_timing", "gptq_debug_kernel_times", "gptq_debug_kernel_kind_name")
@@ -85,6 +86,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_pack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "gptq_unpack_int4": ([P, P, I64, I64, I64, P, P, P], I32),
         "gptq_pack_bits": ([P, P, I64, I64, I64, I32, P, P, P], I32),
+        "gptq_channel_abs_sum": ([P, I64, I64, P, P], I32),
+        "gptq_awq_workspace_bytes": ([I64, I64], SZ),
+        "gptq_awq_search": ([P, I32, I64, I64, P, I64, P, I32, I32, I32, P, P, P, P, P, P, SZ, P],
+                            I32),
         "gptq_unpack_bits": ([P, P, I64, I64, I64, I32, P, P, P], I32),
         "rtn_quantize": ([P, I32, I64, I64, I32, I32, P, P, P, P], I32),
         "gptq_w4a16_gemm": ([P, I64, P, P, P, P, I64, I64, I32, P, P], I32),
@@ -162,7 +167,7 @@ def gptq_set_max_ctas(kind: int, max_ctas: int) -> None:
     _check("gptq_set_max_ctas", load_library().gptq_set_max_ctas(int(kind), int(max_ctas)))
 
 
-N_KERNEL_KINDS = 15
+N_KERNEL_KINDS = 16
 
 
 def gptq_debug_kernel_timing(enable: bool) -> None:
@@ -465,6 +470,45 @@ def gptq_unpack_bits(qweight: torch.Tensor, qzeros: torch.Tensor, d_in: int, n_g
            load_library().gptq_unpack_bits(_ptr(qweight), _ptr(qzeros), m, d_in, n_groups,
                                            int(bits), _ptr(codes), _ptr(zeros), _stream(qweight)))
     return codes, zeros
+
+
+def gptq_channel_abs_sum(X: torch.Tensor, abs_sum=None) -> torch.Tensor:
+    """abs_sum (d fp64) += sum over tokens of |X| (X: n x d fp16)."""
+    _need(X, "X", torch.float16)
+    n, d = X.shape
+    if abs_sum is None:
+        abs_sum = torch.zeros(d, dtype=torch.float64, device=X.device)
+    _need(abs_sum, "abs_sum", torch.float64)
+    _check("gptq_channel_abs_sum",
+           load_library().gptq_channel_abs_sum(_ptr(X), n, d, _ptr(abs_sum), _stream(X)))
+    return abs_sum
+
+
+def gptq_awq_search(W: torch.Tensor, S: torch.Tensor, n_tokens: int, abs_sum: torch.Tensor,
+                    n_grid: int = 20, bits: int = 4, group_size: int = 128,
+                    scaled_outputs: bool = True):
+    """Activation-aware channel scaling chosen by output error.  Returns a
+    LayerResult with losses (n_grid fp64), best (int), alpha, scales (d fp64)
+    and, with scaled_outputs, W_scaled (m x d fp32) and S_scaled (d x d fp32)."""
+    _need(W, "W")
+    _need(S, "S", torch.float32)
+    _need(abs_sum, "abs_sum", torch.float64)
+    m, d = W.shape
+    dev = W.device
+    losses = torch.empty(n_grid, dtype=torch.float64, device=dev)
+    best = torch.empty(1, dtype=torch.int32, device=dev)
+    scales = torch.empty(d, dtype=torch.float64, device=dev)
+    Ws = torch.empty(m, d, dtype=torch.float32, device=dev) if scaled_outputs else None
+    Ss = torch.empty(d, d, dtype=torch.float32, device=dev) if scaled_outputs else None
+    nb = int(load_library().gptq_awq_workspace_bytes(m, d))
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+    _check("gptq_awq_search",
+           load_library().gptq_awq_search(_ptr(W), _wdtype(W), m, d, _ptr(S), int(n_tokens),
+                                          _ptr(abs_sum), int(n_grid), int(bits), int(group_size),
+                                          _ptr(losses), _ptr(best), _ptr(scales), _ptr(Ws),
+                                          _ptr(Ss), _ptr(ws), nb, _stream(W)))
+    return LayerResult(losses=losses, best=best, scales=scales, W_scaled=Ws, S_scaled=Ss,
+                       n_grid=n_grid)
 
 
 def gptq_w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,

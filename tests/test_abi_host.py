@@ -242,3 +242,30 @@ def test_pack_bits_validates_before_launch(lib):
         assert f(FAKE, FAKE, 0, 64, 1, 3, FAKE, FAKE, None) == 2
         assert f(FAKE, FAKE, 4, 64, 0, 3, FAKE, FAKE, None) == 2
     assert Pk(MIS, FAKE, 4, 64, 1, 3, FAKE, FAKE, None) == 1
+
+
+def test_awq_entry_points_validate_before_launch(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-side argument checks with fake pointers run where no GPU is visible")
+    C = lib.gptq_channel_abs_sum
+    assert C(FAKE, 10, 256, None, None) == 1
+    assert C(MIS, 10, 256, FAKE, None) == 1
+    assert C(FAKE, 10, 252, FAKE, None) == 2
+    assert C(FAKE, -1, 256, FAKE, None) == 2
+    assert C(None, 0, 256, FAKE, None) == 0                  # no tokens: nothing to add
+    wb = lib.gptq_awq_workspace_bytes(64, 256)
+    assert wb >= 4 * (256 * 256 + 2 * 64 * 256)
+    A = lib.gptq_awq_search
+
+    def aw(**k):
+        a = dict(W=FAKE, dt=1, m=64, d=256, S=FAKE, n=100, acc=FAKE, grid=20, bits=4, g=128,
+                 losses=FAKE, best=FAKE, scales=FAKE, Ws=None, Ss=None, ws=FAKE, wsb=wb)
+        a.update(k)
+        return A(a["W"], a["dt"], a["m"], a["d"], a["S"], a["n"], a["acc"], a["grid"],
+                 a["bits"], a["g"], a["losses"], a["best"], a["scales"], a["Ws"], a["Ss"],
+                 a["ws"], a["wsb"], None)
+    assert aw(W=None) == 1 and aw(acc=None) == 1 and aw(dt=5) == 1 and aw(Ws=MIS) == 1
+    assert aw(bits=5) == 4 and aw(g=48) == 4 and aw(g=96) == 4
+    assert aw(d=200) == 2 and aw(m=0) == 2 and aw(n=0) == 2 and aw(grid=0) == 2
+    assert aw(wsb=wb - 1) == 1
