@@ -997,10 +997,14 @@ def run_ours_pipelined(a):
 
 def run_w4a16(a):
     """The W4A16 product y = x Q^T of packed INT4 layers (batch a.w4a16 rows
-    of fp16 activations).  Enough distinct layers rotate through the timed
-    loop that their packed bytes exceed L2, so every launch streams its
-    weights from HBM; the roofline is HBM bytes (packed weights, scales, zero
-    points, activations, outputs) per launch over its CUDA-event time."""
+    of fp16 activations) on the tensor cores (gptq_w4a16_matmul), and for
+    batches of at most 4 also the CUDA-core product (gptq_w4a16_gemm).
+    Enough distinct layers rotate through the timed loop that their packed
+    bytes exceed L2, so every launch streams its weights from HBM.  The
+    roofline: HBM bytes per launch (packed weights, scales, zero points,
+    activations, outputs) over the launch's CUDA-event time against the
+    measured copy bandwidth, and 2 m d batch flops against the fp16 (= bf16)
+    tensor peak; the bound is whichever is nearer."""
     ws, rank, local = _dist_init()
     from post_weight_quantization_11_b200 import gptq as G
     G.load_library()
@@ -1021,34 +1025,62 @@ def run_w4a16(a):
         layers.append((qw, sc, qz))
     x = torch.randn(b, d, generator=gen, device=dev).half()
     y = torch.empty(b, m, dtype=torch.float32, device=dev)
-    for i in range(max(3, a.warmup) * L):
+    perm = torch.randperm(d, generator=gen, device=dev).to(torch.int32) if spec.act_order \
+        else None
+    wsb = torch.empty(max(1, G.gptq_w4a16_matmul_workspace_bytes(b, d)), dtype=torch.uint8,
+                      device=dev)
+
+    def tc(i):
         qw, sc, qz = layers[i % L]
-        G.gptq_w4a16_gemm(x, qw, sc, qz, g, None, y)
-    torch.cuda.synchronize()
-    reps = max(a.steps, 1) * L
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    _barrier(ws)
-    with ClockSampler(local) as clk:
+        G.gptq_w4a16_matmul(x, qw, sc, qz, g, perm, y, wsb)
+
+    def cc(i):
+        qw, sc, qz = layers[i % L]
+        G.gptq_w4a16_gemm(x, qw, sc, qz, g, perm, y)
+
+    def timed(fn):
+        for i in range(max(3, a.warmup) * L):
+            fn(i)
+        torch.cuda.synchronize()
+        reps = max(a.steps, 1) * L
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         start.record()
         for i in range(reps):
-            qw, sc, qz = layers[i % L]
-            G.gptq_w4a16_gemm(x, qw, sc, qz, g, None, y)
+            fn(i)
         end.record()
         torch.cuda.synchronize()
-    us = _max_over_ranks(start.elapsed_time(end) * 1e3 / reps, ws)
+        return start.elapsed_time(end) * 1e3 / reps
+
     peaks, src = _peaks()
+    _barrier(ws)
+    with ClockSampler(local) as clk:
+        us = _max_over_ranks(timed(tc), ws)
     bytes_ = per_layer + b * d * 2 + b * m * 4
     gbs = bytes_ / (us * 1e-6) / 1e9
+    tfs = 2.0 * m * d * b / (us * 1e-6) / 1e12
+    hbm, tens = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    t_hbm, t_tc = bytes_ / (hbm * 1e9), 2.0 * m * d * b / (tens * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    roof = ({"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
+            if bound == "hbm" else
+            {"bound": "tensor", "achieved": tfs, "peak": tens, "unit": "TFLOP/s",
+             "frac": tfs / tens})
+    roof.update({"bytes_per_launch": bytes_, "flops_per_launch": 2.0 * m * d * b,
+                 "peak_source": f"hbm_gbs / bf16_tflops (burst) of {src}",
+                 "other": {"GB/s": gbs, "TFLOP/s": tfs}})
     line = {"metric": "W4A16 product weights/s", "value": ws * m * d / (us * 1e-6),
             "unit": "weights/s", "n_gpus": ws, "steps": a.steps, "warmup": a.warmup,
-            "us_per_launch": us, "higher_is_better": True, "scaling": "weak", "dtype": "f32",
-            "data": "synthetic packed layers", "vs_baseline": None,
+            "us_per_launch": us, "higher_is_better": True, "scaling": "weak", "dtype": "f16",
+            "data": "synthetic packed layers", "vs_baseline": None, "kernel": "gptq_w4a16_matmul",
             "config": {"workload": f"{spec.name} ({a.workload}) packed: W {m}x{d} INT4 g{g}, "
-                                   f"batch {b}", "layers_rotated": L},
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks.get("hbm_gbs"),
-                         "unit": "GB/s", "frac": gbs / peaks.get("hbm_gbs"),
-                         "bytes_per_launch": bytes_, "peak_source": f"hbm_gbs of {src}"},
-            "clocks": clk.summary()}
+                                   f"batch {b}, act_order={spec.act_order}",
+                       "layers_rotated": L},
+            "roofline": roof, "clocks": clk.summary()}
+    if b <= 4:
+        us_cc = timed(cc)
+        line["cuda_core_gemv"] = {"us_per_launch": us_cc,
+                                  "GB/s": bytes_ / (us_cc * 1e-6) / 1e9,
+                                  "frac": bytes_ / (us_cc * 1e-6) / 1e9 / hbm}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

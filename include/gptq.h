@@ -379,6 +379,27 @@ int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t* qweight,
                     int64_t d_out, int64_t d_in, int group_size, float* y, void* stream);
 
 /*
+ * W4A16 product on the tensor cores for any batch -- the same product as
+ * gptq_w4a16_gemm ("INT4/INT8 量化推理" sec. 六 on the storage of sec. 一):
+ *   y[b][r] = sum_j x[b][j] Q[r][j],  Q[r][perm[k]] = s[r][k/g] (c[r][k] - z[r][k/g])
+ * The packed words are turned into exact fp16 (c - z) operands in shared
+ * memory and multiplied with the fp16 activations by tcgen05 kind::f16
+ * (fp32 accumulation in TMEM, at most 512 products per accumulation, each
+ * group's sum scaled by its fp16 scale in fp32).
+ * x: batch x d_in fp16 (original column order); y: batch x d_out fp32 out.
+ * perm: d_in int32 or NULL; with perm, ws must hold
+ * gptq_w4a16_matmul_workspace_bytes(batch, d_in) bytes (the activations
+ * gathered into the codes' order); without it ws may be NULL.
+ * group_size: a multiple of 64 dividing d_in, or -1 (smaller groups:
+ * gptq_w4a16_gemm).  1 <= batch <= 2^24; the d limits of gptq_w4a16_gemm.
+ */
+size_t gptq_w4a16_matmul_workspace_bytes(int64_t batch, int64_t d_in);
+int gptq_w4a16_matmul(const uint16_t* x, int64_t batch, const uint32_t* qweight,
+                      const uint16_t* scales, const uint8_t* qzeros, const int32_t* perm,
+                      int64_t d_out, int64_t d_in, int group_size, float* y, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/*
  * Round-to-nearest baseline -- "大模型量化实战（上）" (RTN: every weight
  * rounded on its own) with the min-max group quantizer of "校准艺术" sec. 2.1:
  * the same group parameters and codes as gptq_quantize_layer, taken on the

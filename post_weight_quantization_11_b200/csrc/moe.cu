@@ -14,8 +14,6 @@
 
 namespace gptq {
 
-constexpr int kErrIndex = 0x201;
-
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4* __restrict__ X, int64_t n_rows, int64_t vpr,
                    const int32_t* __restrict__ idx, int64_t n_idx, uint4* __restrict__ out)

@@ -15,6 +15,7 @@
 // only the chain of blocks is sequential.
 #include "common.cuh"
 #include "quant_common.cuh"
+#include "tc_common.cuh"
 #include "update.cuh"
 
 namespace gptq {
@@ -37,7 +38,9 @@ __global__ void init_work_kernel(const T* __restrict__ W, const int32_t* __restr
          i += int64_t(gridDim.x) * blockDim.x) {
         const int64_t r = i / d, k = i - r * d;
         const int64_t src = perm ? int64_t(perm[k]) : k;
-        Wk[i] = float(W[r * d + src]);
+        const bool in = src >= 0 && src < d;          // a bad index is not followed
+        if (!in) atomicCAS(&g_device_status, 0, kErrIndex);
+        Wk[i] = in ? float(W[r * d + src]) : 0.f;
     }
 }
 

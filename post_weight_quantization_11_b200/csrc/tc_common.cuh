@@ -29,6 +29,7 @@ enum DeviceError : int {
     kErrWaitAccEmpty = 0x104, // MMA waited too long for a drained accumulator
     kErrWaitDep = 0x105,      // a task waited too long for a task it depends on
     kErrWaitLeaf = 0x106,     // a role of the factorization leaf waited too long
+    kErrIndex = 0x201,        // an index argument (routing, permutation) was out of range
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)

@@ -19,6 +19,7 @@
 // 16-code chunks of the slice; the slices' partial sums meet in y by atomic
 // adds (y is zeroed first).
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace gptq {
 
@@ -50,7 +51,9 @@ w4a16_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight,
         const int b = idx / klen, kk = idx - b * klen;
         const int64_t k = k0 + kk;
         const int64_t src = perm ? int64_t(perm[k]) : k;
-        xs[b][kk] = ldexpf(__half2float(x[b * d + src]), -4 * (kk & 3));
+        const bool in = src >= 0 && src < d;          // a bad index is not followed
+        if (!in) atomicCAS(&g_device_status, 0, kErrIndex);
+        xs[b][kk] = in ? ldexpf(__half2float(x[b * d + src]), -4 * (kk & 3)) : 0.f;
     }
     __syncthreads();
     const int nch = klen / W4_CHUNK;

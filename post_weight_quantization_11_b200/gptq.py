@@ -36,7 +36,8 @@ EXPORTED = ("gptq_status_string", "gptq_abi_version", "gptq_debug_launch_count",
             "gptq_quantize_workspace_bytes", "gptq_quantize_layer", "gptq_quantize_layer_static",
             "gptq_pack_int4", "gptq_pack_bits", "gptq_unpack_bits",
             "gptq_channel_abs_sum", "gptq_awq_workspace_bytes", "gptq_awq_search",
-            "gptq_unpack_int4", "gptq_w4a16_gemm", "rtn_quantize", "gptq_debug_gemm_nt",
+            "gptq_unpack_int4", "gptq_w4a16_gemm", "gptq_w4a16_matmul_workspace_bytes",
+            "gptq_w4a16_matmul", "rtn_quantize", "gptq_debug_gemm_nt",
             "gptq_debug_chol_task_order", "gptq_debug_div_rn", "gptq_debug_bounded_wait",
             "gptq_debug_kernel_timing", "gptq_debug_kernel_times", "gptq_debug_kernel_kind_name")
 
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gptq_unpack_bits": ([P, P, I64, I64, I64, I32, P, P, P], I32),
         "rtn_quantize": ([P, I32, I64, I64, I32, I32, P, P, P, P], I32),
         "gptq_w4a16_gemm": ([P, I64, P, P, P, P, I64, I64, I32, P, P], I32),
+        "gptq_w4a16_matmul_workspace_bytes": ([I64, I64], SZ),
+        "gptq_w4a16_matmul": ([P, I64, P, P, P, P, I64, I64, I32, P, P, SZ, P], I32),
         "gptq_debug_gemm_nt": ([P, I64, P, I64, P, I64, I64, I64, I64, F32, F32, I32, P], I32),
         "gptq_debug_chol_task_order": ([I64, P, I64], I64),
         "gptq_debug_div_rn": ([P, P, I64, P], I32),
@@ -528,6 +531,36 @@ def gptq_w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor
     _check("gptq_w4a16_gemm",
            load_library().gptq_w4a16_gemm(_ptr(x), b, _ptr(qweight), _ptr(scales), _ptr(qzeros),
                                           _ptr(perm), m, d, int(group_size), _ptr(y), _stream(x)))
+    return y
+
+
+def gptq_w4a16_matmul_workspace_bytes(batch: int, d_in: int) -> int:
+    return int(load_library().gptq_w4a16_matmul_workspace_bytes(int(batch), int(d_in)))
+
+
+def gptq_w4a16_matmul(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                      qzeros: torch.Tensor, group_size: int = 128, perm=None, y=None, ws=None):
+    """y = x Q^T (batch x d_out fp32) from the packed INT4 layer on the tensor
+    cores, any batch; x: batch x d_in fp16 in original column order."""
+    _need(x, "x", torch.float16)
+    _need(qweight, "qweight")
+    _need(scales, "scales", torch.float16)
+    _need(qzeros, "qzeros", torch.uint8)
+    b, d = x.shape
+    m = qweight.shape[0]
+    y = torch.empty(b, m, dtype=torch.float32, device=x.device) if y is None else y
+    _need(y, "y", torch.float32)
+    nb = 0
+    if perm is not None:
+        _need(perm, "perm", torch.int32)
+        nb = int(load_library().gptq_w4a16_matmul_workspace_bytes(b, d))
+        ws = torch.empty(nb, dtype=torch.uint8, device=x.device) if ws is None else ws
+        nb = ws.numel()
+    _check("gptq_w4a16_matmul",
+           load_library().gptq_w4a16_matmul(_ptr(x), b, _ptr(qweight), _ptr(scales), _ptr(qzeros),
+                                            _ptr(perm), m, d, int(group_size), _ptr(y),
+                                            _ptr(ws) if perm is not None else None, nb,
+                                            _stream(x)))
     return y
 
 

@@ -43,12 +43,23 @@ def _layer(rng, m, d, g, act, exact):
     return codes, zeros, sc.view(np.uint16), perm, qw, qz
 
 
-def _run(x, qw, sc16, qz, g, perm):
+def _run(x, qw, sc16, qz, g, perm, tc=False):
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)    # noqa: E731
-    y = G.gptq_w4a16_gemm(t(x), t(qw.view(np.int32)), t(sc16.view(np.float16)), t(qz), g,
-                          None if perm is None else t(perm))
+    fn = G.gptq_w4a16_matmul if tc else G.gptq_w4a16_gemm
+    y = fn(t(x), t(qw.view(np.int32)), t(sc16.view(np.float16)), t(qz), g,
+           None if perm is None else t(perm))
     torch.cuda.synchronize()
     return y.cpu().numpy()
+
+
+def _bound(x, codes, zeros, sc16, d, g, perm):
+    """1e-5 of sum_j |x_j| s (c + z) in original column order"""
+    gi = np.arange(d) // (d if g == -1 else g)
+    s = sc16.view(np.float16).astype(np.float64)[:, gi]
+    mag_sweep = s * (codes.astype(np.float64) + zeros.astype(np.float64)[:, gi])
+    mag = np.empty_like(mag_sweep)
+    mag[:, perm if perm is not None else np.arange(d)] = mag_sweep
+    return 1e-5 * (np.abs(x.astype(np.float64)) @ mag.T)
 
 
 @pytest.mark.parametrize("m,d,g,b,act", [(300, 256, 128, 1, False), (77, 4096, 128, 4, True),
@@ -82,3 +93,49 @@ def test_w4a16_general_within_fp32_bound(m, d, g, b, act):
     mag[:, perm if perm is not None else np.arange(d)] = mag_sweep
     bound = 1e-5 * (np.abs(x.astype(np.float64)) @ mag.T)
     assert (np.abs(y.astype(np.float64) - ref) <= bound).all()
+
+
+# ---- the tensor-core path (gptq_w4a16_matmul), any batch -------------------
+
+@pytest.mark.parametrize("m,d,g,b,act", [(300, 256, 128, 1, False), (77, 4096, 128, 16, True),
+                                         (130, 1024, 64, 37, False), (129, 2048, -1, 129, True),
+                                         (256, 768, 256, 300, False)])
+def test_w4a16_tc_exact_on_representable_values(m, d, g, b, act):
+    rng = np.random.default_rng(3000 + m + d + b)
+    codes, zeros, sc16, perm, qw, qz = _layer(rng, m, d, g, act, exact=True)
+    x = rng.integers(-3, 4, (b, d)).astype(np.float16)
+    y = _run(x, qw, sc16, qz, g, perm, tc=True)
+    ref = oracle.w4a16_matmul(x, qw, qz, sc16, d, g, perm)
+    assert np.array_equal(y.astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("m,d,g,b,act", [(14336, 4096, 128, 1, True), (4096, 14336, 128, 4, False),
+                                         (4096, 4096, 128, 200, True), (11008, 4096, 64, 16, False),
+                                         (4096, 11008, -1, 3, True)])
+def test_w4a16_tc_full_size_within_fp32_bound(m, d, g, b, act):
+    """Layers of the 7B / 8B shapes, act-order permutations on and off."""
+    rng = np.random.default_rng(4000 + m + d + b)
+    codes, zeros, sc16, perm, qw, qz = _layer(rng, m, d, g, act, exact=False)
+    x = rng.standard_normal((b, d)).astype(np.float32)
+    x[:, rng.permutation(d)[: max(1, d // 100)]] *= 40.0
+    x = x.astype(np.float16)
+    y = _run(x, qw, sc16, qz, g, perm, tc=True)
+    ref = oracle.w4a16_matmul(x, qw, qz, sc16, d, g, perm)
+    assert (np.abs(y.astype(np.float64) - ref) <= _bound(x, codes, zeros, sc16, d, g, perm)).all()
+
+
+def test_w4a16_tc_of_a_gptq_layer():
+    """The product of a layer the library quantized and packed (act-order),
+    against the oracle's product of the same packed bytes."""
+    W = (torch.randn(512, 1024) * 0.02).half().to(DEV)
+    X = torch.randn(3000, 1024).half().to(DEV)
+    res = G.quantize_layer_from_inputs(W, X, 4, 128, act_order=True)
+    x = torch.randn(8, 1024).half().to(DEV)
+    y = G.gptq_w4a16_matmul(x, res.qweight, res.scales, res.qzeros, 128, res.perm)
+    torch.cuda.synchronize()
+    t = lambda a: a.cpu().numpy()                                    # noqa: E731
+    qw, qz, sc = t(res.qweight).view(np.uint32), t(res.qzeros), t(res.scales).view(np.uint16)
+    ref = oracle.w4a16_matmul(t(x), qw, qz, sc, 1024, 128, t(res.perm))
+    codes, zeros = oracle.unpack_int4(qw, qz, 1024, 8)
+    assert (np.abs(t(y).astype(np.float64) - ref) <= _bound(t(x), codes, zeros, sc, 1024, 128,
+                                                            t(res.perm))).all()
