@@ -261,6 +261,52 @@ def test_wide_dynamic_groups(gs, act, d):
     print((gs, act, d), st)
 
 
+@pytest.mark.parametrize("act", [False, True])
+def test_sharded_layer_against_the_oracle(monkeypatch, act):
+    """The one-layer-over-ranks driver as three ranks would run it, on real
+    kernels in one process: each emulated rank accumulates S over its token
+    share (unequal shares), the all-reduce is emulated by summing the ranks'
+    S, every rank prepares U and quantizes its share of the rows (an odd row
+    count).  The concatenated codes, scales and zero points against the
+    oracle on the summed S (H-forced protocol), packing bit-exact."""
+    import torch.distributed as dist
+    from post_weight_quantization_11_b200 import sharded
+    world, m, d, n = 3, 301, 512, 3001
+    W = _weights(m, d, torch.float16, 41 + act)
+    X = _gauss_x(n, d, 4, 40.0, 42 + act)
+    Wd, Xd = W.to(DEV), X.to(DEV)
+    monkeypatch.setattr(dist, "all_reduce", lambda *a, **k: None)   # emulated below
+    monkeypatch.setattr(sharded.ShardedLayer, "_sum_over_ranks", lambda self, v, dev: n)
+    ranks = []
+    for r in range(world):
+        monkeypatch.setattr(sharded, "_world", lambda g, r=r: (world, r))
+        t0, t1 = sharded.share(n, world, r)
+        L = sharded.ShardedLayer(m, d, t1 - t0, DEV, act_order=act)
+        L.hessian(Xd[t0:t1].contiguous())
+        ranks.append(L)
+    S_sum = sum(L.S for L in ranks)
+    for L in ranks:
+        L.S.copy_(S_sum)                                  # what the all-reduce leaves
+        lo, hi = L.rows
+        L.quantize(Wd[lo:hi].contiguous())
+    torch.cuda.synchronize()
+    assert all(int(L.info.item()) == 0 for L in ranks)
+    g = dict(codes=np.concatenate([P.to_np(L.codes) for L in ranks]),
+             scales=np.concatenate([P.to_np(L.scales) for L in ranks]),
+             zeros=np.concatenate([P.to_np(L.zeros) for L in ranks]))
+    S64 = P.mirror_upper(P.to_np(S_sum))
+    assert P.rel_fro(S64, oracle.hessian(X.numpy())) <= P.S_TOL
+    ref = oracle.gptq_layer(W.double().numpy(), S64, n, 4, 128, 0.01, act)
+    assert all(np.array_equal(P.to_np(L.perm), ref["perm"]) for L in ranks)
+    P.compare_sweep(g, ref, 128)
+    Wp = np.ascontiguousarray(W.double().numpy()[:, ref["perm"]])
+    P.teacher_forced_check(Wp, ref["U"], g, 4, 128)
+    rq, rz = oracle.pack_int4(g["codes"], g["zeros"])
+    qw = np.concatenate([P.to_np(L.qweight).view(np.uint32) for L in ranks])
+    qz = np.concatenate([P.to_np(L.qzeros) for L in ranks])
+    assert np.array_equal(qw, rq) and np.array_equal(qz, rz)
+
+
 @pytest.mark.parametrize("act_order,d", [(False, 512), (True, 512), (False, 640), (True, 1152)])
 def test_prepare_parity(act_order, d):
     n = 2048

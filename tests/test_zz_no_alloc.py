@@ -33,31 +33,52 @@ def _S(n, d, seed):
     return torch.from_numpy(oracle.hessian(X.numpy()).astype(np.float32)).to(DEV)
 
 
-def _call_static(lib, S, n, act):
+def _call_static(lib, S, n, act, free_mem=None):
+    """One call through the C ABI; outputs are allocated (by torch) before it.
+    free_mem: a list that receives the device's free bytes right before and
+    right after the call (the call itself must allocate nothing)."""
     d = S.shape[0]
     perm = torch.empty(d, dtype=torch.int32, device=DEV)
     U = torch.full((d, d), float("nan"), dtype=torch.float32, device=DEV)
     info = torch.full((1,), -7, dtype=torch.int32, device=DEV)
+    torch.cuda.synchronize()
+    if free_mem is not None:
+        free_mem.append(torch.cuda.mem_get_info()[0])
     st = lib.gptq_prepare_hinv_static(ctypes.c_void_p(S.data_ptr()), d, n, 0.01, int(act),
                                       ctypes.c_void_p(perm.data_ptr()),
                                       ctypes.c_void_p(U.data_ptr()),
                                       ctypes.c_void_p(info.data_ptr()),
                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0, G.gptq_status_string(st)
+    torch.cuda.synchronize()
+    if free_mem is not None:
+        free_mem.append(torch.cuda.mem_get_info()[0])
     return perm, U, info
 
 
 def test_static_scratch_matches_workspace_version(lib):
-    cases = [(2048, 512, 31, True), (1536, 1024, 32, False)]   # two calls in a row
-    for n, d, seed, act in cases:
+    """Two calls in a row, each against the workspace version on the same S.
+    The factorization is deterministic for a given input (no atomics touch
+    its data), so U, perm and info must be equal bit for bit: stale scratch
+    from the previous call would show.  Around every call after the first
+    (which looks up the scratch's address) the device's free memory must not
+    change."""
+    cases = [(2048, 512, 31, True), (1536, 1024, 32, False), (2048, 512, 33, False)]
+    free = []
+    for k, (n, d, seed, act) in enumerate(cases):
         S = _S(n, d, seed)
         p_ref, U_ref, i_ref = G.gptq_prepare_hinv(S, n, 0.01, act)
-        p_st, U_st, i_st = _call_static(lib, S, n, act)
+        p_st, U_st, i_st = _call_static(lib, S, n, act, free if k > 0 else None)
         torch.cuda.synchronize()
         assert int(i_ref.item()) == 0 and int(i_st.item()) == 0
         assert torch.equal(p_ref, p_st)
-        assert P.rel_fro(P.to_np(U_st).astype(np.float64),
-                         P.to_np(U_ref).astype(np.float64)) <= P.U_TOL
+        assert torch.equal(U_st, U_ref)
+        # and both against the oracle's float64 U
+        S64 = P.mirror_upper(P.to_np(S))
+        _, Hd, _, _, st = oracle.finalize(S64, n, 0.01, act)
+        U64, inf = oracle.hinv_upper_chol(Hd)
+        assert P.rel_fro(P.to_np(U_st).astype(np.float64), U64) <= P.U_TOL
+    assert len(free) == 4 and free[0] == free[1] and free[2] == free[3], free
     assert G.gptq_device_status(reset=True) == 0
 
 
