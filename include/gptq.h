@@ -387,9 +387,10 @@ int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t* qweight,
  * (fp32 accumulation in TMEM, at most 512 products per accumulation, each
  * group's sum scaled by its fp16 scale in fp32).
  * x: batch x d_in fp16 (original column order); y: batch x d_out fp32 out.
- * perm: d_in int32 or NULL; with perm, ws must hold
- * gptq_w4a16_matmul_workspace_bytes(batch, d_in) bytes (the activations
- * gathered into the codes' order); without it ws may be NULL.
+ * perm: d_in int32 or NULL.  ws: gptq_w4a16_matmul_workspace_bytes(batch,
+ * d_in) bytes, always (the activations are first gathered into the order in
+ * which the kernel lays out each packed word's columns, through perm when
+ * given).
  * group_size: a multiple of 64 dividing d_in, or -1 (smaller groups:
  * gptq_w4a16_gemm).  1 <= batch <= 2^24; the d limits of gptq_w4a16_gemm.
  */

@@ -7,17 +7,25 @@
 // for any batch of activation rows.  The weights stream from HBM once, as
 // packed nibbles, and become tensor-core operands in shared memory:
 //  * warp 0 loads the packed words by TMA (128 rows x 64 codes = 4 KB per
-//    stage, eight stages deep), warp 1 the activations (N x 64 fp16, 128-byte
+//    stage, sixteen stages deep), warp 1 the activations (N x 64 fp16, 128-byte
 //    swizzle; columns in sweep order, gathered first when perm is given);
-//  * warps 3-6 (one thread per weight row) turn every packed word into one
-//    16-byte chunk of exact fp16 values c - z (the nibble is placed in the
-//    mantissa of 1024.0 and 1024 + z subtracted: small integers, exact) and
-//    store it where the 128-byte swizzle of a K-major operand puts it;
+//  * the dequantization warps (one or two threads per weight row) turn every
+//    packed word into one 16-byte chunk of exact fp16 values c - z: one mask
+//    and OR per pair of nibbles puts nibbles k and k + 4 into the mantissas
+//    of two 1024.0 halves, one subtraction of 1024 + z leaves c - z (small
+//    integers, exact); the chunk is stored where the 128-byte swizzle of a
+//    K-major operand puts it.  Its columns are therefore in the order
+//    (0, 4, 1, 5, 2, 6, 3, 7) of the word; the activations are gathered into
+//    the same order first (with the act-order permutation, when given), and
+//    the product does not depend on the order of K;
 //  * warp 2 issues tcgen05.mma kind::f16 (M = 128 weight rows, N = the batch
 //    tile, K = 16), accumulating one scale chunk (a group, at most 512
 //    columns) per TMEM accumulator, two accumulators in turn;
-//  * warps 7-10 fold each chunk's accumulator into fp32 registers with the
-//    group's fp16 scale, then write y (atomically when K is split).
+//  * four epilogue warps fold each chunk's accumulator into fp32 registers
+//    with the group's fp16 scale, then write y (atomically when K is split).
+// Two shapes: batch tiles up to 32 columns with eight dequantization warps
+// (decode: the dequantization sets the pace), and up to 128 columns with four
+// (the epilogue's 128 accumulators per thread need the registers).
 // Products (c - z) x are exact in fp32; sums are fp32 (each TMEM chunk
 // accumulates at most 512 products).  Every mbarrier wait is bounded.
 #include "common.cuh"
@@ -25,16 +33,21 @@
 
 namespace gptq {
 
-constexpr int WQ_M = 128, WQ_K = 64, WQ_NMAX = 128;
-constexpr int WQ_STAGES = 4, WQ_QSTAGES = 8;
+constexpr int WQ_M = 128, WQ_K = 64, WQ_NBIG = 128;
+constexpr int WQ_STAGES = 4, WQ_QSTAGES = 16;
 constexpr int WQ_CH = 512;                                   // max K per accumulation chunk
 constexpr int WQ_A_BYTES = WQ_M * WQ_K * 2;                  // 16 KB
-constexpr int WQ_B_BYTES = WQ_NMAX * WQ_K * 2;               // 16 KB
+constexpr int WQ_B_BYTES = WQ_NBIG * WQ_K * 2;               // 16 KB (room for the larger tile)
 constexpr int WQ_Q_BYTES = WQ_M * WQ_K / 2;                  // 4 KB
-constexpr int WQ_DEQ_WARPS = 4, WQ_EPI_WARPS = 4;
-constexpr int WQ_THREADS = 32 * (3 + WQ_DEQ_WARPS + WQ_EPI_WARPS);   // 352
+constexpr int WQ_EPI_WARPS = 4;
 constexpr int WQ_SMEM = WQ_STAGES * (WQ_A_BYTES + WQ_B_BYTES) + WQ_QSTAGES * WQ_Q_BYTES + 1024 + 512;
-constexpr uint32_t WQ_TMEM_COLS = 2 * WQ_NMAX;
+
+template <int NMAX> struct WqCfg {
+    static constexpr int DEQ_WARPS = NMAX <= 32 ? 8 : 4;
+    static constexpr int WORDS = 8 / (DEQ_WARPS / 4);          // packed words per thread and stage
+    static constexpr int THREADS = 32 * (3 + DEQ_WARPS + WQ_EPI_WARPS);
+    static constexpr uint32_t TMEM_COLS = 2 * NMAX < 32 ? 32 : 2 * NMAX;
+};
 
 struct WqParams {
     float* y;
@@ -65,13 +78,14 @@ __device__ __forceinline__ WqItem wq_item(const WqParams& p, int q)
     return it;
 }
 
-__device__ __forceinline__ uint32_t wq_half2_bits(uint32_t t)
+// Nibbles j and j + 4 of w (j = 0..3) as the fp16 pair (1024 + c_j, 1024 + c_{j+4})
+__device__ __forceinline__ uint32_t wq_pair_bits(uint32_t w, int j)
 {
-    // (nibble 0, nibble 1) of t as (1024 + c0, 1024 + c1) in fp16
-    return (t & 0x0000000Fu) | ((t & 0x000000F0u) << 12) | 0x64006400u;
+    return ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
 }
 
-__global__ void __launch_bounds__(WQ_THREADS, 1)
+template <int NMAX>
+__global__ void __launch_bounds__(WqCfg<NMAX>::THREADS, 1)
 w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmX,
                 const WqParams p)
 {
@@ -92,13 +106,13 @@ w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < WQ_QSTAGES; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], WQ_DEQ_WARPS); }
-        for (int s = 0; s < WQ_STAGES; ++s) { mbar_init(&afull[s], WQ_DEQ_WARPS + 1); mbar_init(&aempty[s], 1); }
+        for (int s = 0; s < WQ_QSTAGES; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], WqCfg<NMAX>::DEQ_WARPS); }
+        for (int s = 0; s < WQ_STAGES; ++s) { mbar_init(&afull[s], WqCfg<NMAX>::DEQ_WARPS + 1); mbar_init(&aempty[s], 1); }
         for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], WQ_EPI_WARPS); }
         *abort = 0;
         fence_mbar_init();
     }
-    if (warp == 2) tmem_alloc(tmem_slot, WQ_TMEM_COLS);
+    if (warp == 2) tmem_alloc(tmem_slot, WqCfg<NMAX>::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -152,7 +166,7 @@ w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     const uint32_t aph = (ch >> 1) & 1;
                     if (!mbar_wait(&acce[a], aph ^ 1, kErrWaitAccEmpty, abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem + uint32_t(a * WQ_NMAX);
+                    const uint32_t d_tmem = tmem + uint32_t(a * NMAX);
                     uint32_t acc = 0;
                     for (int s = 0; s < spc; ++s) {
                         if (!mbar_wait(&afull[stage], phase, kErrWaitFull, abort)) { ok = false; break; }
@@ -173,10 +187,13 @@ w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
             }
         }
-    } else if (warp < 3 + WQ_DEQ_WARPS) {
-        // dequantization: thread r = weight row r of the tile: the row's 8
-        // packed words of a stage -> the 8 16-byte chunks of its 128-byte row
-        const int r = threadIdx.x - 96;
+    } else if (warp < 3 + WqCfg<NMAX>::DEQ_WARPS) {
+        // dequantization: thread (h, r) = weight row r of the tile, words
+        // h W .. h W + W - 1 of the row's 8 packed words of a stage -> the
+        // same 16-byte chunks of its 128-byte row
+        constexpr int W = WqCfg<NMAX>::WORDS;
+        const int t = threadIdx.x - 96;
+        const int r = t & (WQ_M - 1), h = t >> 7;
         int qs = 0, as = 0;
         uint32_t qph = 0, aph = 0;
         bool ok = true;
@@ -184,35 +201,50 @@ w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const WqItem it = wq_item(p, q);
             const int64_t row = int64_t(it.rt) * WQ_M + r;
             const bool live = row < p.m;
-            for (int s = it.c0 * spc; s < it.c1 * spc; ++s) {
+            // zero points: the item's first group now, every next group one
+            // group ahead (its load overlaps the current group's stages)
+            const int64_t s_begin = int64_t(it.c0) * spc, s_end = int64_t(it.c1) * spc;
+            int64_t gi_cur = (s_begin * WQ_K) / p.gsz;
+            const int64_t gi_last = ((s_end - 1) * WQ_K) / p.gsz;
+            uint32_t zb_cur = live ? uint32_t(p.qzeros[row * Gz + gi_cur / 2]) : 0u;
+            uint32_t zb_next = (live && gi_cur < gi_last) ? uint32_t(p.qzeros[row * Gz + (gi_cur + 1) / 2]) : 0u;
+            for (int64_t s = s_begin; s < s_end; ++s) {
+                const int64_t gi = (s * WQ_K) / p.gsz;
+                if (gi != gi_cur) {
+                    gi_cur = gi;
+                    zb_cur = zb_next;
+                    zb_next = (live && gi_cur < gi_last) ? uint32_t(p.qzeros[row * Gz + (gi_cur + 1) / 2]) : 0u;
+                }
                 if (!mbar_wait(&qfull[qs], qph, kErrWaitFull, abort)) { ok = false; break; }
-                const uint4 w0 = *reinterpret_cast<const uint4*>(sQ + qs * WQ_Q_BYTES + r * 32);
-                const uint4 w1 = *reinterpret_cast<const uint4*>(sQ + qs * WQ_Q_BYTES + r * 32 + 16);
+                uint32_t words[W];
+                {
+                    const uint4* src = reinterpret_cast<const uint4*>(sQ + qs * WQ_Q_BYTES + r * 32 + h * W * 4);
+#pragma unroll
+                    for (int v = 0; v < W / 4; ++v) {
+                        const uint4 q4 = src[v];
+                        words[4 * v] = q4.x; words[4 * v + 1] = q4.y;
+                        words[4 * v + 2] = q4.z; words[4 * v + 3] = q4.w;
+                    }
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&qempty[qs]);
                 if (++qs == WQ_QSTAGES) { qs = 0; qph ^= 1; }
-                const int64_t gi = (int64_t(s) * WQ_K) / p.gsz;
-                uint32_t z = 0;
-                if (live) {
-                    const uint32_t zb = p.qzeros[row * Gz + gi / 2];
-                    z = (gi & 1) ? (zb >> 4) : (zb & 0xFu);
-                }
-                const __half2 zz = __halves2half2(__ushort_as_half(uint16_t(0x6400u | z)),
-                                                  __ushort_as_half(uint16_t(0x6400u | z)));
+                const uint32_t z = (gi_cur & 1) ? (zb_cur >> 4) : (zb_cur & 0xFu);
+                const uint32_t zbits = 0x64006400u | (z << 16) | z;
+                const __half2 zz = *reinterpret_cast<const __half2*>(&zbits);
                 if (!mbar_wait(&aempty[as], aph ^ 1, kErrWaitEmpty, abort)) { ok = false; break; }
                 uint8_t* arow = sA + as * WQ_A_BYTES + r * 128;
-                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t w = words[i];
+                for (int i = 0; i < W; ++i) {
                     uint32_t o[4];
 #pragma unroll
-                    for (int pq = 0; pq < 4; ++pq) {
-                        const uint32_t bits = wq_half2_bits(w >> (8 * pq));
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t bits = wq_pair_bits(words[i], j);
                         const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&bits), zz);
-                        o[pq] = *reinterpret_cast<const uint32_t*>(&v);
+                        o[j] = *reinterpret_cast<const uint32_t*>(&v);
                     }
-                    *reinterpret_cast<uint4*>(arow + ((i ^ (r & 7)) << 4)) =
+                    const int chunk = h * W + i;
+                    *reinterpret_cast<uint4*>(arow + ((chunk ^ (r & 7)) << 4)) =
                         make_uint4(o[0], o[1], o[2], o[3]);
                 }
                 fence_proxy_async_smem();
@@ -227,28 +259,30 @@ w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int r = qr * 32 + lane;
         int ch = 0;
         bool ok = true;
-        float sum[WQ_NMAX];
+        float sum[NMAX];
         for (int q = blockIdx.x; q < p.items && ok; q += P) {
             const WqItem it = wq_item(p, q);
             const int64_t row = int64_t(it.rt) * WQ_M + r;
             const bool live = row < p.m;
 #pragma unroll
-            for (int u = 0; u < WQ_NMAX; ++u) sum[u] = 0.f;
+            for (int u = 0; u < NMAX; ++u) sum[u] = 0.f;
             for (int c = it.c0; c < it.c1; ++c, ++ch) {
                 const int a = ch & 1;
                 const uint32_t aph = (ch >> 1) & 1;
-                if (!mbar_wait(&accf[a], aph, kErrWaitAccFull, abort)) { ok = false; break; }
-                tc_fence_after();
+                // the chunk's scale is requested before the wait, which hides its latency
                 const int64_t gi = (int64_t(c) * p.chunk) / p.gsz;
                 const float sc = live ? __half2float(p.scales[row * G + gi]) : 0.f;
-                const uint32_t base = tmem + uint32_t(a * WQ_NMAX) + (uint32_t(qr * 32) << 16);
+                if (!mbar_wait(&accf[a], aph, kErrWaitAccFull, abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t base = tmem + uint32_t(a * NMAX) + (uint32_t(qr * 32) << 16);
 #pragma unroll
-                for (int cb = 0; cb < WQ_NMAX / 32; ++cb) {
+                for (int cb = 0; cb < (NMAX + 31) / 32; ++cb) {
                     if (cb * 32 < p.ntile) {
                         float v[32];
                         tmem_ld32(base + uint32_t(cb * 32), v);
 #pragma unroll
-                        for (int u = 0; u < 32; ++u) sum[cb * 32 + u] = fmaf(sc, v[u], sum[cb * 32 + u]);
+                        for (int u = 0; u < 32; ++u)
+                            if (cb * 32 + u < NMAX) sum[cb * 32 + u] = fmaf(sc, v[u], sum[cb * 32 + u]);
                     }
                 }
                 tc_fence_before();
@@ -258,7 +292,7 @@ w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (!ok || !live) continue;
             const int64_t b0 = int64_t(it.nt) * p.ntile;
 #pragma unroll
-            for (int u = 0; u < WQ_NMAX; ++u) {
+            for (int u = 0; u < NMAX; ++u) {
                 const int64_t b = b0 + u;
                 if (u < p.ntile && b < p.batch) {
                     if (p.atomic) atomicAdd(p.y + b * p.m + row, sum[u]);
@@ -270,11 +304,15 @@ w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncthreads();
     if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tmem, WQ_TMEM_COLS);
+        tmem_dealloc(tmem, WqCfg<NMAX>::TMEM_COLS);
     }
 }
 
-// xp[b][k] = x[b][perm[k]] (activations in the codes' sweep order)
+// The activations in the order the A operand holds the columns: position
+// 8q + i of a row is column 8q + sigma(i) of the codes (sweep order), with
+// sigma = (0, 4, 1, 5, 2, 6, 3, 7) the order the dequantization writes a
+// packed word's nibbles in; through perm (act-order) when given:
+//   xp[b][8q + i] = x[b][perm[8q + sigma(i)]]
 __global__ void gather_cols_kernel(const __half* __restrict__ x, const int32_t* __restrict__ perm,
                                    int64_t batch, int64_t d, __half* __restrict__ xp)
 {
@@ -282,7 +320,9 @@ __global__ void gather_cols_kernel(const __half* __restrict__ x, const int32_t* 
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += int64_t(gridDim.x) * blockDim.x) {
         const int64_t b = i / d, k = i - b * d;
-        const int32_t pk = perm[k];
+        const int e = int(k & 7);
+        const int64_t ks = (k & ~int64_t(7)) + ((e & 1) ? 4 + (e >> 1) : (e >> 1));
+        const int32_t pk = perm ? perm[ks] : int32_t(ks);
         if (pk >= 0 && pk < d) {
             xp[i] = x[b * d + pk];
         } else {                                   // not followed: zero and record
@@ -297,7 +337,7 @@ __global__ void gather_cols_kernel(const __half* __restrict__ x, const int32_t* 
 extern "C" size_t gptq_w4a16_matmul_workspace_bytes(int64_t batch, int64_t d_in)
 {
     if (batch <= 0 || d_in <= 0) return 0;
-    return gptq::align_up(size_t(batch) * size_t(d_in) * 2, 1024);
+    return gptq::align_up(size_t(batch) * size_t(d_in) * 2, 1024);    // the reordered activations
 }
 
 extern "C" int gptq_w4a16_matmul(const uint16_t* x, int64_t batch, const uint32_t* qweight,
@@ -306,29 +346,28 @@ extern "C" int gptq_w4a16_matmul(const uint16_t* x, int64_t batch, const uint32_
                                  float* y, void* ws, size_t ws_bytes, void* stream)
 {
     using namespace gptq;
-    if (!x || !qweight || !scales || !qzeros || !y) return GPTQ_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(qweight) || !aligned16(y) || (perm && !aligned16(perm)) ||
-        (reinterpret_cast<uintptr_t>(scales) & 1u))
-        return GPTQ_ERR_INVALID_ARG;
-    if (perm && (!ws || !aligned16(ws) || ws_bytes < gptq_w4a16_matmul_workspace_bytes(batch, d_in)))
+    if (!x || !qweight || !scales || !qzeros || !y || !ws) return GPTQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(qweight) || !aligned16(y) || !aligned16(ws) ||
+        (perm && !aligned16(perm)) || (reinterpret_cast<uintptr_t>(scales) & 1u))
         return GPTQ_ERR_INVALID_ARG;
     if (batch < 1 || batch > (int64_t(1) << 24)) return GPTQ_ERR_SHAPE;
     if (d_in < 128 || d_in > kMaxDim || d_in % 128 != 0 || d_out < 1 || d_out > kMaxRows)
         return GPTQ_ERR_SHAPE;
+    if (ws_bytes < gptq_w4a16_matmul_workspace_bytes(batch, d_in)) return GPTQ_ERR_INVALID_ARG;
     const int64_t gsz = (group_size == -1) ? d_in : group_size;
     if (gsz < 64 || gsz % 64 != 0 || d_in % gsz != 0) return GPTQ_ERR_UNSUPPORTED;
     cudaStream_t st = as_stream(stream);
     KernelTimer kt(kKW4A16, st);
-    const __half* xs = reinterpret_cast<const __half*>(x);
-    if (perm) {
-        __half* xp = reinterpret_cast<__half*>(ws);
+    __half* xp = reinterpret_cast<__half*>(ws);
+    {
         const int64_t total = batch * d_in;
         gather_cols_kernel<<<(unsigned)std::min<int64_t>(ceil_div(total, 256),
                                                          int64_t(device_sm_count()) * 16),
-                             256, 0, st>>>(xs, perm, batch, d_in, xp);
+                             256, 0, st>>>(reinterpret_cast<const __half*>(x), perm, batch, d_in,
+                                           xp);
         count_launches();
-        xs = xp;
     }
+    const bool small = ceil_div(batch, 16) * 16 <= 32;          // the decode shape
     WqParams p{};
     p.y = y;
     p.scales = reinterpret_cast<const __half*>(scales);
@@ -337,7 +376,7 @@ extern "C" int gptq_w4a16_matmul(const uint16_t* x, int64_t batch, const uint32_
     p.d = d_in;
     p.gsz = gsz;
     p.batch = batch;
-    p.ntile = (int)std::min<int64_t>(WQ_NMAX, ceil_div(batch, 16) * 16);
+    p.ntile = (int)std::min<int64_t>(small ? 32 : WQ_NBIG, ceil_div(batch, 16) * 16);
     p.n_rt = (int)ceil_div(d_out, WQ_M);
     p.n_nt = (int)ceil_div(batch, p.ntile);
     // accumulation chunk: the largest multiple of 64 columns, at most 512,
@@ -348,9 +387,19 @@ extern "C" int gptq_w4a16_matmul(const uint16_t* x, int64_t batch, const uint32_
     const int nch = (int)(d_in / p.chunk);
     const int sms = device_sm_count();
     const int64_t tiles = int64_t(p.n_rt) * p.n_nt;
-    // split K (in whole chunks) until the items fill the SMs
+    // split K (in whole chunks) when the tiles alone leave SMs idle: the
+    // split count that minimizes rounds x chunks per item, i.e. the longest
+    // CTA's share, among 1 .. nch (fewer splits on ties: fewer atomics)
     int ks = 1;
-    if (tiles < sms) ks = (int)std::min<int64_t>(nch, ceil_div(sms, tiles));
+    if (tiles < 2 * sms) {
+        double best = 1e300;
+        for (int k = 1; k <= nch; ++k) {
+            const int64_t cps = ceil_div(nch, k);
+            const int64_t kk = ceil_div(nch, cps);
+            const double cost = double(ceil_div(tiles * kk, sms)) * double(cps + 1);
+            if (cost < best - 1e-9) { best = cost; ks = (int)kk; }
+        }
+    }
     p.chunks_per_split = (int)ceil_div(nch, ks);
     p.ksplit = (int)ceil_div(nch, p.chunks_per_split);
     p.items = (int)(tiles * p.ksplit);
@@ -362,15 +411,19 @@ extern "C" int gptq_w4a16_matmul(const uint16_t* x, int64_t batch, const uint32_
     if (encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight, (uint64_t)(d_in / 8),
                        (uint64_t)d_out, (uint64_t)(d_in / 8) * 4, WQ_K / 8, WQ_M,
                        CU_TENSOR_MAP_SWIZZLE_NONE) != GPTQ_OK ||
-        encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs, (uint64_t)d_in, (uint64_t)batch,
+        encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xp, (uint64_t)d_in, (uint64_t)batch,
                        (uint64_t)d_in * 2, WQ_K, (uint32_t)p.ntile,
                        CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK)
         return GPTQ_ERR_CUDA;
-    if (cudaFuncSetAttribute(w4a16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             WQ_SMEM) != cudaSuccess)
-        return GPTQ_ERR_CUDA;
     const int grid = std::min(p.items, sms);
-    w4a16_tc_kernel<<<grid, WQ_THREADS, WQ_SMEM, st>>>(tq, tx, p);
-    count_launches();
-    return launch_status();
+    auto run = [&](auto kern, int threads) -> int {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, WQ_SMEM) !=
+            cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        kern<<<grid, threads, WQ_SMEM, st>>>(tq, tx, p);
+        count_launches();
+        return launch_status();
+    };
+    return small ? run(w4a16_tc_kernel<32>, WqCfg<32>::THREADS)
+                 : run(w4a16_tc_kernel<WQ_NBIG>, WqCfg<WQ_NBIG>::THREADS);
 }

@@ -550,17 +550,14 @@ def gptq_w4a16_matmul(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tens
     m = qweight.shape[0]
     y = torch.empty(b, m, dtype=torch.float32, device=x.device) if y is None else y
     _need(y, "y", torch.float32)
-    nb = 0
     if perm is not None:
         _need(perm, "perm", torch.int32)
-        nb = int(load_library().gptq_w4a16_matmul_workspace_bytes(b, d))
-        ws = torch.empty(nb, dtype=torch.uint8, device=x.device) if ws is None else ws
-        nb = ws.numel()
+    nb = int(load_library().gptq_w4a16_matmul_workspace_bytes(b, d))
+    ws = torch.empty(nb, dtype=torch.uint8, device=x.device) if ws is None else ws
     _check("gptq_w4a16_matmul",
            load_library().gptq_w4a16_matmul(_ptr(x), b, _ptr(qweight), _ptr(scales), _ptr(qzeros),
-                                            _ptr(perm), m, d, int(group_size), _ptr(y),
-                                            _ptr(ws) if perm is not None else None, nb,
-                                            _stream(x)))
+                                            _ptr(perm), m, d, int(group_size), _ptr(y), _ptr(ws),
+                                            ws.numel() * ws.element_size(), _stream(x)))
     return y
 
 
