@@ -38,6 +38,7 @@ import numpy as np
 import torch
 
 METRIC = "GPTQ INT4-g128 weights quantized/sec per layer"
+PIPE_H, PIPE_P = 132, 16      # CTA caps of the Hessian and the factorization when layers overlap
 UNIT = "weights/s"
 
 
@@ -550,10 +551,13 @@ def _configs_summary(dev, peaks, steps: int, warmup: int, skip=None) -> dict:
         ms, launches, graph = _time_layer(lay, k, warmup)
         phase = _phase_split(lay, 2)
         bounds = _phase_bounds(lay, peaks)
+        kern = _kernel_entries(lay, peaks, _kernel_times(lay, 1), 1)
         units = lay.mats * lay.m * lay.d
         out[key] = {"workload": desc, "ms_per_layer": ms, "weights_per_s": units / (ms * 1e-3),
                     "steps": k, "launches_per_step": launches, "phase_ms": phase,
                     "phase_bound_ms": bounds, "whole_layer_frac": sum(bounds.values()) / ms,
+                    "kernels": {n: {kk: v[kk] for kk in ("ms", "frac") if kk in v}
+                                for n, v in kern.items()},
                     "info_ok": ok}
         del graph, lay
         torch.cuda.synchronize()
@@ -640,16 +644,15 @@ def run_ours(a):
     # layer's Hessian (dense layers; whole-job throughput over the layers)
     pipelined = None
     if E == 1 and not a.no_pipelined:
-        c0 = G.gptq_debug_launch_count()
         _barrier(ws)
         with ClockSampler(local) as clk_p:
-            pms = _pipelined_ms(lay, a.steps, a.warmup, 132, 16)
+            pms, per_layer = _pipelined_ms(lay, max(a.steps, 10), a.warmup, PIPE_H, PIPE_P,
+                                           not a.eager)
         _barrier(ws)
-        p_launches = (G.gptq_debug_launch_count() - c0) * a.steps // (a.steps + max(3, a.warmup))
         pms = _max_over_ranks(pms, ws)
         pipelined = {"value": ws * units / (pms * 1e-3), "ms_per_layer": pms,
-                     "launches": int(p_launches), "clocks": clk_p.summary(),
-                     "hessian_ctas": 132, "prepare_ctas": 16}
+                     "launches": int(round(per_layer * a.steps)), "clocks": clk_p.summary(),
+                     "hessian_ctas": PIPE_H, "prepare_ctas": PIPE_P}
 
     # end to end through the public API from pinned host memory
     e2e = _e2e(lay, a, ws, dev)
@@ -702,9 +705,10 @@ def run_ours(a):
         "clocks": pipelined["clocks"] if pipelined else clk.summary(),
         "phase_ms": phase,
         "phase_note": "per-phase split of one layer from eager launches",
-        "launch_mode": ("eager, consecutive layers: layer i's preparation on a second stream "
-                        "beside layer i+1's Hessian (persistent grids capped at 132 and 16 "
-                        "CTAs); every layer runs every phase") if pipelined else
+        "launch_mode": (("eager" if a.eager else "cuda_graph") +
+                        f", consecutive layers: layer i's preparation on a second stream beside "
+                        f"layer i+1's Hessian (persistent grids capped at {PIPE_H} and {PIPE_P} "
+                        f"CTAs); every layer runs every phase") if pipelined else
                        ("cuda_graph" if not a.eager else "eager"),
         "single_layer": single,
         # one Hessian serves q/k/v (or up/gate) in a model: the rate of the
@@ -931,13 +935,16 @@ def run_ours_one_layer(a):
         dist.destroy_process_group()
 
 
-def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int) -> float:
-    """ms per layer of consecutive layers with layer i's preparation on a
-    second stream beside layer i+1's Hessian: the factorization is a latency
-    chain that needs few SMs, the Hessian keeps the rest busy.  S, U, perm
-    and info are double-buffered; every layer still runs every phase, and
-    the timed region covers `steps` whole layers (whole-job throughput).
-    The persistent grids are capped at h_ctas / p_ctas CTAs meanwhile."""
+def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int,
+                  graph: bool = True):
+    """(ms per layer, library launches per layer) of consecutive layers with
+    layer i's preparation on a second stream beside layer i+1's Hessian: the
+    factorization is a latency chain that needs few SMs, the Hessian keeps
+    the rest busy.  S, U, perm and info are double-buffered; every layer
+    still runs every phase.  With `graph`, the schedule of `steps` layers
+    (both streams, joined by events) is captured once as a CUDA graph and
+    replayed; otherwise it is launched eagerly.  The persistent grids are
+    capped at h_ctas / p_ctas CTAs meanwhile (the caps are read at capture)."""
     G = lay.G
     dev = lay.S.device
     n = lay.n
@@ -945,10 +952,10 @@ def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int) -> flo
     U2 = [lay.U, torch.empty_like(lay.U)]
     perm2 = [lay.perm, torch.empty_like(lay.perm)]
     info2 = [lay.info, torch.zeros_like(lay.info)]
-    sH = torch.cuda.current_stream(dev)
     sP = torch.cuda.Stream(device=dev)
 
     def run(layers):
+        sH = torch.cuda.current_stream(dev)
         evH = [torch.cuda.Event() for _ in range(layers)]
         evP = [torch.cuda.Event() for _ in range(layers)]
 
@@ -980,21 +987,39 @@ def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int) -> flo
 
     G.gptq_set_max_ctas(G.GPTQ_CTAS_HESSIAN, h_ctas)
     G.gptq_set_max_ctas(G.GPTQ_CTAS_PREPARE, p_ctas)
+    g = None
     try:
         run(max(3, warmup))
         torch.cuda.synchronize()
         assert int(info2[0].item()) == 0 and int(info2[1].item()) == 0
+        c0 = G.gptq_debug_launch_count()
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run(steps)
+            torch.cuda.synchronize()
+            per_layer = (G.gptq_debug_launch_count() - c0) / steps
+            for _ in range(max(1, warmup // 2)):
+                g.replay()
+        else:
+            run(steps)
+            per_layer = (G.gptq_debug_launch_count() - c0) / steps
+        torch.cuda.synchronize()
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        if g is not None:
+            g.replay()
+        else:
+            run(steps)
+        end.record()
         torch.cuda.synchronize()
-        start.record(sH)
-        run(steps)
-        end.record(sH)
-        torch.cuda.synchronize()
+        assert int(info2[0].item()) == 0 and int(info2[1].item()) == 0
         assert G.gptq_device_status(reset=True) == 0
     finally:
         G.gptq_set_max_ctas(G.GPTQ_CTAS_HESSIAN, 0)
         G.gptq_set_max_ctas(G.GPTQ_CTAS_PREPARE, 0)
-    return start.elapsed_time(end) / steps
+    del g
+    return start.elapsed_time(end) / steps, per_layer
 
 
 def run_ours_pipelined(a):
@@ -1008,12 +1033,11 @@ def run_ours_pipelined(a):
     h_ctas, p_ctas = (int(v) for v in a.pipeline.split(","))
     lay = Layer(spec, n, dev, seed_offset=rank)
     m, d = lay.m, lay.d
-    launches0 = G.gptq_debug_launch_count()
     _barrier(ws)
     with ClockSampler(local) as clk:
-        ms = _pipelined_ms(lay, a.steps, a.warmup, h_ctas, p_ctas)
+        ms, per_layer = _pipelined_ms(lay, a.steps, a.warmup, h_ctas, p_ctas, not a.eager)
     _barrier(ws)
-    launches = (G.gptq_debug_launch_count() - launches0) * a.steps // (a.steps + max(3, a.warmup))
+    launches = int(round(per_layer * a.steps))
     ms = _max_over_ranks(ms, ws)
     line = {
         "metric": METRIC, "value": ws * m * d / (ms * 1e-3), "unit": UNIT, "n_gpus": ws,
@@ -1028,7 +1052,8 @@ def run_ours_pipelined(a):
                                 "note": "layer i's preparation overlaps layer i+1's Hessian"},
                    "l2": "inputs larger than L2 (X %.2f GB re-read every layer)" %
                          (n * d * 2 / 1e9)},
-        "gpu_launches": int(launches), "clocks": clk.summary(), "launch_mode": "eager",
+        "gpu_launches": int(launches), "clocks": clk.summary(),
+        "launch_mode": "eager" if a.eager else "cuda_graph",
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -47,6 +47,22 @@ w4a16_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t k0 = int64_t(blockIdx.y) * W4_KS;
     const int klen = (int)(d - k0 < W4_KS ? d - k0 : W4_KS);         // a multiple of 128
+    const int nch = klen / W4_CHUNK;
+    const int64_t row0 = int64_t(blockIdx.x) * (W4_WARPS * W4_ROWS) + warp * W4_ROWS;
+    auto load = [&](int c, uint2 (&q)[W4_ROWS]) {
+        const int64_t gc = k0 / W4_CHUNK + c;
+#pragma unroll
+        for (int r = 0; r < W4_ROWS; ++r) {
+            const int64_t row = row0 + r;
+            q[r] = row < m ? *reinterpret_cast<const uint2*>(qweight + row * (d / 8) + 2 * gc)
+                           : make_uint2(0u, 0u);
+        }
+    };
+    // the lane's first two chunks of weights are requested before the
+    // activations are staged: their latency overlaps the staging below
+    uint2 q0[W4_ROWS], q1[W4_ROWS];
+    if (lane < nch) load(lane, q0);
+    if (lane + 32 < nch) load(lane + 32, q1);
     for (int idx = tid; idx < B * klen; idx += W4_THREADS) {
         const int b = idx / klen, kk = idx - b * klen;
         const int64_t k = k0 + kk;
@@ -56,7 +72,6 @@ w4a16_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight,
         xs[b][kk] = in ? ldexpf(__half2float(x[b * d + src]), -4 * (kk & 3)) : 0.f;
     }
     __syncthreads();
-    const int nch = klen / W4_CHUNK;
     for (int idx = tid; idx < B * nch; idx += W4_THREADS) {
         const int b = idx / nch, c = idx - b * nch;
         float sum = 0.f;
@@ -67,7 +82,6 @@ w4a16_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight,
     __syncthreads();
 
     const int64_t G = d / g, Gz = (G + 1) / 2;
-    const int64_t row0 = int64_t(blockIdx.x) * (W4_WARPS * W4_ROWS) + warp * W4_ROWS;
     float acc[W4_ROWS][B];
 #pragma unroll
     for (int r = 0; r < W4_ROWS; ++r)
@@ -115,24 +129,17 @@ w4a16_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight,
             for (int b = 0; b < B; ++b) acc[r][b] = fmaf(s, fmaf(-z, xsum[b][c], a[b]), acc[r][b]);
         }
     };
-    auto load = [&](int c, uint2 (&q)[W4_ROWS]) {
-        const int64_t gc = k0 / W4_CHUNK + c;
-#pragma unroll
-        for (int r = 0; r < W4_ROWS; ++r) {
-            const int64_t row = row0 + r;
-            q[r] = row < m ? *reinterpret_cast<const uint2*>(qweight + row * (d / 8) + 2 * gc)
-                           : make_uint2(0u, 0u);
-        }
-    };
-    // two chunks per step, both chunks' words requested before either is used,
-    // so each warp keeps 2 KB of weight loads in flight
+    // two chunks per step; the next step's two chunks are requested before
+    // this step's are used, so each warp keeps up to 4 KB of loads in flight
     for (int c = lane; c < nch; c += 64) {
-        uint2 q0[W4_ROWS], q1[W4_ROWS];
-        const bool two = c + 32 < nch;
-        load(c, q0);
-        if (two) load(c + 32, q1);
+        uint2 n0[W4_ROWS], n1[W4_ROWS];
+        const int cn = c + 64;
+        if (cn < nch) load(cn, n0);
+        if (cn + 32 < nch) load(cn + 32, n1);
         chunk(c, q0);
-        if (two) chunk(c + 32, q1);
+        if (c + 32 < nch) chunk(c + 32, q1);
+#pragma unroll
+        for (int r = 0; r < W4_ROWS; ++r) { q0[r] = n0[r]; q1[r] = n1[r]; }
     }
 #pragma unroll
     for (int r = 0; r < W4_ROWS; ++r)

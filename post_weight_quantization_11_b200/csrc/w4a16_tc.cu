@@ -34,19 +34,23 @@
 namespace gptq {
 
 constexpr int WQ_M = 128, WQ_K = 64, WQ_NBIG = 128;
-constexpr int WQ_STAGES = 4, WQ_QSTAGES = 16;
 constexpr int WQ_CH = 512;                                   // max K per accumulation chunk
 constexpr int WQ_A_BYTES = WQ_M * WQ_K * 2;                  // 16 KB
-constexpr int WQ_B_BYTES = WQ_NBIG * WQ_K * 2;               // 16 KB (room for the larger tile)
 constexpr int WQ_Q_BYTES = WQ_M * WQ_K / 2;                  // 4 KB
 constexpr int WQ_EPI_WARPS = 4;
-constexpr int WQ_SMEM = WQ_STAGES * (WQ_A_BYTES + WQ_B_BYTES) + WQ_QSTAGES * WQ_Q_BYTES + 1024 + 512;
 
+// The decode shape (batch tile <= 32) has a small activation tile, so it
+// keeps 8 operand stages (the MMAs' commits come back late relative to the
+// short dequantization of a stage); the large shape keeps 4 of 32 KB.
 template <int NMAX> struct WqCfg {
     static constexpr int DEQ_WARPS = NMAX <= 32 ? 8 : 4;
     static constexpr int WORDS = 8 / (DEQ_WARPS / 4);          // packed words per thread and stage
     static constexpr int THREADS = 32 * (3 + DEQ_WARPS + WQ_EPI_WARPS);
     static constexpr uint32_t TMEM_COLS = 2 * NMAX < 32 ? 32 : 2 * NMAX;
+    static constexpr int STAGES = NMAX <= 32 ? 8 : 4;
+    static constexpr int QSTAGES = NMAX <= 32 ? 8 : 16;
+    static constexpr int B_BYTES = NMAX * WQ_K * 2;            // 4 KB or 16 KB
+    static constexpr int SMEM = STAGES * (WQ_A_BYTES + B_BYTES) + QSTAGES * WQ_Q_BYTES + 1024 + 512;
 };
 
 struct WqParams {
@@ -92,8 +96,10 @@ w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int WQ_STAGES = WqCfg<NMAX>::STAGES, WQ_QSTAGES = WqCfg<NMAX>::QSTAGES;
+    constexpr int WQ_B_BYTES = WqCfg<NMAX>::B_BYTES;
     uint8_t* sA = smem;                                          // stages x 16 KB
-    uint8_t* sB = sA + WQ_STAGES * WQ_A_BYTES;                   // stages x 16 KB
+    uint8_t* sB = sA + WQ_STAGES * WQ_A_BYTES;                   // stages x (4 or 16 KB)
     uint8_t* sQ = sB + WQ_STAGES * WQ_B_BYTES;                   // qstages x 4 KB
     uint64_t* qfull = reinterpret_cast<uint64_t*>(sQ + WQ_QSTAGES * WQ_Q_BYTES);
     uint64_t* qempty = qfull + WQ_QSTAGES;
@@ -416,14 +422,14 @@ extern "C" int gptq_w4a16_matmul(const uint16_t* x, int64_t batch, const uint32_
                        CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK)
         return GPTQ_ERR_CUDA;
     const int grid = std::min(p.items, sms);
-    auto run = [&](auto kern, int threads) -> int {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, WQ_SMEM) !=
+    auto run = [&](auto kern, int threads, int smem) -> int {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
             cudaSuccess)
             return GPTQ_ERR_CUDA;
-        kern<<<grid, threads, WQ_SMEM, st>>>(tq, tx, p);
+        kern<<<grid, threads, smem, st>>>(tq, tx, p);
         count_launches();
         return launch_status();
     };
-    return small ? run(w4a16_tc_kernel<32>, WqCfg<32>::THREADS)
-                 : run(w4a16_tc_kernel<WQ_NBIG>, WqCfg<WQ_NBIG>::THREADS);
+    return small ? run(w4a16_tc_kernel<32>, WqCfg<32>::THREADS, WqCfg<32>::SMEM)
+                 : run(w4a16_tc_kernel<WQ_NBIG>, WqCfg<WQ_NBIG>::THREADS, WqCfg<WQ_NBIG>::SMEM);
 }

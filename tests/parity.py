@@ -10,7 +10,11 @@ Tolerances (written here, used by every parity test):
             bar holds for the free-running comparison, cascades included; at
             other widths it counts the tie flips themselves (the codes the
             oracle decides differently on the GPU's own trajectory), since
-            one flip there moves tens to hundreds of later codes of its row
+            one flip there moves tens to hundreds of later codes of its row;
+            there the scale and zero-point bars are likewise taken on that
+            trajectory (at 2 bits a group made only of earlier columns'
+            cancelling corrections can differ by more than 1e-4 between fp32
+            and fp64 feedback before any code differs)
   * scales: for every group of a row before that row's first code mismatch,
             the GPU's fp16 scale is the fp16 rounding of some value within
             1e-4 relative of the oracle's pre-fp16 scale
@@ -61,12 +65,13 @@ def fp16_range(s_pre: np.ndarray, rel: float):
 
 
 def compare_sweep(gpu: dict, orc: dict, group_size: int, report: dict | None = None,
-                  code_frac: float = CODE_FRAC):
+                  code_frac: float = CODE_FRAC, group_bars: bool = True):
     """gpu/orc: dicts with codes (m x d uint8), scales (m x G uint16 bits),
     zeros (m x G uint8); orc also has s_pre.  Asserts the code and scale
     tolerances and returns statistics.  code_frac: the bar on the free-running
     code mismatches (1.0 where the caller takes the bar on the teacher-forced
-    run instead)."""
+    run instead); group_bars False likewise leaves the scale and zero-point
+    bars to the teacher-forced run (and reports the free-running deviation)."""
     cg, co = gpu["codes"], orc["codes"]
     m, d = co.shape
     mism = cg != co
@@ -82,15 +87,19 @@ def compare_sweep(gpu: dict, orc: dict, group_size: int, report: dict | None = N
     lo, hi = fp16_range(orc["s_pre"], SCALE_REL)
     in_range = (sg >= lo) & (sg <= hi)
     bad = ok_groups & ~in_range
-    assert not bad.any(), f"{int(bad.sum())} scales outside 1e-4 of the oracle's pre-fp16 scale"
     same_s = gpu["scales"] == orc["scales"]
     zdiff = ok_groups & same_s & (gpu["zeros"] != orc["zeros"])
-    assert zdiff.sum() <= CODE_FRAC * max(1, ok_groups.sum()) + 1, \
-        f"{int(zdiff.sum())} zero points differ under equal scales"
     zstep = np.abs(gpu["zeros"].astype(np.int32) - orc["zeros"].astype(np.int32))
-    assert (zstep[zdiff] <= 1).all(), "a zero point differs by more than one step"
+    dev = np.abs(sg.astype(np.float64) / orc["s_pre"].astype(np.float64) - 1.0)
+    if group_bars:
+        assert not bad.any(), f"{int(bad.sum())} scales outside 1e-4 of the oracle's pre-fp16 scale"
+        assert zdiff.sum() <= CODE_FRAC * max(1, ok_groups.sum()) + 1, \
+            f"{int(zdiff.sum())} zero points differ under equal scales"
+        assert (zstep[zdiff] <= 1).all(), "a zero point differs by more than one step"
     st = dict(code_mismatch_frac=frac, rows_with_mismatch=int((first < d).sum()),
-              scale_exact_frac=float(same_s[ok_groups].mean()) if ok_groups.any() else 1.0)
+              scale_exact_frac=float(same_s[ok_groups].mean()) if ok_groups.any() else 1.0,
+              free_scales_off=int(bad.sum()),
+              free_max_scale_dev=float(dev[ok_groups].max()) if ok_groups.any() else 0.0)
     if report is not None:
         report.update(st)
     return st

@@ -56,11 +56,13 @@ def _gpu_layer(W, X, bits=4, group_size=128, act_order=False, damp=0.01):
 def _check_layer(W, X, bits=4, group_size=128, act_order=False, rows=None, code_bar="free"):
     """H-forced protocol: the oracle takes the GPU's S (promoted to fp64).
     code_bar "free": at most 1e-3 of the codes differ in the free-running
-    comparison (every later code a tie flip changes counts too); "forced":
-    the 1e-3 bar counts the codes the oracle decides differently on the GPU's
-    own trajectory (the teacher-forced run), i.e. the tie flips themselves
-    -- the reading for widths other than 4 bits, where one tie flip moves
-    tens to hundreds of later codes of its row."""
+    comparison (every later code a tie flip changes counts too), and the
+    scale and zero-point bars hold there too; "forced": the 1e-3 bar counts
+    the codes the oracle decides differently on the GPU's own trajectory
+    (the teacher-forced run), i.e. the tie flips themselves, and the scale
+    and zero-point bars are those of that run -- the reading for widths
+    other than 4 bits, where one tie flip moves tens to hundreds of later
+    codes of its row."""
     n = X.shape[0]
     g = _gpu_layer(W, X, bits, group_size, act_order)
     assert g["info"] == 0
@@ -73,7 +75,8 @@ def _check_layer(W, X, bits=4, group_size=128, act_order=False, rows=None, code_
     assert P.rel_fro(g["U"].astype(np.float64), ref["U"]) <= P.U_TOL
     st = P.compare_sweep(g, dict(codes=ref["codes"], scales=ref["scales"], zeros=ref["zeros"],
                                  s_pre=ref["s_pre"]), group_size,
-                         code_frac=P.CODE_FRAC if code_bar == "free" else 1.0)
+                         code_frac=P.CODE_FRAC if code_bar == "free" else 1.0,
+                         group_bars=code_bar == "free")
     H64 = 2.0 * S_gpu / n
     perm = ref["perm"]
     lg = P.layer_loss_of(W64, g["codes"], g["scales"], g["zeros"], group_size, perm, H64)
