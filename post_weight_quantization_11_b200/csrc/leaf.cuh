@@ -8,15 +8,16 @@
 
 namespace gptq {
 
-constexpr int PN = 128;            // panel / leaf width
+constexpr int PN = 128;            // leaf width
+constexpr int PW = 8;              // panel width of the leaf's factorization
 // leaf_factor_invert: factor the symmetric block held in `a` (lower triangle
 // read) into L (lower, in `a`) and write X = L^-1 into `xs` (which the caller
-// zeroed): a 4-column right-looking factorization pipelined between a panel
-// warp and update warps (below), then X from the 4x4 diagonal inverses by
-// five doubling levels, X_BC = -X_C (B X_A), as small GEMMs in shared memory.
+// zeroed): an 8-column right-looking factorization pipelined between a panel
+// warp and update warps (below), then X from the 8x8 diagonal inverses by
+// four doubling levels, X_BC = -X_C (B X_A), as small GEMMs in shared memory.
 constexpr int LDA = PN + 4;                  // row stride of the shared 128x128 blocks
 constexpr int LDT = 68;                      // row stride of the doubling temporary
-constexpr int LPC_BYTES = 2 * PN * 16;       // two compact copies of a 4-column panel
+constexpr int LPC_BYTES = 2 * (PW / 4) * PN * 16;   // compact panel copies, two step parities
 constexpr int LTB_BYTES = 64 * LDT * 4;      // tb: doubling temporary, or panel copies + mbarriers
 static_assert(LPC_BYTES + 64 <= LTB_BYTES, "panel copies and barriers fit in tb");
 constexpr size_t LSMEM = sizeof(float) * 2 * PN * LDA + LTB_BYTES;
@@ -105,19 +106,21 @@ __device__ __forceinline__ void rank4_tile(float* __restrict__ a, const float4* 
 // the bounded waits (tc_common.cuh): a wait that gives up records
 // kErrWaitLeaf and every role leaves early; the block is then garbage.
 //
-// Factorization, 4 columns per step c0, software-pipelined across two roles:
-//   warp 0 (panel):   factor and invert the 4x4 pivot block in registers,
-//                     solve the 4 panel entries of every row below (into a,
-//                     and into a compact copy in tb, double-buffered by step
-//                     parity) and publish;
-//   warps 1.. (update): after the publish, first apply the panel's rank-4
-//                     update to the next panel's 4 columns and signal that
+// Factorization, 8 columns per step c0, software-pipelined across two roles:
+//   warp 0 (panel):   factor and invert the 8x8 pivot block in registers,
+//                     solve the 8 panel entries of every row below (into a,
+//                     and into two compact 4-column copies in tb,
+//                     double-buffered by step parity) and publish;
+//   warps 1.. (update): after the publish, first apply the panel's rank-8
+//                     update to the next panel's 8 columns and signal that
 //                     the panel warp may go on, then apply it to the rest of
-//                     the trailing triangle (columns >= c0 + 8, which the
+//                     the trailing triangle (columns >= c0 + 16, which the
 //                     panel warp neither reads nor writes in its next step).
+// Eight columns per step halve the number of steps, hence of hand-offs,
+// against a 4-column panel; the panel warp's solve does twice the work.
 // The hand-offs are mbarriers alternating by step parity: pub[parity]
 // completes when the panel warp has published step c0 and every update warp
-// has finished the trailing update of step c0 - 4 (which orders the updates
+// has finished the trailing update of step c0 - 8 (which orders the updates
 // of consecutive steps), nxt[parity] when every update warp has updated the
 // next panel's columns.  The next use of a barrier always follows a wait that
 // saw its previous phase complete.
@@ -142,19 +145,19 @@ __device__ __forceinline__ void leaf_factor_invert(float* __restrict__ a, float*
     }
     __syncthreads();
     if (warp == 0) {
-        for (int c0 = 0; c0 < PN; c0 += 4) {
-            const int st = c0 >> 2;
+        for (int c0 = 0; c0 < PN; c0 += PW) {
+            const int st = c0 / PW;
             if (c0 > 0 && !mbar_wait(&nxt[(st - 1) & 1], ((st - 1) >> 1) & 1, kErrWaitLeaf, abort))
                 break;
-            // 4x4 diagonal block: Cholesky factor g and its inverse h, in registers
-            float g[4][4], h[4][4];
+            // 8x8 diagonal block: Cholesky factor g and its inverse h, in registers
+            float g[PW][PW], h[PW][PW];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < PW; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) g[i][j] = (j <= i) ? a[(c0 + i) * LDA + c0 + j] : 0.f;
-            float rd[4];
+                for (int j = 0; j < PW; ++j) g[i][j] = (j <= i) ? a[(c0 + i) * LDA + c0 + j] : 0.f;
+            float rd[PW];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < PW; ++j) {
                 const float djj = g[j][j];
                 const bool bad = !(djj > 0.f);
                 if (bad && lane == 0 && info)
@@ -166,16 +169,16 @@ __device__ __forceinline__ void leaf_factor_invert(float* __restrict__ a, float*
                 rd[j] = y;
                 g[j][j] = djj * y;
 #pragma unroll
-                for (int i = j + 1; i < 4; ++i) g[i][j] *= rd[j];
+                for (int i = j + 1; i < PW; ++i) g[i][j] *= rd[j];
 #pragma unroll
-                for (int i = j + 1; i < 4; ++i)
+                for (int i = j + 1; i < PW; ++i)
 #pragma unroll
                     for (int k = j + 1; k <= i; ++k) g[i][k] = fmaf(-g[i][j], g[k][j], g[i][k]);
             }
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {                 // forward substitution, column c
+            for (int c = 0; c < PW; ++c) {                // forward substitution, column c
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
+                for (int r = 0; r < PW; ++r) {
                     if (r < c) { h[r][c] = 0.f; continue; }
                     float t = (r == c) ? 1.f : 0.f;
 #pragma unroll
@@ -183,33 +186,42 @@ __device__ __forceinline__ void leaf_factor_invert(float* __restrict__ a, float*
                     h[r][c] = t * rd[r];
                 }
             }
-            // panel rows below: L[r][c0..c0+3] = A[r][c0..c0+3] h^T
-            float4* pc = pcb + (st & 1) * PN;
-            for (int r = c0 + 4 + lane; r < PN; r += 32) {
-                const float4 v = *reinterpret_cast<const float4*>(a + r * LDA + c0);
-                const float av[4] = {v.x, v.y, v.z, v.w};
-                float o[4];
+            __syncwarp();                                  // every lane has read the pivot block
+            if (lane < PW) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int i = 0; i < PW; ++i)
+                    if (lane == i) {
+                        *reinterpret_cast<float4*>(a + (c0 + i) * LDA + c0) =
+                            make_float4(g[i][0], g[i][1], g[i][2], g[i][3]);
+                        *reinterpret_cast<float4*>(a + (c0 + i) * LDA + c0 + 4) =
+                            make_float4(g[i][4], g[i][5], g[i][6], g[i][7]);
+                        *reinterpret_cast<float4*>(xs + (c0 + i) * LDA + c0) =
+                            make_float4(h[i][0], h[i][1], h[i][2], h[i][3]);
+                        *reinterpret_cast<float4*>(xs + (c0 + i) * LDA + c0 + 4) =
+                            make_float4(h[i][4], h[i][5], h[i][6], h[i][7]);
+                    }
+            }
+            // panel rows below: L[r][c0..c0+7] = A[r][c0..c0+7] h^T, into a and
+            // into the compact copies (columns 0-3 in pc[0..], 4-7 in pc[PN..])
+            float4* pc = pcb + (st & 1) * 2 * PN;
+            for (int r = c0 + PW + lane; r < PN; r += 32) {
+                const float4 v0 = *reinterpret_cast<const float4*>(a + r * LDA + c0);
+                const float4 v1 = *reinterpret_cast<const float4*>(a + r * LDA + c0 + 4);
+                const float av[PW] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                float o[PW];
+#pragma unroll
+                for (int c = 0; c < PW; ++c) {
                     float t = 0.f;
 #pragma unroll
                     for (int k = 0; k <= c; ++k) t = fmaf(av[k], h[c][k], t);
                     o[c] = t;
                 }
-                const float4 lv = make_float4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<float4*>(a + r * LDA + c0) = lv;
-                pc[panel_slot(r)] = lv;
-            }
-            __syncwarp();                                  // every lane has read the pivot block
-            if (lane < 4) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (lane == i) {
-                        *reinterpret_cast<float4*>(a + (c0 + i) * LDA + c0) =
-                            make_float4(g[i][0], g[i][1], g[i][2], g[i][3]);
-                        *reinterpret_cast<float4*>(xs + (c0 + i) * LDA + c0) =
-                            make_float4(h[i][0], h[i][1], h[i][2], h[i][3]);
-                    }
+                const float4 l0 = make_float4(o[0], o[1], o[2], o[3]);
+                const float4 l1 = make_float4(o[4], o[5], o[6], o[7]);
+                *reinterpret_cast<float4*>(a + r * LDA + c0) = l0;
+                *reinterpret_cast<float4*>(a + r * LDA + c0 + 4) = l1;
+                pc[panel_slot(r)] = l0;
+                pc[PN + panel_slot(r)] = l1;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&pub[st & 1]);      // panel published
@@ -217,22 +229,30 @@ __device__ __forceinline__ void leaf_factor_invert(float* __restrict__ a, float*
     } else {
         const int ut = tid - 32;
         if (lane == 0) mbar_arrive(&pub[0]);              // nothing before step 0
-        for (int c0 = 0; c0 < PN; c0 += 4) {
-            const int st = c0 >> 2;
+        for (int c0 = 0; c0 < PN; c0 += PW) {
+            const int st = c0 / PW;
             if (!mbar_wait(&pub[st & 1], (st >> 1) & 1, kErrWaitLeaf, abort)) break;
-            const int nt = (PN - c0 - 4) / 4;              // 4-row tiles below the panel
-            const float4* pc = pcb + (st & 1) * PN;
-            if (ut < nt) rank4_tile(a, pc, c0 + 4 + 4 * ut, c0 + 4);
+            const int nt = (PN - c0 - PW) / 4;             // 4-row tiles below the panel
+            const float4* pc = pcb + (st & 1) * 2 * PN;
+            // the next panel's 8 columns (two tile columns), lower part only
+            for (int t = ut; t < 2 * nt; t += NU) {
+                const int ti = t >> 1, tj = t & 1;
+                if (ti < tj) continue;                     // wholly above the diagonal
+                rank4_tile(a, pc, c0 + PW + 4 * ti, c0 + PW + 4 * tj);
+                rank4_tile(a, pc + PN, c0 + PW + 4 * ti, c0 + PW + 4 * tj);
+            }
             __syncwarp();
-            if (c0 + 4 < PN && lane == 0) mbar_arrive(&nxt[st & 1]);   // next panel's columns
-            const int tiles = nt * (nt - 1) / 2;           // tile columns >= 1: columns >= c0 + 8
+            if (c0 + PW < PN && lane == 0) mbar_arrive(&nxt[st & 1]);   // next panel's columns
+            const int n2 = max(nt - PW / 4, 0);            // tile columns >= c0 + 16
+            const int tiles = n2 * (n2 + 1) / 2;
             for (int t = ut; t < tiles; t += NU) {
                 int ti, tj;
                 tri_index(t, ti, tj);
-                rank4_tile(a, pc, c0 + 8 + 4 * ti, c0 + 8 + 4 * tj);
+                rank4_tile(a, pc, c0 + 2 * PW + 4 * ti, c0 + 2 * PW + 4 * tj);
+                rank4_tile(a, pc + PN, c0 + 2 * PW + 4 * ti, c0 + 2 * PW + 4 * tj);
             }
             __syncwarp();
-            if (c0 + 4 < PN && lane == 0) mbar_arrive(&pub[(st + 1) & 1]);   // next step
+            if (c0 + PW < PN && lane == 0) mbar_arrive(&pub[(st + 1) & 1]);   // next step
         }
     }
     __syncthreads();
@@ -242,8 +262,8 @@ __device__ __forceinline__ void leaf_factor_invert(float* __restrict__ a, float*
     }
     __syncthreads();
 
-    // X from the 4x4 diagonal inverses by doubling: s = 4, 8, ..., 64
-    for (int s = 4; s < PN; s *= 2) {
+    // X from the 8x8 diagonal inverses by doubling: s = 8, 16, 32, 64
+    for (int s = PW; s < PN; s *= 2) {
         const int pairs = PN / (2 * s);
         const int ts = s / 4, tpp = ts * ts;               // 4x4 tiles per pair
         // T = B X_A, B = L[o+s+i][o+k], X_A = X[o+k][o+j] (zero for k < j)
