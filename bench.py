@@ -360,19 +360,20 @@ def _make_layer(workload: str, layer: int, tokens: int, dev, seed_offset=0):
     return lay, desc
 
 
-def _update_flops(m: int, d: int, B: int = 128, outer: int = 4) -> float:
-    """Algorithmic flops of the lazy-batch feedback onto later blocks, as the
-    library schedules it: after each block of B columns the rest of its
-    outer block of outer*B columns (K = B), and after each outer block every
-    column beyond it (K = outer*B); 2 m K N per product."""
+def _update_flops(m: int, d: int, B: int = 128, outer: int = 4, near: bool = True,
+                  far: bool = True) -> float:
+    """Algorithmic flops of the lazy-batch feedback onto later blocks: after
+    each block of B columns the rest of its outer block of outer*B columns
+    (K = B, `near`), and after each outer block every column beyond it
+    (K = outer*B, `far`); 2 m K N per product."""
     f = 0.0
     ob = outer * B
     for j0 in range(0, d, B):
         o0 = j0 // ob * ob
         o1 = min(d, o0 + ob)
-        if j0 + B < o1:
+        if near and j0 + B < o1:
             f += 2.0 * m * B * (o1 - j0 - B)
-        if j0 + B == o1 and o1 < d:
+        if far and j0 + B == o1 and o1 < d:
             f += 2.0 * m * (o1 - o0) * (d - o1)
     return f
 
@@ -435,12 +436,15 @@ def _kernel_entries(lay, peaks, times: dict, steps: int) -> dict:
     uf, nf = t("update_far")
     if un or uf:
         ms = (un or 0.0) + (uf or 0.0)
-        a = E * 3 * _update_flops(m, d) / (ms * 1e-3) / 1e12
+        a = E * 3 * _update_flops(m, d, near=bool(un)) / (ms * 1e-3) / 1e12
         out["update"] = {"bound": "tensor", "ms": ms, "launches": nn + nf, "achieved": a,
                          "peak": tf32, "unit": "TFLOP/s", "frac": a / tf32,
                          "near_ms": un, "far_ms": uf,
-                         "work": "3 x sum of 2 m K N split-TF32 flops of the lazy-batch "
-                                 "schedule (K = 128 near, 512 far)"}
+                         "work": "3 x sum of 2 m K N split-TF32 flops of the tensor-core "
+                                 "updates (K = 512 beyond each outer block" +
+                                 (", K = 128 inside it)" if un else
+                                  "; inside an outer block the sweep kernel updates on the "
+                                  "CUDA cores)")}
     ms, nl = t("sweep")
     if ms:
         b = E * (13.0 * m * d + 4.0 * d * d)
@@ -448,7 +452,10 @@ def _kernel_entries(lay, peaks, times: dict, steps: int) -> dict:
         out["sweep"] = {"bound": "hbm", "ms": ms, "launches": nl, "achieved": a, "peak": hbm,
                         "unit": "GB/s", "frac": a / hbm,
                         "work": "W fp32 in (4 B), codes (1 B) and E split (8 B) out per weight, "
-                                "U diagonal blocks in; issue-bound in practice"}
+                                "U diagonal blocks in; a chain of d dependent column decisions "
+                                "per row in practice" +
+                                ("" if un else "; fused with the fp32 updates inside each "
+                                 "512-column outer block (2 m 128 N flops per block)")}
     ms, nl = t("pack")
     if ms:
         b = E * 1.53 * m * d

@@ -57,9 +57,28 @@ __host__ __device__ __forceinline__ float div_rn_recip(float x, float s, float r
     return fmaf(fmaf(-q, s, x), r, q);
 }
 
+// Round-to-nearest-even to an integer on the FMA pipe (rintf issues on the
+// slower conversion unit): adding and removing 1.5 * 2^23 leaves the sum
+// with a unit last place, so the first add rounds x to an integer, ties to
+// even.  Exact for |x| <= 2^22; beyond that the result stays within 2 of x,
+// which the clamp of every caller (codes in [0, maxq], maxq <= 255) maps to
+// the same code as the exact rounding.
+__device__ __forceinline__ float rne_for_clamp(float x)
+{
+    constexpr float kMagic = 12582912.f;   // 1.5 * 2^23
+    return __fsub_rn(__fadd_rn(x, kMagic), kMagic);
+}
+
+// The integral value of c in [0, 255] as a byte, without a conversion
+// instruction: c + 2^23 holds c in its low mantissa bits.
+__device__ __forceinline__ uint32_t code_byte(float c)
+{
+    return __float_as_uint(__fadd_rn(c, 8388608.f)) & 0xffu;
+}
+
 __device__ __forceinline__ float quant_code_fast(float x, const GroupQ& g, float maxqf)
 {
-    const float c = __fadd_rn(rintf(div_rn_recip(x, g.s, g.r)), g.z);
+    const float c = __fadd_rn(rne_for_clamp(div_rn_recip(x, g.s, g.r)), g.z);
     return fminf(fmaxf(c, 0.f), maxqf);
 }
 

@@ -5,7 +5,7 @@
 //
 // Per 128-column block b (columns j0 .. j0+127, sweep order):
 //   block_sweep:  every row runs the 128 sequential steps with the block's
-//                 columns in registers (16 lanes per row, 8 columns per lane)
+//                 columns in registers (8 lanes per row, 16 columns per lane)
 //                 and U's 128x128 diagonal block in shared memory; writes the
 //                 codes, group scales/zeros, the scaled errors E (rows x 128)
 //                 and accumulates sum E_j^2 per row.
@@ -25,7 +25,8 @@ constexpr int SW_LPR = 8;          // lanes per row
 constexpr int SW_CPL = SW_B / SW_LPR;   // columns per lane (16)
 constexpr int SW_Q4 = SW_CPL / 4;       // float4 chunks per lane (4)
 constexpr int SW_THREADS = 128;
-constexpr int SW_ROWS = 2 * SW_THREADS / SW_LPR;   // rows per CTA (32: two per lane group)
+constexpr int SW_RPL = 2;          // rows per lane group
+constexpr int SW_ROWS = SW_RPL * SW_THREADS / SW_LPR;   // rows per CTA
 constexpr unsigned FULL = 0xffffffffu;
 
 // W_work[r][k] = float(W[r][perm[k]])
@@ -45,9 +46,11 @@ __global__ void init_work_kernel(const T* __restrict__ W, const int32_t* __restr
 }
 
 // One 128-column block of the sweep for all rows.  8 lanes per row, each lane
-// holding 16 consecutive columns of TWO rows in registers (rows g and g+4 of
-// its warp's 8), so every U value a lane reads from shared memory serves two
-// rows and each warp carries two independent decision chains.  U's 128x128
+// holding 16 consecutive columns of SW_RPL rows in registers (rows g, g+4 ..
+// of its warp's rows).  One row per lane group: 16 rows per CTA, so a layer
+// of a few thousand rows puts two CTAs (eight independent decision chains per
+// scheduler pair) on most SMs, and the chains of different warps hide each
+// other's latency.  U's 128x128
 // diagonal block (its strictly-lower part zeroed) and 1/U_jj live in shared
 // memory.  Step j: every lane of a row takes the same fp32 decision on column
 // j (quant_code_fast: no division) and applies w[k] -= E_j U[j][k] to its
@@ -61,6 +64,121 @@ __global__ void init_work_kernel(const T* __restrict__ W, const int32_t* __restr
 // one group per row); the kernel loads them at each group start inside the
 // block and at the block's first column instead of reducing min/max.  GS is
 // then min(group size, 128) and gsz the group size.
+// The 128 sequential steps of one block for this lane's rows: w holds the
+// lane's 16 columns of each row (updated through every earlier column), Us
+// the block's diagonal U block (strictly-lower part zeroed, chunk-major) and
+// rdiag 1/U_jj.  Writes the group scales/zeros of groups starting in the
+// block (dynamic groups) and leaves in Ev/cp the errors and codes of the
+// 16 columns this lane owns, in loss the row's sum of E_j^2 over the block.
+template <int GS, bool STATIC>
+__device__ __forceinline__ void sweep_core(const float* __restrict__ Us,
+                                           const float* __restrict__ rdiag,
+                                           float (&w)[SW_RPL][SW_CPL],
+                                           const int64_t (&row)[SW_RPL],
+                                           const bool (&valid)[SW_RPL], int sub, int src_base,
+                                           int64_t G, int64_t gsz, int64_t j0, float maxqf,
+                                           __half* __restrict__ scales,
+                                           uint8_t* __restrict__ zeros,
+                                           float (&Ev)[SW_RPL][SW_CPL],
+                                           uint32_t (&cp)[SW_RPL][SW_Q4], float (&loss)[SW_RPL])
+{
+    GroupQ gq[SW_RPL];
+#pragma unroll
+    for (int r = 0; r < SW_RPL; ++r) {
+#pragma unroll
+        for (int q = 0; q < SW_Q4; ++q) cp[r][q] = 0u;
+        loss[r] = 0.f;
+        gq[r].s = 1.f; gq[r].z = 0.f; gq[r].r = 1.f; gq[r].h = __float2half(1.f);
+    }
+    float xn[SW_RPL];
+#pragma unroll
+    for (int r = 0; r < SW_RPL; ++r) xn[r] = __shfl_sync(FULL, w[r][0], src_base);
+
+#pragma unroll 1
+    for (int jo = 0; jo < SW_LPR; ++jo) {
+#pragma unroll
+        for (int ji = 0; ji < SW_CPL; ++ji) {
+            const int j = jo * SW_CPL + ji;
+            if (STATIC && ji == 0 && (jo * SW_CPL) % GS == 0) {
+                const int64_t gi = (j0 + j) / gsz;
+#pragma unroll
+                for (int r = 0; r < SW_RPL; ++r) {
+                    if (valid[r]) {
+                        const __half h = scales[row[r] * G + gi];
+                        gq[r].h = h;
+                        gq[r].s = __half2float(h);
+                        gq[r].z = float(zeros[row[r] * G + gi]);
+                        gq[r].r = __frcp_rn(gq[r].s);
+                    }
+                }
+            } else if (ji == 0 && (jo * SW_CPL) % GS == 0) {
+                constexpr int span = GS / SW_CPL;            // lanes covering one group
+                const bool in_group = sub >= jo && sub < jo + span;
+#pragma unroll
+                for (int r = 0; r < SW_RPL; ++r) {
+                    float mn = 0.f, mx = 0.f;
+                    if (in_group) {
+#pragma unroll
+                        for (int q = 0; q < SW_CPL; ++q) { mn = fminf(mn, w[r][q]); mx = fmaxf(mx, w[r][q]); }
+                    }
+#pragma unroll
+                    for (int o = 1; o < SW_LPR; o <<= 1) {
+                        mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+                        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+                    }
+                    gq[r] = group_params(mn, mx, maxqf);
+                    if (valid[r] && sub == jo) {
+                        const int64_t gi = (j0 + j) / GS;
+                        scales[row[r] * G + gi] = gq[r].h;
+                        zeros[row[r] * G + gi] = (uint8_t)gq[r].z;
+                    }
+                }
+            }
+            // next column's values before this column's correction (off the chain)
+            float xpre[SW_RPL];
+#pragma unroll
+            for (int r = 0; r < SW_RPL; ++r) xpre[r] = 0.f;
+            float unext = 0.f;
+#pragma unroll
+            for (int r = 0; r < SW_RPL; ++r) {
+                if (ji + 1 < SW_CPL) xpre[r] = __shfl_sync(FULL, w[r][ji + 1], src_base | jo);
+                else if (jo + 1 < SW_LPR) xpre[r] = __shfl_sync(FULL, w[r][0], src_base | (jo + 1));
+            }
+            if (j + 1 < SW_B) {
+                const int f = (j + 1) >> 2;
+                unext = Us[j * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 + ((j + 1) & 3)];
+            }
+            const float rdj = rdiag[j];
+            float Ej[SW_RPL];
+#pragma unroll
+            for (int r = 0; r < SW_RPL; ++r) {
+                const float x = xn[r];
+                const float c = quant_code_fast(x, gq[r], maxqf);
+                const float q = gq[r].s * (c - gq[r].z);
+                Ej[r] = (x - q) * rdj;
+                loss[r] = fmaf(Ej[r], Ej[r], loss[r]);
+                if (sub == jo) {
+                    Ev[r][ji] = Ej[r];
+                    cp[r][ji / 4] |= code_byte(c) << (8 * (ji % 4));
+                }
+                xn[r] = fmaf(-Ej[r], unext, xpre[r]);
+            }
+            const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B);
+#pragma unroll
+            for (int q4 = 0; q4 < SW_Q4; ++q4) {
+                const float4 u = urow[q4 * SW_LPR + sub];
+#pragma unroll
+                for (int r = 0; r < SW_RPL; ++r) {
+                    w[r][4 * q4 + 0] = fmaf(-Ej[r], u.x, w[r][4 * q4 + 0]);
+                    w[r][4 * q4 + 1] = fmaf(-Ej[r], u.y, w[r][4 * q4 + 1]);
+                    w[r][4 * q4 + 2] = fmaf(-Ej[r], u.z, w[r][4 * q4 + 2]);
+                    w[r][4 * q4 + 3] = fmaf(-Ej[r], u.w, w[r][4 * q4 + 3]);
+                }
+            }
+        }
+    }
+}
+
 template <int GS, bool STATIC>
 __global__ void __launch_bounds__(SW_THREADS)
 block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
@@ -103,16 +221,17 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
 
     const int lane = tid & 31, sub = lane & (SW_LPR - 1);
     const int src_base = lane & ~(SW_LPR - 1);
-    const int64_t rbase = int64_t(blockIdx.x) * SW_ROWS + (tid >> 5) * 8 + (lane >> 3);
-    int64_t row[2];
-    bool valid[2];
+    const int64_t rbase = int64_t(blockIdx.x) * SW_ROWS + (tid >> 5) * (32 / SW_LPR * SW_RPL) +
+                          lane / SW_LPR;
+    int64_t row[SW_RPL];
+    bool valid[SW_RPL];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) { row[r] = rbase + 4 * r; valid[r] = row[r] < m; }
+    for (int r = 0; r < SW_RPL; ++r) { row[r] = rbase + (32 / SW_LPR) * r; valid[r] = row[r] < m; }
     const int64_t G = d / gsz;
 
-    float w[2][SW_CPL];
+    float w[SW_RPL][SW_CPL];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < SW_RPL; ++r) {
         if (valid[r]) {
             const float4* p = reinterpret_cast<const float4*>(Wk + row[r] * d + j0 + SW_CPL * sub);
 #pragma unroll
@@ -127,107 +246,19 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     }
     __syncthreads();
 
-    float Ev[2][SW_CPL];
-    uint32_t cp[2][SW_Q4];
-    float loss[2] = {0.f, 0.f};
-    GroupQ gq[2];
+    float Ev[SW_RPL][SW_CPL];
+    uint32_t cp[SW_RPL][SW_Q4];
+    float loss[SW_RPL];
+    sweep_core<GS, STATIC>(Us, rdiag, w, row, valid, sub, src_base, G, gsz, j0, maxqf, scales,
+                           zeros, Ev, cp, loss);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-#pragma unroll
-        for (int q = 0; q < SW_Q4; ++q) cp[r][q] = 0u;
-        gq[r].s = 1.f; gq[r].z = 0.f; gq[r].r = 1.f; gq[r].h = __float2half(1.f);
-    }
-    float xn[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) xn[r] = __shfl_sync(FULL, w[r][0], src_base);
-
-#pragma unroll 1
-    for (int jo = 0; jo < SW_LPR; ++jo) {
-#pragma unroll
-        for (int ji = 0; ji < SW_CPL; ++ji) {
-            const int j = jo * SW_CPL + ji;
-            if (STATIC && ji == 0 && (jo * SW_CPL) % GS == 0) {
-                const int64_t gi = (j0 + j) / gsz;
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    if (valid[r]) {
-                        const __half h = scales[row[r] * G + gi];
-                        gq[r].h = h;
-                        gq[r].s = __half2float(h);
-                        gq[r].z = float(zeros[row[r] * G + gi]);
-                        gq[r].r = __frcp_rn(gq[r].s);
-                    }
-                }
-            } else if (ji == 0 && (jo * SW_CPL) % GS == 0) {
-                constexpr int span = GS / SW_CPL;            // lanes covering one group
-                const bool in_group = sub >= jo && sub < jo + span;
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    float mn = 0.f, mx = 0.f;
-                    if (in_group) {
-#pragma unroll
-                        for (int q = 0; q < SW_CPL; ++q) { mn = fminf(mn, w[r][q]); mx = fmaxf(mx, w[r][q]); }
-                    }
-#pragma unroll
-                    for (int o = 1; o < SW_LPR; o <<= 1) {
-                        mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
-                        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-                    }
-                    gq[r] = group_params(mn, mx, maxqf);
-                    if (valid[r] && sub == jo) {
-                        const int64_t gi = (j0 + j) / GS;
-                        scales[row[r] * G + gi] = gq[r].h;
-                        zeros[row[r] * G + gi] = (uint8_t)gq[r].z;
-                    }
-                }
-            }
-            // next column's values before this column's correction (off the chain)
-            float xpre[2] = {0.f, 0.f};
-            float unext = 0.f;
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                if (ji + 1 < SW_CPL) xpre[r] = __shfl_sync(FULL, w[r][ji + 1], src_base | jo);
-                else if (jo + 1 < SW_LPR) xpre[r] = __shfl_sync(FULL, w[r][0], src_base | (jo + 1));
-            }
-            if (j + 1 < SW_B) {
-                const int f = (j + 1) >> 2;
-                unext = Us[j * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 + ((j + 1) & 3)];
-            }
-            const float rdj = rdiag[j];
-            float Ej[2];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const float x = xn[r];
-                const float c = quant_code_fast(x, gq[r], maxqf);
-                const float q = gq[r].s * (c - gq[r].z);
-                Ej[r] = (x - q) * rdj;
-                loss[r] = fmaf(Ej[r], Ej[r], loss[r]);
-                if (sub == jo) {
-                    Ev[r][ji] = Ej[r];
-                    cp[r][ji / 4] |= uint32_t(c) << (8 * (ji % 4));
-                }
-                xn[r] = fmaf(-Ej[r], unext, xpre[r]);
-            }
-            const float4* urow = reinterpret_cast<const float4*>(Us + j * SW_B);
-#pragma unroll
-            for (int q4 = 0; q4 < SW_Q4; ++q4) {
-                const float4 u = urow[q4 * SW_LPR + sub];
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    w[r][4 * q4 + 0] = fmaf(-Ej[r], u.x, w[r][4 * q4 + 0]);
-                    w[r][4 * q4 + 1] = fmaf(-Ej[r], u.y, w[r][4 * q4 + 1]);
-                    w[r][4 * q4 + 2] = fmaf(-Ej[r], u.z, w[r][4 * q4 + 2]);
-                    w[r][4 * q4 + 3] = fmaf(-Ej[r], u.w, w[r][4 * q4 + 3]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < SW_RPL; ++r) {
         if (!valid[r]) continue;
-        static_assert(SW_CPL == 16, "codes of a lane are stored as one uint4");
-        *reinterpret_cast<uint4*>(codes + row[r] * d + j0 + SW_CPL * sub) =
-            make_uint4(cp[r][0], cp[r][1], cp[r][2], cp[r][3]);
+        static_assert(SW_CPL % 16 == 0, "codes of a lane are stored as whole uint4");
+#pragma unroll
+        for (int u = 0; u < SW_CPL / 16; ++u)
+            *reinterpret_cast<uint4*>(codes + row[r] * d + j0 + SW_CPL * sub + 16 * u) =
+                make_uint4(cp[r][4 * u], cp[r][4 * u + 1], cp[r][4 * u + 2], cp[r][4 * u + 3]);
         // E split into its TF32 head and fp32 remainder for the tensor-core update
         float4* hdst = reinterpret_cast<float4*>(Eh_out + row[r] * ldE + SW_CPL * sub);
         float4* ldst = reinterpret_cast<float4*>(El_out + row[r] * ldE + SW_CPL * sub);
@@ -243,6 +274,209 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
         }
         if (row_loss && sub == 0)
             row_loss[row[r]] = first_block ? loss[r] : row_loss[row[r]] + loss[r];
+    }
+}
+
+// One 512-column outer block of the sweep, fused: a CTA keeps its 32 rows of
+// the outer block in shared memory, sweeps its 128-column blocks in turn
+// (sweep_core), and after each block applies that block's errors to its own
+// rows' later columns of the outer block on the CUDA cores (fp32 FMA):
+// Ws[:, later] -= E_b U[b rows, later cols].  Rows are independent given U,
+// so this needs no other CTA; it replaces a sweep launch per block and a
+// near-update launch per block but the last.  The errors also leave (as the
+// TF32 head and fp32 remainder) for the tensor-core update of the columns
+// beyond the outer block.
+//   shared memory: Ws  32 rows x (512 + 4) fp32  (the CTA's rows of the outer block)
+//                  Ub  128 x 128 fp32            (diagonal U block, chunk-major, for a
+//                                                 sweep; or an off-diagonal U tile,
+//                                                 row-major, for an update)
+//                  rdiag 128, Es 128 x 32 fp32   (the block's errors, column-major,
+//                                                 row index XOR-swizzled by 4 (j / 16))
+constexpr int OS_WLD = UPD_OUTER * SW_B + 4;
+constexpr size_t OS_SMEM = sizeof(float) * (size_t(SW_ROWS) * OS_WLD + SW_B * SW_B + SW_B +
+                                             SW_B * SW_ROWS);
+static_assert(SW_ROWS == 32 && SW_THREADS == 128, "update tiling: 8 row quads x 16 column quads");
+
+__device__ __forceinline__ int es_index(int k, int lr)
+{
+    return k * SW_ROWS + (lr ^ (((k >> 4) & 7) << 2));
+}
+
+// Diagonal block of U at (j0, j0) into Us (chunk-major rows, strictly-lower
+// part zeroed) and 1 / U_jj into rdiag.
+__device__ __forceinline__ void load_diag_block(const float* __restrict__ U, int64_t d, int64_t j0,
+                                                float* __restrict__ Us, float* __restrict__ rdiag,
+                                                int tid)
+{
+    constexpr int UPT = SW_B * SW_B / 4 / SW_THREADS / 2;   // float4 per thread per half
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+        float4 uv[UPT];
+#pragma unroll
+        for (int i = 0; i < UPT; ++i) {
+            const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
+            uv[i] = *reinterpret_cast<const float4*>(U + (j0 + idx / SW_B) * d + j0 + idx % SW_B);
+        }
+#pragma unroll
+        for (int i = 0; i < UPT; ++i) {
+            const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
+            const int a = idx / SW_B, b = idx % SW_B;
+            float4 v = uv[i];
+            if (b + 0 < a) v.x = 0.f;
+            if (b + 1 < a) v.y = 0.f;
+            if (b + 2 < a) v.z = 0.f;
+            if (b + 3 < a) v.w = 0.f;
+            const int f = b / 4;
+            *reinterpret_cast<float4*>(Us + a * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4) = v;
+        }
+    }
+    if (tid < SW_B) rdiag[tid] = 1.0f / U[(j0 + tid) * d + j0 + tid];
+}
+
+template <int GS, bool STATIC>
+__global__ void __launch_bounds__(SW_THREADS)
+outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
+                   int64_t gsz, int64_t ob0, int nblk, float maxqf, uint8_t* __restrict__ codes,
+                   __half* __restrict__ scales, uint8_t* __restrict__ zeros,
+                   float* __restrict__ Eh_out, float* __restrict__ El_out, int64_t ldE,
+                   float* __restrict__ row_loss, int first_outer)
+{
+    extern __shared__ __align__(16) float smem[];
+    float* Ws = smem;
+    float* Ub = Ws + SW_ROWS * OS_WLD;
+    float* rdiag = Ub + SW_B * SW_B;
+    float* Es = rdiag + SW_B;
+    const int tid = threadIdx.x;
+    const int64_t r0 = int64_t(blockIdx.x) * SW_ROWS;
+    const int ncol4 = nblk * SW_B / 4;
+    for (int i = tid; i < SW_ROWS * ncol4; i += SW_THREADS) {
+        const int rr = i / ncol4, c4 = i - rr * ncol4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r0 + rr < m) v = *reinterpret_cast<const float4*>(Wk + (r0 + rr) * d + ob0 + 4 * c4);
+        *reinterpret_cast<float4*>(Ws + rr * OS_WLD + 4 * c4) = v;
+    }
+    const int lane = tid & 31, sub = lane & (SW_LPR - 1);
+    const int src_base = lane & ~(SW_LPR - 1);
+    const int lbase = (tid >> 5) * (32 / SW_LPR * SW_RPL) + lane / SW_LPR;
+    int lr[SW_RPL];
+    int64_t row[SW_RPL];
+    bool valid[SW_RPL];
+#pragma unroll
+    for (int r = 0; r < SW_RPL; ++r) {
+        lr[r] = lbase + (32 / SW_LPR) * r;
+        row[r] = r0 + lr[r];
+        valid[r] = row[r] < m;
+    }
+    const int64_t G = d / gsz;
+    float tot[SW_RPL];
+#pragma unroll
+    for (int r = 0; r < SW_RPL; ++r) tot[r] = 0.f;
+    // update tiling: 4 rows (rq) x 8 columns {4 cq .. +3, 64 + 4 cq .. +3} per thread
+    const int rq = tid >> 4, cq = tid & 15;
+
+#pragma unroll 1
+    for (int b = 0; b < nblk; ++b) {
+        const int64_t j0 = ob0 + int64_t(b) * SW_B;
+        __syncthreads();                   // Ws rows current, Ub and Es free
+        load_diag_block(U, d, j0, Ub, rdiag, tid);
+        __syncthreads();
+        float w[SW_RPL][SW_CPL];
+#pragma unroll
+        for (int r = 0; r < SW_RPL; ++r) {
+            const float4* p = reinterpret_cast<const float4*>(Ws + lr[r] * OS_WLD + b * SW_B +
+                                                              SW_CPL * sub);
+#pragma unroll
+            for (int q = 0; q < SW_Q4; ++q) {
+                const float4 v = p[q];
+                w[r][4 * q] = v.x; w[r][4 * q + 1] = v.y; w[r][4 * q + 2] = v.z; w[r][4 * q + 3] = v.w;
+            }
+        }
+        float Ev[SW_RPL][SW_CPL];
+        uint32_t cp[SW_RPL][SW_Q4];
+        float loss[SW_RPL];
+        sweep_core<GS, STATIC>(Ub, rdiag, w, row, valid, sub, src_base, G, gsz, j0, maxqf, scales,
+                               zeros, Ev, cp, loss);
+#pragma unroll
+        for (int r = 0; r < SW_RPL; ++r) {
+#pragma unroll
+            for (int i = 0; i < SW_CPL; ++i) Es[es_index(SW_CPL * sub + i, lr[r])] = Ev[r][i];
+            tot[r] += loss[r];
+            if (!valid[r]) continue;
+#pragma unroll
+            for (int u = 0; u < SW_CPL / 16; ++u)
+                *reinterpret_cast<uint4*>(codes + row[r] * d + j0 + SW_CPL * sub + 16 * u) =
+                    make_uint4(cp[r][4 * u], cp[r][4 * u + 1], cp[r][4 * u + 2], cp[r][4 * u + 3]);
+            float4* hdst = reinterpret_cast<float4*>(Eh_out + row[r] * ldE + b * SW_B + SW_CPL * sub);
+            float4* ldst = reinterpret_cast<float4*>(El_out + row[r] * ldE + b * SW_B + SW_CPL * sub);
+#pragma unroll
+            for (int q = 0; q < SW_Q4; ++q) {
+                float4 h, l;
+                h.x = tf32_round(Ev[r][4 * q + 0]); l.x = Ev[r][4 * q + 0] - h.x;
+                h.y = tf32_round(Ev[r][4 * q + 1]); l.y = Ev[r][4 * q + 1] - h.y;
+                h.z = tf32_round(Ev[r][4 * q + 2]); l.z = Ev[r][4 * q + 2] - h.z;
+                h.w = tf32_round(Ev[r][4 * q + 3]); l.w = Ev[r][4 * q + 3] - h.w;
+                hdst[q] = h;
+                ldst[q] = l;
+            }
+        }
+        // the block's errors onto the later columns of the outer block
+#pragma unroll 1
+        for (int b2 = b + 1; b2 < nblk; ++b2) {
+            __syncthreads();               // Es complete; Ub no longer read
+            const int64_t c0 = ob0 + int64_t(b2) * SW_B;
+            {
+                constexpr int UPT = SW_B * SW_B / 4 / SW_THREADS / 2;
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    float4 uv[UPT];
+#pragma unroll
+                    for (int i = 0; i < UPT; ++i) {
+                        const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
+                        uv[i] = *reinterpret_cast<const float4*>(U + (j0 + idx / SW_B) * d + c0 +
+                                                                 idx % SW_B);
+                    }
+#pragma unroll
+                    for (int i = 0; i < UPT; ++i) {
+                        const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
+                        *reinterpret_cast<float4*>(Ub + idx) = uv[i];
+                    }
+                }
+            }
+            __syncthreads();
+            // the block's correction sum E_b U[b, cols] first, then one
+            // subtraction from W (the order of the tensor-core update)
+            float acc[4][8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+#pragma unroll 4
+            for (int k = 0; k < SW_B; ++k) {
+                const float4 e = *reinterpret_cast<const float4*>(Es + es_index(k, 4 * rq));
+                const float4 u0 = *reinterpret_cast<const float4*>(Ub + k * SW_B + 4 * cq);
+                const float4 u1 = *reinterpret_cast<const float4*>(Ub + k * SW_B + 64 + 4 * cq);
+                const float ev[4] = {e.x, e.y, e.z, e.w};
+                const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(ev[i], uv[c], acc[i][c]);
+            }
+            float* wrow = Ws + (4 * rq) * OS_WLD + b2 * SW_B;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float4* p0 = reinterpret_cast<float4*>(wrow + i * OS_WLD + 4 * cq);
+                float4* p1 = reinterpret_cast<float4*>(wrow + i * OS_WLD + 64 + 4 * cq);
+                const float4 a0 = *p0, a1 = *p1;
+                *p0 = make_float4(a0.x - acc[i][0], a0.y - acc[i][1], a0.z - acc[i][2], a0.w - acc[i][3]);
+                *p1 = make_float4(a1.x - acc[i][4], a1.y - acc[i][5], a1.z - acc[i][6], a1.w - acc[i][7]);
+            }
+        }
+    }
+    if (row_loss && sub == 0) {
+#pragma unroll
+        for (int r = 0; r < SW_RPL; ++r)
+            if (valid[r]) row_loss[row[r]] = first_outer ? tot[r] : row_loss[row[r]] + tot[r];
     }
 }
 
@@ -396,6 +630,20 @@ static void launch_sweep(dim3 grid, size_t smem, cudaStream_t st, const float* W
     count_launches();
 }
 
+template <int GS, bool STATIC>
+static void launch_outer(dim3 grid, cudaStream_t st, const float* Wk, const float* U, int64_t m,
+                         int64_t d, int64_t gsz, int64_t ob0, int nblk, float maxqf,
+                         uint8_t* codes, __half* scales, uint8_t* zeros, float* Eh, float* El,
+                         int64_t ldE, float* row_loss, int first)
+{
+    cudaFuncSetAttribute(outer_sweep_kernel<GS, STATIC>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OS_SMEM);
+    KernelTimer kt(kKSweep, st);
+    outer_sweep_kernel<GS, STATIC><<<grid, SW_THREADS, OS_SMEM, st>>>(
+        Wk, U, m, d, gsz, ob0, nblk, maxqf, codes, scales, zeros, Eh, El, ldE, row_loss, first);
+    count_launches();
+}
+
 }  // namespace gptq
 
 extern "C" size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, int block_size)
@@ -491,6 +739,48 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
     // beyond an outer block get the outer block's four blocks at once
     // (K = 512) when it completes.  Every column still receives every earlier
     // column's correction before its own block is swept.
+    // Fused outer blocks: one launch sweeps an outer block's 128-column blocks
+    // and applies each block's errors to the rest of the outer block; the
+    // columns beyond it get the outer block's errors at once (K = 512) on the
+    // tensor cores.  Dynamic groups wider than a block whose starts fall
+    // inside an outer block (256) take the per-block launches below.
+    const int64_t outer = int64_t(UPD_OUTER) * SW_B;
+    if (!wide || gsz % outer == 0) {
+        for (int64_t ob0 = 0; ob0 < d; ob0 += outer) {
+            const int64_t ob1 = std::min<int64_t>(d, ob0 + outer);
+            const int nb = (int)((ob1 - ob0) / SW_B);
+            if (wide && ob0 % gsz == 0) {        // a wide dynamic group starts here
+                KernelTimer kt(kKStaticParams, st);
+                static_params_kernel<<<(unsigned)ceil_div(m * 32, 256), 256, 0, st>>>(
+                    w.Wk, m, d, gsz, ob0 / gsz, 1, maxqf, sc, zeros);
+                count_launches();
+            }
+#define GPTQ_OUTER(GSV, STAT)                                                                   \
+            launch_outer<GSV, STAT>(grid, st, w.Wk, U, m, d, gsz, ob0, nb, maxqf, codes, sc,     \
+                                    zeros, w.upd.Eh, w.upd.El, UPD_LDE, row_loss, ob0 == 0)
+            if (stat) {
+                switch (gsz) {
+                    case 32: GPTQ_OUTER(32, true); break;
+                    case 64: GPTQ_OUTER(64, true); break;
+                    default: GPTQ_OUTER(128, true); break;
+                }
+            } else {
+                switch (gsz) {
+                    case 32: GPTQ_OUTER(32, false); break;
+                    case 64: GPTQ_OUTER(64, false); break;
+                    default: GPTQ_OUTER(128, false); break;
+                }
+            }
+#undef GPTQ_OUTER
+            if (ob1 < d) {
+                KernelTimer kt(kKUpdateFar, st);
+                rc = block_update(w.Wk, &w.upd, m, d, /*e_col0=*/0, /*k_rows=*/ob1 - ob0,
+                                  /*u_row0=*/ob0, /*c_begin=*/ob1, /*c_end=*/d, st);
+                if (rc != GPTQ_OK) return rc;
+            }
+        }
+        return launch_status();
+    }
     const int64_t nblk = d / SW_B;
     for (int64_t b = 0; b < nblk; ++b) {
         const int64_t j0 = b * SW_B;

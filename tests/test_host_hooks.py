@@ -83,3 +83,40 @@ def test_division_free_quotient_is_ieee():
                            f"x={x[bad][0]!r} s={s2[bad][0]!r}")
     # and the decision built on it: rne of the quotient
     assert np.array_equal(np.rint(got), np.rint(want))
+
+
+def test_magic_number_rounding_matches_rint_under_the_clamp():
+    """The sweep's rounding on the FMA pipe: fl(fl(x + 1.5 * 2^23) - 1.5 * 2^23)
+    is round-to-nearest-even for |x| <= 2^22 and, past that, gives the same
+    clamped code as rint (codes in [0, maxq], maxq <= 255).  Float32 numpy
+    arithmetic is IEEE round-to-nearest, as the kernel's __fadd_rn/__fsub_rn."""
+    rng = np.random.default_rng(11)
+    M = np.float32(12582912.0)
+    parts = [np.arange(-600, 601, dtype=np.float32) * np.float32(0.5),      # every half-integer tie
+             rng.uniform(-300, 300, 200000).astype(np.float32),
+             rng.uniform(-2.0 ** 24, 2.0 ** 24, 200000).astype(np.float32)]
+    for e in (22, 23, 24, 30):                                               # around the limits
+        b = np.float32(2.0 ** e)
+        near = (np.array([b, -b], np.float32).view(np.int32)[:, None] +
+                np.arange(-64, 65, dtype=np.int32)[None, :]).ravel().view(np.float32)
+        parts.append(near)
+    parts.append(np.array([3.4e38, -3.4e38, 1e-40, -1e-40, 0.0, -0.0], np.float32))
+    x = np.concatenate(parts).astype(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        trick = ((x + M).astype(np.float32) - M).astype(np.float32)
+    exact = np.rint(x)
+    small = np.abs(x) <= np.float32(2.0 ** 22)
+    assert np.array_equal(trick[small], exact[small])
+    for maxq in (3, 15, 255):
+        for z in sorted({0, 1, maxq // 2, maxq}):
+            zf, mq = np.float32(z), np.float32(maxq)
+            a = np.minimum(np.maximum((trick + zf).astype(np.float32), 0), mq)
+            b = np.minimum(np.maximum((exact + zf).astype(np.float32), 0), mq)
+            assert np.array_equal(a, b), (maxq, z)
+
+
+def test_code_byte_from_float_bits():
+    """An integral c in [0, 255] as a byte: the low 8 bits of fl(c + 2^23)."""
+    c = np.arange(256, dtype=np.float32)
+    got = (c + np.float32(8388608.0)).astype(np.float32).view(np.uint32) & 0xFF
+    assert np.array_equal(got, np.arange(256, dtype=np.uint32))

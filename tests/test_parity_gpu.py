@@ -159,7 +159,7 @@ def test_pack_bits_of_gptq_results_at_3_and_8_bits():
         assert nbytes == m * d * bits // 8 + m * ((G_ * bits + 7) // 8) + 2 * m * G_
 
 
-@pytest.mark.parametrize("n,d", [(512, 256), (777, 384), (64, 128), (4099, 1024)])
+@pytest.mark.parametrize("n,d", [(512, 256), (777, 384), (64, 128), (4099, 1024), (60001, 1152)])
 def test_hessian_parity(n, d):
     X = _gauss_x(n, d, 3, 50.0, d + n)
     S = torch.zeros(d, d, dtype=torch.float32, device=DEV)
