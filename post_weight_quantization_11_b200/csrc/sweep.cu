@@ -280,20 +280,26 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
 // One 512-column outer block of the sweep, fused: a CTA keeps its 32 rows of
 // the outer block in shared memory, sweeps its 128-column blocks in turn
 // (sweep_core), and after each block applies that block's errors to its own
-// rows' later columns of the outer block on the CUDA cores (fp32 FMA):
-// Ws[:, later] -= E_b U[b rows, later cols].  Rows are independent given U,
-// so this needs no other CTA; it replaces a sweep launch per block and a
+// rows' later columns of the outer block on the CUDA cores (fp32 FMA; the
+// correction sum E_b U[b rows, cols] first, then one subtraction from W,
+// the order of the tensor-core update).  Rows are independent given U, so
+// this needs no other CTA; it replaces a sweep launch per block and a
 // near-update launch per block but the last.  The errors also leave (as the
 // TF32 head and fp32 remainder) for the tensor-core update of the columns
 // beyond the outer block.
-//   shared memory: Ws  32 rows x (512 + 4) fp32  (the CTA's rows of the outer block)
-//                  Ub  128 x 128 fp32            (diagonal U block, chunk-major, for a
-//                                                 sweep; or an off-diagonal U tile,
-//                                                 row-major, for an update)
-//                  rdiag 128, Es 128 x 32 fp32   (the block's errors, column-major,
-//                                                 row index XOR-swizzled by 4 (j / 16))
+// The outer block's U tiles -- per block b its diagonal tile, then the tiles
+// (b, b2 > b) -- stream through two shared buffers with 16-byte async
+// copies, each tile's copy issued while the previous tile is in use.  A
+// diagonal tile is stored chunk-major (sweep_core's layout) and its strictly
+// lower part is left as U holds it: sweep_core's corrections to columns
+// already decided are never read.
+//   shared memory: Ws   32 rows x (512 + 4) fp32   (the CTA's rows of the outer block)
+//                  U    2 x (128 x 128 + 128) fp32 (a tile; 1/U_jj after a diagonal one)
+//                  Es   128 x 32 fp32              (the block's errors, column-major,
+//                                                   row index XOR-swizzled by 4 (j / 16))
 constexpr int OS_WLD = UPD_OUTER * SW_B + 4;
-constexpr size_t OS_SMEM = sizeof(float) * (size_t(SW_ROWS) * OS_WLD + SW_B * SW_B + SW_B +
+constexpr int OS_UBUF = SW_B * SW_B + SW_B;
+constexpr size_t OS_SMEM = sizeof(float) * (size_t(SW_ROWS) * OS_WLD + 2 * OS_UBUF +
                                              SW_B * SW_ROWS);
 static_assert(SW_ROWS == 32 && SW_THREADS == 128, "update tiling: 8 row quads x 16 column quads");
 
@@ -302,35 +308,44 @@ __device__ __forceinline__ int es_index(int k, int lr)
     return k * SW_ROWS + (lr ^ (((k >> 4) & 7) << 2));
 }
 
-// Diagonal block of U at (j0, j0) into Us (chunk-major rows, strictly-lower
-// part zeroed) and 1 / U_jj into rdiag.
-__device__ __forceinline__ void load_diag_block(const float* __restrict__ U, int64_t d, int64_t j0,
-                                                float* __restrict__ Us, float* __restrict__ rdiag,
-                                                int tid)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src)
 {
-    constexpr int UPT = SW_B * SW_B / 4 / SW_THREADS / 2;   // float4 per thread per half
-#pragma unroll
-    for (int hb = 0; hb < 2; ++hb) {
-        float4 uv[UPT];
-#pragma unroll
-        for (int i = 0; i < UPT; ++i) {
-            const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
-            uv[i] = *reinterpret_cast<const float4*>(U + (j0 + idx / SW_B) * d + j0 + idx % SW_B);
-        }
-#pragma unroll
-        for (int i = 0; i < UPT; ++i) {
-            const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
-            const int a = idx / SW_B, b = idx % SW_B;
-            float4 v = uv[i];
-            if (b + 0 < a) v.x = 0.f;
-            if (b + 1 < a) v.y = 0.f;
-            if (b + 2 < a) v.z = 0.f;
-            if (b + 3 < a) v.w = 0.f;
-            const int f = b / 4;
-            *reinterpret_cast<float4*>(Us + a * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4) = v;
-        }
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// every committed group but the newest has landed (this thread's copies)
+__device__ __forceinline__ void cp_async_wait_all_but_newest()
+{
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+// Tile t of an outer block of nblk blocks: (b, b2), b2 == b for a diagonal tile.
+__device__ __forceinline__ void os_tile(int t, int nblk, int& b, int& b2)
+{
+    b = 0;
+    while (t >= nblk - b) { t -= nblk - b; ++b; }
+    b2 = b + t;
+}
+
+// Every thread: issue its copies of tile t into buf, and commit them as one group.
+__device__ __forceinline__ void os_issue(const float* __restrict__ U, int64_t d, int64_t ob0,
+                                         int nblk, int t, float* buf, int tid)
+{
+    int b, b2;
+    os_tile(t, nblk, b, b2);
+    const int64_t r0 = ob0 + int64_t(b) * SW_B, c0 = ob0 + int64_t(b2) * SW_B;
+#pragma unroll 4
+    for (int i = 0; i < SW_B * SW_B / 4 / SW_THREADS; ++i) {
+        const int idx = (tid + i * SW_THREADS) * 4;
+        const int a = idx / SW_B, c = idx % SW_B, f = c / 4;
+        const int pos = (b2 == b) ? a * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 : idx;
+        cp_async16(buf + pos, U + (r0 + a) * d + c0 + c);
     }
-    if (tid < SW_B) rdiag[tid] = 1.0f / U[(j0 + tid) * d + j0 + tid];
+    cp_async_commit();
 }
 
 template <int GS, bool STATIC>
@@ -343,18 +358,23 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
 {
     extern __shared__ __align__(16) float smem[];
     float* Ws = smem;
-    float* Ub = Ws + SW_ROWS * OS_WLD;
-    float* rdiag = Ub + SW_B * SW_B;
-    float* Es = rdiag + SW_B;
+    float* Ubuf[2] = {Ws + SW_ROWS * OS_WLD, Ws + SW_ROWS * OS_WLD + OS_UBUF};
+    float* Es = Ubuf[1] + OS_UBUF;
     const int tid = threadIdx.x;
     const int64_t r0 = int64_t(blockIdx.x) * SW_ROWS;
     const int ncol4 = nblk * SW_B / 4;
     for (int i = tid; i < SW_ROWS * ncol4; i += SW_THREADS) {
         const int rr = i / ncol4, c4 = i - rr * ncol4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r0 + rr < m) v = *reinterpret_cast<const float4*>(Wk + (r0 + rr) * d + ob0 + 4 * c4);
-        *reinterpret_cast<float4*>(Ws + rr * OS_WLD + 4 * c4) = v;
+        float* dst = Ws + rr * OS_WLD + 4 * c4;
+        if (r0 + rr < m)
+            cp_async16(dst, Wk + (r0 + rr) * d + ob0 + 4 * c4);
+        else
+            *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    cp_async_commit();
+    const int ntiles = nblk + nblk * (nblk - 1) / 2;
+    os_issue(U, d, ob0, nblk, 0, Ubuf[0], tid);
+
     const int lane = tid & 31, sub = lane & (SW_LPR - 1);
     const int src_base = lane & ~(SW_LPR - 1);
     const int lbase = (tid >> 5) * (32 / SW_LPR * SW_RPL) + lane / SW_LPR;
@@ -374,11 +394,21 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     // update tiling: 4 rows (rq) x 8 columns {4 cq .. +3, 64 + 4 cq .. +3} per thread
     const int rq = tid >> 4, cq = tid & 15;
 
+    int t = 0;                              // the tile in use
 #pragma unroll 1
-    for (int b = 0; b < nblk; ++b) {
+    for (int b = 0; b < nblk; ++b, ++t) {
         const int64_t j0 = ob0 + int64_t(b) * SW_B;
-        __syncthreads();                   // Ws rows current, Ub and Es free
-        load_diag_block(U, d, j0, Ub, rdiag, tid);
+        __syncthreads();                    // nobody reads the other buffer any more
+        if (t + 1 < ntiles) os_issue(U, d, ob0, nblk, t + 1, Ubuf[(t + 1) & 1], tid);
+        else cp_async_commit();
+        cp_async_wait_all_but_newest();
+        __syncthreads();                    // tile t (and the W rows) landed for every thread
+        float* Us = Ubuf[t & 1];
+        float* rdiag = Us + SW_B * SW_B;
+        if (tid < SW_B) {
+            const int f = tid / 4;
+            rdiag[tid] = 1.0f / Us[tid * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 + tid % 4];
+        }
         __syncthreads();
         float w[SW_RPL][SW_CPL];
 #pragma unroll
@@ -394,7 +424,7 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
         float Ev[SW_RPL][SW_CPL];
         uint32_t cp[SW_RPL][SW_Q4];
         float loss[SW_RPL];
-        sweep_core<GS, STATIC>(Ub, rdiag, w, row, valid, sub, src_base, G, gsz, j0, maxqf, scales,
+        sweep_core<GS, STATIC>(Us, rdiag, w, row, valid, sub, src_base, G, gsz, j0, maxqf, scales,
                                zeros, Ev, cp, loss);
 #pragma unroll
         for (int r = 0; r < SW_RPL; ++r) {
@@ -422,45 +452,34 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
         // the block's errors onto the later columns of the outer block
 #pragma unroll 1
         for (int b2 = b + 1; b2 < nblk; ++b2) {
-            __syncthreads();               // Es complete; Ub no longer read
-            const int64_t c0 = ob0 + int64_t(b2) * SW_B;
-            {
-                constexpr int UPT = SW_B * SW_B / 4 / SW_THREADS / 2;
-#pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    float4 uv[UPT];
-#pragma unroll
-                    for (int i = 0; i < UPT; ++i) {
-                        const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
-                        uv[i] = *reinterpret_cast<const float4*>(U + (j0 + idx / SW_B) * d + c0 +
-                                                                 idx % SW_B);
-                    }
-#pragma unroll
-                    for (int i = 0; i < UPT; ++i) {
-                        const int idx = (tid + (hb * UPT + i) * SW_THREADS) * 4;
-                        *reinterpret_cast<float4*>(Ub + idx) = uv[i];
-                    }
-                }
-            }
-            __syncthreads();
-            // the block's correction sum E_b U[b, cols] first, then one
-            // subtraction from W (the order of the tensor-core update)
+            ++t;
+            __syncthreads();                // Es complete; the other buffer is free
+            if (t + 1 < ntiles) os_issue(U, d, ob0, nblk, t + 1, Ubuf[(t + 1) & 1], tid);
+            else cp_async_commit();
+            cp_async_wait_all_but_newest();
+            __syncthreads();                // tile t landed for every thread
+            const float* Ub = Ubuf[t & 1];
             float acc[4][8];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
-#pragma unroll 4
+            float4 e = *reinterpret_cast<const float4*>(Es + es_index(0, 4 * rq));
+            float4 u0 = *reinterpret_cast<const float4*>(Ub + 4 * cq);
+            float4 u1 = *reinterpret_cast<const float4*>(Ub + 64 + 4 * cq);
+#pragma unroll 2
             for (int k = 0; k < SW_B; ++k) {
-                const float4 e = *reinterpret_cast<const float4*>(Es + es_index(k, 4 * rq));
-                const float4 u0 = *reinterpret_cast<const float4*>(Ub + k * SW_B + 4 * cq);
-                const float4 u1 = *reinterpret_cast<const float4*>(Ub + k * SW_B + 64 + 4 * cq);
+                const int kn = (k + 1) & (SW_B - 1);       // the next operands, loaded early
+                const float4 en = *reinterpret_cast<const float4*>(Es + es_index(kn, 4 * rq));
+                const float4 u0n = *reinterpret_cast<const float4*>(Ub + kn * SW_B + 4 * cq);
+                const float4 u1n = *reinterpret_cast<const float4*>(Ub + kn * SW_B + 64 + 4 * cq);
                 const float ev[4] = {e.x, e.y, e.z, e.w};
                 const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
                     for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(ev[i], uv[c], acc[i][c]);
+                e = en; u0 = u0n; u1 = u1n;
             }
             float* wrow = Ws + (4 * rq) * OS_WLD + b2 * SW_B;
 #pragma unroll
