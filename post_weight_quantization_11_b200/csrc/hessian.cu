@@ -28,8 +28,6 @@
 //    memory: the MMA-issuing thread zeroes its rows beyond the end before
 //    the MMAs read it (the rows there belong to the next segment).
 //  * Every mbarrier wait is bounded (see tc_common.cuh).
-#include <atomic>
-
 #include "common.cuh"
 #include "tc_common.cuh"
 
@@ -77,17 +75,6 @@ __device__ __forceinline__ void tile_coords(int t, int& bi, int& bj)
     while (b > 0 && b * (b + 1) > t) --b;
     bj = b;
     bi = t - b * (b + 1);
-}
-
-// Upper-triangle tiles of a square block grid, column-block-major: column
-// block bj holds row blocks bi = 0 .. bj.
-__device__ __forceinline__ void tri_upper_coords(int t, int& bi, int& bj)
-{
-    int b = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
-    while ((b + 1) * (b + 2) / 2 <= t) ++b;
-    while (b > 0 && b * (b + 1) / 2 > t) --b;
-    bj = b;
-    bi = t - b * (b + 1) / 2;
 }
 
 __device__ __forceinline__ HbItem hb_item(const SyrkParams& p, int q)
@@ -266,277 +253,9 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, const SyrkParams p)
     }
 }
 
-// ---- CTA-pair kernel (one row segment) -----------------------------------
-// Output tiles of 256 x 256 computed by a pair of CTAs (a cluster of 2) with
-// tcgen05.mma.cta_group::2, M = N = 256, K = 16: CTA r loads its 128 rows
-// of A (features i0 + 128 r ..) and its 128 columns of B (features
-// j0 + 128 r ..) for every 64-token stage, 32 KB, and receives rows
-// i0 + 128 r .. of the tile over all 256 columns in its TMEM.  Against the
-// single-CTA 128 x 256 tile this is a third less operand traffic per flop
-// (32 KB instead of 48 KB per 64 tokens per SM), which buys six stages in
-// flight instead of four for the same shared memory.
-//   * Both CTAs' copies of a stage complete on the even CTA's full barrier;
-//     only the even CTA arms it (arrive + expect_tx of both CTAs' bytes).
-//   * The even CTA's MMA thread releases a stage, and hands an accumulator
-//     to the epilogues, with commits that arrive in both CTAs.
-//   * The epilogue warps of both CTAs hand an accumulator back on the even
-//     CTA's barrier (8 arrivals per CTA).
-//   * Token splits end at multiples of 64 tokens except at the end of X,
-//     where the tensor map's bounds zero the rows past the end: no box is
-//     cut in shared memory.
-constexpr int H2_STAGES = 6;
-constexpr int H2_HALF_BYTES = 128 * HB_K * 2;               // 16 KB: 128 features x 64 tokens
-constexpr int H2_STAGE_BYTES = 2 * H2_HALF_BYTES;           // A rows + B columns of this CTA
-constexpr int H2_SMEM = H2_STAGES * H2_STAGE_BYTES + 1024 + 256;
-constexpr uint32_t H2_IDESC = make_idesc(0 /*f16*/, 256, 256, 1 /*A MN-major*/, 1 /*B MN*/);
-constexpr int H2_EPI_WARPS = HB_EPI_THREADS / 32;
-
-struct Syrk2Params {
-    float* S;
-    int64_t d;
-    int nb;           // 256-wide blocks
-    int tiles;        // upper-triangle tiles of 256 x 256
-    int items;        // tiles x token splits
-    int64_t n;        // rows of X
-    int64_t per;      // tokens per split (multiple of 64)
-};
-
-__global__ void __launch_bounds__(HB_THREADS, 1)
-hessian_pair_kernel(const __grid_constant__ CUtensorMap tmX, const Syrk2Params p)
-{
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + H2_STAGES * H2_STAGE_BYTES);
-    uint64_t* empty_bar = full_bar + H2_STAGES;
-    uint64_t* accf_bar = empty_bar + H2_STAGES;
-    uint64_t* acce_bar = accf_bar + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + 2);
-    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
-    const int pair = (int)cluster_id_x(), npairs = (int)nclusters_x();
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < H2_STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(&accf_bar[a], 1); mbar_init(&acce_bar[a], 2 * H2_EPI_WARPS); }
-        *abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == 1) tmem_alloc_pair(tmem_slot, HB_TMEM_COLS);
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();               // the peer's barriers exist before any signal reaches them
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            prefetch_tmap(&tmX);
-            const uint32_t full0 = mapa_shared(smem_u32(full_bar), 0);   // the even CTA's
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t armed = 0, armed_par = 0;
-            bool ok = true;
-            for (int q = pair; q < p.items && ok; q += npairs) {
-                const int s = q / p.tiles, t = q - s * p.tiles;
-                int bi, bj;
-                tri_upper_coords(t, bi, bj);
-                const int64_t t0 = int64_t(s) * p.per, t1 = min(p.n, t0 + p.per);
-                const int ra = bi * 256 + (int)rank * 128, rb = bj * 256 + (int)rank * 128;
-                for (int64_t k = t0; k < t1; k += HB_K) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, kErrWaitEmpty, abort)) { ok = false; break; }
-                    uint8_t* sa = smem + stage * H2_STAGE_BYTES;
-                    uint8_t* sb = sa + H2_HALF_BYTES;
-                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * H2_STAGE_BYTES);
-                    const uint32_t fb = full0 + uint32_t(stage) * 8u;
-                    tma_load_2d_pair(sa, &tmX, fb, ra, (int)k);
-                    tma_load_2d_pair(sa + 8192, &tmX, fb, ra + 64, (int)k);
-                    tma_load_2d_pair(sb, &tmX, fb, rb, (int)k);
-                    tma_load_2d_pair(sb + 8192, &tmX, fb, rb + 64, (int)k);
-                    armed |= 1u << stage;
-                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                    if (++stage == H2_STAGES) { stage = 0; phase ^= 1; }
-                }
-            }
-            // every stage this CTA filled has been consumed (so its copies
-            // landed and no release is still on its way) before the exit
-            for (int s = 0; s < H2_STAGES; ++s)
-                if (armed & (1u << s)) mbar_drain(&empty_bar[s], (armed_par >> s) & 1u);
-        }
-    } else if (warp == 1) {
-        if (lane == 0 && rank == 0) {
-            int stage = 0, ch = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int q = pair; q < p.items && ok; q += npairs) {
-                const int s = q / p.tiles;
-                const int64_t t0 = int64_t(s) * p.per, t1 = min(p.n, t0 + p.per);
-                for (int64_t c0 = t0; c0 < t1 && ok; c0 += HB_CHUNK, ++ch) {
-                    const int64_t c1 = min(t1, c0 + HB_CHUNK);
-                    const int a = ch & 1;
-                    const uint32_t aph = (ch >> 1) & 1;
-                    if (!mbar_wait_cluster(&acce_bar[a], aph ^ 1, kErrWaitAccEmpty, abort)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t d_tmem = tmem + uint32_t(a * HB_N);
-                    uint32_t acc = 0;
-                    for (int64_t k = c0; k < c1; k += HB_K) {
-                        if (!mbar_wait(&full_bar[stage], phase, kErrWaitFull, abort)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t sa = smem_u32(smem + stage * H2_STAGE_BYTES);
-                        const uint32_t sb = sa + H2_HALF_BYTES;
-#pragma unroll
-                        for (int kk = 0; kk < HB_K / 16; ++kk) {
-                            const uint64_t da = smem_desc_sw128(sa + kk * 2048, 8192, 1024);
-                            const uint64_t db = smem_desc_sw128(sb + kk * 2048, 8192, 1024);
-                            mma_f16_pair(d_tmem, da, db, H2_IDESC, acc);
-                            acc = 1;
-                        }
-                        mma_commit_pair(&empty_bar[stage], 0x3);
-                        if (++stage == H2_STAGES) { stage = 0; phase ^= 1; }
-                    }
-                    mma_commit_pair(&accf_bar[a], 0x3);
-                }
-            }
-        }
-    } else {
-        const int ew = warp - 2;                 // 0..7
-        const int qr = warp & 3;                 // TMEM lane quarter of this warp
-        const int half = ew >> 2;                // columns [128*half, 128*half + 128)
-        const uint32_t acce0 = mapa_shared(smem_u32(acce_bar), 0);   // the even CTA's
-        int ch = 0;
-        bool ok = true;
-        for (int q = pair; q < p.items && ok; q += npairs) {
-            const int s = q / p.tiles, t = q - s * p.tiles;
-            int bi, bj;
-            tri_upper_coords(t, bi, bj);
-            const int64_t t0 = int64_t(s) * p.per, t1 = min(p.n, t0 + p.per);
-            float sum[128];
-#pragma unroll
-            for (int u = 0; u < 128; ++u) sum[u] = 0.f;
-            for (int64_t c0 = t0; c0 < t1; c0 += HB_CHUNK, ++ch) {
-                const int a = ch & 1;
-                const uint32_t aph = (ch >> 1) & 1;
-                if (!mbar_wait(&accf_bar[a], aph, kErrWaitAccFull, abort)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t base = tmem + uint32_t(a * HB_N + half * 128) + (uint32_t(qr * 32) << 16);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float v[32];
-                    tmem_ld32(base + uint32_t(c * 32), v);
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) sum[c * 32 + u] = __fadd_rn(sum[c * 32 + u], v[u]);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acce0 + uint32_t(a) * 8u);
-            }
-            if (!ok) break;
-            const int64_t i = int64_t(bi) * 256 + rank * 128 + qr * 32 + lane;
-            if (i >= p.d) continue;
-            float* Srow = p.S + i * p.d;
-            const int64_t jb = int64_t(bj) * 256 + half * 128;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int64_t j0 = jb + c * 32;
-                if (j0 >= p.d || j0 + 31 < i) continue;
-#pragma unroll
-                for (int u = 0; u < 32; u += 4) {
-                    const int64_t j = j0 + u;
-                    const float* v = sum + c * 32 + u;
-                    if (j >= i) {
-                        atomicAdd(reinterpret_cast<float4*>(Srow + j),
-                                  make_float4(v[0], v[1], v[2], v[3]));
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if (j + e >= i) atomicAdd(Srow + j + e, v[e]);
-                    }
-                }
-            }
-        }
-    }
-    __syncthreads();
-    cluster_sync_all();               // no signal of either CTA is still on its way to the other
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc_pair(tmem, HB_TMEM_COLS);
-    }
-}
-
 }  // namespace gptq
 
 namespace gptq {
-
-// Clusters of two pair-kernel CTAs that can be resident at once on the
-// current device (cached per device).
-static int pair_clusters_resident(cudaLaunchConfig_t cfg)
-{
-    static std::atomic<int> cache[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64) {
-        const int c = cache[dev].load();
-        if (c > 0) return c;
-    }
-    int ncl = 0;
-    if (cudaOccupancyMaxActiveClusters(&ncl, hessian_pair_kernel, &cfg) != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64 && ncl > 0) cache[dev].store(ncl);
-    return ncl;
-}
-
-// S += X^T X over all n rows of X with the CTA-pair kernel.
-static int hessian_pair_launch(float* S, const uint16_t* X, int64_t n, int64_t d, cudaStream_t st)
-{
-    Syrk2Params p{};
-    p.S = S;
-    p.d = d;
-    p.n = n;
-    p.nb = (int)ceil_div(d, 256);
-    p.tiles = p.nb * (p.nb + 1) / 2;
-    if (cudaFuncSetAttribute(hessian_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             H2_SMEM) != cudaSuccess)
-        return GPTQ_ERR_CUDA;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(HB_THREADS);
-    cfg.dynamicSmemBytes = H2_SMEM;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cfg.gridDim = dim3(2);
-    const int npairs = std::min(persistent_ctas(kCtaHessian) / 2, pair_clusters_resident(cfg));
-    if (npairs < 1) return GPTQ_ERR_CUDA;
-    // token splits by a round model: rounds of npairs items, each as long as
-    // its tokens plus the flush of its tile into S (about 300 tokens' worth)
-    const int64_t ksteps = ceil_div(n, HB_K);
-    int64_t best_s = 1;
-    double best_cost = 1e300;
-    for (int64_t sp = 1; sp <= std::min<int64_t>(ksteps, 256); ++sp) {
-        const int64_t per = ceil_div(ksteps, sp) * HB_K;
-        const int64_t items = int64_t(p.tiles) * ceil_div(n, per);
-        const double cost = double(ceil_div(items, int64_t(npairs))) * double(per + 300);
-        if (cost < best_cost - 1e-9) { best_cost = cost; best_s = sp; }
-    }
-    p.per = ceil_div(ksteps, best_s) * HB_K;
-    const int64_t items = int64_t(p.tiles) * ceil_div(n, p.per);
-    if (items > (int64_t(1) << 30)) return GPTQ_ERR_SHAPE;
-    p.items = (int)items;
-    cfg.gridDim = dim3(2 * (unsigned)std::min<int64_t>(npairs, items));
-
-    CUtensorMap tm;
-    if (encode_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, (uint64_t)d, (uint64_t)n,
-                       (uint64_t)d * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK)
-        return GPTQ_ERR_CUDA;
-    KernelTimer kt(kKHessian, st);
-    if (cudaLaunchKernelEx(&cfg, hessian_pair_kernel, tm, p) != cudaSuccess) return GPTQ_ERR_CUDA;
-    count_launches();
-    return launch_status();
-}
 
 // Launch the accumulation of nseg (<= HB_MAX_SEG) segments [row0[e], row1[e])
 // of the rows of X (n_rows x d) into S + e d^2.  Empty segments get no items.
@@ -621,7 +340,8 @@ extern "C" int gptq_hessian_accumulate(float* S, const uint16_t* X, int64_t n_to
     if (d < 128 || d > kMaxDim || d % 128 != 0 || n_tokens < 0 || n_tokens > (int64_t(1) << 31))
         return GPTQ_ERR_SHAPE;
     if (n_tokens == 0) return GPTQ_OK;
-    const int rc = hessian_pair_launch(S, X, n_tokens, d, as_stream(stream));
+    const int64_t r0 = 0, r1 = n_tokens;
+    const int rc = hessian_launch(S, X, n_tokens, d, 1, &r0, &r1, as_stream(stream));
     if (rc == GPTQ_OK && n_seen) *n_seen += n_tokens;
     return rc;
 }

@@ -331,19 +331,24 @@ __device__ __forceinline__ void os_tile(int t, int nblk, int& b, int& b2)
     b2 = b + t;
 }
 
-// Every thread: issue its copies of tile t into buf, and commit them as one group.
+// Every thread: issue its copies of tile t into buf, and commit them as one
+// group.  Thread tid copies the 16-byte chunk (tid % 32) of rows tid / 32,
+// tid / 32 + 4, ... of the tile.
 __device__ __forceinline__ void os_issue(const float* __restrict__ U, int64_t d, int64_t ob0,
                                          int nblk, int t, float* buf, int tid)
 {
     int b, b2;
     os_tile(t, nblk, b, b2);
-    const int64_t r0 = ob0 + int64_t(b) * SW_B, c0 = ob0 + int64_t(b2) * SW_B;
-#pragma unroll 4
-    for (int i = 0; i < SW_B * SW_B / 4 / SW_THREADS; ++i) {
-        const int idx = (tid + i * SW_THREADS) * 4;
-        const int a = idx / SW_B, c = idx % SW_B, f = c / 4;
-        const int pos = (b2 == b) ? a * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 : idx;
-        cp_async16(buf + pos, U + (r0 + a) * d + c0 + c);
+    const int f = tid & 31;                                  // float4 column of the row
+    const int a0 = tid >> 5;
+    const float* src = U + (ob0 + int64_t(b) * SW_B + a0) * d + ob0 + int64_t(b2) * SW_B + 4 * f;
+    float* dst = buf + a0 * SW_B + (b2 == b ? ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 : 4 * f);
+    constexpr int ROWS_PER_PASS = SW_THREADS / 32;
+#pragma unroll 8
+    for (int i = 0; i < SW_B / ROWS_PER_PASS; ++i) {
+        cp_async16(dst, src);
+        src += ROWS_PER_PASS * d;
+        dst += ROWS_PER_PASS * SW_B;
     }
     cp_async_commit();
 }
@@ -358,8 +363,8 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
 {
     extern __shared__ __align__(16) float smem[];
     float* Ws = smem;
-    float* Ubuf[2] = {Ws + SW_ROWS * OS_WLD, Ws + SW_ROWS * OS_WLD + OS_UBUF};
-    float* Es = Ubuf[1] + OS_UBUF;
+    float* const Ub0 = Ws + SW_ROWS * OS_WLD;          // U buffer i at Ub0 + i * OS_UBUF
+    float* Es = Ub0 + 2 * OS_UBUF;
     const int tid = threadIdx.x;
     const int64_t r0 = int64_t(blockIdx.x) * SW_ROWS;
     const int ncol4 = nblk * SW_B / 4;
@@ -373,7 +378,7 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     }
     cp_async_commit();
     const int ntiles = nblk + nblk * (nblk - 1) / 2;
-    os_issue(U, d, ob0, nblk, 0, Ubuf[0], tid);
+    os_issue(U, d, ob0, nblk, 0, Ub0, tid);
 
     const int lane = tid & 31, sub = lane & (SW_LPR - 1);
     const int src_base = lane & ~(SW_LPR - 1);
@@ -399,11 +404,11 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     for (int b = 0; b < nblk; ++b, ++t) {
         const int64_t j0 = ob0 + int64_t(b) * SW_B;
         __syncthreads();                    // nobody reads the other buffer any more
-        if (t + 1 < ntiles) os_issue(U, d, ob0, nblk, t + 1, Ubuf[(t + 1) & 1], tid);
+        if (t + 1 < ntiles) os_issue(U, d, ob0, nblk, t + 1, Ub0 + ((t + 1) & 1) * OS_UBUF, tid);
         else cp_async_commit();
         cp_async_wait_all_but_newest();
         __syncthreads();                    // tile t (and the W rows) landed for every thread
-        float* Us = Ubuf[t & 1];
+        float* Us = Ub0 + (t & 1) * OS_UBUF;
         float* rdiag = Us + SW_B * SW_B;
         if (tid < SW_B) {
             const int f = tid / 4;
@@ -454,32 +459,27 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
         for (int b2 = b + 1; b2 < nblk; ++b2) {
             ++t;
             __syncthreads();                // Es complete; the other buffer is free
-            if (t + 1 < ntiles) os_issue(U, d, ob0, nblk, t + 1, Ubuf[(t + 1) & 1], tid);
+            if (t + 1 < ntiles) os_issue(U, d, ob0, nblk, t + 1, Ub0 + ((t + 1) & 1) * OS_UBUF, tid);
             else cp_async_commit();
             cp_async_wait_all_but_newest();
             __syncthreads();                // tile t landed for every thread
-            const float* Ub = Ubuf[t & 1];
+            const float* Ub = Ub0 + (t & 1) * OS_UBUF;
             float acc[4][8];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
-            float4 e = *reinterpret_cast<const float4*>(Es + es_index(0, 4 * rq));
-            float4 u0 = *reinterpret_cast<const float4*>(Ub + 4 * cq);
-            float4 u1 = *reinterpret_cast<const float4*>(Ub + 64 + 4 * cq);
-#pragma unroll 2
+#pragma unroll 4
             for (int k = 0; k < SW_B; ++k) {
-                const int kn = (k + 1) & (SW_B - 1);       // the next operands, loaded early
-                const float4 en = *reinterpret_cast<const float4*>(Es + es_index(kn, 4 * rq));
-                const float4 u0n = *reinterpret_cast<const float4*>(Ub + kn * SW_B + 4 * cq);
-                const float4 u1n = *reinterpret_cast<const float4*>(Ub + kn * SW_B + 64 + 4 * cq);
+                const float4 e = *reinterpret_cast<const float4*>(Es + es_index(k, 4 * rq));
+                const float4 u0 = *reinterpret_cast<const float4*>(Ub + k * SW_B + 4 * cq);
+                const float4 u1 = *reinterpret_cast<const float4*>(Ub + k * SW_B + 64 + 4 * cq);
                 const float ev[4] = {e.x, e.y, e.z, e.w};
                 const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
                     for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(ev[i], uv[c], acc[i][c]);
-                e = en; u0 = u0n; u1 = u1n;
             }
             float* wrow = Ws + (4 * rq) * OS_WLD + b2 * SW_B;
 #pragma unroll

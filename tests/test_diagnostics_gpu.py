@@ -27,10 +27,21 @@ def test_kernel_timing_covers_every_launch_kind_and_changes_nothing():
         G.gptq_debug_kernel_timing(False)
     t = G.gptq_debug_kernel_times()
     for kind in ("hessian", "finalize", "factorization", "init_work", "split_u", "sweep",
-                 "update_near", "update_far", "pack"):
+                 "update_far", "pack"):
         assert kind in t and t[kind][0] > 0.0 and t[kind][1] > 0, (kind, t)
-    assert t["sweep"][1] == 1024 // 128
+    # one fused sweep launch per 512-column outer block, no separate near updates
+    assert t["sweep"][1] == 1024 // 512 and "update_near" not in t, t
     assert G.gptq_debug_kernel_times() == {}          # records are consumed
+    # dynamic groups of 256 start inside an outer block: a sweep launch per
+    # 128-column block and a near update after every block but an outer block's last
+    G.gptq_debug_kernel_timing(True)
+    try:
+        G.gptq_quantize_layer(W, res.U, None, 4, 256)
+        torch.cuda.synchronize()
+    finally:
+        G.gptq_debug_kernel_timing(False)
+    t2 = G.gptq_debug_kernel_times()
+    assert t2["sweep"][1] == 1024 // 128 and t2["update_near"][1] == 6, t2
     # S's fp32 atomic adds run in no fixed order when the tokens are split,
     # so the two runs agree to rounding, not bit for bit
     a, b = ref.S.double(), res.S.double()
