@@ -278,34 +278,111 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
 }
 
 // One 512-column outer block of the sweep, fused: a CTA keeps its 32 rows of
-// the outer block in shared memory, sweeps its 128-column blocks in turn
-// (sweep_core), and after each block applies that block's errors to its own
-// rows' later columns of the outer block on the CUDA cores (fp32 FMA; the
-// correction sum E_b U[b rows, cols] first, then one subtraction from W,
-// the order of the tensor-core update).  Rows are independent given U, so
-// this needs no other CTA; it replaces a sweep launch per block and a
+// the outer block in shared memory and sweeps its 128-column blocks in turn
+// (sweep_core); each block's errors are applied to the CTA's rows' later
+// columns of the outer block (for every block pair the correction sum
+// E_b U[b rows, cols] first, then one subtraction from W).  Rows are independent given
+// U, so this needs no other CTA; it replaces a sweep launch per block and a
 // near-update launch per block but the last.  The errors also leave (as the
 // TF32 head and fp32 remainder) for the tensor-core update of the columns
 // beyond the outer block.
-// The outer block's U tiles -- per block b its diagonal tile, then the tiles
-// (b, b2 > b) -- stream through two shared buffers with 16-byte async
-// copies, each tile's copy issued while the previous tile is in use.  A
-// diagonal tile is stored chunk-major (sweep_core's layout) and its strictly
-// lower part is left as U holds it: sweep_core's corrections to columns
-// already decided are never read.
+// Warp roles (8 warps): warps 0-3 sweep; warps 4-7 apply block b-1's errors
+// to blocks b+1.. while block b is swept (phase A), then every warp applies
+// block b's errors to block b+1, the next block to sweep (phase B).  A
+// column receives the corrections of the earlier blocks in block order.
+// U tiles come with 16-byte async copies: the diagonal tile of the next
+// block during phase B, the off-diagonal tiles as 64-row halves through two
+// buffers (the next half copied while one is in use; phase B's tile is
+// copied at the end of phase A).  A diagonal tile is stored chunk-major
+// (sweep_core's layout) and its strictly lower part is left as U holds it:
+// sweep_core's corrections to columns already decided are never read.
+// The updates are m16n8k8 tensor-core products (mma.sync) in split TF32:
+// three products per pair of operands, fp32 accumulation, as the unfused
+// tensor-core update.
 //   shared memory: Ws   32 rows x (512 + 4) fp32   (the CTA's rows of the outer block)
-//                  U    2 x (128 x 128 + 128) fp32 (a tile; 1/U_jj after a diagonal one)
-//                  Es   128 x 32 fp32              (the block's errors, column-major,
-//                                                   row index XOR-swizzled by 4 (j / 16))
+//                  D    128 x 128 + 128 fp32       (diagonal tile, then 1/U_jj)
+//                  H    2 x 64 x (128 + 4) fp32    (halves of off-diagonal tiles)
+//                  Es   32 x (128 + 4) fp32        (a block's errors, row-major)
+constexpr int OS_THREADS = 2 * SW_THREADS;
 constexpr int OS_WLD = UPD_OUTER * SW_B + 4;
-constexpr int OS_UBUF = SW_B * SW_B + SW_B;
-constexpr size_t OS_SMEM = sizeof(float) * (size_t(SW_ROWS) * OS_WLD + 2 * OS_UBUF +
-                                             SW_B * SW_ROWS);
-static_assert(SW_ROWS == 32 && SW_THREADS == 128, "update tiling: 8 row quads x 16 column quads");
+constexpr int OS_DBUF = SW_B * SW_B + SW_B;
+constexpr int OS_HLD = SW_B + 4;                     // row stride of a half tile and of Es
+constexpr int OS_HALF = (SW_B / 2) * OS_HLD;
+constexpr size_t OS_SMEM = sizeof(float) * (size_t(SW_ROWS) * OS_WLD + OS_DBUF + 2 * OS_HALF +
+                                             SW_ROWS * OS_HLD);
+static_assert(SW_ROWS == 32 && SW_THREADS == 128, "update tilings below assume 32 rows");
 
-__device__ __forceinline__ int es_index(int k, int lr)
+// D (16x8, fp32) += A (16x8) B (8x8) on the tensor cores, TF32 inputs (mma.sync).
+__device__ __forceinline__ void mma_tf32_m16n8k8(float (&c)[4], const uint32_t (&a)[4],
+                                                 uint32_t b0, uint32_t b1)
 {
-    return k * SW_ROWS + (lr ^ (((k >> 4) & 7) << 2));
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// x = head + tail: head its TF32 truncation, tail the exact fp32 remainder
+// (whose own TF32 part the tensor core reads); the three products
+// head*head + head*tail + tail*head leave out tail*tail, about 2^-20 of x y.
+__device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo)
+{
+    hi = __float_as_uint(x) & 0xffffe000u;
+    lo = __float_as_uint(x - __uint_as_float(hi));
+}
+
+// acc (this warp's 32 rows x 8 NT columns, as 2 x NT m16n8 tiles) +=
+// E[rows, k0 .. k0 + 64) . Hb[0 .. 64, c0w .. c0w + 8 NT) in split TF32:
+// E row-major in Es (row stride OS_HLD), the half tile row-major in Hb.
+template <int NT>
+__device__ __forceinline__ void os_mma_half(float (&acc)[2][NT][4], const float* Es,
+                                            const float* Hb, int k0, int c0w, int lane)
+{
+    const int g = lane >> 2, tg = lane & 3;
+#pragma unroll 2
+    for (int kk = 0; kk < SW_B / 2; kk += 8) {
+        uint32_t ah[2][4], al[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            const float* er = Es + (16 * mt + g) * OS_HLD + k0 + kk + tg;
+            const float av[4] = {er[0], er[8 * OS_HLD], er[4], er[8 * OS_HLD + 4]};
+#pragma unroll
+            for (int v = 0; v < 4; ++v) tf32_split(av[v], ah[mt][v], al[mt][v]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const float* br = Hb + (kk + tg) * OS_HLD + c0w + 8 * nt + g;
+            uint32_t bh0, bl0, bh1, bl1;
+            tf32_split(br[0], bh0, bl0);
+            tf32_split(br[4 * OS_HLD], bh1, bl1);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                mma_tf32_m16n8k8(acc[mt][nt], ah[mt], bh0, bh1);
+                mma_tf32_m16n8k8(acc[mt][nt], ah[mt], bl0, bl1);
+                mma_tf32_m16n8k8(acc[mt][nt], al[mt], bh0, bh1);
+            }
+        }
+    }
+}
+
+// Ws[rows, b2 block, c0w .. c0w + 8 NT) -= acc
+template <int NT>
+__device__ __forceinline__ void os_mma_subtract(float* Ws, int b2, const float (&acc)[2][NT][4],
+                                                int c0w, int lane)
+{
+    const int g = lane >> 2, tg = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float2* p = reinterpret_cast<float2*>(Ws + (16 * mt + g + 8 * hf) * OS_WLD +
+                                                      b2 * SW_B + c0w + 8 * nt + 2 * tg);
+                const float2 a = *p;
+                *p = make_float2(a.x - acc[mt][nt][2 * hf], a.y - acc[mt][nt][2 * hf + 1]);
+            }
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src)
@@ -317,44 +394,59 @@ __device__ __forceinline__ void cp_async_commit()
 {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
-// every committed group but the newest has landed (this thread's copies)
+// every group this thread committed has landed
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+// every group this thread committed but the newest has landed
 __device__ __forceinline__ void cp_async_wait_all_but_newest()
 {
     asm volatile("cp.async.wait_group 1;" ::: "memory");
 }
-
-// Tile t of an outer block of nblk blocks: (b, b2), b2 == b for a diagonal tile.
-__device__ __forceinline__ void os_tile(int t, int nblk, int& b, int& b2)
+// barrier among the nthreads threads (whole warps) that use this id
+__device__ __forceinline__ void bar_named(int id, int nthreads)
 {
-    b = 0;
-    while (t >= nblk - b) { t -= nblk - b; ++b; }
-    b2 = b + t;
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Every thread: issue its copies of tile t into buf, and commit them as one
-// group.  Thread tid copies the 16-byte chunk (tid % 32) of rows tid / 32,
-// tid / 32 + 4, ... of the tile.
-__device__ __forceinline__ void os_issue(const float* __restrict__ U, int64_t d, int64_t ob0,
-                                         int nblk, int t, float* buf, int tid)
+// Thread t of nthr (a multiple of 32): copies of the diagonal tile at (j0, j0)
+// into D, chunk-major.  Thread t copies the 16-byte chunk (t % 32) of rows
+// t / 32, t / 32 + nthr / 32, ...
+__device__ __forceinline__ void os_copy_diag(const float* __restrict__ U, int64_t d, int64_t j0,
+                                             float* D, int t, int nthr)
 {
-    int b, b2;
-    os_tile(t, nblk, b, b2);
-    const int f = tid & 31;                                  // float4 column of the row
-    const int a0 = tid >> 5;
-    const float* src = U + (ob0 + int64_t(b) * SW_B + a0) * d + ob0 + int64_t(b2) * SW_B + 4 * f;
-    float* dst = buf + a0 * SW_B + (b2 == b ? ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 : 4 * f);
-    constexpr int ROWS_PER_PASS = SW_THREADS / 32;
-#pragma unroll 8
-    for (int i = 0; i < SW_B / ROWS_PER_PASS; ++i) {
+    const int f = t & 31;
+    const int step = nthr >> 5;
+    const float* src = U + (j0 + (t >> 5)) * d + j0 + 4 * f;
+    float* dst = D + (t >> 5) * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4;
+#pragma unroll 4
+    for (int a = t >> 5; a < SW_B; a += step) {
         cp_async16(dst, src);
-        src += ROWS_PER_PASS * d;
-        dst += ROWS_PER_PASS * SW_B;
+        src += step * d;
+        dst += step * SW_B;
     }
-    cp_async_commit();
+}
+
+// Thread t of nthr: copies of rows [k0, k0 + 64) x columns [c0, c0 + 128) of
+// U into H, row-major (row stride OS_HLD).
+__device__ __forceinline__ void os_copy_half(const float* __restrict__ U, int64_t d, int64_t k0,
+                                             int64_t c0, float* H, int t, int nthr)
+{
+    const int f = t & 31;
+    const int step = nthr >> 5;
+    const float* src = U + (k0 + (t >> 5)) * d + c0 + 4 * f;
+    float* dst = H + (t >> 5) * OS_HLD + 4 * f;
+#pragma unroll 4
+    for (int a = t >> 5; a < SW_B / 2; a += step) {
+        cp_async16(dst, src);
+        src += step * d;
+        dst += step * OS_HLD;
+    }
 }
 
 template <int GS, bool STATIC>
-__global__ void __launch_bounds__(SW_THREADS)
+__global__ void __launch_bounds__(OS_THREADS, 1)
 outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, int64_t m, int64_t d,
                    int64_t gsz, int64_t ob0, int nblk, float maxqf, uint8_t* __restrict__ codes,
                    __half* __restrict__ scales, uint8_t* __restrict__ zeros,
@@ -363,26 +455,38 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
 {
     extern __shared__ __align__(16) float smem[];
     float* Ws = smem;
-    float* const Ub0 = Ws + SW_ROWS * OS_WLD;          // U buffer i at Ub0 + i * OS_UBUF
-    float* Es = Ub0 + 2 * OS_UBUF;
+    float* Dt = Ws + SW_ROWS * OS_WLD;
+    float* rdiag = Dt + SW_B * SW_B;
+    float* H0 = Dt + OS_DBUF;                  // half buffer i at H0 + i * OS_HALF
+    float* Es = H0 + 2 * OS_HALF;
     const int tid = threadIdx.x;
+    const bool sweeper = tid < SW_THREADS;
     const int64_t r0 = int64_t(blockIdx.x) * SW_ROWS;
-    const int ncol4 = nblk * SW_B / 4;
-    for (int i = tid; i < SW_ROWS * ncol4; i += SW_THREADS) {
-        const int rr = i / ncol4, c4 = i - rr * ncol4;
-        float* dst = Ws + rr * OS_WLD + 4 * c4;
-        if (r0 + rr < m)
-            cp_async16(dst, Wk + (r0 + rr) * d + ob0 + 4 * c4);
-        else
-            *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    {
+        const int ncol4 = nblk * SW_B / 4;
+        for (int i = tid; i < SW_ROWS * ncol4; i += OS_THREADS) {
+            const int rr = i / ncol4, c4 = i - rr * ncol4;
+            float* dst = Ws + rr * OS_WLD + 4 * c4;
+            if (r0 + rr < m)
+                cp_async16(dst, Wk + (r0 + rr) * d + ob0 + 4 * c4);
+            else
+                *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        os_copy_diag(U, d, ob0, Dt, tid, OS_THREADS);
+        cp_async_commit();
+        cp_async_wait_all();
     }
-    cp_async_commit();
-    const int ntiles = nblk + nblk * (nblk - 1) / 2;
-    os_issue(U, d, ob0, nblk, 0, Ub0, tid);
+    __syncthreads();
+    if (tid < SW_B) {
+        const int f = tid / 4;
+        rdiag[tid] = 1.0f / Dt[tid * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 + tid % 4];
+    }
+    __syncthreads();
 
+    // sweep warps: rows of each lane (sweep_core's mapping)
     const int lane = tid & 31, sub = lane & (SW_LPR - 1);
     const int src_base = lane & ~(SW_LPR - 1);
-    const int lbase = (tid >> 5) * (32 / SW_LPR * SW_RPL) + lane / SW_LPR;
+    const int lbase = ((tid & (SW_THREADS - 1)) >> 5) * (32 / SW_LPR * SW_RPL) + lane / SW_LPR;
     int lr[SW_RPL];
     int64_t row[SW_RPL];
     bool valid[SW_RPL];
@@ -396,103 +500,126 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
     float tot[SW_RPL];
 #pragma unroll
     for (int r = 0; r < SW_RPL; ++r) tot[r] = 0.f;
-    // update tiling: 4 rows (rq) x 8 columns {4 cq .. +3, 64 + 4 cq .. +3} per thread
-    const int rq = tid >> 4, cq = tid & 15;
+    float Ev[SW_RPL][SW_CPL];
 
-    int t = 0;                              // the tile in use
 #pragma unroll 1
-    for (int b = 0; b < nblk; ++b, ++t) {
+    for (int b = 0; b < nblk; ++b) {
         const int64_t j0 = ob0 + int64_t(b) * SW_B;
-        __syncthreads();                    // nobody reads the other buffer any more
-        if (t + 1 < ntiles) os_issue(U, d, ob0, nblk, t + 1, Ub0 + ((t + 1) & 1) * OS_UBUF, tid);
-        else cp_async_commit();
-        cp_async_wait_all_but_newest();
-        __syncthreads();                    // tile t (and the W rows) landed for every thread
-        float* Us = Ub0 + (t & 1) * OS_UBUF;
-        float* rdiag = Us + SW_B * SW_B;
-        if (tid < SW_B) {
-            const int f = tid / 4;
-            rdiag[tid] = 1.0f / Us[tid * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 + tid % 4];
-        }
-        __syncthreads();
-        float w[SW_RPL][SW_CPL];
+        // ---- phase A: sweep block b || block b-1's errors onto blocks b+1 ..
+        if (sweeper) {
+            float w[SW_RPL][SW_CPL];
 #pragma unroll
-        for (int r = 0; r < SW_RPL; ++r) {
-            const float4* p = reinterpret_cast<const float4*>(Ws + lr[r] * OS_WLD + b * SW_B +
-                                                              SW_CPL * sub);
+            for (int r = 0; r < SW_RPL; ++r) {
+                const float4* p = reinterpret_cast<const float4*>(Ws + lr[r] * OS_WLD + b * SW_B +
+                                                                  SW_CPL * sub);
 #pragma unroll
-            for (int q = 0; q < SW_Q4; ++q) {
-                const float4 v = p[q];
-                w[r][4 * q] = v.x; w[r][4 * q + 1] = v.y; w[r][4 * q + 2] = v.z; w[r][4 * q + 3] = v.w;
+                for (int q = 0; q < SW_Q4; ++q) {
+                    const float4 v = p[q];
+                    w[r][4 * q] = v.x; w[r][4 * q + 1] = v.y; w[r][4 * q + 2] = v.z; w[r][4 * q + 3] = v.w;
+                }
             }
-        }
-        float Ev[SW_RPL][SW_CPL];
-        uint32_t cp[SW_RPL][SW_Q4];
-        float loss[SW_RPL];
-        sweep_core<GS, STATIC>(Us, rdiag, w, row, valid, sub, src_base, G, gsz, j0, maxqf, scales,
-                               zeros, Ev, cp, loss);
+            uint32_t cp[SW_RPL][SW_Q4];
+            float loss[SW_RPL];
+            sweep_core<GS, STATIC>(Dt, rdiag, w, row, valid, sub, src_base, G, gsz, j0, maxqf,
+                                   scales, zeros, Ev, cp, loss);
 #pragma unroll
-        for (int r = 0; r < SW_RPL; ++r) {
+            for (int r = 0; r < SW_RPL; ++r) {
+                tot[r] += loss[r];
+                if (!valid[r]) continue;
 #pragma unroll
-            for (int i = 0; i < SW_CPL; ++i) Es[es_index(SW_CPL * sub + i, lr[r])] = Ev[r][i];
-            tot[r] += loss[r];
-            if (!valid[r]) continue;
+                for (int u = 0; u < SW_CPL / 16; ++u)
+                    *reinterpret_cast<uint4*>(codes + row[r] * d + j0 + SW_CPL * sub + 16 * u) =
+                        make_uint4(cp[r][4 * u], cp[r][4 * u + 1], cp[r][4 * u + 2], cp[r][4 * u + 3]);
+                float4* hdst = reinterpret_cast<float4*>(Eh_out + row[r] * ldE + b * SW_B + SW_CPL * sub);
+                float4* ldst = reinterpret_cast<float4*>(El_out + row[r] * ldE + b * SW_B + SW_CPL * sub);
 #pragma unroll
-            for (int u = 0; u < SW_CPL / 16; ++u)
-                *reinterpret_cast<uint4*>(codes + row[r] * d + j0 + SW_CPL * sub + 16 * u) =
-                    make_uint4(cp[r][4 * u], cp[r][4 * u + 1], cp[r][4 * u + 2], cp[r][4 * u + 3]);
-            float4* hdst = reinterpret_cast<float4*>(Eh_out + row[r] * ldE + b * SW_B + SW_CPL * sub);
-            float4* ldst = reinterpret_cast<float4*>(El_out + row[r] * ldE + b * SW_B + SW_CPL * sub);
-#pragma unroll
-            for (int q = 0; q < SW_Q4; ++q) {
-                float4 h, l;
-                h.x = tf32_round(Ev[r][4 * q + 0]); l.x = Ev[r][4 * q + 0] - h.x;
-                h.y = tf32_round(Ev[r][4 * q + 1]); l.y = Ev[r][4 * q + 1] - h.y;
-                h.z = tf32_round(Ev[r][4 * q + 2]); l.z = Ev[r][4 * q + 2] - h.z;
-                h.w = tf32_round(Ev[r][4 * q + 3]); l.w = Ev[r][4 * q + 3] - h.w;
-                hdst[q] = h;
-                ldst[q] = l;
+                for (int q = 0; q < SW_Q4; ++q) {
+                    float4 h, l;
+                    h.x = tf32_round(Ev[r][4 * q + 0]); l.x = Ev[r][4 * q + 0] - h.x;
+                    h.y = tf32_round(Ev[r][4 * q + 1]); l.y = Ev[r][4 * q + 1] - h.y;
+                    h.z = tf32_round(Ev[r][4 * q + 2]); l.z = Ev[r][4 * q + 2] - h.z;
+                    h.w = tf32_round(Ev[r][4 * q + 3]); l.w = Ev[r][4 * q + 3] - h.w;
+                    hdst[q] = h;
+                    ldst[q] = l;
+                }
             }
-        }
-        // the block's errors onto the later columns of the outer block
+        } else {
+            const int ut = tid - SW_THREADS;
+            const int c0w = 32 * (ut >> 5);                     // this warp's 32 columns
+            const int nh = (b >= 1) ? 2 * (nblk - 1 - b) : 0;   // halves of E_{b-1}'s tiles
+            const int64_t kb = j0 - SW_B;                       // U rows of block b-1
+            if (nh > 0) os_copy_half(U, d, kb, j0 + SW_B, H0, ut, SW_THREADS);
+            cp_async_commit();
+            float acc[2][4][4];
 #pragma unroll 1
-        for (int b2 = b + 1; b2 < nblk; ++b2) {
-            ++t;
-            __syncthreads();                // Es complete; the other buffer is free
-            if (t + 1 < ntiles) os_issue(U, d, ob0, nblk, t + 1, Ub0 + ((t + 1) & 1) * OS_UBUF, tid);
-            else cp_async_commit();
-            cp_async_wait_all_but_newest();
-            __syncthreads();                // tile t landed for every thread
-            const float* Ub = Ub0 + (t & 1) * OS_UBUF;
-            float acc[4][8];
+            for (int h = 0; h < nh; ++h) {
+                const int b2 = b + 1 + h / 2, kh = h & 1;
+                if (h + 1 < nh)
+                    os_copy_half(U, d, kb + ((h + 1) & 1) * (SW_B / 2),
+                                 ob0 + int64_t(b + 1 + (h + 1) / 2) * SW_B,
+                                 H0 + ((h + 1) & 1) * OS_HALF, ut, SW_THREADS);
+                cp_async_commit();
+                cp_async_wait_all_but_newest();
+                bar_named(1, SW_THREADS);        // half h landed for every update thread
+                if (kh == 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+                    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
-#pragma unroll 4
-            for (int k = 0; k < SW_B; ++k) {
-                const float4 e = *reinterpret_cast<const float4*>(Es + es_index(k, 4 * rq));
-                const float4 u0 = *reinterpret_cast<const float4*>(Ub + k * SW_B + 4 * cq);
-                const float4 u1 = *reinterpret_cast<const float4*>(Ub + k * SW_B + 64 + 4 * cq);
-                const float ev[4] = {e.x, e.y, e.z, e.w};
-                const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(ev[i], uv[c], acc[i][c]);
+                            for (int v = 0; v < 4; ++v) acc[mt][nt][v] = 0.f;
+                }
+                os_mma_half<4>(acc, Es, H0 + (h & 1) * OS_HALF, kh * (SW_B / 2), c0w, lane);
+                if (kh == 1) os_mma_subtract<4>(Ws, b2, acc, c0w, lane);
+                bar_named(1, SW_THREADS);        // buffer h & 1 free
             }
-            float* wrow = Ws + (4 * rq) * OS_WLD + b2 * SW_B;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float4* p0 = reinterpret_cast<float4*>(wrow + i * OS_WLD + 4 * cq);
-                float4* p1 = reinterpret_cast<float4*>(wrow + i * OS_WLD + 64 + 4 * cq);
-                const float4 a0 = *p0, a1 = *p1;
-                *p0 = make_float4(a0.x - acc[i][0], a0.y - acc[i][1], a0.z - acc[i][2], a0.w - acc[i][3]);
-                *p1 = make_float4(a1.x - acc[i][4], a1.y - acc[i][5], a1.z - acc[i][6], a1.w - acc[i][7]);
+            // phase B's tile (block b's rows, block b+1's columns), copied ahead
+            if (b + 1 < nblk) {
+                os_copy_half(U, d, j0, j0 + SW_B, H0, ut, SW_THREADS);
+                os_copy_half(U, d, j0 + SW_B / 2, j0 + SW_B, H0 + OS_HALF, ut, SW_THREADS);
             }
+            cp_async_commit();
+        }
+        __syncthreads();                         // block b swept; E_{b-1} applied
+        if (b + 1 < nblk) {
+            // ---- phase B: block b's errors onto block b+1, every warp
+            if (sweeper) {
+#pragma unroll
+                for (int r = 0; r < SW_RPL; ++r)
+#pragma unroll
+                    for (int q = 0; q < SW_Q4; ++q)
+                        *reinterpret_cast<float4*>(Es + lr[r] * OS_HLD + SW_CPL * sub + 4 * q) =
+                            make_float4(Ev[r][4 * q], Ev[r][4 * q + 1], Ev[r][4 * q + 2],
+                                        Ev[r][4 * q + 3]);
+                os_copy_diag(U, d, j0 + SW_B, Dt, tid, SW_THREADS);
+                cp_async_commit();
+            } else {
+                cp_async_wait_all();             // phase B's tile
+            }
+            __syncthreads();                     // E_b and the tile visible
+            {
+                const int c0w = 16 * (tid >> 5);                // this warp's 16 columns
+                float acc[2][2][4];
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) acc[mt][nt][v] = 0.f;
+                os_mma_half<2>(acc, Es, H0, 0, c0w, lane);
+                os_mma_half<2>(acc, Es, H0 + OS_HALF, SW_B / 2, c0w, lane);
+                os_mma_subtract<2>(Ws, b + 1, acc, c0w, lane);
+            }
+            if (sweeper) cp_async_wait_all();    // the next diagonal tile
+            __syncthreads();
+            if (tid < SW_B) {
+                const int f = tid / 4;
+                rdiag[tid] = 1.0f / Dt[tid * SW_B + ((f % SW_Q4) * SW_LPR + f / SW_Q4) * 4 + tid % 4];
+            }
+            __syncthreads();
         }
     }
-    if (row_loss && sub == 0) {
+    if (sweeper && row_loss && sub == 0) {
 #pragma unroll
         for (int r = 0; r < SW_RPL; ++r)
             if (valid[r]) row_loss[row[r]] = first_outer ? tot[r] : row_loss[row[r]] + tot[r];
@@ -658,7 +785,7 @@ static void launch_outer(dim3 grid, cudaStream_t st, const float* Wk, const floa
     cudaFuncSetAttribute(outer_sweep_kernel<GS, STATIC>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OS_SMEM);
     KernelTimer kt(kKSweep, st);
-    outer_sweep_kernel<GS, STATIC><<<grid, SW_THREADS, OS_SMEM, st>>>(
+    outer_sweep_kernel<GS, STATIC><<<grid, OS_THREADS, OS_SMEM, st>>>(
         Wk, U, m, d, gsz, ob0, nblk, maxqf, codes, scales, zeros, Eh, El, ldE, row_loss, first);
     count_launches();
 }
