@@ -302,7 +302,7 @@ class MoeLayer:
         self.info = torch.zeros(E, dtype=torch.int32, device=dev)
         self.ws_p = torch.empty(G.gptq_prepare_batched_workspace_bytes(d, E), dtype=torch.uint8,
                                 device=dev)
-        self.ws_q = torch.empty(G.gptq_quantize_workspace_bytes(m, d, 128), dtype=torch.uint8,
+        self.ws_q = torch.empty(E * G.gptq_quantize_workspace_bytes(m, d, 128), dtype=torch.uint8,
                                 device=dev)
         self.codes = torch.empty(E, m, d, dtype=torch.uint8, device=dev)
         self.scales = torch.empty(E, m, d // 128, dtype=torch.float16, device=dev)

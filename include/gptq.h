@@ -306,10 +306,14 @@ int gptq_quantize_layer_static(const void* W, int w_dtype, int64_t d_out, int64_
  *   U: n_mats x d_in x d_in, perm: n_mats x d_in or NULL,
  *   codes: n_mats x d_out x d_in, scales / zeros: n_mats x d_out x G,
  *   row_loss: n_mats x d_out or NULL.
- * Each layer gets exactly the result of gptq_quantize_layer.  The layers
- * run one after the other on the stream and share ONE workspace of
- * gptq_quantize_workspace_bytes(d_out, d_in, block_size) bytes: at these
- * sizes one layer's sweep already fills the GPU (d_out / 32 CTAs per block).
+ * Each layer gets exactly the result of gptq_quantize_layer.  Workspace:
+ * with ws_bytes >= n_mats * gptq_quantize_workspace_bytes(d_out, d_in,
+ * block_size) (layer e's part at e times that size) the layers run
+ * together: each 512-column outer block of every layer is swept in one
+ * launch (their row tiles fill the SMs' waves together), then each layer's
+ * columns beyond it are updated; with a smaller workspace (at least one
+ * layer's) the layers run one after the other and share it.  Dynamic
+ * 256-column groups always take the second schedule.
  * Dynamic groups only (group_size as gptq_quantize_layer).  Every layer's
  * slice must stay 16-byte aligned (GPTQ_ERR_SHAPE otherwise).
  * Pack the stacked codes and zero points with one gptq_pack_int4 call of

@@ -301,15 +301,19 @@ block_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
 // tensor-core update.
 //   shared memory: Ws   32 rows x (512 + 4) fp32   (the CTA's rows of the outer block)
 //                  D    128 x 128 + 128 fp32       (diagonal tile, then 1/U_jj)
-//                  H    2 x 64 x (128 + 4) fp32    (halves of off-diagonal tiles)
+//                  H    2 x 64 x (128 + 8) fp32    (halves of off-diagonal tiles)
 //                  Es   32 x (128 + 4) fp32        (a block's errors, row-major)
 constexpr int OS_THREADS = 2 * SW_THREADS;
 constexpr int OS_WLD = UPD_OUTER * SW_B + 4;
 constexpr int OS_DBUF = SW_B * SW_B + SW_B;
-constexpr int OS_HLD = SW_B + 4;                     // row stride of a half tile and of Es
+// Row strides of a half tile (OS_HLD) and of Es (OS_ELD), so that the 32
+// lanes of an m16n8k8 fragment load hit 32 different banks: lane (g, t) reads
+// Es at 4 g + t and a half tile at 8 t + g (mod 32) past the fragment's base.
+constexpr int OS_HLD = SW_B + 8;
+constexpr int OS_ELD = SW_B + 4;
 constexpr int OS_HALF = (SW_B / 2) * OS_HLD;
 constexpr size_t OS_SMEM = sizeof(float) * (size_t(SW_ROWS) * OS_WLD + OS_DBUF + 2 * OS_HALF +
-                                             SW_ROWS * OS_HLD);
+                                             SW_ROWS * OS_ELD);
 static_assert(SW_ROWS == 32 && SW_THREADS == 128, "update tilings below assume 32 rows");
 
 // D (16x8, fp32) += A (16x8) B (8x8) on the tensor cores, TF32 inputs (mma.sync).
@@ -334,7 +338,8 @@ __device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo)
 
 // acc (this warp's 32 rows x 8 NT columns, as 2 x NT m16n8 tiles) +=
 // E[rows, k0 .. k0 + 64) . Hb[0 .. 64, c0w .. c0w + 8 NT) in split TF32:
-// E row-major in Es (row stride OS_HLD), the half tile row-major in Hb.
+// E row-major in Es (row stride OS_ELD), the half tile row-major in Hb
+// (row stride OS_HLD).
 template <int NT>
 __device__ __forceinline__ void os_mma_half(float (&acc)[2][NT][4], const float* Es,
                                             const float* Hb, int k0, int c0w, int lane)
@@ -345,8 +350,8 @@ __device__ __forceinline__ void os_mma_half(float (&acc)[2][NT][4], const float*
         uint32_t ah[2][4], al[2][4];
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
-            const float* er = Es + (16 * mt + g) * OS_HLD + k0 + kk + tg;
-            const float av[4] = {er[0], er[8 * OS_HLD], er[4], er[8 * OS_HLD + 4]};
+            const float* er = Es + (16 * mt + g) * OS_ELD + k0 + kk + tg;
+            const float av[4] = {er[0], er[8 * OS_ELD], er[4], er[8 * OS_ELD + 4]};
 #pragma unroll
             for (int v = 0; v < 4; ++v) tf32_split(av[v], ah[mt][v], al[mt][v]);
         }
@@ -451,8 +456,22 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
                    int64_t gsz, int64_t ob0, int nblk, float maxqf, uint8_t* __restrict__ codes,
                    __half* __restrict__ scales, uint8_t* __restrict__ zeros,
                    float* __restrict__ Eh_out, float* __restrict__ El_out, int64_t ldE,
-                   float* __restrict__ row_loss, int first_outer)
+                   float* __restrict__ row_loss, int first_outer, int64_t ws_stride,
+                   int64_t u_stride)
 {
+    // matrix blockIdx.y of a batch: working copy and errors ws_stride floats
+    // apart, U u_stride floats apart, the outputs packed one after the other
+    {
+        const int64_t e = blockIdx.y;
+        Wk += e * ws_stride;
+        Eh_out += e * ws_stride;
+        El_out += e * ws_stride;
+        U += e * u_stride;
+        codes += e * m * d;
+        scales += e * m * (d / gsz);
+        zeros += e * m * (d / gsz);
+        if (row_loss) row_loss += e * m;
+    }
     extern __shared__ __align__(16) float smem[];
     float* Ws = smem;
     float* Dt = Ws + SW_ROWS * OS_WLD;
@@ -588,7 +607,7 @@ outer_sweep_kernel(const float* __restrict__ Wk, const float* __restrict__ U, in
                 for (int r = 0; r < SW_RPL; ++r)
 #pragma unroll
                     for (int q = 0; q < SW_Q4; ++q)
-                        *reinterpret_cast<float4*>(Es + lr[r] * OS_HLD + SW_CPL * sub + 4 * q) =
+                        *reinterpret_cast<float4*>(Es + lr[r] * OS_ELD + SW_CPL * sub + 4 * q) =
                             make_float4(Ev[r][4 * q], Ev[r][4 * q + 1], Ev[r][4 * q + 2],
                                         Ev[r][4 * q + 3]);
                 os_copy_diag(U, d, j0 + SW_B, Dt, tid, SW_THREADS);
@@ -780,13 +799,15 @@ template <int GS, bool STATIC>
 static void launch_outer(dim3 grid, cudaStream_t st, const float* Wk, const float* U, int64_t m,
                          int64_t d, int64_t gsz, int64_t ob0, int nblk, float maxqf,
                          uint8_t* codes, __half* scales, uint8_t* zeros, float* Eh, float* El,
-                         int64_t ldE, float* row_loss, int first)
+                         int64_t ldE, float* row_loss, int first, int64_t ws_stride,
+                         int64_t u_stride)
 {
     cudaFuncSetAttribute(outer_sweep_kernel<GS, STATIC>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)OS_SMEM);
     KernelTimer kt(kKSweep, st);
     outer_sweep_kernel<GS, STATIC><<<grid, OS_THREADS, OS_SMEM, st>>>(
-        Wk, U, m, d, gsz, ob0, nblk, maxqf, codes, scales, zeros, Eh, El, ldE, row_loss, first);
+        Wk, U, m, d, gsz, ob0, nblk, maxqf, codes, scales, zeros, Eh, El, ldE, row_loss, first,
+        ws_stride, u_stride);
     count_launches();
 }
 
@@ -824,23 +845,24 @@ static int sweep_group_size(int64_t d, int group_size, bool static_groups, int64
     return GPTQ_ERR_UNSUPPORTED;
 }
 
-static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
-                         const float* U, const int32_t* perm, int bits, int group_size,
-                         int block_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
-                         float* row_loss, void* ws, size_t ws_bytes, void* stream,
-                         bool static_groups)
+// Argument checks of a layer quantization; the group mode on success.
+static int quantize_checks(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
+                           const float* U, const int32_t* perm, int bits, int group_size,
+                           int block_size, const uint8_t* codes, const uint16_t* scales,
+                           const uint8_t* zeros, const float* row_loss, const void* ws,
+                           size_t ws_bytes, bool static_groups, int64_t* gsz, bool* wide,
+                           bool* stat)
 {
     if (!W || !U || !codes || !scales || !zeros || !ws) return GPTQ_ERR_INVALID_ARG;
     int rc = check_quant_args(w_dtype, d_out, d_in, bits);
     if (rc != GPTQ_OK) return rc;
-    int64_t gsz = 0;
-    rc = sweep_group_size(d_in, group_size, static_groups, &gsz);
+    rc = sweep_group_size(d_in, group_size, static_groups, gsz);
     if (rc != GPTQ_OK) return rc;
     // the sweep reads the group parameters instead of reducing them when they
     // are static, one per row, or dynamic but wider than a block (taken just
     // in time at each group's first block by static_params_kernel)
-    const bool wide = !static_groups && gsz > SW_B && gsz < d_in;
-    const bool stat = static_groups || gsz == d_in || wide;
+    *wide = !static_groups && *gsz > SW_B && *gsz < d_in;
+    *stat = static_groups || *gsz == d_in || *wide;
     if (block_size != SW_B) return GPTQ_ERR_UNSUPPORTED;
     if (!aligned16(W) || !aligned16(U) || !aligned16(codes) || !aligned16(scales) ||
         !aligned16(zeros) || !aligned16(ws) || (perm && !aligned16(perm)) ||
@@ -848,10 +870,16 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
         return GPTQ_ERR_INVALID_ARG;
     if (ws_bytes < gptq_quantize_workspace_bytes(d_out, d_in, block_size))
         return GPTQ_ERR_INVALID_ARG;
-    cudaStream_t st = as_stream(stream);
-    QuantWs w;
-    quant_layout(d_out, d_in, reinterpret_cast<char*>(ws), &w);
-    const int64_t m = d_out, d = d_in;
+    return GPTQ_OK;
+}
+
+// Per matrix, before the sweep: the fp32 working copy in sweep order, the
+// group parameters when they are taken from the rows before the sweep, and
+// U's TF32 split for the tensor-core updates.
+static int quantize_prepare(const void* W, int w_dtype, int64_t m, int64_t d, const float* U,
+                            const int32_t* perm, int64_t gsz, bool stat, bool wide, float maxqf,
+                            __half* sc, uint8_t* zeros, QuantWs& w, cudaStream_t st)
+{
     {
         const int64_t total = m * d;
         const unsigned grid = (unsigned)std::min<int64_t>(ceil_div(total, 256), 148 * 16);
@@ -864,8 +892,6 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
                                                           m, d, w.Wk);
         count_launches();
     }
-    const float maxqf = float((1 << bits) - 1);
-    __half* sc = reinterpret_cast<__half*>(scales);
     if (stat && !wide) {
         const int64_t warps = m * (d / gsz);
         KernelTimer kt(kKStaticParams, st);
@@ -873,60 +899,103 @@ static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in
             w.Wk, m, d, gsz, 0, d / gsz, maxqf, sc, zeros);
         count_launches();
     }
-    {
-        KernelTimer kt(kKSplitU, st);
-        rc = update_prepare_u(U, d, &w.upd, st);
-    }
-    if (rc != GPTQ_OK) return rc;
-    const dim3 grid((unsigned)ceil_div(m, SW_ROWS));
-    const size_t smem = sizeof(float) * (SW_B * SW_B + SW_B);
-    // Deferred (two-level) error feedback: after each 128-column block only the
-    // rest of its 512-column outer block is updated (K = 128); the columns
-    // beyond an outer block get the outer block's four blocks at once
-    // (K = 512) when it completes.  Every column still receives every earlier
-    // column's correction before its own block is swept.
-    // Fused outer blocks: one launch sweeps an outer block's 128-column blocks
-    // and applies each block's errors to the rest of the outer block; the
-    // columns beyond it get the outer block's errors at once (K = 512) on the
-    // tensor cores.  Dynamic groups wider than a block whose starts fall
-    // inside an outer block (256) take the per-block launches below.
+    KernelTimer kt(kKSplitU, st);
+    return update_prepare_u(U, d, &w.upd, st);
+}
+
+// Fused outer blocks, for n_mats matrices at once (matrix e's workspace
+// ws_stride bytes after matrix 0's, its U d^2 floats after, its outputs
+// packed): one launch sweeps an outer block's 128-column blocks of every
+// matrix and applies each block's errors to the rest of the outer block; the
+// columns beyond it get the outer block's errors at once (K = 512) on the
+// tensor cores.  Not for dynamic groups whose starts fall inside an outer
+// block (256 columns).
+static int quantize_fused(int64_t n_mats, int64_t m, int64_t d, const float* U, int64_t gsz,
+                          bool stat, bool wide, float maxqf, uint8_t* codes, __half* sc,
+                          uint8_t* zeros, float* row_loss, char* ws0, size_t ws_stride,
+                          cudaStream_t st)
+{
     const int64_t outer = int64_t(UPD_OUTER) * SW_B;
-    if (!wide || gsz % outer == 0) {
-        for (int64_t ob0 = 0; ob0 < d; ob0 += outer) {
-            const int64_t ob1 = std::min<int64_t>(d, ob0 + outer);
-            const int nb = (int)((ob1 - ob0) / SW_B);
-            if (wide && ob0 % gsz == 0) {        // a wide dynamic group starts here
+    const int64_t G = d / gsz;
+    const dim3 grid((unsigned)ceil_div(m, SW_ROWS), (unsigned)n_mats);
+    QuantWs w0;
+    quant_layout(m, d, ws0, &w0);
+    for (int64_t ob0 = 0; ob0 < d; ob0 += outer) {
+        const int64_t ob1 = std::min<int64_t>(d, ob0 + outer);
+        const int nb = (int)((ob1 - ob0) / SW_B);
+        if (wide && ob0 % gsz == 0) {            // a wide dynamic group starts here
+            for (int64_t e = 0; e < n_mats; ++e) {
+                QuantWs w;
+                quant_layout(m, d, ws0 + e * ws_stride, &w);
                 KernelTimer kt(kKStaticParams, st);
                 static_params_kernel<<<(unsigned)ceil_div(m * 32, 256), 256, 0, st>>>(
-                    w.Wk, m, d, gsz, ob0 / gsz, 1, maxqf, sc, zeros);
+                    w.Wk, m, d, gsz, ob0 / gsz, 1, maxqf, sc + e * m * G, zeros + e * m * G);
                 count_launches();
             }
+        }
 #define GPTQ_OUTER(GSV, STAT)                                                                   \
-            launch_outer<GSV, STAT>(grid, st, w.Wk, U, m, d, gsz, ob0, nb, maxqf, codes, sc,     \
-                                    zeros, w.upd.Eh, w.upd.El, UPD_LDE, row_loss, ob0 == 0)
-            if (stat) {
-                switch (gsz) {
-                    case 32: GPTQ_OUTER(32, true); break;
-                    case 64: GPTQ_OUTER(64, true); break;
-                    default: GPTQ_OUTER(128, true); break;
-                }
-            } else {
-                switch (gsz) {
-                    case 32: GPTQ_OUTER(32, false); break;
-                    case 64: GPTQ_OUTER(64, false); break;
-                    default: GPTQ_OUTER(128, false); break;
-                }
+        launch_outer<GSV, STAT>(grid, st, w0.Wk, U, m, d, gsz, ob0, nb, maxqf, codes, sc, zeros, \
+                                w0.upd.Eh, w0.upd.El, UPD_LDE, row_loss, ob0 == 0,               \
+                                int64_t(ws_stride / sizeof(float)), d * d)
+        if (stat) {
+            switch (gsz) {
+                case 32: GPTQ_OUTER(32, true); break;
+                case 64: GPTQ_OUTER(64, true); break;
+                default: GPTQ_OUTER(128, true); break;
             }
+        } else {
+            switch (gsz) {
+                case 32: GPTQ_OUTER(32, false); break;
+                case 64: GPTQ_OUTER(64, false); break;
+                default: GPTQ_OUTER(128, false); break;
+            }
+        }
 #undef GPTQ_OUTER
-            if (ob1 < d) {
+        if (ob1 < d) {
+            for (int64_t e = 0; e < n_mats; ++e) {
+                QuantWs w;
+                quant_layout(m, d, ws0 + e * ws_stride, &w);
                 KernelTimer kt(kKUpdateFar, st);
-                rc = block_update(w.Wk, &w.upd, m, d, /*e_col0=*/0, /*k_rows=*/ob1 - ob0,
-                                  /*u_row0=*/ob0, /*c_begin=*/ob1, /*c_end=*/d, st);
+                const int rc = block_update(w.Wk, &w.upd, m, d, /*e_col0=*/0, /*k_rows=*/ob1 - ob0,
+                                           /*u_row0=*/ob0, /*c_begin=*/ob1, /*c_end=*/d, st);
                 if (rc != GPTQ_OK) return rc;
             }
         }
-        return launch_status();
     }
+    return launch_status();
+}
+
+static int quantize_impl(const void* W, int w_dtype, int64_t d_out, int64_t d_in,
+                         const float* U, const int32_t* perm, int bits, int group_size,
+                         int block_size, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
+                         float* row_loss, void* ws, size_t ws_bytes, void* stream,
+                         bool static_groups)
+{
+    int64_t gsz = 0;
+    bool wide = false, stat = false;
+    int rc = quantize_checks(W, w_dtype, d_out, d_in, U, perm, bits, group_size, block_size, codes,
+                             scales, zeros, row_loss, ws, ws_bytes, static_groups, &gsz, &wide,
+                             &stat);
+    if (rc != GPTQ_OK) return rc;
+    cudaStream_t st = as_stream(stream);
+    QuantWs w;
+    quant_layout(d_out, d_in, reinterpret_cast<char*>(ws), &w);
+    const int64_t m = d_out, d = d_in;
+    const float maxqf = float((1 << bits) - 1);
+    __half* sc = reinterpret_cast<__half*>(scales);
+    rc = quantize_prepare(W, w_dtype, m, d, U, perm, gsz, stat, wide, maxqf, sc, zeros, w, st);
+    if (rc != GPTQ_OK) return rc;
+    const int64_t outer = int64_t(UPD_OUTER) * SW_B;
+    if (!wide || gsz % outer == 0)
+        return quantize_fused(1, m, d, U, gsz, stat, wide, maxqf, codes, sc, zeros, row_loss,
+                              reinterpret_cast<char*>(ws), 0, st);
+    // Dynamic groups of 256 columns: a sweep launch per 128-column block, the
+    // rest of the outer block updated after each (K = 128), the columns
+    // beyond an outer block after its last block (K = 512).  Every column
+    // still receives every earlier column's correction before its own block
+    // is swept.
+    const dim3 grid((unsigned)ceil_div(m, SW_ROWS));
+    const size_t smem = sizeof(float) * (SW_B * SW_B + SW_B);
     const int64_t nblk = d / SW_B;
     for (int64_t b = 0; b < nblk; ++b) {
         const int64_t j0 = b * SW_B;
@@ -1016,8 +1085,35 @@ extern "C" int gptq_quantize_layer_batched(const void* W, int w_dtype, int64_t n
     if ((d_out * d_in * int64_t(wb)) % 16 || (d_out * G * 2) % 16 || (d_out * G) % 16 ||
         (row_loss && (d_out * 4) % 16) || (perm && (d_in * 4) % 16))
         return GPTQ_ERR_SHAPE;
-    // one layer after the other on the stream: each fills the GPU on its own
-    // (d_out / 32 sweep CTAs per block), and they share the one workspace
+    // With a workspace per matrix (n_mats times the single-matrix size), every
+    // outer block is one fused launch over all the matrices (their row tiles
+    // fill the SMs' waves together) followed by each matrix's far update;
+    // otherwise one matrix after the other shares the one workspace.
+    const size_t single = gptq_quantize_workspace_bytes(d_out, d_in, block_size);
+    if (n_mats > 1 && single > 0 && ws && ws_bytes / size_t(n_mats) >= single) {
+        bool wide = false, stat = false;
+        int64_t g2 = 0;
+        rc = quantize_checks(W, w_dtype, d_out, d_in, U, perm, bits, group_size, block_size,
+                             codes, scales, zeros, row_loss, ws, single, false, &g2, &wide, &stat);
+        if (rc != GPTQ_OK) return rc;
+        if (!wide || g2 % (int64_t(UPD_OUTER) * SW_B) == 0) {
+            cudaStream_t st = as_stream(stream);
+            const float maxqf = float((1 << bits) - 1);
+            __half* sc = reinterpret_cast<__half*>(scales);
+            char* ws0 = reinterpret_cast<char*>(ws);
+            for (int64_t e = 0; e < n_mats; ++e) {
+                QuantWs w;
+                quant_layout(d_out, d_in, ws0 + e * single, &w);
+                rc = quantize_prepare(reinterpret_cast<const char*>(W) + e * d_out * d_in * int64_t(wb),
+                                      w_dtype, d_out, d_in, U + e * d_in * d_in,
+                                      perm ? perm + e * d_in : nullptr, g2, stat, wide, maxqf,
+                                      sc + e * d_out * G, zeros + e * d_out * G, w, st);
+                if (rc != GPTQ_OK) return rc;
+            }
+            return quantize_fused(n_mats, d_out, d_in, U, g2, stat, wide, maxqf, codes, sc, zeros,
+                                  row_loss, ws0, single, st);
+        }
+    }
     for (int64_t e = 0; e < n_mats; ++e) {
         rc = quantize_impl(reinterpret_cast<const char*>(W) + e * d_out * d_in * int64_t(wb),
                            w_dtype, d_out, d_in, U + e * d_in * d_in,

@@ -370,10 +370,13 @@ def gptq_prepare_hinv_batched(S: torch.Tensor, n_tokens, damp_rel: float = 0.01,
 
 def gptq_quantize_layer_batched(W: torch.Tensor, U: torch.Tensor, perm=None, bits: int = 4,
                                 group_size: int = 128, block_size: int = 128, codes=None,
-                                scales=None, zeros=None, row_loss=None, ws=None):
+                                scales=None, zeros=None, row_loss=None, ws=None,
+                                shared_workspace: bool = False):
     """gptq_quantize_layer over E stacked layers (W: E x m x d, U: E x d x d,
-    perm: E x d or None) sharing one workspace.  Returns (codes E x m x d,
-    scales E x m x G, zeros E x m x G, row_loss E x m)."""
+    perm: E x d or None).  By default one workspace per layer (the layers are
+    swept together); shared_workspace: one workspace, the layers one after
+    the other.  Returns (codes E x m x d, scales E x m x G, zeros E x m x G,
+    row_loss E x m)."""
     _need(W, "W")
     _need(U, "U", torch.float32)
     E, m, d = W.shape
@@ -383,7 +386,7 @@ def gptq_quantize_layer_batched(W: torch.Tensor, U: torch.Tensor, perm=None, bit
     scales = torch.empty(E, m, G, dtype=torch.float16, device=dev) if scales is None else scales
     zeros = torch.empty(E, m, G, dtype=torch.uint8, device=dev) if zeros is None else zeros
     row_loss = torch.empty(E, m, dtype=torch.float32, device=dev) if row_loss is None else row_loss
-    nb = gptq_quantize_workspace_bytes(m, d, block_size)
+    nb = gptq_quantize_workspace_bytes(m, d, block_size) * (1 if shared_workspace else E)
     ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev) if ws is None else ws
     if perm is not None:
         _need(perm, "perm", torch.int32)

@@ -128,29 +128,35 @@ def test_batched_prepare_reports_each_matrix_pivot():
     assert inf[0] == 0 and inf[1] == 0 and inf[2] != 0
 
 
-@pytest.mark.parametrize("act_order,dtype", [(False, torch.float16), (True, torch.float32)])
-def test_batched_quantize_equals_single_and_oracle(act_order, dtype):
+@pytest.mark.parametrize("act_order,dtype,gs,shared", [
+    (False, torch.float16, 128, False),   # a workspace per layer: the layers swept together
+    (True, torch.float32, 128, False),
+    (False, torch.float16, 64, False),
+    (False, torch.float16, 128, True),    # one shared workspace: one layer after the other
+    (False, torch.float16, 256, False),   # 256-column dynamic groups: per-block launches
+])
+def test_batched_quantize_equals_single_and_oracle(act_order, dtype, gs, shared):
     S, lens = _expert_set(d=512, lens=(2000, 400, 1500), seed=40)
     E, d = S.shape[0], S.shape[1]
     m = 200
     W = torch.stack([_weights(m, d, dtype, 50 + e) for e in range(E)]).to(DEV).contiguous()
     perm, U, info = G.gptq_prepare_hinv_batched(S, lens, 0.01, act_order)
-    codes, scales, zeros, loss = G.gptq_quantize_layer_batched(W, U, perm if act_order else None,
-                                                               4, 128)
+    codes, scales, zeros, loss = G.gptq_quantize_layer_batched(
+        W, U, perm if act_order else None, 4, gs, shared_workspace=shared)
     torch.cuda.synchronize()
     for e in range(E):
         c, s, z, l = G.gptq_quantize_layer(W[e].contiguous(), U[e].contiguous(),
-                                           perm[e].contiguous() if act_order else None, 4, 128)
+                                           perm[e].contiguous() if act_order else None, 4, gs)
         torch.cuda.synchronize()
         assert torch.equal(codes[e], c) and torch.equal(scales[e], s)
         assert torch.equal(zeros[e], z) and torch.equal(loss[e], l)
         # against the oracle's sweep with the same U (the H-forced protocol)
         Wp = np.ascontiguousarray(W[e].double().cpu().numpy()[:, P.to_np(perm[e])])
         U64 = P.to_np(U[e]).astype(np.float64)
-        ref = oracle.quantize_rows(Wp, U64, 4, 128)
+        ref = oracle.quantize_rows(Wp, U64, 4, gs)
         gpu = dict(codes=P.to_np(codes[e]), scales=P.to_np(scales[e]), zeros=P.to_np(zeros[e]))
-        P.compare_sweep(gpu, ref, 128)
-        P.teacher_forced_check(Wp, U64, gpu, 4, 128)
+        P.compare_sweep(gpu, ref, gs)
+        P.teacher_forced_check(Wp, U64, gpu, 4, gs)
     qw, qz = G.gptq_pack_int4(codes.view(E * m, d), zeros.view(E * m, -1))
     rq, rz = oracle.pack_int4(P.to_np(codes).reshape(E * m, d), P.to_np(zeros).reshape(E * m, -1))
     assert np.array_equal(P.to_np(qw).view(np.uint32), rq) and np.array_equal(P.to_np(qz), rz)
