@@ -647,14 +647,15 @@ def run_ours(a):
     torch.cuda.synchronize()
     k1_ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in k1)
 
-    # consecutive layers with each layer's preparation beside the next
-    # layer's Hessian (dense layers; whole-job throughput over the layers)
+    # consecutive layers (exactly K of them, one per step) with every
+    # layer's preparation on a second stream, layer i quantized after layer
+    # i+2's Hessian (dense layers; whole-job throughput over the layers);
+    # with fewer than 3 layers there is nothing to overlap
     pipelined = None
-    if E == 1 and not a.no_pipelined:
+    if E == 1 and not a.no_pipelined and a.steps >= 3:
         _barrier(ws)
         with ClockSampler(local) as clk_p:
-            pms, per_layer = _pipelined_ms(lay, max(a.steps, 10), a.warmup, PIPE_H, PIPE_P,
-                                           not a.eager)
+            pms, per_layer = _pipelined_ms(lay, a.steps, a.warmup, PIPE_H, PIPE_P, not a.eager)
         _barrier(ws)
         pms = _max_over_ranks(pms, ws)
         pipelined = {"value": ws * units / (pms * 1e-3), "ms_per_layer": pms,
@@ -713,9 +714,10 @@ def run_ours(a):
         "phase_ms": phase,
         "phase_note": "per-phase split of one layer from eager launches",
         "launch_mode": (("eager" if a.eager else "cuda_graph") +
-                        f", consecutive layers: layer i's preparation on a second stream beside "
-                        f"layer i+1's Hessian (persistent grids capped at {PIPE_H} and {PIPE_P} "
-                        f"CTAs); every layer runs every phase") if pipelined else
+                        f", consecutive layers: every layer's preparation on a second stream, "
+                        f"layer i quantized after layer i+2's Hessian (persistent grids capped "
+                        f"at {PIPE_H} CTAs for the Hessian and the updates, {PIPE_P} for the "
+                        f"factorization); every layer runs every phase") if pipelined else
                        ("cuda_graph" if not a.eager else "eager"),
         "single_layer": single,
         # one Hessian serves q/k/v (or up/gate) in a model: the rate of the
@@ -943,22 +945,29 @@ def run_ours_one_layer(a):
 
 
 def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int,
-                  graph: bool = True):
+                  graph: bool = True, lag: int = 2):
     """(ms per layer, library launches per layer) of consecutive layers with
-    layer i's preparation on a second stream beside layer i+1's Hessian: the
-    factorization is a latency chain that needs few SMs, the Hessian keeps
-    the rest busy.  S, U, perm and info are double-buffered; every layer
-    still runs every phase.  With `graph`, the schedule of `steps` layers
-    (both streams, joined by events) is captured once as a CUDA graph and
-    replayed; otherwise it is launched eagerly.  The persistent grids are
-    capped at h_ctas / p_ctas CTAs meanwhile (the caps are read at capture)."""
+    each layer's preparation on a second stream: the factorization is a
+    latency chain that needs few SMs, the Hessian and the quantization keep
+    the rest busy.  Layer i is quantized after layer i + lag's Hessian, so
+    its preparation (on p_ctas CTAs, slower than on the whole GPU) has lag
+    Hessians and lag - 1 quantizations to finish in; preparations follow one
+    another on their stream.  S, U, perm and info rotate through lag + 1
+    buffers (layer i's S is overwritten by layer i + lag + 1's Hessian,
+    which runs after layer i's quantization, which waits for its
+    preparation).  Every layer still runs every phase.  With `graph`, the
+    schedule of `steps` layers (both streams, joined by events) is captured
+    once as a CUDA graph and replayed; otherwise it is launched eagerly.  The
+    persistent grids are capped at h_ctas (Hessian, updates) / p_ctas
+    (factorization) CTAs meanwhile (the caps are read at capture)."""
     G = lay.G
     dev = lay.S.device
     n = lay.n
-    S2 = [lay.S, torch.zeros_like(lay.S)]
-    U2 = [lay.U, torch.empty_like(lay.U)]
-    perm2 = [lay.perm, torch.empty_like(lay.perm)]
-    info2 = [lay.info, torch.zeros_like(lay.info)]
+    nb = lag + 1
+    S2 = [lay.S] + [torch.zeros_like(lay.S) for _ in range(lag)]
+    U2 = [lay.U] + [torch.empty_like(lay.U) for _ in range(lag)]
+    perm2 = [lay.perm] + [torch.empty_like(lay.perm) for _ in range(lag)]
+    info2 = [lay.info] + [torch.zeros_like(lay.info) for _ in range(lag)]
     sP = torch.cuda.Stream(device=dev)
 
     def run(layers):
@@ -967,38 +976,41 @@ def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int,
         evP = [torch.cuda.Event() for _ in range(layers)]
 
         def hess(i):
-            S2[i % 2].zero_()
-            G.gptq_hessian_accumulate(S2[i % 2], lay.X)
+            S2[i % nb].zero_()
+            G.gptq_hessian_accumulate(S2[i % nb], lay.X)
             evH[i].record(sH)
 
         def prep(i):
             sP.wait_event(evH[i])
             with torch.cuda.stream(sP):
-                G.gptq_prepare_hinv(S2[i % 2], n, 0.01, lay.act_order, perm2[i % 2], U2[i % 2],
-                                    info2[i % 2], lay.ws_p)
+                G.gptq_prepare_hinv(S2[i % nb], n, 0.01, lay.act_order, perm2[i % nb],
+                                    U2[i % nb], info2[i % nb], lay.ws_p)
             evP[i].record(sP)
 
         def quant(i):
             sH.wait_event(evP[i])
-            G.gptq_quantize_layer(lay.W, U2[i % 2], perm2[i % 2] if lay.act_order else None, 4,
-                                  128, 128, lay.codes, lay.scales, lay.zeros, lay.loss, lay.ws_q)
+            G.gptq_quantize_layer(lay.W, U2[i % nb], perm2[i % nb] if lay.act_order else None,
+                                  4, 128, 128, lay.codes, lay.scales, lay.zeros, lay.loss,
+                                  lay.ws_q)
             G.gptq_pack_int4(lay.codes, lay.zeros, lay.qweight, lay.qzeros)
 
-        hess(0)
-        prep(0)
+        for i in range(min(lag, layers)):
+            hess(i)
+            prep(i)
         for i in range(layers):
-            if i + 1 < layers:
-                hess(i + 1)           # beside prep(i) on the other stream
-                prep(i + 1)
+            if i + lag < layers:
+                hess(i + lag)         # beside the preparations on the other stream
+                prep(i + lag)
             quant(i)
 
     G.gptq_set_max_ctas(G.GPTQ_CTAS_HESSIAN, h_ctas)
+    G.gptq_set_max_ctas(G.GPTQ_CTAS_QUANTIZE, h_ctas)   # the SMs the preparation leaves
     G.gptq_set_max_ctas(G.GPTQ_CTAS_PREPARE, p_ctas)
     g = None
     try:
         run(max(3, warmup))
         torch.cuda.synchronize()
-        assert int(info2[0].item()) == 0 and int(info2[1].item()) == 0
+        assert all(int(x.item()) == 0 for x in info2)
         c0 = G.gptq_debug_launch_count()
         if graph:
             g = torch.cuda.CUDAGraph()
@@ -1020,10 +1032,11 @@ def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int,
             run(steps)
         end.record()
         torch.cuda.synchronize()
-        assert int(info2[0].item()) == 0 and int(info2[1].item()) == 0
+        assert all(int(x.item()) == 0 for x in info2)
         assert G.gptq_device_status(reset=True) == 0
     finally:
         G.gptq_set_max_ctas(G.GPTQ_CTAS_HESSIAN, 0)
+        G.gptq_set_max_ctas(G.GPTQ_CTAS_QUANTIZE, 0)
         G.gptq_set_max_ctas(G.GPTQ_CTAS_PREPARE, 0)
     del g
     return start.elapsed_time(end) / steps, per_layer

@@ -69,14 +69,17 @@ int gptq_device_status(int32_t* status_out, int reset);
 /*
  * Launch configuration (no counterpart on the pages): caps the CTAs of the
  * library's persistent kernels of one kind -- GPTQ_CTAS_HESSIAN (the Hessian
- * accumulation) or GPTQ_CTAS_PREPARE (the factorization in
- * gptq_prepare_hinv) -- at max_ctas (0: one per SM, the default).  A caller
- * that runs one layer's preparation beside the next layer's Hessian on two
- * streams gives each a share of the SMs this way; both kernels are correct
- * for any count.  Process-wide, read at each launch; not synchronized with
- * launches in flight.  Returns GPTQ_OK or GPTQ_ERR_INVALID_ARG.
+ * accumulation), GPTQ_CTAS_PREPARE (the factorization in gptq_prepare_hinv)
+ * or GPTQ_CTAS_QUANTIZE (the tensor-core updates in gptq_quantize_layer) --
+ * at max_ctas (0: one per SM, the default).  A caller that runs one layer's
+ * preparation beside the next layer's Hessian and quantization on two
+ * streams gives each a share of the SMs this way (a persistent grid larger
+ * than the SMs left to it would run its last CTAs after the others); every
+ * kernel is correct for any count.  Process-wide, read at each launch; not
+ * synchronized with launches in flight.  Returns GPTQ_OK or
+ * GPTQ_ERR_INVALID_ARG.
  */
-enum { GPTQ_CTAS_HESSIAN = 0, GPTQ_CTAS_PREPARE = 1 };
+enum { GPTQ_CTAS_HESSIAN = 0, GPTQ_CTAS_PREPARE = 1, GPTQ_CTAS_QUANTIZE = 2 };
 int gptq_set_max_ctas(int kind, int max_ctas);
 
 /*

@@ -34,7 +34,7 @@ int device_sm_count();
 
 // Persistent-grid caps set by gptq_set_max_ctas (0: none): the CTAs a
 // persistent kernel of that kind launches are min(SMs, cap).
-enum CtaKind : int { kCtaHessian = 0, kCtaPrepare = 1, kCtaKinds = 2 };
+enum CtaKind : int { kCtaHessian = 0, kCtaPrepare = 1, kCtaQuantize = 2, kCtaKinds = 3 };
 int persistent_ctas(int kind);
 
 // Diagnostics (gptq_debug_kernel_timing): kinds of the library's launches.

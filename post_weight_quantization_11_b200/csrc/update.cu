@@ -277,7 +277,7 @@ int block_update(float* Wk, const UpdateWs* w, int64_t m, int64_t d, int64_t e_c
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
             cudaSuccess)
             return GPTQ_ERR_CUDA;
-        const int grid = std::min(p.items, device_sm_count());
+        const int grid = std::min(p.items, persistent_ctas(kCtaQuantize));
         kern<<<grid, UB_THREADS, smem, st>>>(tEh, tEl, tUh, tUl, p);
         return GPTQ_OK;
     };

@@ -161,7 +161,7 @@ def gptq_device_status(reset: bool = True) -> int:
     return int(v.value)
 
 
-GPTQ_CTAS_HESSIAN, GPTQ_CTAS_PREPARE = 0, 1
+GPTQ_CTAS_HESSIAN, GPTQ_CTAS_PREPARE, GPTQ_CTAS_QUANTIZE = 0, 1, 2
 
 
 def gptq_set_max_ctas(kind: int, max_ctas: int) -> None:

@@ -39,7 +39,8 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_cta_caps(lib):
-    assert lib.gptq_set_max_ctas(2, 10) == 1 and lib.gptq_set_max_ctas(-1, 10) == 1
+    assert lib.gptq_set_max_ctas(3, 10) == 1 and lib.gptq_set_max_ctas(-1, 10) == 1
+    assert lib.gptq_set_max_ctas(2, 10) == 0 and lib.gptq_set_max_ctas(2, 0) == 0
     assert lib.gptq_set_max_ctas(0, -1) == 1
     assert lib.gptq_set_max_ctas(0, 32) == 0 and lib.gptq_set_max_ctas(1, 16) == 0
     assert lib.gptq_set_max_ctas(0, 0) == 0 and lib.gptq_set_max_ctas(1, 0) == 0

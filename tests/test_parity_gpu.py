@@ -402,6 +402,18 @@ def test_cta_caps_keep_the_results():
     a, b = P.to_np(S1).astype(np.float64), P.to_np(S0).astype(np.float64)
     assert P.rel_fro(np.triu(a), np.triu(b)) <= 1e-6
     assert torch.equal(U1, U0)
+    # the quantization's persistent updates on 20 CTAs: every tile's
+    # arithmetic is the same whichever CTA computes it (codes bit for bit)
+    W = _weights(384, d, torch.float16, 52).to(DEV)
+    ref = G.gptq_quantize_layer(W, U0, None, 4, 128)
+    try:
+        G.gptq_set_max_ctas(G.GPTQ_CTAS_QUANTIZE, 20)
+        got = G.gptq_quantize_layer(W, U0, None, 4, 128)
+        torch.cuda.synchronize()
+    finally:
+        G.gptq_set_max_ctas(G.GPTQ_CTAS_QUANTIZE, 0)
+    for x, y in zip(got, ref):
+        assert torch.equal(x, y)
 
 
 def test_prepare_reports_non_pd():
