@@ -373,12 +373,15 @@ int gptq_unpack_bits(const uint32_t* qweight, const uint8_t* qzeros, int64_t d_o
  * of the same page:
  *   y[b][r] = sum_j x[b][j] Q[r][j],  Q[r][perm[k]] = s[r][k/g] (c[r][k] - z[r][k/g])
  * with c, z unpacked from qweight / qzeros (gptq_pack_int4's layout, codes in
- * sweep order) and s the fp16 scales.  Products and sums are fp32; the
- * dequantized weights are exact.
+ * sweep order) and s the fp16 scales.  Products and sums are fp32 (the
+ * products on the tensor cores, m16n8k16, exact); the dequantized weights
+ * are exact.  Decode-sized: every CTA requests its rows' packed bytes for
+ * one 2048-column slice at once (bulk copies), the slices' partial sums
+ * meet in y by atomic adds.
  * x: batch x d_in fp16 (original column order); y: batch x d_out fp32 output
  * (overwritten).  perm: d_in int32 or NULL (identity), as gptq_prepare_hinv
  * returned it.  group_size: a multiple of 32 dividing d_in, or -1 (one group
- * per row).  batch in 1..4 (decode-sized; larger batches are UNSUPPORTED).
+ * per row).  batch in 1..8 (decode-sized; larger batches are UNSUPPORTED).
  * Requires d_in % 128 == 0, 128 <= d_in <= 32768, 1 <= d_out <= 2^24.
  */
 int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t* qweight,

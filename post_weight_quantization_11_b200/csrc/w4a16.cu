@@ -4,160 +4,198 @@
 //
 //   y[b][r] = sum_j x[b][j] Q[r][j],   Q[r][perm[k]] = s[r][k/g] (c[r][k] - z[r][k/g])
 //
-// for a small batch of activation rows (decode).  The weights stream from
-// HBM once; every product is fp32 with exact dequantization:
-//  * a code c in nibble i (0..3) of a 16-bit half of a packed word becomes
-//    the fp32 value c 16^i with one AND/OR and one subtraction (the bits go
-//    into the mantissa of 2^23), and the activation it meets is stored
-//    pre-multiplied by 16^-i (a power of two: exact), so c x needs no
-//    integer conversion;
-//  * per 16-code chunk (inside one group, g >= 16) the lane forms
-//    a = sum c x and adds s (a - z sum x) to its row's sum, the chunk's
-//    sum x taken once per CTA.
-// CTA: 8 warps x 4 rows, one K-slice of 2048 columns whose activations
-// (permuted to sweep order, pre-scaled) sit in shared memory; lanes take
-// 16-code chunks of the slice; the slices' partial sums meet in y by atomic
-// adds (y is zeroed first).
+// for a decode-sized batch (1..8 activation rows).  The weights stream from
+// HBM once, and a decode product is that stream: every CTA asks for all of
+// its packed bytes at once (one 1-D bulk copy per row onto one mbarrier), so
+// each SM has tens of KB in flight from the start.
+//  * CTA: 32 rows x one K-slice of 2048 columns; 8 warps = 2 row tiles of 16
+//    x 4 K-quarters; the slices' partial sums meet in y by atomic adds (y is
+//    zeroed first).
+//  * Products on the tensor cores, m16n8k16 mma.sync, fp16 x fp16 -> fp32
+//    (exact products, fp32 sums): the 16 x 16 weight fragment of a block of
+//    16 columns is two packed words per row; a word's nibble pair (j, j+4)
+//    becomes the fp16 pair (1024 + c_j, 1024 + c_{j+4}) by one AND/OR, and
+//    subtracting 1024 + z leaves the exact c - z.  Lane (g, t) takes pair
+//    t of each word, so the fragment's columns 2t, 2t+1, 2t+8, 2t+9 are the
+//    block's columns t, t+4, 8+t, 12+t: the activations are gathered into
+//    that order once per CTA (through perm), batch columns past the batch
+//    zero.
+//  * Per group (a multiple of 32 columns) the fp32 partial of each row is
+//    scaled by its fp16 scale in fp32; a warp's quarter is at most 512
+//    columns, so no accumulator sums more than 512 products.
+#include <atomic>
+
 #include "common.cuh"
 #include "tc_common.cuh"
 
 namespace gptq {
 
-constexpr int W4_KS = 2048;                 // columns per K-slice (CTA)
-constexpr int W4_WARPS = 8, W4_ROWS = 4;    // rows per warp
-constexpr int W4_THREADS = W4_WARPS * 32;
-constexpr int W4_CHUNK = 16;                // codes per lane step (two packed words)
-constexpr unsigned W4_FULL = 0xffffffffu;
+constexpr int WD_KS = 2048;                   // columns per K-slice (CTA)
+constexpr int WD_ROWS = 32;                   // rows per CTA
+constexpr int WD_THREADS = 256;               // 8 warps: 2 row tiles x 4 K-quarters
+constexpr int WD_WLD = WD_KS / 8 + 4;         // words per shared row (rows 4 banks apart)
+constexpr int WD_NB = 8;                      // batch columns of the mma (n = 8)
+constexpr size_t WD_SMEM = size_t(WD_ROWS) * WD_WLD * 4 + size_t(WD_KS) * WD_NB * 2 +
+                           4 * WD_ROWS * WD_NB * 4 + 16;
 
-__device__ __forceinline__ float nib16(uint32_t v, int i)
+// One 1-D bulk copy global -> shared completing on an mbarrier (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar)
 {
-    // c 16^i for the nibble i (0..3) of the low 16 bits of v, exactly
-    return __int_as_float(0x4B000000u | (v & (0xFu << (4 * i)))) - 8388608.0f;
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
-template <int B>
-__global__ void __launch_bounds__(W4_THREADS)
-w4a16_kernel(const __half* __restrict__ x, const uint32_t* __restrict__ qweight,
-             const __half* __restrict__ scales, const uint8_t* __restrict__ qzeros,
-             const int32_t* __restrict__ perm, int64_t m, int64_t d, int64_t g,
-             float* __restrict__ y)
+// D (16x8 fp32) += A (16x16 fp16, row) B (16x8 fp16, col)
+__device__ __forceinline__ void mma_f16_m16n8k16(float (&c)[4], const uint32_t (&a)[4],
+                                                 uint32_t b0, uint32_t b1)
 {
-    __shared__ __align__(16) float xs[B][W4_KS];               // pre-scaled x, sweep order
-    __shared__ float xsum[B][W4_KS / W4_CHUNK];                 // per-chunk sum of x
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t k0 = int64_t(blockIdx.y) * W4_KS;
-    const int klen = (int)(d - k0 < W4_KS ? d - k0 : W4_KS);         // a multiple of 128
-    const int nch = klen / W4_CHUNK;
-    const int64_t row0 = int64_t(blockIdx.x) * (W4_WARPS * W4_ROWS) + warp * W4_ROWS;
-    auto load = [&](int c, uint2 (&q)[W4_ROWS]) {
-        const int64_t gc = k0 / W4_CHUNK + c;
-#pragma unroll
-        for (int r = 0; r < W4_ROWS; ++r) {
-            const int64_t row = row0 + r;
-            q[r] = row < m ? *reinterpret_cast<const uint2*>(qweight + row * (d / 8) + 2 * gc)
-                           : make_uint2(0u, 0u);
-        }
-    };
-    // the lane's first two chunks of weights are requested before the
-    // activations are staged: their latency overlaps the staging below
-    uint2 q0[W4_ROWS], q1[W4_ROWS];
-    if (lane < nch) load(lane, q0);
-    if (lane + 32 < nch) load(lane + 32, q1);
-    for (int idx = tid; idx < B * klen; idx += W4_THREADS) {
-        const int b = idx / klen, kk = idx - b * klen;
-        const int64_t k = k0 + kk;
-        const int64_t src = perm ? int64_t(perm[k]) : k;
-        const bool in = src >= 0 && src < d;          // a bad index is not followed
-        if (!in) atomicCAS(&g_device_status, 0, kErrIndex);
-        xs[b][kk] = in ? ldexpf(__half2float(x[b * d + src]), -4 * (kk & 3)) : 0.f;
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Nibbles (j, j+4) of w as the fp16 pair (c_j - z, c_{j+4} - z), exact:
+// zz = the fp16 pair (1024 + z, 1024 + z) as bits.
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int j, uint32_t zz)
+{
+    const uint32_t v = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+    const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&v),
+                              *reinterpret_cast<const __half2*>(&zz));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__global__ void __launch_bounds__(WD_THREADS)
+w4a16_dec_kernel(const __half* __restrict__ x, int batch, const uint32_t* __restrict__ qweight,
+                 const __half* __restrict__ scales, const uint8_t* __restrict__ qzeros,
+                 const int32_t* __restrict__ perm, int64_t m, int64_t d, int64_t g,
+                 float* __restrict__ y)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint32_t* Wsm = reinterpret_cast<uint32_t*>(smem);
+    __half* Xs = reinterpret_cast<__half*>(smem + size_t(WD_ROWS) * WD_WLD * 4);
+    float* red = reinterpret_cast<float*>(smem + size_t(WD_ROWS) * WD_WLD * 4 +
+                                          size_t(WD_KS) * WD_NB * 2);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(red + 4 * WD_ROWS * WD_NB);
+    __shared__ int abort_flag;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t r0 = int64_t(blockIdx.x) * WD_ROWS;
+    const int64_t k0 = int64_t(blockIdx.y) * WD_KS;
+    const int klen = (int)min(int64_t(WD_KS), d - k0);     // a multiple of 128
+    const int rows = (int)min(int64_t(WD_ROWS), m - r0);
+    const int64_t wpr = d / 8;                             // packed words per row
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
     }
     __syncthreads();
-    for (int idx = tid; idx < B * nch; idx += W4_THREADS) {
-        const int b = idx / nch, c = idx - b * nch;
-        float sum = 0.f;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar, uint32_t(rows) * uint32_t(klen / 2));
+        for (int r = 0; r < rows; ++r)
+            bulk_load(Wsm + r * WD_WLD, qweight + (r0 + r) * wpr + k0 / 8, uint32_t(klen / 2), bar);
+    }
+    for (int i = tid; i < (WD_ROWS - rows) * (WD_KS / 8); i += WD_THREADS)
+        Wsm[(rows + i / (WD_KS / 8)) * WD_WLD + i % (WD_KS / 8)] = 0u;   // rows past m
+    // activations of the slice in fragment order: element (q, n, L) at
+    // (q * 8 + n) * 16 + L is column 16 q + p(L) of batch row n, with
+    // p(2t + e) = t + 4 e and p(8 + 2t + e) = 8 + t + 4 e (columns < 2^15:
+    // 32-bit indices)
+    {
+        constexpr int PER = WD_KS / WD_THREADS;            // slots per thread
+        int src[PER];
 #pragma unroll
-        for (int t = 0; t < W4_CHUNK; ++t) sum += ldexpf(xs[b][c * W4_CHUNK + t], 4 * (t & 3));
-        xsum[b][c] = sum;
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + u * WD_THREADS;            // slot (q, L) of the slice
+            const int L = i & 15;
+            const int p = 8 * (L >> 3) + ((L & 7) >> 1) + 4 * (L & 1);
+            const int col = int(k0) + (i & ~15) + p;
+            src[u] = (i < klen) ? (perm ? perm[col] : col) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + u * WD_THREADS;
+            if (i >= klen) continue;
+            const bool ok = src[u] >= 0 && src[u] < int(d);
+            if (!ok) atomicCAS(&g_device_status, 0, kErrIndex);   // a bad index is not followed
+            __half* dst = Xs + (i >> 4) * (WD_NB * 16) + (i & 15);
+#pragma unroll
+            for (int n = 0; n < WD_NB; ++n)
+                dst[n * 16] = (n < batch && ok) ? x[n * int(d) + src[u]] : __float2half(0.f);
+        }
     }
     __syncthreads();
+    mbar_wait(bar, 0, kErrWaitFull, &abort_flag);
 
-    const int64_t G = d / g, Gz = (G + 1) / 2;
-    float acc[W4_ROWS][B];
-#pragma unroll
-    for (int r = 0; r < W4_ROWS; ++r)
-#pragma unroll
-        for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
-
-    // one chunk of 16 codes for the warp's rows, packed words already loaded
-    auto chunk = [&](int c, const uint2 (&q)[W4_ROWS]) {
-        const int64_t gc = k0 / W4_CHUNK + c;                   // chunk index in the row
-        const int64_t gi = gc * W4_CHUNK / g;                   // its group
-        float xv[B][W4_CHUNK];
-#pragma unroll
-        for (int b = 0; b < B; ++b)
-#pragma unroll
-            for (int t4 = 0; t4 < W4_CHUNK / 4; ++t4) {
-                const float4 v = *reinterpret_cast<const float4*>(&xs[b][c * W4_CHUNK + 4 * t4]);
-                xv[b][4 * t4] = v.x; xv[b][4 * t4 + 1] = v.y;
-                xv[b][4 * t4 + 2] = v.z; xv[b][4 * t4 + 3] = v.w;
+    const int mt = warp & 1, kq = warp >> 1;               // row tile, K quarter
+    const int gq = lane >> 2, tq = lane & 3;
+    const int qlen = klen / 4;                             // a multiple of 32
+    const int kb0 = kq * qlen;
+    const int ra = 16 * mt + gq, rb = ra + 8;              // CTA-local rows
+    const bool va = ra < rows, vb = rb < rows;
+    const int gi = int(g);
+    const int64_t G = d / g, Gb = (G + 1) / 2;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};                   // (ra, 2tq), (ra, 2tq+1), (rb, 2tq), (rb, 2tq+1)
+    float part[4] = {0.f, 0.f, 0.f, 0.f};
+    float sa = 0.f, sb = 0.f;
+    uint32_t za = 0u, zb = 0u;
+    int grp = (int(k0) + kb0) / gi;                         // the group of the next block
+    int rem = (int(k0) + kb0) - grp * gi;                   // its column inside the group
+    --grp;
+    for (int kb = kb0; kb < kb0 + qlen; kb += 16, rem += 16) {
+        if (kb == kb0 || rem == gi) {                      // a group starts (or the quarter)
+            if (kb != kb0) {
+                acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
+                acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
+                part[0] = part[1] = part[2] = part[3] = 0.f;
             }
-#pragma unroll
-        for (int r = 0; r < W4_ROWS; ++r) {
-            const int64_t row = row0 + r;
-            if (row >= m) continue;
-            const float s = __half2float(scales[row * G + gi]);
-            const uint32_t zb = qzeros[row * Gz + gi / 2];
-            const float z = float((gi & 1) ? (zb >> 4) : (zb & 0xFu));
-            float a[B];
-#pragma unroll
-            for (int b = 0; b < B; ++b) a[b] = 0.f;
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-                const uint32_t word = w ? q[r].y : q[r].x;
-                const uint32_t hi = word >> 16;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float flo = nib16(word, i), fhi = nib16(hi, i);
-#pragma unroll
-                    for (int b = 0; b < B; ++b) {
-                        a[b] = fmaf(flo, xv[b][8 * w + i], a[b]);
-                        a[b] = fmaf(fhi, xv[b][8 * w + 4 + i], a[b]);
-                    }
-                }
+            if (rem == gi) rem = 0;
+            ++grp;
+            uint32_t zra = 0u, zrb = 0u;
+            sa = 0.f; sb = 0.f;
+            if (va) {
+                zra = (qzeros[(r0 + ra) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
+                sa = __half2float(scales[(r0 + ra) * G + grp]);
             }
-#pragma unroll
-            for (int b = 0; b < B; ++b) acc[r][b] = fmaf(s, fmaf(-z, xsum[b][c], a[b]), acc[r][b]);
+            if (vb) {
+                zrb = (qzeros[(r0 + rb) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
+                sb = __half2float(scales[(r0 + rb) * G + grp]);
+            }
+            const uint32_t ha = __half_as_ushort(__float2half(1024.f + float(zra)));
+            const uint32_t hb = __half_as_ushort(__float2half(1024.f + float(zrb)));
+            za = ha | (ha << 16);
+            zb = hb | (hb << 16);
         }
-    };
-    // two chunks per step; the next step's two chunks are requested before
-    // this step's are used, so each warp keeps up to 4 KB of loads in flight
-    for (int c = lane; c < nch; c += 64) {
-        uint2 n0[W4_ROWS], n1[W4_ROWS];
-        const int cn = c + 64;
-        if (cn < nch) load(cn, n0);
-        if (cn + 32 < nch) load(cn + 32, n1);
-        chunk(c, q0);
-        if (c + 32 < nch) chunk(c + 32, q1);
-#pragma unroll
-        for (int r = 0; r < W4_ROWS; ++r) { q0[r] = n0[r]; q1[r] = n1[r]; }
+        const uint2 wa = *reinterpret_cast<const uint2*>(Wsm + ra * WD_WLD + kb / 8);
+        const uint2 wb = *reinterpret_cast<const uint2*>(Wsm + rb * WD_WLD + kb / 8);
+        uint32_t a[4];
+        a[0] = nib_pair(wa.x, tq, za);                     // row ra, columns t, t+4
+        a[1] = nib_pair(wb.x, tq, zb);                     // row rb
+        a[2] = nib_pair(wa.y, tq, za);                     // row ra, columns 8+t, 12+t
+        a[3] = nib_pair(wb.y, tq, zb);
+        const __half* xb = Xs + ((kb >> 4) * WD_NB + gq) * 16;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xb + 2 * tq);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xb + 8 + 2 * tq);
+        mma_f16_m16n8k16(part, a, b0, b1);
     }
+    acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
+    acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
+    float* rq = red + kq * WD_ROWS * WD_NB;
+    rq[ra * WD_NB + 2 * tq] = acc[0];
+    rq[ra * WD_NB + 2 * tq + 1] = acc[1];
+    rq[rb * WD_NB + 2 * tq] = acc[2];
+    rq[rb * WD_NB + 2 * tq + 1] = acc[3];
+    __syncthreads();
+    const int rr = tid >> 3, cc = tid & 7;                 // one output per thread
+    if (rr < rows && cc < batch) {
+        float v = 0.f;
 #pragma unroll
-    for (int r = 0; r < W4_ROWS; ++r)
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            float v = acc[r][b];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(W4_FULL, v, o);
-            acc[r][b] = v;
-        }
-    if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < W4_ROWS; ++r) {
-            const int64_t row = row0 + r;
-            if (row < m)
-#pragma unroll
-                for (int b = 0; b < B; ++b) atomicAdd(y + b * m + row, acc[r][b]);
-        }
+        for (int k = 0; k < 4; ++k) v += red[k * WD_ROWS * WD_NB + rr * WD_NB + cc];
+        atomicAdd(&y[int64_t(cc) * m + r0 + rr], v);
     }
 }
 
@@ -173,7 +211,7 @@ extern "C" int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t*
     if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(qzeros) ||
         !aligned16(y) || (perm && !aligned16(perm)))
         return GPTQ_ERR_INVALID_ARG;
-    if (batch < 1 || batch > 4) return GPTQ_ERR_UNSUPPORTED;
+    if (batch < 1 || batch > WD_NB) return GPTQ_ERR_UNSUPPORTED;
     if (d_in < 128 || d_in > kMaxDim || d_in % 128 != 0 || d_out < 1 || d_out > kMaxRows)
         return GPTQ_ERR_SHAPE;
     const int64_t g = (group_size == -1) ? d_in : group_size;
@@ -182,15 +220,21 @@ extern "C" int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t*
     KernelTimer kt(kKW4A16, st);
     if (cudaMemsetAsync(y, 0, sizeof(float) * size_t(batch) * size_t(d_out), st) != cudaSuccess)
         return GPTQ_ERR_CUDA;
-    const dim3 grid((unsigned)ceil_div(d_out, W4_WARPS * W4_ROWS), (unsigned)ceil_div(d_in, W4_KS));
-    const __half* xh = reinterpret_cast<const __half*>(x);
-    const __half* sh = reinterpret_cast<const __half*>(scales);
-    switch (batch) {
-        case 1: w4a16_kernel<1><<<grid, W4_THREADS, 0, st>>>(xh, qweight, sh, qzeros, perm, d_out, d_in, g, y); break;
-        case 2: w4a16_kernel<2><<<grid, W4_THREADS, 0, st>>>(xh, qweight, sh, qzeros, perm, d_out, d_in, g, y); break;
-        case 3: w4a16_kernel<3><<<grid, W4_THREADS, 0, st>>>(xh, qweight, sh, qzeros, perm, d_out, d_in, g, y); break;
-        default: w4a16_kernel<4><<<grid, W4_THREADS, 0, st>>>(xh, qweight, sh, qzeros, perm, d_out, d_in, g, y); break;
+    {   // the shared-memory opt-in, once per device
+        static std::atomic<bool> done[64];
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
+        if (dev < 0 || dev >= 64 || !done[dev].load()) {
+            if (cudaFuncSetAttribute(w4a16_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)WD_SMEM) != cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            if (dev >= 0 && dev < 64) done[dev].store(true);
+        }
     }
+    const dim3 grid((unsigned)ceil_div(d_out, WD_ROWS), (unsigned)ceil_div(d_in, WD_KS));
+    w4a16_dec_kernel<<<grid, WD_THREADS, WD_SMEM, st>>>(
+        reinterpret_cast<const __half*>(x), (int)batch, qweight,
+        reinterpret_cast<const __half*>(scales), qzeros, perm, d_out, d_in, g, y);
     count_launches();
     return launch_status();
 }

@@ -520,7 +520,7 @@ def gptq_awq_search(W: torch.Tensor, S: torch.Tensor, n_tokens: int, abs_sum: to
 def gptq_w4a16_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
                     qzeros: torch.Tensor, group_size: int = 128, perm=None, y=None):
     """y = x Q^T (batch x d_out fp32) from the packed INT4 layer; x: batch x
-    d_in fp16 in original column order, batch 1..4."""
+    d_in fp16 in original column order, batch 1..8."""
     _need(x, "x", torch.float16)
     _need(qweight, "qweight")
     _need(scales, "scales", torch.float16)

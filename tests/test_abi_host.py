@@ -149,7 +149,7 @@ def test_validation_rejects_before_launch(lib):
     W4 = lib.gptq_w4a16_gemm
     assert W4(None, 1, FAKE, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 1
     assert W4(FAKE, 1, MIS, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 1
-    assert W4(FAKE, 5, FAKE, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 4
+    assert W4(FAKE, 9, FAKE, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 4
     assert W4(FAKE, 0, FAKE, FAKE, FAKE, None, 64, 256, 128, FAKE, None) == 4
     assert W4(FAKE, 1, FAKE, FAKE, FAKE, None, 64, 200, 128, FAKE, None) == 2
     assert W4(FAKE, 1, FAKE, FAKE, FAKE, None, 0, 256, 128, FAKE, None) == 2

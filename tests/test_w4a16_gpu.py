@@ -64,7 +64,8 @@ def _bound(x, codes, zeros, sc16, d, g, perm):
 
 @pytest.mark.parametrize("m,d,g,b,act", [(300, 256, 128, 1, False), (77, 4096, 128, 4, True),
                                          (33, 14336, 64, 2, False), (129, 1024, 32, 3, True),
-                                         (50, 2048, -1, 1, True)])
+                                         (50, 2048, -1, 1, True), (257, 4096, 32, 5, True),
+                                         (64, 6144, 128, 8, False)])
 def test_w4a16_exact_on_representable_values(m, d, g, b, act):
     rng = np.random.default_rng(1000 + m + d)
     codes, zeros, sc16, perm, qw, qz = _layer(rng, m, d, g, act, exact=True)
@@ -76,7 +77,8 @@ def test_w4a16_exact_on_representable_values(m, d, g, b, act):
 
 @pytest.mark.parametrize("m,d,g,b,act", [(300, 256, 128, 1, False), (77, 4096, 128, 4, True),
                                          (33, 14336, 64, 2, False), (129, 6144, 256, 2, True),
-                                         (50, 2048, -1, 3, False)])
+                                         (50, 2048, -1, 3, False), (200, 4096, 128, 8, True),
+                                         (31, 2304, 64, 6, False)])
 def test_w4a16_general_within_fp32_bound(m, d, g, b, act):
     rng = np.random.default_rng(2000 + m + d)
     codes, zeros, sc16, perm, qw, qz = _layer(rng, m, d, g, act, exact=False)
