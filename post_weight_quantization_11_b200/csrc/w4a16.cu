@@ -8,9 +8,11 @@
 // HBM once, and a decode product is that stream: every CTA asks for all of
 // its packed bytes at once (one 1-D bulk copy per row onto one mbarrier), so
 // each SM has tens of KB in flight from the start.
-//  * CTA: 32 rows x one K-slice of 2048 columns; 8 warps = 2 row tiles of 16
-//    x 4 K-quarters; the slices' partial sums meet in y by atomic adds (y is
-//    zeroed first).
+//  * CTA: one K-slice of 2048 columns and every gridDim.x-th tile of 32 rows
+//    (persistent over row tiles: the slice's activations are gathered once,
+//    the next tile's bytes are copied into the second of two buffers while
+//    this one is multiplied); 8 warps = 2 row halves of 16 x 4 K-quarters;
+//    the slices' partial sums meet in y by atomic adds (y is zeroed first).
 //  * Products on the tensor cores, m16n8k16 mma.sync, fp16 x fp16 -> fp32
 //    (exact products, fp32 sums): the 16 x 16 weight fragment of a block of
 //    16 columns is two packed words per row; a word's nibble pair (j, j+4)
@@ -35,8 +37,8 @@ constexpr int WD_ROWS = 32;                   // rows per CTA
 constexpr int WD_THREADS = 256;               // 8 warps: 2 row tiles x 4 K-quarters
 constexpr int WD_WLD = WD_KS / 8 + 4;         // words per shared row (rows 4 banks apart)
 constexpr int WD_NB = 8;                      // batch columns of the mma (n = 8)
-constexpr size_t WD_SMEM = size_t(WD_ROWS) * WD_WLD * 4 + size_t(WD_KS) * WD_NB * 2 +
-                           4 * WD_ROWS * WD_NB * 4 + 16;
+constexpr size_t WD_WBUF = size_t(WD_ROWS) * WD_WLD * 4;   // one row tile's packed slice
+constexpr size_t WD_SMEM = 2 * WD_WBUF + size_t(WD_KS) * WD_NB * 2 + 4 * WD_ROWS * WD_NB * 4 + 16;
 
 // One 1-D bulk copy global -> shared completing on an mbarrier (no multicast).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
@@ -76,31 +78,34 @@ w4a16_dec_kernel(const __half* __restrict__ x, int batch, const uint32_t* __rest
                  float* __restrict__ y)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t* Wsm = reinterpret_cast<uint32_t*>(smem);
-    __half* Xs = reinterpret_cast<__half*>(smem + size_t(WD_ROWS) * WD_WLD * 4);
-    float* red = reinterpret_cast<float*>(smem + size_t(WD_ROWS) * WD_WLD * 4 +
-                                          size_t(WD_KS) * WD_NB * 2);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(red + 4 * WD_ROWS * WD_NB);
+    uint32_t* Wb0 = reinterpret_cast<uint32_t*>(smem);      // buffer i at Wb0 + i * WD_WBUF / 4
+    __half* Xs = reinterpret_cast<__half*>(smem + 2 * WD_WBUF);
+    float* red = reinterpret_cast<float*>(smem + 2 * WD_WBUF + size_t(WD_KS) * WD_NB * 2);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(red + 4 * WD_ROWS * WD_NB);   // two
     __shared__ int abort_flag;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t r0 = int64_t(blockIdx.x) * WD_ROWS;
     const int64_t k0 = int64_t(blockIdx.y) * WD_KS;
     const int klen = (int)min(int64_t(WD_KS), d - k0);     // a multiple of 128
-    const int rows = (int)min(int64_t(WD_ROWS), m - r0);
     const int64_t wpr = d / 8;                             // packed words per row
+    const int64_t ntiles = (m + WD_ROWS - 1) / WD_ROWS;
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar, uint32_t(rows) * uint32_t(klen / 2));
+    // thread 0: the copies of row tile `tile` into buffer `buf`
+    auto issue = [&](int64_t tile, int buf) {
+        const int64_t r0 = tile * WD_ROWS;
+        const int rows = (int)min(int64_t(WD_ROWS), m - r0);
+        uint32_t* W = Wb0 + buf * (WD_WBUF / 4);
+        mbar_arrive_expect_tx(&bar[buf], uint32_t(rows) * uint32_t(klen / 2));
         for (int r = 0; r < rows; ++r)
-            bulk_load(Wsm + r * WD_WLD, qweight + (r0 + r) * wpr + k0 / 8, uint32_t(klen / 2), bar);
-    }
-    for (int i = tid; i < (WD_ROWS - rows) * (WD_KS / 8); i += WD_THREADS)
-        Wsm[(rows + i / (WD_KS / 8)) * WD_WLD + i % (WD_KS / 8)] = 0u;   // rows past m
+            bulk_load(W + r * WD_WLD, qweight + (r0 + r) * wpr + k0 / 8, uint32_t(klen / 2),
+                      &bar[buf]);
+    };
+    if (tid == 0 && int64_t(blockIdx.x) < ntiles) issue(blockIdx.x, 0);
     // activations of the slice in fragment order: element (q, n, L) at
     // (q * 8 + n) * 16 + L is column 16 q + p(L) of batch row n, with
     // p(2t + e) = t + 4 e and p(8 + 2t + e) = 8 + t + 4 e (columns < 2^15:
@@ -129,73 +134,82 @@ w4a16_dec_kernel(const __half* __restrict__ x, int batch, const uint32_t* __rest
         }
     }
     __syncthreads();
-    mbar_wait(bar, 0, kErrWaitFull, &abort_flag);
 
-    const int mt = warp & 1, kq = warp >> 1;               // row tile, K quarter
+    const int mt = warp & 1, kq = warp >> 1;               // row half, K quarter
     const int gq = lane >> 2, tq = lane & 3;
     const int qlen = klen / 4;                             // a multiple of 32
     const int kb0 = kq * qlen;
-    const int ra = 16 * mt + gq, rb = ra + 8;              // CTA-local rows
-    const bool va = ra < rows, vb = rb < rows;
+    const int ra = 16 * mt + gq, rb = ra + 8;              // rows inside the tile
     const int gi = int(g);
     const int64_t G = d / g, Gb = (G + 1) / 2;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};                   // (ra, 2tq), (ra, 2tq+1), (rb, 2tq), (rb, 2tq+1)
-    float part[4] = {0.f, 0.f, 0.f, 0.f};
-    float sa = 0.f, sb = 0.f;
-    uint32_t za = 0u, zb = 0u;
-    int grp = (int(k0) + kb0) / gi;                         // the group of the next block
-    int rem = (int(k0) + kb0) - grp * gi;                   // its column inside the group
-    --grp;
-    for (int kb = kb0; kb < kb0 + qlen; kb += 16, rem += 16) {
-        if (kb == kb0 || rem == gi) {                      // a group starts (or the quarter)
-            if (kb != kb0) {
-                acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
-                acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
-                part[0] = part[1] = part[2] = part[3] = 0.f;
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int buf = it & 1;
+        if (tid == 0 && tile + gridDim.x < ntiles) issue(tile + gridDim.x, buf ^ 1);
+        mbar_wait(&bar[buf], uint32_t((it >> 1) & 1), kErrWaitFull, &abort_flag);
+        const uint32_t* Wsm = Wb0 + buf * (WD_WBUF / 4);
+        const int64_t r0 = tile * WD_ROWS;
+        const int rows = (int)min(int64_t(WD_ROWS), m - r0);
+        const bool va = ra < rows, vb = rb < rows;        // rows past m: stale words, no output
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};               // (ra, 2tq), (ra, 2tq+1), (rb, 2tq), (rb, 2tq+1)
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+        float sa = 0.f, sb = 0.f;
+        uint32_t za = 0u, zb = 0u;
+        int grp = (int(k0) + kb0) / gi;                     // the group of the next block
+        int rem = (int(k0) + kb0) - grp * gi;               // its column inside the group
+        --grp;
+        for (int kb = kb0; kb < kb0 + qlen; kb += 16, rem += 16) {
+            if (kb == kb0 || rem == gi) {                  // a group starts (or the quarter)
+                if (kb != kb0) {
+                    acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
+                    acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
+                    part[0] = part[1] = part[2] = part[3] = 0.f;
+                }
+                if (rem == gi) rem = 0;
+                ++grp;
+                uint32_t zra = 0u, zrb = 0u;
+                sa = 0.f; sb = 0.f;
+                if (va) {
+                    zra = (qzeros[(r0 + ra) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
+                    sa = __half2float(scales[(r0 + ra) * G + grp]);
+                }
+                if (vb) {
+                    zrb = (qzeros[(r0 + rb) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
+                    sb = __half2float(scales[(r0 + rb) * G + grp]);
+                }
+                const uint32_t ha = __half_as_ushort(__float2half(1024.f + float(zra)));
+                const uint32_t hb = __half_as_ushort(__float2half(1024.f + float(zrb)));
+                za = ha | (ha << 16);
+                zb = hb | (hb << 16);
             }
-            if (rem == gi) rem = 0;
-            ++grp;
-            uint32_t zra = 0u, zrb = 0u;
-            sa = 0.f; sb = 0.f;
-            if (va) {
-                zra = (qzeros[(r0 + ra) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
-                sa = __half2float(scales[(r0 + ra) * G + grp]);
-            }
-            if (vb) {
-                zrb = (qzeros[(r0 + rb) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
-                sb = __half2float(scales[(r0 + rb) * G + grp]);
-            }
-            const uint32_t ha = __half_as_ushort(__float2half(1024.f + float(zra)));
-            const uint32_t hb = __half_as_ushort(__float2half(1024.f + float(zrb)));
-            za = ha | (ha << 16);
-            zb = hb | (hb << 16);
+            const uint2 wa = *reinterpret_cast<const uint2*>(Wsm + ra * WD_WLD + kb / 8);
+            const uint2 wb = *reinterpret_cast<const uint2*>(Wsm + rb * WD_WLD + kb / 8);
+            uint32_t a[4];
+            a[0] = nib_pair(wa.x, tq, za);                 // row ra, columns t, t+4
+            a[1] = nib_pair(wb.x, tq, zb);                 // row rb
+            a[2] = nib_pair(wa.y, tq, za);                 // row ra, columns 8+t, 12+t
+            a[3] = nib_pair(wb.y, tq, zb);
+            const __half* xb = Xs + ((kb >> 4) * WD_NB + gq) * 16;
+            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xb + 2 * tq);
+            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xb + 8 + 2 * tq);
+            mma_f16_m16n8k16(part, a, b0, b1);
         }
-        const uint2 wa = *reinterpret_cast<const uint2*>(Wsm + ra * WD_WLD + kb / 8);
-        const uint2 wb = *reinterpret_cast<const uint2*>(Wsm + rb * WD_WLD + kb / 8);
-        uint32_t a[4];
-        a[0] = nib_pair(wa.x, tq, za);                     // row ra, columns t, t+4
-        a[1] = nib_pair(wb.x, tq, zb);                     // row rb
-        a[2] = nib_pair(wa.y, tq, za);                     // row ra, columns 8+t, 12+t
-        a[3] = nib_pair(wb.y, tq, zb);
-        const __half* xb = Xs + ((kb >> 4) * WD_NB + gq) * 16;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xb + 2 * tq);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xb + 8 + 2 * tq);
-        mma_f16_m16n8k16(part, a, b0, b1);
-    }
-    acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
-    acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
-    float* rq = red + kq * WD_ROWS * WD_NB;
-    rq[ra * WD_NB + 2 * tq] = acc[0];
-    rq[ra * WD_NB + 2 * tq + 1] = acc[1];
-    rq[rb * WD_NB + 2 * tq] = acc[2];
-    rq[rb * WD_NB + 2 * tq + 1] = acc[3];
-    __syncthreads();
-    const int rr = tid >> 3, cc = tid & 7;                 // one output per thread
-    if (rr < rows && cc < batch) {
-        float v = 0.f;
+        acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
+        acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
+        float* rq = red + kq * WD_ROWS * WD_NB;
+        rq[ra * WD_NB + 2 * tq] = acc[0];
+        rq[ra * WD_NB + 2 * tq + 1] = acc[1];
+        rq[rb * WD_NB + 2 * tq] = acc[2];
+        rq[rb * WD_NB + 2 * tq + 1] = acc[3];
+        __syncthreads();
+        const int rr = tid >> 3, cc = tid & 7;             // one output per thread
+        if (rr < rows && cc < batch) {
+            float v = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) v += red[k * WD_ROWS * WD_NB + rr * WD_NB + cc];
-        atomicAdd(&y[int64_t(cc) * m + r0 + rr], v);
+            for (int k = 0; k < 4; ++k) v += red[k * WD_ROWS * WD_NB + rr * WD_NB + cc];
+            atomicAdd(&y[int64_t(cc) * m + r0 + rr], v);
+        }
+        __syncthreads();                                   // red and this buffer free again
     }
 }
 
@@ -231,7 +245,10 @@ extern "C" int gptq_w4a16_gemm(const uint16_t* x, int64_t batch, const uint32_t*
             if (dev >= 0 && dev < 64) done[dev].store(true);
         }
     }
-    const dim3 grid((unsigned)ceil_div(d_out, WD_ROWS), (unsigned)ceil_div(d_in, WD_KS));
+    // persistent over row tiles: two CTAs per SM over the slices
+    const int64_t slices = ceil_div(d_in, WD_KS), tiles = ceil_div(d_out, WD_ROWS);
+    const int64_t per_slice = std::max<int64_t>(1, ceil_div(2 * int64_t(device_sm_count()), slices));
+    const dim3 grid((unsigned)std::min(tiles, per_slice), (unsigned)slices);
     w4a16_dec_kernel<<<grid, WD_THREADS, WD_SMEM, st>>>(
         reinterpret_cast<const __half*>(x), (int)batch, qweight,
         reinterpret_cast<const __half*>(scales), qzeros, perm, d_out, d_in, g, y);
