@@ -237,7 +237,7 @@ int gptq_prepare_hinv_static(const float* S, int64_t d, int64_t n_tokens, float 
  * ws: gptq_prepare_batched_workspace_bytes(d, n_mats) bytes of scratch
  *    (n_mats times the single-matrix workspace, about 2 d^2 fp32 each).
  * Requires the d limits of gptq_prepare_hinv, 1 <= n_mats <= 4096 and
- * n_mats * d < 2^31.
+ * 2 n_mats d < 2^31.
  */
 size_t gptq_prepare_batched_workspace_bytes(int64_t d, int64_t n_mats);
 int gptq_prepare_hinv_batched(const float* S, int64_t n_mats, int64_t d, const int64_t* n_tokens,

@@ -15,6 +15,16 @@
 // the transpose, sum_k (X_kj)^T L_ik^T, so that every operand is read
 // K-major: they read Y = X^T, which they also write.
 //
+// Operands are stored split by the task that writes them, so a consumer's
+// TMA brings both parts and no thread touches them on the way to the MMA:
+// the tile holds the head hi = rna_tf32(x) in place of x and the remainder
+// x - hi sits in a tile nothing else uses -- the mirrored tile (c, r) for a
+// tile (r, c) off the diagonal of A (L and the S tasks' partial sums) and of
+// Y (X^T and the I tasks' partial sums), A's diagonal tile (j, j) (free once
+// F(j) has read it) for Y_jj, and a second d x 128 plane of Xc for X_jj.
+// The heads and remainders are the values a split in shared memory would
+// give, so the products are unchanged; U is written from the fp32 results.
+//
 // Scheduling: tasks are numbered in an order in which every dependency of
 // a task has a smaller number, and each CTA claims the next number from an
 // atomic counter.  A CTA waits (bounded) only for tasks with smaller
@@ -36,10 +46,11 @@
 // E matrices advance side by side on the SMs.
 //
 // CTA roles (320 threads): warp 0 TMA producer (also waits for the
-// dependencies), warp 1 MMA issuer, warps 2-9 split each landed fp32 chunk
-// into TF32 head / remainder and fold the previous product's TMEM
-// accumulator into registers (row m, 64 columns per thread), then write the
-// task's results through shared memory.  The leaf runs on all 320 threads
+// dependencies; four boxes per 32-wide K chunk: both parts of both
+// operands), warp 1 MMA issuer, warps 2-9 fold each product's TMEM
+// accumulator into registers (row m, 64 columns per thread) while the MMAs
+// fill the other accumulator, then write the task's results, split, through
+// shared memory.  The leaf runs on all 320 threads
 // (warp 0 as its panel warp, warps 1-9 as its update warps).
 #include "chol_dag.cuh"
 #include "leaf.cuh"
@@ -63,6 +74,7 @@ enum : int { kMapA = 0, kMapX = 1, kMapY = 2 };
 struct CdParams {
     float* A;
     float* Xc;
+    float* Xl;       // remainders of Xc (a second plane, E d x 128)
     float* Y;
     float* U;
     int* flagL;      // T x T: L_ij is final (for i == j: X_jj is in Xc)
@@ -84,6 +96,7 @@ __device__ __forceinline__ CdParams cd_matrix(const CdParams& p, int e)
     const int64_t dd = p.d * p.d, TT = int64_t(p.T) * p.T;
     q.A = p.A + e * dd;
     q.Xc = p.Xc + e * p.d * 128;
+    q.Xl = p.Xl + e * p.d * 128;
     q.Y = p.Y + e * dd;
     q.U = p.U + e * dd;
     q.flagL = p.flagL + e * 2 * TT;
@@ -94,11 +107,26 @@ __device__ __forceinline__ CdParams cd_matrix(const CdParams& p, int e)
 }
 
 struct CdProduct {
-    int ma, ra, ca;      // A operand: tensor map, first row, first column
-    int mb, rb, cb;      // B operand
+    int ma, ra, ca;      // A operand (heads): tensor map, first row, first column
+    int mb, rb, cb;      // B operand (heads)
     const int* f1;       // flags to acquire first (nullptr: none)
     const int* f2;
+    int mal, ral, cal;   // where the A operand's remainders are
+    int mbl, rbl, cbl;   // where the B operand's remainders are
 };
+
+// The tile holding the remainders of the operand tile at (map, tile row r,
+// tile column c) of matrix 0 (see the header): mirrored off the diagonal, A's
+// diagonal tile for Y's diagonal, the second plane for Xc (rows E d further).
+__device__ __forceinline__ void cd_lo_tile(const CdParams& p, int map, int r, int c, int& lmap,
+                                           int& lr, int& lc)
+{
+    if (map == kMapX) { lmap = kMapX; lr = r + p.E * (int)p.d; lc = c; return; }
+    const int tr = r / CD_T, tc = c / CD_T;
+    lmap = (map == kMapY && tr == tc) ? kMapA : map;
+    lr = tc * CD_T;
+    lc = tr * CD_T;
+}
 
 // Task number -> (type, i, j); see the order above.  Host and device (the
 // library's task-order test hook calls it on the host).
@@ -145,8 +173,12 @@ __device__ __forceinline__ CdProduct cd_product(const CdParams& p, int type, int
         r = CdProduct{kMapX, i * CD_T, 0, kMapY, j * CD_T, i * CD_T, &p.flagL[i * T + i],
                       nullptr};
     }
+    cd_lo_tile(p, r.ma, r.ra, r.ca, r.mal, r.ral, r.cal);
+    cd_lo_tile(p, r.mb, r.rb, r.cb, r.mbl, r.rbl, r.cbl);
     r.ra += p.roff;
     r.rb += p.roff;
+    r.ral += p.roff;
+    r.rbl += p.roff;
     return r;
 }
 
@@ -180,6 +212,43 @@ __device__ __forceinline__ void cd_tile_out_transposed(const float* sb, float* d
         for (int q = 0; q < CD_T / 32; ++q) dst[c * ld + 32 * q + lane] = sb[(32 * q + lane) * LDA + c];
 }
 
+// TF32 head (round to nearest) and fp32 remainder of x: the operand split
+__device__ __forceinline__ void cd_split(float x, float& hi, float& lo)
+{
+    hi = tf32_round(x);
+    lo = x - hi;
+}
+
+// cd_tile_out with the heads to dh and the remainders to dl (same layout)
+__device__ __forceinline__ void cd_tile_out_split(const float* sb, float* dh, float* dl,
+                                                  int64_t ld, int warp, int lane)
+{
+    for (int r = warp; r < CD_T; r += CD_THREADS / 32) {
+        const float4 v = *reinterpret_cast<const float4*>(sb + r * LDA + 4 * lane);
+        float4 h, l;
+        cd_split(v.x, h.x, l.x);
+        cd_split(v.y, h.y, l.y);
+        cd_split(v.z, h.z, l.z);
+        cd_split(v.w, h.w, l.w);
+        *reinterpret_cast<float4*>(dh + r * ld + 4 * lane) = h;
+        *reinterpret_cast<float4*>(dl + r * ld + 4 * lane) = l;
+    }
+}
+
+// cd_tile_out_transposed with the heads to dh and the remainders to dl
+__device__ __forceinline__ void cd_tile_out_transposed_split(const float* sb, float* dh, float* dl,
+                                                             int64_t ld, int warp, int lane)
+{
+    for (int c = warp; c < CD_T; c += CD_THREADS / 32)
+#pragma unroll
+        for (int q = 0; q < CD_T / 32; ++q) {
+            float h, l;
+            cd_split(sb[(32 * q + lane) * LDA + c], h, l);
+            dh[c * ld + 32 * q + lane] = h;
+            dl[c * ld + 32 * q + lane] = l;
+        }
+}
+
 __device__ __forceinline__ void cd_tile_zero(float* dst, int64_t ld, int warp, int lane)
 {
     for (int r = warp; r < CD_T; r += CD_THREADS / 32)
@@ -194,8 +263,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + CD_PIPE_BYTES);
-    uint64_t* conv_bar = full_bar + CD_STAGES;
-    uint64_t* empty_bar = conv_bar + CD_STAGES;
+    uint64_t* empty_bar = full_bar + CD_STAGES;
     uint64_t* accf_bar = empty_bar + CD_STAGES;
     uint64_t* acce_bar = accf_bar + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce_bar + 2);
@@ -212,7 +280,6 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     if (tid == 0) {
         for (int s = 0; s < CD_STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&conv_bar[s], 256);
             mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < 2; ++a) { mbar_init(&accf_bar[a], 1); mbar_init(&acce_bar[a], 256); }
@@ -226,8 +293,8 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const uint32_t tmem = *tmem_slot;
 
     // pipeline state of each role, carried across tasks
-    int pr_stage = 0, cv_stage = 0, mm_stage = 0;
-    uint32_t pr_phase = 0, cv_phase = 0, mm_phase = 0;
+    int pr_stage = 0, mm_stage = 0;
+    uint32_t pr_phase = 0, mm_phase = 0;
     uint32_t armed = 0, armed_par = 0;
     int mm_it = 0, ep_it = 0;
     // warps 2-9: tile row m = qrow*32 + lane (TMEM lane quarter of the warp),
@@ -248,6 +315,8 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     fence_proxy_async_global();
                     const CUtensorMap* ma = pr.ma == kMapA ? &tmA : pr.ma == kMapX ? &tmX : &tmY;
                     const CUtensorMap* mb = pr.mb == kMapA ? &tmA : pr.mb == kMapX ? &tmX : &tmY;
+                    const CUtensorMap* mal = pr.mal == kMapA ? &tmA : pr.mal == kMapX ? &tmX : &tmY;
+                    const CUtensorMap* mbl = pr.mbl == kMapA ? &tmA : pr.mbl == kMapX ? &tmX : &tmY;
                     bool ok = true;
                     for (int kc = 0; kc < CD_T / CD_KC; ++kc) {
                         if (!mbar_wait(&empty_bar[pr_stage], pr_phase ^ 1, kErrWaitEmpty, abort)) {
@@ -255,10 +324,14 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                             break;
                         }
                         uint8_t* st = smem + pr_stage * CD_STAGE_BYTES;
-                        mbar_arrive_expect_tx(&full_bar[pr_stage], 2 * CD_TILE_BYTES);
+                        mbar_arrive_expect_tx(&full_bar[pr_stage], 4 * CD_TILE_BYTES);
                         tma_load_2d(st, ma, &full_bar[pr_stage], pr.ca + kc * CD_KC, pr.ra);
+                        tma_load_2d(st + CD_TILE_BYTES, mal, &full_bar[pr_stage],
+                                    pr.cal + kc * CD_KC, pr.ral);
                         tma_load_2d(st + 2 * CD_TILE_BYTES, mb, &full_bar[pr_stage],
                                     pr.cb + kc * CD_KC, pr.rb);
+                        tma_load_2d(st + 3 * CD_TILE_BYTES, mbl, &full_bar[pr_stage],
+                                    pr.cbl + kc * CD_KC, pr.rbl);
                         armed |= 1u << pr_stage;
                         armed_par = (armed_par & ~(1u << pr_stage)) | (pr_phase << pr_stage);
                         if (++pr_stage == CD_STAGES) { pr_stage = 0; pr_phase ^= 1; }
@@ -277,7 +350,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     const uint32_t d_tmem = tmem + uint32_t(a * CD_T);
                     uint32_t accum = 0;
                     for (int kc = 0; kc < CD_T / CD_KC; ++kc) {
-                        if (!mbar_wait(&conv_bar[mm_stage], mm_phase, kErrWaitFull, abort)) {
+                        if (!mbar_wait(&full_bar[mm_stage], mm_phase, kErrWaitFull, abort)) {
                             ok = false;
                             break;
                         }
@@ -304,58 +377,23 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
             }
         } else {
-            // warps 2-9: split the chunks of product q, then fold product q-1
-            // (the MMA of q-1 overlaps the split of q)
-            const int ct = tid - 64;
-            bool ok = true;
-            for (int qi = 0; qi <= n && ok; ++qi) {
-                if (qi < n) {
-                    for (int kc = 0; kc < CD_T / CD_KC; ++kc) {
-                        if (!mbar_wait(&full_bar[cv_stage], cv_phase, kErrWaitFull, abort)) {
-                            ok = false;
-                            break;
-                        }
-                        uint8_t* st = smem + cv_stage * CD_STAGE_BYTES;
+            // warps 2-9: fold each product as its accumulator fills (the MMAs
+            // of the next product run into the other accumulator meanwhile)
+            for (int qi = 0; qi < n; ++qi) {
+                const int a = ep_it & 1;
+                const uint32_t aph = (ep_it >> 1) & 1;
+                ++ep_it;
+                if (!mbar_wait(&accf_bar[a], aph, kErrWaitAccFull, abort)) break;
+                tc_fence_after();
 #pragma unroll
-                        for (int op = 0; op < 2; ++op) {
-                            float4* hi = reinterpret_cast<float4*>(st + op * 2 * CD_TILE_BYTES);
-                            float4* lo = reinterpret_cast<float4*>(st + op * 2 * CD_TILE_BYTES +
-                                                                   CD_TILE_BYTES);
-#pragma unroll
-                            for (int u = 0; u < CD_TILE_BYTES / 16 / 256; ++u) {
-                                const int e = ct + 256 * u;
-                                const float4 x = hi[e];
-                                float4 hv, lv;
-                                hv.x = tf32_round(x.x); lv.x = x.x - hv.x;
-                                hv.y = tf32_round(x.y); lv.y = x.y - hv.y;
-                                hv.z = tf32_round(x.z); lv.z = x.z - hv.z;
-                                hv.w = tf32_round(x.w); lv.w = x.w - hv.w;
-                                hi[e] = hv;
-                                lo[e] = lv;
-                            }
-                        }
-                        fence_proxy_async_smem();
-                        mbar_arrive(&conv_bar[cv_stage]);
-                        if (++cv_stage == CD_STAGES) { cv_stage = 0; cv_phase ^= 1; }
-                    }
-                    if (!ok) break;
+                for (int cc = 0; cc < 2; ++cc) {
+                    float v[32];
+                    tmem_ld32(tmem + uint32_t(a * CD_T + (2 * half + cc) * 32) +
+                                  (uint32_t(qrow * 32) << 16), v);
+                    epi(v, cc);
                 }
-                if (qi > 0) {
-                    const int a = ep_it & 1;
-                    const uint32_t aph = (ep_it >> 1) & 1;
-                    ++ep_it;
-                    if (!mbar_wait(&accf_bar[a], aph, kErrWaitAccFull, abort)) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        float v[32];
-                        tmem_ld32(tmem + uint32_t(a * CD_T + (2 * half + cc) * 32) +
-                                      (uint32_t(qrow * 32) << 16), v);
-                        epi(v, cc);
-                    }
-                    tc_fence_before();
-                    mbar_arrive(&acce_bar[a]);
-                }
+                tc_fence_before();
+                mbar_arrive(&acce_bar[a]);
             }
         }
     };
@@ -430,8 +468,14 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             // X_jj first: the S tasks of column j wait only for it
             for (int idx = tid * 4; idx < CD_T * CD_T; idx += CD_THREADS * 4) {
                 const int r = idx / CD_T, c = idx % CD_T;
-                *reinterpret_cast<float4*>(q.Xc + (c0 + r) * CD_T + c) =
-                    *reinterpret_cast<const float4*>(lx + r * LDA + c);
+                const float4 v = *reinterpret_cast<const float4*>(lx + r * LDA + c);
+                float4 h, l;
+                cd_split(v.x, h.x, l.x);
+                cd_split(v.y, h.y, l.y);
+                cd_split(v.z, h.z, l.z);
+                cd_split(v.w, h.w, l.w);
+                *reinterpret_cast<float4*>(q.Xc + (c0 + r) * CD_T + c) = h;
+                *reinterpret_cast<float4*>(q.Xl + (c0 + r) * CD_T + c) = l;
             }
             fence_proxy_async_global();
             __syncthreads();
@@ -439,15 +483,17 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 __threadfence();
                 st_release_gpu(&q.flagL[tj * T + tj], 1);
             }
-            // then Y_jj = X_jj^T and the diagonal tile of U
-            cd_tile_out_transposed(lx, q.Y + c0 * d + c0, d, warp, lane);
+            // then Y_jj = X_jj^T (remainders into A's diagonal tile, which
+            // nothing reads any more) and the diagonal tile of U
+            cd_tile_out_transposed_split(lx, q.Y + c0 * d + c0, q.A + c0 * d + c0, d, warp, lane);
             cd_tile_out_reversed(lx, q.U + (d - CD_T - c0) * d + (d - CD_T - c0), d, warp, lane);
             release(&q.flagY[tj * T + tj]);
         } else if (type == kTaskS) {
-            if (n1 > 0) {             // A_ij - sum back into A: the final product reads it
+            {   // A_ij - sum back into A, split (remainders in the mirrored
+                // tile): the final product reads it
                 stage_acc();
                 __syncthreads();
-                cd_tile_out(sb, q.A + r0 * d + c0, d, warp, lane);
+                cd_tile_out_split(sb, q.A + r0 * d + c0, q.A + c0 * d + r0, d, warp, lane);
                 fence_proxy_async_global();
                 fence_proxy_async_smem();
                 __syncthreads();
@@ -460,13 +506,13 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
             });
             __syncthreads();
-            cd_tile_out(sb, q.A + r0 * d + c0, d, warp, lane);
+            cd_tile_out_split(sb, q.A + r0 * d + c0, q.A + c0 * d + r0, d, warp, lane);
             release(&q.flagL[ti * T + tj]);
         } else {
             // the sum's transpose into the Y_ji tile: the final product reads it
             stage_acc();
             __syncthreads();
-            cd_tile_out(sb, q.Y + c0 * d + r0, d, warp, lane);
+            cd_tile_out_split(sb, q.Y + c0 * d + r0, q.Y + r0 * d + c0, d, warp, lane);
             fence_proxy_async_global();
             fence_proxy_async_smem();
             __syncthreads();
@@ -478,7 +524,7 @@ chol_dag_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         make_float4(-v[4 * u], -v[4 * u + 1], -v[4 * u + 2], -v[4 * u + 3]);
             });
             __syncthreads();
-            cd_tile_out_transposed(sb, q.Y + c0 * d + r0, d, warp, lane);
+            cd_tile_out_transposed_split(sb, q.Y + c0 * d + r0, q.Y + r0 * d + c0, d, warp, lane);
             cd_tile_out_reversed(sb, q.U + (d - CD_T - r0) * d + (d - CD_T - c0), d, warp, lane);
             release(&q.flagY[tj * T + ti]);
         }
@@ -505,10 +551,12 @@ int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d,
 {
     if (d < CD_T || d % CD_T) return GPTQ_ERR_SHAPE;
     const int T = (int)(d / CD_T);
-    if (E < 1 || E * d > (int64_t(1) << 31) - 1 || E * T * T > (int64_t(1) << 30))
+    // 2 E d: the rows of Xc's two planes, int32 TMA coordinates
+    if (E < 1 || 2 * E * d > (int64_t(1) << 31) - 1 || E * T * T > (int64_t(1) << 30))
         return GPTQ_ERR_SHAPE;
     CdParams p{};
     p.A = A; p.Xc = Xc; p.Y = Y; p.U = U;
+    p.Xl = Xc + E * d * CD_T;          // the remainder plane
     int* s = reinterpret_cast<int*>(sync);
     p.flagL = s;
     p.flagY = s + size_t(T) * T;
@@ -526,7 +574,7 @@ int chol_inv_dag(float* A, float* Xc, float* Y, float* U, void* sync, int64_t d,
     const uint64_t rows = uint64_t(E) * uint64_t(d);
     if (encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, A, (uint64_t)d, rows,
                        (uint64_t)d * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
-        encode_tmap_2d(&tX, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Xc, (uint64_t)CD_T, rows,
+        encode_tmap_2d(&tX, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Xc, (uint64_t)CD_T, 2 * rows,
                        (uint64_t)CD_T * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK ||
         encode_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, (uint64_t)d, rows,
                        (uint64_t)d * 4, CD_KC, CD_T, CU_TENSOR_MAP_SWIZZLE_128B) != GPTQ_OK)

@@ -26,7 +26,7 @@ constexpr int TW = 128;            // tile width of the factorization
 struct PrepWs {
     float* A;      // d x d reversed damped H (lower tiles), then L
     float* Y;      // d x d, (L^-1)^T in the upper tiles
-    float* Xc;     // d x 128, the diagonal tiles of L^-1
+    float* Xc;     // 2 d x 128, the diagonal tiles of L^-1 (TF32 heads, then remainders)
     void* sync;    // dependency flags of the factorization
     float* keys;   // d
     float* lam;    // 1
@@ -34,14 +34,15 @@ struct PrepWs {
 };
 
 // Workspace of a batch of E matrices (E = 1: one layer); matrix e's parts at
-// e d^2 (A, Y), e d 128 (Xc), e d (keys, pid) and 4 e (lam).
+// e d^2 (A, Y), e d 128 (each of Xc's two planes), e d (keys, pid) and 4 e
+// (lam).
 static size_t prep_layout(int64_t d, int64_t E, char* base, PrepWs* w)
 {
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 1024); return o; };
     size_t oA = take(sizeof(float) * d * d * E);
     size_t oY = take(sizeof(float) * d * d * E);
-    size_t oX = take(sizeof(float) * d * TW * E);
+    size_t oX = take(sizeof(float) * d * TW * E * 2);
     size_t oS = take(chol_dag_sync_bytes(d, E));
     size_t oK = take(sizeof(float) * d * E);
     size_t oL = take(sizeof(float) * 4 * E);
@@ -216,7 +217,7 @@ extern "C" int gptq_prepare_hinv_batched(const float* S, int64_t n_mats, int64_t
     int rc = prepare_check_args(S, d, damp_rel, act_order, perm, U, info);
     if (rc != GPTQ_OK) return rc;
     if (!n_tokens || !ws || !aligned16(ws)) return GPTQ_ERR_INVALID_ARG;
-    if (n_mats < 1 || n_mats > 4096 || n_mats * d > (int64_t(1) << 31) - 1)
+    if (n_mats < 1 || n_mats > 4096 || 2 * n_mats * d > (int64_t(1) << 31) - 1)
         return GPTQ_ERR_SHAPE;
     for (int64_t e = 0; e < n_mats; ++e)
         if (n_tokens[e] <= 0) return GPTQ_ERR_SHAPE;
