@@ -5,9 +5,9 @@ A step is one pass of the whole hot path over one layer whose inputs are
 resident in HBM: zero S, accumulate S = X^T X over all calibration tokens,
 prepare U (damp, factor, invert), sweep all columns with error feedback, and
 pack to INT4.  The timed region runs K consecutive layers, each through
-every phase, with layer i's preparation (a latency chain on 16 CTAs) on a
-second stream beside layer i+1's Hessian (132 CTAs); value = layers' weights
-/ that time.  The single-layer step, replayed as a CUDA graph with nothing
+every phase, with layer i's preparation (a latency chain on 12 CTAs) on a
+second stream beside the next layers' Hessians (136 CTAs); value = layers'
+weights / that time.  The single-layer step, replayed as a CUDA graph with nothing
 overlapped, is reported beside it (single_layer).  Default workload: the 7B attention projection (W 4096 x 4096
 fp16, X 262144 tokens x 4096 fp16 with 1 % outlier channels), synthetic and
 seeded.  Under torchrun every rank quantizes its own independent layer (weak
@@ -38,7 +38,7 @@ import numpy as np
 import torch
 
 METRIC = "GPTQ INT4-g128 weights quantized/sec per layer"
-PIPE_H, PIPE_P = 132, 16      # CTA caps of the Hessian and the factorization when layers overlap
+PIPE_H, PIPE_P = 136, 12      # CTA caps of the Hessian and the factorization when layers overlap
 UNIT = "weights/s"
 
 
@@ -717,7 +717,8 @@ def run_ours(a):
                         f", consecutive layers: every layer's preparation on a second stream, "
                         f"layer i quantized after layer i+2's Hessian (persistent grids capped "
                         f"at {PIPE_H} CTAs for the Hessian and the updates, {PIPE_P} for the "
-                        f"factorization); every layer runs every phase") if pipelined else
+                        f"factorization but the last two layers', which have no Hessian left "
+                        f"beside them); every layer runs every phase") if pipelined else
                        ("cuda_graph" if not a.eager else "eager"),
         "single_layer": single,
         # one Hessian serves q/k/v (or up/gate) in a model: the rate of the
@@ -945,7 +946,7 @@ def run_ours_one_layer(a):
 
 
 def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int,
-                  graph: bool = True, lag: int = 2):
+                  graph: bool = True, lag: int = 2, uncap_tail: bool = True):
     """(ms per layer, library launches per layer) of consecutive layers with
     each layer's preparation on a second stream: the factorization is a
     latency chain that needs few SMs, the Hessian and the quantization keep
@@ -959,7 +960,10 @@ def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int,
     schedule of `steps` layers (both streams, joined by events) is captured
     once as a CUDA graph and replayed; otherwise it is launched eagerly.  The
     persistent grids are capped at h_ctas (Hessian, updates) / p_ctas
-    (factorization) CTAs meanwhile (the caps are read at capture)."""
+    (factorization) CTAs meanwhile (the caps are read at capture), except
+    for the preparations of the last `lag` layers: no Hessian is left to
+    run beside them (the last one ends while the first of them starts), so
+    they take the whole GPU rather than draining on p_ctas CTAs."""
     G = lay.G
     dev = lay.S.device
     n = lay.n
@@ -981,11 +985,16 @@ def _pipelined_ms(lay, steps: int, warmup: int, h_ctas: int, p_ctas: int,
             evH[i].record(sH)
 
         def prep(i):
+            tail = uncap_tail and i >= layers - lag   # no Hessian left to share the SMs with
+            if tail:
+                G.gptq_set_max_ctas(G.GPTQ_CTAS_PREPARE, 0)
             sP.wait_event(evH[i])
             with torch.cuda.stream(sP):
                 G.gptq_prepare_hinv(S2[i % nb], n, 0.01, lay.act_order, perm2[i % nb],
                                     U2[i % nb], info2[i % nb], lay.ws_p)
             evP[i].record(sP)
+            if tail:
+                G.gptq_set_max_ctas(G.GPTQ_CTAS_PREPARE, p_ctas)
 
         def quant(i):
             sH.wait_event(evP[i])
