@@ -116,7 +116,7 @@ struct CdProduct {
 };
 
 // The tile holding the remainders of the operand tile at (map, tile row r,
-// tile column c) of matrix 0 (see the header): mirrored off the diagonal, A's
+// tile column c) of matrix 0 (see the top of this file): mirrored off the diagonal, A's
 // diagonal tile for Y's diagonal, the second plane for Xc (rows E d further).
 __device__ __forceinline__ void cd_lo_tile(const CdParams& p, int map, int r, int c, int& lmap,
                                            int& lr, int& lc)
@@ -182,15 +182,8 @@ __device__ __forceinline__ CdProduct cd_product(const CdParams& p, int type, int
     return r;
 }
 
-// Tile copies between the shared staging tile sb (128 x LDA floats) and
-// global memory, one warp per row so that every store is coalesced.
-__device__ __forceinline__ void cd_tile_out(const float* sb, float* dst, int64_t ld, int warp,
-                                            int lane)
-{
-    for (int r = warp; r < CD_T; r += CD_THREADS / 32)
-        *reinterpret_cast<float4*>(dst + r * ld + 4 * lane) =
-            *reinterpret_cast<const float4*>(sb + r * LDA + 4 * lane);
-}
+// Tile copies from the shared staging tile sb (128 x LDA floats) to global
+// memory, one warp per row (or column) so that every store is coalesced.
 
 // dst[127 - r][127 - c] = sb[r][c]  (a tile of U from a tile of X)
 __device__ __forceinline__ void cd_tile_out_reversed(const float* sb, float* dst, int64_t ld,
@@ -203,15 +196,6 @@ __device__ __forceinline__ void cd_tile_out_reversed(const float* sb, float* dst
     }
 }
 
-// dst[c][r] = sb[r][c]  (lanes along r: coalesced stores, 4-way bank conflicts)
-__device__ __forceinline__ void cd_tile_out_transposed(const float* sb, float* dst, int64_t ld,
-                                                       int warp, int lane)
-{
-    for (int c = warp; c < CD_T; c += CD_THREADS / 32)
-#pragma unroll
-        for (int q = 0; q < CD_T / 32; ++q) dst[c * ld + 32 * q + lane] = sb[(32 * q + lane) * LDA + c];
-}
-
 // TF32 head (round to nearest) and fp32 remainder of x: the operand split
 __device__ __forceinline__ void cd_split(float x, float& hi, float& lo)
 {
@@ -219,7 +203,7 @@ __device__ __forceinline__ void cd_split(float x, float& hi, float& lo)
     lo = x - hi;
 }
 
-// cd_tile_out with the heads to dh and the remainders to dl (same layout)
+// dh[r][c] = head of sb[r][c], dl[r][c] = its remainder
 __device__ __forceinline__ void cd_tile_out_split(const float* sb, float* dh, float* dl,
                                                   int64_t ld, int warp, int lane)
 {
@@ -235,7 +219,8 @@ __device__ __forceinline__ void cd_tile_out_split(const float* sb, float* dh, fl
     }
 }
 
-// cd_tile_out_transposed with the heads to dh and the remainders to dl
+// dh[c][r] = head of sb[r][c], dl[c][r] = its remainder (lanes along r:
+// coalesced stores, 4-way bank conflicts on the reads)
 __device__ __forceinline__ void cd_tile_out_transposed_split(const float* sb, float* dh, float* dl,
                                                              int64_t ld, int warp, int lane)
 {
