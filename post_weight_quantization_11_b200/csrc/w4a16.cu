@@ -152,50 +152,52 @@ w4a16_dec_kernel(const __half* __restrict__ x, int batch, const uint32_t* __rest
         const int rows = (int)min(int64_t(WD_ROWS), m - r0);
         const bool va = ra < rows, vb = rb < rows;        // rows past m: stale words, no output
         float acc[4] = {0.f, 0.f, 0.f, 0.f};               // (ra, 2tq), (ra, 2tq+1), (rb, 2tq), (rb, 2tq+1)
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-        float sa = 0.f, sb = 0.f;
-        uint32_t za = 0u, zb = 0u;
-        int grp = (int(k0) + kb0) / gi;                     // the group of the next block
-        int rem = (int(k0) + kb0) - grp * gi;               // its column inside the group
-        --grp;
-        for (int kb = kb0; kb < kb0 + qlen; kb += 16, rem += 16) {
-            if (kb == kb0 || rem == gi) {                  // a group starts (or the quarter)
-                if (kb != kb0) {
-                    acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
-                    acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
-                    part[0] = part[1] = part[2] = part[3] = 0.f;
-                }
-                if (rem == gi) rem = 0;
-                ++grp;
-                uint32_t zra = 0u, zrb = 0u;
-                sa = 0.f; sb = 0.f;
-                if (va) {
-                    zra = (qzeros[(r0 + ra) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
-                    sa = __half2float(scales[(r0 + ra) * G + grp]);
-                }
-                if (vb) {
-                    zrb = (qzeros[(r0 + rb) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
-                    sb = __half2float(scales[(r0 + rb) * G + grp]);
-                }
-                const uint32_t ha = __half_as_ushort(__float2half(1024.f + float(zra)));
-                const uint32_t hb = __half_as_ushort(__float2half(1024.f + float(zrb)));
-                za = ha | (ha << 16);
-                zb = hb | (hb << 16);
+        // the quarter in segments of one group each (a group may start before
+        // the quarter or end after it): the group's scales and zero points,
+        // then its blocks of 16 columns with no per-block bookkeeping
+        const int kend = kb0 + qlen;
+        int col = int(k0) + kb0;                           // absolute column of kb
+        int grp = col / gi;
+        for (int kb = kb0; kb < kend; ++grp) {
+            const int seg_end = min(kend, kb + (grp + 1) * gi - col);
+            uint32_t zra = 0u, zrb = 0u;
+            float sa = 0.f, sb = 0.f;
+            if (va) {
+                zra = (qzeros[(r0 + ra) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
+                sa = __half2float(scales[(r0 + ra) * G + grp]);
             }
-            const uint2 wa = *reinterpret_cast<const uint2*>(Wsm + ra * WD_WLD + kb / 8);
-            const uint2 wb = *reinterpret_cast<const uint2*>(Wsm + rb * WD_WLD + kb / 8);
-            uint32_t a[4];
-            a[0] = nib_pair(wa.x, tq, za);                 // row ra, columns t, t+4
-            a[1] = nib_pair(wb.x, tq, zb);                 // row rb
-            a[2] = nib_pair(wa.y, tq, za);                 // row ra, columns 8+t, 12+t
-            a[3] = nib_pair(wb.y, tq, zb);
+            if (vb) {
+                zrb = (qzeros[(r0 + rb) * Gb + grp / 2] >> (4 * (grp & 1))) & 0xFu;
+                sb = __half2float(scales[(r0 + rb) * G + grp]);
+            }
+            const uint32_t ha = __half_as_ushort(__float2half(1024.f + float(zra)));
+            const uint32_t hb = __half_as_ushort(__float2half(1024.f + float(zrb)));
+            const uint32_t za = ha | (ha << 16), zb = hb | (hb << 16);
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint32_t* pa = Wsm + ra * WD_WLD + kb / 8;
+            const uint32_t* pb = Wsm + rb * WD_WLD + kb / 8;
             const __half* xb = Xs + ((kb >> 4) * WD_NB + gq) * 16;
-            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xb + 2 * tq);
-            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xb + 8 + 2 * tq);
-            mma_f16_m16n8k16(part, a, b0, b1);
+#pragma unroll 4
+            for (int k = kb; k < seg_end; k += 16) {
+                const uint2 wa = *reinterpret_cast<const uint2*>(pa);
+                const uint2 wb = *reinterpret_cast<const uint2*>(pb);
+                uint32_t a[4];
+                a[0] = nib_pair(wa.x, tq, za);             // row ra, columns t, t+4
+                a[1] = nib_pair(wb.x, tq, zb);             // row rb
+                a[2] = nib_pair(wa.y, tq, za);             // row ra, columns 8+t, 12+t
+                a[3] = nib_pair(wb.y, tq, zb);
+                const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xb + 2 * tq);
+                const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xb + 8 + 2 * tq);
+                mma_f16_m16n8k16(part, a, b0, b1);
+                pa += 2;
+                pb += 2;
+                xb += WD_NB * 16;
+            }
+            acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
+            acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
+            col += seg_end - kb;
+            kb = seg_end;
         }
-        acc[0] = fmaf(sa, part[0], acc[0]); acc[1] = fmaf(sa, part[1], acc[1]);
-        acc[2] = fmaf(sb, part[2], acc[2]); acc[3] = fmaf(sb, part[3], acc[3]);
         float* rq = red + kq * WD_ROWS * WD_NB;
         rq[ra * WD_NB + 2 * tq] = acc[0];
         rq[ra * WD_NB + 2 * tq + 1] = acc[1];
