@@ -57,7 +57,11 @@ def test_status_strings_and_version(lib):
 def test_workspace_sizes(lib):
     for d in (128, 256, 4096, 14336):
         b = G.gptq_prepare_workspace_bytes(d)
-        assert b >= 2 * 4 * d * d and b % 256 == 0
+        # A and Y (d x d each) and Xc's two planes of d x 128 fp32
+        assert b >= 2 * 4 * d * d + 2 * 4 * d * 128 and b % 256 == 0
+    # the allocation-free entry point's fixed 16 MiB scratch covers every d
+    # it accepts (d <= 1024, per include/gptq.h)
+    assert G.gptq_prepare_workspace_bytes(1024) <= 16 << 20
     for m, d in ((1, 128), (300, 256), (4096, 4096), (14336, 4096)):
         b = G.gptq_quantize_workspace_bytes(m, d, 128)
         assert b >= 4 * m * d + 4 * m * 128
